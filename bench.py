@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the chunked SSD forward: tokens/s and TFLOP/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c1] [--impl ours|reference]
+
+One step is one ``ssd_fwd`` call over the whole workload (all chunked steps:
+cumsum, intra-chunk output, chunk states, state passing, output correction)
+with inputs already resident in HBM.  The default workload is the Mamba-2
+2.7B-shaped layer (b8 L2048 H80 P64 N128 G1 Q64, bf16 in / fp32 accumulate).
+Rank 0 prints one JSON line.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronize, timed with CUDA events on the launching stream; the
+maximum over ranks is reported.  The inputs and outputs (hundreds of MB)
+are larger than the 126 MB L2, so no flush is needed between steps.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica
+of the workload: the (batch, head) units are independent and need no
+exchange, so there is no collective on the data path ("weak" scaling).
+
+``--impl reference`` times the fp64 CPU oracle instead (host cores, bounded
+samples of the same workload), as the comparison arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import ssd_inputs as si  # noqa: E402
+
+METRIC = "SSD fwd tokens/s and TFLOP/s (% of bf16 tensor roofline) at L=2K–16K, 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def work(shape: si.SSDShape, num_seqs):
+    """Algorithmic FLOPs (full Q x Q tiles, C.B^T once per group; and the
+    causal-half count) and minimum HBM bytes (each tensor touched once)."""
+    s = shape
+    b, L, H, P, N, G, Q = s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.chunk_size
+    c = -(-L // Q)
+    full = (2 * Q * Q * N * c * G * b + 2 * Q * Q * P * c * H * b + 4 * Q * N * P * c * H * b
+            + 2 * N * P * c * H * b + 2 * P * b * L * H)
+    causal = (Q * (Q + 1) * N * c * G * b + Q * (Q + 1) * P * c * H * b + 4 * Q * N * P * c * H * b
+              + 2 * N * P * c * H * b + 2 * P * b * L * H)
+    e = 2 if s.dtype == "bf16" else 4
+    nbytes = 2 * b * L * H * P * e + 2 * b * L * G * N * e + 4 * b * L * H + 4 * H * (2 if s.has_D else 1)
+    nbytes += 4 * H * P * N * (num_seqs if s.packed is not None else b)  # final states
+    if s.h0_std > 0:
+        nbytes += 4 * b * H * P * N
+    if s.packed is not None:
+        nbytes += 4 * b * L
+    return {"flops": full, "flops_causal": causal, "bytes": nbytes}
+
+
+def describe(shape: si.SSDShape) -> str:
+    s = shape
+    desc = (f"{s.name}: SSD fwd b{s.batch} L{s.seqlen} H{s.nheads} P{s.headdim} N{s.dstate} "
+            f"G{s.ngroups} Q{s.chunk_size} {s.dtype}")
+    if s.packed:
+        desc += f" packed lengths~U{list(s.packed)}"
+    if s.h0_std > 0:
+        desc += f" h0~N(0,{s.h0_std}^2)"
+    return desc
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("uuid,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str, period_ms: int = 50):
+        self.uuid = uuid
+        self.period_ms = period_ms
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", str(self.period_ms)], stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.uuid and self.uuid not in parts[0]:
+                continue
+            rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[6:10]) if v.lower() == "active"})
+        loaded = [v for v in sm if mx and v >= 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_uuid(dev) -> str:
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return ""
+
+
+def traffic_from_profiles(kernel_file: str, kernel: str, workload: str):
+    """dram read+write bytes per launch from a committed ncu summary, if it was
+    taken on the kernel source as it is now."""
+    path = os.path.join(ROOT, "profiles", f"{workload}_{kernel}_dram.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    src = os.path.join(ROOT, "mamba_ssd_chunked_03_b200", "csrc", kernel_file)
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if kv.get("source_sha256") != sha:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample(d, shape, target_s: float, max_units=None):
+    """Time the fp64 oracle on the first U (batch, head) units of the workload,
+    U chosen so the run takes about ``target_s`` seconds.  Returns
+    (tokens/s, units, seconds, threads)."""
+    import oracle  # test infrastructure: only this CPU-baseline leg uses it here
+    f = {k: oracle.as_f32(d[k]) for k in ("x", "dt", "A", "B", "C", "D", "initial_states")}
+    si_ = d.get("seq_idx")
+    seq = None if si_ is None else oracle.as_i32(si_)
+    threads = oracle.max_threads()
+    total_units = shape.batch * shape.nheads
+    t = time.perf_counter()
+    oracle.ssd_fwd(f["x"], f["dt"], f["A"], f["B"], f["C"], f["D"], f["initial_states"], seq, d.get("num_seqs"),
+                   units=list(range(min(threads, total_units))))
+    t_wave = max(time.perf_counter() - t, 1e-3)
+    waves = max(1, int(target_s / t_wave))
+    U = min(total_units, waves * threads) if max_units is None else min(total_units, max_units)
+    t = time.perf_counter()
+    oracle.ssd_fwd(f["x"], f["dt"], f["A"], f["B"], f["C"], f["D"], f["initial_states"], seq, d.get("num_seqs"),
+                   units=list(range(U)))
+    el = time.perf_counter() - t
+    tokens = U * shape.seqlen / shape.nheads
+    return tokens / el, U, el, min(threads, U)
+
+
+def run_reference(args, shape):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    d = si.make_inputs(shape)
+    f = {k: oracle.as_f32(d[k]) for k in ("x", "dt", "A", "B", "C", "D", "initial_states")}
+    seq = None if d.get("seq_idx") is None else oracle.as_i32(d["seq_idx"])
+    threads = oracle.max_threads()
+    U = min(shape.batch * shape.nheads, threads)
+    units = list(range(U))
+
+    def step():
+        oracle.ssd_fwd(f["x"], f["dt"], f["A"], f["B"], f["C"], f["D"], f["initial_states"], seq,
+                       d.get("num_seqs"), units=units)
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t
+    tokens = U * shape.seqlen / shape.nheads * args.steps
+    value = tokens / el
+    w = work(shape, d.get("num_seqs"))
+    sample = (f"first {U} of {shape.batch * shape.nheads} (batch, head) units per step "
+              f"= {U * shape.seqlen} head-tokens = {U * shape.seqlen / shape.nheads:.1f} tokens")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": describe(shape), "sample": sample},
+        "tflops": value / shape.tokens * w["flops"] / 1e12,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(threads, U), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="c1", choices=sorted(si.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--generic", action="store_true", help="force the generic CUDA-core kernels")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    shape = si.CONFIGS[args.config]
+
+    if args.impl == "reference":
+        return run_reference(args, shape)
+
+    import mamba_ssd_chunked_03_b200 as ssd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+
+    host = si.make_inputs(shape, seed=shape.seed + rank)
+    num_seqs = host.get("num_seqs")
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
+    b, L, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
+    y = torch.empty_like(g["x"])
+    rows = num_seqs if shape.packed is not None else b
+    final = torch.empty(rows, H, P, N, device=dev, dtype=torch.float32)
+    ws_bytes = ssd.workspace_size(g["x"], g["B"], shape.chunk_size, g.get("seq_idx"), num_seqs, True,
+                                  generic=args.generic)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    launches_per_call = ssd.launch_count(g["x"], g["B"], shape.chunk_size, g.get("seq_idx"), num_seqs, True,
+                                         generic=args.generic)
+    path = ssd.kernel_path(g["x"], g["B"], shape.chunk_size, generic=args.generic)
+
+    K = args.steps
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+    def step(events=None):
+        ssd.fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk_size=shape.chunk_size,
+                initial_states=g["initial_states"], seq_idx=g.get("seq_idx"), num_seqs=num_seqs,
+                y=y, final_states=final, workspace=ws, generic=args.generic, timing_events=events)
+
+    for _ in range(args.warmup):
+        step()
+    for a_, c_ in kev:  # torch creates the underlying cudaEvent on first record
+        a_.record()
+        c_.record()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(gpu_uuid(dev))
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        step(kev[i])
+    e1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clock_stats = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    kernel_ms = sum(a.elapsed_time(c) for a, c in kev) / K
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end to end through the public API: pinned host inputs -> device -> fwd -> host
+    names = [k for k in ("x", "dt", "A", "B", "C", "D", "initial_states", "seq_idx") if host.get(k) is not None]
+    pinned = {k: host[k].pin_memory() for k in names}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    f_host = torch.empty(final.shape, dtype=final.dtype).pin_memory()
+    h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in names)
+    d2h = y_host.numel() * y_host.element_size() + f_host.numel() * f_host.element_size()
+
+    def e2e_step():
+        for k in names:
+            g[k].copy_(pinned[k], non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        f_host.copy_(final, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    E = max(3, min(K, 50))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(E):
+        e2e_step()
+    a1.record()
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+
+    w = work(shape, num_seqs)
+    peaks = load_peaks()
+    ms_step = ms / K
+    tokens_job = shape.tokens * world
+    value = tokens_job / (ms_step / 1e3)
+    t_hbm = w["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = w["flops"] / (peaks["bf16_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        achieved = w["bytes"] / (kernel_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"]}
+    else:
+        achieved = w["flops"] / (kernel_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "peak_source": peaks["source"]}
+    kfile = "ssd_tc.cu" if path == "tcgen05" else "ssd_generic.cu"
+    roof["kernel"] = "ssd_fwd_tc" if path == "tcgen05" else "generic (all kernels of the call)"
+    roof["kernel_ms"] = kernel_ms
+    roof["traffic"] = traffic_from_profiles(kfile, path, shape.name)
+    roof["algorithmic_bytes"] = w["bytes"]
+    roof["algorithmic_flops"] = w["flops"]
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if shape.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": describe(shape), "batch": b, "seqlen": L, "nheads": H, "headdim": P,
+                   "dstate": N, "ngroups": shape.ngroups, "chunk_size": shape.chunk_size,
+                   "l2": f"no flush: inputs+outputs {w['bytes'] / 1e6:.0f} MB per step > 126 MB L2",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "tflops": {"full": w["flops"] * world / (ms_step / 1e3) / 1e12,
+                   "causal": w["flops_causal"] * world / (ms_step / 1e3) / 1e12},
+        "kernel_path": path,
+        "roofline": roof,
+        "e2e": {"value": tokens_job / (e2e_ms / E / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": E},
+        "gpu_launches": launches_per_call * K,
+        "clocks": clock_stats,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, U, el, cores = oracle_sample(host, shape, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"first {U} of {b * H} (batch, head) units of the workload, "
+                                          f"{U * L / H:.1f} tokens, {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,144 @@
+/*
+ * ssd.h -- C ABI of libssd, the chunked SSD (structured state space duality)
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * What one call computes, per batch row b and head h, with group
+ * g = h / (nheads / ngroups) (contiguous heads share B and C):
+ *
+ *   h_t = a_t h_{t-1} + dt_t x_t B_t^T        state, headdim x dstate
+ *   y_t = h_t C_t + D_h x_t                    output, headdim
+ *   a_t = exp(dt_t A_h), or 0 at the first token of a new packed sequence
+ *
+ * with h_{-1} = initial_states[b,h] (or 0).  Sources, by page title:
+ *  - "22 · Mamba 2 — Transformers are SSMs" (paper story), section 3.1 (the
+ *    scalar-A recurrence), section 3.2 (the dual form Y = (L o C B^T)(dt x)),
+ *    section 4.1 (block decomposition into intra- and inter-chunk parts).
+ *  - "SSM 家族全景图（下）：Mamba-2 与 Jamba", section 三.4 (the four chunked
+ *    steps) and the closing question (a_t = exp(Delta_t A)).
+ *  - "从Transformer的二次复杂度困境到Mamba的线性突围", continuous SSM
+ *    equations (the D feed-through).
+ *  - "Transformers与SSMs的隐藏联系", section 4.2 (packed sequences: the
+ *    transition is set to zero at each boundary).
+ *
+ * The result is computed with the chunked algorithm: an in-chunk cumulative
+ * sum of dt*A, the masked decay-weighted C B^T "attention" inside each chunk,
+ * per-chunk states, a scan of states across chunks, and an output correction
+ * from each chunk's carried state.  Chunking re-associates the same sums, so
+ * the result equals the recurrence up to rounding for every chunk size.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or retains them, and keeps no global state, so
+ *    calls are re-entrant and may run concurrently on different streams with
+ *    different workspaces.
+ *  - Tensors are dense and contiguous, row-major in the order given.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL means
+ *    the legacy default stream) and the call returns without synchronising.
+ *  - Arguments are validated on the host before anything is enqueued; a
+ *    rejected call enqueues nothing.  Nothing on the device traps or asserts.
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SSD_OK = 0,
+  SSD_ERR_INVALID_ARG = 1,  /* null required pointer, bad size, bad alignment, bad enum */
+  SSD_ERR_UNSUPPORTED = 2,  /* valid arguments outside the implemented shape set */
+  SSD_ERR_WORKSPACE = 3,    /* workspace missing or smaller than ssd_fwd_workspace_size() */
+  SSD_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed (see cudaGetLastError) */
+  SSD_ERR_TIMEOUT = 5       /* reserved: a bounded device-side wait gave up */
+} ssd_status;
+
+/* Element type of x, B, C and y.  dt, A, D, initial_states and final_states
+ * are always fp32. */
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+
+/* flags */
+#define SSD_FLAG_GENERIC 1u /* use the generic (CUDA-core, fp32) kernels even where
+                               the tensor-core kernels apply; for cross-checks */
+
+typedef struct {
+  /* sizes: b = batch, L = seqlen, H = nheads, P = headdim, N = dstate,
+   * G = ngroups (H % G == 0), Q = chunk_size (a power of two, 16..256).
+   * L need not be a multiple of Q (the last chunk is short). */
+  int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk_size;
+  ssd_dtype dtype;
+  uint32_t flags;                 /* SSD_FLAG_* or 0 */
+
+  const void* x;                  /* (b,L,H,P) dtype                                  */
+  const float* dt;                /* (b,L,H) fp32, the step size used as given (> 0)  */
+  const float* A;                 /* (H) fp32, continuous decay rate (expected < 0)   */
+  const void* B;                  /* (b,L,G,N) dtype, input projection ("keys")       */
+  const void* C;                  /* (b,L,G,N) dtype, output projection ("queries")   */
+  const float* D;                 /* (H) fp32 skip weight, or NULL for D = 0          */
+  const float* initial_states;    /* (b,H,P,N) fp32 state before token 0, or NULL = 0.
+                                     With seq_idx it applies to each row's first
+                                     sequence only.                                  */
+  const int32_t* seq_idx;         /* (b,L) int32 packed-sequence ids, or NULL.
+                                     Precondition: non-decreasing along each row, ids
+                                     in [0, num_seqs), a sequence never spans rows.
+                                     A change of id starts a new sequence (a_t = 0). */
+  int64_t num_seqs;               /* number of sequence ids; required (> 0) iff seq_idx */
+
+  void* y;                        /* (b,L,H,P) dtype, output                          */
+  float* final_states;            /* output or NULL: (b,H,P,N) fp32 state after the
+                                     last token; with seq_idx (num_seqs,H,P,N), the
+                                     state after each sequence's last token (ids that
+                                     do not occur get zeros)                         */
+
+  void* workspace;                /* device scratch of at least
+                                     ssd_fwd_workspace_size(args) bytes, 256-byte
+                                     aligned; may be NULL when that size is 0.  Its
+                                     contents on entry do not matter.                */
+  size_t workspace_bytes;
+
+  void* timing_events[2];         /* optional pair of cudaEvent_t (as void*), or NULLs:
+                                     recorded on `stream` right before and right after
+                                     the main kernel of the call (the fused tensor-core
+                                     kernel, or all generic kernels together), so a
+                                     caller can time it without a profiler.  Owned by
+                                     the caller; both or neither.                    */
+} ssd_fwd_args;
+
+/* Bytes of device workspace ssd_fwd needs for these sizes and options (only
+ * the size fields, dtype, flags and the presence of seq_idx/final_states are
+ * read; pointers may be NULL).  Returns 0 if the sizes are invalid. */
+SSD_API size_t ssd_fwd_workspace_size(const ssd_fwd_args* args);
+
+/* Enqueue the SSD forward on `stream`.  Returns SSD_OK once the work is
+ * enqueued, or an error code; on error nothing was enqueued except for
+ * SSD_ERR_CUDA from a later launch, in which case outputs are undefined. */
+SSD_API ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream);
+
+/* Number of kernels ssd_fwd enqueues for these arguments (memsets excluded),
+ * or 0 if the sizes are invalid. */
+SSD_API int ssd_fwd_launch_count(const ssd_fwd_args* args);
+
+/* Name of the kernel path ssd_fwd would take for these arguments
+ * ("generic", "tcgen05"), or "invalid". Static string. */
+SSD_API const char* ssd_fwd_path(const ssd_fwd_args* args);
+
+/* Static, human-readable text for a status code. */
+SSD_API const char* ssd_status_string(ssd_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+SSD_API int ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H_ */

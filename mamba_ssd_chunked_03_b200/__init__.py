@@ -1,0 +1,202 @@
+"""Chunked SSD (Mamba-2 structured state space duality) forward on B200.
+
+Thin Python binding over the C ABI in ``include/ssd.h`` (``libssd.so``, built
+in-tree by ``mamba_ssd_chunked_03_b200/build.py``).  This module only marshals
+arguments: it checks tensor placement, dtypes and shapes, allocates outputs
+and the workspace with PyTorch on the current stream, and calls ``ssd_fwd``.
+Every step of the forward runs in the library's CUDA kernels; there is no
+Python or CPU fallback, and importing fails loudly if the library is missing.
+
+    y, final_states = fwd(x, dt, A, B, C, D, chunk_size=64,
+                          initial_states=None, seq_idx=None, num_seqs=None)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = ["fwd", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
+           "SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED", "SSD_ERR_WORKSPACE", "SSD_ERR_CUDA",
+           "SSD_F32", "SSD_BF16", "SSD_FLAG_GENERIC"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
+
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_WORKSPACE, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(6)
+SSD_F32, SSD_BF16 = 0, 1
+SSD_FLAG_GENERIC = 1
+
+
+class Args(ctypes.Structure):
+    """Mirror of ``ssd_fwd_args``."""
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups", "chunk_size")] + [
+        ("dtype", ctypes.c_int),
+        ("flags", ctypes.c_uint32),
+        ("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("A", ctypes.c_void_p),
+        ("B", ctypes.c_void_p), ("C", ctypes.c_void_p), ("D", ctypes.c_void_p),
+        ("initial_states", ctypes.c_void_p), ("seq_idx", ctypes.c_void_p),
+        ("num_seqs", ctypes.c_int64),
+        ("y", ctypes.c_void_p), ("final_states", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("timing_events", ctypes.c_void_p * 2),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python mamba_ssd_chunked_03_b200/build.py` "
+            "(there is no fallback implementation)")
+    L = ctypes.CDLL(LIB_PATH)
+    L.ssd_fwd.argtypes = [ctypes.POINTER(Args), ctypes.c_void_p]
+    L.ssd_fwd.restype = ctypes.c_int
+    L.ssd_fwd_workspace_size.argtypes = [ctypes.POINTER(Args)]
+    L.ssd_fwd_workspace_size.restype = ctypes.c_size_t
+    L.ssd_fwd_launch_count.argtypes = [ctypes.POINTER(Args)]
+    L.ssd_fwd_launch_count.restype = ctypes.c_int
+    L.ssd_fwd_path.argtypes = [ctypes.POINTER(Args)]
+    L.ssd_fwd_path.restype = ctypes.c_char_p
+    L.ssd_status_string.argtypes = [ctypes.c_int]
+    L.ssd_status_string.restype = ctypes.c_char_p
+    L.ssd_version.restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        super().__init__(f"ssd_fwd failed: {lib.ssd_status_string(status).decode()} (status {status})")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def make_args(x, dt, A, B, C, D=None, chunk_size: int = 64, initial_states=None, seq_idx=None,
+              num_seqs: Optional[int] = None, y=None, final_states=None, workspace=None,
+              workspace_bytes: int = 0, generic: bool = False) -> Args:
+    """Fill an ``ssd_fwd_args`` from tensors (shapes read from x and B)."""
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    a = Args()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk_size = b, L, H, P, N, G, int(chunk_size)
+    a.dtype = SSD_BF16 if x.dtype == torch.bfloat16 else SSD_F32
+    a.flags = SSD_FLAG_GENERIC if generic else 0
+    a.x, a.dt, a.A, a.B, a.C, a.D = _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D)
+    a.initial_states, a.seq_idx = _ptr(initial_states), _ptr(seq_idx)
+    a.num_seqs = int(num_seqs) if seq_idx is not None else 0
+    a.y, a.final_states = _ptr(y), _ptr(final_states)
+    a.workspace, a.workspace_bytes = _ptr(workspace), int(workspace_bytes)
+    return a
+
+
+def _check(x, dt, A, B, C, D, initial_states, seq_idx):
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    if x.dim() != 4 or B.dim() != 4 or C.dim() != 4 or dt.dim() != 3 or A.dim() != 1:
+        raise ValueError("expected x (b,L,H,P), dt (b,L,H), A (H), B and C (b,L,G,N)")
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if tuple(B.shape) != (b, L, G, N) or tuple(C.shape) != (b, L, G, N):
+        raise ValueError("B and C must be (b, L, G, N)")
+    if tuple(dt.shape) != (b, L, H) or tuple(A.shape) != (H,):
+        raise ValueError("dt must be (b, L, H) and A (H,)")
+    if B.dtype != x.dtype or C.dtype != x.dtype:
+        raise TypeError("B and C must have x's dtype")
+    if dt.dtype != torch.float32 or A.dtype != torch.float32:
+        raise TypeError("dt and A must be float32")
+    if D is not None and (D.dtype != torch.float32 or tuple(D.shape) != (H,)):
+        raise ValueError("D must be float32 (H,)")
+    if initial_states is not None and (initial_states.dtype != torch.float32
+                                       or tuple(initial_states.shape) != (b, H, P, N)):
+        raise ValueError("initial_states must be float32 (b, H, P, N)")
+    if seq_idx is not None and (seq_idx.dtype != torch.int32 or tuple(seq_idx.shape) != (b, L)):
+        raise ValueError("seq_idx must be int32 (b, L)")
+    dev = x.device
+    for name, t in (("x", x), ("dt", dt), ("A", A), ("B", B), ("C", C), ("D", D),
+                    ("initial_states", initial_states), ("seq_idx", seq_idx)):
+        if t is None:
+            continue
+        if t.device != dev or dev.type != "cuda":
+            raise ValueError(f"{name} must be a CUDA tensor on {dev}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def workspace_size(x, B, chunk_size: int, seq_idx=None, num_seqs=None, final_states: bool = True,
+                   generic: bool = False) -> int:
+    """Workspace bytes for these shapes (tensors only supply shapes/dtype)."""
+    a = make_args(x, None, None, B, None, chunk_size=chunk_size, seq_idx=seq_idx, num_seqs=num_seqs,
+                  generic=generic)
+    if final_states:
+        a.final_states = 1 << 8  # presence only; the size query does not dereference
+    return int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
+
+
+def launch_count(x, B, chunk_size: int, seq_idx=None, num_seqs=None, final_states: bool = True,
+                 generic: bool = False) -> int:
+    """Kernels one ``fwd`` call enqueues for these shapes."""
+    a = make_args(x, None, None, B, None, chunk_size=chunk_size, seq_idx=seq_idx, num_seqs=num_seqs,
+                  generic=generic)
+    if final_states:
+        a.final_states = 1 << 8  # presence only; the query does not dereference
+    return int(lib.ssd_fwd_launch_count(ctypes.byref(a)))
+
+
+def kernel_path(x, B, chunk_size: int, generic: bool = False) -> str:
+    a = make_args(x, None, None, B, None, chunk_size=chunk_size, generic=generic)
+    return lib.ssd_fwd_path(ctypes.byref(a)).decode()
+
+
+def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+        D: Optional[torch.Tensor] = None, chunk_size: int = 64,
+        initial_states: Optional[torch.Tensor] = None, seq_idx: Optional[torch.Tensor] = None,
+        num_seqs: Optional[int] = None, return_final_states: bool = True,
+        y: Optional[torch.Tensor] = None, final_states: Optional[torch.Tensor] = None,
+        workspace: Optional[torch.Tensor] = None, generic: bool = False,
+        timing_events: Optional[tuple] = None):
+    """SSD forward.  Returns (y, final_states or None).
+
+    x (b,L,H,P) fp32|bf16, dt (b,L,H) fp32, A (H) fp32, B/C (b,L,G,N) x.dtype,
+    D (H) fp32 or None, initial_states (b,H,P,N) fp32 or None,
+    seq_idx (b,L) int32 (non-decreasing per row) or None; with seq_idx,
+    final_states is (num_seqs,H,P,N), else (b,H,P,N).
+    ``y``, ``final_states`` and ``workspace`` may be passed preallocated.
+    ``timing_events``: optional (start, end) torch.cuda.Event pair recorded on
+    the current stream around the call's main kernel.
+    """
+    _check(x, dt, A, B, C, D, initial_states, seq_idx)
+    b, L, H, P = x.shape
+    N = B.shape[3]
+    if seq_idx is not None and num_seqs is None:
+        num_seqs = int(seq_idx.max().item()) + 1
+    if y is None:
+        y = torch.empty_like(x)
+    if return_final_states and final_states is None:
+        rows = num_seqs if seq_idx is not None else b
+        final_states = torch.empty(rows, H, P, N, device=x.device, dtype=torch.float32)
+    if not return_final_states:
+        final_states = None
+    a = make_args(x, dt, A, B, C, D, chunk_size, initial_states, seq_idx, num_seqs, y, final_states,
+                  generic=generic)
+    need = int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
+    if need > 0:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    if timing_events is not None:
+        h0_, h1_ = timing_events[0].cuda_event, timing_events[1].cuda_event
+        if not h0_ or not h1_:
+            raise ValueError("timing events must have been recorded once (torch creates them lazily)")
+        a.timing_events[0], a.timing_events[1] = h0_, h1_
+    stream = torch.cuda.current_stream(x.device).cuda_stream
+    st = lib.ssd_fwd(ctypes.byref(a), ctypes.c_void_p(stream))
+    if st != SSD_OK:
+        raise SSDError(st)
+    return y, final_states

@@ -1,0 +1,38 @@
+// Internal declarations shared by the libssd translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssd.h"
+
+namespace ssd {
+
+// Resolved problem description (validated sizes, typed pointers).
+struct Problem {
+  int64_t b, L, H, P, N, G, Q, nc;  // nc = ceil(L / Q) chunks per row
+  int64_t hpg;                      // heads per group, H / G
+  ssd_dtype dtype;
+  const void* x;
+  const float* dt;
+  const float* A;
+  const void* B;
+  const void* C;
+  const float* D;
+  const float* h0;
+  const int32_t* seq;
+  int64_t num_seqs;
+  void* y;
+  float* final_states;
+};
+
+constexpr size_t kWsAlign = 256;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---- generic (CUDA-core, fp32) path: ssd_generic.cu ----
+size_t generic_workspace_bytes(const Problem& p);
+cudaError_t generic_forward(const Problem& p, void* ws, cudaStream_t stream);
+int generic_launch_count(const Problem& p);
+
+}  // namespace ssd

@@ -1,0 +1,135 @@
+"""The C-ABI library: loads, exports every declared symbol, validates on the
+host.  CPU only: no call here reaches a kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mamba_ssd_chunked_03_b200 as ssd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"SSD_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert "ssd_fwd" in names and "ssd_fwd_workspace_size" in names
+    raw = ctypes.CDLL(ssd.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings_and_version():
+    for s in range(6):
+        assert ssd.lib.ssd_status_string(s)
+    assert ssd.lib.ssd_status_string(99) == b"unknown status"
+    assert ssd.lib.ssd_version() >= 100
+
+
+def base_args(**kw):
+    a = ssd.Args()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk_size = 2, 100, 4, 64, 128, 2, 64
+    a.dtype = ssd.SSD_BF16
+    fake = 1 << 20  # never dereferenced: every case below is rejected on the host
+    a.x = a.dt = a.A = a.B = a.C = a.y = fake
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def call(a):
+    return ssd.lib.ssd_fwd(ctypes.byref(a), None)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("batch", 0, ssd.SSD_ERR_INVALID_ARG),
+    ("seqlen", -1, ssd.SSD_ERR_INVALID_ARG),
+    ("nheads", 0, ssd.SSD_ERR_INVALID_ARG),
+    ("ngroups", 3, ssd.SSD_ERR_INVALID_ARG),       # H % G != 0
+    ("chunk_size", 48, ssd.SSD_ERR_INVALID_ARG),   # not a power of two
+    ("chunk_size", 8, ssd.SSD_ERR_INVALID_ARG),    # below 16
+    ("chunk_size", 512, ssd.SSD_ERR_INVALID_ARG),  # above 256
+    ("dtype", 7, ssd.SSD_ERR_INVALID_ARG),
+    ("flags", 4, ssd.SSD_ERR_INVALID_ARG),
+    ("headdim", 12, ssd.SSD_ERR_UNSUPPORTED),
+    ("dstate", 512, ssd.SSD_ERR_UNSUPPORTED),
+    ("x", None, ssd.SSD_ERR_INVALID_ARG),
+    ("dt", None, ssd.SSD_ERR_INVALID_ARG),
+    ("A", None, ssd.SSD_ERR_INVALID_ARG),
+    ("B", None, ssd.SSD_ERR_INVALID_ARG),
+    ("C", None, ssd.SSD_ERR_INVALID_ARG),
+    ("y", None, ssd.SSD_ERR_INVALID_ARG),
+    ("x", (1 << 20) + 8, ssd.SSD_ERR_INVALID_ARG),  # misaligned
+    ("final_states", (1 << 20) + 4, ssd.SSD_ERR_INVALID_ARG),
+])
+def test_bad_argument_rejected(field, value, status):
+    assert call(base_args(**{field: value})) == status
+
+
+def test_seq_idx_needs_num_seqs():
+    assert call(base_args(seq_idx=1 << 20, num_seqs=0)) == ssd.SSD_ERR_INVALID_ARG
+
+
+def test_null_args_pointer():
+    assert ssd.lib.ssd_fwd(None, None) == ssd.SSD_ERR_INVALID_ARG
+    assert ssd.lib.ssd_fwd_workspace_size(None) == 0
+
+
+def test_workspace_checked_before_launch():
+    a = base_args()
+    need = ssd.lib.ssd_fwd_workspace_size(ctypes.byref(a))
+    assert need > 0
+    assert call(a) == ssd.SSD_ERR_WORKSPACE                 # none given
+    a.workspace, a.workspace_bytes = 1 << 24, need - 1
+    assert call(a) == ssd.SSD_ERR_WORKSPACE                 # one byte short
+    a.workspace, a.workspace_bytes = (1 << 24) + 16, need
+    assert call(a) == ssd.SSD_ERR_INVALID_ARG               # not 256-byte aligned
+
+
+def test_workspace_size_is_pure_and_monotone():
+    a = base_args()
+    w1 = ssd.lib.ssd_fwd_workspace_size(ctypes.byref(a))
+    a.seqlen = 1000
+    w2 = ssd.lib.ssd_fwd_workspace_size(ctypes.byref(a))
+    assert w2 > w1
+    a.chunk_size = 48
+    assert ssd.lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 0
+
+
+def test_kernel_path_query():
+    a = base_args()
+    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) in (b"generic", b"tcgen05")
+    a.flags = ssd.SSD_FLAG_GENERIC
+    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"generic"
+    a.chunk_size = 3
+    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"invalid"
+
+
+def test_struct_layout_matches_header():
+    # 7 int64 sizes, dtype + flags, 8 pointers, num_seqs, 2 outputs, workspace + bytes
+    assert ctypes.sizeof(ssd.Args) == 7 * 8 + 4 + 4 + 8 * 8 + 8 + 2 * 8 + 8 + 8 + 2 * 8
+    assert ssd.Args.x.offset == 64 and ssd.Args.num_seqs.offset == 128
+    assert ssd.Args.timing_events.offset == 168
+
+
+def test_timing_events_both_or_neither():
+    a = base_args()
+    a.timing_events[0] = 1 << 12
+    assert call(a) == ssd.SSD_ERR_INVALID_ARG
+
+
+def test_launch_count_query():
+    a = base_args()
+    n = ssd.lib.ssd_fwd_launch_count(ctypes.byref(a))
+    assert n >= 1
+    a.chunk_size = 3
+    assert ssd.lib.ssd_fwd_launch_count(ctypes.byref(a)) == 0
