@@ -123,6 +123,29 @@ SSD_API size_t ssd_fwd_workspace_size(const ssd_fwd_args* args);
  * SSD_ERR_CUDA from a later launch, in which case outputs are undefined. */
 SSD_API ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream);
 
+/* ssd_fwd for callers that cannot allocate device memory when they call:
+ * identical arguments and results (it always runs the generic CUDA-core
+ * kernels), but the workspace fields are ignored and no memory is allocated
+ * or freed.  Meant for code where no device allocator is reachable or allowed
+ * once work has started, such as a plugin inside a host runtime that owns all
+ * device memory, or a latency-critical loop that must not call cudaMalloc.
+ * The pages describe no such entry point; it has no counterpart there.
+ *
+ * Scratch comes from one fixed 32 MiB device array inside the library.  Every
+ * GPU that loads this part of the library keeps that array until the process
+ * exits.  Problems whose generic workspace (ssd_fwd_workspace_size with
+ * SSD_FLAG_GENERIC) exceeds 32 MiB are rejected with SSD_ERR_WORKSPACE before
+ * anything is enqueued.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.  A failed lookup returns SSD_ERR_CUDA.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents; each call rewrites every part it reads (and clears what must
+ *    start at zero), so sequential calls are independent.  Calls that overlap
+ *    on the GPU (other streams, other host threads) race on the array:
+ *    serialise them. */
+SSD_API ssd_status ssd_fwd_noalloc(const ssd_fwd_args* args, void* stream);
+
 /* Number of kernels ssd_fwd enqueues for these arguments (memsets excluded),
  * or 0 if the sizes are invalid. */
 SSD_API int ssd_fwd_launch_count(const ssd_fwd_args* args);
