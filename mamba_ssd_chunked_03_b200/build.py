@@ -68,10 +68,30 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     return LIB
 
 
+PROBE_SRC = os.path.join(ROOT, "tests", "cuda", "tc_probe.cu")
+PROBE_LIB = os.path.join(ROOT, "tests", "cuda", "libtcprobe.so")
+
+
+def build_probe(force: bool = False, verbose: bool = False) -> str:
+    """Test-only library probing the tcgen05 building blocks (tests/cuda)."""
+    deps = [PROBE_SRC, os.path.join(CSRC, "sm100.cuh"), os.path.abspath(__file__)]
+    if (not force and os.path.exists(PROBE_LIB)
+            and os.path.getmtime(PROBE_LIB) >= max(os.path.getmtime(d) for d in deps)):
+        return PROBE_LIB
+    tmp = PROBE_LIB + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-I", CSRC, "-shared", "-o", tmp, PROBE_SRC, "-cudart", "static"]
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, PROBE_LIB)
+    return PROBE_LIB
+
+
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     args = ap.parse_args()
     print(build(force=args.force, verbose=args.verbose))
+    print(build_probe(force=args.force, verbose=args.verbose))
     sys.exit(0)

@@ -72,17 +72,18 @@ extern "C" {
 size_t ssd_fwd_workspace_size(const ssd_fwd_args* args) {
   if (ssd::check_sizes(args) != SSD_OK) return 0;
   const ssd::Problem p = ssd::resolve(args);
-  return ssd::generic_workspace_bytes(p);
+  return ssd::tc_supported(p, args->flags) ? ssd::tc_workspace_bytes(p) : ssd::generic_workspace_bytes(p);
 }
 
 int ssd_fwd_launch_count(const ssd_fwd_args* args) {
   if (ssd::check_sizes(args) != SSD_OK) return 0;
-  return ssd::generic_launch_count(ssd::resolve(args));
+  const ssd::Problem p = ssd::resolve(args);
+  return ssd::tc_supported(p, args->flags) ? ssd::tc_launch_count(p) : ssd::generic_launch_count(p);
 }
 
 const char* ssd_fwd_path(const ssd_fwd_args* args) {
   if (ssd::check_sizes(args) != SSD_OK) return "invalid";
-  return "generic";
+  return ssd::tc_supported(ssd::resolve(args), args->flags) ? "tcgen05" : "generic";
 }
 
 ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream) {
@@ -97,12 +98,14 @@ ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream) {
       !ssd::aligned(a->final_states, 16))
     return SSD_ERR_INVALID_ARG;
   const ssd::Problem p = ssd::resolve(a);
-  const size_t need = ssd::generic_workspace_bytes(p);
+  const bool tc = ssd::tc_supported(p, a->flags);
+  const size_t need = tc ? ssd::tc_workspace_bytes(p) : ssd::generic_workspace_bytes(p);
   if (need > 0 && (!a->workspace || a->workspace_bytes < need)) return SSD_ERR_WORKSPACE;
   if (!ssd::aligned(a->workspace, ssd::kWsAlign)) return SSD_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaEvent_t ev0 = static_cast<cudaEvent_t>(a->timing_events[0]);
   cudaEvent_t ev1 = static_cast<cudaEvent_t>(a->timing_events[1]);
+  if (tc) return ssd::tc_forward(p, a->workspace, s, ev0, ev1) == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
   if (ev0 && cudaEventRecord(ev0, s) != cudaSuccess) return SSD_ERR_CUDA;
   const cudaError_t err = ssd::generic_forward(p, a->workspace, s);
   if (err != cudaSuccess) return SSD_ERR_CUDA;

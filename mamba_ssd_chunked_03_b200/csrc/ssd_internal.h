@@ -35,4 +35,10 @@ size_t generic_workspace_bytes(const Problem& p);
 cudaError_t generic_forward(const Problem& p, void* ws, cudaStream_t stream);
 int generic_launch_count(const Problem& p);
 
+// ---- fused tensor-core path: ssd_tc.cu ----
+bool tc_supported(const Problem& p, uint32_t flags);
+size_t tc_workspace_bytes(const Problem& p);
+int tc_launch_count(const Problem& p);
+cudaError_t tc_forward(const Problem& p, void* ws, cudaStream_t stream, cudaEvent_t ev0, cudaEvent_t ev1);
+
 }  // namespace ssd

@@ -1,0 +1,593 @@
+// Exact fused chunked SSD forward on sm_100a tensor cores (tcgen05 + TMEM +
+// TMA).  It forms every intra-chunk decay exp(cs_t - cs_s) separately, so it
+// is valid for any decay; the launch processes only the (batch row, head)
+// units that the fast kernel (ssd_tc_fast.cu) leaves out because some chunk's
+// decay range is too wide to factorise.  The host also owns the tensor-map
+// helper and the workspace carve-up shared by both kernels.
+//
+// One CTA owns one (batch row, head) and walks its chunks in order, keeping
+// the running state on chip, so the only HBM traffic is the inputs and y.
+// Per chunk of Q = 64 tokens (headdim P = 64, state size N in {128, 256}):
+//
+//   MMA1  CB  = C B^T                     (Q x Q,  K = N)    -> TMEM, fp32
+//   mask  W   = CB o exp(cs_t - cs_s) dt_s [s <= t, same seq] + D_h I   -> smem bf16
+//   scale X~  = diag(exp(cs_e - cs_s) dt_s [same seq as e]) X            -> smem bf16
+//   MMA2  Yd  = W X                        (Q x P,  K = Q)    -> TMEM
+//   MMA3  Yo  = C H_c^T                    (Q x P,  K = N)    -> TMEM
+//   MMA4  S^T = B^T X~                     (N x P,  K = Q)    -> TMEM
+//   state H_{c+1} = keep exp(cs_e) H_c + S           (fp32, registers; bf16 copy in smem)
+//   out   y_t = Yd_t + keep_t exp(cs_t) Yo_t          (bf16)
+//
+// These are the four chunked steps of "SSM 家族全景图（下）：Mamba-2 与 Jamba"
+// section 三.4 (intra-chunk output, chunk state, state passing, correction
+// from the chunk's true initial state) on the dual form of "22 · Mamba 2 —
+// Transformers are SSMs" section 3.2 (W is the decay-masked C B^T).  The D
+// skip of "从Transformer的二次复杂度困境到Mamba的线性突围" is folded into the
+// diagonal of W, so W X also yields D x.  cs is the in-chunk cumulative sum of
+// dt A, kept in log2 units so each decay is one exp2 of a difference with the
+// later token first (never above 1).  keep / same-seq factors implement the
+// zero transition at packed-sequence boundaries ("Transformers与SSMs的隐藏联系"
+// section 4.2).
+//
+// Warp roles (192 threads):  warp 0 TMA producer, warp 1 MMA issuer (one
+// thread), warps 2-5 compute (cumsum, mask, scale, state update, epilogue).
+// Every wait is bounded; a CTA that times out records the error, drains its
+// own copies and MMAs, frees its TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "sm100.cuh"
+#include "ssd_internal.h"
+#include "ssd_tc_common.cuh"
+
+namespace ssd {
+
+namespace tc {
+
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once per process through the
+// runtime (no link-time dependency on libcuda).
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+}  // namespace
+
+bool make_map_3d(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer};
+  const cuuint64_t strides[2] = {(cuuint64_t)(inner * 2), (cuuint64_t)(inner * 2 * rows)};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+namespace {
+
+using namespace sm100;
+using namespace tc;
+
+template <int NS>
+struct Cfg {
+  static constexpr int Q = 64, P = 64, NB = NS / 64;
+  static constexpr int kThreads = 192;
+  static constexpr uint32_t kTile = 8192;  // 64 rows x 128 B
+  static constexpr uint32_t oC = 0;
+  static constexpr uint32_t oB = oC + NB * kTile;
+  static constexpr uint32_t oX = oB + NB * kTile;
+  static constexpr uint32_t oW = oX + kTile;
+  static constexpr uint32_t oXt = oW + kTile;
+  static constexpr uint32_t oH = oXt + kTile;
+  static constexpr uint32_t oEnd = oH + NB * kTile;
+  // N = 128: 2 CTAs per SM (TMEM 256 columns each); the request is padded so a
+  // third CTA never fits next to them.  N = 256: 1 CTA per SM.
+  static constexpr uint32_t kSmemBytes = (NS <= 128 ? (oEnd + 1024 > 80 * 1024 ? oEnd + 1024 : 80 * 1024)
+                                                    : oEnd + 1024);
+  static constexpr uint32_t tCB = 0, tYd = 64, tYo = 128, tS = 192;
+  static constexpr uint32_t kTmemCols = NS <= 128 ? 256 : 512;
+  static constexpr uint32_t kStageBytes = 2 * NB * kTile + kTile;
+  static constexpr int kMinBlocks = NS <= 128 ? 2 : 1;
+};
+
+struct TcArgs {
+  int64_t b, L, H, G, hpg, nc;
+  const float* dt;
+  const float* A;
+  const float* D;
+  const float* h0;
+  const int32_t* seq;
+  __nv_bfloat16* y;
+  float* final_states;
+  const uint8_t* ok;  // per (b, chunk, head) flags of the fast kernel; may be null
+  int* err;
+};
+
+struct __align__(8) Smem {
+  uint64_t full, empty, cb_full, s_full, y_full;
+  uint64_t cb_free, w_ready, xt_ready, h_ready, s_free, y_free;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int never;  // stays 0: a flag for waits that must not be cut short
+  float cs2[64];   // in-chunk cumulative sum of dt*A, log2 units
+  float dts[64];
+  int seqs[64];
+  float warp_tot;
+};
+
+template <int NS>
+__global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
+    k_ssd_fwd_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+                 const __grid_constant__ CUtensorMap tm_c, const TcArgs a) {
+  using K = Cfg<NS>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                       ~uintptr_t(1023));
+  __shared__ Smem s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t unit = blockIdx.x;
+  const int64_t b = unit / a.H, h = unit % a.H;
+  const int64_t g = h / a.hpg;
+  const int nc = (int)a.nc;
+
+  // units whose chunks are all within the fast kernel's range are done there
+  if (a.ok) {
+    bool all_ok = true;
+    for (int c = tid; c < nc; c += blockDim.x) all_ok &= a.ok[(b * a.nc + c) * a.H + h] != 0;
+    if (__syncthreads_and(all_ok)) return;
+  }
+
+  if (tid == 0) {
+    mbar_init(&s.full, 1);
+    mbar_init(&s.empty, 1);
+    mbar_init(&s.cb_full, 1);
+    mbar_init(&s.s_full, 1);
+    mbar_init(&s.y_full, 1);
+    mbar_init(&s.cb_free, 128);
+    mbar_init(&s.w_ready, 128);
+    mbar_init(&s.xt_ready, 128);
+    mbar_init(&s.h_ready, 128);
+    mbar_init(&s.s_free, 128);
+    mbar_init(&s.y_free, 128);
+    mbar_init(&s.drain, 1);
+    // a CTA of this launch already gave up: every wait below returns at once
+    s.abort_flag = *reinterpret_cast<volatile int*>(a.err) != 0;
+    s.never = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_c);
+  }
+  if (warp == 0) {
+    tmem_alloc(&s.tmem_base, K::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int* abort_flag = &s.abort_flag;
+  volatile int* never = &s.never;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int c = 0; c < nc; ++c) {
+        if (c > 0 && !mbar_wait(&s.empty, (c - 1) & 1, abort_flag, kWaitLimitNs)) break;
+        const int t0 = c * K::Q;
+        mbar_arrive_expect_tx(&s.full, K::kStageBytes);
+        for (int j = 0; j < K::NB; ++j) {
+          tma_load_3d(sm + K::oC + j * K::kTile, &tm_c, &s.full, (int)(g * NS + 64 * j), t0, (int)b);
+          tma_load_3d(sm + K::oB + j * K::kTile, &tm_b, &s.full, (int)(g * NS + 64 * j), t0, (int)b);
+        }
+        tma_load_3d(sm + K::oX, &tm_x, &s.full, (int)(h * K::P), t0, (int)b);
+        issued = c + 1;
+      }
+      if (*abort_flag && issued > 0) {
+        // let this CTA's own copies land before the shared memory is released
+        mbar_wait(&s.full, (issued - 1) & 1, never, kWaitLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB), aX = smem_u32(sm + K::oX);
+      const uint32_t aW = smem_u32(sm + K::oW), aXt = smem_u32(sm + K::oXt), aH = smem_u32(sm + K::oH);
+      constexpr uint32_t id_cb = idesc_bf16(64, 64, 0, 0);
+      constexpr uint32_t id_wx = idesc_bf16(64, 64, 0, 1);
+      constexpr uint32_t id_st = idesc_bf16(128, 64, 1, 1);
+      bool ok = true;
+      for (int c = 0; c < nc && ok; ++c) {
+        const uint32_t par = c & 1, ppar = (c - 1) & 1;
+        ok = mbar_wait(&s.full, par, abort_flag, kWaitLimitNs);
+        if (ok && c > 0) ok = mbar_wait(&s.cb_free, ppar, abort_flag, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+        // MMA1: CB = C B^T, K = N in steps of 16
+#pragma unroll
+        for (int kk = 0; kk < NS / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * K::kTile + (kk & 3) * 32;
+          mma_bf16_ss(tmem + K::tCB, sw128_desc(aC + koff, 16, 1024), sw128_desc(aB + koff, 16, 1024), id_cb,
+                      kk > 0);
+        }
+        mma_commit(&s.cb_full);
+        // MMA3: Yo = C H_c^T (H stored [n][p], MN-major B operand), K = N
+        ok = mbar_wait(&s.h_ready, par, abort_flag, kWaitLimitNs);
+        if (ok && c > 0) ok = mbar_wait(&s.y_free, ppar, abort_flag, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < NS / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * K::kTile + (kk & 3) * 32;
+          mma_bf16_ss(tmem + K::tYo, sw128_desc(aC + koff, 16, 1024), sw128_desc(aH + kk * 2048, K::kTile, 1024),
+                      id_wx, kk > 0);
+        }
+        // MMA4: S^T = B^T X~ (both MN-major), M = 128 state rows per half
+        ok = mbar_wait(&s.xt_ready, par, abort_flag, kWaitLimitNs);
+        if (ok && c > 0) ok = mbar_wait(&s.s_free, ppar, abort_flag, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int hf = 0; hf < NS / 128; ++hf) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_bf16_ss(tmem + K::tS + hf * 64, sw128_desc(aB + hf * 2 * K::kTile + kk * 2048, K::kTile, 1024),
+                        sw128_desc(aXt + kk * 2048, K::kTile, 1024), id_st, kk > 0);
+          }
+        }
+        mma_commit(&s.s_full);
+        // MMA2: Yd = W X, K = Q
+        ok = mbar_wait(&s.w_ready, par, abort_flag, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_bf16_ss(tmem + K::tYd, sw128_desc(aW + kk * 32, 16, 1024), sw128_desc(aX + kk * 2048, K::kTile, 1024),
+                      id_wx, kk > 0);
+        }
+        mma_commit(&s.y_full);
+        mma_commit(&s.empty);
+      }
+      // all MMAs issued by this thread must finish before TMEM is released
+      mma_commit(&s.drain);
+      mbar_wait(&s.drain, 0, never, kWaitLimitNs);
+    }
+  } else {
+    // ------------------------------------------------------------ compute warps
+    const int wt = tid - 64;      // 0..127
+    const int q = warp & 3;       // TMEM lane quadrant this warp may access
+    const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+    const float a2 = a.A[h] * kLog2e;
+    const float dskip = a.D ? a.D[h] : 0.f;
+    const int64_t rowbase = b * a.L;
+    // state rows this thread owns: n = 32q + lane (+128 for the second half)
+    constexpr int NH = NS / 128;
+    float Hs[NH][64];
+    {
+      const int n0 = 32 * q + lane;
+#pragma unroll
+      for (int hf = 0; hf < NH; ++hf) {
+        const int n = n0 + 128 * hf;
+#pragma unroll
+        for (int p = 0; p < 64; ++p)
+          Hs[hf][p] = a.h0 ? a.h0[((b * a.H + h) * 64 + p) * NS + n] : 0.f;
+        // bf16 copy, row n of the [N][64] MN-major operand
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint4 v;
+          v.x = pack_bf16x2(Hs[hf][8 * j + 0], Hs[hf][8 * j + 1]);
+          v.y = pack_bf16x2(Hs[hf][8 * j + 2], Hs[hf][8 * j + 3]);
+          v.z = pack_bf16x2(Hs[hf][8 * j + 4], Hs[hf][8 * j + 5]);
+          v.w = pack_bf16x2(Hs[hf][8 * j + 6], Hs[hf][8 * j + 7]);
+          *reinterpret_cast<uint4*>(sm + K::oH + sw128((uint32_t)n * 128 + j * 16)) = v;
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&s.h_ready);
+    }
+    const int seq_first = a.seq ? a.seq[rowbase] : 0;
+    // dt (and seq id) for the next chunk are fetched one chunk ahead
+    float dt_next = 0.f;
+    int seq_next = 0;
+    if (wt < 64 && wt < a.L) {
+      dt_next = a.dt[(rowbase + wt) * a.H + h];
+      seq_next = a.seq ? a.seq[rowbase + wt] : 0;
+    }
+    bool failed = false;
+    for (int c = 0; c < nc; ++c) {
+      // agreement point: the 128 compute threads leave the loop together, so
+      // no thread is left waiting at a named barrier for one that has gone
+      if (named_barrier_any(2, 128, failed)) {
+        failed = true;
+        break;
+      }
+      const uint32_t par = c & 1;
+      const int t0 = c * 64;
+      const int nvalid = (int)((int64_t)(c + 1) * 64 <= a.L ? 64 : a.L - t0);
+      const int e = nvalid - 1;
+      // ---- in-chunk cumulative sum of dt*A (threads 0..63 = warps 2, 3)
+      if (wt < 64) {
+        const float dtv = wt < nvalid ? dt_next : 0.f;
+        const int sq = wt < nvalid ? seq_next : -1;
+        if ((int64_t)t0 + 64 + wt < a.L) {
+          dt_next = a.dt[(rowbase + t0 + 64 + wt) * a.H + h];
+          seq_next = a.seq ? a.seq[rowbase + t0 + 64 + wt] : 0;
+        }
+        float v = dtv * a2;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
+        }
+        if (wt == 31) s.warp_tot = v;
+        named_barrier_sync(1, 128);
+        if (wt >= 32) v += s.warp_tot;
+        s.cs2[wt] = v;
+        s.dts[wt] = dtv;
+        s.seqs[wt] = sq;
+      } else {
+        named_barrier_sync(1, 128);
+      }
+      named_barrier_sync(1, 128);
+      const float cs_e = s.cs2[e];
+      const int seq_e = s.seqs[e];
+      const int seq_prev = t0 > 0 ? (a.seq ? a.seq[rowbase + t0 - 1] : 0) : seq_first;
+
+      if (!mbar_wait(&s.full, par, abort_flag, kWaitLimitNs)) {
+        failed = true;
+        continue;
+      }
+      // ---- scale pass: X~[s][p] = x[s][p] * exp2(cs_e - cs_s) dt_s
+      {
+        const int srow = wt >> 1, hf = wt & 1;
+        float w = 0.f;
+        if (srow < nvalid && s.seqs[srow] == seq_e) w = exp2f(cs_e - s.cs2[srow]) * s.dts[srow];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t off = sw128((uint32_t)srow * 128 + (4 * hf + j) * 16);
+          uint4 v = *reinterpret_cast<const uint4*>(sm + K::oX + off);
+          float f0, f1;
+          unpack_bf16x2(v.x, f0, f1);
+          v.x = pack_bf16x2(f0 * w, f1 * w);
+          unpack_bf16x2(v.y, f0, f1);
+          v.y = pack_bf16x2(f0 * w, f1 * w);
+          unpack_bf16x2(v.z, f0, f1);
+          v.z = pack_bf16x2(f0 * w, f1 * w);
+          unpack_bf16x2(v.w, f0, f1);
+          v.w = pack_bf16x2(f0 * w, f1 * w);
+          *reinterpret_cast<uint4*>(sm + K::oXt + off) = v;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&s.xt_ready);
+      }
+      // ---- mask pass: W = CB o decay o mask (+ D on the diagonal)
+      if (!mbar_wait(&s.cb_full, par, abort_flag, kWaitLimitNs)) {
+        failed = true;
+        continue;
+      }
+      tc_fence_after();
+      {
+        uint32_t r[32];
+        SSD_TMEM_LD_16x32bx2_X32_HALF32(tq + K::tCB, r);
+        SSD_TMEM_WAIT_LD_32(r);
+        tc_fence_before();
+        mbar_arrive(&s.cb_free);
+        const int t = 16 * q + (lane & 15);
+        const int s0 = 32 * (lane >> 4);
+        const float cs_t = s.cs2[t];
+        const int seq_t = s.seqs[t];
+        const bool trow = t < nvalid;
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          float w2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int sc = s0 + j + u;
+            float v = 0.f;
+            if (trow && sc <= t && s.seqs[sc] == seq_t)
+              v = __uint_as_float(r[j + u]) * exp2f(cs_t - s.cs2[sc]) * s.dts[sc];
+            if (trow && sc == t) v += dskip;
+            w2[u] = v;
+          }
+          packed[j >> 1] = pack_bf16x2(w2[0], w2[1]);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t off = sw128((uint32_t)t * 128 + (4 * (lane >> 4) + j) * 16);
+          *reinterpret_cast<uint4*>(sm + K::oW + off) =
+              make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&s.w_ready);
+      }
+      // ---- state update: H = keep exp2(cs_e) H + S   (S^T rows n = 32q + lane)
+      if (!mbar_wait(&s.s_full, par, abort_flag, kWaitLimitNs)) {
+        failed = true;
+        continue;
+      }
+      tc_fence_after();
+      {
+        const float dec = (seq_e == seq_prev) ? exp2f(cs_e) : 0.f;
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t r[32];
+            SSD_TMEM_LD_32x32b_X32(tq + K::tS + hf * 64 + half * 32, r);
+            SSD_TMEM_WAIT_LD_32(r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              Hs[hf][half * 32 + j] = fmaf(dec, Hs[hf][half * 32 + j], __uint_as_float(r[j]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&s.s_free);
+      }
+      // ---- wait for Yd / Yo (MMA3 of this chunk no longer reads H), publish H
+      if (!mbar_wait(&s.y_full, par, abort_flag, kWaitLimitNs)) {
+        failed = true;
+        continue;
+      }
+      tc_fence_after();
+      if (c + 1 < nc) {
+        const int n0 = 32 * q + lane;
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf) {
+          const int n = n0 + 128 * hf;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint4 v;
+            v.x = pack_bf16x2(Hs[hf][8 * j + 0], Hs[hf][8 * j + 1]);
+            v.y = pack_bf16x2(Hs[hf][8 * j + 2], Hs[hf][8 * j + 3]);
+            v.z = pack_bf16x2(Hs[hf][8 * j + 4], Hs[hf][8 * j + 5]);
+            v.w = pack_bf16x2(Hs[hf][8 * j + 6], Hs[hf][8 * j + 7]);
+            *reinterpret_cast<uint4*>(sm + K::oH + sw128((uint32_t)n * 128 + j * 16)) = v;
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&s.h_ready);
+      }
+      // ---- epilogue: y = Yd + keep_t exp2(cs_t) Yo
+      {
+        uint32_t rd[32], ro[32];
+        SSD_TMEM_LD_16x32bx2_X32_HALF32(tq + K::tYd, rd);
+        SSD_TMEM_WAIT_LD_32(rd);
+        SSD_TMEM_LD_16x32bx2_X32_HALF32(tq + K::tYo, ro);
+        SSD_TMEM_WAIT_LD_32(ro);
+        tc_fence_before();
+        mbar_arrive(&s.y_free);
+        const int t = 16 * q + (lane & 15);
+        const int p0 = 32 * (lane >> 4);
+        if (t < nvalid) {
+          const float sc = (s.seqs[t] == seq_prev) ? exp2f(s.cs2[t]) : 0.f;
+          uint32_t packed[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2)
+            packed[j >> 1] = pack_bf16x2(fmaf(sc, __uint_as_float(ro[j]), __uint_as_float(rd[j])),
+                                         fmaf(sc, __uint_as_float(ro[j + 1]), __uint_as_float(rd[j + 1])));
+          uint4* dst = reinterpret_cast<uint4*>(a.y + ((rowbase + t0 + t) * a.H + h) * 64 + p0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+        }
+      }
+    }
+    if (!failed && a.final_states && !a.seq) {
+      const int n0 = 32 * q + lane;
+#pragma unroll
+      for (int hf = 0; hf < NH; ++hf) {
+        const int n = n0 + 128 * hf;
+        float* dst = a.final_states + ((b * a.H + h) * 64) * NS + n;
+#pragma unroll
+        for (int p = 0; p < 64; ++p) dst[(int64_t)p * NS] = Hs[hf][p];
+      }
+    }
+  }
+
+  if (*abort_flag && tid == 0) atomicExch(a.err, 1);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
+}
+
+// ---------------------------------------------------------------- host side
+template <int NS>
+cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
+  CUtensorMap tx, tb, tc_;
+  if (!make_map_3d(&tx, p.x, p.H * p.P, p.L, p.b) || !make_map_3d(&tb, p.B, p.G * p.N, p.L, p.b) ||
+      !make_map_3d(&tc_, p.C, p.G * p.N, p.L, p.b))
+    return cudaErrorInvalidValue;
+  TcArgs a;
+  a.b = p.b;
+  a.L = p.L;
+  a.H = p.H;
+  a.G = p.G;
+  a.hpg = p.hpg;
+  a.nc = p.nc;
+  a.dt = p.dt;
+  a.A = p.A;
+  a.D = p.D;
+  a.h0 = p.h0;
+  a.seq = p.seq;
+  a.y = static_cast<__nv_bfloat16*>(p.y);
+  a.final_states = p.final_states;
+  a.ok = w.ok;
+  a.err = w.err;
+  cudaError_t e = cudaFuncSetAttribute(k_ssd_fwd_tc<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Cfg<NS>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  k_ssd_fwd_tc<NS><<<(unsigned)(p.b * p.H), Cfg<NS>::kThreads, Cfg<NS>::kSmemBytes, st>>>(tx, tb, tc_, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t tc_workspace_need(const Problem& p) {
+  size_t off = kWsAlign;                                                        // error word
+  off = align_up(off + sizeof(__nv_bfloat16) * (size_t)(p.b * p.nc * p.G * 64 * 64), kWsAlign);  // W'
+  off = align_up(off + (size_t)(p.b * p.nc * p.H), kWsAlign);                   // range flags
+  return off;
+}
+
+TcWorkspace tc_carve(const Problem& p, void* ws) {
+  char* base = static_cast<char*>(ws);
+  TcWorkspace w;
+  w.err = reinterpret_cast<int*>(base);
+  size_t off = kWsAlign;
+  w.wp = reinterpret_cast<__nv_bfloat16*>(base + off);
+  off = align_up(off + sizeof(__nv_bfloat16) * (size_t)(p.b * p.nc * p.G * 64 * 64), kWsAlign);
+  w.ok = reinterpret_cast<uint8_t*>(base + off);
+  return w;
+}
+
+bool tc_supported(const Problem& p, uint32_t flags) {
+  if (flags & SSD_FLAG_GENERIC) return false;
+  if (p.dtype != SSD_BF16) return false;
+  if (p.P != 64 || p.Q != 64) return false;
+  if (p.N != 128 && p.N != 256) return false;
+  if (p.seq) return false;
+  // TMA coordinates are 32-bit
+  if (p.b * p.nc * p.G * 64 >= ((int64_t)1 << 31) || p.L >= ((int64_t)1 << 31)) return false;
+  return true;
+}
+
+size_t tc_workspace_bytes(const Problem& p) { return tc_workspace_need(p); }
+
+int tc_launch_count(const Problem&) { return 3; }
+
+cudaError_t tc_forward(const Problem& p, void* ws, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
+  const TcWorkspace w = tc_carve(p, ws);
+  cudaError_t e = cudaMemsetAsync(w.err, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
+  if ((e = tc_fast_forward(p, w, st)) != cudaSuccess) return e;
+  e = p.N == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st);
+  if (e != cudaSuccess) return e;
+  if (ev1) e = cudaEventRecord(ev1, st);
+  return e;
+}
+
+}  // namespace ssd

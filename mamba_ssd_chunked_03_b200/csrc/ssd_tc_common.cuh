@@ -1,0 +1,72 @@
+// Pieces shared by the tensor-core SSD kernels (ssd_tc.cu, ssd_tc_fast.cu):
+// constants, kernel argument blocks, the workspace carve-up and TMA tensor
+// map creation.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssd_internal.h"
+
+namespace ssd {
+namespace tc {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per bounded wait
+// Largest |cs_t - m| (log2 units, m = the chunk's midpoint cumulative sum)
+// for which the factorised decay is used: 2^100 stays far inside fp32/bf16.
+constexpr float kRangeLog2 = 100.f;
+
+struct CbArgs {
+  int64_t L, H, G, hpg, nc;
+  const float* dt;
+  const float* A;
+  const int32_t* seq;
+  __nv_bfloat16* wp;  // (b, nc, G, 64, 64) masked C B^T
+  uint8_t* ok;        // (b, nc, H) chunk within the factorisable range
+  int* err;
+};
+
+struct FastArgs {
+  int64_t L, H, G, hpg, nc;
+  const float* dt;
+  const float* A;
+  const float* D;
+  const float* h0;
+  __nv_bfloat16* y;
+  float* final_states;
+  const uint8_t* ok;
+  int* err;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void unpack_bf16x2(uint32_t u, float& lo, float& hi) {
+  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
+  lo = __low2float(v);
+  hi = __high2float(v);
+}
+
+// 3-D bf16 tensor map over (outer, rows, inner) with a 64 x 64 x 1 box and
+// 128-byte swizzle; rows past `rows` read as zeros.
+bool make_map_3d(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t outer);
+
+}  // namespace tc
+
+// Workspace of the tensor-core path, carved from the caller's buffer.
+struct TcWorkspace {
+  int* err;               // nonzero after a kernel gave up on a bounded wait
+  __nv_bfloat16* wp;      // masked C B^T per (b, chunk, group)
+  uint8_t* ok;            // per (b, chunk, head) range flags
+};
+
+TcWorkspace tc_carve(const Problem& p, void* ws);
+size_t tc_workspace_need(const Problem& p);
+cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st);
+
+}  // namespace ssd

@@ -1,0 +1,139 @@
+// Test-only probe of the tcgen05 building blocks used by the fused SSD kernel:
+// one CTA computes D = A B^T (A: M x K, B: N x K, bf16, row-major in global
+// memory) with the shared-memory layouts, descriptors, MMA shapes and TMEM
+// load shapes of each step of that kernel, and writes D (M x N, fp32) back in
+// logical order.  The tests compare D with a float64 matmul.
+//
+// mode 0: M=64,  N=64, K=128  A K-major (2 x 64-wide K blocks), B K-major      (C B^T)
+// mode 1: M=64,  N=64, K=64   A K-major,                        B MN-major     (W X)
+// mode 2: M=64,  N=64, K=128  A K-major (2 K blocks),           B MN-major     (C H^T)
+// mode 3: M=128, N=64, K=64   A MN-major (2 x 64-wide M blocks), B MN-major    (B^T X~)
+// modes 0-2 read TMEM with the 16-lane x2 shape, mode 3 with 32x32b.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sm100.cuh"
+
+using namespace ssd::sm100;
+
+namespace {
+
+
+__global__ void __launch_bounds__(128) probe_kernel(int mode, const __nv_bfloat16* __restrict__ A,
+                                                    const __nv_bfloat16* __restrict__ B, float* __restrict__ D,
+                                                    int* __restrict__ err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-align the dynamic smem base
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = smem;                 // 32 KB
+  unsigned char* sB = smem + 32768;         // 16 KB
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  int M = 64, N = 64, K = 128;
+  if (mode == 1) K = 64;
+  if (mode == 3) { M = 128; K = 64; }
+
+  // ---- stage A and B in shared memory with the kernel's layouts
+  for (int i = tid; i < M * K; i += 128) {
+    const int m = i / K, k = i % K;
+    const __nv_bfloat16 v = A[m * K + k];
+    uint32_t off;
+    if (mode == 3) {  // MN-major: blocks of 64 m, rows = k, 128 B per row
+      off = (m / 64) * 8192 + k * 128 + (m % 64) * 2;
+    } else {          // K-major: blocks of 64 k, rows = m, 128 B per row
+      off = (k / 64) * 8192 + m * 128 + (k % 64) * 2;
+    }
+    *reinterpret_cast<__nv_bfloat16*>(sA + sw128(off)) = v;
+  }
+  for (int i = tid; i < N * K; i += 128) {
+    const int n = i / K, k = i % K;
+    const __nv_bfloat16 v = B[n * K + k];
+    uint32_t off;
+    if (mode == 0) {  // K-major: blocks of 64 k, rows = n
+      off = (k / 64) * 8192 + n * 128 + (k % 64) * 2;
+    } else {          // MN-major: rows = k, 64 n per row
+      off = k * 128 + n * 2;
+    }
+    *reinterpret_cast<__nv_bfloat16*>(sB + sw128(off)) = v;
+  }
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (tid == 0) {
+    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+    for (int kk = 0; kk < K / 16; ++kk) {
+      uint64_t ad, bd;
+      uint32_t id;
+      if (mode == 3) {
+        ad = sw128_desc(a0 + kk * 16 * 128, 8192, 1024);
+        bd = sw128_desc(b0 + kk * 16 * 128, 8192, 1024);
+        id = idesc_bf16(128, 64, 1, 1);
+      } else {
+        ad = sw128_desc(a0 + (kk / 4) * 8192 + (kk % 4) * 32, 16, 1024);
+        if (mode == 0) {
+          bd = sw128_desc(b0 + (kk / 4) * 8192 + (kk % 4) * 32, 16, 1024);
+          id = idesc_bf16(64, 64, 0, 0);
+        } else {
+          bd = sw128_desc(b0 + kk * 16 * 128, 8192, 1024);
+          id = idesc_bf16(64, 64, 0, 1);
+        }
+      }
+      mma_bf16_ss(tmem, ad, bd, id, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&bar);
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(&bar, 0, &abort_flag, 1000000000ull);
+  tc_fence_after();
+  if (!ok) {
+    if (tid == 0) *err = 1;
+  } else {
+    const int q = warp;  // TMEM lane quadrant of this warp
+    uint32_t r[32];
+    if (mode == 3) {
+      for (int half = 0; half < 2; ++half) {
+        SSD_TMEM_LD_32x32b_X32(tmem + ((uint32_t)(32 * q) << 16) + half * 32, r);
+        SSD_TMEM_WAIT_LD_32(r);
+        const int m = 32 * q + lane;
+        for (int j = 0; j < 32; ++j) D[m * N + half * 32 + j] = __uint_as_float(r[j]);
+      }
+    } else {
+      SSD_TMEM_LD_16x32bx2_X32_HALF32(tmem + ((uint32_t)(32 * q) << 16), r);
+      SSD_TMEM_WAIT_LD_32(r);
+      const int m = 16 * q + (lane % 16);
+      const int n0 = (lane / 16) * 32;
+      for (int j = 0; j < 32; ++j) D[m * N + n0 + j] = __uint_as_float(r[j]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+}  // namespace
+
+extern "C" __attribute__((visibility("default"))) int tc_probe_mma(int mode, const void* A, const void* B,
+                                                                   float* D, int* err, void* stream) {
+  if (mode < 0 || mode > 3) return 1;
+  const size_t smem = 32768 + 16384 + 1024;
+  if (cudaFuncSetAttribute(probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return 2;
+  probe_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
+      mode, static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), D, err);
+  return cudaGetLastError() == cudaSuccess ? 0 : 3;
+}

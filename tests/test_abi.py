@@ -96,7 +96,7 @@ def test_workspace_checked_before_launch():
 
 
 def test_workspace_size_is_pure_and_monotone():
-    a = base_args()
+    a = base_args(flags=ssd.SSD_FLAG_GENERIC)
     w1 = ssd.lib.ssd_fwd_workspace_size(ctypes.byref(a))
     a.seqlen = 1000
     w2 = ssd.lib.ssd_fwd_workspace_size(ctypes.byref(a))

@@ -125,6 +125,23 @@ def test_generic_flag_matches_default_path():
     assert rel_l2(y1, y2) <= 1e-2 and state_err(f1, f2) <= 1e-2
 
 
+@pytest.mark.parametrize("N", [128, 256])
+def test_strong_decay_heads_take_the_exact_kernel(N):
+    """Heads whose in-chunk decay is too steep for the factorised fast kernel
+    (dt*A ~ -30 per token) are handled by the exact kernel in the same call;
+    the other heads by the fast kernel.  Both must match the oracle."""
+    s = si.SSDShape("steep", 2, 300, 4, 64, N, 2, 64, "bf16", h0_std=0.2, seed=31)
+    d = si.make_inputs(s)
+    d["dt"][:, :, 0] = 2.0
+    d["A"][0] = -16.0
+    d["dt"][0, 100:140, 3] = 1.5   # one steep stretch in one row of head 3
+    d["A"][3] = -12.0
+    y, f = run_gpu(d, 64)
+    yr, fr = run_oracle(d)
+    assert rel_l2(y, yr) <= 1e-2, rel_l2(y, yr)
+    assert state_err(f, fr) <= 1e-2, state_err(f, fr)
+
+
 def test_rejected_call_raises_and_leaves_outputs():
     s = si.SSDShape("r", 1, 64, 2, 64, 64, 1, 64, "bf16", seed=1)
     g = to_dev(si.make_inputs(s))
