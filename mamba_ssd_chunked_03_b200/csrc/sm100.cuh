@@ -48,6 +48,20 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As mbar_test, but a thread whose phase is not complete may sleep up to
+// `hint_ns` waiting for it instead of returning at once, so waiting warps do
+// not take issue slots from working ones.
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 
 // Bounded wait for the phase with the given parity.  Gives up once *abort is
 // set by another thread or after `limit_ns` of waiting, sets *abort and
@@ -56,12 +70,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           uint64_t limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_test(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      *abort = 1;
-      return false;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_test_sleep(bar, parity, 20000)) return true;
+    if ((i & 7) == 0) {  // the abort flag and the clock are checked every 8 tries
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        return false;
+      }
     }
   }
 }

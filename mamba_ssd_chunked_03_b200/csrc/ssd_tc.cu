@@ -1,9 +1,10 @@
 // Exact fused chunked SSD forward on sm_100a tensor cores (tcgen05 + TMEM +
 // TMA).  It forms every intra-chunk decay exp(cs_t - cs_s) separately, so it
-// is valid for any decay; the launch processes only the (batch row, head)
-// units that the fast kernel (ssd_tc_fast.cu) leaves out because some chunk's
-// decay range is too wide to factorise.  The host also owns the tensor-map
-// helper and the workspace carve-up shared by both kernels.
+// is valid for any decay.  It runs after the fast kernel (ssd_tc_fast.cu) as a
+// small persistent grid over the list of (batch row, head) units the fast
+// kernel could not factorise, and overwrites their outputs; with an empty
+// list every CTA exits at once.  This file also holds the tensor-map helper
+// and the workspace carve-up shared by both kernels.
 //
 // One CTA owns one (batch row, head) and walks its chunks in order, keeping
 // the running state on chip, so the only HBM traffic is the inputs and y.
@@ -118,7 +119,8 @@ struct TcArgs {
   const int32_t* seq;
   __nv_bfloat16* y;
   float* final_states;
-  const uint8_t* ok;  // per (b, chunk, head) flags of the fast kernel; may be null
+  const int* failed_count;  // units to process, listed by the fast kernel
+  const int* failed_list;
   int* err;
 };
 
@@ -145,35 +147,15 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
                                                        ~uintptr_t(1023));
   __shared__ Smem s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t unit = blockIdx.x;
-  const int64_t b = unit / a.H, h = unit % a.H;
-  const int64_t g = h / a.hpg;
   const int nc = (int)a.nc;
-
-  // units whose chunks are all within the fast kernel's range are done there
-  if (a.ok) {
-    bool all_ok = true;
-    for (int c = tid; c < nc; c += blockDim.x) all_ok &= a.ok[(b * a.nc + c) * a.H + h] != 0;
-    if (__syncthreads_and(all_ok)) return;
-  }
+  // a small persistent grid walks the list of units the fast kernel could not do
+  const int count = *reinterpret_cast<const volatile int*>(a.failed_count);
+  if ((int)blockIdx.x >= count) return;  // uniform: every thread reads the same count
 
   if (tid == 0) {
-    mbar_init(&s.full, 1);
-    mbar_init(&s.empty, 1);
-    mbar_init(&s.cb_full, 1);
-    mbar_init(&s.s_full, 1);
-    mbar_init(&s.y_full, 1);
-    mbar_init(&s.cb_free, 128);
-    mbar_init(&s.w_ready, 128);
-    mbar_init(&s.xt_ready, 128);
-    mbar_init(&s.h_ready, 128);
-    mbar_init(&s.s_free, 128);
-    mbar_init(&s.y_free, 128);
-    mbar_init(&s.drain, 1);
     // a CTA of this launch already gave up: every wait below returns at once
     s.abort_flag = *reinterpret_cast<volatile int*>(a.err) != 0;
     s.never = 0;
-    fence_mbar_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_b);
     tma_prefetch_desc(&tm_c);
@@ -188,6 +170,27 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
   const uint32_t tmem = s.tmem_base;
   volatile int* abort_flag = &s.abort_flag;
   volatile int* never = &s.never;
+
+  for (int it = blockIdx.x; it < count; it += gridDim.x) {
+  const int64_t unit = a.failed_list[it];
+  const int64_t b = unit / a.H, h = unit % a.H;
+  const int64_t g = h / a.hpg;
+  if (tid == 0) {  // fresh barriers per unit (all earlier phases have completed)
+    mbar_init(&s.full, 1);
+    mbar_init(&s.empty, 1);
+    mbar_init(&s.cb_full, 1);
+    mbar_init(&s.s_full, 1);
+    mbar_init(&s.y_full, 1);
+    mbar_init(&s.cb_free, 128);
+    mbar_init(&s.w_ready, 128);
+    mbar_init(&s.xt_ready, 128);
+    mbar_init(&s.h_ready, 128);
+    mbar_init(&s.s_free, 128);
+    mbar_init(&s.y_free, 128);
+    mbar_init(&s.drain, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -506,10 +509,11 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
     }
   }
 
-  if (*abort_flag && tid == 0) atomicExch(a.err, 1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  }  // units
+  if (*abort_flag && tid == 0) atomicExch(a.err, 1);
   if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
 }
 
@@ -534,21 +538,27 @@ cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
   a.seq = p.seq;
   a.y = static_cast<__nv_bfloat16*>(p.y);
   a.final_states = p.final_states;
-  a.ok = w.ok;
+  a.failed_count = w.failed_count;
+  a.failed_list = w.failed_list;
   a.err = w.err;
   cudaError_t e = cudaFuncSetAttribute(k_ssd_fwd_tc<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Cfg<NS>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  k_ssd_fwd_tc<NS><<<(unsigned)(p.b * p.H), Cfg<NS>::kThreads, Cfg<NS>::kSmemBytes, st>>>(tx, tb, tc_, a);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  const int64_t grid = p.b * p.H < (int64_t)Cfg<NS>::kMinBlocks * sms ? p.b * p.H : (int64_t)Cfg<NS>::kMinBlocks * sms;
+  k_ssd_fwd_tc<NS><<<(unsigned)grid, Cfg<NS>::kThreads, Cfg<NS>::kSmemBytes, st>>>(tx, tb, tc_, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t tc_workspace_need(const Problem& p) {
-  size_t off = kWsAlign;                                                        // error word
+  size_t off = kWsAlign;                                                        // error word, count
   off = align_up(off + sizeof(__nv_bfloat16) * (size_t)(p.b * p.nc * p.G * 64 * 64), kWsAlign);  // W'
-  off = align_up(off + (size_t)(p.b * p.nc * p.H), kWsAlign);                   // range flags
+  off = align_up(off + sizeof(int) * (size_t)(p.b * p.H), kWsAlign);            // failed units
   return off;
 }
 
@@ -556,10 +566,11 @@ TcWorkspace tc_carve(const Problem& p, void* ws) {
   char* base = static_cast<char*>(ws);
   TcWorkspace w;
   w.err = reinterpret_cast<int*>(base);
+  w.failed_count = reinterpret_cast<int*>(base) + 1;
   size_t off = kWsAlign;
   w.wp = reinterpret_cast<__nv_bfloat16*>(base + off);
   off = align_up(off + sizeof(__nv_bfloat16) * (size_t)(p.b * p.nc * p.G * 64 * 64), kWsAlign);
-  w.ok = reinterpret_cast<uint8_t*>(base + off);
+  w.failed_list = reinterpret_cast<int*>(base + off);
   return w;
 }
 
@@ -580,7 +591,7 @@ int tc_launch_count(const Problem&) { return 3; }
 
 cudaError_t tc_forward(const Problem& p, void* ws, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
   const TcWorkspace w = tc_carve(p, ws);
-  cudaError_t e = cudaMemsetAsync(w.err, 0, sizeof(int), st);
+  cudaError_t e = cudaMemsetAsync(w.err, 0, 2 * sizeof(int), st);
   if (e != cudaSuccess) return e;
   if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
   if ((e = tc_fast_forward(p, w, st)) != cudaSuccess) return e;

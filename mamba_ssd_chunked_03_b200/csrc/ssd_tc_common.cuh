@@ -20,12 +20,9 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per bounded wait
 constexpr float kRangeLog2 = 100.f;
 
 struct CbArgs {
-  int64_t L, H, G, hpg, nc;
-  const float* dt;
-  const float* A;
+  int64_t L, G, nc;
   const int32_t* seq;
   __nv_bfloat16* wp;  // (b, nc, G, 64, 64) masked C B^T
-  uint8_t* ok;        // (b, nc, H) chunk within the factorisable range
   int* err;
 };
 
@@ -37,7 +34,8 @@ struct FastArgs {
   const float* h0;
   __nv_bfloat16* y;
   float* final_states;
-  const uint8_t* ok;
+  int* failed_count;  // units whose decay range could not be factorised ...
+  int* failed_list;   // ... listed here for the exact kernel
   int* err;
 };
 
@@ -61,8 +59,9 @@ bool make_map_3d(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, 
 // Workspace of the tensor-core path, carved from the caller's buffer.
 struct TcWorkspace {
   int* err;               // nonzero after a kernel gave up on a bounded wait
+  int* failed_count;      // next to err: both are cleared by one memset per call
   __nv_bfloat16* wp;      // masked C B^T per (b, chunk, group)
-  uint8_t* ok;            // per (b, chunk, head) range flags
+  int* failed_list;       // (b*H) units for the exact kernel
 };
 
 TcWorkspace tc_carve(const Problem& p, void* ws);

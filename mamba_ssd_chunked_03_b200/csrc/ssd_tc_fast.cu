@@ -9,31 +9,37 @@
 //                             packed sequence, else 0          (bf16, 64 x 64)
 //   (the masked C B^T of the dual form, "22 · Mamba 2 — Transformers are
 //   SSMs" section 3.2), computed once and shared by all heads of the group.
-//   It also flags, per (chunk, head), whether the chunk's in-chunk cumulative
-//   decay stays within +-kRangeLog2 of its midpoint value (see below).
 //
 // k_ssd_fwd_fast (one CTA per (batch row, head), chunks in order, the running
 //   state kept on chip).  With cs_t the in-chunk cumulative sum of dt*A (log2
 //   units) and m = cs at the chunk's midpoint, the decay between tokens s <= t
 //   factorises as exp2(cs_t - cs_s) = u_t v_s / dt_s with
 //       u_t = exp2(cs_t - m),   v_s = exp2(m - cs_s) dt_s,
-//   both within 2^+-kRangeLog2 when the chunk is flagged in range.  Then
+//   both within 2^+-kRangeLog2 when the chunk's cumsum stays that close to m.
+//   Then
 //       X'  = diag(v) X                                      (one scaling pass)
-//       Yd  = W' X' + C (e^m H_c)^T                          (one accumulator)
-//       y_t = u_t Yd_t + D_h x_t
+//       Yd  = (W' + diag(D_h / dt)) X' + C (e^m H_c)^T       (one accumulator)
+//       y_t = u_t Yd_t
 //       S'  = B^T X',   H_{c+1} = exp2(cs_e) H_c + exp2(cs_e - m) S'
 //   which are the four chunked steps of "SSM 家族全景图（下）：Mamba-2 与 Jamba"
-//   section 三.4: the intra-chunk output (W' X' scaled by u), the chunk state
+//   section 三.4 plus the D skip ("从Transformer的二次复杂度困境到Mamba的线性突围",
+//   continuous SSM equations; u_t (D/dt_t) v_t x_t = D x_t since u_t v_t = dt_t):
+//   the intra-chunk output (W' X' scaled by u), the chunk state
 //   (S'), the state passing (H), and the correction from the chunk's true
 //   initial state (the C H^T term, whose per-row factor exp2(cs_t) equals
-//   u_t e^m).  A (batch row, head) unit with any chunk out of range is left to
-//   the exact kernel (ssd_tc.cu), which forms every decay separately.
+//   u_t e^m).  A (batch row, head) unit with any chunk out of that range is
+//   appended to a list; the exact kernel (ssd_tc.cu), which forms every decay
+//   separately, then recomputes those units and overwrites their outputs.
 //
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer (one
-// thread), warps 2-9 compute.  W'/x tiles, Yd, S and the bf16 state copy are
-// double-buffered so chunk c's MMAs overlap chunk c-1's state update and
-// epilogue.  Every wait is bounded; a CTA that times out records the error,
-// drains its copies and MMAs, frees its TMEM and exits.
+// Warp roles (320 threads): warp 0 computes the in-chunk cumulative sums and
+// factor vectors two chunks ahead and issues the TMA loads (x in a 3-deep
+// ring, scaled in place; W' and C 2-deep; B one tile; each refilled as soon as
+// its last reader is done);
+// warp 1 issues the MMAs (one thread); warps 2-9 scale x, update the state and
+// write y.  Yd and S are double-buffered in TMEM so chunk c's MMAs
+// overlap chunk c-1's state update and epilogue.  Every wait is bounded; a
+// CTA that times out records the error, drains its copies and MMAs, frees its
+// TMEM and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -116,28 +122,6 @@ __global__ void __launch_bounds__(128) k_chunk_cb(const __grid_constant__ CUtens
   }
   __syncwarp();
 
-  // per-(chunk, head) range flags: warp w handles heads w, w+4, ... of the group
-  for (int64_t hh = warp; hh < a.hpg; hh += 4) {
-    const int64_t h = g * a.hpg + hh;
-    const float a2 = a.A[h] * kLog2e;
-    float x0 = 0.f, x1 = 0.f;
-    const int i0 = 2 * lane, i1 = 2 * lane + 1;
-    if (i0 < nvalid) x0 = a.dt[(rowbase + t0 + i0) * a.H + h] * a2;
-    if (i1 < nvalid) x1 = a.dt[(rowbase + t0 + i1) * a.H + h] * a2;
-    float v = x0 + x1;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float u = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += u;
-    }
-    const float cs1 = v, cs0 = v - x1;  // inclusive sums at tokens 2l+1 and 2l
-    const float mid = __shfl_sync(0xffffffffu, cs1, 15);  // token 31
-    float dev = fmaxf(fabsf(cs0 - mid), fabsf(cs1 - mid));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
-    if (lane == 0) a.ok[(b * a.nc + c) * a.H + h] = (dev <= kRangeLog2) ? 1 : 0;
-  }
-
   // W' = masked C B^T -> bf16, row-major 64 x 64 per (b, c, g)
   const bool ok = mbar_wait(&bar_mma, 0, abort_p, kWaitLimitNs);
   tc_fence_after();
@@ -179,13 +163,12 @@ struct FastCfg {
   static constexpr int NB = NS / 64, NH = NS / 128;
   static constexpr int kThreads = 320;
   static constexpr uint32_t kTile = 8192;
-  static constexpr uint32_t oW = 0;                    // [2] W' tiles
-  static constexpr uint32_t oX = oW + 2 * kTile;       // [2] x tiles
-  static constexpr uint32_t oC = oX + 2 * kTile;       // C, NB tiles
-  static constexpr uint32_t oB = oC + NB * kTile;      // B, NB tiles
-  static constexpr uint32_t oXp = oB + NB * kTile;     // X' = diag(v) x
-  static constexpr uint32_t oH = oXp + kTile;          // [2] bf16 e^m H, NB tiles each
-  static constexpr uint32_t oEnd = oH + 2 * NB * kTile;
+  static constexpr uint32_t oX = 0;                          // [3] x tiles, scaled in place to X'
+  static constexpr uint32_t oW = oX + 3 * kTile;             // [2] W' tiles
+  static constexpr uint32_t oB = oW + 2 * kTile;             // B, NB tiles
+  static constexpr uint32_t oC = oB + NB * kTile;            // [2] C, NB tiles each
+  static constexpr uint32_t oH = oC + 2 * NB * kTile;        // bf16 e^m H, NB tiles
+  static constexpr uint32_t oEnd = oH + NB * kTile;
   static constexpr uint32_t kSmemBytes = oEnd + 1024;
   // TMEM columns: Yd[2] (M = 64 layout) then S^T[2] (M = 128 rows per half)
   static constexpr uint32_t tYd0 = 0, tS0 = 128;
@@ -195,17 +178,17 @@ struct FastCfg {
 };
 
 struct __align__(8) FastSmem {
-  uint64_t full_x[2], empty_x[2], full_cb, cb_free, xp_ready, xp_free;
-  uint64_t s_full[2], s_free[2], h_ready[2], h_free[2], y_full[2], y_free[2];
-  uint64_t drain;
+  uint64_t full_x[3], x_empty[3], full_w[2], w_empty[2], full_b, b_free, full_c[2], c_free[2];
+  uint64_t scan_full[4], scan_empty[4], xp_ready, h_ready, h_free;
+  uint64_t s_full[2], s_free[2], y_full[2], y_free[2], drain;
   uint32_t tmem_base;
   int abort_flag;
   int never;
-  float cs2[64];
-  float u[2][64];
-  float v[64];
-  float sc[2][4];  // per chunk parity: E = 2^m, f = 2^(cs_e - m), d = 2^cs_e
-  float warp_tot;
+  int unit_bad;
+  float u[4][64];   // per scan slot: exp2(cs_t - m)
+  float v[4][64];   // per scan slot: exp2(m - cs_s) dt_s
+  float dt[4][64];  // per scan slot: dt (0 past the end of the sequence)
+  float sc[4][4];   // per scan slot: E = 2^m, f = 2^(cs_e - m), d = 2^cs_e
 };
 
 template <int NS>
@@ -223,30 +206,36 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
   const int64_t b = unit / a.H, h = unit % a.H;
   const int64_t g = h / a.hpg;
   const int nc = (int)a.nc;
-
-  // units with any chunk out of the factorisable range belong to the exact kernel
-  bool in_range = true;
-  for (int c = tid; c < nc; c += blockDim.x) in_range &= a.ok[(b * a.nc + c) * a.H + h] != 0;
-  if (!__syncthreads_and(in_range)) return;
+  const int64_t rowbase = b * a.L;
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s.scan_full[i], 32);
+      mbar_init(&s.scan_empty[i], 256);
+    }
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&s.full_x[i], 1);
-      mbar_init(&s.empty_x[i], 1 + 256);
+      mbar_init(&s.x_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.full_c[i], 1);
+      mbar_init(&s.c_free[i], 1);
+      mbar_init(&s.full_w[i], 1);
+      mbar_init(&s.w_empty[i], 1);
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.s_free[i], 256);
-      mbar_init(&s.h_ready[i], 256);
-      mbar_init(&s.h_free[i], 1);
       mbar_init(&s.y_full[i], 1);
       mbar_init(&s.y_free[i], 256);
     }
-    mbar_init(&s.full_cb, 1);
-    mbar_init(&s.cb_free, 1);
+    mbar_init(&s.full_b, 1);
+    mbar_init(&s.b_free, 1);
     mbar_init(&s.xp_ready, 256);
-    mbar_init(&s.xp_free, 1);
+    mbar_init(&s.h_ready, 256);
+    mbar_init(&s.h_free, 1);
     mbar_init(&s.drain, 1);
     s.abort_flag = *reinterpret_cast<volatile int*>(a.err) != 0;
     s.never = 0;
+    s.unit_bad = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_b);
@@ -265,43 +254,136 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
   volatile int* never = &s.never;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int last_x = -1, last_cb = -1;
-      for (int c = 0; c < nc; ++c) {
-        const int i = c & 1;
-        const int t0 = c * 64;
-        if (c >= 2 && !mbar_wait(&s.empty_x[i], ((c - 2) >> 1) & 1, abort_flag, kWaitLimitNs)) break;
-        mbar_arrive_expect_tx(&s.full_x[i], 2 * K::kTile);
-        tma_load_3d(sm + K::oW + i * K::kTile, &tm_w, &s.full_x[i], 0, (int)(((b * a.nc + c) * a.G + g) * 64), 0);
-        tma_load_3d(sm + K::oX + i * K::kTile, &tm_x, &s.full_x[i], (int)(h * 64), t0, (int)b);
-        last_x = c;
-        if (c >= 1 && !mbar_wait(&s.cb_free, (c - 1) & 1, abort_flag, kWaitLimitNs)) break;
-        mbar_arrive_expect_tx(&s.full_cb, 2 * K::NB * K::kTile);
-        for (int j = 0; j < K::NB; ++j) {
-          tma_load_3d(sm + K::oC + j * K::kTile, &tm_c, &s.full_cb, (int)(g * NS + 64 * j), t0, (int)b);
-          tma_load_3d(sm + K::oB + j * K::kTile, &tm_b, &s.full_cb, (int)(g * NS + 64 * j), t0, (int)b);
+    // ------------------------------------------------ scan + TMA producer warp
+    const float a2 = a.A[h] * kLog2e;
+    float p0 = 0.f, p1 = 0.f;  // dt of tokens 2*lane, 2*lane+1 of the next chunk to scan
+    auto load_dt = [&](int c) {
+      const int64_t t = (int64_t)c * 64 + 2 * lane;
+      p0 = (c < nc && t < a.L) ? a.dt[(rowbase + t) * a.H + h] : 0.f;
+      p1 = (c < nc && t + 1 < a.L) ? a.dt[(rowbase + t + 1) * a.H + h] : 0.f;
+    };
+    load_dt(0);
+    int scanned = 0;
+    // in-chunk cumulative sum (log2 units), factor vectors and chunk scalars
+    auto scan_next = [&]() -> bool {
+      const int c = scanned;
+      const int slot = c & 3;
+      if (c >= 4 && !mbar_wait(&s.scan_empty[slot], ((c - 4) >> 2) & 1, abort_flag, kWaitLimitNs)) return false;
+      const float d0 = p0, d1 = p1;
+      load_dt(c + 1);
+      const float x0 = d0 * a2, x1 = d1 * a2;
+      float v = x0 + x1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      const float cs1 = v, cs0 = v - x1;
+      const float m = __shfl_sync(0xffffffffu, cs1, 15);  // token 31
+      const int nvalid = (int)((int64_t)(c + 1) * 64 <= a.L ? 64 : a.L - (int64_t)c * 64);
+      const int e = nvalid - 1;
+      const float cse = __shfl_sync(0xffffffffu, (e & 1) ? cs1 : cs0, e >> 1);
+      float dev = fmaxf(fabsf(cs0 - m), fabsf(cs1 - m));
+      // D x_t is carried through u_t v_t = dt_t, which needs dt_t != 0
+      if ((2 * lane < nvalid && d0 == 0.f) || (2 * lane + 1 < nvalid && d1 == 0.f)) dev = INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
+      if (!(dev <= kRangeLog2) && lane == 0) s.unit_bad = 1;
+      s.u[slot][2 * lane] = exp2f(cs0 - m);
+      s.u[slot][2 * lane + 1] = exp2f(cs1 - m);
+      s.v[slot][2 * lane] = exp2f(m - cs0) * d0;
+      s.v[slot][2 * lane + 1] = exp2f(m - cs1) * d1;
+      s.dt[slot][2 * lane] = d0;
+      s.dt[slot][2 * lane + 1] = d1;
+      if (lane == 0) {
+        s.sc[slot][0] = exp2f(m);
+        s.sc[slot][1] = exp2f(cse - m);
+        s.sc[slot][2] = exp2f(cse);
+      }
+      mbar_arrive(&s.scan_full[slot]);
+      ++scanned;
+      return true;
+    };
+    int last_x = -1, last_w = -1, last_b = -1, last_c = -1;
+    auto issue_x = [&](int c) {
+      const int sl = c % 3;
+      mbar_arrive_expect_tx(&s.full_x[sl], K::kTile);
+      tma_load_3d(sm + K::oX + sl * K::kTile, &tm_x, &s.full_x[sl], (int)(h * 64), c * 64, (int)b);
+      last_x = c;
+    };
+    auto issue_w = [&](int c) {
+      mbar_arrive_expect_tx(&s.full_w[c & 1], K::kTile);
+      tma_load_3d(sm + K::oW + (c & 1) * K::kTile, &tm_w, &s.full_w[c & 1], 0,
+                  (int)(((b * a.nc + c) * a.G + g) * 64), 0);
+      last_w = c;
+    };
+    auto issue_b = [&](int c) {
+      mbar_arrive_expect_tx(&s.full_b, K::NB * K::kTile);
+      for (int j = 0; j < K::NB; ++j)
+        tma_load_3d(sm + K::oB + j * K::kTile, &tm_b, &s.full_b, (int)(g * NS + 64 * j), c * 64, (int)b);
+      last_b = c;
+    };
+    auto issue_c = [&](int c) {
+      uint64_t* bar = &s.full_c[c & 1];
+      mbar_arrive_expect_tx(bar, K::NB * K::kTile);
+      for (int j = 0; j < K::NB; ++j)
+        tma_load_3d(sm + K::oC + ((c & 1) * K::NB + j) * K::kTile, &tm_c, bar, (int)(g * NS + 64 * j), c * 64,
+                    (int)b);
+      last_c = c;
+    };
+    bool ok = true;
+    for (int k = 0; k < 2 && k < nc && ok; ++k) ok = scan_next();
+    if (lane == 0 && ok) {
+      for (int c = 0; c < 3 && c < nc; ++c) issue_x(c);
+      for (int c = 0; c < 2 && c < nc; ++c) {
+        issue_w(c);
+        issue_c(c);
+      }
+      issue_b(0);
+    }
+    // each resource of chunk c is refilled for a later chunk as soon as its
+    // last reader is done: W' after W' X', B and x (scaled in place) after
+    // B^T X', C after C H^T
+    for (int c = 0; c < nc && ok; ++c) {
+      if (scanned < nc) ok = scan_next();  // chunk c + 2
+      if (lane == 0 && ok) {
+        if (c + 2 < nc) {
+          ok = mbar_wait(&s.w_empty[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
+          if (ok) issue_w(c + 2);
         }
-        last_cb = c;
+        if (ok && c + 1 < nc) {
+          ok = mbar_wait(&s.b_free, c & 1, abort_flag, kWaitLimitNs);
+          if (ok) issue_b(c + 1);
+        }
+        if (ok && c + 3 < nc) {
+          ok = mbar_wait(&s.x_empty[c % 3], (c / 3) & 1, abort_flag, kWaitLimitNs);
+          if (ok) issue_x(c + 3);
+        }
+        if (ok && c + 2 < nc) {
+          ok = mbar_wait(&s.c_free[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
+          if (ok) issue_c(c + 2);
+        }
       }
-      if (*abort_flag) {  // let this CTA's own copies land before its smem is released
-        if (last_x >= 0) mbar_wait(&s.full_x[last_x & 1], (last_x >> 1) & 1, never, kWaitLimitNs);
-        if (last_cb >= 0) mbar_wait(&s.full_cb, last_cb & 1, never, kWaitLimitNs);
-      }
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (lane == 0 && *abort_flag) {  // let this CTA's own copies land before its smem is released
+      if (last_x >= 0) mbar_wait(&s.full_x[last_x % 3], (last_x / 3) & 1, never, kWaitLimitNs);
+      if (last_w >= 0) mbar_wait(&s.full_w[last_w & 1], (last_w >> 1) & 1, never, kWaitLimitNs);
+      if (last_b >= 0) mbar_wait(&s.full_b, last_b & 1, never, kWaitLimitNs);
+      if (last_c >= 0) mbar_wait(&s.full_c[last_c & 1], (last_c >> 1) & 1, never, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t aW = smem_u32(sm + K::oW), aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB);
-      const uint32_t aXp = smem_u32(sm + K::oXp), aH = smem_u32(sm + K::oH);
+      const uint32_t aX = smem_u32(sm + K::oX), aH = smem_u32(sm + K::oH);
       constexpr uint32_t id_64 = idesc_bf16(64, 64, 0, 1);    // A K-major, B MN-major, M = 64
       constexpr uint32_t id_st = idesc_bf16(128, 64, 1, 1);   // both MN-major, M = 128
       for (int c = 0; c < nc; ++c) {
         const int i = c & 1;
-        const uint32_t pb = (c >> 1) & 1, ps = c & 1, pp = ((c - 2) >> 1) & 1;
-        bool ok = mbar_wait(&s.full_x[i], pb, abort_flag, kWaitLimitNs);
-        ok = ok && mbar_wait(&s.xp_ready, ps, abort_flag, kWaitLimitNs);
-        ok = ok && mbar_wait(&s.full_cb, ps, abort_flag, kWaitLimitNs);
+        const uint32_t ph = (c >> 1) & 1, p1 = c & 1, pp = ((c - 2) >> 1) & 1;
+        bool ok = mbar_wait(&s.full_w[i], ph, abort_flag, kWaitLimitNs);
+        ok = ok && mbar_wait(&s.xp_ready, p1, abort_flag, kWaitLimitNs);
         if (c >= 2) {
           ok = ok && mbar_wait(&s.y_free[i], pp, abort_flag, kWaitLimitNs);
           ok = ok && mbar_wait(&s.s_free[i], pp, abort_flag, kWaitLimitNs);
@@ -310,33 +392,39 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
         tc_fence_after();
         const uint32_t yd = tmem + K::tYd0 + 64 * i;
         const uint32_t st = tmem + K::tS0 + K::kSCols * i;
+        const uint32_t aXc = aX + (c % 3) * K::kTile;  // X' of this chunk
         // Yd = W' X'   (K = 64 tokens)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16_ss(yd, sw128_desc(aW + i * K::kTile + kk * 32, 16, 1024),
-                      sw128_desc(aXp + kk * 2048, K::kTile, 1024), id_64, kk > 0);
+                      sw128_desc(aXc + kk * 2048, K::kTile, 1024), id_64, kk > 0);
+        mma_commit(&s.w_empty[i]);
         // S'^T = B^T X'   (M = 128 state rows per half, K = 64 tokens)
+        if (!mbar_wait(&s.full_b, p1, abort_flag, kWaitLimitNs)) break;
+        tc_fence_after();
 #pragma unroll
         for (int hf = 0; hf < K::NH; ++hf)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_ss(st + 64 * hf, sw128_desc(aB + hf * 2 * K::kTile + kk * 2048, K::kTile, 1024),
-                        sw128_desc(aXp + kk * 2048, K::kTile, 1024), id_st, kk > 0);
+                        sw128_desc(aXc + kk * 2048, K::kTile, 1024), id_st, kk > 0);
         mma_commit(&s.s_full[i]);
-        mma_commit(&s.xp_free);
+        mma_commit(&s.b_free);
+        mma_commit(&s.x_empty[c % 3]);
         // Yd += C (e^m H_c)^T   (K = N)
-        if (!mbar_wait(&s.h_ready[i], pb, abort_flag, kWaitLimitNs)) break;
+        ok = mbar_wait(&s.h_ready, p1, abort_flag, kWaitLimitNs);
+        ok = ok && mbar_wait(&s.full_c[i], ph, abort_flag, kWaitLimitNs);
+        if (!ok) break;
         tc_fence_after();
+        const uint32_t aCi = aC + i * K::NB * K::kTile;
 #pragma unroll
         for (int kk = 0; kk < NS / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * K::kTile + (kk & 3) * 32;
-          mma_bf16_ss(yd, sw128_desc(aC + koff, 16, 1024),
-                      sw128_desc(aH + i * K::NB * K::kTile + kk * 2048, K::kTile, 1024), id_64, 1);
+          mma_bf16_ss(yd, sw128_desc(aCi + koff, 16, 1024), sw128_desc(aH + kk * 2048, K::kTile, 1024), id_64, 1);
         }
         mma_commit(&s.y_full[i]);
-        mma_commit(&s.h_free[i]);
-        mma_commit(&s.cb_free);
-        mma_commit(&s.empty_x[i]);
+        mma_commit(&s.h_free);
+        mma_commit(&s.c_free[i]);
       }
       mma_commit(&s.drain);
       mbar_wait(&s.drain, 0, never, kWaitLimitNs);
@@ -347,9 +435,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     const int q = warp & 3;             // TMEM lane quadrant
     const int hq = (warp - 2) >> 2;     // which half of the 64 columns
     const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
-    const float a2 = a.A[h] * kLog2e;
     const float dskip = a.D ? a.D[h] : 0.f;
-    const int64_t rowbase = b * a.L;
     const int n0 = 32 * q + lane;       // state row(s): n0 (+128)
     const int pc0 = 32 * hq;            // state columns [pc0, pc0 + 32)
     float H[K::NH][32];
@@ -358,10 +444,6 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
 #pragma unroll
       for (int j = 0; j < 32; ++j)
         H[hf][j] = a.h0 ? a.h0[((b * a.H + h) * 64 + pc0 + j) * NS + n0 + 128 * hf] : 0.f;
-
-    float dt_next = 0.f;
-    if (wt < 64 && wt < a.L) dt_next = a.dt[(rowbase + wt) * a.H + h];
-    float d_prev = 0.f, f_prev = 0.f;  // chunk c-1 scalars
     bool failed = false;
 
     for (int c = 0; c <= nc; ++c) {
@@ -369,116 +451,88 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
         failed = true;
         break;
       }
-      float E_c = 0.f;
       if (c < nc) {
-        const int i = c & 1;
-        const int t0 = c * 64;
-        const int nvalid = (int)((int64_t)(c + 1) * 64 <= a.L ? 64 : a.L - t0);
-        // ---- in-chunk cumulative sum and the factor vectors u, v
-        if (wt < 64) {
-          const float dtv = wt < nvalid ? dt_next : 0.f;
-          if ((int64_t)t0 + 64 + wt < a.L) dt_next = a.dt[(rowbase + t0 + 64 + wt) * a.H + h];
-          float x = dtv * a2;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const float u = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += u;
-          }
-          if (wt == 31) s.warp_tot = x;
-          named_barrier_sync(1, 256);
-          if (wt >= 32) x += s.warp_tot;
-          s.cs2[wt] = x;
-          named_barrier_sync(1, 256);
-          const float m = s.cs2[31];
-          const float cse = s.cs2[nvalid - 1];
-          s.u[i][wt] = exp2f(x - m);
-          s.v[wt] = exp2f(m - x) * dtv;
-          if (wt == 0) {
-            s.sc[i][0] = exp2f(m);
-            s.sc[i][1] = exp2f(cse - m);
-            s.sc[i][2] = exp2f(cse);
-          }
-        } else {
-          named_barrier_sync(1, 256);
-          named_barrier_sync(1, 256);
-        }
-        named_barrier_sync(1, 256);
-        E_c = s.sc[i][0];
-        // ---- X' = diag(v) x for chunk c
-        if (!mbar_wait(&s.full_x[i], (c >> 1) & 1, abort_flag, kWaitLimitNs) ||
-            (c >= 1 && !mbar_wait(&s.xp_free, (c - 1) & 1, abort_flag, kWaitLimitNs))) {
+        // ---- X' = diag(v) x for chunk c (in place), and D folded into W's diagonal
+        const int sl = c & 3, ix = c % 3, iw = c & 1;
+        if (!mbar_wait(&s.scan_full[sl], (c >> 2) & 1, abort_flag, kWaitLimitNs) ||
+            !mbar_wait(&s.full_x[ix], (c / 3) & 1, abort_flag, kWaitLimitNs) ||
+            !mbar_wait(&s.full_w[iw], (c >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           continue;
         }
-        {
-          const int srow = wt >> 2, j4 = wt & 3;
-          const float w = s.v[srow];
+        const int srow = wt >> 2, j4 = wt & 3;
+        const __nv_bfloat162 w2 = __float2bfloat162_rn(s.v[sl][srow]);
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            const uint32_t off = sw128((uint32_t)srow * 128 + (2 * j4 + jj) * 16);
-            uint4 vv = *reinterpret_cast<const uint4*>(sm + K::oX + i * K::kTile + off);
-            float f0, f1;
-            unpack_bf16x2(vv.x, f0, f1);
-            vv.x = pack_bf16x2(f0 * w, f1 * w);
-            unpack_bf16x2(vv.y, f0, f1);
-            vv.y = pack_bf16x2(f0 * w, f1 * w);
-            unpack_bf16x2(vv.z, f0, f1);
-            vv.z = pack_bf16x2(f0 * w, f1 * w);
-            unpack_bf16x2(vv.w, f0, f1);
-            vv.w = pack_bf16x2(f0 * w, f1 * w);
-            *reinterpret_cast<uint4*>(sm + K::oXp + off) = vv;
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(&s.xp_ready);
+        for (int jj = 0; jj < 2; ++jj) {
+          uint4* px = reinterpret_cast<uint4*>(sm + K::oX + ix * K::kTile +
+                                               sw128((uint32_t)srow * 128 + (2 * j4 + jj) * 16));
+          uint4 vv = *px;
+          __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&vv);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) e2[k] = __hmul2(e2[k], w2);
+          *px = vv;
         }
+        if (wt < 64) {
+          // W'[t][t] += D / dt_t, so that u_t (W' X')_t includes D x_t (u_t v_t = dt_t)
+          const float dtt = s.dt[sl][wt];
+          if (dtt != 0.f && dskip != 0.f) {
+            __nv_bfloat16* dg = reinterpret_cast<__nv_bfloat16*>(
+                sm + K::oW + iw * K::kTile + sw128((uint32_t)wt * 128 + (wt >> 3) * 16) + (wt & 7) * 2);
+            *dg = __float2bfloat16_rn(__bfloat162float(*dg) + dskip / dtt);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&s.xp_ready);
       }
-      // ---- state update for chunk c-1, then publish e^m H_c for chunk c
+      // ---- state update for chunk c-1
       if (c >= 1) {
-        const int ip = (c - 1) & 1;
+        const int ip = (c - 1) & 1, slp = (c - 1) & 3;
         if (!mbar_wait(&s.s_full[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           continue;
         }
         tc_fence_after();
+        const float dd = s.sc[slp][2], ff = s.sc[slp][1];
 #pragma unroll
         for (int hf = 0; hf < K::NH; ++hf) {
           uint32_t r[32];
           SSD_TMEM_LD_32x32b_X32(tq + K::tS0 + K::kSCols * ip + 64 * hf + pc0, r);
           SSD_TMEM_WAIT_LD_32(r);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) H[hf][j] = fmaf(d_prev, H[hf][j], f_prev * __uint_as_float(r[j]));
+          for (int j = 0; j < 32; ++j) H[hf][j] = fmaf(dd, H[hf][j], ff * __uint_as_float(r[j]));
         }
         tc_fence_before();
         mbar_arrive(&s.s_free[ip]);
       }
+      // ---- publish e^m H_c (bf16) for chunk c's C H^T product
       if (c < nc) {
-        const int i = c & 1;
-        if (c >= 2 && !mbar_wait(&s.h_free[i], ((c - 2) >> 1) & 1, abort_flag, kWaitLimitNs)) {
+        if (c >= 1 && !mbar_wait(&s.h_free, (c - 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           continue;
         }
+        const float E = s.sc[c & 3][0];
 #pragma unroll
         for (int hf = 0; hf < K::NH; ++hf) {
           const uint32_t row = (uint32_t)(n0 + 128 * hf);
-          unsigned char* base = sm + K::oH + i * K::NB * K::kTile + row * 128;
+          unsigned char* base = sm + K::oH + row * 128;
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) {
             uint4 vv;
-            vv.x = pack_bf16x2(E_c * H[hf][8 * jj + 0], E_c * H[hf][8 * jj + 1]);
-            vv.y = pack_bf16x2(E_c * H[hf][8 * jj + 2], E_c * H[hf][8 * jj + 3]);
-            vv.z = pack_bf16x2(E_c * H[hf][8 * jj + 4], E_c * H[hf][8 * jj + 5]);
-            vv.w = pack_bf16x2(E_c * H[hf][8 * jj + 6], E_c * H[hf][8 * jj + 7]);
+            vv.x = pack_bf16x2(E * H[hf][8 * jj + 0], E * H[hf][8 * jj + 1]);
+            vv.y = pack_bf16x2(E * H[hf][8 * jj + 2], E * H[hf][8 * jj + 3]);
+            vv.z = pack_bf16x2(E * H[hf][8 * jj + 4], E * H[hf][8 * jj + 5]);
+            vv.w = pack_bf16x2(E * H[hf][8 * jj + 6], E * H[hf][8 * jj + 7]);
             const uint32_t chunk = (uint32_t)(pc0 / 8 + jj);
             *reinterpret_cast<uint4*>(base + ((chunk ^ (row & 7)) << 4)) = vv;
           }
         }
         fence_proxy_async_smem();
-        mbar_arrive(&s.h_ready[i]);
+        mbar_arrive(&s.h_ready);
       }
       // ---- epilogue for chunk c-1: y = u_t Yd + D x
       if (c >= 1) {
-        const int ip = (c - 1) & 1;
-        const int t0p = (c - 1) * 64;
+        const int ip = (c - 1) & 1, slp = (c - 1) & 3;
+        const int64_t t0p = (int64_t)(c - 1) * 64;
         const int nvp = (int)((int64_t)c * 64 <= a.L ? 64 : a.L - t0p);
         if (!mbar_wait(&s.y_full[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
@@ -493,32 +547,16 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
         const int t = 16 * q + (lane & 15);
         const int p0 = 16 * hq + 32 * (lane >> 4);
         if (t < nvp) {
-          const float ut = s.u[ip][t];
-          const unsigned char* xrow = sm + K::oX + ip * K::kTile + (uint32_t)t * 128;
+          const float ut = s.u[slp][t];
           uint32_t packed[8];
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            const uint32_t chunk = (uint32_t)(p0 / 8 + jj);
-            const uint4 xv = *reinterpret_cast<const uint4*>(xrow + ((chunk ^ (t & 7)) << 4));
-            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              float x0, x1;
-              unpack_bf16x2(xw[k], x0, x1);
-              const int j = 8 * jj + 2 * k;
-              packed[4 * jj + k] = pack_bf16x2(fmaf(ut, __uint_as_float(r[j]), dskip * x0),
-                                               fmaf(ut, __uint_as_float(r[j + 1]), dskip * x1));
-            }
-          }
+          for (int j = 0; j < 8; ++j)
+            packed[j] = pack_bf16x2(ut * __uint_as_float(r[2 * j]), ut * __uint_as_float(r[2 * j + 1]));
           uint4* dst = reinterpret_cast<uint4*>(a.y + ((rowbase + t0p + t) * a.H + h) * 64 + p0);
           dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         }
-        mbar_arrive(&s.empty_x[ip]);
-      }
-      if (c < nc) {
-        d_prev = s.sc[c & 1][2];
-        f_prev = s.sc[c & 1][1];
+        mbar_arrive(&s.scan_empty[slp]);
       }
     }
     if (!failed && a.final_states) {
@@ -531,10 +569,14 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     }
   }
 
-  if (*abort_flag && tid == 0) atomicExch(a.err, 1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (tid == 0) {
+    if (*abort_flag) atomicExch(a.err, 1);
+    // a chunk's decay range was too wide to factorise: the exact kernel redoes this unit
+    if (s.unit_bad) a.failed_list[atomicAdd(a.failed_count, 1)] = (int)unit;
+  }
   if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
 }
 
@@ -546,15 +588,10 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st)
     return cudaErrorInvalidValue;
   CbArgs ca;
   ca.L = p.L;
-  ca.H = p.H;
   ca.G = p.G;
-  ca.hpg = p.hpg;
   ca.nc = p.nc;
-  ca.dt = p.dt;
-  ca.A = p.A;
   ca.seq = p.seq;
   ca.wp = w.wp;
-  ca.ok = w.ok;
   ca.err = w.err;
   cudaError_t e = cudaFuncSetAttribute(k_chunk_cb<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)CbCfg<NS>::kSmemBytes);
@@ -574,7 +611,8 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st)
   fa.h0 = p.h0;
   fa.y = static_cast<__nv_bfloat16*>(p.y);
   fa.final_states = p.final_states;
-  fa.ok = w.ok;
+  fa.failed_count = w.failed_count;
+  fa.failed_list = w.failed_list;
   fa.err = w.err;
   e = cudaFuncSetAttribute(k_ssd_fwd_fast<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)FastCfg<NS>::kSmemBytes);

@@ -142,6 +142,18 @@ def test_strong_decay_heads_take_the_exact_kernel(N):
     assert state_err(f, fr) <= 1e-2, state_err(f, fr)
 
 
+def test_zero_step_tokens():
+    """dt = 0 tokens (a_t = 1, no input) still get their D x term."""
+    s = si.SSDShape("dt0", 1, 200, 4, 64, 128, 1, 64, "bf16", h0_std=0.1, seed=41)
+    d = si.make_inputs(s)
+    d["dt"][0, 10:20, 1] = 0.0
+    d["dt"][0, 150, 2] = 0.0
+    y, f = run_gpu(d, 64)
+    yr, fr = run_oracle(d)
+    assert rel_l2(y, yr) <= 1e-2, rel_l2(y, yr)
+    assert state_err(f, fr) <= 1e-2, state_err(f, fr)
+
+
 def test_rejected_call_raises_and_leaves_outputs():
     s = si.SSDShape("r", 1, 64, 2, 64, 64, 1, 64, "bf16", seed=1)
     g = to_dev(si.make_inputs(s))
