@@ -1,4 +1,5 @@
-// Pieces shared by the tensor-core SSD kernels (ssd_tc.cu, ssd_tc_fast.cu):
+// Pieces shared by the tensor-core SSD kernels (ssd_tc.cu, ssd_tc_fast.cu,
+// ssd_tc_pair.cu):
 // constants, kernel argument blocks, the workspace carve-up and TMA tensor
 // map creation.
 #pragma once
@@ -67,5 +68,11 @@ struct TcWorkspace {
 TcWorkspace tc_carve(const Problem& p, void* ws);
 size_t tc_workspace_need(const Problem& p);
 cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st);
+
+// two heads per CTA (ssd_tc_pair.cu): N = 128 and an even number of heads per group
+bool tc_pair_supported(const Problem& p);
+cudaError_t tc_pair_launch(const Problem& p, const TcWorkspace& w, const CUtensorMap& tx, const CUtensorMap& tb,
+                           const CUtensorMap& tc_, const CUtensorMap& tw, const CUtensorMap& ty,
+                           const tc::FastArgs& fa, cudaStream_t st);
 
 }  // namespace ssd

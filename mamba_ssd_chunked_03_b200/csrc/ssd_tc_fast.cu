@@ -179,7 +179,9 @@ struct FastCfg {
 
 struct __align__(8) FastSmem {
   uint64_t full_x[3], x_empty[3], full_w[2], w_empty[2], full_b, b_free, full_c[2], c_free[2];
-  uint64_t scan_full[4], scan_empty[4], xp_ready, h_ready, h_free;
+  // xp_ready is a ring like the x tiles it announces, so it cannot complete a
+  // second phase before the MMA thread has seen the first
+  uint64_t scan_full[4], scan_empty[4], xp_ready[3], h_ready, h_free;
   uint64_t s_full[2], s_free[2], y_full[2], y_free[2], drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -216,6 +218,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     for (int i = 0; i < 3; ++i) {
       mbar_init(&s.full_x[i], 1);
       mbar_init(&s.x_empty[i], 1);
+      mbar_init(&s.xp_ready[i], 256);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.full_c[i], 1);
@@ -229,7 +232,6 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     }
     mbar_init(&s.full_b, 1);
     mbar_init(&s.b_free, 1);
-    mbar_init(&s.xp_ready, 256);
     mbar_init(&s.h_ready, 256);
     mbar_init(&s.h_free, 1);
     mbar_init(&s.drain, 1);
@@ -270,7 +272,6 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
       const int slot = c & 3;
       if (c >= 4 && !mbar_wait(&s.scan_empty[slot], ((c - 4) >> 2) & 1, abort_flag, kWaitLimitNs)) return false;
       const float d0 = p0, d1 = p1;
-      load_dt(c + 1);
       const float x0 = d0 * a2, x1 = d1 * a2;
       float v = x0 + x1;
 #pragma unroll
@@ -301,6 +302,9 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
         s.sc[slot][2] = exp2f(cse);
       }
       mbar_arrive(&s.scan_full[slot]);
+      // the next chunk's dt is fetched only now: a release arrive waits for this
+      // thread's loads in flight, which would otherwise stall it for a full load
+      load_dt(c + 1);
       ++scanned;
       return true;
     };
@@ -383,7 +387,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
         const int i = c & 1;
         const uint32_t ph = (c >> 1) & 1, p1 = c & 1, pp = ((c - 2) >> 1) & 1;
         bool ok = mbar_wait(&s.full_w[i], ph, abort_flag, kWaitLimitNs);
-        ok = ok && mbar_wait(&s.xp_ready, p1, abort_flag, kWaitLimitNs);
+        ok = ok && mbar_wait(&s.xp_ready[c % 3], (c / 3) & 1, abort_flag, kWaitLimitNs);
         if (c >= 2) {
           ok = ok && mbar_wait(&s.y_free[i], pp, abort_flag, kWaitLimitNs);
           ok = ok && mbar_wait(&s.s_free[i], pp, abort_flag, kWaitLimitNs);
@@ -482,7 +486,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
           }
         }
         fence_proxy_async_smem();
-        mbar_arrive(&s.xp_ready);
+        mbar_arrive(&s.xp_ready[ix]);
       }
       // ---- state update for chunk c-1
       if (c >= 1) {
@@ -614,6 +618,11 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st)
   fa.failed_count = w.failed_count;
   fa.failed_list = w.failed_list;
   fa.err = w.err;
+  if (NS == 128 && tc_pair_supported(p)) {
+    CUtensorMap ty;
+    if (!make_map_3d(&ty, p.y, p.H * p.P, p.L, p.b)) return cudaErrorInvalidValue;
+    return tc_pair_launch(p, w, tx, tb, tc_, tw, ty, fa, st);
+  }
   e = cudaFuncSetAttribute(k_ssd_fwd_fast<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)FastCfg<NS>::kSmemBytes);
   if (e != cudaSuccess) return e;
