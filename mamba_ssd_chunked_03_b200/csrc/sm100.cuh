@@ -67,12 +67,10 @@ __device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, 
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity.  Gives up once *abort is
-// set by another thread or after `limit_ns` of waiting, sets *abort and
-// returns false; every waiter in the CTA then drains out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint64_t limit_ns) {
-  if (mbar_test(bar, parity)) return true;
+// Slow path of mbar_wait, kept out of line so that the many wait sites of a
+// kernel stay small in the instruction cache.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                   uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_test_sleep(bar, parity, 20000)) return true;
@@ -84,6 +82,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       }
     }
   }
+}
+
+// Bounded wait for the phase with the given parity.  Gives up once *abort is
+// set by another thread or after `limit_ns` of waiting, sets *abort and
+// returns false; every waiter in the CTA then drains out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns) {
+  if (mbar_test(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort, limit_ns);
 }
 
 // ------------------------------------------------------------------ fences
@@ -125,6 +132,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "%4}], [%5];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Bring one box of a tensor into L2 ahead of its load; nothing waits on it.
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 
 // Bulk tensor store of one box from shared memory, tracked by this thread's

@@ -81,6 +81,18 @@ bool make_map_3d(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_map_dt(CUtensorMap* m, const float* dt, int64_t H, int64_t L, int64_t b) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || (H * 4) % 16 != 0) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)b};
+  const cuuint64_t strides[2] = {(cuuint64_t)(H * 4), (cuuint64_t)(H * 4 * L)};
+  const cuuint32_t box[3] = {4, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(dt), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tc
 
 namespace {

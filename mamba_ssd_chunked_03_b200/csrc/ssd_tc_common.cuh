@@ -54,6 +54,9 @@ __device__ __forceinline__ void unpack_bf16x2(uint32_t u, float& lo, float& hi) 
 // 3-D bf16 tensor map over (outer, rows, inner) with a 64 x 64 x 1 box and
 // 128-byte swizzle; rows past `rows` read as zeros.
 bool make_map_3d(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t outer);
+// fp32 tensor map over dt (b, L, H) with a 4-head x 64-token box, no swizzle;
+// needs H * 4 bytes to be a multiple of 16.  Tokens past L read as zeros.
+bool make_map_dt(CUtensorMap* m, const float* dt, int64_t H, int64_t L, int64_t b);
 
 }  // namespace tc
 
@@ -69,10 +72,11 @@ TcWorkspace tc_carve(const Problem& p, void* ws);
 size_t tc_workspace_need(const Problem& p);
 cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st);
 
-// two heads per CTA (ssd_tc_pair.cu): N = 128 and an even number of heads per group
+// two heads per CTA (ssd_tc_pair.cu): N = 128, an even number of heads per
+// group and H a multiple of 4
 bool tc_pair_supported(const Problem& p);
 cudaError_t tc_pair_launch(const Problem& p, const TcWorkspace& w, const CUtensorMap& tx, const CUtensorMap& tb,
                            const CUtensorMap& tc_, const CUtensorMap& tw, const CUtensorMap& ty,
-                           const tc::FastArgs& fa, cudaStream_t st);
+                           const CUtensorMap& tdt, const tc::FastArgs& fa, cudaStream_t st);
 
 }  // namespace ssd

@@ -619,9 +619,10 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st)
   fa.failed_list = w.failed_list;
   fa.err = w.err;
   if (NS == 128 && tc_pair_supported(p)) {
-    CUtensorMap ty;
-    if (!make_map_3d(&ty, p.y, p.H * p.P, p.L, p.b)) return cudaErrorInvalidValue;
-    return tc_pair_launch(p, w, tx, tb, tc_, tw, ty, fa, st);
+    CUtensorMap ty, tdt;
+    if (!make_map_3d(&ty, p.y, p.H * p.P, p.L, p.b) || !make_map_dt(&tdt, p.dt, p.H, p.L, p.b))
+      return cudaErrorInvalidValue;
+    return tc_pair_launch(p, w, tx, tb, tc_, tw, ty, tdt, fa, st);
   }
   e = cudaFuncSetAttribute(k_ssd_fwd_fast<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)FastCfg<NS>::kSmemBytes);
