@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
       const int seq_e = s.seqs[e];
       const int seq_prev = t0 > 0 ? (a.seq ? a.seq[rowbase + t0 - 1] : 0) : seq_first;
 
-      if (!mbar_wait(&s.full, par, abort_flag, kWaitLimitNs)) {
+      if (!mbar_wait_warp(&s.full, par, abort_flag, kWaitLimitNs)) {
         failed = true;
         continue;
       }
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
         mbar_arrive(&s.xt_ready);
       }
       // ---- mask pass: W = CB o decay o mask (+ D on the diagonal)
-      if (!mbar_wait(&s.cb_full, par, abort_flag, kWaitLimitNs)) {
+      if (!mbar_wait_warp(&s.cb_full, par, abort_flag, kWaitLimitNs)) {
         failed = true;
         continue;
       }
@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
         mbar_arrive(&s.w_ready);
       }
       // ---- state update: H = keep exp2(cs_e) H + S   (S^T rows n = 32q + lane)
-      if (!mbar_wait(&s.s_full, par, abort_flag, kWaitLimitNs)) {
+      if (!mbar_wait_warp(&s.s_full, par, abort_flag, kWaitLimitNs)) {
         failed = true;
         continue;
       }
@@ -461,7 +461,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
         mbar_arrive(&s.s_free);
       }
       // ---- wait for Yd / Yo (MMA3 of this chunk no longer reads H), publish H
-      if (!mbar_wait(&s.y_full, par, abort_flag, kWaitLimitNs)) {
+      if (!mbar_wait_warp(&s.y_full, par, abort_flag, kWaitLimitNs)) {
         failed = true;
         continue;
       }

@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(128) k_chunk_cb(const __grid_constant__ CUtens
   __syncwarp();
 
   // W' = masked C B^T -> bf16, row-major 64 x 64 per (b, c, g)
-  const bool ok = mbar_wait(&bar_mma, 0, abort_p, kWaitLimitNs);
+  const bool ok = mbar_wait_warp(&bar_mma, 0, abort_p, kWaitLimitNs);
   tc_fence_after();
   if (ok) {
     const int q = warp;
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     auto scan_next = [&]() -> bool {
       const int c = scanned;
       const int slot = c & 3;
-      if (c >= 4 && !mbar_wait(&s.scan_empty[slot], ((c - 4) >> 2) & 1, abort_flag, kWaitLimitNs)) return false;
+      if (c >= 4 && !mbar_wait_warp(&s.scan_empty[slot], ((c - 4) >> 2) & 1, abort_flag, kWaitLimitNs)) return false;
       const float d0 = p0, d1 = p1;
       const float x0 = d0 * a2, x1 = d1 * a2;
       float v = x0 + x1;
@@ -458,9 +458,9 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
       if (c < nc) {
         // ---- X' = diag(v) x for chunk c (in place), and D folded into W's diagonal
         const int sl = c & 3, ix = c % 3, iw = c & 1;
-        if (!mbar_wait(&s.scan_full[sl], (c >> 2) & 1, abort_flag, kWaitLimitNs) ||
-            !mbar_wait(&s.full_x[ix], (c / 3) & 1, abort_flag, kWaitLimitNs) ||
-            !mbar_wait(&s.full_w[iw], (c >> 1) & 1, abort_flag, kWaitLimitNs)) {
+        if (!mbar_wait_warp(&s.scan_full[sl], (c >> 2) & 1, abort_flag, kWaitLimitNs) ||
+            !mbar_wait_warp(&s.full_x[ix], (c / 3) & 1, abort_flag, kWaitLimitNs) ||
+            !mbar_wait_warp(&s.full_w[iw], (c >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           continue;
         }
@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
       // ---- state update for chunk c-1
       if (c >= 1) {
         const int ip = (c - 1) & 1, slp = (c - 1) & 3;
-        if (!mbar_wait(&s.s_full[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
+        if (!mbar_wait_warp(&s.s_full[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           continue;
         }
@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
       }
       // ---- publish e^m H_c (bf16) for chunk c's C H^T product
       if (c < nc) {
-        if (c >= 1 && !mbar_wait(&s.h_free, (c - 1) & 1, abort_flag, kWaitLimitNs)) {
+        if (c >= 1 && !mbar_wait_warp(&s.h_free, (c - 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           continue;
         }
@@ -538,7 +538,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
         const int ip = (c - 1) & 1, slp = (c - 1) & 3;
         const int64_t t0p = (int64_t)(c - 1) * 64;
         const int nvp = (int)((int64_t)c * 64 <= a.L ? 64 : a.L - t0p);
-        if (!mbar_wait(&s.y_full[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
+        if (!mbar_wait_warp(&s.y_full[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           continue;
         }

@@ -190,8 +190,11 @@ __global__ void __launch_bounds__(512, 1)
         for (int j = 0; j < 2; ++j) tma_prefetch_l2_3d(&tm_x, (int)((h0 + j) * 64), c * 64, (int)b);
       };
       if (!*abort_flag) {
+        #pragma unroll 1
         for (int c = 3; c < 6 && c < nc; ++c) prefetch_x(c);
+        #pragma unroll 1
         for (int c = 0; c < 3 && c < nc; ++c) issue_x(c);  // slot 3 starts free
+        #pragma unroll 1
         for (int c = 0; c < 2 && c < nc; ++c) {
           issue_wb(c);
           issue_c(c);
@@ -199,6 +202,7 @@ __global__ void __launch_bounds__(512, 1)
       }
       bool ok = !*abort_flag;
       // each tile is refilled for a later chunk as soon as its last reader is done
+      #pragma unroll 1
       for (int c = 0; c < nc && ok; ++c) {
         if (c + 2 < nc) {
           ok = mbar_wait(&s.s_full[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
@@ -215,10 +219,13 @@ __global__ void __launch_bounds__(512, 1)
       }
       if (*abort_flag) {  // let this CTA's own copies land before its smem is released
         // (within one ring-depth window every slot holds a single chunk)
+        #pragma unroll 1
         for (int c = last_x - 3 < 0 ? 0 : last_x - 3; c <= last_x; ++c)
           mbar_wait(&s.full_x[c & 3], (c >> 2) & 1, never, kWaitLimitNs);
+        #pragma unroll 1
         for (int c = last_wb - 1 < 0 ? 0 : last_wb - 1; c <= last_wb; ++c)
           mbar_wait(&s.full_wb[c & 1], (c >> 1) & 1, never, kWaitLimitNs);
+        #pragma unroll 1
         for (int c = last_c - 1 < 0 ? 0 : last_c - 1; c <= last_c; ++c)
           mbar_wait(&s.full_c[c & 1], (c >> 1) & 1, never, kWaitLimitNs);
       }
@@ -230,6 +237,7 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t aX = smem_u32(sm + K::oX), aH = smem_u32(sm + K::oH);
       constexpr uint32_t id_y = idesc_bf16(64, 128, 0, 1);    // A K-major, B MN-major (2 heads)
       constexpr uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // both MN-major
+      #pragma unroll 1
       for (int c = 0; c < nc; ++c) {
         const int i = c & 1;
         const uint32_t ph = (c >> 1) & 1;
@@ -288,11 +296,13 @@ __global__ void __launch_bounds__(512, 1)
       last_dt = c;
     };
     if (lane == 0 && !*abort_flag)
+      #pragma unroll 1
       for (int c = 0; c < 8 && c < nc; ++c) issue_dt(c);
+    #pragma unroll 1
     for (int c = 0; c < nc; ++c) {
       const int slot = c & 3;
-      if (c >= 4 && !mbar_wait(&s.scan_empty[slot], ((c - 4) >> 2) & 1, abort_flag, kWaitLimitNs)) break;
-      if (!mbar_wait(&s.full_dt[c & 7], (c >> 3) & 1, abort_flag, kWaitLimitNs)) break;
+      if (c >= 4 && !mbar_wait_warp(&s.scan_empty[slot], ((c - 4) >> 2) & 1, abort_flag, kWaitLimitNs)) break;
+      if (!mbar_wait_warp(&s.full_dt[c & 7], (c >> 3) & 1, abort_flag, kWaitLimitNs)) break;
       const float* dts = reinterpret_cast<const float*>(sm + K::oDt + (c & 7) * K::kDtBox);
       const int nvalid = (int)((int64_t)(c + 1) * 64 <= a.L ? 64 : a.L - (int64_t)c * 64);
       float d[4], cs[4];
@@ -343,11 +353,13 @@ __global__ void __launch_bounds__(512, 1)
       mbar_arrive(&s.scan_full[slot]);
     }
     if (lane == 0 && *abort_flag)  // let the dt copies in flight land
+      #pragma unroll 1
       for (int c = last_dt - 7 < 0 ? 0 : last_dt - 7; c <= last_dt; ++c)
         mbar_wait(&s.full_dt[c & 7], (c >> 3) & 1, never, kWaitLimitNs);
   } else if (warp == 3) {
     // ------------------------------------------------------------ y stores
     if (lane == 0) {
+      #pragma unroll 1
       for (int c = 0; c < nc; ++c) {
         const int sl = c & 3;
         if (!mbar_wait(&s.y_staged[sl], (c >> 2) & 1, abort_flag, kWaitLimitNs)) break;
@@ -365,18 +377,14 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
     const int te = 16 * q + (lane & 15);   // epilogue row (token) of this thread
     const int half = lane >> 4;            // epilogue columns p in [32 half, 32 half + 32)
-    bool failed = false;
-    for (int c = 0; c <= nc; ++c) {
-      if (named_barrier_any(2, 128, failed)) break;
+    #pragma unroll 1
+    for (int c = 1; c <= nc; ++c) {
       // ---- epilogue for chunk c-1, both heads: y = u_t Yd + (D / v_t) X'_t, written over X'
       if (c >= 1) {
         const int ip = (c - 1) & 1, slp = (c - 1) & 3;
-        if (!mbar_wait(&s.mma_done[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
-          failed = true;
-          continue;
-        }
+        if (!mbar_wait_warp(&s.mma_done[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) break;
         tc_fence_after();
-#pragma unroll 1
+        #pragma unroll 1
         for (int j = 0; j < 2; ++j) {
           uint32_t r[32];
           SSD_TMEM_LD_16x32bx2_X32_HALF32(tq + K::tYd0 + 128 * ip + 64 * j, r);
@@ -421,8 +429,8 @@ __global__ void __launch_bounds__(512, 1)
     // 128-byte row in place, at the swizzled positions of its 16-byte columns
     auto scale_chunk = [&](int cc) -> bool {
       const int sl = cc & 3;
-      if (!mbar_wait(&s.scan_full[sl], (cc >> 2) & 1, abort_flag, kWaitLimitNs) ||
-          !mbar_wait(&s.full_x[sl], (cc >> 2) & 1, abort_flag, kWaitLimitNs))
+      if (!mbar_wait_warp(&s.scan_full[sl], (cc >> 2) & 1, abort_flag, kWaitLimitNs) ||
+          !mbar_wait_warp(&s.full_x[sl], (cc >> 2) & 1, abort_flag, kWaitLimitNs))
         return false;
       const __nv_bfloat162 w2 = __float2bfloat162_rn(s.v[sl][j][srow]);
       unsigned char* row = sm + K::oX + (sl * 2 + j) * K::kTile + srow * 128;
@@ -443,17 +451,14 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
     for (int p = 0; p < 64; ++p) H[p] = a.h0 ? a.h0[((b * a.H + h) * 64 + p) * NS + n] : 0.f;
     bool failed = nc > 0 && !scale_chunk(0);
-    for (int c = 0; c <= nc; ++c) {
-      if (named_barrier_any(3 + j, 128, failed)) {
-        failed = true;
-        break;
-      }
+    #pragma unroll 1
+    for (int c = 0; c <= nc && !failed; ++c) {
       // ---- state update for chunk c-1
       if (c >= 1) {
         const int ip = (c - 1) & 1, slp = (c - 1) & 3;
-        if (!mbar_wait(&s.s_full[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
+        if (!mbar_wait_warp(&s.s_full[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
-          continue;
+          break;
         }
         tc_fence_after();
         const float dd = s.sc[slp][j][2], ff = s.sc[slp][j][1];
@@ -472,10 +477,10 @@ __global__ void __launch_bounds__(512, 1)
       // ---- publish e^m H (bf16) for chunk c's C H^T product
       if (c < nc) {
         const int i = c & 1;
-        if (!mbar_wait(&s.scan_full[c & 3], (c >> 2) & 1, abort_flag, kWaitLimitNs) ||
-            (c >= 2 && !mbar_wait(&s.mma_done[i], ((c - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        if (!mbar_wait_warp(&s.scan_full[c & 3], (c >> 2) & 1, abort_flag, kWaitLimitNs) ||
+            (c >= 2 && !mbar_wait_warp(&s.mma_done[i], ((c - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
           failed = true;
-          continue;
+          break;
         }
         const float E = s.sc[c & 3][j][0];
         unsigned char* base = sm + K::oH + (i * 2 + j) * K::kHTile + (uint32_t)n * 128;
@@ -494,7 +499,7 @@ __global__ void __launch_bounds__(512, 1)
       // ---- X' of chunk c+1, which the next MMAs wait for
       if (c + 1 < nc && !scale_chunk(c + 1)) {
         failed = true;
-        continue;
+        break;
       }
     }
     if (!failed && a.final_states) {
