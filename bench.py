@@ -173,6 +173,17 @@ def traffic_from_profiles(kernel_file: str, kernel: str, workload: str):
         return None
 
 
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """The largest of every rank's ``value`` (each rank times its own replica;
+    the job takes as long as its slowest rank).  Without a process group the
+    value is returned as is."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------------------- CPU oracle timing
 
 def oracle_sample(d, shape, target_s: float, max_units=None):
@@ -289,6 +300,7 @@ def main():
     launches_per_call = ssd.launch_count(g["x"], g["B"], shape.chunk_size, g.get("seq_idx"), num_seqs, True,
                                          generic=args.generic)
     path = ssd.kernel_path(g["x"], g["B"], shape.chunk_size, generic=args.generic)
+    main_kernel = ssd.main_kernel(g["x"], g["dt"], g["B"], shape.chunk_size, generic=args.generic)
 
     K = args.steps
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -321,10 +333,7 @@ def main():
     clock_stats = clocks.stop()
     ms = e0.elapsed_time(e1)
     kernel_ms = sum(a.elapsed_time(c) for a, c in kev) / K
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, dev)
 
     # end to end through the public API: pinned host inputs -> device -> fwd -> host
     names = [k for k in ("x", "dt", "A", "B", "C", "D", "initial_states", "seq_idx") if host.get(k) is not None]
@@ -354,10 +363,8 @@ def main():
     a1.record()
     torch.cuda.synchronize()
     e2e_ms = a0.elapsed_time(a1)
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
 
     w = work(shape, num_seqs)
@@ -375,10 +382,11 @@ def main():
         achieved = w["flops"] / (kernel_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "peak_source": peaks["source"]}
-    kfile = "ssd_tc.cu" if path == "tcgen05" else "ssd_generic.cu"
-    roof["kernel"] = "ssd_fwd_tc" if path == "tcgen05" else "generic (all kernels of the call)"
+    kfile = {"k_ssd_fwd_pair": "ssd_tc_pair.cu", "k_ssd_fwd_fast": "ssd_tc_fast.cu"}.get(main_kernel,
+                                                                                      "ssd_generic.cu")
+    roof["kernel"] = main_kernel if path == "tcgen05" else "generic (all kernels of the call)"
     roof["kernel_ms"] = kernel_ms
-    roof["traffic"] = traffic_from_profiles(kfile, path, shape.name)
+    roof["traffic"] = traffic_from_profiles(kfile, main_kernel, shape.name)
     roof["algorithmic_bytes"] = w["bytes"]
     roof["algorithmic_flops"] = w["flops"]
 

@@ -154,6 +154,13 @@ SSD_API int ssd_fwd_launch_count(const ssd_fwd_args* args);
  * ("generic", "tcgen05"), or "invalid". Static string. */
 SSD_API const char* ssd_fwd_path(const ssd_fwd_args* args);
 
+/* Name of the fused kernel that dominates the call on the tensor-core path
+ * ("k_ssd_fwd_pair": two heads per CTA, N = 128, an even number of heads per
+ * group, H a multiple of 4 and dt 16-byte aligned; "k_ssd_fwd_fast": one head
+ * per CTA otherwise), "generic" on the generic path, or "invalid".  It is the
+ * kernel that timing_events bracket.  Static string; no device work. */
+SSD_API const char* ssd_fwd_main_kernel(const ssd_fwd_args* args);
+
 /* Static, human-readable text for a status code. */
 SSD_API const char* ssd_status_string(ssd_status status);
 

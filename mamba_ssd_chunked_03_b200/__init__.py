@@ -59,6 +59,8 @@ def _load() -> ctypes.CDLL:
     L.ssd_fwd_launch_count.restype = ctypes.c_int
     L.ssd_fwd_path.argtypes = [ctypes.POINTER(Args)]
     L.ssd_fwd_path.restype = ctypes.c_char_p
+    L.ssd_fwd_main_kernel.argtypes = [ctypes.POINTER(Args)]
+    L.ssd_fwd_main_kernel.restype = ctypes.c_char_p
     L.ssd_status_string.argtypes = [ctypes.c_int]
     L.ssd_status_string.restype = ctypes.c_char_p
     L.ssd_version.restype = ctypes.c_int
@@ -152,6 +154,13 @@ def launch_count(x, B, chunk_size: int, seq_idx=None, num_seqs=None, final_state
 def kernel_path(x, B, chunk_size: int, generic: bool = False) -> str:
     a = make_args(x, None, None, B, None, chunk_size=chunk_size, generic=generic)
     return lib.ssd_fwd_path(ctypes.byref(a)).decode()
+
+
+def main_kernel(x, dt, B, chunk_size: int, generic: bool = False) -> str:
+    """Name of the fused kernel a call with these tensors is dominated by
+    (the one ``timing_events`` bracket)."""
+    a = make_args(x, dt, None, B, None, chunk_size=chunk_size, generic=generic)
+    return lib.ssd_fwd_main_kernel(ctypes.byref(a)).decode()
 
 
 def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,

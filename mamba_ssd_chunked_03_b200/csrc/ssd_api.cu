@@ -86,6 +86,12 @@ const char* ssd_fwd_path(const ssd_fwd_args* args) {
   return ssd::tc_supported(ssd::resolve(args), args->flags) ? "tcgen05" : "generic";
 }
 
+const char* ssd_fwd_main_kernel(const ssd_fwd_args* args) {
+  if (ssd::check_sizes(args) != SSD_OK) return "invalid";
+  const ssd::Problem p = ssd::resolve(args);
+  return ssd::tc_supported(p, args->flags) ? ssd::tc_main_kernel(p) : "generic";
+}
+
 ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream) {
   ssd_status st = ssd::check_sizes(args);
   if (st != SSD_OK) return st;

@@ -605,12 +605,8 @@ cudaError_t tc_forward(const Problem& p, void* ws, cudaStream_t st, cudaEvent_t 
   const TcWorkspace w = tc_carve(p, ws);
   cudaError_t e = cudaMemsetAsync(w.err, 0, 2 * sizeof(int), st);
   if (e != cudaSuccess) return e;
-  if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
-  if ((e = tc_fast_forward(p, w, st)) != cudaSuccess) return e;
-  e = p.N == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st);
-  if (e != cudaSuccess) return e;
-  if (ev1) e = cudaEventRecord(ev1, st);
-  return e;
+  if ((e = tc_fast_forward(p, w, st, ev0, ev1)) != cudaSuccess) return e;
+  return p.N == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st);
 }
 
 }  // namespace ssd

@@ -70,7 +70,9 @@ struct TcWorkspace {
 
 TcWorkspace tc_carve(const Problem& p, void* ws);
 size_t tc_workspace_need(const Problem& p);
-cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st);
+// chunk C B^T kernel, then the fused kernel, bracketed by ev0 / ev1 if given
+cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0 = nullptr,
+                            cudaEvent_t ev1 = nullptr);
 
 // two heads per CTA (ssd_tc_pair.cu): N = 128, an even number of heads per
 // group and H a multiple of 4

@@ -584,8 +584,9 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
   if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
 }
 
+// ev0 / ev1 (optional) are recorded right before and after the fused kernel.
 template <int NS>
-cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
+cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
   CUtensorMap tx, tb, tc_, tw;
   if (!make_map_3d(&tx, p.x, p.H * p.P, p.L, p.b) || !make_map_3d(&tb, p.B, p.G * p.N, p.L, p.b) ||
       !make_map_3d(&tc_, p.C, p.G * p.N, p.L, p.b) || !make_map_3d(&tw, w.wp, 64, p.b * p.nc * p.G * 64, 1))
@@ -622,20 +623,29 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st)
     CUtensorMap ty, tdt;
     if (!make_map_3d(&ty, p.y, p.H * p.P, p.L, p.b) || !make_map_dt(&tdt, p.dt, p.H, p.L, p.b))
       return cudaErrorInvalidValue;
-    return tc_pair_launch(p, w, tx, tb, tc_, tw, ty, tdt, fa, st);
+    if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
+    if ((e = tc_pair_launch(p, w, tx, tb, tc_, tw, ty, tdt, fa, st)) != cudaSuccess) return e;
+    return ev1 ? cudaEventRecord(ev1, st) : cudaSuccess;
   }
   e = cudaFuncSetAttribute(k_ssd_fwd_fast<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)FastCfg<NS>::kSmemBytes);
   if (e != cudaSuccess) return e;
+  if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
   k_ssd_fwd_fast<NS><<<(unsigned)(p.b * p.H), FastCfg<NS>::kThreads, FastCfg<NS>::kSmemBytes, st>>>(tx, tb, tc_,
                                                                                                       tw, fa);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return ev1 ? cudaEventRecord(ev1, st) : cudaSuccess;
 }
 
 }  // namespace
 
-cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
-  return p.N == 128 ? launch_fast<128>(p, w, st) : launch_fast<256>(p, w, st);
+const char* tc_main_kernel(const Problem& p) {
+  return p.N == 128 && tc_pair_supported(p) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
+}
+
+cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0,
+                            cudaEvent_t ev1) {
+  return p.N == 128 ? launch_fast<128>(p, w, st, ev0, ev1) : launch_fast<256>(p, w, st, ev0, ev1);
 }
 
 }  // namespace ssd

@@ -526,7 +526,10 @@ __global__ void __launch_bounds__(512, 1)
 
 }  // namespace
 
-bool tc_pair_supported(const Problem& p) { return p.N == 128 && p.hpg % 2 == 0 && p.H % 4 == 0; }
+// dt is read by TMA, whose base address must be 16-byte aligned
+bool tc_pair_supported(const Problem& p) {
+  return p.N == 128 && p.hpg % 2 == 0 && p.H % 4 == 0 && reinterpret_cast<uintptr_t>(p.dt) % 16 == 0;
+}
 
 cudaError_t tc_pair_launch(const Problem& p, const TcWorkspace& w, const CUtensorMap& tx, const CUtensorMap& tb,
                            const CUtensorMap& tc_, const CUtensorMap& tw, const CUtensorMap& ty,
