@@ -59,7 +59,7 @@ typedef enum {
   SSD_ERR_UNSUPPORTED = 2,  /* valid arguments outside the implemented shape set */
   SSD_ERR_WORKSPACE = 3,    /* workspace missing or smaller than ssd_fwd_workspace_size() */
   SSD_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed (see cudaGetLastError) */
-  SSD_ERR_TIMEOUT = 5       /* reserved: a bounded device-side wait gave up */
+  SSD_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (ssd_fwd_device_status) */
 } ssd_status;
 
 /* Element type of x, B, C and y.  dt, A, D, initial_states and final_states
@@ -160,6 +160,16 @@ SSD_API const char* ssd_fwd_path(const ssd_fwd_args* args);
  * per CTA otherwise), "generic" on the generic path, or "invalid".  It is the
  * kernel that timing_events bracket.  Static string; no device work. */
 SSD_API const char* ssd_fwd_main_kernel(const ssd_fwd_args* args);
+
+/* After an ssd_fwd call with these arguments: waits for `stream`, then reads
+ * the error word the tensor-core kernels keep at the start of the workspace.
+ * Returns SSD_ERR_TIMEOUT if a bounded device-side wait of that call gave up
+ * (every wait is limited to about a second; the call's outputs are then
+ * undefined, and the next ssd_fwd on the same workspace clears the word),
+ * SSD_OK otherwise; always SSD_OK on the generic path, whose kernels do not
+ * wait on one another.  Synchronous; reads 4 bytes; SSD_ERR_CUDA if the
+ * synchronisation or the read fails.  No counterpart in the pages. */
+SSD_API ssd_status ssd_fwd_device_status(const ssd_fwd_args* args, void* stream);
 
 /* Static, human-readable text for a status code. */
 SSD_API const char* ssd_status_string(ssd_status status);

@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
     L.ssd_fwd_workspace_size.restype = ctypes.c_size_t
     L.ssd_fwd_launch_count.argtypes = [ctypes.POINTER(Args)]
     L.ssd_fwd_launch_count.restype = ctypes.c_int
+    L.ssd_fwd_device_status.argtypes = [ctypes.POINTER(Args), ctypes.c_void_p]
+    L.ssd_fwd_device_status.restype = ctypes.c_int
     L.ssd_fwd_path.argtypes = [ctypes.POINTER(Args)]
     L.ssd_fwd_path.restype = ctypes.c_char_p
     L.ssd_fwd_main_kernel.argtypes = [ctypes.POINTER(Args)]
@@ -139,6 +141,16 @@ def workspace_size(x, B, chunk_size: int, seq_idx=None, num_seqs=None, final_sta
     if final_states:
         a.final_states = 1 << 8  # presence only; the size query does not dereference
     return int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
+
+
+def device_status(x, B, chunk_size: int, workspace: torch.Tensor, generic: bool = False) -> int:
+    """Synchronise the current stream and report whether the last call that
+    used ``workspace`` had a device-side wait give up (``SSD_ERR_TIMEOUT``)
+    or not (``SSD_OK``)."""
+    a = make_args(x, None, None, B, None, chunk_size=chunk_size, generic=generic)
+    a.workspace = workspace.data_ptr()
+    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(lib.ssd_fwd_device_status(ctypes.byref(a), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))
 
 
 def launch_count(x, B, chunk_size: int, seq_idx=None, num_seqs=None, final_states: bool = True,

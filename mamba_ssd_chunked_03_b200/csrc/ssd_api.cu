@@ -86,6 +86,19 @@ const char* ssd_fwd_path(const ssd_fwd_args* args) {
   return ssd::tc_supported(ssd::resolve(args), args->flags) ? "tcgen05" : "generic";
 }
 
+ssd_status ssd_fwd_device_status(const ssd_fwd_args* args, void* stream) {
+  ssd_status st = ssd::check_sizes(args);
+  if (st != SSD_OK) return st;
+  const ssd::Problem p = ssd::resolve(args);
+  if (!ssd::tc_supported(p, args->flags)) return SSD_OK;
+  if (!args->workspace) return SSD_ERR_WORKSPACE;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSD_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, ssd::tc_error_word(p, args->workspace), sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SSD_ERR_CUDA;
+  return word ? SSD_ERR_TIMEOUT : SSD_OK;
+}
+
 const char* ssd_fwd_main_kernel(const ssd_fwd_args* args) {
   if (ssd::check_sizes(args) != SSD_OK) return "invalid";
   const ssd::Problem p = ssd::resolve(args);

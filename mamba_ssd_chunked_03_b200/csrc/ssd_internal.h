@@ -39,6 +39,8 @@ int generic_launch_count(const Problem& p);
 bool tc_supported(const Problem& p, uint32_t flags);
 size_t tc_workspace_bytes(const Problem& p);
 int tc_launch_count(const Problem& p);
+// device address of the tensor-core path's error word inside the workspace
+const int* tc_error_word(const Problem& p, const void* ws);
 // name of the fused kernel the tensor-core path launches for p
 const char* tc_main_kernel(const Problem& p);
 cudaError_t tc_forward(const Problem& p, void* ws, cudaStream_t stream, cudaEvent_t ev0, cudaEvent_t ev1);

@@ -586,6 +586,10 @@ TcWorkspace tc_carve(const Problem& p, void* ws) {
   return w;
 }
 
+const int* tc_error_word(const Problem& p, const void* ws) {
+  return tc_carve(p, const_cast<void*>(ws)).err;
+}
+
 bool tc_supported(const Problem& p, uint32_t flags) {
   if (flags & SSD_FLAG_GENERIC) return false;
   if (p.dtype != SSD_BF16) return false;

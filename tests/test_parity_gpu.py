@@ -117,6 +117,17 @@ def test_chunk_size_invariance_on_gpu():
         assert state_err(f, fr) <= 1e-5, (Q, state_err(f, fr))
 
 
+def test_device_status_reports_no_timeout_after_a_normal_call():
+    s = si.SSDShape("st", 2, 300, 8, 64, 128, 1, 64, "bf16", h0_std=0.1, seed=8)
+    g = to_dev(si.make_inputs(s))
+    assert ssd.main_kernel(g["x"], g["dt"], g["B"], 64) == "k_ssd_fwd_pair"
+    need = ssd.workspace_size(g["x"], g["B"], 64)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")  # the call must clear its error word
+    ssd.fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk_size=64,
+            initial_states=g["initial_states"], workspace=ws)
+    assert ssd.device_status(g["x"], g["B"], 64, ws) == ssd.SSD_OK
+
+
 def test_generic_flag_matches_default_path():
     s = si.SSDShape("g", 2, 333, 4, 64, 128, 1, 64, "bf16", h0_std=0.1, seed=6)
     d = si.make_inputs(s)
