@@ -567,23 +567,32 @@ cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
 
 }  // namespace
 
-size_t tc_workspace_need(const Problem& p) {
-  size_t off = kWsAlign;                                                        // error word, count
-  off = align_up(off + sizeof(__nv_bfloat16) * (size_t)(p.b * p.nc * p.G * 64 * 64), kWsAlign);  // W'
-  off = align_up(off + sizeof(int) * (size_t)(p.b * p.H), kWsAlign);            // failed units
-  return off;
-}
-
-TcWorkspace tc_carve(const Problem& p, void* ws) {
-  char* base = static_cast<char*>(ws);
+// Layout: [err, failed_count, (two-head kernel: flags, pair marks)] cleared per
+// call | W' | failed units | (two-head kernel: state hand-over buffers)
+TcWorkspace tc_carve(const Problem& p, void* ws, size_t* total) {
+  const uintptr_t base = reinterpret_cast<uintptr_t>(ws);
+  const bool pair = tc_pair_shape_ok(p);
   TcWorkspace w;
   w.err = reinterpret_cast<int*>(base);
-  w.failed_count = reinterpret_cast<int*>(base) + 1;
-  size_t off = kWsAlign;
+  w.failed_count = reinterpret_cast<int*>(base + sizeof(int));
+  w.flags = pair ? reinterpret_cast<int*>(base + 2 * sizeof(int)) : nullptr;
+  w.pair_bad = pair ? reinterpret_cast<int*>(base + (2 + 8 * (size_t)kPairGridMax) * sizeof(int)) : nullptr;
+  w.zero_bytes = sizeof(int) * (2 + (pair ? 8 * (size_t)kPairGridMax + (size_t)(p.b * p.H / 2) : 0));
+  size_t off = align_up(w.zero_bytes, kWsAlign);
   w.wp = reinterpret_cast<__nv_bfloat16*>(base + off);
   off = align_up(off + sizeof(__nv_bfloat16) * (size_t)(p.b * p.nc * p.G * 64 * 64), kWsAlign);
   w.failed_list = reinterpret_cast<int*>(base + off);
+  off = align_up(off + sizeof(int) * (size_t)(p.b * p.H), kWsAlign);
+  w.handoff = pair ? reinterpret_cast<float*>(base + off) : nullptr;
+  if (pair) off = align_up(off + sizeof(float) * (size_t)kPairGridMax * kPairHandoffFloats, kWsAlign);
+  if (total) *total = off;
   return w;
+}
+
+size_t tc_workspace_need(const Problem& p) {
+  size_t total = 0;
+  tc_carve(p, nullptr, &total);
+  return total;
 }
 
 const int* tc_error_word(const Problem& p, const void* ws) {
@@ -607,7 +616,7 @@ int tc_launch_count(const Problem&) { return 3; }
 
 cudaError_t tc_forward(const Problem& p, void* ws, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
   const TcWorkspace w = tc_carve(p, ws);
-  cudaError_t e = cudaMemsetAsync(w.err, 0, 2 * sizeof(int), st);
+  cudaError_t e = cudaMemsetAsync(w.err, 0, w.zero_bytes, st);
   if (e != cudaSuccess) return e;
   if ((e = tc_fast_forward(p, w, st, ev0, ev1)) != cudaSuccess) return e;
   return p.N == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st);

@@ -16,8 +16,9 @@ namespace tc {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per bounded wait
-// Largest |cs_t - m| (log2 units, m = the chunk's midpoint cumulative sum)
-// for which the factorised decay is used: 2^100 stays far inside fp32/bf16.
+// Largest |cs_t - r| (log2 units) for the point r the decay factorisation is
+// taken about (the chunk's middle token in ssd_tc_fast.cu, its first in
+// ssd_tc_pair.cu): 2^100 stays far inside fp32/bf16.
 constexpr float kRangeLog2 = 100.f;
 
 struct CbArgs {
@@ -28,7 +29,7 @@ struct CbArgs {
 };
 
 struct FastArgs {
-  int64_t L, H, G, hpg, nc;
+  int64_t L, H, G, hpg, nc, batch;
   const float* dt;
   const float* A;
   const float* D;
@@ -38,7 +39,15 @@ struct FastArgs {
   int* failed_count;  // units whose decay range could not be factorised ...
   int* failed_list;   // ... listed here for the exact kernel
   int* err;
+  // two-head kernel only: state hand-over between the CTAs that share a pair
+  float* handoff;  // [grid][2 heads][128 states][64 p] fp32
+  int* flags;      // [grid][8 state warps]: 1 once that warp's part of the hand-over is written
+  int* pair_bad;   // [b * H / 2]: 1 once a pair was put on the exact kernel's list
 };
+
+// persistent grid of the two-head kernel, at most; per-CTA hand-over size
+constexpr int kPairGridMax = 256;
+constexpr int kPairHandoffFloats = 2 * 128 * 64;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -63,19 +72,26 @@ bool make_map_dt(CUtensorMap* m, const float* dt, int64_t H, int64_t L, int64_t 
 // Workspace of the tensor-core path, carved from the caller's buffer.
 struct TcWorkspace {
   int* err;               // nonzero after a kernel gave up on a bounded wait
-  int* failed_count;      // next to err: both are cleared by one memset per call
+  int* failed_count;      // next to err; err .. zero_bytes is cleared by one memset per call
+  int* flags;             // two-head kernel: hand-over flags (kPairGridMax x 8), or null
+  int* pair_bad;          // two-head kernel: per-pair exact-kernel marks, or null
+  size_t zero_bytes;
   __nv_bfloat16* wp;      // masked C B^T per (b, chunk, group)
   int* failed_list;       // (b*H) units for the exact kernel
+  float* handoff;         // two-head kernel: kPairGridMax x kPairHandoffFloats, or null
 };
 
-TcWorkspace tc_carve(const Problem& p, void* ws);
+// carve the caller's workspace (ws may be null to only size it: *total)
+TcWorkspace tc_carve(const Problem& p, void* ws, size_t* total = nullptr);
 size_t tc_workspace_need(const Problem& p);
 // chunk C B^T kernel, then the fused kernel, bracketed by ev0 / ev1 if given
 cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0 = nullptr,
                             cudaEvent_t ev1 = nullptr);
 
 // two heads per CTA (ssd_tc_pair.cu): N = 128, an even number of heads per
-// group and H a multiple of 4
+// group and H a multiple of 4 (shape only) ...
+bool tc_pair_shape_ok(const Problem& p);
+// ... and a 16-byte aligned dt
 bool tc_pair_supported(const Problem& p);
 cudaError_t tc_pair_launch(const Problem& p, const TcWorkspace& w, const CUtensorMap& tx, const CUtensorMap& tb,
                            const CUtensorMap& tc_, const CUtensorMap& tw, const CUtensorMap& ty,

@@ -619,6 +619,10 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
   fa.failed_count = w.failed_count;
   fa.failed_list = w.failed_list;
   fa.err = w.err;
+  fa.batch = p.b;
+  fa.handoff = w.handoff;
+  fa.flags = w.flags;
+  fa.pair_bad = w.pair_bad;
   if (NS == 128 && tc_pair_supported(p)) {
     CUtensorMap ty, tdt;
     if (!make_map_3d(&ty, p.y, p.H * p.P, p.L, p.b) || !make_map_dt(&tdt, p.dt, p.H, p.L, p.b))

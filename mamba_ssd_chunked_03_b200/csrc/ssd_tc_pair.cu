@@ -6,10 +6,16 @@
 //
 //   Yd   = W' [X'_h | X'_h+1]                     (M = 64 tokens,  K = 64 tokens)
 //   S'^T = B^T [X'_h | X'_h+1]                    (M = 128 states, K = 64 tokens)
-//   Yd  += C [e^m H_h | e^m H_h+1]^T              (M = 64 tokens,  K = N)
-//   y_t  = u_t Yd_t + D x_t,   H <- exp2(cs_e) H + exp2(cs_e - m) S'
+//   Yd  += C [H_h | H_h+1]^T                      (M = 64 tokens,  K = N)
+//   y_t  = u_t Yd_t + D x_t,   H <- 2^cs_e (H + S')
 //
-// (per head; u, v, m, cs as in ssd_tc_fast.cu).  The chunked steps are those
+// per head, with cs_t the in-chunk cumulative sum of dt A (log2 units),
+// u_t = 2^cs_t, v_s = 2^-cs_s dt_s and X' = diag(v) x: u_t v_s = exp of the
+// decay from s to t times dt_s.  The factors are taken about the chunk's
+// first token (ssd_tc_fast.cu takes them about its middle), so the state
+// enters the C H^T product as it is, with no per-chunk rescaling; a chunk
+// whose total decay exceeds 2^kRangeLog2 sends the pair to the exact kernel.
+// The chunked steps are those
 // of "SSM 家族全景图（下）：Mamba-2 与 Jamba" section 三.4; the D feed-through
 // is from "从Transformer的二次复杂度困境到Mamba的线性突围" (continuous SSM).
 //
@@ -33,6 +39,15 @@
 // x tiles sit in a 4-deep ring; W'+B, C, the e^m H tiles, Yd and S are
 // double-buffered.  Every wait is bounded; a CTA that times out records the
 // error, drains its copies, stores and MMAs, frees its TMEM and exits.
+//
+// The grid is persistent: with G CTAs, CTA i owns the contiguous range
+// [i T / G, (i+1) T / G) of the T = pairs x chunks steps in pair-major order,
+// so every CTA gets the same number of chunk steps.  A pair split between CTAs
+// i and i+1 hands its fp32 state over through global memory (per state warp:
+// data, then a release flag).  Each CTA runs the head of its last pair first
+// and the tail of its first pair last, so a tail normally finds its hand-over
+// long written.  Every warp role walks the CTA's segments as one sequence of
+// chunks, so the pipelines run across segment boundaries without draining.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -68,6 +83,8 @@ struct PairCfg {
   static constexpr uint32_t tYd0 = 0, tS0 = 256, kTmemCols = 512;
 };
 
+constexpr int kPairMaxSeg = 32;  // segments (pairs touched) per CTA, at most
+
 // Ring barriers are indexed like the buffers they guard, so no barrier can
 // complete a second phase before every waiter has seen the first.
 struct __align__(16) PairSmem {
@@ -85,16 +102,35 @@ struct __align__(16) PairSmem {
   uint32_t tmem_base;
   int abort_flag;
   int never;
-  int unit_bad;
+  int nseg, total;                       // segments of this CTA and their chunk count
+  // per segment: pair, batch row, first head, group, first chunk, length, first step
+  int seg_pair[kPairMaxSeg], seg_b[kPairMaxSeg], seg_h0[kPairMaxSeg], seg_grp[kPairMaxSeg];
+  int seg_c0[kPairMaxSeg], seg_len[kPairMaxSeg], seg_g0[kPairMaxSeg];
   alignas(16) float u[4][2][64];  // written as float4
   alignas(16) float v[4][2][64];
   alignas(16) float g[4][2][64];  // D / v_t: D x_t = g_t X'_t
-  float sc[4][2][4];  // E = 2^m, f = 2^(cs_e - m), d = 2^cs_e
+  float sc[4][2][4];  // [0]: d = 2^cs_e, the chunk's total decay
 };
 
 static_assert(offsetof(PairSmem, u) % 16 == 0 && offsetof(PairSmem, v) % 16 == 0 &&
                   offsetof(PairSmem, g) % 16 == 0,
               "scan results are stored as float4");
+
+// Position of one of a CTA's step streams (each role walks its steps in
+// order): segment k, chunk c.  next() moves to the following step.
+struct PairCursor {
+  int k, c;
+  __device__ __forceinline__ void start(const PairSmem& s) {
+    k = 0;
+    c = s.seg_c0[0];
+  }
+  __device__ __forceinline__ void next(const PairSmem& s) {
+    if (++c == s.seg_c0[k] + s.seg_len[k] && k + 1 < s.nseg) {
+      ++k;
+      c = s.seg_c0[k];
+    }
+  }
+};
 
 __global__ void __launch_bounds__(512, 1)
     k_ssd_fwd_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
@@ -109,9 +145,6 @@ __global__ void __launch_bounds__(512, 1)
   __shared__ PairSmem s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t pairs = a.H / 2;
-  const int64_t b = blockIdx.x / pairs;
-  const int64_t h0 = (blockIdx.x % pairs) * 2;  // heads h0, h0 + 1
-  const int64_t g = h0 / a.hpg;
   const int nc = (int)a.nc;
 
   if (tid == 0) {
@@ -135,7 +168,39 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(&s.drain, 1);
     s.abort_flag = *reinterpret_cast<volatile int*>(a.err) != 0;
     s.never = 0;
-    s.unit_bad = 0;
+    // this CTA's range of (pair, chunk) steps, as segments in processing order:
+    // the head of the last pair, the whole pairs, the tail of the first pair
+    // (steps, pairs and chunks fit in 32 bits: the launch checks b * H * nc)
+    const int64_t T = a.batch * pairs * a.nc;
+    const int start = (int)((int64_t)blockIdx.x * T / gridDim.x);
+    const int end = (int)(((int64_t)blockIdx.x + 1) * T / gridDim.x);
+    const int ncs = nc, npr = (int)pairs, hpg = (int)a.hpg;
+    int n = 0, tot = 0;
+    auto add = [&](int pr, int c0, int len) {
+      if (n < kPairMaxSeg && len > 0) {
+        s.seg_pair[n] = pr;
+        s.seg_b[n] = pr / npr;
+        s.seg_h0[n] = (pr % npr) * 2;
+        s.seg_grp[n] = (pr % npr) * 2 / hpg;
+        s.seg_c0[n] = c0;
+        s.seg_len[n] = len;
+        s.seg_g0[n] = tot;
+        tot += len;
+        ++n;
+      }
+    };
+    if (end > start) {
+      const int p0 = start / ncs, c0 = start % ncs, q = (end - 1) / ncs, cq = (end - 1) % ncs + 1;
+      if (q == p0) {
+        add(p0, c0, cq - c0);
+      } else {
+        add(q, 0, cq);
+        for (int pr = p0 + 1; pr < q; ++pr) add(pr, 0, ncs);
+        add(p0, c0, ncs - c0);
+      }
+    }
+    s.nseg = n;
+    s.total = tot;
     fence_mbar_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_b);
@@ -154,48 +219,61 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = s.tmem_base;
   volatile int* abort_flag = &s.abort_flag;
   volatile int* never = &s.never;
+  const int total = s.total;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA loads
     if (lane == 0) {
       int last_x = -1, last_wb = -1, last_c = -1;
-      auto issue_x = [&](int c) {
-        const int sl = c & 3;
+      // (the argument is this CTA's step number; each stream has a cursor on
+      // its pair and chunk, advanced as the stream issues its steps in order)
+      PairCursor ux, uwb, uc, upf;
+      ux.start(s);
+      uwb.start(s);
+      uc.start(s);
+      upf.start(s);
+      for (int k = 0; k < 3; ++k) upf.next(s);
+      auto issue_x = [&](int gg) {
+        const int sl = gg & 3, bb = s.seg_b[ux.k], hh = s.seg_h0[ux.k];
         mbar_arrive_expect_tx(&s.full_x[sl], 2 * K::kTile);
         for (int j = 0; j < 2; ++j)
-          tma_load_3d(sm + K::oX + (sl * 2 + j) * K::kTile, &tm_x, &s.full_x[sl], (int)((h0 + j) * 64), c * 64,
-                      (int)b);
-        last_x = c;
+          tma_load_3d(sm + K::oX + (sl * 2 + j) * K::kTile, &tm_x, &s.full_x[sl], (hh + j) * 64, ux.c * 64, bb);
+        ux.next(s);
+        last_x = gg;
       };
-      auto issue_wb = [&](int c) {
-        const int i = c & 1;
+      auto issue_wb = [&](int gg) {
+        const int i = gg & 1, bb = s.seg_b[uwb.k], grp = s.seg_grp[uwb.k];
         mbar_arrive_expect_tx(&s.full_wb[i], (1 + K::NB) * K::kTile);
-        tma_load_3d(sm + K::oW + i * K::kTile, &tm_w, &s.full_wb[i], 0, (int)(((b * a.nc + c) * a.G + g) * 64), 0);
+        tma_load_3d(sm + K::oW + i * K::kTile, &tm_w, &s.full_wb[i], 0, ((bb * nc + uwb.c) * (int)a.G + grp) * 64, 0);
         for (int jb = 0; jb < K::NB; ++jb)
-          tma_load_3d(sm + K::oB + (i * K::NB + jb) * K::kTile, &tm_b, &s.full_wb[i], (int)(g * NS + 64 * jb),
-                      c * 64, (int)b);
-        last_wb = c;
+          tma_load_3d(sm + K::oB + (i * K::NB + jb) * K::kTile, &tm_b, &s.full_wb[i], grp * NS + 64 * jb,
+                      uwb.c * 64, bb);
+        uwb.next(s);
+        last_wb = gg;
       };
-      auto issue_c = [&](int c) {
-        const int i = c & 1;
+      auto issue_c = [&](int gg) {
+        const int i = gg & 1, bb = s.seg_b[uc.k], grp = s.seg_grp[uc.k];
         mbar_arrive_expect_tx(&s.full_c[i], K::NB * K::kTile);
         for (int jb = 0; jb < K::NB; ++jb)
-          tma_load_3d(sm + K::oC + (i * K::NB + jb) * K::kTile, &tm_c, &s.full_c[i], (int)(g * NS + 64 * jb),
-                      c * 64, (int)b);
-        last_c = c;
+          tma_load_3d(sm + K::oC + (i * K::NB + jb) * K::kTile, &tm_c, &s.full_c[i], grp * NS + 64 * jb,
+                      uc.c * 64, bb);
+        uc.next(s);
+        last_c = gg;
       };
       // x comes from HBM and takes several chunk periods to arrive; L2
       // prefetches run 6 chunks ahead of use, the loads into the ring 3
-      auto prefetch_x = [&](int c) {
-        for (int j = 0; j < 2; ++j) tma_prefetch_l2_3d(&tm_x, (int)((h0 + j) * 64), c * 64, (int)b);
+      auto prefetch_x = [&](int) {
+        const int bb = s.seg_b[upf.k], hh = s.seg_h0[upf.k];
+        for (int j = 0; j < 2; ++j) tma_prefetch_l2_3d(&tm_x, (hh + j) * 64, upf.c * 64, bb);
+        upf.next(s);
       };
       if (!*abort_flag) {
         #pragma unroll 1
-        for (int c = 3; c < 6 && c < nc; ++c) prefetch_x(c);
+        for (int c = 3; c < 6 && c < total; ++c) prefetch_x(c);
         #pragma unroll 1
-        for (int c = 0; c < 3 && c < nc; ++c) issue_x(c);  // slot 3 starts free
+        for (int c = 0; c < 3 && c < total; ++c) issue_x(c);  // slot 3 starts free
         #pragma unroll 1
-        for (int c = 0; c < 2 && c < nc; ++c) {
+        for (int c = 0; c < 2 && c < total; ++c) {
           issue_wb(c);
           issue_c(c);
         }
@@ -203,18 +281,18 @@ __global__ void __launch_bounds__(512, 1)
       bool ok = !*abort_flag;
       // each tile is refilled for a later chunk as soon as its last reader is done
       #pragma unroll 1
-      for (int c = 0; c < nc && ok; ++c) {
-        if (c + 2 < nc) {
+      for (int c = 0; c < total && ok; ++c) {
+        if (c + 2 < total) {
           ok = mbar_wait(&s.s_full[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
           if (ok) issue_wb(c + 2);
           ok = ok && mbar_wait(&s.mma_done[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
           if (ok) issue_c(c + 2);
         }
-        // x of chunk c + 3 goes where chunk c - 1 was, once its y tile has been stored
-        if (ok && c + 3 < nc) {
+        // x of step c + 3 goes where step c - 1 was, once its y tile has been stored
+        if (ok && c + 3 < total) {
           ok = c < 1 || mbar_wait(&s.x_empty[(c - 1) & 3], ((c - 1) >> 2) & 1, abort_flag, kWaitLimitNs);
           if (ok) issue_x(c + 3);
-          if (ok && c + 6 < nc) prefetch_x(c + 6);
+          if (ok && c + 6 < total) prefetch_x(c + 6);
         }
       }
       if (*abort_flag) {  // let this CTA's own copies land before its smem is released
@@ -238,7 +316,7 @@ __global__ void __launch_bounds__(512, 1)
       constexpr uint32_t id_y = idesc_bf16(64, 128, 0, 1);    // A K-major, B MN-major (2 heads)
       constexpr uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // both MN-major
       #pragma unroll 1
-      for (int c = 0; c < nc; ++c) {
+      for (int c = 0; c < total; ++c) {
         const int i = c & 1;
         const uint32_t ph = (c >> 1) & 1;
         bool ok = mbar_wait(&s.full_wb[i], ph, abort_flag, kWaitLimitNs);
@@ -285,33 +363,44 @@ __global__ void __launch_bounds__(512, 1)
     // arrives by TMA (a box of 4 heads from the multiple of 4 at or below h0)
     // so that no register load is in flight when the results are released.
     const int j = lane >> 4, l16 = lane & 15;
-    const int hx = (int)(h0 & ~int64_t(3));
-    const int col = (int)(h0 - hx) + j;
-    const float a2 = a.A[h0 + j] * kLog2e;
-    const float dsk = a.D ? a.D[h0 + j] : 0.f;
     int last_dt = -1;
-    auto issue_dt = [&](int c) {
-      mbar_arrive_expect_tx(&s.full_dt[c & 7], K::kDtBox);
-      tma_load_3d(sm + K::oDt + (c & 7) * K::kDtBox, &tm_dt, &s.full_dt[c & 7], hx, c * 64, (int)b);
-      last_dt = c;
+    PairCursor ud, us;
+    ud.start(s);
+    us.start(s);
+    auto issue_dt = [&](int gg) {
+      mbar_arrive_expect_tx(&s.full_dt[gg & 7], K::kDtBox);
+      tma_load_3d(sm + K::oDt + (gg & 7) * K::kDtBox, &tm_dt, &s.full_dt[gg & 7], s.seg_h0[ud.k] & ~3, ud.c * 64,
+                  s.seg_b[ud.k]);
+      ud.next(s);
+      last_dt = gg;
     };
     if (lane == 0 && !*abort_flag)
       #pragma unroll 1
-      for (int c = 0; c < 8 && c < nc; ++c) issue_dt(c);
+      for (int c = 0; c < 8 && c < total; ++c) issue_dt(c);
+    int cur_seg = -1, col = 0;
+    float a2 = 0.f, dsk = 0.f;
     #pragma unroll 1
-    for (int c = 0; c < nc; ++c) {
-      const int slot = c & 3;
-      if (c >= 4 && !mbar_wait_warp(&s.scan_empty[slot], ((c - 4) >> 2) & 1, abort_flag, kWaitLimitNs)) break;
-      if (!mbar_wait_warp(&s.full_dt[c & 7], (c >> 3) & 1, abort_flag, kWaitLimitNs)) break;
-      const float* dts = reinterpret_cast<const float*>(sm + K::oDt + (c & 7) * K::kDtBox);
+    for (int g = 0; g < total; ++g, us.next(s)) {
+      const int slot = g & 3;
+      const int hh = s.seg_h0[us.k];
+      if (us.k != cur_seg) {  // a new pair: its heads' A and D
+        cur_seg = us.k;
+        col = (hh & 3) + j;
+        a2 = a.A[hh + j] * kLog2e;
+        dsk = a.D ? a.D[hh + j] : 0.f;
+      }
+      if (g >= 4 && !mbar_wait_warp(&s.scan_empty[slot], ((g - 4) >> 2) & 1, abort_flag, kWaitLimitNs)) break;
+      if (!mbar_wait_warp(&s.full_dt[g & 7], (g >> 3) & 1, abort_flag, kWaitLimitNs)) break;
+      const float* dts = reinterpret_cast<const float*>(sm + K::oDt + (g & 7) * K::kDtBox);
+      const int c = us.c;
       const int nvalid = (int)((int64_t)(c + 1) * 64 <= a.L ? 64 : a.L - (int64_t)c * 64);
       float d[4], cs[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) d[k] = dts[(4 * l16 + k) * 4 + col];
       __syncwarp();
-      if (lane == 0 && c + 8 < nc) {  // the slot has been read: refill it 8 chunks ahead
+      if (lane == 0 && g + 8 < total) {  // the slot has been read: refill it 8 steps ahead
         fence_proxy_async_smem();
-        issue_dt(c + 8);
+        issue_dt(g + 8);
       }
       cs[0] = d[0] * a2;
 #pragma unroll
@@ -325,7 +414,6 @@ __global__ void __launch_bounds__(512, 1)
       const float excl = incl - cs[3];
 #pragma unroll
       for (int k = 0; k < 4; ++k) cs[k] += excl;
-      const float m = __shfl_sync(0xffffffffu, cs[3], 7, 16);  // token 31
       const int e = nvalid - 1;
       const float mine = (e & 3) == 0 ? cs[0] : (e & 3) == 1 ? cs[1] : (e & 3) == 2 ? cs[2] : cs[3];
       const float cse = __shfl_sync(0xffffffffu, mine, e >> 2, 16);
@@ -333,22 +421,27 @@ __global__ void __launch_bounds__(512, 1)
       bool bad = false;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        u4[k] = exp2f(cs[k] - m);
-        v4[k] = exp2f(m - cs[k]) * d[k];
+        u4[k] = exp2f(cs[k]);
+        v4[k] = exp2f(-cs[k]) * d[k];
         // D x_t is recovered from X'_t = v_t x_t, so a valid token needs v_t well
         // inside the normal range (the fast division is exact to 2 ulp there)
         g4[k] = dsk != 0.f ? __fdividef(dsk, v4[k]) : 0.f;
-        bad |= !(fabsf(cs[k] - m) <= kRangeLog2) ||
+        bad |= !(fabsf(cs[k]) <= kRangeLog2) ||
                (dsk != 0.f && 4 * l16 + k < nvalid && !(fabsf(v4[k]) >= 1e-30f && fabsf(v4[k]) <= 1e30f));
       }
-      if (__any_sync(0xffffffffu, bad) && lane == 0) s.unit_bad = 1;
+      // a chunk the factorised form cannot take: the exact kernel redoes the
+      // pair (once, however many chunks or CTAs find it)
+      if (__any_sync(0xffffffffu, bad) && lane == 0 && atomicExch(&a.pair_bad[s.seg_pair[us.k]], 1) == 0) {
+        const int at = atomicAdd(a.failed_count, 2);
+        const int unit = s.seg_b[us.k] * (int)a.H + hh;
+        a.failed_list[at] = unit;
+        a.failed_list[at + 1] = unit + 1;
+      }
       *reinterpret_cast<float4*>(&s.u[slot][j][4 * l16]) = make_float4(u4[0], u4[1], u4[2], u4[3]);
       *reinterpret_cast<float4*>(&s.v[slot][j][4 * l16]) = make_float4(v4[0], v4[1], v4[2], v4[3]);
       *reinterpret_cast<float4*>(&s.g[slot][j][4 * l16]) = make_float4(g4[0], g4[1], g4[2], g4[3]);
       if (l16 == 0) {
-        s.sc[slot][j][0] = exp2f(m);
-        s.sc[slot][j][1] = exp2f(cse - m);
-        s.sc[slot][j][2] = exp2f(cse);
+        s.sc[slot][j][0] = exp2f(cse);
       }
       mbar_arrive(&s.scan_full[slot]);
     }
@@ -359,12 +452,15 @@ __global__ void __launch_bounds__(512, 1)
   } else if (warp == 3) {
     // ------------------------------------------------------------ y stores
     if (lane == 0) {
+      PairCursor uy;
+      uy.start(s);
       #pragma unroll 1
-      for (int c = 0; c < nc; ++c) {
+      for (int c = 0; c < total; ++c, uy.next(s)) {
         const int sl = c & 3;
         if (!mbar_wait(&s.y_staged[sl], (c >> 2) & 1, abort_flag, kWaitLimitNs)) break;
         for (int j = 0; j < 2; ++j)
-          tma_store_3d(&tm_y, sm + K::oX + (sl * 2 + j) * K::kTile, (int)((h0 + j) * 64), c * 64, (int)b);
+          tma_store_3d(&tm_y, sm + K::oX + (sl * 2 + j) * K::kTile, (s.seg_h0[uy.k] + j) * 64, uy.c * 64,
+                       s.seg_b[uy.k]);
         bulk_commit_group();
         bulk_wait_read<0>();  // the tiles have been read out: the slot may be refilled
         mbar_arrive(&s.x_empty[sl]);
@@ -378,8 +474,8 @@ __global__ void __launch_bounds__(512, 1)
     const int te = 16 * q + (lane & 15);   // epilogue row (token) of this thread
     const int half = lane >> 4;            // epilogue columns p in [32 half, 32 half + 32)
     #pragma unroll 1
-    for (int c = 1; c <= nc; ++c) {
-      // ---- epilogue for chunk c-1, both heads: y = u_t Yd + (D / v_t) X'_t, written over X'
+    for (int c = 1; c <= total; ++c) {
+      // ---- epilogue for step c-1, both heads: y = u_t Yd + (D / v_t) X'_t, written over X'
       if (c >= 1) {
         const int ip = (c - 1) & 1, slp = (c - 1) & 3;
         if (!mbar_wait_warp(&s.mma_done[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) break;
@@ -418,14 +514,14 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else {
     // ------------------------------------------------ per-head state warps
-    const int j = (warp - 8) >> 2;       // head h0 + j
-    const int64_t h = h0 + j;
+    const int j = (warp - 8) >> 2;       // head h0 + j of the current pair
     const int q = warp & 3;              // TMEM lane quadrant
     const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
     const int n = 32 * q + lane;         // state row
+    const int uw = warp - 8;             // this warp's part of a state hand-over
     const int ut = tid - 256 - 128 * j;  // 0..127 within this head's group
     const int srow = ut >> 1, shalf = ut & 1;
-    // X' = diag(v) x for chunk cc of this head: each thread scales half a
+    // X' = diag(v) x for step cc of this head: each thread scales half a
     // 128-byte row in place, at the swizzled positions of its 16-byte columns
     auto scale_chunk = [&](int cc) -> bool {
       const int sl = cc & 3;
@@ -448,87 +544,146 @@ __global__ void __launch_bounds__(512, 1)
       return true;
     };
     float H[64];
+    // state at the start of segment k: h0 (or zero) at a pair's first chunk,
+    // otherwise this warp's part of the hand-over the previous CTA wrote
+    auto seg_begin = [&](int k) -> bool {
+      const int64_t h = s.seg_h0[k] + j, bb = s.seg_b[k];
+      if (s.seg_c0[k] == 0) {
+        if (a.h0) {
+          const float* src = a.h0 + ((bb * a.H + h) * 64) * NS + n;
 #pragma unroll
-    for (int p = 0; p < 64; ++p) H[p] = a.h0 ? a.h0[((b * a.H + h) * 64 + p) * NS + n] : 0.f;
-    bool failed = nc > 0 && !scale_chunk(0);
+          for (int p = 0; p < 64; ++p) H[p] = src[p * NS];
+        } else {
+#pragma unroll
+          for (int p = 0; p < 64; ++p) H[p] = 0.f;
+        }
+        return true;
+      }
+      const int slot = (int)blockIdx.x - 1;
+      bool ok = true;
+      if (lane == 0) ok = wait_flag_acquire(a.flags + slot * 8 + uw, abort_flag, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      const float4* src =
+          reinterpret_cast<const float4*>(a.handoff + (size_t)slot * kPairHandoffFloats + ((size_t)j * 128 + n) * 64);
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        const float4 v = __ldcg(src + p);
+        H[4 * p] = v.x;
+        H[4 * p + 1] = v.y;
+        H[4 * p + 2] = v.z;
+        H[4 * p + 3] = v.w;
+      }
+      return true;
+    };
+    // state at the end of segment k: the pair's final state, or the hand-over
+    // to the next CTA (data, then this warp's release flag)
+    auto seg_end = [&](int k) {
+      const int64_t h = s.seg_h0[k] + j, bb = s.seg_b[k];
+      if (s.seg_c0[k] + s.seg_len[k] == nc) {
+        if (a.final_states) {
+          float* dst = a.final_states + ((bb * a.H + h) * 64) * NS + n;
+#pragma unroll
+          for (int p = 0; p < 64; ++p) dst[(int64_t)p * NS] = H[p];
+        }
+        return;
+      }
+      float4* dst = reinterpret_cast<float4*>(a.handoff + (size_t)blockIdx.x * kPairHandoffFloats +
+                                              ((size_t)j * 128 + n) * 64);
+#pragma unroll
+      for (int p = 0; p < 16; ++p) __stcg(dst + p, make_float4(H[4 * p], H[4 * p + 1], H[4 * p + 2], H[4 * p + 3]));
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) store_flag_release(a.flags + (int)blockIdx.x * 8 + uw, 1);
+    };
+    // Steps in order: publish e^m H for step g (the state before g), scale the
+    // x tile of step g+1, then fold step g's chunk state into H.
+    bool failed = total > 0 && !scale_chunk(0);
+    const int nseg = s.nseg;
     #pragma unroll 1
-    for (int c = 0; c <= nc && !failed; ++c) {
-      // ---- state update for chunk c-1
-      if (c >= 1) {
-        const int ip = (c - 1) & 1, slp = (c - 1) & 3;
-        if (!mbar_wait_warp(&s.s_full[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
+    for (int k = 0; k < nseg && !failed; ++k) {
+      if (!seg_begin(k)) {
+        failed = true;
+        break;
+      }
+      const int g_end = s.seg_g0[k] + s.seg_len[k];
+      #pragma unroll 1
+      for (int g = s.seg_g0[k]; g < g_end; ++g) {
+        const int i = g & 1;
+        // ---- publish H (bf16) for step g's C H^T product
+        if (!mbar_wait_warp(&s.scan_full[g & 3], (g >> 2) & 1, abort_flag, kWaitLimitNs) ||
+            (g >= 2 && !mbar_wait_warp(&s.mma_done[i], ((g - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
+          failed = true;
+          break;
+        }
+        {
+          unsigned char* base = sm + K::oH + (i * 2 + j) * K::kHTile + (uint32_t)n * 128;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            uint4 vv;
+            vv.x = pack_bf16x2(H[8 * kk + 0], H[8 * kk + 1]);
+            vv.y = pack_bf16x2(H[8 * kk + 2], H[8 * kk + 3]);
+            vv.z = pack_bf16x2(H[8 * kk + 4], H[8 * kk + 5]);
+            vv.w = pack_bf16x2(H[8 * kk + 6], H[8 * kk + 7]);
+            *reinterpret_cast<uint4*>(base + ((kk ^ (n & 7)) << 4)) = vv;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&s.h_ready[i]);
+        }
+        // ---- X' of step g+1, which the next MMAs wait for
+        if (g + 1 < total && !scale_chunk(g + 1)) {
+          failed = true;
+          break;
+        }
+        // ---- state update with step g's chunk state
+        if (!mbar_wait_warp(&s.s_full[i], (g >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           break;
         }
         tc_fence_after();
-        const float dd = s.sc[slp][j][2], ff = s.sc[slp][j][1];
+        {
+          // H <- d (H + S'), two lanes of fp32 per instruction
+          const float dd = s.sc[g & 3][j][0];
+          const float2 d2 = make_float2(dd, dd);
 #pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          uint32_t r[32];
-          SSD_TMEM_LD_32x32b_X32(tq + K::tS0 + 128 * ip + 64 * j + 32 * hlf, r);
-          SSD_TMEM_WAIT_LD_32(r);
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            uint32_t r[32];
+            SSD_TMEM_LD_32x32b_X32(tq + K::tS0 + 128 * i + 64 * j + 32 * hlf, r);
+            SSD_TMEM_WAIT_LD_32(r);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) H[32 * hlf + k] = fmaf(dd, H[32 * hlf + k], ff * __uint_as_float(r[k]));
+            for (int kk = 0; kk < 32; kk += 2) {
+              const float2 h2 = __fadd2_rn(make_float2(H[32 * hlf + kk], H[32 * hlf + kk + 1]),
+                                           make_float2(__uint_as_float(r[kk]), __uint_as_float(r[kk + 1])));
+              const float2 o2 = __fmul2_rn(d2, h2);
+              H[32 * hlf + kk] = o2.x;
+              H[32 * hlf + kk + 1] = o2.y;
+            }
+          }
         }
         tc_fence_before();
-        mbar_arrive(&s.acc_free[ip]);     // this thread's reads of S of chunk c-1 are done
-        mbar_arrive(&s.scan_empty[slp]);  // and of that chunk's scalars
+        mbar_arrive(&s.acc_free[i]);        // this thread's reads of S of step g are done
+        mbar_arrive(&s.scan_empty[g & 3]);  // and of that step's scalars
       }
-      // ---- publish e^m H (bf16) for chunk c's C H^T product
-      if (c < nc) {
-        const int i = c & 1;
-        if (!mbar_wait_warp(&s.scan_full[c & 3], (c >> 2) & 1, abort_flag, kWaitLimitNs) ||
-            (c >= 2 && !mbar_wait_warp(&s.mma_done[i], ((c - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
-          failed = true;
-          break;
-        }
-        const float E = s.sc[c & 3][j][0];
-        unsigned char* base = sm + K::oH + (i * 2 + j) * K::kHTile + (uint32_t)n * 128;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          uint4 vv;
-          vv.x = pack_bf16x2(E * H[8 * k + 0], E * H[8 * k + 1]);
-          vv.y = pack_bf16x2(E * H[8 * k + 2], E * H[8 * k + 3]);
-          vv.z = pack_bf16x2(E * H[8 * k + 4], E * H[8 * k + 5]);
-          vv.w = pack_bf16x2(E * H[8 * k + 6], E * H[8 * k + 7]);
-          *reinterpret_cast<uint4*>(base + ((k ^ (n & 7)) << 4)) = vv;
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&s.h_ready[i]);
-      }
-      // ---- X' of chunk c+1, which the next MMAs wait for
-      if (c + 1 < nc && !scale_chunk(c + 1)) {
-        failed = true;
-        break;
-      }
-    }
-    if (!failed && a.final_states) {
-      float* dst = a.final_states + ((b * a.H + h) * 64) * NS + n;
-#pragma unroll
-      for (int p = 0; p < 64; ++p) dst[(int64_t)p * NS] = H[p];
+      if (!failed) seg_end(k);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid == 0) {
-    if (*abort_flag) atomicExch(a.err, 1);
-    // a chunk's decay range was too wide to factorise: the exact kernel redoes both heads
-    if (s.unit_bad) {
-      const int at = atomicAdd(a.failed_count, 2);
-      a.failed_list[at] = (int)(b * a.H + h0);
-      a.failed_list[at + 1] = (int)(b * a.H + h0 + 1);
-    }
-  }
+  if (tid == 0 && *abort_flag) atomicExch(a.err, 1);
   if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
 }
 
 }  // namespace
 
+// (the kernel counts its (pair, chunk) steps in 32-bit integers)
+bool tc_pair_shape_ok(const Problem& p) {
+  return p.N == 128 && p.hpg % 2 == 0 && p.H % 4 == 0 && (p.b * p.H / 2) * p.nc < ((int64_t)1 << 30);
+}
+
 // dt is read by TMA, whose base address must be 16-byte aligned
 bool tc_pair_supported(const Problem& p) {
-  return p.N == 128 && p.hpg % 2 == 0 && p.H % 4 == 0 && reinterpret_cast<uintptr_t>(p.dt) % 16 == 0;
+  return tc_pair_shape_ok(p) && reinterpret_cast<uintptr_t>(p.dt) % 16 == 0;
 }
 
 cudaError_t tc_pair_launch(const Problem& p, const TcWorkspace& w, const CUtensorMap& tx, const CUtensorMap& tb,
@@ -537,9 +692,22 @@ cudaError_t tc_pair_launch(const Problem& p, const TcWorkspace& w, const CUtenso
   cudaError_t e = cudaFuncSetAttribute(k_ssd_fwd_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)PairCfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  (void)w;
-  k_ssd_fwd_pair<<<(unsigned)(p.b * p.H / 2), PairCfg::kThreads, PairCfg::kSmemBytes, st>>>(tx, tb, tc_, tw, ty,
-                                                                                            tdt, fa);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  // one CTA per SM over equal ranges of the pair-major steps; if a CTA would
+  // touch more pairs than its segment table holds, one CTA per pair instead
+  // (whole pairs only: no hand-over)
+  const int64_t npairs = p.b * p.H / 2;
+  int64_t grid = npairs < sms ? npairs : sms;
+  if (grid > kPairGridMax) grid = kPairGridMax;
+  if ((npairs + grid - 1) / grid + 2 > kPairMaxSeg) grid = npairs;
+  tc::FastArgs a = fa;
+  a.batch = p.b;
+  a.handoff = w.handoff;
+  a.flags = w.flags;
+  a.pair_bad = w.pair_bad;
+  k_ssd_fwd_pair<<<(unsigned)grid, PairCfg::kThreads, PairCfg::kSmemBytes, st>>>(tx, tb, tc_, tw, ty, tdt, a);
   return cudaGetLastError();
 }
 

@@ -31,6 +31,10 @@ SMALL = [
     (1, 777, 4, 64, 64, 1, 128, 0.0),
     (1, 100, 2, 256, 256, 1, 256, 0.1),
     (2, 255, 4, 64, 128, 1, 256, 0.0),
+    # more head pairs than SMs: the two-head kernel splits pairs between CTAs
+    # and hands the state over (4 chunks per row; ragged 13-chunk rows)
+    (4, 200, 80, 64, 128, 1, 64, 0.1),
+    (2, 777, 160, 64, 128, 2, 64, 0.0),
 ]
 
 
