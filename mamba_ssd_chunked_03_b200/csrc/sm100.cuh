@@ -52,6 +52,19 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of a phase (never suspends the thread); several probes
+// issued back to back overlap their latencies.
+__device__ __forceinline__ bool mbar_probe(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // As mbar_test, but a thread whose phase is not complete may sleep up to
 // `hint_ns` waiting for it instead of returning at once, so waiting warps do
 // not take issue slots from working ones.
@@ -261,6 +274,16 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
         "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),          \
         "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),          \
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                                               \
+      : "r"(taddr))
+
+// 32 lanes x 32 bit, 16 columns: thread i reads lane base + i, columns
+// [c, c+16) into r[0..15]
+#define SSD_TMEM_LD_32x32b_X16(taddr, r)                                                                     \
+  asm volatile(                                                                                              \
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];" \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),      \
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),            \
+        "=r"(r[15])                                                                                         \
       : "r"(taddr))
 
 // 16 lanes x 32 bit, twice: threads 0-15 read lanes base..base+15 at columns

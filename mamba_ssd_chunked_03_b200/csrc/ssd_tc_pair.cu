@@ -523,11 +523,10 @@ __global__ void __launch_bounds__(512, 1)
     const int srow = ut >> 1, shalf = ut & 1;
     // X' = diag(v) x for step cc of this head: each thread scales half a
     // 128-byte row in place, at the swizzled positions of its 16-byte columns
-    auto scale_chunk = [&](int cc) -> bool {
+    // (the caller has seen scan_full and full_x of step cc; it fences and
+    // arrives on xp_ready)
+    auto scale_tile = [&](int cc) {
       const int sl = cc & 3;
-      if (!mbar_wait_warp(&s.scan_full[sl], (cc >> 2) & 1, abort_flag, kWaitLimitNs) ||
-          !mbar_wait_warp(&s.full_x[sl], (cc >> 2) & 1, abort_flag, kWaitLimitNs))
-        return false;
       const __nv_bfloat162 w2 = __float2bfloat162_rn(s.v[sl][j][srow]);
       unsigned char* row = sm + K::oX + (sl * 2 + j) * K::kTile + srow * 128;
 #pragma unroll
@@ -539,6 +538,13 @@ __global__ void __launch_bounds__(512, 1)
         for (int q2 = 0; q2 < 4; ++q2) e2[q2] = __hmul2(e2[q2], w2);
         *px = vv;
       }
+    };
+    auto scale_chunk = [&](int cc) -> bool {
+      const int sl = cc & 3;
+      if (!mbar_wait_warp(&s.scan_full[sl], (cc >> 2) & 1, abort_flag, kWaitLimitNs) ||
+          !mbar_wait_warp(&s.full_x[sl], (cc >> 2) & 1, abort_flag, kWaitLimitNs))
+        return false;
+      scale_tile(cc);
       fence_proxy_async_smem();
       mbar_arrive(&s.xp_ready[sl]);
       return true;
@@ -608,10 +614,15 @@ __global__ void __launch_bounds__(512, 1)
       const int g_end = s.seg_g0[k] + s.seg_len[k];
       #pragma unroll 1
       for (int g = s.seg_g0[k]; g < g_end; ++g) {
-        const int i = g & 1;
-        // ---- publish H (bf16) for step g's C H^T product
-        if (!mbar_wait_warp(&s.scan_full[g & 3], (g >> 2) & 1, abort_flag, kWaitLimitNs) ||
-            (g >= 2 && !mbar_wait_warp(&s.mma_done[i], ((g - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        const int i = g & 1, n1 = g + 1, s1 = n1 & 3;
+        const bool more = n1 < total;
+        // the barriers this step's publish and the next tile's scaling need,
+        // probed together (their latencies overlap), then waited for if not yet
+        const bool d_ok = g < 2 || mbar_probe(&s.mma_done[i], ((g - 2) >> 1) & 1);
+        const bool v_ok = !more || mbar_probe(&s.scan_full[s1], (n1 >> 2) & 1);
+        const bool x_ok = !more || mbar_probe(&s.full_x[s1], (n1 >> 2) & 1);
+        if (!__all_sync(0xffffffffu, d_ok) &&
+            !mbar_wait_warp(&s.mma_done[i], ((g - 2) >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           break;
         }
@@ -626,13 +637,20 @@ __global__ void __launch_bounds__(512, 1)
             vv.w = pack_bf16x2(H[8 * kk + 6], H[8 * kk + 7]);
             *reinterpret_cast<uint4*>(base + ((kk ^ (n & 7)) << 4)) = vv;
           }
-          fence_proxy_async_smem();
-          mbar_arrive(&s.h_ready[i]);
         }
-        // ---- X' of step g+1, which the next MMAs wait for
-        if (g + 1 < total && !scale_chunk(g + 1)) {
-          failed = true;
-          break;
+        fence_proxy_async_smem();
+        mbar_arrive(&s.h_ready[i]);
+        if (more) {
+          if ((!__all_sync(0xffffffffu, v_ok) &&
+               !mbar_wait_warp(&s.scan_full[s1], (n1 >> 2) & 1, abort_flag, kWaitLimitNs)) ||
+              (!__all_sync(0xffffffffu, x_ok) &&
+               !mbar_wait_warp(&s.full_x[s1], (n1 >> 2) & 1, abort_flag, kWaitLimitNs))) {
+            failed = true;
+            break;
+          }
+          scale_tile(n1);
+          fence_proxy_async_smem();
+          mbar_arrive(&s.xp_ready[s1]);
         }
         // ---- state update with step g's chunk state
         if (!mbar_wait_warp(&s.s_full[i], (g >> 1) & 1, abort_flag, kWaitLimitNs)) {
