@@ -596,25 +596,27 @@ size_t tc_workspace_need(const Problem& p) {
 }
 
 const int* tc_error_word(const Problem& p, const void* ws) {
-  return tc_carve(p, const_cast<void*>(ws)).err;
+  return tc_carve(tc_tiles(p), const_cast<void*>(ws)).err;
 }
 
 bool tc_supported(const Problem& p, uint32_t flags) {
   if (flags & SSD_FLAG_GENERIC) return false;
   if (p.dtype != SSD_BF16) return false;
-  if (p.P != 64 || p.Q != 64) return false;
+  if (p.P != 64 || (p.Q != 64 && p.Q != 128 && p.Q != 256)) return false;
   if (p.N != 128 && p.N != 256) return false;
   if (p.seq) return false;
   // TMA coordinates are 32-bit
-  if (p.b * p.nc * p.G * 64 >= ((int64_t)1 << 31) || p.L >= ((int64_t)1 << 31)) return false;
+  const Problem t = tc_tiles(p);
+  if (t.b * t.nc * t.G * 64 >= ((int64_t)1 << 31) || t.L >= ((int64_t)1 << 31)) return false;
   return true;
 }
 
-size_t tc_workspace_bytes(const Problem& p) { return tc_workspace_need(p); }
+size_t tc_workspace_bytes(const Problem& p) { return tc_workspace_need(tc_tiles(p)); }
 
 int tc_launch_count(const Problem&) { return 3; }
 
-cudaError_t tc_forward(const Problem& p, void* ws, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
+cudaError_t tc_forward(const Problem& pq, void* ws, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
+  const Problem p = tc_tiles(pq);
   const TcWorkspace w = tc_carve(p, ws);
   cudaError_t e = cudaMemsetAsync(w.err, 0, w.zero_bytes, st);
   if (e != cudaSuccess) return e;

@@ -69,6 +69,19 @@ bool make_map_dt(CUtensorMap* m, const float* dt, int64_t H, int64_t L, int64_t 
 
 }  // namespace tc
 
+// The tensor-core kernels work on 64-token chunks.  A chunk of Q = 128 or 256
+// tokens is computed as Q/64 consecutive 64-token chunks: the chunked
+// decomposition is an exact re-association of the recurrence, so refining
+// the chunks changes only the rounding, not the result.  Every tensor-core
+// entry point (ssd_tc.cu, ssd_tc_fast.cu) turns the problem into its
+// 64-token form first.
+inline Problem tc_tiles(const Problem& p) {
+  Problem t = p;
+  t.Q = 64;
+  t.nc = (p.L + 63) / 64;
+  return t;
+}
+
 // Workspace of the tensor-core path, carved from the caller's buffer.
 struct TcWorkspace {
   int* err;               // nonzero after a kernel gave up on a bounded wait

@@ -644,7 +644,7 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
 }  // namespace
 
 const char* tc_main_kernel(const Problem& p) {
-  return p.N == 128 && tc_pair_supported(p) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
+  return p.N == 128 && tc_pair_supported(tc_tiles(p)) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
 }
 
 cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0,
