@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nc = (int)a.nc;
   // a small persistent grid walks the list of units the fast kernel could not do
+  griddep_wait();  // the list comes from the fused kernel launched before this one
   const int count = *reinterpret_cast<const volatile int*>(a.failed_count);
   if ((int)blockIdx.x >= count) return;  // uniform: every thread reads the same count
 
@@ -561,8 +562,8 @@ cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return cudaErrorInvalidValue;
   const int64_t grid = p.b * p.H < (int64_t)Cfg<NS>::kMinBlocks * sms ? p.b * p.H : (int64_t)Cfg<NS>::kMinBlocks * sms;
-  k_ssd_fwd_tc<NS><<<(unsigned)grid, Cfg<NS>::kThreads, Cfg<NS>::kSmemBytes, st>>>(tx, tb, tc_, a);
-  return cudaGetLastError();
+  return launch_dependent(k_ssd_fwd_tc<NS>, (unsigned)grid, Cfg<NS>::kThreads, Cfg<NS>::kSmemBytes, st, tx, tb, tc_,
+                          a);
 }
 
 }  // namespace

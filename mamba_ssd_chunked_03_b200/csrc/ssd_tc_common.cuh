@@ -69,6 +69,25 @@ bool make_map_dt(CUtensorMap* m, const float* dt, int64_t H, int64_t L, int64_t 
 
 }  // namespace tc
 
+// Launch `kernel` so that it may start while the previous kernel on the
+// stream is still running (programmatic dependent launch): the kernel calls
+// griddep_wait() before it reads what that kernel wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                             Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // The tensor-core kernels work on 64-token chunks.  A chunk of Q = 128 or 256
 // tokens is computed as Q/64 consecutive 64-token chunks: the chunked
 // decomposition is an exact re-association of the recurrence, so refining

@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(128) k_chunk_cb(const __grid_constant__ CUtens
   __shared__ int abort_flag;
   __shared__ int never;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  griddep_launch_dependents();  // the fused kernel may set up while this grid runs
   const int64_t r = blockIdx.x;
   const int64_t g = r % a.G;
   const int64_t c = (r / a.G) % a.nc;
@@ -204,6 +205,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
                                                        ~uintptr_t(1023));
   __shared__ FastSmem s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  griddep_launch_dependents();  // the exact kernel may set up while this grid runs
   const int64_t unit = blockIdx.x;
   const int64_t b = unit / a.H, h = unit % a.H;
   const int64_t g = h / a.hpg;
@@ -339,6 +341,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     for (int k = 0; k < 2 && k < nc && ok; ++k) ok = scan_next();
     if (lane == 0 && ok) {
       for (int c = 0; c < 3 && c < nc; ++c) issue_x(c);
+      griddep_wait();  // W' comes from the C B^T kernel launched before this one
       for (int c = 0; c < 2 && c < nc; ++c) {
         issue_w(c);
         issue_c(c);
@@ -635,9 +638,9 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
                            (int)FastCfg<NS>::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
-  k_ssd_fwd_fast<NS><<<(unsigned)(p.b * p.H), FastCfg<NS>::kThreads, FastCfg<NS>::kSmemBytes, st>>>(tx, tb, tc_,
-                                                                                                      tw, fa);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = launch_dependent(k_ssd_fwd_fast<NS>, (unsigned)(p.b * p.H), FastCfg<NS>::kThreads, FastCfg<NS>::kSmemBytes, st,
+                       tx, tb, tc_, tw, fa);
+  if (e != cudaSuccess) return e;
   return ev1 ? cudaEventRecord(ev1, st) : cudaSuccess;
 }
 

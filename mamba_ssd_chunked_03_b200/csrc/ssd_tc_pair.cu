@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(512, 1)
                                                        ~uintptr_t(1023));
   __shared__ PairSmem s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  griddep_launch_dependents();  // the exact kernel may set up while this grid runs
   const int64_t pairs = a.H / 2;
   const int nc = (int)a.nc;
 
@@ -272,6 +273,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int c = 3; c < 6 && c < total; ++c) prefetch_x(c);
         #pragma unroll 1
         for (int c = 0; c < 3 && c < total; ++c) issue_x(c);  // slot 3 starts free
+        griddep_wait();  // W' comes from the C B^T kernel launched before this one
         #pragma unroll 1
         for (int c = 0; c < 2 && c < total; ++c) {
           issue_wb(c);
@@ -725,8 +727,8 @@ cudaError_t tc_pair_launch(const Problem& p, const TcWorkspace& w, const CUtenso
   a.handoff = w.handoff;
   a.flags = w.flags;
   a.pair_bad = w.pair_bad;
-  k_ssd_fwd_pair<<<(unsigned)grid, PairCfg::kThreads, PairCfg::kSmemBytes, st>>>(tx, tb, tc_, tw, ty, tdt, a);
-  return cudaGetLastError();
+  return launch_dependent(k_ssd_fwd_pair, (unsigned)grid, PairCfg::kThreads, PairCfg::kSmemBytes, st, tx, tb, tc_, tw,
+                          ty, tdt, a);
 }
 
 }  // namespace ssd
