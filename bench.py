@@ -299,8 +299,10 @@ def main():
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     launches_per_call = ssd.launch_count(g["x"], g["B"], shape.chunk_size, g.get("seq_idx"), num_seqs, True,
                                          generic=args.generic)
-    path = ssd.kernel_path(g["x"], g["B"], shape.chunk_size, generic=args.generic)
-    main_kernel = ssd.main_kernel(g["x"], g["dt"], g["B"], shape.chunk_size, generic=args.generic)
+    path = ssd.kernel_path(g["x"], g["B"], shape.chunk_size, generic=args.generic, seq_idx=g.get("seq_idx"),
+                           num_seqs=num_seqs)
+    main_kernel = ssd.main_kernel(g["x"], g["dt"], g["B"], shape.chunk_size, generic=args.generic,
+                                  seq_idx=g.get("seq_idx"), num_seqs=num_seqs)
 
     K = args.steps
     # the fused kernel's own duration is timed in a separate loop: events

@@ -163,15 +163,17 @@ def launch_count(x, B, chunk_size: int, seq_idx=None, num_seqs=None, final_state
     return int(lib.ssd_fwd_launch_count(ctypes.byref(a)))
 
 
-def kernel_path(x, B, chunk_size: int, generic: bool = False) -> str:
-    a = make_args(x, None, None, B, None, chunk_size=chunk_size, generic=generic)
+def kernel_path(x, B, chunk_size: int, generic: bool = False, seq_idx=None, num_seqs=None) -> str:
+    a = make_args(x, None, None, B, None, chunk_size=chunk_size, seq_idx=seq_idx, num_seqs=num_seqs,
+                  generic=generic)
     return lib.ssd_fwd_path(ctypes.byref(a)).decode()
 
 
-def main_kernel(x, dt, B, chunk_size: int, generic: bool = False) -> str:
+def main_kernel(x, dt, B, chunk_size: int, generic: bool = False, seq_idx=None, num_seqs=None) -> str:
     """Name of the fused kernel a call with these tensors is dominated by
     (the one ``timing_events`` bracket)."""
-    a = make_args(x, dt, None, B, None, chunk_size=chunk_size, generic=generic)
+    a = make_args(x, dt, None, B, None, chunk_size=chunk_size, seq_idx=seq_idx, num_seqs=num_seqs,
+                  generic=generic)
     return lib.ssd_fwd_main_kernel(ctypes.byref(a)).decode()
 
 
