@@ -81,6 +81,18 @@ bool make_map_3d(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_map_bc(CUtensorMap* m, const void* base, int64_t N, int64_t G, int64_t L, int64_t b) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)N, (cuuint64_t)G, (cuuint64_t)L, (cuuint64_t)b};
+  const cuuint64_t strides[3] = {(cuuint64_t)(N * 2), (cuuint64_t)(G * N * 2), (cuuint64_t)(L * G * N * 2)};
+  const cuuint32_t box[4] = {64, 1, 64, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map_dt(CUtensorMap* m, const float* dt, int64_t H, int64_t L, int64_t b) {
   EncodeTiledFn enc = encode_fn();
   if (!enc || (H * 4) % 16 != 0) return false;
@@ -124,6 +136,7 @@ struct Cfg {
 
 struct TcArgs {
   int64_t b, L, H, G, hpg, nc;
+  int64_t Nr;  // the problem's d_state (<= NS; state rows past it are zero padding)
   const float* dt;
   const float* A;
   const float* D;
@@ -214,8 +227,8 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
         const int t0 = c * K::Q;
         mbar_arrive_expect_tx(&s.full, K::kStageBytes);
         for (int j = 0; j < K::NB; ++j) {
-          tma_load_3d(sm + K::oC + j * K::kTile, &tm_c, &s.full, (int)(g * NS + 64 * j), t0, (int)b);
-          tma_load_3d(sm + K::oB + j * K::kTile, &tm_b, &s.full, (int)(g * NS + 64 * j), t0, (int)b);
+          tma_load_4d(sm + K::oC + j * K::kTile, &tm_c, &s.full, 64 * j, (int)g, t0, (int)b);
+          tma_load_4d(sm + K::oB + j * K::kTile, &tm_b, &s.full, 64 * j, (int)g, t0, (int)b);
         }
         tma_load_3d(sm + K::oX, &tm_x, &s.full, (int)(h * K::P), t0, (int)b);
         issued = c + 1;
@@ -307,7 +320,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
         const int n = n0 + 128 * hf;
 #pragma unroll
         for (int p = 0; p < 64; ++p)
-          Hs[hf][p] = a.h0 ? a.h0[((b * a.H + h) * 64 + p) * NS + n] : 0.f;
+          Hs[hf][p] = a.h0 && n < a.Nr ? a.h0[((b * a.H + h) * 64 + p) * a.Nr + n] : 0.f;
         // bf16 copy, row n of the [N][64] MN-major operand
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -515,9 +528,11 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
 #pragma unroll
       for (int hf = 0; hf < NH; ++hf) {
         const int n = n0 + 128 * hf;
-        float* dst = a.final_states + ((b * a.H + h) * 64) * NS + n;
+        if (n < a.Nr) {
+          float* dst = a.final_states + ((b * a.H + h) * 64) * a.Nr + n;
 #pragma unroll
-        for (int p = 0; p < 64; ++p) dst[(int64_t)p * NS] = Hs[hf][p];
+          for (int p = 0; p < 64; ++p) dst[(int64_t)p * a.Nr] = Hs[hf][p];
+        }
       }
     }
   }
@@ -534,8 +549,8 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
 template <int NS>
 cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
   CUtensorMap tx, tb, tc_;
-  if (!make_map_3d(&tx, p.x, p.H * p.P, p.L, p.b) || !make_map_3d(&tb, p.B, p.G * p.N, p.L, p.b) ||
-      !make_map_3d(&tc_, p.C, p.G * p.N, p.L, p.b))
+  if (!make_map_3d(&tx, p.x, p.H * p.P, p.L, p.b) || !make_map_bc(&tb, p.B, p.N, p.G, p.L, p.b) ||
+      !make_map_bc(&tc_, p.C, p.N, p.G, p.L, p.b))
     return cudaErrorInvalidValue;
   TcArgs a;
   a.b = p.b;
@@ -548,6 +563,7 @@ cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
   a.A = p.A;
   a.D = p.D;
   a.h0 = p.h0;
+  a.Nr = p.N;
   a.seq = p.seq;
   a.y = static_cast<__nv_bfloat16*>(p.y);
   a.final_states = p.final_states;
@@ -604,7 +620,7 @@ bool tc_supported(const Problem& p, uint32_t flags) {
   if (flags & SSD_FLAG_GENERIC) return false;
   if (p.dtype != SSD_BF16) return false;
   if (p.P != 64 || (p.Q != 64 && p.Q != 128 && p.Q != 256)) return false;
-  if (p.N != 128 && p.N != 256) return false;
+  if (p.N != 64 && p.N != 128 && p.N != 256) return false;  // 64 runs zero-padded as 128
   if (p.seq) return false;
   // TMA coordinates are 32-bit
   const Problem t = tc_tiles(p);
@@ -622,7 +638,7 @@ cudaError_t tc_forward(const Problem& pq, void* ws, cudaStream_t st, cudaEvent_t
   cudaError_t e = cudaMemsetAsync(w.err, 0, w.zero_bytes, st);
   if (e != cudaSuccess) return e;
   if ((e = tc_fast_forward(p, w, st, ev0, ev1)) != cudaSuccess) return e;
-  return p.N == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st);
+  return tc_kernel_n(p) == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st);
 }
 
 }  // namespace ssd

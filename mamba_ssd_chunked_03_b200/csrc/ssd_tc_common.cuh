@@ -30,6 +30,7 @@ struct CbArgs {
 
 struct FastArgs {
   int64_t L, H, G, hpg, nc, batch;
+  int64_t Nr;  // the problem's d_state (<= the kernel's N; rows past it are zero padding)
   const float* dt;
   const float* A;
   const float* D;
@@ -63,6 +64,11 @@ __device__ __forceinline__ void unpack_bf16x2(uint32_t u, float& lo, float& hi) 
 // 3-D bf16 tensor map over (outer, rows, inner) with a 64 x 64 x 1 box and
 // 128-byte swizzle; rows past `rows` read as zeros.
 bool make_map_3d(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t outer);
+// bf16 tensor map over B or C (b, L, G, N) as 4-D (n, group, token, row) with
+// a 64 x 1 x 64 x 1 box and 128-byte swizzle: a box at n = 64 of an N = 64
+// tensor lies outside it and reads as zeros, which is how the kernels built
+// for N = 128 run N = 64 (the state is zero-padded to 128 rows).
+bool make_map_bc(CUtensorMap* m, const void* base, int64_t N, int64_t G, int64_t L, int64_t b);
 // fp32 tensor map over dt (b, L, H) with a 4-head x 64-token box, no swizzle;
 // needs H * 4 bytes to be a multiple of 16.  Tokens past L read as zeros.
 bool make_map_dt(CUtensorMap* m, const float* dt, int64_t H, int64_t L, int64_t b);
@@ -94,6 +100,9 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned b
 // the chunks changes only the rounding, not the result.  Every tensor-core
 // entry point (ssd_tc.cu, ssd_tc_fast.cu) turns the problem into its
 // 64-token form first.
+// d_state the kernels are built for: 64 runs zero-padded as 128
+inline int tc_kernel_n(const Problem& p) { return p.N == 256 ? 256 : 128; }
+
 inline Problem tc_tiles(const Problem& p) {
   Problem t = p;
   t.Q = 64;

@@ -104,8 +104,8 @@ __global__ void __launch_bounds__(128) k_chunk_cb(const __grid_constant__ CUtens
   if (tid == 0) {
     mbar_arrive_expect_tx(&bar_full, 2 * K::NB * K::kTile);
     for (int j = 0; j < K::NB; ++j) {
-      tma_load_3d(sm + K::oC + j * K::kTile, &tm_c, &bar_full, (int)(g * NS + 64 * j), t0, (int)b);
-      tma_load_3d(sm + K::oB + j * K::kTile, &tm_b, &bar_full, (int)(g * NS + 64 * j), t0, (int)b);
+      tma_load_4d(sm + K::oC + j * K::kTile, &tm_c, &bar_full, 64 * j, (int)g, t0, (int)b);
+      tma_load_4d(sm + K::oB + j * K::kTile, &tm_b, &bar_full, 64 * j, (int)g, t0, (int)b);
     }
     if (mbar_wait(&bar_full, 0, abort_p, kWaitLimitNs)) {
       tc_fence_after();
@@ -326,15 +326,14 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     auto issue_b = [&](int c) {
       mbar_arrive_expect_tx(&s.full_b, K::NB * K::kTile);
       for (int j = 0; j < K::NB; ++j)
-        tma_load_3d(sm + K::oB + j * K::kTile, &tm_b, &s.full_b, (int)(g * NS + 64 * j), c * 64, (int)b);
+        tma_load_4d(sm + K::oB + j * K::kTile, &tm_b, &s.full_b, 64 * j, (int)g, c * 64, (int)b);
       last_b = c;
     };
     auto issue_c = [&](int c) {
       uint64_t* bar = &s.full_c[c & 1];
       mbar_arrive_expect_tx(bar, K::NB * K::kTile);
       for (int j = 0; j < K::NB; ++j)
-        tma_load_3d(sm + K::oC + ((c & 1) * K::NB + j) * K::kTile, &tm_c, bar, (int)(g * NS + 64 * j), c * 64,
-                    (int)b);
+        tma_load_4d(sm + K::oC + ((c & 1) * K::NB + j) * K::kTile, &tm_c, bar, 64 * j, (int)g, c * 64, (int)b);
       last_c = c;
     };
     bool ok = true;
@@ -450,7 +449,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     for (int hf = 0; hf < K::NH; ++hf)
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        H[hf][j] = a.h0 ? a.h0[((b * a.H + h) * 64 + pc0 + j) * NS + n0 + 128 * hf] : 0.f;
+        H[hf][j] = a.h0 && n0 + 128 * hf < a.Nr ? a.h0[((b * a.H + h) * 64 + pc0 + j) * a.Nr + n0 + 128 * hf] : 0.f;
     bool failed = false;
 
     for (int c = 0; c <= nc; ++c) {
@@ -569,9 +568,10 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     if (!failed && a.final_states) {
 #pragma unroll
       for (int hf = 0; hf < K::NH; ++hf) {
-        float* dst = a.final_states + ((b * a.H + h) * 64 + pc0) * NS + n0 + 128 * hf;
+        if (n0 + 128 * hf >= a.Nr) continue;
+        float* dst = a.final_states + ((b * a.H + h) * 64 + pc0) * a.Nr + n0 + 128 * hf;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(int64_t)j * NS] = H[hf][j];
+        for (int j = 0; j < 32; ++j) dst[(int64_t)j * a.Nr] = H[hf][j];
       }
     }
   }
@@ -591,8 +591,8 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
 template <int NS>
 cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
   CUtensorMap tx, tb, tc_, tw;
-  if (!make_map_3d(&tx, p.x, p.H * p.P, p.L, p.b) || !make_map_3d(&tb, p.B, p.G * p.N, p.L, p.b) ||
-      !make_map_3d(&tc_, p.C, p.G * p.N, p.L, p.b) || !make_map_3d(&tw, w.wp, 64, p.b * p.nc * p.G * 64, 1))
+  if (!make_map_3d(&tx, p.x, p.H * p.P, p.L, p.b) || !make_map_bc(&tb, p.B, p.N, p.G, p.L, p.b) ||
+      !make_map_bc(&tc_, p.C, p.N, p.G, p.L, p.b) || !make_map_3d(&tw, w.wp, 64, p.b * p.nc * p.G * 64, 1))
     return cudaErrorInvalidValue;
   CbArgs ca;
   ca.L = p.L;
@@ -617,6 +617,7 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
   fa.A = p.A;
   fa.D = p.D;
   fa.h0 = p.h0;
+  fa.Nr = p.N;
   fa.y = static_cast<__nv_bfloat16*>(p.y);
   fa.final_states = p.final_states;
   fa.failed_count = w.failed_count;
@@ -647,12 +648,12 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
 }  // namespace
 
 const char* tc_main_kernel(const Problem& p) {
-  return p.N == 128 && tc_pair_supported(tc_tiles(p)) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
+  return tc_kernel_n(p) == 128 && tc_pair_supported(tc_tiles(p)) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
 }
 
 cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0,
                             cudaEvent_t ev1) {
-  return p.N == 128 ? launch_fast<128>(p, w, st, ev0, ev1) : launch_fast<256>(p, w, st, ev0, ev1);
+  return tc_kernel_n(p) == 128 ? launch_fast<128>(p, w, st, ev0, ev1) : launch_fast<256>(p, w, st, ev0, ev1);
 }
 
 }  // namespace ssd

@@ -247,8 +247,8 @@ __global__ void __launch_bounds__(512, 1)
         mbar_arrive_expect_tx(&s.full_wb[i], (1 + K::NB) * K::kTile);
         tma_load_3d(sm + K::oW + i * K::kTile, &tm_w, &s.full_wb[i], 0, ((bb * nc + uwb.c) * (int)a.G + grp) * 64, 0);
         for (int jb = 0; jb < K::NB; ++jb)
-          tma_load_3d(sm + K::oB + (i * K::NB + jb) * K::kTile, &tm_b, &s.full_wb[i], grp * NS + 64 * jb,
-                      uwb.c * 64, bb);
+          tma_load_4d(sm + K::oB + (i * K::NB + jb) * K::kTile, &tm_b, &s.full_wb[i], 64 * jb, grp, uwb.c * 64,
+                      bb);
         uwb.next(s);
         last_wb = gg;
       };
@@ -256,8 +256,7 @@ __global__ void __launch_bounds__(512, 1)
         const int i = gg & 1, bb = s.seg_b[uc.k], grp = s.seg_grp[uc.k];
         mbar_arrive_expect_tx(&s.full_c[i], K::NB * K::kTile);
         for (int jb = 0; jb < K::NB; ++jb)
-          tma_load_3d(sm + K::oC + (i * K::NB + jb) * K::kTile, &tm_c, &s.full_c[i], grp * NS + 64 * jb,
-                      uc.c * 64, bb);
+          tma_load_4d(sm + K::oC + (i * K::NB + jb) * K::kTile, &tm_c, &s.full_c[i], 64 * jb, grp, uc.c * 64, bb);
         uc.next(s);
         last_c = gg;
       };
@@ -557,10 +556,10 @@ __global__ void __launch_bounds__(512, 1)
     auto seg_begin = [&](int k) -> bool {
       const int64_t h = s.seg_h0[k] + j, bb = s.seg_b[k];
       if (s.seg_c0[k] == 0) {
-        if (a.h0) {
-          const float* src = a.h0 + ((bb * a.H + h) * 64) * NS + n;
+        if (a.h0 && n < a.Nr) {
+          const float* src = a.h0 + ((bb * a.H + h) * 64) * a.Nr + n;
 #pragma unroll
-          for (int p = 0; p < 64; ++p) H[p] = src[p * NS];
+          for (int p = 0; p < 64; ++p) H[p] = src[p * a.Nr];
         } else {
 #pragma unroll
           for (int p = 0; p < 64; ++p) H[p] = 0.f;
@@ -588,10 +587,10 @@ __global__ void __launch_bounds__(512, 1)
     auto seg_end = [&](int k) {
       const int64_t h = s.seg_h0[k] + j, bb = s.seg_b[k];
       if (s.seg_c0[k] + s.seg_len[k] == nc) {
-        if (a.final_states) {
-          float* dst = a.final_states + ((bb * a.H + h) * 64) * NS + n;
+        if (a.final_states && n < a.Nr) {
+          float* dst = a.final_states + ((bb * a.H + h) * 64) * a.Nr + n;
 #pragma unroll
-          for (int p = 0; p < 64; ++p) dst[(int64_t)p * NS] = H[p];
+          for (int p = 0; p < 64; ++p) dst[(int64_t)p * a.Nr] = H[p];
         }
         return;
       }
@@ -698,7 +697,7 @@ __global__ void __launch_bounds__(512, 1)
 
 // (the kernel counts its (pair, chunk) steps in 32-bit integers)
 bool tc_pair_shape_ok(const Problem& p) {
-  return p.N == 128 && p.hpg % 2 == 0 && p.H % 4 == 0 && (p.b * p.H / 2) * p.nc < ((int64_t)1 << 30);
+  return tc_kernel_n(p) == 128 && p.hpg % 2 == 0 && p.H % 4 == 0 && (p.b * p.H / 2) * p.nc < ((int64_t)1 << 30);
 }
 
 // dt is read by TMA, whose base address must be 16-byte aligned

@@ -35,6 +35,8 @@ SMALL = [
     # and hands the state over (4 chunks per row; ragged 13-chunk rows)
     (4, 200, 80, 64, 128, 1, 64, 0.1),
     (2, 777, 160, 64, 128, 2, 64, 0.0),
+    # N = 64 on the two-head kernel (state zero-padded to 128 rows), with hand-over
+    (4, 200, 80, 64, 64, 1, 64, 0.1),
 ]
 
 
@@ -119,6 +121,43 @@ def test_chunk_size_invariance_on_gpu():
         y, f = run_gpu(d, Q)
         assert rel_l2(y, yr) <= 1e-5, (Q, rel_l2(y, yr))
         assert state_err(f, fr) <= 1e-5, (Q, state_err(f, fr))
+
+
+@pytest.mark.parametrize("case", [
+    # b, L, H, P, N, G, Q, h0_std: N = 128 shapes the two-head kernel does not take
+    (1, 300, 6, 64, 128, 3, 64, 0.2),    # H not a multiple of 4
+    (2, 200, 3, 64, 128, 1, 64, 0.0),    # an odd number of heads per group
+    (1, 300, 3, 64, 64, 1, 64, 0.2),     # N = 64, zero-padded to 128 rows
+], ids=_id)
+def test_single_head_kernel_takes_the_other_n128_shapes(case):
+    b, L, H, P, N, G, Q, h0 = case
+    shape = si.SSDShape("sh", b, L, H, P, N, G, Q, "bf16", h0_std=h0, seed=H * 10 + G)
+    d = si.make_inputs(shape)
+    g = to_dev(d)
+    assert ssd.main_kernel(g["x"], g["dt"], g["B"], Q) == "k_ssd_fwd_fast"
+    y, f = run_gpu(d, Q)
+    yr, fr = run_oracle(d)
+    assert rel_l2(y, yr) <= 1e-2, rel_l2(y, yr)
+    assert state_err(f, fr) <= 1e-2, state_err(f, fr)
+
+
+def test_unaligned_dt_takes_the_single_head_kernel():
+    """The two-head kernel reads dt by TMA (16-byte aligned base); a dt view
+    that starts 4 bytes into its storage goes to the single-head kernel."""
+    s = si.SSDShape("ua", 2, 300, 8, 64, 128, 1, 64, "bf16", h0_std=0.1, seed=12)
+    d = si.make_inputs(s)
+    g = to_dev(d)
+    store = torch.empty(g["dt"].numel() + 1, device="cuda", dtype=torch.float32)
+    dt = store[1:].view_as(g["dt"])
+    dt.copy_(g["dt"])
+    assert dt.data_ptr() % 16 != 0
+    assert ssd.main_kernel(g["x"], dt, g["B"], 64) == "k_ssd_fwd_fast"
+    assert ssd.main_kernel(g["x"], g["dt"], g["B"], 64) == "k_ssd_fwd_pair"
+    y, f = ssd.fwd(g["x"], dt, g["A"], g["B"], g["C"], g["D"], chunk_size=64, initial_states=g["initial_states"])
+    torch.cuda.synchronize()
+    yr, fr = run_oracle(d)
+    assert rel_l2(y.float().cpu().numpy(), yr) <= 1e-2
+    assert state_err(f.cpu().numpy(), fr) <= 1e-2
 
 
 def test_device_status_reports_no_timeout_after_a_normal_call():
