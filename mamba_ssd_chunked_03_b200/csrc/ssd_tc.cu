@@ -30,6 +30,12 @@
 // zero transition at packed-sequence boundaries ("Transformers与SSMs的隐藏联系"
 // section 4.2).
 //
+// Packed sequences (seq_idx) run on this kernel alone, over every unit: it
+// also writes each sequence's final state, from the updated state when the
+// sequence ends on a chunk's last token, and otherwise from the state at the
+// chunk's start plus the sequence's own tokens of the chunk (CUDA cores,
+// while the chunk's x and B tiles are still held).
+//
 // Warp roles (192 threads):  warp 0 TMA producer, warp 1 MMA issuer (one
 // thread), warps 2-5 compute (cumsum, mask, scale, state update, epilogue).
 // Every wait is bounded; a CTA that times out records the error, drains its
@@ -144,8 +150,9 @@ struct TcArgs {
   const int32_t* seq;
   __nv_bfloat16* y;
   float* final_states;
-  const int* failed_count;  // units to process, listed by the fast kernel
+  const int* failed_count;  // units to process, listed by the fast kernel ...
   const int* failed_list;
+  int all_units;            // ... or, if set, every unit (packed sequences)
   int* err;
 };
 
@@ -175,7 +182,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
   const int nc = (int)a.nc;
   // a small persistent grid walks the list of units the fast kernel could not do
   griddep_wait();  // the list comes from the fused kernel launched before this one
-  const int count = *reinterpret_cast<const volatile int*>(a.failed_count);
+  const int count = a.all_units ? (int)(a.b * a.H) : *reinterpret_cast<const volatile int*>(a.failed_count);
   if ((int)blockIdx.x >= count) return;  // uniform: every thread reads the same count
 
   if (tid == 0) {
@@ -198,7 +205,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
   volatile int* never = &s.never;
 
   for (int it = blockIdx.x; it < count; it += gridDim.x) {
-  const int64_t unit = a.failed_list[it];
+  const int64_t unit = a.all_units ? it : a.failed_list[it];
   const int64_t b = unit / a.H, h = unit % a.H;
   const int64_t g = h / a.hpg;
   if (tid == 0) {  // fresh barriers per unit (all earlier phases have completed)
@@ -407,6 +414,57 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
           v.w = pack_bf16x2(f0 * w, f1 * w);
           *reinterpret_cast<uint4*>(sm + K::oXt + off) = v;
         }
+        // sequences that end inside this chunk before its last token: their
+        // final state is the decayed carry (same sequence as the chunk's
+        // start) plus their own tokens' terms.  x and B stay valid until the
+        // MMAs of this chunk, which wait for xt_ready below, are done.
+        if (a.seq && a.final_states) {
+          const int n0 = 32 * q + lane;
+          for (int t = 0; t < e; ++t) {
+            const int sq = s.seqs[t];
+            if (sq == s.seqs[t + 1]) continue;
+            int ts = t;
+            while (ts > 0 && s.seqs[ts - 1] == sq) --ts;
+            const float cst = s.cs2[t];
+            const float carry = (ts == 0 && sq == seq_prev) ? exp2f(cst) : 0.f;
+#pragma unroll
+            for (int pb = 0; pb < 64; pb += 16) {
+              float acc[NH][16];
+#pragma unroll
+              for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+                for (int k = 0; k < 16; ++k) acc[hf][k] = carry * Hs[hf][pb + k];
+              for (int si = ts; si <= t; ++si) {
+                const float w = exp2f(cst - s.cs2[si]) * s.dts[si];
+                const uint4 xa = *reinterpret_cast<const uint4*>(sm + K::oX + sw128((uint32_t)si * 128 + (pb / 8) * 16));
+                const uint4 xb =
+                    *reinterpret_cast<const uint4*>(sm + K::oX + sw128((uint32_t)si * 128 + (pb / 8 + 1) * 16));
+                const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+                float xv[16];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) unpack_bf16x2(xw[k], xv[2 * k], xv[2 * k + 1]);
+#pragma unroll
+                for (int hf = 0; hf < NH; ++hf) {
+                  const int n = n0 + 128 * hf;
+                  const float bv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                      sm + K::oB + (n >> 6) * K::kTile + sw128((uint32_t)si * 128 + (n & 63) * 2)));
+                  const float wb = w * bv;
+#pragma unroll
+                  for (int k = 0; k < 16; ++k) acc[hf][k] = fmaf(wb, xv[k], acc[hf][k]);
+                }
+              }
+#pragma unroll
+              for (int hf = 0; hf < NH; ++hf) {
+                const int n = n0 + 128 * hf;
+                if (n < a.Nr) {
+                  float* dst = a.final_states + (((int64_t)sq * a.H + h) * 64 + pb) * a.Nr + n;
+#pragma unroll
+                  for (int k = 0; k < 16; ++k) dst[(int64_t)k * a.Nr] = acc[hf][k];
+                }
+              }
+            }
+          }
+        }
         fence_proxy_async_smem();
         mbar_arrive(&s.xt_ready);
       }
@@ -473,6 +531,20 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
         }
         tc_fence_before();
         mbar_arrive(&s.s_free);
+        // the sequence of the chunk's last token ends there: its final state
+        if (a.seq && a.final_states &&
+            ((int64_t)t0 + e + 1 >= a.L || a.seq[rowbase + t0 + e + 1] != seq_e)) {
+          const int n0 = 32 * q + lane;
+#pragma unroll
+          for (int hf = 0; hf < NH; ++hf) {
+            const int n = n0 + 128 * hf;
+            if (n < a.Nr) {
+              float* dst = a.final_states + (((int64_t)seq_e * a.H + h) * 64) * a.Nr + n;
+#pragma unroll
+              for (int p = 0; p < 64; ++p) dst[(int64_t)p * a.Nr] = Hs[hf][p];
+            }
+          }
+        }
       }
       // ---- wait for Yd / Yo (MMA3 of this chunk no longer reads H), publish H
       if (!mbar_wait_warp(&s.y_full, par, abort_flag, kWaitLimitNs)) {
@@ -569,6 +641,7 @@ cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
   a.final_states = p.final_states;
   a.failed_count = w.failed_count;
   a.failed_list = w.failed_list;
+  a.all_units = p.seq != nullptr;
   a.err = w.err;
   cudaError_t e = cudaFuncSetAttribute(k_ssd_fwd_tc<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Cfg<NS>::kSmemBytes);
@@ -621,7 +694,7 @@ bool tc_supported(const Problem& p, uint32_t flags) {
   if (p.dtype != SSD_BF16) return false;
   if (p.P != 64 || (p.Q != 64 && p.Q != 128 && p.Q != 256)) return false;
   if (p.N != 64 && p.N != 128 && p.N != 256) return false;  // 64 runs zero-padded as 128
-  if (p.seq) return false;
+  // packed sequences: the exact kernel alone (see its header), for Q >= 64
   // TMA coordinates are 32-bit
   const Problem t = tc_tiles(p);
   if (t.b * t.nc * t.G * 64 >= ((int64_t)1 << 31) || t.L >= ((int64_t)1 << 31)) return false;
@@ -630,13 +703,24 @@ bool tc_supported(const Problem& p, uint32_t flags) {
 
 size_t tc_workspace_bytes(const Problem& p) { return tc_workspace_need(tc_tiles(p)); }
 
-int tc_launch_count(const Problem&) { return 3; }
+int tc_launch_count(const Problem& p) { return p.seq ? 1 : 3; }
 
 cudaError_t tc_forward(const Problem& pq, void* ws, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
   const Problem p = tc_tiles(pq);
   const TcWorkspace w = tc_carve(p, ws);
   cudaError_t e = cudaMemsetAsync(w.err, 0, w.zero_bytes, st);
   if (e != cudaSuccess) return e;
+  if (p.seq) {
+    // packed sequences: every unit on the exact kernel; sequence ids that never
+    // occur keep zero final states
+    if (p.final_states &&
+        (e = cudaMemsetAsync(p.final_states, 0, sizeof(float) * (size_t)(p.num_seqs * p.H * p.P * p.N), st)) !=
+            cudaSuccess)
+      return e;
+    if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
+    if ((e = (tc_kernel_n(p) == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st))) != cudaSuccess) return e;
+    return ev1 ? cudaEventRecord(ev1, st) : cudaSuccess;
+  }
   if ((e = tc_fast_forward(p, w, st, ev0, ev1)) != cudaSuccess) return e;
   return tc_kernel_n(p) == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st);
 }

@@ -648,6 +648,7 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
 }  // namespace
 
 const char* tc_main_kernel(const Problem& p) {
+  if (p.seq) return "k_ssd_fwd_tc";
   return tc_kernel_n(p) == 128 && tc_pair_supported(tc_tiles(p)) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
 }
 

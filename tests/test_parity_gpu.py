@@ -91,6 +91,43 @@ def test_packed(case, dtype):
     assert state_err(f, fr) <= TOL[dtype], state_err(f, fr)
 
 
+PACKED_TC = [
+    # per-row lengths, N, Q, h0_std: bf16 with Q >= 64 runs on the exact tensor-core kernel
+    ([[5, 16, 16, 27, 64, 1, 1, 30]], 128, 64, 0.3),   # ends mid-chunk, on chunk edges, 1-token sequences
+    ([[100, 37, 1, 118], [256]], 256, 64, 0.2),         # two rows, ids numbered across rows
+    ([[300, 212]], 128, 256, 0.0),                      # one boundary, 256-token chunks
+    ([[64, 64, 1, 63, 64, 60]], 64, 128, 0.1),          # N = 64 (zero-padded), ends before chunk edges
+]
+
+
+@pytest.mark.parametrize("case", PACKED_TC, ids=lambda c: f"N{c[1]}_Q{c[2]}_rows{len(c[0])}_n{sum(map(len, c[0]))}")
+def test_packed_on_the_tensor_core_path(case):
+    rows, N, Q, h0 = case
+    L = sum(rows[0])
+    shape = si.SSDShape("packed_tc", len(rows), L, 4, 64, N, 2, Q, "bf16", h0_std=h0, seed=L + N)
+    d = si.make_inputs(shape)
+    d["seq_idx"], d["num_seqs"] = si.seq_idx_from_lengths(rows)
+    g = to_dev(d)
+    assert ssd.kernel_path(g["x"], g["B"], Q, seq_idx=g["seq_idx"], num_seqs=d["num_seqs"]) == "tcgen05"
+    y, f = run_gpu(d, Q)
+    yr, fr = run_oracle(d)
+    assert f.shape == fr.shape == (d["num_seqs"], 4, 64, N)
+    assert rel_l2(y, yr) <= 1e-2, rel_l2(y, yr)
+    assert state_err(f, fr) <= 1e-2, state_err(f, fr)
+
+
+def test_packed_absent_ids_get_zero_states_on_the_tensor_core_path():
+    shape = si.SSDShape("packed", 1, 160, 2, 64, 128, 1, 64, "bf16", seed=19)
+    d = si.make_inputs(shape)
+    sq = torch.tensor([[0] * 70 + [2] * 90], dtype=torch.int32)  # ids 1 and 3 never occur
+    d["seq_idx"], d["num_seqs"] = sq, 4
+    y, f = run_gpu(d, 64)
+    yr, fr = run_oracle(d)
+    assert rel_l2(y, yr) <= 1e-2
+    assert not f[1].any() and not f[3].any()
+    assert state_err(f, fr) <= 1e-2
+
+
 def test_packed_absent_ids_get_zero_states():
     shape = si.SSDShape("packed", 1, 96, 2, 64, 64, 1, 32, "bf16", seed=9)
     d = si.make_inputs(shape)
