@@ -277,6 +277,18 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem desc], bf16 inputs, fp32 accumulate.  A (M = 128)
+// sits one row per TMEM lane, two bf16 of K per 32-bit column (lower K in the
+// low half); a K-step of 16 advances the A address by 8 columns.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive on `bar` once every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -348,6 +360,50 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                  "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])                                          \
                :                                                                                            \
                : "memory")
+
+// 16 lanes x 256 bit (8 columns), 4 repeats along the columns: thread i gets
+// lane base + i/4 at columns 2(i%4), 2(i%4)+1 in r[4j], r[4j+1] and lane
+// base + 8 + i/4 at the same columns in r[4j+2], r[4j+3] (columns offset by 8j)
+// -- the accumulator fragment of mma.sync m16n8.
+#define SSD_TMEM_LD_16x256b_X4(taddr, r)                                                                     \
+  asm volatile(                                                                                              \
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];" \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),      \
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),            \
+        "=r"(r[15])                                                                                         \
+      : "r"(taddr))
+
+// 32 lanes x 32 bit, 32 consecutive columns: thread i writes lane base + i.
+#define SSD_TMEM_ST_32x32b_X32(taddr, r)                                                                     \
+  asm volatile(                                                                                              \
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16," \
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),                     \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),       \
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),          \
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),         \
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                    \
+      : "memory")
+
+// 16 lanes x 128 bit (4 columns), 4 repeats along the columns: thread i
+// writes r[2j] to lane base + i/4 and r[2j+1] to lane base + 8 + i/4, both at
+// column 4j + i%4.
+#define SSD_TMEM_ST_16x128b_X4(taddr, r)                                                                     \
+  asm volatile("tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),     \
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])        \
+               : "memory")
+
+// This thread's tcgen05.st have completed (before a fence and a barrier hand
+// the columns to the MMA).
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Transpose an 8 x 8 matrix of 16-bit values held across the warp: thread i
+// holds row i/4, columns 2(i%4) (low half) and 2(i%4)+1 (high half), before
+// and after.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
 
 // ------------------------------------------------------------------ descriptors
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.

@@ -14,10 +14,11 @@ pytestmark = pytest.mark.gpu
 
 LIB = os.path.join(os.path.dirname(os.path.abspath(__file__)), "cuda", "libtcprobe.so")
 
-SHAPES = {0: (64, 64, 128), 1: (64, 64, 64), 2: (64, 64, 128), 3: (128, 64, 64)}
+SHAPES = {0: (64, 64, 128), 1: (64, 64, 64), 2: (64, 64, 128), 3: (128, 64, 64),
+          4: (128, 64, 64), 5: (128, 64, 128), 6: (128, 64, 64)}
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", list(SHAPES))
 def test_mma_mode(mode):
     lib = ctypes.CDLL(LIB)
     lib.tc_probe_mma.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -38,3 +39,48 @@ def test_mma_mode(mode):
     assert np.isfinite(got).all(), "unwritten outputs"
     rel = np.abs(got - want).max() / np.abs(want).max()
     assert rel < 1e-5, (mode, rel)
+
+
+def _expected_layout():
+    """The lane / column maps the kernels assume (the mma.sync m16n8 fragment)."""
+    exp = np.zeros(4128, dtype=np.int64)
+    for t in range(128):  # 16x256b.x4 load after filling (lane << 16) | column
+        q, i = divmod(t, 32)
+        for j in range(4):
+            for e in range(4):
+                lane = 32 * q + i // 4 + 8 * (e >> 1)
+                col = 8 * j + 2 * (i % 4) + (e & 1)
+                exp[t * 16 + 4 * j + e] = (lane << 16) | col
+    for lane in range(128):  # 16x128b.x4 store of (thread << 8) | register
+        q, l = divmod(lane, 32)
+        for c in range(16):
+            if l >= 16:
+                exp[2048 + lane * 16 + c] = 0xFFFFFFFF
+                continue
+            e, r = divmod(l, 8)
+            i = 4 * r + c % 4
+            exp[2048 + lane * 16 + c] = ((32 * q + i) << 8) | (2 * (c // 4) + e)
+    for i in range(32):  # 8 x 8 transpose: element ids row * 8 + column
+        lo = 2 * (i % 4) * 8 + i // 4
+        hi = (2 * (i % 4) + 1) * 8 + i // 4
+        exp[4096 + i] = lo | (hi << 16)
+    return exp
+
+
+def test_fragment_layouts():
+    lib = ctypes.CDLL(LIB)
+    lib.tc_probe_layout.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    out = torch.zeros(4128, dtype=torch.int32, device="cuda")
+    assert lib.tc_probe_layout(out.data_ptr(), torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().astype(np.int64) & 0xFFFFFFFF
+    exp = _expected_layout()
+    bad = np.nonzero(got != exp)[0]
+    if len(bad):
+        dump = os.environ.get("SSD_PROBE_DUMP")
+        if dump:
+            np.save(dump, got)
+        names = ["16x256b load", "16x128b store", "8x8 transpose"]
+        first = {n: [(int(k), hex(int(got[k])), hex(int(exp[k]))) for k in bad
+                     if (0 if k < 2048 else 1 if k < 4096 else 2) == ni][:4] for ni, n in enumerate(names)}
+        raise AssertionError(f"{len(bad)} mismatches: {first}")
