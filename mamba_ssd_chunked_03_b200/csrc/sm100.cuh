@@ -277,6 +277,19 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// One lane of the (converged) warp: true there, false on the others.  Work
+// that only one lane may do (an MMA issue, a commit) goes under it while the
+// operands it uses are computed by the whole warp, so they stay warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc], bf16 inputs, fp32 accumulate.  A (M = 128)
 // sits one row per TMEM lane, two bf16 of K per 32-bit column (lower K in the
 // low half); a K-step of 16 advances the A address by 8 columns.
@@ -384,6 +397,14 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                    \
       : "memory")
 
+// 32 lanes x 32 bit, 16 consecutive columns: thread i writes lane base + i.
+#define SSD_TMEM_ST_32x32b_X16(taddr, r)                                                                     \
+  asm volatile(                                                                                              \
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" \
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),    \
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])            \
+      : "memory")
+
 // 16 lanes x 128 bit (4 columns), 4 repeats along the columns: thread i
 // writes r[2j] to lane base + i/4 and r[2j+1] to lane base + 8 + i/4, both at
 // column 4j + i%4.
@@ -403,6 +424,23 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
   uint32_t d;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
   return d;
+}
+
+// Four 8 x 8 matrices of 16-bit values, transposed on the way between shared
+// memory and registers.  Thread 8k + r gives the shared address of row r of
+// matrix k (16 bytes: 8 values); register k of thread i holds column i/4 of
+// matrix k at rows 2(i%4) (low half) and 2(i%4)+1 (high half) -- the fragment
+// of its transpose.  stmatrix writes the same correspondence in reverse.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, const uint32_t (&r)[4]) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
 }
 
 // ------------------------------------------------------------------ descriptors

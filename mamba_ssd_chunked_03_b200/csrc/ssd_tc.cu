@@ -666,8 +666,9 @@ TcWorkspace tc_carve(const Problem& p, void* ws, size_t* total) {
   w.err = reinterpret_cast<int*>(base);
   w.failed_count = reinterpret_cast<int*>(base + sizeof(int));
   w.flags = pair ? reinterpret_cast<int*>(base + 2 * sizeof(int)) : nullptr;
-  w.pair_bad = pair ? reinterpret_cast<int*>(base + (2 + 8 * (size_t)kPairGridMax) * sizeof(int)) : nullptr;
-  w.zero_bytes = sizeof(int) * (2 + (pair ? 8 * (size_t)kPairGridMax + (size_t)(p.b * p.H / 2) : 0));
+  const size_t nflags = (size_t)kPairFlagsPerCta * kPairGridMax;
+  w.pair_bad = pair ? reinterpret_cast<int*>(base + (2 + nflags) * sizeof(int)) : nullptr;
+  w.zero_bytes = sizeof(int) * (2 + (pair ? nflags + (size_t)(p.b * p.H / 2) : 0));
   size_t off = align_up(w.zero_bytes, kWsAlign);
   w.wp = reinterpret_cast<__nv_bfloat16*>(base + off);
   off = align_up(off + sizeof(__nv_bfloat16) * (size_t)(p.b * p.nc * p.G * 64 * 64), kWsAlign);

@@ -42,13 +42,14 @@ struct FastArgs {
   int* err;
   // two-head kernel only: state hand-over between the CTAs that share a pair
   float* handoff;  // [grid][2 heads][128 states][64 p] fp32
-  int* flags;      // [grid][8 state warps]: 1 once that warp's part of the hand-over is written
+  int* flags;      // [grid][kPairFlagsPerCta state warps]: 1 once that warp's part of the hand-over is written
   int* pair_bad;   // [b * H / 2]: 1 once a pair was put on the exact kernel's list
 };
 
 // persistent grid of the two-head kernel, at most; per-CTA hand-over size
 constexpr int kPairGridMax = 256;
 constexpr int kPairHandoffFloats = 2 * 128 * 64;
+constexpr int kPairFlagsPerCta = 8;  // one per state warp
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -114,7 +115,7 @@ inline Problem tc_tiles(const Problem& p) {
 struct TcWorkspace {
   int* err;               // nonzero after a kernel gave up on a bounded wait
   int* failed_count;      // next to err; err .. zero_bytes is cleared by one memset per call
-  int* flags;             // two-head kernel: hand-over flags (kPairGridMax x 8), or null
+  int* flags;             // two-head kernel: hand-over flags (kPairGridMax x kPairFlagsPerCta), or null
   int* pair_bad;          // two-head kernel: per-pair exact-kernel marks, or null
   size_t zero_bytes;
   __nv_bfloat16* wp;      // masked C B^T per (b, chunk, group)

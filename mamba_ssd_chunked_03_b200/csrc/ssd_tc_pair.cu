@@ -311,52 +311,57 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      const uint32_t aW = smem_u32(sm + K::oW), aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB);
-      const uint32_t aX = smem_u32(sm + K::oX), aH = smem_u32(sm + K::oH);
-      constexpr uint32_t id_y = idesc_bf16(64, 128, 0, 1);    // A K-major, B MN-major (2 heads)
-      constexpr uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // both MN-major
-      #pragma unroll 1
-      for (int c = 0; c < total; ++c) {
-        const int i = c & 1;
-        const uint32_t ph = (c >> 1) & 1;
-        bool ok = mbar_wait(&s.full_wb[i], ph, abort_flag, kWaitLimitNs);
-        ok = ok && mbar_wait(&s.xp_ready[c & 3], (c >> 2) & 1, abort_flag, kWaitLimitNs);
-        if (c >= 2) ok = ok && mbar_wait(&s.acc_free[i], ((c - 2) >> 1) & 1, abort_flag, kWaitLimitNs);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t yd = tmem + K::tYd0 + 128 * i;
-        const uint32_t st = tmem + K::tS0 + 128 * i;
-        const uint32_t aXp = aX + (c & 3) * 2 * K::kTile;  // X' of both heads, this chunk
+    // The whole warp walks the loop and forms the descriptors (warp-uniform
+    // values); one elected lane issues the MMAs and commits.
+    const uint32_t aW = smem_u32(sm + K::oW), aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB);
+    const uint32_t aX = smem_u32(sm + K::oX), aH = smem_u32(sm + K::oH);
+    constexpr uint32_t id_y = idesc_bf16(64, 128, 0, 1);    // A K-major, B MN-major (2 heads)
+    constexpr uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // both MN-major
+    #pragma unroll 1
+    for (int c = 0; c < total; ++c) {
+      const int i = c & 1;
+      const uint32_t ph = (c >> 1) & 1;
+      bool ok = mbar_wait_warp(&s.full_wb[i], ph, abort_flag, kWaitLimitNs);
+      ok = ok && mbar_wait_warp(&s.xp_ready[c & 3], (c >> 2) & 1, abort_flag, kWaitLimitNs);
+      if (c >= 2) ok = ok && mbar_wait_warp(&s.acc_free[i], ((c - 2) >> 1) & 1, abort_flag, kWaitLimitNs);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t yd = tmem + K::tYd0 + 128 * i;
+      const uint32_t st = tmem + K::tS0 + 128 * i;
+      // X' of both heads, this chunk; a K step of 16 tokens is 16 rows (2048 B)
+      const uint64_t dxp = sw128_desc(aX + (c & 3) * 2 * K::kTile, K::kTile, 1024);
+      const uint64_t dw = sw128_desc(aW + i * K::kTile, 16, 1024);  // a K step is 32 B along the row
+      const uint64_t db = sw128_desc(aB + i * K::NB * K::kTile, K::kTile, 1024);
+      if (elect_one()) {
         // Yd = W' [X'_0 | X'_1]   (K = 64 tokens)
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(yd, sw128_desc(aW + i * K::kTile + kk * 32, 16, 1024),
-                      sw128_desc(aXp + kk * 2048, K::kTile, 1024), id_y, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(yd, dw + 2 * kk, dxp + 128 * kk, id_y, kk > 0);
         // S'^T = B^T [X'_0 | X'_1]   (M = 128 states, K = 64 tokens)
-        const uint32_t aBi = aB + i * K::NB * K::kTile;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(st, sw128_desc(aBi + kk * 2048, K::kTile, 1024), sw128_desc(aXp + kk * 2048, K::kTile, 1024),
-                      id_s, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(st, db + 128 * kk, dxp + 128 * kk, id_s, kk > 0);
         mma_commit(&s.s_full[i]);
-        // Yd += C [e^m H_0 | e^m H_1]^T   (K = N)
-        ok = mbar_wait(&s.h_ready[i], ph, abort_flag, kWaitLimitNs);
-        ok = ok && mbar_wait(&s.full_c[i], ph, abort_flag, kWaitLimitNs);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t aCi = aC + i * K::NB * K::kTile;
-        const uint32_t aHi = aH + i * 2 * K::kHTile;
+      }
+      __syncwarp();
+      // Yd += C [e^m H_0 | e^m H_1]^T   (K = N)
+      ok = mbar_wait_warp(&s.h_ready[i], ph, abort_flag, kWaitLimitNs);
+      ok = ok && mbar_wait_warp(&s.full_c[i], ph, abort_flag, kWaitLimitNs);
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t dc = sw128_desc(aC + i * K::NB * K::kTile, 16, 1024);
+      const uint64_t dh = sw128_desc(aH + i * 2 * K::kHTile, K::kHTile, 1024);
+      if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < NS / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * K::kTile + (kk & 3) * 32;
-          mma_bf16_ss(yd, sw128_desc(aCi + koff, 16, 1024), sw128_desc(aHi + kk * 2048, K::kHTile, 1024), id_y, 1);
-        }
+        for (int kk = 0; kk < NS / 16; ++kk)
+          mma_bf16_ss(yd, dc + ((kk >> 2) * K::kTile + (kk & 3) * 32) / 16, dh + 128 * kk, id_y, 1);
         mma_commit(&s.mma_done[i]);
       }
+      __syncwarp();
+    }
+    if (elect_one()) {
       mma_commit(&s.drain);
       mbar_wait(&s.drain, 0, never, kWaitLimitNs);
     }
+    __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------------------ dt scan
     // lanes 0-15 take head h0, lanes 16-31 head h0 + 1; each lane owns 4
@@ -568,7 +573,7 @@ __global__ void __launch_bounds__(512, 1)
       }
       const int slot = (int)blockIdx.x - 1;
       bool ok = true;
-      if (lane == 0) ok = wait_flag_acquire(a.flags + slot * 8 + uw, abort_flag, kWaitLimitNs);
+      if (lane == 0) ok = wait_flag_acquire(a.flags + slot * kPairFlagsPerCta + uw, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) return false;
       const float4* src =
           reinterpret_cast<const float4*>(a.handoff + (size_t)slot * kPairHandoffFloats + ((size_t)j * 128 + n) * 64);
@@ -600,7 +605,7 @@ __global__ void __launch_bounds__(512, 1)
       for (int p = 0; p < 16; ++p) __stcg(dst + p, make_float4(H[4 * p], H[4 * p + 1], H[4 * p + 2], H[4 * p + 3]));
       __threadfence();
       __syncwarp();
-      if (lane == 0) store_flag_release(a.flags + (int)blockIdx.x * 8 + uw, 1);
+      if (lane == 0) store_flag_release(a.flags + (int)blockIdx.x * kPairFlagsPerCta + uw, 1);
     };
     // Steps in order: publish e^m H for step g (the state before g), scale the
     // x tile of step g+1, then fold step g's chunk state into H.

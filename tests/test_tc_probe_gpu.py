@@ -43,7 +43,7 @@ def test_mma_mode(mode):
 
 def _expected_layout():
     """The lane / column maps the kernels assume (the mma.sync m16n8 fragment)."""
-    exp = np.zeros(4128, dtype=np.int64)
+    exp = np.zeros(4384, dtype=np.int64)
     for t in range(128):  # 16x256b.x4 load after filling (lane << 16) | column
         q, i = divmod(t, 32)
         for j in range(4):
@@ -64,13 +64,24 @@ def _expected_layout():
         lo = 2 * (i % 4) * 8 + i // 4
         hi = (2 * (i % 4) + 1) * 8 + i // 4
         exp[4096 + i] = lo | (hi << 16)
+    for i in range(32):  # ldmatrix.x4.trans: column i/4 of matrix k, rows 2(i%4), 2(i%4)+1
+        for k in range(4):
+            lo = 64 * k + 8 * (2 * (i % 4)) + i // 4
+            exp[4128 + 4 * i + k] = lo | ((lo + 8) << 16)
+    for e in range(128):  # stmatrix.x4.trans: shared row r of matrix k holds column r of the fragment
+        vals = []
+        for h in range(2):
+            k, rc = divmod(2 * e + h, 64)
+            r, c = divmod(rc, 8)
+            vals.append(64 * k + 8 * c + r)
+        exp[4256 + e] = vals[0] | (vals[1] << 16)
     return exp
 
 
 def test_fragment_layouts():
     lib = ctypes.CDLL(LIB)
     lib.tc_probe_layout.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
-    out = torch.zeros(4128, dtype=torch.int32, device="cuda")
+    out = torch.zeros(4384, dtype=torch.int32, device="cuda")
     assert lib.tc_probe_layout(out.data_ptr(), torch.cuda.current_stream().cuda_stream) == 0
     torch.cuda.synchronize()
     got = out.cpu().numpy().astype(np.int64) & 0xFFFFFFFF
@@ -80,7 +91,30 @@ def test_fragment_layouts():
         dump = os.environ.get("SSD_PROBE_DUMP")
         if dump:
             np.save(dump, got)
-        names = ["16x256b load", "16x128b store", "8x8 transpose"]
-        first = {n: [(int(k), hex(int(got[k])), hex(int(exp[k]))) for k in bad
-                     if (0 if k < 2048 else 1 if k < 4096 else 2) == ni][:4] for ni, n in enumerate(names)}
+        names = ["16x256b load", "16x128b store", "8x8 transpose", "ldmatrix.trans", "stmatrix.trans"]
+        part = lambda k: 0 if k < 2048 else 1 if k < 4096 else 2 if k < 4128 else 3 if k < 4256 else 4
+        first = {n: [(int(k), hex(int(got[k])), hex(int(exp[k]))) for k in bad if part(k) == ni][:4]
+                 for ni, n in enumerate(names)}
         raise AssertionError(f"{len(bad)} mismatches: {first}")
+
+
+def test_mma_issue_rate_is_recorded():
+    """Times 64 back-to-back MMAs per shape, alone and beside other warps'
+    TMEM or shared-memory traffic (a measurement, printed; the test only
+    checks that every variant completed)."""
+    lib = ctypes.CDLL(LIB)
+    lib.tc_probe_mma_rate.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    names = ["A tmem N64", "A tmem N128", "A tmem N256", "A smem N64", "A tmem N192 (B MN)",
+             "chunk sequence"]
+    loads = {0: "alone", 1: "tmem ld", 2: "smem ldst", 4: "tmem st", 8: "fma", 15: "all"}
+    for v, name in enumerate(names):
+        for ld, lname in loads.items():
+            if ld and v not in (0, 5):
+                continue
+            out = torch.zeros(2 + 128, dtype=torch.int64, device="cuda")
+            for _ in range(3):  # warm the instruction cache
+                assert lib.tc_probe_mma_rate(v, ld, out.data_ptr(), torch.cuda.current_stream().cuda_stream) == 0
+            torch.cuda.synchronize()
+            issue, done = (int(t) for t in out[:2].cpu())
+            assert done > 0, name
+            print(f"mma rate {name} [{lname}]: issue {issue / 64:.1f} cycles/MMA, complete {done / 64:.1f} cycles/MMA")
