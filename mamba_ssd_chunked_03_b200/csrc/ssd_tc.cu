@@ -247,68 +247,81 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB), aX = smem_u32(sm + K::oX);
-      const uint32_t aW = smem_u32(sm + K::oW), aXt = smem_u32(sm + K::oXt), aH = smem_u32(sm + K::oH);
-      constexpr uint32_t id_cb = idesc_bf16(64, 64, 0, 0);
-      constexpr uint32_t id_wx = idesc_bf16(64, 64, 0, 1);
-      constexpr uint32_t id_st = idesc_bf16(128, 64, 1, 1);
-      bool ok = true;
-      for (int c = 0; c < nc && ok; ++c) {
-        const uint32_t par = c & 1, ppar = (c - 1) & 1;
-        ok = mbar_wait(&s.full, par, abort_flag, kWaitLimitNs);
-        if (ok && c > 0) ok = mbar_wait(&s.cb_free, ppar, abort_flag, kWaitLimitNs);
-        if (!ok) break;
-        tc_fence_after();
-        // MMA1: CB = C B^T, K = N in steps of 16
+    // The whole warp walks the loop and forms the descriptors (warp-uniform
+    // values); one elected lane issues the MMAs and commits.
+    const uint32_t aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB), aX = smem_u32(sm + K::oX);
+    const uint32_t aW = smem_u32(sm + K::oW), aXt = smem_u32(sm + K::oXt), aH = smem_u32(sm + K::oH);
+    constexpr uint32_t id_cb = idesc_bf16(64, 64, 0, 0);
+    constexpr uint32_t id_wx = idesc_bf16(64, 64, 0, 1);
+    constexpr uint32_t id_st = idesc_bf16(128, 64, 1, 1);
+    const uint64_t dc = sw128_desc(aC, 16, 1024), dbk = sw128_desc(aB, 16, 1024);  // K-major: 32 B per K step
+    const uint64_t dbm = sw128_desc(aB, K::kTile, 1024), dh = sw128_desc(aH, K::kTile, 1024);  // MN-major: 2048 B
+    const uint64_t dxt = sw128_desc(aXt, K::kTile, 1024), dx = sw128_desc(aX, K::kTile, 1024);
+    const uint64_t dw = sw128_desc(aW, 16, 1024);
+    bool ok = true;
+    for (int c = 0; c < nc && ok; ++c) {
+      const uint32_t par = c & 1, ppar = (c - 1) & 1;
+      ok = mbar_wait_warp(&s.full, par, abort_flag, kWaitLimitNs);
+      if (ok && c > 0) ok = mbar_wait_warp(&s.cb_free, ppar, abort_flag, kWaitLimitNs);
+      if (!ok) break;
+      tc_fence_after();
+      // MMA1: CB = C B^T, K = N in steps of 16
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < NS / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * K::kTile + (kk & 3) * 32;
-          mma_bf16_ss(tmem + K::tCB, sw128_desc(aC + koff, 16, 1024), sw128_desc(aB + koff, 16, 1024), id_cb,
-                      kk > 0);
+          const uint32_t koff = ((kk >> 2) * K::kTile + (kk & 3) * 32) / 16;
+          mma_bf16_ss(tmem + K::tCB, dc + koff, dbk + koff, id_cb, kk > 0);
         }
         mma_commit(&s.cb_full);
-        // MMA3: Yo = C H_c^T (H stored [n][p], MN-major B operand), K = N
-        ok = mbar_wait(&s.h_ready, par, abort_flag, kWaitLimitNs);
-        if (ok && c > 0) ok = mbar_wait(&s.y_free, ppar, abort_flag, kWaitLimitNs);
-        if (!ok) break;
-        tc_fence_after();
+      }
+      __syncwarp();
+      // MMA3: Yo = C H_c^T (H stored [n][p], MN-major B operand), K = N
+      ok = mbar_wait_warp(&s.h_ready, par, abort_flag, kWaitLimitNs);
+      if (ok && c > 0) ok = mbar_wait_warp(&s.y_free, ppar, abort_flag, kWaitLimitNs);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < NS / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * K::kTile + (kk & 3) * 32;
-          mma_bf16_ss(tmem + K::tYo, sw128_desc(aC + koff, 16, 1024), sw128_desc(aH + kk * 2048, K::kTile, 1024),
-                      id_wx, kk > 0);
+          const uint32_t koff = ((kk >> 2) * K::kTile + (kk & 3) * 32) / 16;
+          mma_bf16_ss(tmem + K::tYo, dc + koff, dh + 128 * kk, id_wx, kk > 0);
         }
-        // MMA4: S^T = B^T X~ (both MN-major), M = 128 state rows per half
-        ok = mbar_wait(&s.xt_ready, par, abort_flag, kWaitLimitNs);
-        if (ok && c > 0) ok = mbar_wait(&s.s_free, ppar, abort_flag, kWaitLimitNs);
-        if (!ok) break;
-        tc_fence_after();
+      }
+      __syncwarp();
+      // MMA4: S^T = B^T X~ (both MN-major), M = 128 state rows per half
+      ok = mbar_wait_warp(&s.xt_ready, par, abort_flag, kWaitLimitNs);
+      if (ok && c > 0) ok = mbar_wait_warp(&s.s_free, ppar, abort_flag, kWaitLimitNs);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
         for (int hf = 0; hf < NS / 128; ++hf) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16_ss(tmem + K::tS + hf * 64, sw128_desc(aB + hf * 2 * K::kTile + kk * 2048, K::kTile, 1024),
-                        sw128_desc(aXt + kk * 2048, K::kTile, 1024), id_st, kk > 0);
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tmem + K::tS + hf * 64, dbm + (hf * 2 * K::kTile) / 16 + 128 * kk, dxt + 128 * kk, id_st,
+                        kk > 0);
         }
         mma_commit(&s.s_full);
-        // MMA2: Yd = W X, K = Q
-        ok = mbar_wait(&s.w_ready, par, abort_flag, kWaitLimitNs);
-        if (!ok) break;
-        tc_fence_after();
+      }
+      __syncwarp();
+      // MMA2: Yd = W X, K = Q
+      ok = mbar_wait_warp(&s.w_ready, par, abort_flag, kWaitLimitNs);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_bf16_ss(tmem + K::tYd, sw128_desc(aW + kk * 32, 16, 1024), sw128_desc(aX + kk * 2048, K::kTile, 1024),
-                      id_wx, kk > 0);
-        }
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(tmem + K::tYd, dw + 2 * kk, dx + 128 * kk, id_wx, kk > 0);
         mma_commit(&s.y_full);
         mma_commit(&s.empty);
       }
-      // all MMAs issued by this thread must finish before TMEM is released
+      __syncwarp();
+    }
+    // all MMAs issued by this warp must finish before TMEM is released
+    if (elect_one()) {
       mma_commit(&s.drain);
       mbar_wait(&s.drain, 0, never, kWaitLimitNs);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ compute warps
     const int wt = tid - 64;      // 0..127

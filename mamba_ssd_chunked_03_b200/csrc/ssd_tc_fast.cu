@@ -380,61 +380,71 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t aW = smem_u32(sm + K::oW), aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB);
-      const uint32_t aX = smem_u32(sm + K::oX), aH = smem_u32(sm + K::oH);
-      constexpr uint32_t id_64 = idesc_bf16(64, 64, 0, 1);    // A K-major, B MN-major, M = 64
-      constexpr uint32_t id_st = idesc_bf16(128, 64, 1, 1);   // both MN-major, M = 128
-      for (int c = 0; c < nc; ++c) {
-        const int i = c & 1;
-        const uint32_t ph = (c >> 1) & 1, p1 = c & 1, pp = ((c - 2) >> 1) & 1;
-        bool ok = mbar_wait(&s.full_w[i], ph, abort_flag, kWaitLimitNs);
-        ok = ok && mbar_wait(&s.xp_ready[c % 3], (c / 3) & 1, abort_flag, kWaitLimitNs);
-        if (c >= 2) {
-          ok = ok && mbar_wait(&s.y_free[i], pp, abort_flag, kWaitLimitNs);
-          ok = ok && mbar_wait(&s.s_free[i], pp, abort_flag, kWaitLimitNs);
-        }
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t yd = tmem + K::tYd0 + 64 * i;
-        const uint32_t st = tmem + K::tS0 + K::kSCols * i;
-        const uint32_t aXc = aX + (c % 3) * K::kTile;  // X' of this chunk
-        // Yd = W' X'   (K = 64 tokens)
+    // The whole warp walks the loop and forms the descriptors (warp-uniform
+    // values); one elected lane issues the MMAs and commits.
+    const uint32_t aW = smem_u32(sm + K::oW), aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB);
+    const uint32_t aX = smem_u32(sm + K::oX), aH = smem_u32(sm + K::oH);
+    constexpr uint32_t id_64 = idesc_bf16(64, 64, 0, 1);    // A K-major, B MN-major, M = 64
+    constexpr uint32_t id_st = idesc_bf16(128, 64, 1, 1);   // both MN-major, M = 128
+    const uint64_t db = sw128_desc(aB, K::kTile, 1024);     // a K step of 16 tokens: 2048 B
+    const uint64_t dh = sw128_desc(aH, K::kTile, 1024);
+    for (int c = 0; c < nc; ++c) {
+      const int i = c & 1;
+      const uint32_t ph = (c >> 1) & 1, p1 = c & 1, pp = ((c - 2) >> 1) & 1;
+      bool ok = mbar_wait_warp(&s.full_w[i], ph, abort_flag, kWaitLimitNs);
+      ok = ok && mbar_wait_warp(&s.xp_ready[c % 3], (c / 3) & 1, abort_flag, kWaitLimitNs);
+      if (c >= 2) {
+        ok = ok && mbar_wait_warp(&s.y_free[i], pp, abort_flag, kWaitLimitNs);
+        ok = ok && mbar_wait_warp(&s.s_free[i], pp, abort_flag, kWaitLimitNs);
+      }
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t yd = tmem + K::tYd0 + 64 * i;
+      const uint32_t st = tmem + K::tS0 + K::kSCols * i;
+      const uint64_t dx = sw128_desc(aX + (c % 3) * K::kTile, K::kTile, 1024);  // X' of this chunk
+      const uint64_t dw = sw128_desc(aW + i * K::kTile, 16, 1024);             // a K step: 32 B
+      // Yd = W' X'   (K = 64 tokens)
+      if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(yd, sw128_desc(aW + i * K::kTile + kk * 32, 16, 1024),
-                      sw128_desc(aXc + kk * 2048, K::kTile, 1024), id_64, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(yd, dw + 2 * kk, dx + 128 * kk, id_64, kk > 0);
         mma_commit(&s.w_empty[i]);
-        // S'^T = B^T X'   (M = 128 state rows per half, K = 64 tokens)
-        if (!mbar_wait(&s.full_b, p1, abort_flag, kWaitLimitNs)) break;
-        tc_fence_after();
+      }
+      __syncwarp();
+      // S'^T = B^T X'   (M = 128 state rows per half, K = 64 tokens)
+      if (!mbar_wait_warp(&s.full_b, p1, abort_flag, kWaitLimitNs)) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
         for (int hf = 0; hf < K::NH; ++hf)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(st + 64 * hf, sw128_desc(aB + hf * 2 * K::kTile + kk * 2048, K::kTile, 1024),
-                        sw128_desc(aXc + kk * 2048, K::kTile, 1024), id_st, kk > 0);
+            mma_bf16_ss(st + 64 * hf, db + (hf * 2 * K::kTile) / 16 + 128 * kk, dx + 128 * kk, id_st, kk > 0);
         mma_commit(&s.s_full[i]);
         mma_commit(&s.b_free);
         mma_commit(&s.x_empty[c % 3]);
-        // Yd += C (e^m H_c)^T   (K = N)
-        ok = mbar_wait(&s.h_ready, p1, abort_flag, kWaitLimitNs);
-        ok = ok && mbar_wait(&s.full_c[i], ph, abort_flag, kWaitLimitNs);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t aCi = aC + i * K::NB * K::kTile;
+      }
+      __syncwarp();
+      // Yd += C (e^m H_c)^T   (K = N)
+      ok = mbar_wait_warp(&s.h_ready, p1, abort_flag, kWaitLimitNs);
+      ok = ok && mbar_wait_warp(&s.full_c[i], ph, abort_flag, kWaitLimitNs);
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t dc = sw128_desc(aC + i * K::NB * K::kTile, 16, 1024);
+      if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < NS / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * K::kTile + (kk & 3) * 32;
-          mma_bf16_ss(yd, sw128_desc(aCi + koff, 16, 1024), sw128_desc(aH + kk * 2048, K::kTile, 1024), id_64, 1);
-        }
+        for (int kk = 0; kk < NS / 16; ++kk)
+          mma_bf16_ss(yd, dc + ((kk >> 2) * K::kTile + (kk & 3) * 32) / 16, dh + 128 * kk, id_64, 1);
         mma_commit(&s.y_full[i]);
         mma_commit(&s.h_free);
         mma_commit(&s.c_free[i]);
       }
+      __syncwarp();
+    }
+    if (elect_one()) {
       mma_commit(&s.drain);
       mbar_wait(&s.drain, 0, never, kWaitLimitNs);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ compute warps
     const int wt = tid - 64;            // 0..255
