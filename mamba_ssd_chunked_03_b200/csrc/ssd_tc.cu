@@ -671,7 +671,8 @@ cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
 }  // namespace
 
 // Layout: [err, failed_count, (two-head kernel: flags, pair marks)] cleared per
-// call | W' | failed units | (two-head kernel: state hand-over buffers)
+// call | W' | failed units | (two-head kernel: state hand-over buffers, total
+// decays)
 TcWorkspace tc_carve(const Problem& p, void* ws, size_t* total) {
   const uintptr_t base = reinterpret_cast<uintptr_t>(ws);
   const bool pair = tc_pair_shape_ok(p);
@@ -689,6 +690,8 @@ TcWorkspace tc_carve(const Problem& p, void* ws, size_t* total) {
   off = align_up(off + sizeof(int) * (size_t)(p.b * p.H), kWsAlign);
   w.handoff = pair ? reinterpret_cast<float*>(base + off) : nullptr;
   if (pair) off = align_up(off + sizeof(float) * (size_t)kPairGridMax * kPairHandoffFloats, kWsAlign);
+  w.seg_decay = pair ? reinterpret_cast<float*>(base + off) : nullptr;
+  if (pair) off = align_up(off + sizeof(float) * (size_t)kPairGridMax * 2, kWsAlign);
   if (total) *total = off;
   return w;
 }
@@ -717,7 +720,11 @@ bool tc_supported(const Problem& p, uint32_t flags) {
 
 size_t tc_workspace_bytes(const Problem& p) { return tc_workspace_need(tc_tiles(p)); }
 
-int tc_launch_count(const Problem& p) { return p.seq ? 1 : 3; }
+int tc_launch_count(const Problem& p) {
+  if (p.seq) return 1;
+  const Problem t = tc_tiles(p);
+  return tc_kernel_n(t) == 128 && tc_pair_supported(t) && tc_pair_split(t) ? 4 : 3;
+}
 
 cudaError_t tc_forward(const Problem& pq, void* ws, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
   const Problem p = tc_tiles(pq);

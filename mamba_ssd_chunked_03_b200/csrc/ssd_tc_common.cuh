@@ -44,6 +44,10 @@ struct FastArgs {
   float* handoff;  // [grid][2 heads][128 states][64 p] fp32
   int* flags;      // [grid][kPairFlagsPerCta state warps]: 1 once that warp's part of the hand-over is written
   int* pair_bad;   // [b * H / 2]: 1 once a pair was put on the exact kernel's list
+  // split mode (a state-only pass first): the CTA's local end state goes to
+  // handoff, its total decay per head to seg_decay [grid][2]
+  int split;
+  float* seg_decay;
 };
 
 // persistent grid of the two-head kernel, at most; per-CTA hand-over size
@@ -121,6 +125,7 @@ struct TcWorkspace {
   __nv_bfloat16* wp;      // masked C B^T per (b, chunk, group)
   int* failed_list;       // (b*H) units for the exact kernel
   float* handoff;         // two-head kernel: kPairGridMax x kPairHandoffFloats, or null
+  float* seg_decay;       // two-head kernel: kPairGridMax x 2 total decays (split mode), or null
 };
 
 // carve the caller's workspace (ws may be null to only size it: *total)
@@ -135,6 +140,9 @@ cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t
 bool tc_pair_shape_ok(const Problem& p);
 // ... and a 16-byte aligned dt
 bool tc_pair_supported(const Problem& p);
+// whether the two-head kernel runs split: a state-only pass over every CTA's
+// range first, so that no CTA waits for another (fewer pairs than SMs)
+bool tc_pair_split(const Problem& p);
 cudaError_t tc_pair_launch(const Problem& p, const TcWorkspace& w, const CUtensorMap& tx, const CUtensorMap& tb,
                            const CUtensorMap& tc_, const CUtensorMap& tw, const CUtensorMap& ty,
                            const CUtensorMap& tdt, const tc::FastArgs& fa, cudaStream_t st);

@@ -106,6 +106,7 @@ struct __align__(16) PairSmem {
   // per segment: pair, batch row, first head, group, first chunk, length, first step
   int seg_pair[kPairMaxSeg], seg_b[kPairMaxSeg], seg_h0[kPairMaxSeg], seg_grp[kPairMaxSeg];
   int seg_c0[kPairMaxSeg], seg_len[kPairMaxSeg], seg_g0[kPairMaxSeg];
+  int seg_i0[kPairMaxSeg];  // split mode: the first CTA whose range holds the segment's pair start
   alignas(16) float u[4][2][64];  // written as float4
   alignas(16) float v[4][2][64];
   alignas(16) float g[4][2][64];  // D / v_t: D x_t = g_t X'_t
@@ -132,6 +133,12 @@ struct PairCursor {
   }
 };
 
+// kStateOnly: the state-only pass of split mode.  Each CTA takes only the
+// segment of its range that ends inside a pair (there is at most one: the
+// head of its last pair), runs it from a zero state with x and B alone (no
+// W', C, y) and leaves the end state in handoff and the segment's total decay
+// per head in seg_decay.
+template <bool kStateOnly>
 __global__ void __launch_bounds__(512, 1)
     k_ssd_fwd_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_w,
@@ -153,7 +160,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&s.full_x[i], 1);
       mbar_init(&s.x_empty[i], 1);
       mbar_init(&s.scan_full[i], 32);
-      mbar_init(&s.scan_empty[i], 384);  // scale/epilogue warps and state warps
+      mbar_init(&s.scan_empty[i], kStateOnly ? 256 : 384);  // epilogue warps and state warps
       mbar_init(&s.xp_ready[i], 256);  // both heads' state warps
       mbar_init(&s.y_staged[i], 128);
     }
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.mma_done[i], 1);
       mbar_init(&s.h_ready[i], 256);
-      mbar_init(&s.acc_free[i], 384);  // epilogue (Yd) and state (S) readers
+      mbar_init(&s.acc_free[i], kStateOnly ? 256 : 384);  // epilogue (Yd) and state (S) readers
     }
     for (int i = 0; i < 8; ++i) mbar_init(&s.full_dt[i], 1);
     mbar_init(&s.drain, 1);
@@ -198,6 +205,22 @@ __global__ void __launch_bounds__(512, 1)
         add(q, 0, cq);
         for (int pr = p0 + 1; pr < q; ++pr) add(pr, 0, ncs);
         add(p0, c0, ncs - c0);
+      }
+    }
+    if (kStateOnly) {  // only a segment that ends inside its pair
+      if (n > 0 && s.seg_c0[0] + s.seg_len[0] < ncs) {
+        n = 1;
+        tot = s.seg_len[0];
+      } else {
+        n = tot = 0;
+      }
+    } else if (a.split) {
+      // the CTAs before this one that hold a part of the segment's pair
+      for (int k = 0; k < n; ++k) {
+        const int64_t s0 = (int64_t)s.seg_pair[k] * ncs;
+        int i0 = (int)blockIdx.x;
+        while (i0 > 0 && (int64_t)i0 * T / gridDim.x > s0) --i0;
+        s.seg_i0[k] = i0;
       }
     }
     s.nseg = n;
@@ -244,8 +267,10 @@ __global__ void __launch_bounds__(512, 1)
       };
       auto issue_wb = [&](int gg) {
         const int i = gg & 1, bb = s.seg_b[uwb.k], grp = s.seg_grp[uwb.k];
-        mbar_arrive_expect_tx(&s.full_wb[i], (1 + K::NB) * K::kTile);
-        tma_load_3d(sm + K::oW + i * K::kTile, &tm_w, &s.full_wb[i], 0, ((bb * nc + uwb.c) * (int)a.G + grp) * 64, 0);
+        mbar_arrive_expect_tx(&s.full_wb[i], (kStateOnly ? K::NB : 1 + K::NB) * K::kTile);
+        if (!kStateOnly)
+          tma_load_3d(sm + K::oW + i * K::kTile, &tm_w, &s.full_wb[i], 0, ((bb * nc + uwb.c) * (int)a.G + grp) * 64,
+                      0);
         for (int jb = 0; jb < K::NB; ++jb)
           tma_load_4d(sm + K::oB + (i * K::NB + jb) * K::kTile, &tm_b, &s.full_wb[i], 64 * jb, grp, uwb.c * 64,
                       bb);
@@ -272,11 +297,11 @@ __global__ void __launch_bounds__(512, 1)
         for (int c = 3; c < 6 && c < total; ++c) prefetch_x(c);
         #pragma unroll 1
         for (int c = 0; c < 3 && c < total; ++c) issue_x(c);  // slot 3 starts free
-        griddep_wait();  // W' comes from the C B^T kernel launched before this one
+        if (!kStateOnly) griddep_wait();  // W' comes from the C B^T kernel launched before this one
         #pragma unroll 1
         for (int c = 0; c < 2 && c < total; ++c) {
           issue_wb(c);
-          issue_c(c);
+          if (!kStateOnly) issue_c(c);
         }
       }
       bool ok = !*abort_flag;
@@ -286,8 +311,10 @@ __global__ void __launch_bounds__(512, 1)
         if (c + 2 < total) {
           ok = mbar_wait(&s.s_full[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
           if (ok) issue_wb(c + 2);
-          ok = ok && mbar_wait(&s.mma_done[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
-          if (ok) issue_c(c + 2);
+          if (!kStateOnly) {
+            ok = ok && mbar_wait(&s.mma_done[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
+            if (ok) issue_c(c + 2);
+          }
         }
         // x of step c + 3 goes where step c - 1 was, once its y tile has been stored
         if (ok && c + 3 < total) {
@@ -334,14 +361,18 @@ __global__ void __launch_bounds__(512, 1)
       const uint64_t db = sw128_desc(aB + i * K::NB * K::kTile, K::kTile, 1024);
       if (elect_one()) {
         // Yd = W' [X'_0 | X'_1]   (K = 64 tokens)
+        if (!kStateOnly) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(yd, dw + 2 * kk, dxp + 128 * kk, id_y, kk > 0);
+          for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(yd, dw + 2 * kk, dxp + 128 * kk, id_y, kk > 0);
+        }
         // S'^T = B^T [X'_0 | X'_1]   (M = 128 states, K = 64 tokens)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(st, db + 128 * kk, dxp + 128 * kk, id_s, kk > 0);
         mma_commit(&s.s_full[i]);
+        if (kStateOnly) mma_commit(&s.x_empty[c & 3]);  // X' read: the slot may be refilled
       }
       __syncwarp();
+      if (kStateOnly) continue;
       // Yd += C [e^m H_0 | e^m H_1]^T   (K = N)
       ok = mbar_wait_warp(&s.h_ready[i], ph, abort_flag, kWaitLimitNs);
       ok = ok && mbar_wait_warp(&s.full_c[i], ph, abort_flag, kWaitLimitNs);
@@ -457,7 +488,8 @@ __global__ void __launch_bounds__(512, 1)
         mbar_wait(&s.full_dt[c & 7], (c >> 3) & 1, never, kWaitLimitNs);
   } else if (warp == 3) {
     // ------------------------------------------------------------ y stores
-    if (lane == 0) {
+    // (the state-only pass stores no y: its MMAs free the x slots)
+    if (!kStateOnly && lane == 0) {
       PairCursor uy;
       uy.start(s);
       #pragma unroll 1
@@ -475,47 +507,49 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp < 8) {
     // ------------------------------------------------ epilogue warps (both heads)
-    const int q = warp & 3;              // TMEM lane quadrant
-    const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
-    const int te = 16 * q + (lane & 15);   // epilogue row (token) of this thread
-    const int half = lane >> 4;            // epilogue columns p in [32 half, 32 half + 32)
-    #pragma unroll 1
-    for (int c = 1; c <= total; ++c) {
-      // ---- epilogue for step c-1, both heads: y = u_t Yd + (D / v_t) X'_t, written over X'
-      if (c >= 1) {
-        const int ip = (c - 1) & 1, slp = (c - 1) & 3;
-        if (!mbar_wait_warp(&s.mma_done[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) break;
-        tc_fence_after();
-        #pragma unroll 1
-        for (int j = 0; j < 2; ++j) {
-          uint32_t r[32];
-          SSD_TMEM_LD_16x32bx2_X32_HALF32(tq + K::tYd0 + 128 * ip + 64 * j, r);
-          SSD_TMEM_WAIT_LD_32(r);
-          const float ut = s.u[slp][j][te], gt = s.g[slp][j][te];
-          unsigned char* row = sm + K::oX + (slp * 2 + j) * K::kTile + te * 128;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            // 16-byte column 4 half + k of row te, at its swizzled position
-            uint4* px = reinterpret_cast<uint4*>(row + (((4 * half + k) ^ (te & 7)) << 4));
-            const uint4 xv = *px;
-            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-            uint32_t o[4];
-#pragma unroll
-            for (int k2 = 0; k2 < 4; ++k2) {
-              float x0, x1;
-              unpack_bf16x2(xw[k2], x0, x1);
-              const int jj = 8 * k + 2 * k2;
-              o[k2] = pack_bf16x2(fmaf(ut, __uint_as_float(r[jj]), gt * x0),
-                                  fmaf(ut, __uint_as_float(r[jj + 1]), gt * x1));
+    if constexpr (!kStateOnly) {
+      const int q = warp & 3;              // TMEM lane quadrant
+      const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+      const int te = 16 * q + (lane & 15);   // epilogue row (token) of this thread
+      const int half = lane >> 4;            // epilogue columns p in [32 half, 32 half + 32)
+      #pragma unroll 1
+      for (int c = 1; c <= total; ++c) {
+        // ---- epilogue for step c-1, both heads: y = u_t Yd + (D / v_t) X'_t, written over X'
+        if (c >= 1) {
+          const int ip = (c - 1) & 1, slp = (c - 1) & 3;
+          if (!mbar_wait_warp(&s.mma_done[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+          tc_fence_after();
+          #pragma unroll 1
+          for (int j = 0; j < 2; ++j) {
+            uint32_t r[32];
+            SSD_TMEM_LD_16x32bx2_X32_HALF32(tq + K::tYd0 + 128 * ip + 64 * j, r);
+            SSD_TMEM_WAIT_LD_32(r);
+            const float ut = s.u[slp][j][te], gt = s.g[slp][j][te];
+            unsigned char* row = sm + K::oX + (slp * 2 + j) * K::kTile + te * 128;
+  #pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              // 16-byte column 4 half + k of row te, at its swizzled position
+              uint4* px = reinterpret_cast<uint4*>(row + (((4 * half + k) ^ (te & 7)) << 4));
+              const uint4 xv = *px;
+              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+              uint32_t o[4];
+  #pragma unroll
+              for (int k2 = 0; k2 < 4; ++k2) {
+                float x0, x1;
+                unpack_bf16x2(xw[k2], x0, x1);
+                const int jj = 8 * k + 2 * k2;
+                o[k2] = pack_bf16x2(fmaf(ut, __uint_as_float(r[jj]), gt * x0),
+                                    fmaf(ut, __uint_as_float(r[jj + 1]), gt * x1));
+              }
+              *px = make_uint4(o[0], o[1], o[2], o[3]);
             }
-            *px = make_uint4(o[0], o[1], o[2], o[3]);
           }
+          tc_fence_before();
+          mbar_arrive(&s.acc_free[ip]);  // this thread's reads of Yd of chunk c-1 are done
+          fence_proxy_async_smem();
+          mbar_arrive(&s.y_staged[slp]);
+          mbar_arrive(&s.scan_empty[slp]);
         }
-        tc_fence_before();
-        mbar_arrive(&s.acc_free[ip]);  // this thread's reads of Yd of chunk c-1 are done
-        fence_proxy_async_smem();
-        mbar_arrive(&s.y_staged[slp]);
-        mbar_arrive(&s.scan_empty[slp]);
       }
     }
   } else {
@@ -556,11 +590,21 @@ __global__ void __launch_bounds__(512, 1)
       return true;
     };
     float H[64];
+    float dprod = 1.f;  // state-only pass: the segment's total decay so far
     // state at the start of segment k: h0 (or zero) at a pair's first chunk,
-    // otherwise this warp's part of the hand-over the previous CTA wrote
+    // otherwise this warp's part of the hand-over the previous CTA wrote, or
+    // in split mode h0 carried through the state-only pass's local states of
+    // the CTAs before this one (each: H <- decay H + S).  The state-only pass
+    // itself starts every segment from zero.
     auto seg_begin = [&](int k) -> bool {
       const int64_t h = s.seg_h0[k] + j, bb = s.seg_b[k];
-      if (s.seg_c0[k] == 0) {
+      if (kStateOnly) {
+#pragma unroll
+        for (int p = 0; p < 64; ++p) H[p] = 0.f;
+        dprod = 1.f;
+        return true;
+      }
+      if (s.seg_c0[k] == 0 || a.split) {
         if (a.h0 && n < a.Nr) {
           const float* src = a.h0 + ((bb * a.H + h) * 64) * a.Nr + n;
 #pragma unroll
@@ -568,6 +612,22 @@ __global__ void __launch_bounds__(512, 1)
         } else {
 #pragma unroll
           for (int p = 0; p < 64; ++p) H[p] = 0.f;
+        }
+        if (s.seg_c0[k] == 0) return true;
+        griddep_wait();  // the state-only pass launched before this kernel
+        #pragma unroll 1
+        for (int ip = s.seg_i0[k]; ip < (int)blockIdx.x; ++ip) {
+          const float dd = __ldcg(a.seg_decay + 2 * ip + j);
+          const float4* src =
+              reinterpret_cast<const float4*>(a.handoff + (size_t)ip * kPairHandoffFloats + ((size_t)j * 128 + n) * 64);
+#pragma unroll
+          for (int p = 0; p < 16; ++p) {
+            const float4 v = __ldcg(src + p);
+            H[4 * p] = fmaf(dd, H[4 * p], v.x);
+            H[4 * p + 1] = fmaf(dd, H[4 * p + 1], v.y);
+            H[4 * p + 2] = fmaf(dd, H[4 * p + 2], v.z);
+            H[4 * p + 3] = fmaf(dd, H[4 * p + 3], v.w);
+          }
         }
         return true;
       }
@@ -591,6 +651,14 @@ __global__ void __launch_bounds__(512, 1)
     // to the next CTA (data, then this warp's release flag)
     auto seg_end = [&](int k) {
       const int64_t h = s.seg_h0[k] + j, bb = s.seg_b[k];
+      if (kStateOnly) {  // the local end state and the total decay, for the CTAs after this one
+        float4* dst = reinterpret_cast<float4*>(a.handoff + (size_t)blockIdx.x * kPairHandoffFloats +
+                                                ((size_t)j * 128 + n) * 64);
+#pragma unroll
+        for (int p = 0; p < 16; ++p) __stcg(dst + p, make_float4(H[4 * p], H[4 * p + 1], H[4 * p + 2], H[4 * p + 3]));
+        if (n == 0) __stcg(a.seg_decay + 2 * blockIdx.x + j, dprod);
+        return;
+      }
       if (s.seg_c0[k] + s.seg_len[k] == nc) {
         if (a.final_states && n < a.Nr) {
           float* dst = a.final_states + ((bb * a.H + h) * 64) * a.Nr + n;
@@ -599,6 +667,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         return;
       }
+      if (a.split) return;  // the CTAs after this one start from the state-only pass
       float4* dst = reinterpret_cast<float4*>(a.handoff + (size_t)blockIdx.x * kPairHandoffFloats +
                                               ((size_t)j * 128 + n) * 64);
 #pragma unroll
@@ -624,28 +693,30 @@ __global__ void __launch_bounds__(512, 1)
         const bool more = n1 < total;
         // the barriers this step's publish and the next tile's scaling need,
         // probed together (their latencies overlap), then waited for if not yet
-        const bool d_ok = g < 2 || mbar_probe(&s.mma_done[i], ((g - 2) >> 1) & 1);
+        const bool d_ok = kStateOnly || g < 2 || mbar_probe(&s.mma_done[i], ((g - 2) >> 1) & 1);
         const bool v_ok = !more || mbar_probe(&s.scan_full[s1], (n1 >> 2) & 1);
         const bool x_ok = !more || mbar_probe(&s.full_x[s1], (n1 >> 2) & 1);
-        if (!__all_sync(0xffffffffu, d_ok) &&
-            !mbar_wait_warp(&s.mma_done[i], ((g - 2) >> 1) & 1, abort_flag, kWaitLimitNs)) {
-          failed = true;
-          break;
-        }
-        {
-          unsigned char* base = sm + K::oH + (i * 2 + j) * K::kHTile + (uint32_t)n * 128;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            uint4 vv;
-            vv.x = pack_bf16x2(H[8 * kk + 0], H[8 * kk + 1]);
-            vv.y = pack_bf16x2(H[8 * kk + 2], H[8 * kk + 3]);
-            vv.z = pack_bf16x2(H[8 * kk + 4], H[8 * kk + 5]);
-            vv.w = pack_bf16x2(H[8 * kk + 6], H[8 * kk + 7]);
-            *reinterpret_cast<uint4*>(base + ((kk ^ (n & 7)) << 4)) = vv;
+        if constexpr (!kStateOnly) {
+          if (!__all_sync(0xffffffffu, d_ok) &&
+              !mbar_wait_warp(&s.mma_done[i], ((g - 2) >> 1) & 1, abort_flag, kWaitLimitNs)) {
+            failed = true;
+            break;
           }
+          {
+            unsigned char* base = sm + K::oH + (i * 2 + j) * K::kHTile + (uint32_t)n * 128;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              uint4 vv;
+              vv.x = pack_bf16x2(H[8 * kk + 0], H[8 * kk + 1]);
+              vv.y = pack_bf16x2(H[8 * kk + 2], H[8 * kk + 3]);
+              vv.z = pack_bf16x2(H[8 * kk + 4], H[8 * kk + 5]);
+              vv.w = pack_bf16x2(H[8 * kk + 6], H[8 * kk + 7]);
+              *reinterpret_cast<uint4*>(base + ((kk ^ (n & 7)) << 4)) = vv;
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&s.h_ready[i]);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&s.h_ready[i]);
         if (more) {
           if ((!__all_sync(0xffffffffu, v_ok) &&
                !mbar_wait_warp(&s.scan_full[s1], (n1 >> 2) & 1, abort_flag, kWaitLimitNs)) ||
@@ -668,6 +739,7 @@ __global__ void __launch_bounds__(512, 1)
           // H <- d (H + S'), two lanes of fp32 per instruction
           const float dd = s.sc[g & 3][j][0];
           const float2 d2 = make_float2(dd, dd);
+          if (kStateOnly) dprod *= dd;
 #pragma unroll
           for (int hlf = 0; hlf < 2; ++hlf) {
             uint32_t r[32];
@@ -695,6 +767,9 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   if (tid == 0 && *abort_flag) atomicExch(a.err, 1);
+  // the state-only pass completes only after the grid before it (the C B^T
+  // kernel), so the kernel after it may rely on both once it has waited
+  if (kStateOnly && tid == 0) griddep_wait();
   if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
 }
 
@@ -710,29 +785,58 @@ bool tc_pair_supported(const Problem& p) {
   return tc_pair_shape_ok(p) && reinterpret_cast<uintptr_t>(p.dt) % 16 == 0;
 }
 
+static int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return sms;
+}
+
+// Split when the pairs alone would leave SMs idle and every SM gets at least
+// two chunk steps; the state-only pass then costs about a third of a step per
+// step, against SMs that would otherwise do nothing.
+bool tc_pair_split(const Problem& p) {
+  const int sms = sm_count();
+  const int64_t npairs = p.b * p.H / 2;
+  return sms > 0 && npairs < sms && npairs * p.nc >= 2 * (int64_t)sms;
+}
+
 cudaError_t tc_pair_launch(const Problem& p, const TcWorkspace& w, const CUtensorMap& tx, const CUtensorMap& tb,
                            const CUtensorMap& tc_, const CUtensorMap& tw, const CUtensorMap& ty,
                            const CUtensorMap& tdt, const tc::FastArgs& fa, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(k_ssd_fwd_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)PairCfg::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  // one CTA per SM over equal ranges of the pair-major steps; if a CTA would
-  // touch more pairs than its segment table holds, one CTA per pair instead
-  // (whole pairs only: no hand-over)
-  const int64_t npairs = p.b * p.H / 2;
-  int64_t grid = npairs < sms ? npairs : sms;
-  if (grid > kPairGridMax) grid = kPairGridMax;
-  if ((npairs + grid - 1) / grid + 2 > kPairMaxSeg) grid = npairs;
+  cudaError_t e;
+  for (auto* k : {k_ssd_fwd_pair<false>, k_ssd_fwd_pair<true>})
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PairCfg::kSmemBytes)) !=
+        cudaSuccess)
+      return e;
+  const int sms = sm_count();
+  if (sms == 0) return cudaErrorInvalidValue;
   tc::FastArgs a = fa;
   a.batch = p.b;
   a.handoff = w.handoff;
   a.flags = w.flags;
   a.pair_bad = w.pair_bad;
-  return launch_dependent(k_ssd_fwd_pair, (unsigned)grid, PairCfg::kThreads, PairCfg::kSmemBytes, st, tx, tb, tc_, tw,
-                          ty, tdt, a);
+  a.seg_decay = w.seg_decay;
+  a.split = 0;
+  const int64_t npairs = p.b * p.H / 2;
+  if (tc_pair_split(p)) {
+    // one CTA per SM over equal ranges of the steps, the state-only pass first
+    int64_t grid = sms < kPairGridMax ? sms : kPairGridMax;
+    a.split = 1;
+    if ((e = launch_dependent(k_ssd_fwd_pair<true>, (unsigned)grid, PairCfg::kThreads, PairCfg::kSmemBytes, st, tx,
+                              tb, tc_, tw, ty, tdt, a)) != cudaSuccess)
+      return e;
+    return launch_dependent(k_ssd_fwd_pair<false>, (unsigned)grid, PairCfg::kThreads, PairCfg::kSmemBytes, st, tx,
+                            tb, tc_, tw, ty, tdt, a);
+  }
+  // one CTA per SM over equal ranges of the pair-major steps; if a CTA would
+  // touch more pairs than its segment table holds, one CTA per pair instead
+  // (whole pairs only: no hand-over)
+  int64_t grid = npairs < sms ? npairs : sms;
+  if (grid > kPairGridMax) grid = kPairGridMax;
+  if ((npairs + grid - 1) / grid + 2 > kPairMaxSeg) grid = npairs;
+  return launch_dependent(k_ssd_fwd_pair<false>, (unsigned)grid, PairCfg::kThreads, PairCfg::kSmemBytes, st, tx, tb,
+                          tc_, tw, ty, tdt, a);
 }
 
 }  // namespace ssd

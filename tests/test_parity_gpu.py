@@ -178,6 +178,27 @@ def test_single_head_kernel_takes_the_other_n128_shapes(case):
     assert state_err(f, fr) <= 1e-2, state_err(f, fr)
 
 
+@pytest.mark.parametrize("case", [
+    # b, L, H, P, N, G, Q, h0_std: fewer head pairs than SMs and at least two
+    # chunk steps per SM, so the two-head kernel runs split (a state-only pass
+    # first; each CTA folds the local states of the CTAs before it)
+    (1, 8192, 8, 64, 128, 1, 64, 0.3),     # 4 pairs of 128 chunks: each pair over ~37 CTAs
+    (1, 12000, 4, 64, 128, 2, 128, 0.0),   # two groups, a ragged tail, Q = 128
+    (2, 4800, 4, 64, 64, 1, 256, 0.2),     # two rows, N = 64 zero-padded
+], ids=_id)
+def test_split_two_head_kernel(case):
+    b, L, H, P, N, G, Q, h0 = case
+    shape = si.SSDShape("split", b, L, H, P, N, G, Q, "bf16", h0_std=h0, seed=L + H)
+    d = si.make_inputs(shape)
+    g = to_dev(d)
+    assert ssd.main_kernel(g["x"], g["dt"], g["B"], Q) == "k_ssd_fwd_pair"
+    assert ssd.launch_count(g["x"], g["B"], Q) == 4  # C B^T, state-only pass, fused, exact
+    y, f = run_gpu(d, Q)
+    yr, fr = run_oracle(d)
+    assert rel_l2(y, yr) <= 1e-2, rel_l2(y, yr)
+    assert state_err(f, fr) <= 1e-2, state_err(f, fr)
+
+
 def test_unaligned_dt_takes_the_single_head_kernel():
     """The two-head kernel reads dt by TMA (16-byte aligned base); a dt view
     that starts 4 bytes into its storage goes to the single-head kernel."""
