@@ -30,11 +30,13 @@
 // zero transition at packed-sequence boundaries ("Transformers与SSMs的隐藏联系"
 // section 4.2).
 //
-// Packed sequences (seq_idx) run on this kernel alone, over every unit: it
-// also writes each sequence's final state, from the updated state when the
-// sequence ends on a chunk's last token, and otherwise from the state at the
-// chunk's start plus the sequence's own tokens of the chunk (CUDA cores,
-// while the chunk's x and B tiles are still held).
+// Packed sequences (seq_idx): the fast path runs them per sequence; this
+// kernel takes the (batch row, head) units it hands back, or every unit when
+// the ids do not form increasing runs.  It then also writes each sequence's
+// final state, from the updated state when the sequence ends on a chunk's
+// last token, and otherwise from the state at the chunk's start plus the
+// sequence's own tokens of the chunk (CUDA cores, while the chunk's x and B
+// tiles are still held).
 //
 // Warp roles (192 threads):  warp 0 TMA producer, warp 1 MMA issuer (one
 // thread), warps 2-5 compute (cumsum, mask, scale, state update, epilogue).
@@ -152,7 +154,8 @@ struct TcArgs {
   float* final_states;
   const int* failed_count;  // units to process, listed by the fast kernel ...
   const int* failed_list;
-  int all_units;            // ... or, if set, every unit (packed sequences)
+  int all_units;            // ... or, if set, every unit
+  int64_t num_seqs;         // packed sequences: final states of ids outside [0, num_seqs) are not written
   int* err;
 };
 
@@ -469,7 +472,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
 #pragma unroll
               for (int hf = 0; hf < NH; ++hf) {
                 const int n = n0 + 128 * hf;
-                if (n < a.Nr) {
+                if (n < a.Nr && sq >= 0 && sq < a.num_seqs) {
                   float* dst = a.final_states + (((int64_t)sq * a.H + h) * 64 + pb) * a.Nr + n;
 #pragma unroll
                   for (int k = 0; k < 16; ++k) dst[(int64_t)k * a.Nr] = acc[hf][k];
@@ -545,7 +548,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
         tc_fence_before();
         mbar_arrive(&s.s_free);
         // the sequence of the chunk's last token ends there: its final state
-        if (a.seq && a.final_states &&
+        if (a.seq && a.final_states && seq_e >= 0 && seq_e < a.num_seqs &&
             ((int64_t)t0 + e + 1 >= a.L || a.seq[rowbase + t0 + e + 1] != seq_e)) {
           const int n0 = 32 * q + lane;
 #pragma unroll
@@ -631,8 +634,9 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
 }
 
 // ---------------------------------------------------------------- host side
+// all_units: every (batch row, head), else the units the fast kernel listed
 template <int NS>
-cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
+cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st, bool all_units) {
   CUtensorMap tx, tb, tc_;
   if (!make_map_3d(&tx, p.x, p.H * p.P, p.L, p.b) || !make_map_bc(&tb, p.B, p.N, p.G, p.L, p.b) ||
       !make_map_bc(&tc_, p.C, p.N, p.G, p.L, p.b))
@@ -654,7 +658,8 @@ cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
   a.final_states = p.final_states;
   a.failed_count = w.failed_count;
   a.failed_list = w.failed_list;
-  a.all_units = p.seq != nullptr;
+  a.all_units = all_units;
+  a.num_seqs = p.seq ? p.num_seqs : 0;
   a.err = w.err;
   cudaError_t e = cudaFuncSetAttribute(k_ssd_fwd_tc<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Cfg<NS>::kSmemBytes);
@@ -682,12 +687,29 @@ TcWorkspace tc_carve(const Problem& p, void* ws, size_t* total) {
   w.flags = pair ? reinterpret_cast<int*>(base + 2 * sizeof(int)) : nullptr;
   const size_t nflags = (size_t)kPairFlagsPerCta * kPairGridMax;
   w.pair_bad = pair ? reinterpret_cast<int*>(base + (2 + nflags) * sizeof(int)) : nullptr;
-  w.zero_bytes = sizeof(int) * (2 + (pair ? nflags + (size_t)(p.b * p.H / 2) : 0));
+  size_t zero_ints = 2 + (pair ? nflags + (size_t)(p.b * p.H / 2) : 0);
+  w.unit_bad = p.seq ? reinterpret_cast<int*>(base + zero_ints * sizeof(int)) : nullptr;
+  if (p.seq) zero_ints += (size_t)(p.b * p.H);
+  w.zero_bytes = sizeof(int) * zero_ints;
   size_t off = align_up(w.zero_bytes, kWsAlign);
   w.wp = reinterpret_cast<__nv_bfloat16*>(base + off);
-  off = align_up(off + sizeof(__nv_bfloat16) * (size_t)(p.b * p.nc * p.G * 64 * 64), kWsAlign);
+  // packed sequences: the runs' chunks, at most b * nc + num_seqs (one partial chunk per run)
+  const int64_t chunks = p.b * p.nc + (p.seq ? p.num_seqs : 0);
+  off = align_up(off + sizeof(__nv_bfloat16) * (size_t)(chunks * p.G * 64 * 64), kWsAlign);
   w.failed_list = reinterpret_cast<int*>(base + off);
   off = align_up(off + sizeof(int) * (size_t)(p.b * p.H), kWsAlign);
+  w.runs = tc::RunList{};
+  if (p.seq) {
+    const size_t ns = (size_t)p.num_seqs;
+    int* r = reinterpret_cast<int*>(base + off);
+    w.runs.count = r;
+    w.runs.b = r + 1;
+    w.runs.t0 = r + 1 + ns;
+    w.runs.len = r + 1 + 2 * ns;
+    w.runs.id = r + 1 + 3 * ns;
+    w.runs.c0 = r + 1 + 4 * ns;
+    off = align_up(off + sizeof(int) * (2 + 5 * ns), kWsAlign);
+  }
   w.handoff = pair ? reinterpret_cast<float*>(base + off) : nullptr;
   if (pair) off = align_up(off + sizeof(float) * (size_t)kPairGridMax * kPairHandoffFloats, kWsAlign);
   w.seg_decay = pair ? reinterpret_cast<float*>(base + off) : nullptr;
@@ -711,17 +733,17 @@ bool tc_supported(const Problem& p, uint32_t flags) {
   if (p.dtype != SSD_BF16) return false;
   if (p.P != 64 || (p.Q != 64 && p.Q != 128 && p.Q != 256)) return false;
   if (p.N != 64 && p.N != 128 && p.N != 256) return false;  // 64 runs zero-padded as 128
-  // packed sequences: the exact kernel alone (see its header), for Q >= 64
-  // TMA coordinates are 32-bit
+  // TMA coordinates are 32-bit (W' rows: packed sequences add one partial chunk per run)
   const Problem t = tc_tiles(p);
-  if (t.b * t.nc * t.G * 64 >= ((int64_t)1 << 31) || t.L >= ((int64_t)1 << 31)) return false;
+  const int64_t chunks = t.b * t.nc + (p.seq ? p.num_seqs : 0);
+  if (chunks * t.G * 64 >= ((int64_t)1 << 31) || t.L >= ((int64_t)1 << 31)) return false;
   return true;
 }
 
 size_t tc_workspace_bytes(const Problem& p) { return tc_workspace_need(tc_tiles(p)); }
 
 int tc_launch_count(const Problem& p) {
-  if (p.seq) return 1;
+  if (p.seq) return 4;  // run list, C B^T per run chunk, fused per (run, head), exact
   const Problem t = tc_tiles(p);
   return tc_kernel_n(t) == 128 && tc_pair_supported(t) && tc_pair_split(t) ? 4 : 3;
 }
@@ -731,19 +753,13 @@ cudaError_t tc_forward(const Problem& pq, void* ws, cudaStream_t st, cudaEvent_t
   const TcWorkspace w = tc_carve(p, ws);
   cudaError_t e = cudaMemsetAsync(w.err, 0, w.zero_bytes, st);
   if (e != cudaSuccess) return e;
-  if (p.seq) {
-    // packed sequences: every unit on the exact kernel; sequence ids that never
-    // occur keep zero final states
-    if (p.final_states &&
-        (e = cudaMemsetAsync(p.final_states, 0, sizeof(float) * (size_t)(p.num_seqs * p.H * p.P * p.N), st)) !=
-            cudaSuccess)
-      return e;
-    if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
-    if ((e = (tc_kernel_n(p) == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st))) != cudaSuccess) return e;
-    return ev1 ? cudaEventRecord(ev1, st) : cudaSuccess;
-  }
+  // packed sequences: ids that never occur keep zero final states
+  if (p.seq && p.final_states &&
+      (e = cudaMemsetAsync(p.final_states, 0, sizeof(float) * (size_t)(p.num_seqs * p.H * p.P * p.N), st)) !=
+          cudaSuccess)
+    return e;
   if ((e = tc_fast_forward(p, w, st, ev0, ev1)) != cudaSuccess) return e;
-  return tc_kernel_n(p) == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st);
+  return tc_kernel_n(p) == 128 ? launch<128>(p, w, st, false) : launch<256>(p, w, st, false);
 }
 
 }  // namespace ssd

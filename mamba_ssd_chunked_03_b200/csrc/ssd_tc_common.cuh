@@ -21,11 +21,27 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per bounded wait
 // ssd_tc_pair.cu): 2^100 stays far inside fp32/bf16.
 constexpr float kRangeLog2 = 100.f;
 
+// Packed sequences run one sequence at a time ("runs"): every maximal run of
+// equal seq_idx in a batch row is chunked from its own first token, so no chunk
+// straddles a boundary and the runs are independent problems.  k_seq_runs
+// fills this list in the workspace.
+struct RunList {
+  int* count;  // runs, or 0 when the ids are not strictly increasing runs in
+               // [0, num_seqs) (every unit then goes to the exact kernel)
+  int* b;      // [num_seqs] batch row of run r
+  int* t0;     // [num_seqs] its first token in the row
+  int* len;    // [num_seqs] its tokens
+  int* id;     // [num_seqs] its sequence id
+  int* c0;     // [num_seqs + 1] its first chunk in the flattened chunk list
+};
+
 struct CbArgs {
   int64_t L, G, nc;
   const int32_t* seq;
-  __nv_bfloat16* wp;  // (b, nc, G, 64, 64) masked C B^T
+  __nv_bfloat16* wp;  // (chunks, G, 64, 64) masked C B^T; chunks = b * nc, or the runs' chunks
   int* err;
+  int varlen;         // chunks are the runs' chunks (RunList)
+  RunList runs;
 };
 
 struct FastArgs {
@@ -48,6 +64,11 @@ struct FastArgs {
   // handoff, its total decay per head to seg_decay [grid][2]
   int split;
   float* seg_decay;
+  // single-head kernel, packed sequences: one CTA per (run, head); a unit
+  // the factorised form cannot take marks its (row, head) once in unit_bad
+  int varlen;
+  RunList runs;
+  int* unit_bad;
 };
 
 // persistent grid of the two-head kernel, at most; per-CTA hand-over size
@@ -126,6 +147,8 @@ struct TcWorkspace {
   int* failed_list;       // (b*H) units for the exact kernel
   float* handoff;         // two-head kernel: kPairGridMax x kPairHandoffFloats, or null
   float* seg_decay;       // two-head kernel: kPairGridMax x 2 total decays (split mode), or null
+  tc::RunList runs;       // packed sequences: the run list, else null pointers
+  int* unit_bad;          // packed sequences: [b * H] exact-kernel marks (cleared per call), or null
 };
 
 // carve the caller's workspace (ws may be null to only size it: *total)

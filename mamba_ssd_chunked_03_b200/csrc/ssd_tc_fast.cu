@@ -54,6 +54,106 @@ namespace {
 using namespace sm100;
 using namespace tc;
 
+// ============================================================== k_seq_runs
+// One CTA lists the runs of equal seq_idx: in row-major token order, a run
+// starts at every token whose id differs from the token before it in the same
+// row ("Transformers与SSMs的隐藏联系" section 4.2: the decay is cut exactly
+// there).  Each run is an independent problem: its state starts from h0 if it
+// is its row's first run, else from zero, and its final state is that
+// sequence's.  The list is usable when the ids are strictly increasing along
+// it and lie in [0, num_seqs) (each id one run); otherwise count = 0 and every
+// (row, head) unit is put on the exact kernel's list.
+struct SeqRunArgs {
+  const int32_t* seq;
+  int64_t b, L, H, num_seqs;
+  RunList runs;
+  int* failed_count;
+  int* failed_list;
+};
+
+// exclusive prefix sum over the 1024 threads of the block; *total gets the sum
+__device__ __forceinline__ int64_t block_exclusive_scan(int64_t v, int64_t* total, int64_t* warp_sums) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int64_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) warp_sums[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    int64_t w = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    warp_sums[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int64_t before = (wid > 0 ? warp_sums[wid - 1] : 0) + incl - v;
+  *total = warp_sums[31];
+  __syncthreads();  // warp_sums may be reused by the caller's next scan
+  return before;
+}
+
+__global__ void __launch_bounds__(1024) k_seq_runs(const SeqRunArgs a) {
+  __shared__ int64_t warp_sums[32];
+  __shared__ int bad;
+  const int tid = threadIdx.x;
+  if (tid == 0) bad = 0;
+  const int64_t total = a.b * a.L;
+  const int64_t per = (total + 1023) / 1024;
+  const int64_t lo = tid * per < total ? tid * per : total;
+  const int64_t hi = lo + per < total ? lo + per : total;
+  auto is_start = [&](int64_t i) { return i % a.L == 0 || a.seq[i] != a.seq[i - 1]; };
+  int64_t cnt = 0;
+  for (int64_t i = lo; i < hi; ++i) cnt += is_start(i);
+  int64_t nr = 0;
+  int64_t k = block_exclusive_scan(cnt, &nr, warp_sums);
+  const bool fits = nr <= a.num_seqs;
+  if (fits)
+    for (int64_t i = lo; i < hi; ++i)
+      if (is_start(i)) {
+        a.runs.b[k] = (int)(i / a.L);
+        a.runs.t0[k] = (int)(i % a.L);
+        a.runs.id[k] = a.seq[i];
+        ++k;
+      }
+  __syncthreads();
+  // lengths, the id checks and the chunk counts, per block of runs
+  const int64_t rper = (nr + 1023) / 1024;
+  const int64_t rlo = fits && tid * rper < nr ? tid * rper : nr;
+  const int64_t rhi = fits && rlo + rper < nr ? rlo + rper : nr;
+  int64_t chunks = 0;
+  for (int64_t r = rlo; r < rhi; ++r) {
+    const bool last_in_row = r + 1 >= nr || a.runs.b[r + 1] != a.runs.b[r];
+    const int len = last_in_row ? (int)(a.L - a.runs.t0[r]) : a.runs.t0[r + 1] - a.runs.t0[r];
+    a.runs.len[r] = len;
+    const int id = a.runs.id[r];
+    if (id < 0 || id >= a.num_seqs || (r > 0 && id <= a.runs.id[r - 1])) bad = 1;
+    chunks += (len + 63) / 64;
+  }
+  int64_t nchunks = 0;
+  int64_t c = block_exclusive_scan(chunks, &nchunks, warp_sums);
+  for (int64_t r = rlo; r < rhi; ++r) {
+    a.runs.c0[r] = (int)c;
+    c += (a.runs.len[r] + 63) / 64;
+  }
+  if (tid == 0 && fits) a.runs.c0[nr] = (int)nchunks;
+  __syncthreads();
+  if (!fits || bad) {
+    for (int64_t u = tid; u < a.b * a.H; u += 1024) a.failed_list[u] = (int)u;
+    if (tid == 0) {
+      *a.runs.count = 0;
+      *a.failed_count = (int)(a.b * a.H);
+    }
+  } else if (tid == 0) {
+    *a.runs.count = (int)nr;
+  }
+}
+
 // ============================================================== k_chunk_cb
 template <int NS>
 struct CbCfg {
@@ -76,12 +176,31 @@ __global__ void __launch_bounds__(128) k_chunk_cb(const __grid_constant__ CUtens
   __shared__ int never;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   griddep_launch_dependents();  // the fused kernel may set up while this grid runs
+  // tile r = chunk * G + g; the chunk is (row, 64-token chunk) or, for packed
+  // sequences, (run, 64-token chunk of the run)
   const int64_t r = blockIdx.x;
   const int64_t g = r % a.G;
-  const int64_t c = (r / a.G) % a.nc;
-  const int64_t b = r / (a.G * a.nc);
-  const int t0 = (int)(c * 64);
-  const int nvalid = (int)((c + 1) * 64 <= a.L ? 64 : a.L - t0);
+  int64_t b;
+  int t0, nvalid;
+  if (a.varlen) {
+    const int nrun = *a.runs.count;
+    const int64_t ch = r / a.G;
+    if (nrun == 0 || ch >= a.runs.c0[nrun]) return;  // past the runs' chunks (uniform)
+    int lo = 0, hi = nrun - 1;  // the run holding chunk ch: the last with c0 <= ch
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.runs.c0[mid] <= ch) lo = mid; else hi = mid - 1;
+    }
+    const int c = (int)(ch - a.runs.c0[lo]);
+    b = a.runs.b[lo];
+    t0 = a.runs.t0[lo] + 64 * c;
+    nvalid = a.runs.len[lo] - 64 * c < 64 ? a.runs.len[lo] - 64 * c : 64;
+  } else {
+    const int64_t c = (r / a.G) % a.nc;
+    b = r / (a.G * a.nc);
+    t0 = (int)(c * 64);
+    nvalid = (int)((c + 1) * 64 <= a.L ? 64 : a.L - t0);
+  }
   const int64_t rowbase = b * a.L;
 
   if (tid == 0) {
@@ -206,11 +325,31 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
   __shared__ FastSmem s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   griddep_launch_dependents();  // the exact kernel may set up while this grid runs
+  // the unit: (batch row, head), or for packed sequences (run, head) -- tokens
+  // [t_base, t_base + len) of row b, chunked from t_base
   const int64_t unit = blockIdx.x;
-  const int64_t b = unit / a.H, h = unit % a.H;
+  const int64_t h = unit % a.H;
+  int64_t b, out_row, cbase;
+  int t_base, len;
+  if (a.varlen) {
+    const int64_t ru = unit / a.H;
+    if (ru >= *a.runs.count) return;  // past the runs (uniform)
+    b = a.runs.b[ru];
+    t_base = a.runs.t0[ru];
+    len = a.runs.len[ru];
+    out_row = a.runs.id[ru];       // final state: the sequence's
+    cbase = a.runs.c0[ru];         // W' of the run's chunks
+  } else {
+    b = unit / a.H;
+    t_base = 0;
+    len = (int)a.L;
+    out_row = b;
+    cbase = b * a.nc;
+  }
+  const bool first = t_base == 0;  // h0 is the state before a row's first token
   const int64_t g = h / a.hpg;
-  const int nc = (int)a.nc;
-  const int64_t rowbase = b * a.L;
+  const int nc = (len + 63) / 64;
+  const int64_t rowbase = b * a.L + t_base;
 
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) {
@@ -263,8 +402,8 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     float p0 = 0.f, p1 = 0.f;  // dt of tokens 2*lane, 2*lane+1 of the next chunk to scan
     auto load_dt = [&](int c) {
       const int64_t t = (int64_t)c * 64 + 2 * lane;
-      p0 = (c < nc && t < a.L) ? a.dt[(rowbase + t) * a.H + h] : 0.f;
-      p1 = (c < nc && t + 1 < a.L) ? a.dt[(rowbase + t + 1) * a.H + h] : 0.f;
+      p0 = (c < nc && t < len) ? a.dt[(rowbase + t) * a.H + h] : 0.f;
+      p1 = (c < nc && t + 1 < len) ? a.dt[(rowbase + t + 1) * a.H + h] : 0.f;
     };
     load_dt(0);
     int scanned = 0;
@@ -283,7 +422,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
       }
       const float cs1 = v, cs0 = v - x1;
       const float m = __shfl_sync(0xffffffffu, cs1, 15);  // token 31
-      const int nvalid = (int)((int64_t)(c + 1) * 64 <= a.L ? 64 : a.L - (int64_t)c * 64);
+      const int nvalid = (c + 1) * 64 <= len ? 64 : len - c * 64;
       const int e = nvalid - 1;
       const float cse = __shfl_sync(0xffffffffu, (e & 1) ? cs1 : cs0, e >> 1);
       float dev = fmaxf(fabsf(cs0 - m), fabsf(cs1 - m));
@@ -314,26 +453,27 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     auto issue_x = [&](int c) {
       const int sl = c % 3;
       mbar_arrive_expect_tx(&s.full_x[sl], K::kTile);
-      tma_load_3d(sm + K::oX + sl * K::kTile, &tm_x, &s.full_x[sl], (int)(h * 64), c * 64, (int)b);
+      tma_load_3d(sm + K::oX + sl * K::kTile, &tm_x, &s.full_x[sl], (int)(h * 64), t_base + c * 64, (int)b);
       last_x = c;
     };
     auto issue_w = [&](int c) {
       mbar_arrive_expect_tx(&s.full_w[c & 1], K::kTile);
       tma_load_3d(sm + K::oW + (c & 1) * K::kTile, &tm_w, &s.full_w[c & 1], 0,
-                  (int)(((b * a.nc + c) * a.G + g) * 64), 0);
+                  (int)(((cbase + c) * a.G + g) * 64), 0);
       last_w = c;
     };
     auto issue_b = [&](int c) {
       mbar_arrive_expect_tx(&s.full_b, K::NB * K::kTile);
       for (int j = 0; j < K::NB; ++j)
-        tma_load_4d(sm + K::oB + j * K::kTile, &tm_b, &s.full_b, 64 * j, (int)g, c * 64, (int)b);
+        tma_load_4d(sm + K::oB + j * K::kTile, &tm_b, &s.full_b, 64 * j, (int)g, t_base + c * 64, (int)b);
       last_b = c;
     };
     auto issue_c = [&](int c) {
       uint64_t* bar = &s.full_c[c & 1];
       mbar_arrive_expect_tx(bar, K::NB * K::kTile);
       for (int j = 0; j < K::NB; ++j)
-        tma_load_4d(sm + K::oC + ((c & 1) * K::NB + j) * K::kTile, &tm_c, bar, 64 * j, (int)g, c * 64, (int)b);
+        tma_load_4d(sm + K::oC + ((c & 1) * K::NB + j) * K::kTile, &tm_c, bar, 64 * j, (int)g, t_base + c * 64,
+                    (int)b);
       last_c = c;
     };
     bool ok = true;
@@ -459,7 +599,9 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
     for (int hf = 0; hf < K::NH; ++hf)
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        H[hf][j] = a.h0 && n0 + 128 * hf < a.Nr ? a.h0[((b * a.H + h) * 64 + pc0 + j) * a.Nr + n0 + 128 * hf] : 0.f;
+        H[hf][j] = a.h0 && first && n0 + 128 * hf < a.Nr
+                       ? a.h0[((b * a.H + h) * 64 + pc0 + j) * a.Nr + n0 + 128 * hf]
+                       : 0.f;
     bool failed = false;
 
     for (int c = 0; c <= nc; ++c) {
@@ -549,7 +691,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
       if (c >= 1) {
         const int ip = (c - 1) & 1, slp = (c - 1) & 3;
         const int64_t t0p = (int64_t)(c - 1) * 64;
-        const int nvp = (int)((int64_t)c * 64 <= a.L ? 64 : a.L - t0p);
+        const int nvp = c * 64 <= len ? 64 : (int)(len - t0p);
         if (!mbar_wait_warp(&s.y_full[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           continue;
@@ -579,7 +721,7 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
 #pragma unroll
       for (int hf = 0; hf < K::NH; ++hf) {
         if (n0 + 128 * hf >= a.Nr) continue;
-        float* dst = a.final_states + ((b * a.H + h) * 64 + pc0) * a.Nr + n0 + 128 * hf;
+        float* dst = a.final_states + ((out_row * a.H + h) * 64 + pc0) * a.Nr + n0 + 128 * hf;
 #pragma unroll
         for (int j = 0; j < 32; ++j) dst[(int64_t)j * a.Nr] = H[hf][j];
       }
@@ -591,33 +733,57 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
   tc_fence_after();
   if (tid == 0) {
     if (*abort_flag) atomicExch(a.err, 1);
-    // a chunk's decay range was too wide to factorise: the exact kernel redoes this unit
-    if (s.unit_bad) a.failed_list[atomicAdd(a.failed_count, 1)] = (int)unit;
+    // a chunk's decay range was too wide to factorise: the exact kernel redoes
+    // this unit (for packed sequences, the run's whole (row, head), once)
+    if (s.unit_bad) {
+      const int64_t rowunit = b * a.H + h;
+      if (!a.varlen) a.failed_list[atomicAdd(a.failed_count, 1)] = (int)unit;
+      else if (atomicExch(&a.unit_bad[rowunit], 1) == 0) a.failed_list[atomicAdd(a.failed_count, 1)] = (int)rowunit;
+    }
   }
   if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
 }
 
 // ev0 / ev1 (optional) are recorded right before and after the fused kernel.
+// Packed sequences (seq_idx): the run list first, then W' per run chunk and
+// the single-head kernel per (run, head).
 template <int NS>
 cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
+  const bool varlen = p.seq != nullptr;
+  const int64_t chunks = p.b * p.nc + (varlen ? p.num_seqs : 0);  // W' tiles per group, at most
   CUtensorMap tx, tb, tc_, tw;
   if (!make_map_3d(&tx, p.x, p.H * p.P, p.L, p.b) || !make_map_bc(&tb, p.B, p.N, p.G, p.L, p.b) ||
-      !make_map_bc(&tc_, p.C, p.N, p.G, p.L, p.b) || !make_map_3d(&tw, w.wp, 64, p.b * p.nc * p.G * 64, 1))
+      !make_map_bc(&tc_, p.C, p.N, p.G, p.L, p.b) || !make_map_3d(&tw, w.wp, 64, chunks * p.G * 64, 1))
     return cudaErrorInvalidValue;
-  CbArgs ca;
+  cudaError_t e;
+  if (varlen) {
+    SeqRunArgs sa;
+    sa.seq = p.seq;
+    sa.b = p.b;
+    sa.L = p.L;
+    sa.H = p.H;
+    sa.num_seqs = p.num_seqs;
+    sa.runs = w.runs;
+    sa.failed_count = w.failed_count;
+    sa.failed_list = w.failed_list;
+    k_seq_runs<<<1, 1024, 0, st>>>(sa);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  CbArgs ca{};
   ca.L = p.L;
   ca.G = p.G;
   ca.nc = p.nc;
-  ca.seq = p.seq;
+  ca.seq = nullptr;  // a run never crosses a sequence boundary
   ca.wp = w.wp;
   ca.err = w.err;
-  cudaError_t e = cudaFuncSetAttribute(k_chunk_cb<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)CbCfg<NS>::kSmemBytes);
+  ca.varlen = varlen;
+  ca.runs = w.runs;
+  e = cudaFuncSetAttribute(k_chunk_cb<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CbCfg<NS>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  k_chunk_cb<NS><<<(unsigned)(p.b * p.nc * p.G), 128, CbCfg<NS>::kSmemBytes, st>>>(tb, tc_, ca);
+  k_chunk_cb<NS><<<(unsigned)(chunks * p.G), 128, CbCfg<NS>::kSmemBytes, st>>>(tb, tc_, ca);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  FastArgs fa;
+  FastArgs fa{};
   fa.L = p.L;
   fa.H = p.H;
   fa.G = p.G;
@@ -637,7 +803,10 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
   fa.handoff = w.handoff;
   fa.flags = w.flags;
   fa.pair_bad = w.pair_bad;
-  if (NS == 128 && tc_pair_supported(p)) {
+  fa.varlen = varlen;
+  fa.runs = w.runs;
+  fa.unit_bad = w.unit_bad;
+  if (!varlen && NS == 128 && tc_pair_supported(p)) {
     CUtensorMap ty, tdt;
     if (!make_map_3d(&ty, p.y, p.H * p.P, p.L, p.b) || !make_map_dt(&tdt, p.dt, p.H, p.L, p.b))
       return cudaErrorInvalidValue;
@@ -649,8 +818,9 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
                            (int)FastCfg<NS>::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
-  e = launch_dependent(k_ssd_fwd_fast<NS>, (unsigned)(p.b * p.H), FastCfg<NS>::kThreads, FastCfg<NS>::kSmemBytes, st,
-                       tx, tb, tc_, tw, fa);
+  const int64_t units = (varlen ? p.num_seqs : p.b) * p.H;  // (run, head): at most num_seqs runs
+  e = launch_dependent(k_ssd_fwd_fast<NS>, (unsigned)units, FastCfg<NS>::kThreads, FastCfg<NS>::kSmemBytes, st, tx,
+                       tb, tc_, tw, fa);
   if (e != cudaSuccess) return e;
   return ev1 ? cudaEventRecord(ev1, st) : cudaSuccess;
 }
@@ -658,7 +828,7 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
 }  // namespace
 
 const char* tc_main_kernel(const Problem& p) {
-  if (p.seq) return "k_ssd_fwd_tc";
+  if (p.seq) return "k_ssd_fwd_fast";  // per (run, head)
   return tc_kernel_n(p) == 128 && tc_pair_supported(tc_tiles(p)) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
 }
 

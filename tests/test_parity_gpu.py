@@ -254,6 +254,39 @@ def test_strong_decay_heads_take_the_exact_kernel(N):
     assert state_err(f, fr) <= 1e-2, state_err(f, fr)
 
 
+@pytest.mark.parametrize("N", [128, 256])
+def test_packed_strong_decay_runs_take_the_exact_kernel(N):
+    """Packed sequences run per (sequence, head) on the fast kernel; a head
+    with a steep stretch inside one sequence sends its (row, head) to the exact
+    kernel, which redoes the whole row for that head.  Two sequences share the
+    steep head's row, so the exact kernel rewrites outputs the fast kernel also
+    wrote; both rows and every sequence's final state must match the oracle."""
+    s = si.SSDShape("steep_packed", 2, 320, 4, 64, N, 2, 64, "bf16", h0_std=0.2, seed=33)
+    d = si.make_inputs(s)
+    d["seq_idx"], d["num_seqs"] = si.seq_idx_from_lengths([[130, 190], [64, 100, 156]])
+    d["dt"][0, 140:180, 3] = 1.5   # inside the second sequence of row 0
+    d["A"][3] = -12.0
+    g = to_dev(d)
+    assert ssd.main_kernel(g["x"], g["dt"], g["B"], 64, seq_idx=g["seq_idx"], num_seqs=d["num_seqs"]) == "k_ssd_fwd_fast"
+    y, f = run_gpu(d, 64)
+    yr, fr = run_oracle(d)
+    assert rel_l2(y, yr) <= 1e-2, rel_l2(y, yr)
+    assert state_err(f, fr) <= 1e-2, state_err(f, fr)
+
+
+def test_packed_ids_out_of_order_take_the_exact_kernel():
+    """Sequence ids that do not increase along the tokens cannot be listed as
+    independent runs; every unit then goes to the exact kernel."""
+    s = si.SSDShape("packed_order", 1, 240, 4, 64, 128, 1, 64, "bf16", h0_std=0.3, seed=35)
+    d = si.make_inputs(s)
+    d["seq_idx"] = torch.tensor([[2] * 50 + [0] * 100 + [1] * 90], dtype=torch.int32)
+    d["num_seqs"] = 3
+    y, f = run_gpu(d, 64)
+    yr, fr = run_oracle(d)
+    assert rel_l2(y, yr) <= 1e-2, rel_l2(y, yr)
+    assert state_err(f, fr) <= 1e-2, state_err(f, fr)
+
+
 def test_zero_step_tokens():
     """dt = 0 tokens (a_t = 1, no input) still get their D x term."""
     s = si.SSDShape("dt0", 1, 200, 4, 64, 128, 1, 64, "bf16", h0_std=0.1, seed=41)
