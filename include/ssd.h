@@ -90,7 +90,10 @@ typedef struct {
   const int32_t* seq_idx;         /* (b,L) int32 packed-sequence ids, or NULL.
                                      Precondition: non-decreasing along each row, ids
                                      in [0, num_seqs), a sequence never spans rows.
-                                     A change of id starts a new sequence (a_t = 0). */
+                                     A change of id starts a new sequence (a_t = 0).
+                                     Ids increasing from row to row (each id one
+                                     run) run per sequence on the fast kernels;
+                                     other orders on a slower per-(row, head) one. */
   int64_t num_seqs;               /* number of sequence ids; required (> 0) iff seq_idx */
 
   void* y;                        /* (b,L,H,P) dtype, output                          */
