@@ -152,9 +152,8 @@ struct TcArgs {
   const int32_t* seq;
   __nv_bfloat16* y;
   float* final_states;
-  const int* failed_count;  // units to process, listed by the fast kernel ...
+  const int* failed_count;  // units to process, listed by the fast kernel
   const int* failed_list;
-  int all_units;            // ... or, if set, every unit
   int64_t num_seqs;         // packed sequences: final states of ids outside [0, num_seqs) are not written
   int* err;
 };
@@ -185,7 +184,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
   const int nc = (int)a.nc;
   // a small persistent grid walks the list of units the fast kernel could not do
   griddep_wait();  // the list comes from the fused kernel launched before this one
-  const int count = a.all_units ? (int)(a.b * a.H) : *reinterpret_cast<const volatile int*>(a.failed_count);
+  const int count = *reinterpret_cast<const volatile int*>(a.failed_count);
   if ((int)blockIdx.x >= count) return;  // uniform: every thread reads the same count
 
   if (tid == 0) {
@@ -208,7 +207,7 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
   volatile int* never = &s.never;
 
   for (int it = blockIdx.x; it < count; it += gridDim.x) {
-  const int64_t unit = a.all_units ? it : a.failed_list[it];
+  const int64_t unit = a.failed_list[it];
   const int64_t b = unit / a.H, h = unit % a.H;
   const int64_t g = h / a.hpg;
   if (tid == 0) {  // fresh barriers per unit (all earlier phases have completed)
@@ -634,9 +633,8 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
 }
 
 // ---------------------------------------------------------------- host side
-// all_units: every (batch row, head), else the units the fast kernel listed
 template <int NS>
-cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st, bool all_units) {
+cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
   CUtensorMap tx, tb, tc_;
   if (!make_map_3d(&tx, p.x, p.H * p.P, p.L, p.b) || !make_map_bc(&tb, p.B, p.N, p.G, p.L, p.b) ||
       !make_map_bc(&tc_, p.C, p.N, p.G, p.L, p.b))
@@ -658,7 +656,6 @@ cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st, bool
   a.final_states = p.final_states;
   a.failed_count = w.failed_count;
   a.failed_list = w.failed_list;
-  a.all_units = all_units;
   a.num_seqs = p.seq ? p.num_seqs : 0;
   a.err = w.err;
   cudaError_t e = cudaFuncSetAttribute(k_ssd_fwd_tc<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -759,7 +756,7 @@ cudaError_t tc_forward(const Problem& pq, void* ws, cudaStream_t st, cudaEvent_t
           cudaSuccess)
     return e;
   if ((e = tc_fast_forward(p, w, st, ev0, ev1)) != cudaSuccess) return e;
-  return tc_kernel_n(p) == 128 ? launch<128>(p, w, st, false) : launch<256>(p, w, st, false);
+  return tc_kernel_n(p) == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st);
 }
 
 }  // namespace ssd
