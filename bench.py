@@ -254,6 +254,112 @@ def run_reference(args, shape):
     return 0
 
 
+# ----------------------------------------------------------------------------- decode step
+
+def run_step(args, dist, dev, world, rank):
+    """``--op step``: the recurrent (decode) step ``ssd_step`` on one token per
+    row for ``--step-batch`` rows of the c1 head layout (H 80, P 64, N 128,
+    G 1, bf16), the fp32 state resident in HBM and updated in place.  Bound by
+    HBM on the state: 8 b H P N bytes read and written per step."""
+    import mamba_ssd_chunked_03_b200 as ssd
+    b, H, P, N, G = args.step_batch, 80, 64, 128, 1
+    shape = si.SSDShape("decode", b, 1, H, P, N, G, 64, "bf16", h0_std=0.5, seed=11 + rank)
+    host = si.make_inputs(shape)
+    inputs = {k: host[k][:, 0].contiguous() for k in ("x", "dt", "B", "C")}
+    g = {k: v.to(dev) for k, v in inputs.items()}
+    A, D = host["A"].to(dev), host["D"].to(dev)
+    state = host["initial_states"].to(dev)
+    y = torch.empty_like(g["x"])
+
+    def step():
+        ssd.step(g["x"], g["dt"], A, g["B"], g["C"], D, state, y=y)
+
+    K = args.steps
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_uuid(dev))
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clock_stats = clocks.stop()
+    ms_step = max_over_ranks(e0.elapsed_time(e1), dist, dev) / K
+
+    # end to end: this step's inputs from pinned host memory, y back; the state
+    # stays on the device (it is the decode cache)
+    pinned = {k: v.pin_memory() for k, v in inputs.items()}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = y_host.numel() * y_host.element_size()
+
+    def e2e_step():
+        for k in pinned:
+            g[k].copy_(pinned[k], non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    E = max(3, min(K, 50))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(E):
+        e2e_step()
+    a1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev) / E
+
+    state_bytes = b * H * P * N * 4
+    nbytes = 2 * state_bytes + 2 * b * H * P * 2 + 2 * b * G * N * 2 + b * H * 4
+    peaks = load_peaks()
+    achieved = nbytes / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": "SSD decode step (one token per row), rows/s", "value": b * world / (ms_step / 1e3),
+        "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"decode step: b{b} H{H} P{P} N{N} G{G} bf16, fp32 state in HBM "
+                               f"({state_bytes / 1e6:.0f} MB)",
+                   "l2": f"no flush: state {state_bytes / 1e6:.0f} MB > 126 MB L2",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                     "frac_datasheet": achieved / DATASHEET_HBM_GBS, "kernel": "k_ssd_step",
+                     "kernel_ms": ms_step, "traffic": None, "algorithmic_bytes": nbytes},
+        "e2e": {"value": b * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": E},
+        "gpu_launches": K,
+        "clocks": clock_stats,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle  # test infrastructure: only this CPU-baseline leg uses it here
+        f = {k: oracle.as_f32(host[k]) for k in ("x", "dt", "A", "B", "C", "D", "initial_states")}
+        threads = oracle.max_threads()
+        reps, t = 0, time.perf_counter()
+        while True:
+            oracle.ssd_fwd(f["x"], f["dt"], f["A"], f["B"], f["C"], f["D"], f["initial_states"])
+            reps += 1
+            el = time.perf_counter() - t
+            if el >= min(args.cpu_seconds, 10.0):
+                break
+        line["cpu_baseline"] = {"value": reps * b / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{reps} whole steps of the workload (all {b} rows), {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def main():
@@ -266,6 +372,9 @@ def main():
     ap.add_argument("--generic", action="store_true", help="force the generic CUDA-core kernels")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--op", default="fwd", choices=["fwd", "step"],
+                    help="fwd: the chunked forward (default); step: the recurrent decode step")
+    ap.add_argument("--step-batch", type=int, default=256, help="rows of the decode step (--op step)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -288,6 +397,8 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    if args.op == "step":
+        return run_step(args, dist, dev, world, rank)
 
     host = si.make_inputs(shape, seed=shape.seed + rank)
     num_seqs = host.get("num_seqs")

@@ -174,6 +174,36 @@ SSD_API const char* ssd_fwd_main_kernel(const ssd_fwd_args* args);
  * synchronisation or the read fails.  No counterpart in the pages. */
 SSD_API ssd_status ssd_fwd_device_status(const ssd_fwd_args* args, void* stream);
 
+/* One recurrent step (decode): one new token per batch row against a running
+ * state held by the caller, per row b and head h (group g as above):
+ *
+ *   state[b,h] <- exp(dt[b,h] A_h) state[b,h] + dt[b,h] x[b,h] B[b,g]^T
+ *   y[b,h]      = state[b,h] C[b,g] + D_h x[b,h]
+ *
+ * the recurrent form of the same model ("22 · Mamba 2 — Transformers are
+ * SSMs" section 3.1; the D feed-through as above).  It equals ssd_fwd over
+ * one token (L = 1) with initial_states = state and final_states written
+ * back to state.  Sizes as in ssd_fwd_args with dstate a multiple of 4 and at
+ * most 256 (else SSD_ERR_UNSUPPORTED).  All pointers are device pointers
+ * owned by the caller; state is read and written in place (16-byte aligned),
+ * B and C must be aligned to 4 elements.  Asynchronous on `stream`; nothing
+ * is enqueued when the arguments are rejected. */
+typedef struct {
+  int64_t batch, nheads, headdim, dstate, ngroups;
+  ssd_dtype dtype;      /* of x, B, C and y */
+  const void* x;        /* (b,H,P) dtype, this step's input                  */
+  const float* dt;      /* (b,H) fp32 step sizes                             */
+  const float* A;       /* (H) fp32 per-head decay rates                     */
+  const void* B;        /* (b,G,N) dtype                                     */
+  const void* C;        /* (b,G,N) dtype                                     */
+  const float* D;       /* (H) fp32 skip weight, or NULL for D = 0           */
+  float* state;         /* (b,H,P,N) fp32, the state before the step; holds
+                           the state after it on return                      */
+  void* y;              /* (b,H,P) dtype, output                             */
+} ssd_step_args;
+
+SSD_API ssd_status ssd_step(const ssd_step_args* args, void* stream);
+
 /* Static, human-readable text for a status code. */
 SSD_API const char* ssd_status_string(ssd_status status);
 

@@ -9,6 +9,7 @@ Python or CPU fallback, and importing fails loudly if the library is missing.
 
     y, final_states = fwd(x, dt, A, B, C, D, chunk_size=64,
                           initial_states=None, seq_idx=None, num_seqs=None)
+    y_t = step(x_t, dt_t, A, B_t, C_t, D, state)   # one decode step, state in place
 """
 from __future__ import annotations
 
@@ -18,7 +19,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["fwd", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
+__all__ = ["fwd", "step", "StepArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
            "SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED", "SSD_ERR_WORKSPACE", "SSD_ERR_CUDA",
            "SSD_F32", "SSD_BF16", "SSD_FLAG_GENERIC"]
 
@@ -45,6 +46,16 @@ class Args(ctypes.Structure):
     ]
 
 
+class StepArgs(ctypes.Structure):
+    """Mirror of ``ssd_step_args``."""
+    _fields_ = [(n, ctypes.c_int64) for n in ("batch", "nheads", "headdim", "dstate", "ngroups")] + [
+        ("dtype", ctypes.c_int),
+        ("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("A", ctypes.c_void_p),
+        ("B", ctypes.c_void_p), ("C", ctypes.c_void_p), ("D", ctypes.c_void_p),
+        ("state", ctypes.c_void_p), ("y", ctypes.c_void_p),
+    ]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -63,6 +74,8 @@ def _load() -> ctypes.CDLL:
     L.ssd_fwd_path.restype = ctypes.c_char_p
     L.ssd_fwd_main_kernel.argtypes = [ctypes.POINTER(Args)]
     L.ssd_fwd_main_kernel.restype = ctypes.c_char_p
+    L.ssd_step.argtypes = [ctypes.POINTER(StepArgs), ctypes.c_void_p]
+    L.ssd_step.restype = ctypes.c_int
     L.ssd_status_string.argtypes = [ctypes.c_int]
     L.ssd_status_string.restype = ctypes.c_char_p
     L.ssd_version.restype = ctypes.c_int
@@ -223,3 +236,36 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     if st != SSD_OK:
         raise SSDError(st)
     return y, final_states
+
+
+def step(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+         D: Optional[torch.Tensor], state: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One recurrent (decode) step via ``ssd_step``: x (b,H,P), dt (b,H), A (H),
+    B and C (b,G,N), D (H) or None, state (b,H,P,N) fp32, updated in place.
+    Returns y (b,H,P) in x's dtype."""
+    if x.dim() != 3 or dt.dim() != 2 or B.dim() != 3 or C.dim() != 3 or state.dim() != 4:
+        raise ValueError("expected x (b,H,P), dt (b,H), B and C (b,G,N), state (b,H,P,N)")
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    if tuple(dt.shape) != (b, H) or tuple(A.shape) != (H,) or tuple(C.shape) != (b, G, N) \
+            or tuple(B.shape) != (b, G, N) or tuple(state.shape) != (b, H, P, N):
+        raise ValueError("shapes do not match x (b,H,P) and B (b,G,N)")
+    if x.dtype not in (torch.float32, torch.bfloat16) or B.dtype != x.dtype or C.dtype != x.dtype:
+        raise TypeError("x, B and C must all be float32 or all bfloat16")
+    if dt.dtype != torch.float32 or A.dtype != torch.float32 or state.dtype != torch.float32 \
+            or (D is not None and (D.dtype != torch.float32 or tuple(D.shape) != (H,))):
+        raise TypeError("dt, A, D and state must be float32 (D of shape (H,))")
+    for name, t in (("x", x), ("dt", dt), ("A", A), ("B", B), ("C", C), ("D", D), ("state", state)):
+        if t is not None and (t.device != x.device or x.device.type != "cuda" or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor on {x.device}")
+    if y is None:
+        y = torch.empty_like(x)
+    a = StepArgs()
+    a.batch, a.nheads, a.headdim, a.dstate, a.ngroups = b, H, P, N, G
+    a.dtype = SSD_BF16 if x.dtype == torch.bfloat16 else SSD_F32
+    a.x, a.dt, a.A, a.B, a.C, a.D = _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D)
+    a.state, a.y = _ptr(state), _ptr(y)
+    st = lib.ssd_step(ctypes.byref(a), ctypes.c_void_p(torch.cuda.current_stream(x.device).cuda_stream))
+    if st != SSD_OK:
+        raise SSDError(st)
+    return y

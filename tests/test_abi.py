@@ -133,3 +133,63 @@ def test_launch_count_query():
     assert n >= 1
     a.chunk_size = 3
     assert ssd.lib.ssd_fwd_launch_count(ctypes.byref(a)) == 0
+
+
+def _c_layout(fields, struct):
+    """offsetof/sizeof of a header struct, from a C program compiled here."""
+    import subprocess
+    import tempfile
+    body = "\n".join(f'printf("%zu\\n", offsetof({struct}, {f}));' for f in fields)
+    src = (f'#include <stddef.h>\n#include <stdio.h>\n#include "ssd.h"\n'
+           f'int main(void) {{ {body} printf("%zu\\n", sizeof({struct})); return 0; }}\n')
+    with tempfile.TemporaryDirectory() as tmp:
+        c, exe = os.path.join(tmp, "l.c"), os.path.join(tmp, "l")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()
+    return [int(v) for v in out]
+
+
+def test_step_struct_layout_matches_the_compiled_header():
+    names = [f[0] for f in ssd.StepArgs._fields_]
+    got = _c_layout(names, "ssd_step_args")
+    assert got[:-1] == [getattr(ssd.StepArgs, n).offset for n in names]
+    assert got[-1] == ctypes.sizeof(ssd.StepArgs)
+
+
+def test_fwd_struct_layout_matches_the_compiled_header():
+    names = [f[0] for f in ssd.Args._fields_]
+    got = _c_layout(names, "ssd_fwd_args")
+    assert got[:-1] == [getattr(ssd.Args, n).offset for n in names]
+    assert got[-1] == ctypes.sizeof(ssd.Args)
+
+
+def _step_args(**kw):
+    a = ssd.StepArgs()
+    a.batch, a.nheads, a.headdim, a.dstate, a.ngroups = 2, 4, 64, 128, 2
+    a.dtype = ssd.SSD_BF16
+    # placeholders that are never dereferenced: every case below is rejected on the host
+    for i, n in enumerate(("x", "dt", "A", "B", "C", "D", "state", "y")):
+        setattr(a, n, 4096 * (i + 1))
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({"batch": 0}, ssd.SSD_ERR_INVALID_ARG),
+    ({"nheads": 6, "ngroups": 4}, ssd.SSD_ERR_INVALID_ARG),
+    ({"dtype": 7}, ssd.SSD_ERR_INVALID_ARG),
+    ({"x": None}, ssd.SSD_ERR_INVALID_ARG),
+    ({"state": None}, ssd.SSD_ERR_INVALID_ARG),
+    ({"state": 4096 + 8}, ssd.SSD_ERR_INVALID_ARG),   # not 16-byte aligned
+    ({"B": 4096 + 4}, ssd.SSD_ERR_INVALID_ARG),       # not aligned to 4 bf16
+    ({"dstate": 130}, ssd.SSD_ERR_UNSUPPORTED),
+    ({"dstate": 512}, ssd.SSD_ERR_UNSUPPORTED),
+])
+def test_step_rejects_bad_arguments(kw, status):
+    assert ssd.lib.ssd_step(ctypes.byref(_step_args(**kw)), None) == status
+
+
+def test_step_null_args_pointer():
+    assert ssd.lib.ssd_step(None, None) == ssd.SSD_ERR_INVALID_ARG
