@@ -204,6 +204,31 @@ typedef struct {
 
 SSD_API ssd_status ssd_step(const ssd_step_args* args, void* stream);
 
+/* Sequence parallelism: a sequence split over R ranks, rank k holding a
+ * contiguous range of the tokens of every row.  The recurrence is affine in
+ * the state, so over rank k's range h_out = D_k h_in + S_k, with S_k the
+ * range's end state from a zero state (ssd_fwd without initial_states) and
+ * D_k its total decay.  Rank r starts from h0 carried through ranks 0..r-1.
+ * This is the state passing of "SSM 家族全景图（下）：Mamba-2 与 Jamba"
+ * section 三.4 with a rank's range as one chunk.  Packed sequences are not
+ * split this way.  Both calls are asynchronous on `stream`; device pointers
+ * owned by the caller; nothing is enqueued when the arguments are rejected. */
+
+/* out (b,H) fp32 = exp(A_h * sum_t dt[b,t,h]) over the seqlen tokens of dt
+ * (b,L,H) fp32; A (H) fp32.  (The sum is taken in fp64.) */
+SSD_API ssd_status ssd_total_decay(const float* dt, const float* A, float* out, int64_t batch, int64_t seqlen,
+                                   int64_t nheads, void* stream);
+
+/* out (b,H,P,N) fp32 = initial_states (or 0 when NULL) carried through
+ * ranks 0..rank-1: H <- decays[k] * H + states[k] for k = 0..rank-1, with
+ * states (R,b,H,P,N) fp32 (S_k) and decays (R,b,H) fp32 (D_k); states and
+ * decays may be NULL when rank = 0.  headdim * dstate a multiple of 4
+ * (SSD_ERR_UNSUPPORTED otherwise); states, initial_states and out 16-byte
+ * aligned.  out must not overlap the inputs. */
+SSD_API ssd_status ssd_state_fold(const float* states, const float* decays, const float* initial_states,
+                                  float* out, int64_t rank, int64_t batch, int64_t nheads, int64_t headdim,
+                                  int64_t dstate, void* stream);
+
 /* Static, human-readable text for a status code. */
 SSD_API const char* ssd_status_string(ssd_status status);
 

@@ -19,7 +19,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["fwd", "step", "StepArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
+__all__ = ["fwd", "step", "StepArgs", "total_decay", "state_fold", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
            "SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED", "SSD_ERR_WORKSPACE", "SSD_ERR_CUDA",
            "SSD_F32", "SSD_BF16", "SSD_FLAG_GENERIC"]
 
@@ -76,6 +76,11 @@ def _load() -> ctypes.CDLL:
     L.ssd_fwd_main_kernel.restype = ctypes.c_char_p
     L.ssd_step.argtypes = [ctypes.POINTER(StepArgs), ctypes.c_void_p]
     L.ssd_step.restype = ctypes.c_int
+    L.ssd_total_decay.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int64] * 3 + [
+        ctypes.c_void_p]
+    L.ssd_total_decay.restype = ctypes.c_int
+    L.ssd_state_fold.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 5 + [ctypes.c_void_p]
+    L.ssd_state_fold.restype = ctypes.c_int
     L.ssd_status_string.argtypes = [ctypes.c_int]
     L.ssd_status_string.restype = ctypes.c_char_p
     L.ssd_version.restype = ctypes.c_int
@@ -269,3 +274,47 @@ def step(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C:
     if st != SSD_OK:
         raise SSDError(st)
     return y
+
+
+def _stream(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def total_decay(dt: torch.Tensor, A: torch.Tensor) -> torch.Tensor:
+    """``ssd_total_decay``: exp(A_h * sum_t dt[b,t,h]) as a (b,H) fp32 tensor."""
+    if dt.dim() != 3 or dt.dtype != torch.float32 or A.dtype != torch.float32 or tuple(A.shape) != (dt.shape[2],):
+        raise ValueError("dt must be float32 (b,L,H) and A float32 (H,)")
+    if not (dt.is_cuda and A.is_cuda and dt.is_contiguous() and A.is_contiguous()):
+        raise ValueError("dt and A must be contiguous CUDA tensors")
+    b, L, H = dt.shape
+    out = torch.empty(b, H, device=dt.device, dtype=torch.float32)
+    st = lib.ssd_total_decay(dt.data_ptr(), A.data_ptr(), out.data_ptr(), b, L, H, _stream(dt))
+    if st != SSD_OK:
+        raise SSDError(st)
+    return out
+
+
+def state_fold(states: Optional[torch.Tensor], decays: Optional[torch.Tensor],
+               initial_states: Optional[torch.Tensor], rank: int, shape) -> torch.Tensor:
+    """``ssd_state_fold``: initial_states (or 0) carried through ranks
+    0..rank-1 of states (R,b,H,P,N) and decays (R,b,H); shape = (b,H,P,N)."""
+    b, H, P, N = shape
+    dev = next(t.device for t in (states, initial_states, decays) if t is not None) if (
+        states is not None or initial_states is not None) else torch.device("cuda")
+    for name, t, want in (("states", states, None), ("decays", decays, None),
+                          ("initial_states", initial_states, (b, H, P, N))):
+        if t is None:
+            continue
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+        if want is not None and tuple(t.shape) != want:
+            raise ValueError(f"{name} must be {want}")
+    if rank > 0 and (states is None or decays is None or states.shape[0] < rank or decays.shape[0] < rank
+                     or tuple(states.shape[1:]) != (b, H, P, N) or tuple(decays.shape[1:]) != (b, H)):
+        raise ValueError("states (R,b,H,P,N) and decays (R,b,H) with R >= rank are needed for rank > 0")
+    out = torch.empty(b, H, P, N, device=dev, dtype=torch.float32)
+    st = lib.ssd_state_fold(_ptr(states), _ptr(decays), _ptr(initial_states), out.data_ptr(), int(rank), b, H, P, N,
+                            _stream(out))
+    if st != SSD_OK:
+        raise SSDError(st)
+    return out

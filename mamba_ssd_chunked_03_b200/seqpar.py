@@ -1,0 +1,77 @@
+"""Sequence parallelism for the SSD forward over ``torch.distributed`` ranks.
+
+Each of R ranks holds a contiguous range of the tokens of every row
+(x (b, L_r, H, P), dt, B, C alike).  The recurrence is affine in the state,
+so over rank k's range it is h_out = D_k h_in + S_k:
+
+1. every rank runs its range from a zero state: S_k = its end state, and
+   D_k = exp(A_h * sum of its dt) (``ssd_total_decay``);
+2. the ranks all-gather (S_k, D_k) -- the one exchange step;
+3. rank r starts from h0 carried through ranks 0..r-1 (``ssd_state_fold``)
+   and runs its range again from that state, which gives its y and the state
+   at its range's end (rank R-1's is the sequence's final state).
+
+That is the state passing of "SSM 家族全景图（下）：Mamba-2 与 Jamba" section
+三.4 with a rank's range as one chunk.  All arithmetic runs in the library's
+kernels; this module only calls them and moves the states between ranks.
+Packed sequences (seq_idx) are not split this way.
+
+The three per-rank operations are taken from ``ops`` (default: the library),
+so the exchange logic can be exercised on CPU ranks with another
+implementation of them.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import fwd, state_fold, total_decay
+
+
+class LibraryOps:
+    """The per-rank operations, on the library's kernels."""
+
+    @staticmethod
+    def local_forward(x, dt, A, B, C, D, chunk_size, initial_states):
+        return fwd(x, dt, A, B, C, D, chunk_size=chunk_size, initial_states=initial_states)
+
+    @staticmethod
+    def total_decay(dt, A):
+        return total_decay(dt, A)
+
+    @staticmethod
+    def state_fold(states, decays, initial_states, rank, shape):
+        return state_fold(states, decays, initial_states, rank, shape)
+
+
+def local_summary(x, dt, A, B, C, D, chunk_size: int = 64, ops=LibraryOps):
+    """(S, D_total) of this rank's range: its end state from a zero state and
+    its total decay, (b,H,P,N) and (b,H) fp32."""
+    _, S = ops.local_forward(x, dt, A, B, C, D, chunk_size, None)
+    return S, ops.total_decay(dt, A)
+
+
+def carry_in(states, decays, initial_states, rank: int, shape, ops=LibraryOps):
+    """The state before rank ``rank``'s first token, from the gathered
+    summaries of ranks 0..rank-1 (states (R,b,H,P,N), decays (R,b,H))."""
+    return ops.state_fold(states, decays, initial_states, rank, shape)
+
+
+def fwd_seqpar(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+               D: Optional[torch.Tensor], chunk_size: int = 64, initial_states: Optional[torch.Tensor] = None,
+               group=None, ops=LibraryOps):
+    """The forward of this rank's token range of a sequence split over the
+    ranks of ``group``, in rank order.  ``initial_states`` (the state before
+    the sequence's first token, or None) must be the same on every rank.
+    Returns (y of this rank's tokens, the state at the end of its range)."""
+    import torch.distributed as dist
+    R = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    S, dec = local_summary(x, dt, A, B, C, D, chunk_size, ops)
+    all_S = [torch.empty_like(S) for _ in range(R)]
+    all_d = [torch.empty_like(dec) for _ in range(R)]
+    dist.all_gather(all_S, S.contiguous(), group=group)
+    dist.all_gather(all_d, dec.contiguous(), group=group)
+    h_in = carry_in(torch.stack(all_S), torch.stack(all_d), initial_states, r, tuple(S.shape), ops)
+    return ops.local_forward(x, dt, A, B, C, D, chunk_size, h_in)

@@ -1,0 +1,117 @@
+"""Sequence parallelism on the CPU: the composition rule the split relies on,
+pinned on the oracle, and the exchange logic of ``seqpar.fwd_seqpar`` on two
+gloo ranks (with the per-rank operations done by the oracle, since these
+ranks have no GPU).
+
+The rule: over a contiguous token range the recurrence is affine in the
+state, h_out = D h_in + S, with S the range's end state from a zero state and
+D = exp(A sum dt); a sequence split into ranges and carried through them
+equals the sequence run whole."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+import ssd_inputs as si
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _split(d, lo, hi):
+    return {k: (v[:, lo:hi].contiguous() if k in ("x", "dt", "B", "C") else v) for k, v in d.items()}
+
+
+def _whole(d):
+    return oracle.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["initial_states"])
+
+
+class OracleOps:
+    """The per-rank operations of seqpar, on the oracle (fp64)."""
+
+    @staticmethod
+    def local_forward(x, dt, A, B, C, D, chunk_size, initial_states):
+        y, f = oracle.ssd_fwd(x, dt, A, B, C, D, initial_states)
+        return torch.from_numpy(y), torch.from_numpy(f).float()
+
+    @staticmethod
+    def total_decay(dt, A):
+        s = dt.double().sum(dim=1)  # (b, H)
+        return torch.exp(A.double()[None, :] * s).float()
+
+    @staticmethod
+    def state_fold(states, decays, initial_states, rank, shape):
+        h = torch.zeros(shape, dtype=torch.float64) if initial_states is None else initial_states.double().clone()
+        for k in range(rank):
+            h = decays[k].double()[:, :, None, None] * h + states[k].double()
+        return h.float()
+
+
+@pytest.mark.parametrize("cuts", [[0, 90, 91, 200], [0, 64, 128, 200], [0, 200]])
+def test_split_sequence_composes_to_the_whole(cuts):
+    shape = si.SSDShape("sp", 2, 200, 3, 8, 8, 1, 64, "f32", h0_std=0.5, seed=5)
+    d = si.make_inputs(shape)
+    yw, fw = _whole(d)
+    h = d["initial_states"].double().numpy()
+    ys = []
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        p = _split(d, lo, hi)
+        # the range's summary: end state from zero, total decay
+        _, S = oracle.ssd_fwd(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], None)
+        Dk = np.exp(p["A"].double().numpy()[None, :] * p["dt"].double().numpy().sum(axis=1))
+        y, f = oracle.ssd_fwd(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], torch.from_numpy(h).float())
+        ys.append(y)
+        h_next = Dk[:, :, None, None] * h + S
+        # the carried state is the range's true end state
+        assert np.abs(h_next - f).max() <= 1e-5 * max(1.0, np.abs(f).max())
+        h = h_next
+    y = np.concatenate(ys, axis=1)
+    assert np.abs(y - yw).max() <= 1e-5 * max(1.0, np.abs(yw).max())
+    assert np.abs(h - fw).max() <= 1e-5 * max(1.0, np.abs(fw).max())
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, cuts, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from mamba_ssd_chunked_03_b200 import seqpar
+        shape = si.SSDShape("sp", 2, 200, 3, 8, 8, 1, 64, "f32", h0_std=0.5, seed=5)
+        d = si.make_inputs(shape)
+        p = _split(d, cuts[rank], cuts[rank + 1])
+        y, f = seqpar.fwd_seqpar(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], 64, d["initial_states"],
+                                 ops=OracleOps)
+        out[rank] = (np.asarray(y), np.asarray(f))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_fwd_seqpar_two_gloo_ranks():
+    cuts = [0, 117, 200]
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_rank_main, args=(r, 2, port, cuts, out)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(180)
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        shape = si.SSDShape("sp", 2, 200, 3, 8, 8, 1, 64, "f32", h0_std=0.5, seed=5)
+        yw, fw = _whole(si.make_inputs(shape))
+        y = np.concatenate([out[0][0], out[1][0]], axis=1)
+        assert np.abs(y - yw).max() <= 1e-5 * max(1.0, np.abs(yw).max())
+        assert np.abs(out[1][1] - fw).max() <= 1e-5 * max(1.0, np.abs(fw).max())
