@@ -38,8 +38,9 @@
 // sequence's own tokens of the chunk (CUDA cores, while the chunk's x and B
 // tiles are still held).
 //
-// Warp roles (192 threads):  warp 0 TMA producer, warp 1 MMA issuer (one
-// thread), warps 2-5 compute (cumsum, mask, scale, state update, epilogue).
+// Warp roles (192 threads):  warp 0 TMA producer, warp 1 MMA issuer (the warp
+// forms the descriptors, one elected lane issues), warps 2-5 compute (cumsum,
+// mask, scale, state update, epilogue).
 // Every wait is bounded; a CTA that times out records the error, drains its
 // own copies and MMAs, frees its TMEM and exits.
 #include <cuda.h>

@@ -1,17 +1,21 @@
 // Fast fused chunked SSD forward on sm_100a (tcgen05 + TMEM + TMA), for the
 // common case where every chunk's decay range is moderate.
 //
-// Two kernels:
+// Three kernels:
 //
-// k_chunk_cb (one CTA per batch row, chunk, B/C group): the head-independent
+// k_seq_runs (packed sequences only): lists each sequence as a run (row,
+//   first token, length, id), so that every sequence is chunked from its own
+//   first token and the two kernels below take it as an independent problem.
+//
+// k_chunk_cb (one CTA per chunk -- of a batch row, or of a run -- and B/C group): the head-independent
 //   part of the intra-chunk "attention",
 //       W'[t][s] = C_t . B_s  if s <= t, both tokens valid and in the same
 //                             packed sequence, else 0          (bf16, 64 x 64)
 //   (the masked C B^T of the dual form, "22 · Mamba 2 — Transformers are
 //   SSMs" section 3.2), computed once and shared by all heads of the group.
 //
-// k_ssd_fwd_fast (one CTA per (batch row, head), chunks in order, the running
-//   state kept on chip).  With cs_t the in-chunk cumulative sum of dt*A (log2
+// k_ssd_fwd_fast (one CTA per (batch row, head), or per (run, head), chunks in
+//   order, the running state kept on chip).  With cs_t the in-chunk cumulative sum of dt*A (log2
 //   units) and m = cs at the chunk's midpoint, the decay between tokens s <= t
 //   factorises as exp2(cs_t - cs_s) = u_t v_s / dt_s with
 //       u_t = exp2(cs_t - m),   v_s = exp2(m - cs_s) dt_s,
@@ -35,7 +39,8 @@
 // factor vectors two chunks ahead and issues the TMA loads (x in a 3-deep
 // ring, scaled in place; W' and C 2-deep; B one tile; each refilled as soon as
 // its last reader is done);
-// warp 1 issues the MMAs (one thread); warps 2-9 scale x, update the state and
+// warp 1 issues the MMAs (the whole warp forms the descriptors, one elected
+// lane issues); warps 2-9 scale x, update the state and
 // write y.  Yd and S are double-buffered in TMEM so chunk c's MMAs
 // overlap chunk c-1's state update and epilogue.  Every wait is bounded; a
 // CTA that times out records the error, drains its copies and MMAs, frees its

@@ -28,7 +28,7 @@
 // the barriers it needs:
 //   warp 0      TMA loads (one thread): x 3 chunks ahead (L2 prefetch 6 ahead),
 //               W', B, C 2 ahead
-//   warp 1      MMA issue (one thread)
+//   warp 1      MMA issue (descriptors formed by the warp, one elected lane issues)
 //   warp 2      dt scan of both heads: u, v, D / v and the chunk scalars; it
 //               also loads dt by TMA into an 8-deep ring of its own
 //   warp 3      y stores (one thread); frees an x slot once its tile is read out
