@@ -11,6 +11,8 @@ Contents:
                               ``ssd_oracle.c``); this is the oracle proper.
   * ``matrix_form.ssd_matrix_form`` -- y = M x with the semiseparable matrix M
                               written out (tiny inputs; a pin for the oracle).
+  * ``block.conv1d_silu``, ``block.gate`` -- the Mamba-2 block pieces around the SSD
+                              (causal depthwise conv1d + SiLU; the SiLU gate).
   * ``chunked.ssd_chunked``  -- the four chunked steps written out literally in
                               fp64 numpy (a pin for the decomposition the CUDA
                               kernels use).

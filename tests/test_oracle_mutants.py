@@ -66,3 +66,45 @@ def test_mutant_is_caught(name):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"no pin rejects the planted mistake {name}"
+
+
+# ----------------------------------------------------------------------------- block pieces
+# Planted mistakes in a copy of oracle/block.py (conv1d + SiLU, gate): each must
+# fail some pin of tests/test_block_oracle_pins.py.
+BLOCK_MUTANTS = {
+    "tap_direction_reversed": ("pre += w[None, None, :, k] * src", "pre += w[None, None, :, K - 1 - k] * src"),
+    "taps_shifted_by_one": ("shift = K - 1 - k", "shift = K - k"),
+    "bias_dropped": ("pre = np.zeros((b, L, C)) if bias is None", "pre = np.zeros((b, L, C)) if True"),
+    "packing_cut_ignored": ("            src *= same[:, :, None]\n", ""),
+    "silu_sign_flipped": ("return v / (1.0 + np.exp(-v))", "return v / (1.0 + np.exp(v))"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BLOCK_MUTANTS))
+def test_block_mutant_fails_a_pin(name, monkeypatch, tmp_path):
+    import importlib.util
+    import sys
+
+    import oracle.block
+    import test_block_oracle_pins as bpins
+    src = open(oracle.block.__file__).read()
+    old, new = BLOCK_MUTANTS[name]
+    assert src.count(old) == 1, name
+    path = tmp_path / "block_mutant.py"
+    path.write_text(src.replace(old, new))
+    spec = importlib.util.spec_from_file_location("oracle.block_mutant", path)
+    mod = importlib.util.module_from_spec(spec)
+    mod.__package__ = "oracle"
+    spec.loader.exec_module(mod)
+    monkeypatch.setattr(bpins, "block", mod)
+    pins_run = [lambda: bpins.test_silu_is_x_times_the_logistic(),
+                *[functools.partial(bpins.test_each_channel_is_a_numpy_convolution, K) for K in (1, 2, 4)],
+                bpins.test_an_impulse_gives_back_the_filter, bpins.test_the_first_token_sees_only_itself,
+                bpins.test_packed_sequences_equal_their_parts_run_alone, bpins.test_gate]
+    failed = 0
+    for pin in pins_run:
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed > 0, f"no pin caught {name}"
