@@ -360,6 +360,101 @@ def run_step(args, dist, dev, world, rank):
     return 0
 
 
+# ----------------------------------------------------------------------------- block piece: conv1d + SiLU
+
+def run_conv(args, dist, dev, world, rank):
+    """``--op conv``: the Mamba-2 block's causal depthwise conv1d + SiLU on c1's
+    xBC tensor (b 8, L 2048, channels H P + 2 G N = 5376, width 4, bf16).
+    Bound by HBM: u read and out written once."""
+    import mamba_ssd_chunked_03_b200 as ssd
+    b, L, C, K = 8, 2048, 80 * 64 + 2 * 1 * 128, 4
+    gen = torch.Generator().manual_seed(13 + rank)
+    u_h = torch.randn(b, L, C, generator=gen).to(torch.bfloat16)
+    w_h = torch.randn(C, K, generator=gen) * 0.5
+    bias_h = torch.randn(C, generator=gen) * 0.1
+    u, w, bias = u_h.to(dev), w_h.to(dev), bias_h.to(dev)
+    out = torch.empty_like(u)
+
+    def step():
+        ssd.conv1d_silu(u, w, bias, out=out)
+
+    K_ = args.steps
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_uuid(dev))
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K_):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clock_stats = clocks.stop()
+    ms_step = max_over_ranks(e0.elapsed_time(e1), dist, dev) / K_
+
+    pinned, out_host = u_h.pin_memory(), torch.empty_like(u_h).pin_memory()
+
+    def e2e_step():
+        u.copy_(pinned, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    E = max(3, min(K_, 50))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(E):
+        e2e_step()
+    a1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev) / E
+
+    nbytes = 2 * b * L * C * 2 + C * K * 4 + C * 4
+    peaks = load_peaks()
+    achieved = nbytes / (ms_step / 1e3) / 1e9
+    tokens = b * L
+    line = {
+        "metric": "Mamba-2 block causal conv1d + SiLU tokens/s", "value": tokens * world / (ms_step / 1e3),
+        "unit": "tokens/s", "n_gpus": world, "steps": K_, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"conv1d+SiLU: b{b} L{L} channels {C} (c1 xBC) width {K} bf16",
+                   "l2": f"no flush: u + out {nbytes / 1e6:.0f} MB > 126 MB L2",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                     "frac_datasheet": achieved / DATASHEET_HBM_GBS, "kernel": "k_conv1d_silu",
+                     "kernel_ms": ms_step, "traffic": None, "algorithmic_bytes": nbytes},
+        "e2e": {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": b * L * C * 2, "d2h_bytes_per_step": b * L * C * 2, "steps": E},
+        "gpu_launches": K_,
+        "clocks": clock_stats,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import block  # test infrastructure: only this CPU-baseline leg uses it here
+        reps, t = 0, time.perf_counter()
+        while True:
+            block.conv1d_silu(u_h[:1], w_h, bias_h)  # one batch row per repetition
+            reps += 1
+            el = time.perf_counter() - t
+            if el >= min(args.cpu_seconds, 10.0):
+                break
+        line["cpu_baseline"] = {"value": reps * L / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{reps} batch rows of {L} tokens (numpy, one process), {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def main():
@@ -372,8 +467,9 @@ def main():
     ap.add_argument("--generic", action="store_true", help="force the generic CUDA-core kernels")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--op", default="fwd", choices=["fwd", "step"],
-                    help="fwd: the chunked forward (default); step: the recurrent decode step")
+    ap.add_argument("--op", default="fwd", choices=["fwd", "step", "conv"],
+                    help="fwd: the chunked forward (default); step: the recurrent decode step; "
+                         "conv: the block's causal conv1d + SiLU")
     ap.add_argument("--step-batch", type=int, default=256, help="rows of the decode step (--op step)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -399,6 +495,8 @@ def main():
     torch.cuda.set_device(dev)
     if args.op == "step":
         return run_step(args, dist, dev, world, rank)
+    if args.op == "conv":
+        return run_conv(args, dist, dev, world, rank)
 
     host = si.make_inputs(shape, seed=shape.seed + rank)
     num_seqs = host.get("num_seqs")

@@ -114,6 +114,11 @@ typedef struct {
                                      kernel, or all generic kernels together), so a
                                      caller can time it without a profiler.  Owned by
                                      the caller; both or neither.                    */
+  const void* z;                  /* (b,L,H,P) dtype gate, or NULL: y is returned as
+                                     y * SiLU(z) (SiLU(v) = v / (1 + e^-v)), the
+                                     Mamba-2 block's gate path multiplied in where y
+                                     is formed ("SSM 家族全景图（下）：Mamba-2 与
+                                     Jamba", section 5).                             */
 } ssd_fwd_args;
 
 /* Bytes of device workspace ssd_fwd needs for these sizes and options (only
@@ -228,6 +233,31 @@ SSD_API ssd_status ssd_total_decay(const float* dt, const float* A, float* out, 
 SSD_API ssd_status ssd_state_fold(const float* states, const float* decays, const float* initial_states,
                                   float* out, int64_t rank, int64_t batch, int64_t nheads, int64_t headdim,
                                   int64_t dstate, void* stream);
+
+/* The Mamba-2 block's causal depthwise convolution followed by SiLU, the
+ * piece before the SSD on its main path ("SSM 家族全景图（下）：Mamba-2 与
+ * Jamba", section 5, the block's data flow):
+ *
+ *   out[b,t,c] = SiLU(bias_c + sum_{k<K} weight[c,k] u[b, t-(K-1)+k, c])
+ *
+ * with SiLU(v) = v / (1 + e^-v), zeros before the first token and, with
+ * seq_idx, no tap reaching into an earlier packed sequence.  K = width,
+ * 1..4, and channels a multiple of 8 (bf16) or 4 (fp32) (else
+ * SSD_ERR_UNSUPPORTED); u and out 16-byte aligned and not overlapping.
+ * Asynchronous on `stream`; device pointers owned by the caller; nothing is
+ * enqueued when the arguments are rejected. */
+typedef struct {
+  int64_t batch, seqlen, channels, width;
+  ssd_dtype dtype;         /* of u and out */
+  const void* u;           /* (b,L,channels) dtype                          */
+  const float* weight;     /* (channels,width) fp32, tap k multiplies token
+                              t-(width-1)+k                                */
+  const float* bias;       /* (channels) fp32, or NULL for 0                */
+  const int32_t* seq_idx;  /* (b,L) int32 packed-sequence ids, or NULL      */
+  void* out;               /* (b,L,channels) dtype                          */
+} ssd_conv_args;
+
+SSD_API ssd_status ssd_conv1d_silu(const ssd_conv_args* args, void* stream);
 
 /* Static, human-readable text for a status code. */
 SSD_API const char* ssd_status_string(ssd_status status);

@@ -19,7 +19,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["fwd", "step", "StepArgs", "total_decay", "state_fold", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
+__all__ = ["fwd", "step", "StepArgs", "total_decay", "state_fold", "conv1d_silu", "ConvArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
            "SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED", "SSD_ERR_WORKSPACE", "SSD_ERR_CUDA",
            "SSD_F32", "SSD_BF16", "SSD_FLAG_GENERIC"]
 
@@ -43,6 +43,7 @@ class Args(ctypes.Structure):
         ("y", ctypes.c_void_p), ("final_states", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("timing_events", ctypes.c_void_p * 2),
+        ("z", ctypes.c_void_p),
     ]
 
 
@@ -53,6 +54,15 @@ class StepArgs(ctypes.Structure):
         ("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("A", ctypes.c_void_p),
         ("B", ctypes.c_void_p), ("C", ctypes.c_void_p), ("D", ctypes.c_void_p),
         ("state", ctypes.c_void_p), ("y", ctypes.c_void_p),
+    ]
+
+
+class ConvArgs(ctypes.Structure):
+    """Mirror of ``ssd_conv_args``."""
+    _fields_ = [(n, ctypes.c_int64) for n in ("batch", "seqlen", "channels", "width")] + [
+        ("dtype", ctypes.c_int),
+        ("u", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+        ("seq_idx", ctypes.c_void_p), ("out", ctypes.c_void_p),
     ]
 
 
@@ -76,6 +86,8 @@ def _load() -> ctypes.CDLL:
     L.ssd_fwd_main_kernel.restype = ctypes.c_char_p
     L.ssd_step.argtypes = [ctypes.POINTER(StepArgs), ctypes.c_void_p]
     L.ssd_step.restype = ctypes.c_int
+    L.ssd_conv1d_silu.argtypes = [ctypes.POINTER(ConvArgs), ctypes.c_void_p]
+    L.ssd_conv1d_silu.restype = ctypes.c_int
     L.ssd_total_decay.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int64] * 3 + [
         ctypes.c_void_p]
     L.ssd_total_decay.restype = ctypes.c_int
@@ -102,7 +114,7 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 def make_args(x, dt, A, B, C, D=None, chunk_size: int = 64, initial_states=None, seq_idx=None,
               num_seqs: Optional[int] = None, y=None, final_states=None, workspace=None,
-              workspace_bytes: int = 0, generic: bool = False) -> Args:
+              workspace_bytes: int = 0, generic: bool = False, z=None) -> Args:
     """Fill an ``ssd_fwd_args`` from tensors (shapes read from x and B)."""
     b, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
@@ -115,6 +127,7 @@ def make_args(x, dt, A, B, C, D=None, chunk_size: int = 64, initial_states=None,
     a.num_seqs = int(num_seqs) if seq_idx is not None else 0
     a.y, a.final_states = _ptr(y), _ptr(final_states)
     a.workspace, a.workspace_bytes = _ptr(workspace), int(workspace_bytes)
+    a.z = _ptr(z)
     return a
 
 
@@ -201,7 +214,7 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
         num_seqs: Optional[int] = None, return_final_states: bool = True,
         y: Optional[torch.Tensor] = None, final_states: Optional[torch.Tensor] = None,
         workspace: Optional[torch.Tensor] = None, generic: bool = False,
-        timing_events: Optional[tuple] = None):
+        timing_events: Optional[tuple] = None, z: Optional[torch.Tensor] = None):
     """SSD forward.  Returns (y, final_states or None).
 
     x (b,L,H,P) fp32|bf16, dt (b,L,H) fp32, A (H) fp32, B/C (b,L,G,N) x.dtype,
@@ -211,8 +224,13 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     ``y``, ``final_states`` and ``workspace`` may be passed preallocated.
     ``timing_events``: optional (start, end) torch.cuda.Event pair recorded on
     the current stream around the call's main kernel.
+    ``z`` (b,L,H,P) x.dtype or None: the block's gate, y is returned as
+    y * SiLU(z).
     """
     _check(x, dt, A, B, C, D, initial_states, seq_idx)
+    if z is not None and (z.dtype != x.dtype or tuple(z.shape) != tuple(x.shape) or z.device != x.device
+                          or not z.is_contiguous()):
+        raise ValueError("z must be a contiguous tensor like x")
     b, L, H, P = x.shape
     N = B.shape[3]
     if seq_idx is not None and num_seqs is None:
@@ -225,7 +243,7 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     if not return_final_states:
         final_states = None
     a = make_args(x, dt, A, B, C, D, chunk_size, initial_states, seq_idx, num_seqs, y, final_states,
-                  generic=generic)
+                  generic=generic, z=z)
     need = int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
     if need > 0:
         if workspace is None or workspace.numel() * workspace.element_size() < need:
@@ -315,6 +333,34 @@ def state_fold(states: Optional[torch.Tensor], decays: Optional[torch.Tensor],
     out = torch.empty(b, H, P, N, device=dev, dtype=torch.float32)
     st = lib.ssd_state_fold(_ptr(states), _ptr(decays), _ptr(initial_states), out.data_ptr(), int(rank), b, H, P, N,
                             _stream(out))
+    if st != SSD_OK:
+        raise SSDError(st)
+    return out
+
+
+def conv1d_silu(u: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                seq_idx: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """``ssd_conv1d_silu``: SiLU of the causal depthwise convolution of u
+    (b,L,C) with weight (C,K) fp32 and bias (C) fp32 or None; seq_idx (b,L)
+    int32 keeps taps inside each packed sequence.  Returns (b,L,C) in u's dtype."""
+    if u.dim() != 3 or weight.dim() != 2 or weight.shape[0] != u.shape[2]:
+        raise ValueError("expected u (b,L,C) and weight (C,K)")
+    if u.dtype not in (torch.float32, torch.bfloat16) or weight.dtype != torch.float32 \
+            or (bias is not None and (bias.dtype != torch.float32 or tuple(bias.shape) != (u.shape[2],))):
+        raise TypeError("u float32 or bfloat16; weight and bias float32 (bias of shape (C,))")
+    if seq_idx is not None and (seq_idx.dtype != torch.int32 or tuple(seq_idx.shape) != tuple(u.shape[:2])):
+        raise ValueError("seq_idx must be int32 (b,L)")
+    for name, t in (("u", u), ("weight", weight), ("bias", bias), ("seq_idx", seq_idx)):
+        if t is not None and (t.device != u.device or u.device.type != "cuda" or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor on {u.device}")
+    if out is None:
+        out = torch.empty_like(u)
+    a = ConvArgs()
+    a.batch, a.seqlen, a.channels = u.shape
+    a.width = weight.shape[1]
+    a.dtype = SSD_BF16 if u.dtype == torch.bfloat16 else SSD_F32
+    a.u, a.weight, a.bias, a.seq_idx, a.out = _ptr(u), _ptr(weight), _ptr(bias), _ptr(seq_idx), _ptr(out)
+    st = lib.ssd_conv1d_silu(ctypes.byref(a), _stream(u))
     if st != SSD_OK:
         raise SSDError(st)
     return out

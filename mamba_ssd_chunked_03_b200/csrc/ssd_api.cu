@@ -58,6 +58,7 @@ Problem resolve(const ssd_fwd_args* a) {
   p.D = a->D;
   p.h0 = a->initial_states;
   p.seq = a->seq_idx;
+  p.z = a->z;
   p.num_seqs = a->seq_idx ? a->num_seqs : 0;
   p.y = a->y;
   p.final_states = a->final_states;

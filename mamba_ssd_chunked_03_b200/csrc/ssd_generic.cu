@@ -318,7 +318,12 @@ __global__ void __launch_bounds__(kThreads) k_chunk_scan(Problem pr, const float
       const int p = pp0 + tx * 4 + j;
       if (p >= pr.P) continue;
       const int64_t off = ((b * pr.L + t0 + t) * pr.H + h) * pr.P + p;
-      y[off] = from_f<T>(fmaf(d, to_f(x[off]), acc[i][j]));
+      float v = fmaf(d, to_f(x[off]), acc[i][j]);
+      if (pr.z) {  // the gate: y * SiLU(z)
+        const float zv = to_f(static_cast<const T*>(pr.z)[off]);
+        v *= zv / (1.f + expf(-zv));
+      }
+      y[off] = from_f<T>(v);
     }
   }
 }

@@ -24,6 +24,7 @@ struct Problem {
   int64_t num_seqs;
   void* y;
   float* final_states;
+  const void* z;  // gate: y * SiLU(z), or null
 };
 
 constexpr size_t kWsAlign = 256;

@@ -156,6 +156,7 @@ struct TcArgs {
   const int* failed_count;  // units to process, listed by the fast kernel
   const int* failed_list;
   int64_t num_seqs;         // packed sequences: final states of ids outside [0, num_seqs) are not written
+  const __nv_bfloat16* z;   // gate: y * SiLU(z), or null
   int* err;
 };
 
@@ -599,12 +600,21 @@ __global__ void __launch_bounds__(192, Cfg<NS>::kMinBlocks)
         const int p0 = 32 * (lane >> 4);
         if (t < nvalid) {
           const float sc = (s.seqs[t] == seq_prev) ? exp2f(s.cs2[t]) : 0.f;
+          const int64_t yoff = ((rowbase + t0 + t) * a.H + h) * 64 + p0;
           uint32_t packed[16];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2)
-            packed[j >> 1] = pack_bf16x2(fmaf(sc, __uint_as_float(ro[j]), __uint_as_float(rd[j])),
-                                         fmaf(sc, __uint_as_float(ro[j + 1]), __uint_as_float(rd[j + 1])));
-          uint4* dst = reinterpret_cast<uint4*>(a.y + ((rowbase + t0 + t) * a.H + h) * 64 + p0);
+          for (int j = 0; j < 32; j += 2) {
+            float v0 = fmaf(sc, __uint_as_float(ro[j]), __uint_as_float(rd[j]));
+            float v1 = fmaf(sc, __uint_as_float(ro[j + 1]), __uint_as_float(rd[j + 1]));
+            if (a.z) {  // the gate: y * SiLU(z)
+              float z0, z1;
+              unpack_bf16x2(reinterpret_cast<const uint32_t*>(a.z + yoff)[j >> 1], z0, z1);
+              v0 *= silu(z0);
+              v1 *= silu(z1);
+            }
+            packed[j >> 1] = pack_bf16x2(v0, v1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(a.y + yoff);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
@@ -658,6 +668,7 @@ cudaError_t launch(const Problem& p, const TcWorkspace& w, cudaStream_t st) {
   a.failed_count = w.failed_count;
   a.failed_list = w.failed_list;
   a.num_seqs = p.seq ? p.num_seqs : 0;
+  a.z = static_cast<const __nv_bfloat16*>(p.z);
   a.err = w.err;
   cudaError_t e = cudaFuncSetAttribute(k_ssd_fwd_tc<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Cfg<NS>::kSmemBytes);
@@ -731,6 +742,7 @@ bool tc_supported(const Problem& p, uint32_t flags) {
   if (p.dtype != SSD_BF16) return false;
   if (p.P != 64 || (p.Q != 64 && p.Q != 128 && p.Q != 256)) return false;
   if (p.N != 64 && p.N != 128 && p.N != 256) return false;  // 64 runs zero-padded as 128
+  if (p.z && reinterpret_cast<uintptr_t>(p.z) % 16 != 0) return false;  // the gate is read in 16-byte vectors
   // TMA coordinates are 32-bit (W' rows: packed sequences add one partial chunk per run)
   const Problem t = tc_tiles(p);
   const int64_t chunks = t.b * t.nc + (p.seq ? p.num_seqs : 0);
@@ -743,7 +755,7 @@ size_t tc_workspace_bytes(const Problem& p) { return tc_workspace_need(tc_tiles(
 int tc_launch_count(const Problem& p) {
   if (p.seq) return 4;  // run list, C B^T per run chunk, fused per (run, head), exact
   const Problem t = tc_tiles(p);
-  return tc_kernel_n(t) == 128 && tc_pair_supported(t) && tc_pair_split(t) ? 4 : 3;
+  return tc_kernel_n(t) == 128 && !t.z && tc_pair_supported(t) && tc_pair_split(t) ? 4 : 3;
 }
 
 cudaError_t tc_forward(const Problem& pq, void* ws, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {

@@ -69,6 +69,7 @@ struct FastArgs {
   int varlen;
   RunList runs;
   int* unit_bad;
+  const __nv_bfloat16* z;  // gate (b, L, H, 64): y * SiLU(z), or null
 };
 
 // persistent grid of the two-head kernel, at most; per-CTA hand-over size
@@ -80,6 +81,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
+
+// the block's gate nonlinearity, SiLU(v) = v / (1 + e^-v)
+__device__ __forceinline__ float silu(float v) { return v / (1.f + expf(-v)); }
 
 __device__ __forceinline__ void unpack_bf16x2(uint32_t u, float& lo, float& hi) {
   __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);

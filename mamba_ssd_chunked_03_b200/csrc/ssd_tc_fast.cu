@@ -711,11 +711,28 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
         const int p0 = 16 * hq + 32 * (lane >> 4);
         if (t < nvp) {
           const float ut = s.u[slp][t];
+          const int64_t yoff = ((rowbase + t0p + t) * a.H + h) * 64 + p0;
+          float gz[16];  // the gate: SiLU(z), or 1
+          if (a.z) {
+            const uint4* zp = reinterpret_cast<const uint4*>(a.z + yoff);
+            const uint4 z0 = zp[0], z1 = zp[1];
+            const uint32_t zw[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              unpack_bf16x2(zw[j], gz[2 * j], gz[2 * j + 1]);
+              gz[2 * j] = silu(gz[2 * j]);
+              gz[2 * j + 1] = silu(gz[2 * j + 1]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) gz[j] = 1.f;
+          }
           uint32_t packed[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            packed[j] = pack_bf16x2(ut * __uint_as_float(r[2 * j]), ut * __uint_as_float(r[2 * j + 1]));
-          uint4* dst = reinterpret_cast<uint4*>(a.y + ((rowbase + t0p + t) * a.H + h) * 64 + p0);
+            packed[j] = pack_bf16x2(ut * __uint_as_float(r[2 * j]) * gz[2 * j],
+                                    ut * __uint_as_float(r[2 * j + 1]) * gz[2 * j + 1]);
+          uint4* dst = reinterpret_cast<uint4*>(a.y + yoff);
           dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         }
@@ -809,9 +826,11 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
   fa.flags = w.flags;
   fa.pair_bad = w.pair_bad;
   fa.varlen = varlen;
+  fa.z = static_cast<const __nv_bfloat16*>(p.z);
   fa.runs = w.runs;
   fa.unit_bad = w.unit_bad;
-  if (!varlen && NS == 128 && tc_pair_supported(p)) {
+  // (a gated call takes the single-head kernel, whose epilogue applies the gate)
+  if (!varlen && !p.z && NS == 128 && tc_pair_supported(p)) {
     CUtensorMap ty, tdt;
     if (!make_map_3d(&ty, p.y, p.H * p.P, p.L, p.b) || !make_map_dt(&tdt, p.dt, p.H, p.L, p.b))
       return cudaErrorInvalidValue;
@@ -834,7 +853,7 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
 
 const char* tc_main_kernel(const Problem& p) {
   if (p.seq) return "k_ssd_fwd_fast";  // per (run, head)
-  return tc_kernel_n(p) == 128 && tc_pair_supported(tc_tiles(p)) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
+  return tc_kernel_n(p) == 128 && !p.z && tc_pair_supported(tc_tiles(p)) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
 }
 
 cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0,

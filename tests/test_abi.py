@@ -115,8 +115,8 @@ def test_kernel_path_query():
 
 
 def test_struct_layout_matches_header():
-    # 7 int64 sizes, dtype + flags, 8 pointers, num_seqs, 2 outputs, workspace + bytes
-    assert ctypes.sizeof(ssd.Args) == 7 * 8 + 4 + 4 + 8 * 8 + 8 + 2 * 8 + 8 + 8 + 2 * 8
+    # 7 int64 sizes, dtype + flags, 8 pointers, num_seqs, 2 outputs, workspace + bytes, events, z
+    assert ctypes.sizeof(ssd.Args) == 7 * 8 + 4 + 4 + 8 * 8 + 8 + 2 * 8 + 8 + 8 + 2 * 8 + 8
     assert ssd.Args.x.offset == 64 and ssd.Args.num_seqs.offset == 128
     assert ssd.Args.timing_events.offset == 168
 
@@ -193,3 +193,33 @@ def test_step_rejects_bad_arguments(kw, status):
 
 def test_step_null_args_pointer():
     assert ssd.lib.ssd_step(None, None) == ssd.SSD_ERR_INVALID_ARG
+
+
+def _conv_args(**kw):
+    a = ssd.ConvArgs()
+    a.batch, a.seqlen, a.channels, a.width = 2, 64, 64, 4
+    a.dtype = ssd.SSD_BF16
+    for i, n in enumerate(("u", "weight", "bias", "seq_idx", "out")):  # never dereferenced: all rejected
+        setattr(a, n, 4096 * (i + 1))
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({"batch": 0}, ssd.SSD_ERR_INVALID_ARG),
+    ({"width": 0}, ssd.SSD_ERR_INVALID_ARG),
+    ({"u": None}, ssd.SSD_ERR_INVALID_ARG),
+    ({"out": 4096 + 8}, ssd.SSD_ERR_INVALID_ARG),
+    ({"width": 5}, ssd.SSD_ERR_UNSUPPORTED),
+    ({"channels": 60}, ssd.SSD_ERR_UNSUPPORTED),   # not a multiple of 8 bf16
+])
+def test_conv_rejects_bad_arguments(kw, status):
+    assert ssd.lib.ssd_conv1d_silu(ctypes.byref(_conv_args(**kw)), None) == status
+
+
+def test_conv_struct_layout_matches_the_compiled_header():
+    names = [f[0] for f in ssd.ConvArgs._fields_]
+    got = _c_layout(names, "ssd_conv_args")
+    assert got[:-1] == [getattr(ssd.ConvArgs, n).offset for n in names]
+    assert got[-1] == ctypes.sizeof(ssd.ConvArgs)
