@@ -71,11 +71,7 @@ struct Vec<float> {
   }
 };
 
-// SiLU with the fast exponential and division intrinsics (a few ulp; the
-// output is rounded to bf16 or compared at 1e-5): the kernel's cost is
-// instructions per element, and the IEEE forms would triple them.  For very
-// negative v the quotient underflows to 0, the limit of SiLU there.
-__device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.f + __expf(-v)); }
+__device__ __forceinline__ float silu(float v) { return v / (1.f + expf(-v)); }
 
 // grid: (channel vectors / kConvThreads, token strips, batch rows)
 template <typename T, int K>
@@ -85,10 +81,9 @@ __global__ void __launch_bounds__(kConvThreads) k_conv1d_silu(const ConvArgs a) 
   if (c0 >= a.C) return;
   const int64_t b = blockIdx.z;
   const int64_t t0 = (int64_t)blockIdx.y * kStrip;
-  // u and out do not overlap (a precondition), so loads may run ahead of stores
-  const T* __restrict__ u = static_cast<const T*>(a.u) + b * a.L * a.C + c0;
-  T* __restrict__ out = static_cast<T*>(a.out) + b * a.L * a.C + c0;
-  const int32_t* __restrict__ seq = a.seq ? a.seq + b * a.L : nullptr;
+  const T* u = static_cast<const T*>(a.u) + b * a.L * a.C + c0;
+  T* out = static_cast<T*>(a.out) + b * a.L * a.C + c0;
+  const int32_t* seq = a.seq ? a.seq + b * a.L : nullptr;
   float w[V][K], bias[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) {
@@ -113,7 +108,6 @@ __global__ void __launch_bounds__(kConvThreads) k_conv1d_silu(const ConvArgs a) 
     }
   }
   const int64_t t_end = t0 + kStrip < a.L ? t0 + kStrip : a.L;
-#pragma unroll 2
   for (int64_t t = t0; t < t_end; ++t) {
     float cur[V];
     Vec<T>::load(u + t * a.C, cur);
