@@ -13,6 +13,8 @@ Contents:
                               written out (tiny inputs; a pin for the oracle).
   * ``block.conv1d_silu``, ``block.gate`` -- the Mamba-2 block pieces around the SSD
                               (causal depthwise conv1d + SiLU; the SiLU gate).
+  * ``backward.ssd_bwd``     -- the backward pass: the adjoint of the recurrence
+                              (derived; the pages give no formulas), fp64.
   * ``chunked.ssd_chunked``  -- the four chunked steps written out literally in
                               fp64 numpy (a pin for the decomposition the CUDA
                               kernels use).

@@ -108,3 +108,47 @@ def test_block_mutant_fails_a_pin(name, monkeypatch, tmp_path):
         except AssertionError:
             failed += 1
     assert failed > 0, f"no pin caught {name}"
+
+
+# ----------------------------------------------------------------------------- backward
+# Planted mistakes in a copy of oracle/backward.py: each must fail some pin of
+# tests/test_backward_oracle_pins.py.
+BACKWARD_MUTANTS = {
+    "carry_dropped": ("Gt = a[:, t + 1, :, None, None] * Gt", "Gt = 0.0 * Gt"),
+    "dh0_not_decayed": ("dh0 = None if h0 is None else a[:, 0, :, None, None] * Gt",
+                        "dh0 = None if h0 is None else Gt"),
+    "ddt_decay_term_dropped": ("ddt[:, t] = g_in + A[None, :] * a[:, t] * g_dec", "ddt[:, t] = g_in"),
+    "dA_without_dt": ("dA += np.sum(dt[:, t] * a[:, t] * g_dec, axis=0)", "dA += np.sum(a[:, t] * g_dec, axis=0)"),
+    "dB_not_summed_over_group": ("dB[:, :, grp[h_]] += dBh[:, :, h_]", "dB[:, :, grp[h_]] = dBh[:, :, h_]"),
+    "reset_ignored": ("a = np.where(reset[:, :, None], 0.0, a)", "a = a"),
+    "skip_term_dropped_from_dx": ("dx += Dv[None, None, :, None] * dy", "dx += 0.0 * dy"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BACKWARD_MUTANTS))
+def test_backward_mutant_fails_a_pin(name, monkeypatch, tmp_path):
+    import importlib.util
+
+    import oracle.backward
+    import test_backward_oracle_pins as bw
+    src = open(oracle.backward.__file__).read()
+    old, new = BACKWARD_MUTANTS[name]
+    assert src.count(old) == 1, name
+    path = tmp_path / "backward_mutant.py"
+    path.write_text(src.replace(old, new))
+    spec = importlib.util.spec_from_file_location("oracle.backward_mutant", path)
+    mod = importlib.util.module_from_spec(spec)
+    mod.__package__ = "oracle"
+    spec.loader.exec_module(mod)
+    monkeypatch.setattr(bw, "backward", mod)
+    failed = 0
+    for case in bw.CASES:
+        try:
+            bw.test_backward_matches_autograd(case)
+        except AssertionError:
+            failed += 1
+    try:
+        bw.test_backward_matches_finite_differences_of_the_forward_oracle()
+    except AssertionError:
+        failed += 1
+    assert failed > 0, f"no pin caught {name}"
