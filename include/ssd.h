@@ -242,7 +242,7 @@ SSD_API ssd_status ssd_state_fold(const float* states, const float* decays, cons
  *
  * with SiLU(v) = v / (1 + e^-v), zeros before the first token and, with
  * seq_idx, no tap reaching into an earlier packed sequence.  K = width,
- * 1..4, and channels a multiple of 8 (bf16) or 4 (fp32) (else
+ * 1..4, and channels a multiple of 4 (else
  * SSD_ERR_UNSUPPORTED); u and out 16-byte aligned and not overlapping.
  * Asynchronous on `stream`; device pointers owned by the caller; nothing is
  * enqueued when the arguments are rejected. */

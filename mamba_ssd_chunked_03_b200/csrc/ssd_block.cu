@@ -7,8 +7,8 @@
 // reaches into an earlier sequence (the same cut as the SSD's decay).
 //
 // Bound by HBM: u read once (plus a K-1 token halo per strip, from L2) and
-// out written once.  A thread owns one 16-byte vector of channels (8 bf16 or
-// 4 fp32) over a strip of kStrip tokens; its filter taps, bias and the K-1
+// out written once.  A thread owns one vector of 4 channels (8 bytes of bf16,
+// 16 of fp32) over a strip of kStrip tokens; its filter taps, bias and the K-1
 // previous inputs (with their sequence ids) stay in registers while it walks
 // the strip.  Consecutive threads take consecutive channel vectors, so every
 // load and store of a warp is contiguous.
@@ -38,25 +38,21 @@ template <typename T>
 struct Vec;
 template <>
 struct Vec<__nv_bfloat16> {
-  static constexpr int n = 8;
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 q = *reinterpret_cast<const uint4*>(p);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
-      v[2 * i] = __low2float(h);
-      v[2 * i + 1] = __high2float(h);
-    }
+  static constexpr int n = 4;  // 8-byte vectors: half the registers of 16-byte ones, twice the resident warps
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[4]) {
+    const uint2 q = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&q.x);
+    const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162*>(&q.y);
+    v[0] = __low2float(h0);
+    v[1] = __high2float(h0);
+    v[2] = __low2float(h1);
+    v[3] = __high2float(h1);
   }
-  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[8]) {
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-      w[i] = *reinterpret_cast<const uint32_t*>(&h);
-    }
-    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[4]) {
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
+    const __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
+    *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<const uint32_t*>(&h0),
+                                              *reinterpret_cast<const uint32_t*>(&h1));
   }
 };
 template <>
@@ -172,8 +168,7 @@ extern "C" SSD_API ssd_status ssd_conv1d_silu(const ssd_conv_args* a, void* stre
   if (a->batch <= 0 || a->seqlen <= 0 || a->channels <= 0 || a->width <= 0) return SSD_ERR_INVALID_ARG;
   if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
   if (!aligned16(a->u) || !aligned16(a->out)) return SSD_ERR_INVALID_ARG;
-  const int V = a->dtype == SSD_BF16 ? 8 : 4;
-  if (a->width > kMaxWidth || a->channels % V != 0) return SSD_ERR_UNSUPPORTED;
+  if (a->width > kMaxWidth || a->channels % 4 != 0) return SSD_ERR_UNSUPPORTED;
   if (a->batch > 65535 || (a->seqlen + kStrip - 1) / kStrip > 65535) return SSD_ERR_UNSUPPORTED;
   const cudaError_t e = a->dtype == SSD_BF16 ? launch_conv<__nv_bfloat16>(a, static_cast<cudaStream_t>(stream))
                                              : launch_conv<float>(a, static_cast<cudaStream_t>(stream));

@@ -212,7 +212,7 @@ def _conv_args(**kw):
     ({"u": None}, ssd.SSD_ERR_INVALID_ARG),
     ({"out": 4096 + 8}, ssd.SSD_ERR_INVALID_ARG),
     ({"width": 5}, ssd.SSD_ERR_UNSUPPORTED),
-    ({"channels": 60}, ssd.SSD_ERR_UNSUPPORTED),   # not a multiple of 8 bf16
+    ({"channels": 62}, ssd.SSD_ERR_UNSUPPORTED),   # not a multiple of 4
 ])
 def test_conv_rejects_bad_arguments(kw, status):
     assert ssd.lib.ssd_conv1d_silu(ctypes.byref(_conv_args(**kw)), None) == status
