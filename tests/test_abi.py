@@ -223,3 +223,32 @@ def test_conv_struct_layout_matches_the_compiled_header():
     got = _c_layout(names, "ssd_conv_args")
     assert got[:-1] == [getattr(ssd.ConvArgs, n).offset for n in names]
     assert got[-1] == ctypes.sizeof(ssd.ConvArgs)
+
+
+def test_packed_dispatch_queries():
+    """Packed sequences take the per-sequence fast path: run list, C B^T per
+    run chunk, the single-head kernel per (run, head), the exact kernel."""
+    a = base_args(seq_idx=1 << 21, num_seqs=8)
+    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"tcgen05"
+    assert ssd.lib.ssd_fwd_main_kernel(ctypes.byref(a)) == b"k_ssd_fwd_fast"
+    assert ssd.lib.ssd_fwd_launch_count(ctypes.byref(a)) == 4
+
+
+def test_gated_dispatch_queries():
+    """A gated call leaves the two-head kernel; an unaligned gate leaves the
+    tensor-core path (its epilogues read z in 16-byte vectors)."""
+    a = base_args(nheads=8, ngroups=1)
+    two_head = ssd.lib.ssd_fwd_main_kernel(ctypes.byref(a))
+    a.z = 1 << 22
+    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"tcgen05"
+    assert ssd.lib.ssd_fwd_main_kernel(ctypes.byref(a)) == b"k_ssd_fwd_fast"
+    assert two_head in (b"k_ssd_fwd_pair", b"k_ssd_fwd_fast")  # the pair kernel also needs dt 16-byte aligned
+    a.z = (1 << 22) + 8
+    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"generic"
+
+
+def test_workspace_grows_with_packed_sequences():
+    a = base_args()
+    plain = ssd.lib.ssd_fwd_workspace_size(ctypes.byref(a))
+    a.seq_idx, a.num_seqs = 1 << 21, 50
+    assert ssd.lib.ssd_fwd_workspace_size(ctypes.byref(a)) > plain
