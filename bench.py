@@ -212,10 +212,55 @@ def oracle_sample(d, shape, target_s: float, max_units=None):
     return tokens / el, U, el, min(threads, U)
 
 
+def run_reference_op(args):
+    """``--impl reference`` for ``--op step`` / ``--op conv``: the oracle on the
+    same workload as the GPU arm, timed on the host cores."""
+    import oracle
+    if args.op == "step":
+        b, H, P, N, G = args.step_batch, 80, 64, 128, 1
+        shape = si.SSDShape("decode", b, 1, H, P, N, G, 64, "bf16", h0_std=0.5, seed=11)
+        d = si.make_inputs(shape)
+        f = {k: oracle.as_f32(d[k]) for k in ("x", "dt", "A", "B", "C", "D", "initial_states")}
+        run = lambda: oracle.ssd_fwd(f["x"], f["dt"], f["A"], f["B"], f["C"], f["D"], f["initial_states"])
+        per_step, metric = b, "SSD decode step (one token per row), rows/s"
+        workload = f"decode step: b{b} H{H} P{P} N{N} G{G} bf16, fp32 state"
+        cores = oracle.max_threads()
+    else:
+        from oracle import block
+        b, L, C, K = 8, 2048, 80 * 64 + 2 * 1 * 128, 4
+        gen = torch.Generator().manual_seed(13)
+        u = torch.randn(1, L, C, generator=gen).to(torch.bfloat16)  # one batch row per repetition
+        w, bias = torch.randn(C, K, generator=gen) * 0.5, torch.randn(C, generator=gen) * 0.1
+        run = lambda: block.conv1d_silu(u, w, bias)
+        per_step, metric = L, "Mamba-2 block causal conv1d + SiLU tokens/s"
+        workload = f"conv1d+SiLU: one batch row of b{b} L{L} channels {C} width {K} bf16"
+        cores = 1
+    for _ in range(args.warmup):
+        run()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    el = time.perf_counter() - t
+    value = per_step * args.steps / el
+    sample = f"{args.steps} repetitions of {workload}"
+    line = {
+        "impl": "reference", "metric": metric, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args, shape):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    if args.op != "fwd":
+        return run_reference_op(args)
     import oracle
     d = si.make_inputs(shape)
     f = {k: oracle.as_f32(d[k]) for k in ("x", "dt", "A", "B", "C", "D", "initial_states")}
