@@ -69,6 +69,9 @@ typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
 /* flags */
 #define SSD_FLAG_GENERIC 1u /* use the generic (CUDA-core, fp32) kernels even where
                                the tensor-core kernels apply; for cross-checks */
+#define SSD_FLAG_CHECK_SEQ 2u /* check the seq_idx precondition first: ssd_fwd copies
+                                 seq_idx to the host (waiting for `stream`) and
+                                 returns ssd_check_seq_idx's verdict if it fails */
 
 typedef struct {
   /* sizes: b = batch, L = seqlen, H = nheads, P = headdim, N = dstate,
@@ -258,6 +261,13 @@ typedef struct {
 } ssd_conv_args;
 
 SSD_API ssd_status ssd_conv1d_silu(const ssd_conv_args* args, void* stream);
+
+/* The seq_idx precondition, on a HOST copy (b,L) int32: ids in [0, num_seqs),
+ * non-decreasing along each row, and no id in two rows.  SSD_OK, or
+ * SSD_ERR_INVALID_ARG at the first violation (or for a null pointer or a
+ * non-positive size).  Synchronous, host only; ssd_fwd runs it when
+ * SSD_FLAG_CHECK_SEQ is set. */
+SSD_API ssd_status ssd_check_seq_idx(const int32_t* seq_idx_host, int64_t batch, int64_t seqlen, int64_t num_seqs);
 
 /* Static, human-readable text for a status code. */
 SSD_API const char* ssd_status_string(ssd_status status);

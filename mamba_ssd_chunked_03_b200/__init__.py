@@ -28,6 +28,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
 SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_WORKSPACE, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(6)
 SSD_F32, SSD_BF16 = 0, 1
 SSD_FLAG_GENERIC = 1
+SSD_FLAG_CHECK_SEQ = 2
 
 
 class Args(ctypes.Structure):
@@ -93,6 +94,8 @@ def _load() -> ctypes.CDLL:
     L.ssd_total_decay.restype = ctypes.c_int
     L.ssd_state_fold.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 5 + [ctypes.c_void_p]
     L.ssd_state_fold.restype = ctypes.c_int
+    L.ssd_check_seq_idx.argtypes = [ctypes.c_void_p] + [ctypes.c_int64] * 3
+    L.ssd_check_seq_idx.restype = ctypes.c_int
     L.ssd_status_string.argtypes = [ctypes.c_int]
     L.ssd_status_string.restype = ctypes.c_char_p
     L.ssd_version.restype = ctypes.c_int
@@ -214,7 +217,7 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
         num_seqs: Optional[int] = None, return_final_states: bool = True,
         y: Optional[torch.Tensor] = None, final_states: Optional[torch.Tensor] = None,
         workspace: Optional[torch.Tensor] = None, generic: bool = False,
-        timing_events: Optional[tuple] = None, z: Optional[torch.Tensor] = None):
+        timing_events: Optional[tuple] = None, z: Optional[torch.Tensor] = None, check_seq: bool = False):
     """SSD forward.  Returns (y, final_states or None).
 
     x (b,L,H,P) fp32|bf16, dt (b,L,H) fp32, A (H) fp32, B/C (b,L,G,N) x.dtype,
@@ -226,6 +229,8 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     the current stream around the call's main kernel.
     ``z`` (b,L,H,P) x.dtype or None: the block's gate, y is returned as
     y * SiLU(z).
+    ``check_seq``: check the seq_idx precondition on a host copy first
+    (synchronous; raises SSDError on a violation).
     """
     _check(x, dt, A, B, C, D, initial_states, seq_idx)
     if z is not None and (z.dtype != x.dtype or tuple(z.shape) != tuple(x.shape) or z.device != x.device
@@ -244,6 +249,8 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
         final_states = None
     a = make_args(x, dt, A, B, C, D, chunk_size, initial_states, seq_idx, num_seqs, y, final_states,
                   generic=generic, z=z)
+    if check_seq:
+        a.flags |= SSD_FLAG_CHECK_SEQ
     need = int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
     if need > 0:
         if workspace is None or workspace.numel() * workspace.element_size() < need:

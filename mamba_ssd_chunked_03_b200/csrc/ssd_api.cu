@@ -2,6 +2,8 @@
 // The operation and its sources are described in include/ssd.h.
 #include <cuda_runtime.h>
 
+#include <vector>
+
 #include "ssd.h"
 #include "ssd_internal.h"
 
@@ -20,7 +22,7 @@ ssd_status check_sizes(const ssd_fwd_args* a) {
   if (a->nheads % a->ngroups != 0) return SSD_ERR_INVALID_ARG;
   if (!is_pow2(a->chunk_size) || a->chunk_size < 16 || a->chunk_size > 256) return SSD_ERR_INVALID_ARG;
   if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
-  if (a->flags & ~SSD_FLAG_GENERIC) return SSD_ERR_INVALID_ARG;
+  if (a->flags & ~(SSD_FLAG_GENERIC | SSD_FLAG_CHECK_SEQ)) return SSD_ERR_INVALID_ARG;
   if (a->seq_idx && a->num_seqs <= 0) return SSD_ERR_INVALID_ARG;
   if (a->seq_idx && a->num_seqs > (int64_t)1 << 31) return SSD_ERR_INVALID_ARG;
   // implemented shape set
@@ -123,6 +125,15 @@ ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream) {
   if (need > 0 && (!a->workspace || a->workspace_bytes < need)) return SSD_ERR_WORKSPACE;
   if (!ssd::aligned(a->workspace, ssd::kWsAlign)) return SSD_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((a->flags & SSD_FLAG_CHECK_SEQ) && a->seq_idx) {
+    std::vector<int32_t> host((size_t)(a->batch * a->seqlen));
+    if (cudaMemcpyAsync(host.data(), a->seq_idx, host.size() * sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return SSD_ERR_CUDA;
+    const ssd_status cs = ssd_check_seq_idx(host.data(), a->batch, a->seqlen, a->num_seqs);
+    if (cs != SSD_OK) return cs;
+  }
   cudaEvent_t ev0 = static_cast<cudaEvent_t>(a->timing_events[0]);
   cudaEvent_t ev1 = static_cast<cudaEvent_t>(a->timing_events[1]);
   if (tc) return ssd::tc_forward(p, a->workspace, s, ev0, ev1) == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
@@ -130,6 +141,21 @@ ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream) {
   const cudaError_t err = ssd::generic_forward(p, a->workspace, s);
   if (err != cudaSuccess) return SSD_ERR_CUDA;
   if (ev1 && cudaEventRecord(ev1, s) != cudaSuccess) return SSD_ERR_CUDA;
+  return SSD_OK;
+}
+
+ssd_status ssd_check_seq_idx(const int32_t* seq, int64_t batch, int64_t seqlen, int64_t num_seqs) {
+  if (!seq || batch <= 0 || seqlen <= 0 || num_seqs <= 0) return SSD_ERR_INVALID_ARG;
+  std::vector<int64_t> row_of((size_t)num_seqs, -1);  // the row each id was seen in
+  for (int64_t r = 0; r < batch; ++r) {
+    for (int64_t t = 0; t < seqlen; ++t) {
+      const int32_t id = seq[r * seqlen + t];
+      if (id < 0 || id >= num_seqs) return SSD_ERR_INVALID_ARG;
+      if (t > 0 && id < seq[r * seqlen + t - 1]) return SSD_ERR_INVALID_ARG;  // decreasing along the row
+      if (row_of[(size_t)id] != -1 && row_of[(size_t)id] != r) return SSD_ERR_INVALID_ARG;  // in two rows
+      row_of[(size_t)id] = r;
+    }
+  }
   return SSD_OK;
 }
 

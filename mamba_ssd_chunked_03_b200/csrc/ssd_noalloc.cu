@@ -53,9 +53,10 @@ void* scratch_on_current_device() {
 extern "C" ssd_status ssd_fwd_noalloc(const ssd_fwd_args* args, void* stream) {
   if (!args) return SSD_ERR_INVALID_ARG;
   // Same argument rules as ssd_fwd; workspace fields and the kernel-path flag
-  // are ignored (this entry point always runs the generic kernels).
+  // are ignored (this entry point always runs the generic kernels).  The
+  // seq_idx check, if asked for, uses host memory only.
   ssd_fwd_args a = *args;
-  a.flags = SSD_FLAG_GENERIC;
+  a.flags = SSD_FLAG_GENERIC | (args->flags & SSD_FLAG_CHECK_SEQ);
   a.workspace = nullptr;
   a.workspace_bytes = 0;
   const size_t need = ssd_fwd_workspace_size(&a);

@@ -252,3 +252,35 @@ def test_workspace_grows_with_packed_sequences():
     plain = ssd.lib.ssd_fwd_workspace_size(ctypes.byref(a))
     a.seq_idx, a.num_seqs = 1 << 21, 50
     assert ssd.lib.ssd_fwd_workspace_size(ctypes.byref(a)) > plain
+
+
+def _check_seq(rows, num_seqs):
+    import numpy as np
+    arr = np.ascontiguousarray(np.array(rows, dtype=np.int32))
+    return ssd.lib.ssd_check_seq_idx(arr.ctypes.data, arr.shape[0], arr.shape[1], num_seqs)
+
+
+@pytest.mark.parametrize("rows,num_seqs,status", [
+    ([[0, 0, 1, 1, 2]], 3, ssd.SSD_OK),
+    ([[0, 0, 1], [2, 2, 3]], 4, ssd.SSD_OK),
+    ([[0, 0, 2]], 5, ssd.SSD_OK),                      # ids that never occur are allowed
+    ([[0, 1, 0]], 2, ssd.SSD_ERR_INVALID_ARG),         # decreasing along a row
+    ([[0, 0, 3]], 3, ssd.SSD_ERR_INVALID_ARG),         # id outside [0, num_seqs)
+    ([[-1, 0, 0]], 3, ssd.SSD_ERR_INVALID_ARG),
+    ([[0, 0, 1], [1, 1, 2]], 3, ssd.SSD_ERR_INVALID_ARG),  # id 1 in two rows
+])
+def test_seq_idx_precondition_check(rows, num_seqs, status):
+    assert _check_seq(rows, num_seqs) == status
+
+
+def test_seq_idx_check_rejects_null_and_bad_sizes():
+    assert ssd.lib.ssd_check_seq_idx(None, 1, 1, 1) == ssd.SSD_ERR_INVALID_ARG
+    assert _check_seq([[0]], 0) == ssd.SSD_ERR_INVALID_ARG
+
+
+def test_check_flag_is_accepted_and_unknown_flags_rejected():
+    a = base_args()
+    a.flags = ssd.SSD_FLAG_CHECK_SEQ
+    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"tcgen05"
+    a.flags = 4
+    assert call(a) == ssd.SSD_ERR_INVALID_ARG
