@@ -14,7 +14,10 @@ Contents:
   * ``block.conv1d_silu``, ``block.gate`` -- the Mamba-2 block pieces around the SSD
                               (causal depthwise conv1d + SiLU; the SiLU gate).
   * ``backward.ssd_bwd``     -- the backward pass: the adjoint of the recurrence
-                              (derived; the pages give no formulas), fp64.
+                              (derived; the pages give no formulas), fp64 numpy.
+  * ``ssd_bwd``              -- the same adjoint in C + OpenMP (``ssd_oracle.c``),
+                              states recomputed from 64-token checkpoints, for
+                              larger inputs.
   * ``chunked.ssd_chunked``  -- the four chunked steps written out literally in
                               fp64 numpy (a pin for the decomposition the CUDA
                               kernels use).
@@ -55,6 +58,9 @@ def load_library(path: str) -> ctypes.CDLL:
     i64, vp = ctypes.c_int64, ctypes.c_void_p
     f.argtypes = [i64] * 6 + [vp] * 8 + [i64, vp, vp, vp, i64, ctypes.c_int]
     f.restype = ctypes.c_int
+    g = lib.oracle_ssd_bwd
+    g.argtypes = [i64] * 6 + [vp] * 17 + [ctypes.c_int]
+    g.restype = ctypes.c_int
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
 
@@ -140,3 +146,39 @@ def ssd_fwd(x, dt, A, B, C, D=None, initial_states=None, seq_idx=None, num_seqs=
     if rc != 0:
         raise RuntimeError(f"oracle_ssd_fwd failed with code {rc}")
     return y, final
+
+
+def ssd_bwd(x, dt, A, B, C, D=None, initial_states=None, dy=None, dfinal=None, seq_idx=None,
+            nthreads: int = 0) -> dict:
+    """The backward pass in C (fp64, OpenMP over (b, h)): gradients of
+    sum(dy * y) + sum(dfinal * final) as a dict like ``backward.ssd_bwd``."""
+    x32, dt32, A32, B32, C32 = (as_f32(v) for v in (x, dt, A, B, C))
+    D32, h032, si = as_f32(D), as_f32(initial_states), as_i32(seq_idx)
+    dy32, df32 = as_f32(dy), as_f32(dfinal)
+    b, L, H, P = x32.shape
+    G, N = B32.shape[2], B32.shape[3]
+    assert dy32.shape == (b, L, H, P)
+    dx = np.zeros((b, L, H, P))
+    ddt = np.zeros((b, L, H))
+    dBh = np.zeros((b, L, H, N))
+    dCh = np.zeros((b, L, H, N))
+    dA_u = np.zeros(b * H)
+    dD_u = np.zeros(b * H)
+    dh0 = np.zeros((b, H, P, N)) if h032 is not None else None
+
+    def ptr(a):
+        return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+    rc = _get_lib().oracle_ssd_bwd(b, L, H, P, N, G, ptr(x32), ptr(dt32), ptr(A32), ptr(B32), ptr(C32),
+                                   ptr(D32), ptr(h032), ptr(si), ptr(dy32), ptr(df32), ptr(dx), ptr(ddt),
+                                   ptr(dBh), ptr(dCh), ptr(dA_u), ptr(dD_u), ptr(dh0), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_ssd_bwd failed with code {rc}")
+    grp = np.arange(H) // (H // G)
+    dB = np.zeros((b, L, G, N))
+    dC = np.zeros((b, L, G, N))
+    for h in range(H):
+        dB[:, :, grp[h]] += dBh[:, :, h]
+        dC[:, :, grp[h]] += dCh[:, :, h]
+    return {"dx": dx, "ddt": ddt, "dA": dA_u.reshape(b, H).sum(axis=0), "dB": dB, "dC": dC,
+            "dD": None if D32 is None else dD_u.reshape(b, H).sum(axis=0), "dh0": dh0}

@@ -99,3 +99,30 @@ def test_backward_matches_finite_differences_of_the_forward_oracle():
         fd = (loss(plus) - loss(minus)) / (2 * eps)
         an = float(got[names[key]][idx])
         assert abs(fd - an) <= 1e-4 * max(1.0, abs(an)), (key, fd, an)
+
+
+@pytest.mark.parametrize("case", CASES + [(2, 200, 4, 8, 16, 2, 0.4, True, True, None),
+                                          (1, 300, 2, 8, 8, 1, 0.2, True, False, [[70, 1, 100, 129]])],
+                         ids=lambda c: f"b{c[0]}L{c[1]}H{c[2]}G{c[5]}{'_packed' if c[9] else ''}")
+def test_c_backward_matches_the_numpy_backward(case):
+    """The C backward (checkpointed recompute) agrees with the numpy one,
+    which autograd and finite differences pin; L up to 300 spans several
+    64-token checkpoints."""
+    b, L, H, P, N, G, h0s, withD, withF, packed = case
+    d = si.make_inputs(si.SSDShape("bwd_c", b, L, H, P, N, G, 64, "f32", h0_std=h0s, seed=L + H))
+    if not withD:
+        d["D"] = None
+    if packed is not None:
+        d["seq_idx"], d["num_seqs"] = si.seq_idx_from_lengths(packed)
+    rng = np.random.default_rng(L + 1)
+    f32 = lambda a: a.astype(np.float32).astype(np.float64)
+    dy = f32(rng.standard_normal((b, L, H, P)))
+    dfinal = f32(rng.standard_normal((b, H, P, N))) if withF else None
+    args = (d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["initial_states"])
+    want = backward.ssd_bwd(*args, dy, dfinal, d.get("seq_idx"))
+    got = oracle.ssd_bwd(*args, dy=dy, dfinal=dfinal, seq_idx=d.get("seq_idx"))
+    for k, w in want.items():
+        if w is None:
+            assert got[k] is None, k
+            continue
+        assert np.allclose(got[k], w, rtol=1e-11, atol=1e-11 * max(1.0, np.abs(w).max())), k
