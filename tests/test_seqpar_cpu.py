@@ -98,13 +98,14 @@ def _rank_main(rank, world, port, cuts, out):
         dist.destroy_process_group()
 
 
-def test_fwd_seqpar_two_gloo_ranks():
-    cuts = [0, 117, 200]
+@pytest.mark.parametrize("cuts", [[0, 117, 200], [0, 64, 65, 200]], ids=["2_ranks", "3_ranks"])
+def test_fwd_seqpar_gloo_ranks(cuts):
+    world = len(cuts) - 1
     ctx = mp.get_context("spawn")
     with ctx.Manager() as m:
         out = m.dict()
         port = _free_port()
-        procs = [ctx.Process(target=_rank_main, args=(r, 2, port, cuts, out)) for r in range(2)]
+        procs = [ctx.Process(target=_rank_main, args=(r, world, port, cuts, out)) for r in range(world)]
         for p in procs:
             p.start()
         for p in procs:
@@ -112,6 +113,6 @@ def test_fwd_seqpar_two_gloo_ranks():
         assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
         shape = si.SSDShape("sp", 2, 200, 3, 8, 8, 1, 64, "f32", h0_std=0.5, seed=5)
         yw, fw = _whole(si.make_inputs(shape))
-        y = np.concatenate([out[0][0], out[1][0]], axis=1)
+        y = np.concatenate([out[r][0] for r in range(world)], axis=1)
         assert np.abs(y - yw).max() <= 1e-5 * max(1.0, np.abs(yw).max())
-        assert np.abs(out[1][1] - fw).max() <= 1e-5 * max(1.0, np.abs(fw).max())
+        assert np.abs(out[world - 1][1] - fw).max() <= 1e-5 * max(1.0, np.abs(fw).max())
