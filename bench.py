@@ -46,6 +46,8 @@ DATASHEET_HBM_GBS = 8000.0
 DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
+# fp32 FMA throughput of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (max SM clock)
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -216,6 +218,8 @@ def run_reference_op(args):
     """``--impl reference`` for ``--op step`` / ``--op conv``: the oracle on the
     same workload as the GPU arm, timed on the host cores."""
     import oracle
+    if args.op == "bwd":
+        return run_reference_bwd(args)
     if args.op == "step":
         b, H, P, N, G = args.step_batch, 80, 64, 128, 1
         shape = si.SSDShape("decode", b, 1, H, P, N, G, 64, "bf16", h0_std=0.5, seed=11)
@@ -500,6 +504,192 @@ def run_conv(args, dist, dev, world, rank):
     return 0
 
 
+# ----------------------------------------------------------------------------- backward
+
+BWD_SHAPE = si.SSDShape("c1_bwd", 8, 2048, 80, 64, 128, 1, 64, "bf16", seed=1001)
+BWD_WORKLOAD = "SSD bwd on the c1 layout: b8 L2048 H80 P64 N128 G1 bf16, from dy, fp32 gradients"
+
+
+def bwd_flops(b, L, H, P, N, Q):
+    """Algorithmic FLOPs (2 per multiply-add) of the backward's two per-chunk
+    kernels, (k_bwd_chunk_states, k_bwd_chunk), for chunk length Q.  Per chunk
+    of Qc tokens, with T2 = Qc (Qc + 1) / 2 lower-triangle pairs:
+    k_bwd_chunk_states forms two P x N sums of Qc outer products (2 Qc P N);
+    k_bwd_chunk forms C B^T and dy x^T on the triangle (T2 (N + P)), Lam B^T
+    and h_in C^T (2 Qc P N), the triangle products for dx, dB, dC
+    (T2 (P + 2 N)), the state terms of dB and dC (2 Qc P N) and <Lam, h_in>
+    (P N)."""
+    states = chunk = 0
+    for c in range(-(-L // Q)):
+        qc = min(Q, L - c * Q)
+        t2 = qc * (qc + 1) // 2
+        states += 2 * qc * P * N
+        chunk += t2 * (3 * N + 2 * P) + 4 * qc * P * N + P * N
+    return 2 * b * H * states, 2 * b * H * chunk
+
+
+def bwd_inputs(shape, rank=0):
+    host = si.make_inputs(shape, seed=shape.seed + rank)
+    g = torch.Generator().manual_seed(shape.seed + 17 + rank)
+    host["dy"] = torch.randn(*host["x"].shape, generator=g).to(host["x"].dtype)
+    return host
+
+
+def bwd_oracle_sample(host, shape, target_s: float):
+    """The C backward oracle on batch row 0 and its first U heads, U grown
+    by waves of the host's threads until a run takes about ``target_s``.
+    Returns (tokens/s, U, seconds, threads)."""
+    import oracle  # test infrastructure: only the CPU-baseline legs use it here
+    threads = oracle.max_threads()
+
+    def run(U):
+        sl = {k: host[k][:1, :, :U].contiguous() for k in ("x", "dt", "dy")}
+        A, D = host["A"][:U].contiguous(), host["D"][:U].contiguous()
+        B, C = host["B"][:1], host["C"][:1]
+        t = time.perf_counter()
+        oracle.ssd_bwd(sl["x"], sl["dt"], A, B, C, D, None, sl["dy"], None, None)
+        return time.perf_counter() - t
+
+    U = min(shape.nheads, threads)
+    el = run(U)
+    while el < target_s / 2 and U < shape.nheads:
+        U = min(shape.nheads, U * 2)
+        el = run(U)
+    return U * shape.seqlen / shape.nheads / el, U, el, min(threads, U)
+
+
+def run_reference_bwd(args):
+    """``--impl reference --op bwd``: the C backward oracle on a bounded sample
+    (batch row 0, the first heads) of the backward workload."""
+    shape = BWD_SHAPE
+    host = bwd_inputs(shape)
+    per_run = []
+    for i in range(args.warmup + args.steps):
+        v, U, el, cores = bwd_oracle_sample(host, shape, 2.0)
+        if i >= args.warmup:
+            per_run.append((v, U, el, cores))
+    value = statistics.median(r[0] for r in per_run)
+    U, cores = per_run[-1][1], per_run[-1][3]
+    sample = f"batch row 0, heads 0..{U - 1} of {shape.nheads} ({U * shape.seqlen} head-tokens) per step"
+    line = {
+        "impl": "reference", "metric": "SSD bwd tokens/s", "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.median(r[2] for r in per_run) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": BWD_WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_bwd(args, dist, dev, world, rank):
+    """``--op bwd``: the backward ``ssd_bwd`` on c1's layout (b 8, L 2048,
+    H 80, P 64, N 128, G 1, bf16) from a random dy, all gradients in fp32.
+    Its kernels run on the CUDA cores, so the roofline is fp32 FMA throughput
+    (bound "alu") on k_bwd_chunk, the dominant kernel."""
+    import mamba_ssd_chunked_03_b200 as ssd
+    shape = BWD_SHAPE
+    b, L, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
+    host = bwd_inputs(shape, rank)
+    names = ("x", "dt", "B", "C", "dy")
+    g = {k: host[k].to(dev) for k in names}
+    A, D = host["A"].to(dev), host["D"].to(dev)
+    ws = torch.empty(ssd.bwd_workspace_size(g["x"], g["B"]), dtype=torch.uint8, device=dev)
+    pl = {"Q": 64}
+    for q in (64, 32, 16, 8):  # the library's own choice for chunk_size 0
+        if ssd.bwd_workspace_size(g["x"], g["B"], chunk_size=q) == ws.numel():
+            pl["Q"] = q
+            break
+    K = args.steps
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for e0_, e1_ in events:  # torch creates an event on its first record
+        e0_.record()
+        e1_.record()
+    out = {}
+
+    def step(ev=None):
+        out.update(ssd.bwd(g["x"], g["dt"], A, g["B"], g["C"], D, g["dy"], workspace=ws, timing_events=ev))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_uuid(dev))
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        step(events[i])
+    e1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clock_stats = clocks.stop()
+    ms_step = max_over_ranks(e0.elapsed_time(e1), dist, dev) / K
+    per = sorted(a.elapsed_time(z) for a, z in events)
+    kernel_ms = max_over_ranks(sum(per) / K, dist, dev)
+
+    pinned = {k: host[k].pin_memory() for k in names}
+    grads_host = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items() if v is not None}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = sum(v.numel() * v.element_size() for v in grads_host.values())
+
+    def e2e_step():
+        for k in names:
+            g[k].copy_(pinned[k], non_blocking=True)
+        step()
+        for k, v in grads_host.items():
+            v.copy_(out[k], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    E = max(3, min(K, 20))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(E):
+        e2e_step()
+    a1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev) / E
+
+    f_states, f_chunk = bwd_flops(b, L, H, P, N, pl["Q"])
+    achieved = f_chunk / (kernel_ms / 1e3) / 1e12
+    tokens = b * L
+    line = {
+        "metric": "SSD bwd tokens/s", "value": tokens * world / (ms_step / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": BWD_WORKLOAD,
+                   "l2": "no flush: inputs, gradients and the per-chunk states (GBs) exceed the 126 MB L2",
+                   "parallelism": "replicas" if world > 1 else "single GPU", "bwd_chunk": pl["Q"]},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                     "frac": achieved / FP32_PEAK_TFLOPS,
+                     "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz",
+                     "kernel": "k_bwd_chunk", "kernel_ms": kernel_ms,
+                     "kernel_ms_p10_p50_p90": [per[int(0.1 * (K - 1))], per[int(0.5 * (K - 1))],
+                                               per[int(0.9 * (K - 1))]],
+                     "traffic": None, "algorithmic_flops": f_chunk, "states_kernel_flops": f_states},
+        "e2e": {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": E},
+        "gpu_launches": 5 * K,
+        "clocks": clock_stats,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, U, el, cores = bwd_oracle_sample(host, shape, min(args.cpu_seconds, 10.0))
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"batch row 0, heads 0..{U - 1} of {H}, {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def main():
@@ -512,9 +702,9 @@ def main():
     ap.add_argument("--generic", action="store_true", help="force the generic CUDA-core kernels")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--op", default="fwd", choices=["fwd", "step", "conv"],
+    ap.add_argument("--op", default="fwd", choices=["fwd", "step", "conv", "bwd"],
                     help="fwd: the chunked forward (default); step: the recurrent decode step; "
-                         "conv: the block's causal conv1d + SiLU")
+                         "conv: the block's causal conv1d + SiLU; bwd: the backward on c1's layout")
     ap.add_argument("--step-batch", type=int, default=256, help="rows of the decode step (--op step)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -542,6 +732,8 @@ def main():
         return run_step(args, dist, dev, world, rank)
     if args.op == "conv":
         return run_conv(args, dist, dev, world, rank)
+    if args.op == "bwd":
+        return run_bwd(args, dist, dev, world, rank)
 
     host = si.make_inputs(shape, seed=shape.seed + rank)
     num_seqs = host.get("num_seqs")

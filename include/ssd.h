@@ -262,6 +262,83 @@ typedef struct {
 
 SSD_API ssd_status ssd_conv1d_silu(const ssd_conv_args* args, void* stream);
 
+/* The backward pass of ssd_fwd: the gradients of a loss with respect to every
+ * input, given dy = dLoss/dy and optionally dfinal = dLoss/dfinal_states.
+ * The pages give the forward recurrence (sources above) and say that the
+ * backward recomputes the forward's states rather than storing them ("从
+ * Transformer的二次复杂度困境到Mamba的线性突围", the hardware-aware algorithm:
+ * recomputation); the gradients are the adjoint of that recurrence.  With
+ * G_t = dLoss/dh_t, swept from the last token (G_{L-1} also receives dfinal):
+ *
+ *   G_t   = dy_t C_t^T + a_{t+1} G_{t+1}
+ *   dx_t  = dt_t G_t B_t + D_h dy_t
+ *   dB_t  = sum over the group's heads of dt_t G_t^T x_t
+ *   dC_t  = sum over the group's heads of h_t^T dy_t
+ *   ddt_t = <G_t, x_t B_t^T> + A_h a_t <G_t, h_{t-1}>
+ *   dA_h  = sum_{b,t} dt_t a_t <G_t, h_{t-1}>
+ *   dD_h  = sum_{b,t} <dy_t, x_t>
+ *   dinitial_states = a_0 G_0
+ *
+ * (<.,.> sums over all entries; a token that starts a packed sequence has
+ * a_t = 0 and passes no gradient to h_{t-1}, to its decay or to A.)  It is
+ * computed chunk by chunk: the states entering each chunk are recomputed, the
+ * adjoint state is carried backwards across chunks, and every chunk then
+ * forms its gradients from its own tokens and those two states.  All
+ * arithmetic is fp32; every gradient is written as fp32, whatever the input
+ * dtype.  Chunking re-associates the same sums, so the result equals the
+ * adjoint recurrence up to rounding for every chunk size. */
+typedef struct {
+  /* sizes as in ssd_fwd_args; headdim and dstate at most 256.  chunk_size is
+   * the chunk length of the backward itself, unrelated to the forward's: 0
+   * lets the library choose (64, halved while its shared memory would not
+   * fit), or 1..64 (SSD_ERR_UNSUPPORTED if that does not fit). */
+  int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk_size;
+  ssd_dtype dtype;                /* of x, B, C and dy                                */
+  const void* x;                  /* (b,L,H,P) dtype                                  */
+  const float* dt;                /* (b,L,H) fp32                                     */
+  const float* A;                 /* (H) fp32                                         */
+  const void* B;                  /* (b,L,G,N) dtype                                  */
+  const void* C;                  /* (b,L,G,N) dtype                                  */
+  const float* D;                 /* (H) fp32, or NULL for D = 0                      */
+  const float* initial_states;    /* (b,H,P,N) fp32, or NULL = 0                      */
+  const int32_t* seq_idx;         /* (b,L) int32 packed-sequence ids, or NULL; the
+                                     precondition of ssd_fwd_args (not checked)       */
+  const void* dy;                 /* (b,L,H,P) dtype, dLoss/dy                        */
+  const float* dfinal_states;     /* (b,H,P,N) fp32 dLoss/dfinal_states, or NULL = 0.
+                                     Not with seq_idx (SSD_ERR_UNSUPPORTED).          */
+  float* dx;                      /* (b,L,H,P) fp32, output                           */
+  float* ddt;                     /* (b,L,H) fp32, output                             */
+  float* dA;                      /* (H) fp32, output                                 */
+  float* dB;                      /* (b,L,G,N) fp32, output                           */
+  float* dC;                      /* (b,L,G,N) fp32, output                           */
+  float* dD;                      /* (H) fp32 output, or NULL to skip                 */
+  float* dinitial_states;         /* (b,H,P,N) fp32 output, or NULL to skip (written
+                                     also when initial_states is NULL: the gradient
+                                     at a zero initial state)                        */
+  void* workspace;                /* device scratch of ssd_bwd_workspace_size(args)
+                                     bytes, 256-byte aligned; contents on entry do
+                                     not matter                                      */
+  size_t workspace_bytes;
+  void* timing_events[2];         /* optional pair of cudaEvent_t (as void*), or NULLs:
+                                     recorded on `stream` right before and right after
+                                     k_bwd_chunk, the kernel that dominates the call.
+                                     Both or neither.                                */
+} ssd_bwd_args;
+
+/* Bytes of device workspace ssd_bwd needs (only sizes, chunk_size and dtype
+ * are read), or 0 if the sizes are invalid or unsupported. */
+SSD_API size_t ssd_bwd_workspace_size(const ssd_bwd_args* args);
+
+/* Enqueue the backward on `stream`: five kernels, no allocation, no memset.
+ * All pointers are device pointers owned by the caller; outputs must not
+ * overlap inputs or the workspace.  Returns SSD_OK once enqueued;
+ * SSD_ERR_INVALID_ARG for a null required pointer, a bad size or enum, or a
+ * misaligned workspace or a single timing event; SSD_ERR_UNSUPPORTED as
+ * described above;
+ * SSD_ERR_WORKSPACE when the workspace is missing or too small; SSD_ERR_CUDA
+ * when a launch fails (outputs then undefined). */
+SSD_API ssd_status ssd_bwd(const ssd_bwd_args* args, void* stream);
+
 /* The seq_idx precondition, on a HOST copy (b,L) int32: ids in [0, num_seqs),
  * non-decreasing along each row, and no id in two rows.  SSD_OK, or
  * SSD_ERR_INVALID_ARG at the first violation (or for a null pointer or a

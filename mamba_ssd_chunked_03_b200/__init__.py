@@ -10,6 +10,8 @@ Python or CPU fallback, and importing fails loudly if the library is missing.
     y, final_states = fwd(x, dt, A, B, C, D, chunk_size=64,
                           initial_states=None, seq_idx=None, num_seqs=None)
     y_t = step(x_t, dt_t, A, B_t, C_t, D, state)   # one decode step, state in place
+    grads = bwd(x, dt, A, B, C, D, dy)              # the backward (fp32 gradients)
+    y, final_states = ssd_chunked(x, dt, A, B, C, D)  # differentiable: fwd, then bwd
 """
 from __future__ import annotations
 
@@ -19,7 +21,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["fwd", "step", "StepArgs", "total_decay", "state_fold", "conv1d_silu", "ConvArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
+__all__ = ["fwd", "bwd", "BwdArgs", "ssd_chunked", "step", "StepArgs", "total_decay", "state_fold", "conv1d_silu", "ConvArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
            "SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED", "SSD_ERR_WORKSPACE", "SSD_ERR_CUDA",
            "SSD_F32", "SSD_BF16", "SSD_FLAG_GENERIC"]
 
@@ -67,6 +69,23 @@ class ConvArgs(ctypes.Structure):
     ]
 
 
+class BwdArgs(ctypes.Structure):
+    """Mirror of ``ssd_bwd_args``."""
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups", "chunk_size")] + [
+        ("dtype", ctypes.c_int),
+        ("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("A", ctypes.c_void_p),
+        ("B", ctypes.c_void_p), ("C", ctypes.c_void_p), ("D", ctypes.c_void_p),
+        ("initial_states", ctypes.c_void_p), ("seq_idx", ctypes.c_void_p),
+        ("dy", ctypes.c_void_p), ("dfinal_states", ctypes.c_void_p),
+        ("dx", ctypes.c_void_p), ("ddt", ctypes.c_void_p), ("dA", ctypes.c_void_p),
+        ("dB", ctypes.c_void_p), ("dC", ctypes.c_void_p), ("dD", ctypes.c_void_p),
+        ("dinitial_states", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("timing_events", ctypes.c_void_p * 2),
+    ]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -87,6 +106,10 @@ def _load() -> ctypes.CDLL:
     L.ssd_fwd_main_kernel.restype = ctypes.c_char_p
     L.ssd_step.argtypes = [ctypes.POINTER(StepArgs), ctypes.c_void_p]
     L.ssd_step.restype = ctypes.c_int
+    L.ssd_bwd.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_void_p]
+    L.ssd_bwd.restype = ctypes.c_int
+    L.ssd_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs)]
+    L.ssd_bwd_workspace_size.restype = ctypes.c_size_t
     L.ssd_conv1d_silu.argtypes = [ctypes.POINTER(ConvArgs), ctypes.c_void_p]
     L.ssd_conv1d_silu.restype = ctypes.c_int
     L.ssd_total_decay.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int64] * 3 + [
@@ -371,3 +394,109 @@ def conv1d_silu(u: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tens
     if st != SSD_OK:
         raise SSDError(st)
     return out
+
+
+def make_bwd_args(x, dt, A, B, C, D=None, dy=None, initial_states=None, seq_idx=None, dfinal_states=None,
+                  chunk_size: int = 0) -> BwdArgs:
+    """Fill an ``ssd_bwd_args`` from tensors (shapes read from x and B); the
+    gradient and workspace pointers are left NULL."""
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    a = BwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk_size = b, L, H, P, N, G, int(chunk_size)
+    a.dtype = SSD_BF16 if x.dtype == torch.bfloat16 else SSD_F32
+    a.x, a.dt, a.A, a.B, a.C, a.D = _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D)
+    a.initial_states, a.seq_idx = _ptr(initial_states), _ptr(seq_idx)
+    a.dy, a.dfinal_states = _ptr(dy), _ptr(dfinal_states)
+    return a
+
+
+def bwd_workspace_size(x, B, chunk_size: int = 0) -> int:
+    """Workspace bytes ``ssd_bwd`` needs for these shapes (0: not supported)."""
+    a = make_bwd_args(x, None, None, B, None, chunk_size=chunk_size)
+    return int(lib.ssd_bwd_workspace_size(ctypes.byref(a)))
+
+
+def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+        D: Optional[torch.Tensor], dy: torch.Tensor, initial_states: Optional[torch.Tensor] = None,
+        seq_idx: Optional[torch.Tensor] = None, dfinal_states: Optional[torch.Tensor] = None,
+        chunk_size: int = 0, want_dD: bool = True, want_dinitial_states: Optional[bool] = None,
+        workspace: Optional[torch.Tensor] = None, timing_events: Optional[tuple] = None) -> dict:
+    """The SSD backward via ``ssd_bwd``: gradients of a loss given
+    dy = dLoss/dy (like x) and dfinal_states = dLoss/dfinal_states
+    ((b,H,P,N) fp32 or None; not with seq_idx).  Inputs as for ``fwd``.
+    Returns a dict of fp32 tensors dx, ddt, dA, dB, dC, dD (None unless
+    ``want_dD``) and dinitial_states (by default only when initial_states
+    is given).  ``chunk_size`` is the backward's own chunk length (0: the
+    library chooses).  ``timing_events``: optional (start, end)
+    torch.cuda.Event pair recorded around the dominant kernel."""
+    _check(x, dt, A, B, C, D, initial_states, seq_idx)
+    if dy.dtype != x.dtype or tuple(dy.shape) != tuple(x.shape) or dy.device != x.device or not dy.is_contiguous():
+        raise ValueError("dy must be a contiguous tensor like x")
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if dfinal_states is not None and (dfinal_states.dtype != torch.float32 or tuple(dfinal_states.shape) != (b, H, P, N)
+                                      or dfinal_states.device != x.device or not dfinal_states.is_contiguous()):
+        raise ValueError("dfinal_states must be a contiguous float32 (b, H, P, N) tensor on x's device")
+    if want_dinitial_states is None:
+        want_dinitial_states = initial_states is not None
+    f32 = dict(device=x.device, dtype=torch.float32)
+    g = {"dx": torch.empty(b, L, H, P, **f32), "ddt": torch.empty(b, L, H, **f32), "dA": torch.empty(H, **f32),
+         "dB": torch.empty(b, L, G, N, **f32), "dC": torch.empty(b, L, G, N, **f32),
+         "dD": torch.empty(H, **f32) if want_dD else None,
+         "dinitial_states": torch.empty(b, H, P, N, **f32) if want_dinitial_states else None}
+    a = make_bwd_args(x, dt, A, B, C, D, dy, initial_states, seq_idx, dfinal_states, chunk_size)
+    a.dx, a.ddt, a.dA, a.dB, a.dC = (_ptr(g[k]) for k in ("dx", "ddt", "dA", "dB", "dC"))
+    a.dD, a.dinitial_states = _ptr(g["dD"]), _ptr(g["dinitial_states"])
+    need = int(lib.ssd_bwd_workspace_size(ctypes.byref(a)))
+    if need == 0:
+        raise SSDError(SSD_ERR_UNSUPPORTED)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    if timing_events is not None:
+        h0_, h1_ = timing_events[0].cuda_event, timing_events[1].cuda_event
+        if not h0_ or not h1_:
+            raise ValueError("timing events must have been recorded once (torch creates them lazily)")
+        a.timing_events[0], a.timing_events[1] = h0_, h1_
+    st = lib.ssd_bwd(ctypes.byref(a), _stream(x))
+    if st != SSD_OK:
+        raise SSDError(st)
+    return g
+
+
+class _SSDChunked(torch.autograd.Function):
+    """``fwd`` forward, ``bwd`` backward; gradients returned in each input's dtype."""
+
+    @staticmethod
+    def forward(ctx, x, dt, A, B, C, D, initial_states, seq_idx, num_seqs, chunk_size):
+        ctx.set_materialize_grads(False)
+        y, fin = fwd(x, dt, A, B, C, D, chunk_size=chunk_size, initial_states=initial_states, seq_idx=seq_idx,
+                     num_seqs=num_seqs)
+        ctx.save_for_backward(x, dt, A, B, C, D, initial_states, seq_idx)
+        return y, fin
+
+    @staticmethod
+    def backward(ctx, dy, dfin):
+        x, dt, A, B, C, D, h0, seq = ctx.saved_tensors
+        if seq is not None and dfin is not None:
+            raise NotImplementedError("the gradient through per-sequence final states is not supported")
+        dy = torch.zeros_like(x) if dy is None else dy.to(x.dtype).contiguous()
+        dfin = None if dfin is None else dfin.to(torch.float32).contiguous()
+        need = ctx.needs_input_grad
+        g = bwd(x, dt, A, B, C, D, dy, initial_states=h0, seq_idx=seq, dfinal_states=dfin,
+                want_dD=D is not None and need[5], want_dinitial_states=h0 is not None and need[6])
+        return (g["dx"].to(x.dtype), g["ddt"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype), g["dD"],
+                g["dinitial_states"], None, None, None)
+
+
+def ssd_chunked(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+                D: Optional[torch.Tensor] = None, chunk_size: int = 64,
+                initial_states: Optional[torch.Tensor] = None, seq_idx: Optional[torch.Tensor] = None,
+                num_seqs: Optional[int] = None):
+    """Differentiable SSD forward: returns (y, final_states) like ``fwd``, and
+    its backward runs ``ssd_bwd`` (the states are recomputed, nothing but the
+    inputs is kept).  With seq_idx the final states carry no gradient."""
+    if seq_idx is not None and num_seqs is None:
+        num_seqs = int(seq_idx.max().item()) + 1
+    return _SSDChunked.apply(x, dt, A, B, C, D, initial_states, seq_idx, num_seqs, chunk_size)

@@ -1,0 +1,34 @@
+// ssd_bwd and ssd_bwd_workspace_size: the backward kernels of ssd_bwd.cuh,
+// launched on the caller's stream.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ssd.h"
+#include "ssd_bwd.cuh"
+
+namespace {
+
+struct CudaLaunch {
+  cudaStream_t stream;
+  bool operator()(void (*kern)(ssd::bwd::KArgs), unsigned grid, size_t smem, const ssd::bwd::KArgs& k) const {
+    if (grid == 0) return true;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute((const void*)kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return false;
+    kern<<<grid, ssd::bwd::kThreads, smem, stream>>>(k);
+    return cudaGetLastError() == cudaSuccess;
+  }
+  bool record(void* event) const { return cudaEventRecord(static_cast<cudaEvent_t>(event), stream) == cudaSuccess; }
+};
+
+}  // namespace
+
+extern "C" SSD_API size_t ssd_bwd_workspace_size(const ssd_bwd_args* a) {
+  ssd::bwd::Plan pl;
+  return ssd::bwd::plan(a, &pl) == SSD_OK ? pl.total : 0;
+}
+
+extern "C" SSD_API ssd_status ssd_bwd(const ssd_bwd_args* a, void* stream) {
+  CudaLaunch launch{static_cast<cudaStream_t>(stream)};
+  return ssd::bwd::run(a, launch);
+}

@@ -1,0 +1,79 @@
+"""Cases, inputs and the comparison rule shared by the backward tests (the
+host emulation in ``test_bwd_emu_cpu.py`` and the GPU parity tests in
+``test_zz_bwd_gpu.py``)."""
+import numpy as np
+import torch
+
+import oracle
+import ssd_inputs as si
+
+# The kernels compute in fp32 and the oracle in fp64 on the same (fp32- or
+# bf16-valued) inputs, so the gap is fp32 rounding in sums of at most
+# Q + P + N terms per stage, a few of them chained (measured below 1e-6
+# relative at these sizes); both bounds leave a wide margin over that.
+REL_L2 = 1e-5
+MAX_ABS = 1e-4
+KEYS = ("dx", "ddt", "dA", "dB", "dC", "dD", "dh0")
+
+CASES = [
+    # id, (b, L, H, P, N, G), dtype, h0 std, dfinal, packed (lo, hi) or per-row lengths, D, chunk
+    ("f32_ragged_Q16", (1, 50, 2, 8, 16, 1), "f32", 0.5, True, None, True, 16),
+    ("f32_groups_auto", (2, 150, 4, 24, 40, 2), "f32", 0.3, True, None, True, 0),
+    ("bf16_packed", (2, 150, 4, 16, 32, 2), "bf16", 0.0, False, (5, 40), False, 0),
+    # sequences starting exactly at a chunk start, one-token sequences, a row starting with two of them
+    ("f32_packed_edges", (2, 64, 2, 8, 8, 1), "f32", 0.4, False, [[16, 1, 15, 32], [1, 1, 30, 2, 30]], True, 16),
+    ("f32_chunk1", (1, 7, 2, 4, 4, 2), "f32", 0.5, True, None, True, 1),
+    ("f32_one_token", (2, 1, 2, 4, 8, 1), "f32", 0.5, True, None, True, 0),
+    # dstate 256 at headdim 64: a 64-token chunk does not fit one CTA's shared memory, 32 does
+    ("bf16_N256_chunk32", (1, 70, 2, 64, 256, 1), "bf16", 0.2, True, None, True, 0),
+    ("f32_hpg4", (1, 40, 8, 8, 16, 2), "f32", 0.0, True, None, True, 8),
+]
+
+
+def dy_like(b, L, H, P, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(b, L, H, P, generator=g).to(dtype)
+
+
+def dfinal_like(b, H, P, N, seed):
+    g = torch.Generator().manual_seed(seed + 1)
+    return torch.randn(b, H, P, N, generator=g)
+
+
+def inputs(b, L, H, P, N, G, dtype="f32", h0=0.0, packed=None, seed=1, has_D=True, lengths=None):
+    d = si.make_inputs(si.SSDShape("bwd", b, L, H, P, N, G, 64, dtype, h0_std=h0, packed=packed,
+                                   seed=seed, has_D=has_D))
+    if lengths is not None:
+        d["seq_idx"], d["num_seqs"] = si.seq_idx_from_lengths(lengths)
+    return d
+
+
+def case_inputs(case):
+    """(inputs, dy, dfinal, chunk) of one CASES entry."""
+    name, (b, L, H, P, N, G), dtype, h0, with_df, packed, with_D, chunk = case
+    d = inputs(b, L, H, P, N, G, dtype, h0, packed if isinstance(packed, tuple) else None, seed=L * 3 + H,
+               has_D=with_D, lengths=packed if isinstance(packed, list) else None)
+    dy = dy_like(b, L, H, P, d["x"].dtype, L + P)
+    dfinal = dfinal_like(b, H, P, N, L) if with_df else None
+    return d, dy, dfinal, chunk
+
+
+def oracle_bwd(d, dy, dfinal):
+    return oracle.ssd_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["initial_states"], dy, dfinal,
+                          d["seq_idx"])
+
+
+def compare(out, ref, keys=KEYS):
+    """Every gradient the oracle gives: finite, within REL_L2 in relative L2
+    and within MAX_ABS * max(1, max |ref|) element by element."""
+    for k in keys:
+        if ref.get(k) is None:
+            continue
+        got = np.asarray(out[k], dtype=np.float64)
+        want = ref[k]
+        assert got.shape == want.shape, f"{k}: shape {got.shape} != {want.shape}"
+        assert np.isfinite(got).all(), f"{k}: non-finite values"
+        rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+        mad = np.abs(got - want).max()
+        assert rel <= REL_L2, f"{k}: rel L2 {rel:.3g}"
+        assert mad <= MAX_ABS * max(1.0, np.abs(want).max()), f"{k}: max abs {mad:.3g}"

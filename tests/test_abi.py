@@ -284,3 +284,63 @@ def test_check_flag_is_accepted_and_unknown_flags_rejected():
     assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"tcgen05"
     a.flags = 4
     assert call(a) == ssd.SSD_ERR_INVALID_ARG
+
+
+def test_bwd_struct_layout_matches_the_compiled_header():
+    names = [f[0] for f in ssd.BwdArgs._fields_]
+    got = _c_layout(names, "ssd_bwd_args")
+    assert got[:-1] == [getattr(ssd.BwdArgs, n).offset for n in names]
+    assert got[-1] == ctypes.sizeof(ssd.BwdArgs)
+
+
+def _bwd_args(**kw):
+    a = ssd.BwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk_size = 2, 100, 4, 64, 128, 2, 0
+    a.dtype = ssd.SSD_BF16
+    # placeholders that are never dereferenced: every case below is rejected on the host
+    for i, n in enumerate(("x", "dt", "A", "B", "C", "dy", "dx", "ddt", "dA", "dB", "dC")):
+        setattr(a, n, 4096 * (i + 1))
+    a.workspace = 1 << 30
+    a.workspace_bytes = ssd.lib.ssd_bwd_workspace_size(ctypes.byref(a))
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({"batch": 0}, ssd.SSD_ERR_INVALID_ARG),
+    ({"nheads": 6, "ngroups": 4}, ssd.SSD_ERR_INVALID_ARG),
+    ({"dtype": 7}, ssd.SSD_ERR_INVALID_ARG),
+    ({"chunk_size": -1}, ssd.SSD_ERR_INVALID_ARG),
+    ({"x": None}, ssd.SSD_ERR_INVALID_ARG),
+    ({"dy": None}, ssd.SSD_ERR_INVALID_ARG),
+    ({"dC": None}, ssd.SSD_ERR_INVALID_ARG),
+    ({"workspace": None}, ssd.SSD_ERR_WORKSPACE),
+    ({"workspace_bytes": 1024}, ssd.SSD_ERR_WORKSPACE),
+    ({"workspace": (1 << 30) + 64}, ssd.SSD_ERR_INVALID_ARG),  # not 256-byte aligned
+    ({"seq_idx": 1 << 24, "dfinal_states": 1 << 25}, ssd.SSD_ERR_UNSUPPORTED),
+    ({"headdim": 257}, ssd.SSD_ERR_UNSUPPORTED),
+    ({"chunk_size": 65}, ssd.SSD_ERR_UNSUPPORTED),
+    ({"timing_events": (ctypes.c_void_p * 2)(1 << 12, None)}, ssd.SSD_ERR_INVALID_ARG),  # one event only
+])
+def test_bwd_rejects_bad_arguments(kw, status):
+    assert ssd.lib.ssd_bwd(ctypes.byref(_bwd_args(**kw)), None) == status
+
+
+def test_bwd_null_args_pointer():
+    assert ssd.lib.ssd_bwd(None, None) == ssd.SSD_ERR_INVALID_ARG
+    assert ssd.lib.ssd_bwd_workspace_size(None) == 0
+
+
+def test_bwd_workspace_size():
+    size = lambda **kw: ssd.lib.ssd_bwd_workspace_size(ctypes.byref(_bwd_args(**kw)))
+    assert size() > 0 and size() % 256 == 0
+    assert size(seqlen=200) > size()
+    assert size(batch=0) == 0 and size(headdim=300) == 0
+    # states per chunk dominate: b*H*ceil(L/Q)*P*N*4 bytes twice, plus dB and dC per head
+    b, L, H, P, N = 2, 100, 4, 64, 128
+    assert size(chunk_size=64) >= 2 * b * H * 2 * P * N * 4 + 2 * b * L * H * N * 4
+    assert size(chunk_size=16) > size(chunk_size=64)
+    # dstate 256 does not fit a 64-token chunk: the library halves it
+    assert size(dstate=256) == size(dstate=256, chunk_size=32)
+    assert size(dstate=256, chunk_size=64) == 0

@@ -1,0 +1,152 @@
+"""The backward kernels (``csrc/ssd_bwd.cuh``) run on the CPU through the
+test-only emulation in ``tests/emu`` and compared with the fp64 backward
+oracle, before any GPU runs them.
+
+The emulator compiles the kernels' own source with g++ under
+AddressSanitizer + UBSan (exact-size buffers: any access past an input,
+output, workspace or shared-memory buffer aborts) or ThreadSanitizer (real
+threads: a shared-memory race aborts), and fills outputs, workspace and
+shared memory with NaN first, so a value read before it was written shows up.
+Each block's threads also run in reverse order once, which exposes a missing
+barrier in the other direction.  Planted mistakes in a copy of the kernels
+must be caught.  The GPU parity tests (``test_zz_bwd_gpu.py``) run the same
+kernels compiled by nvcc."""
+import os
+import re
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+
+import emu_bwd
+from bwd_cases import CASES, KEYS, case_inputs, compare, dfinal_like, dy_like, inputs, oracle_bwd
+
+pytestmark = pytest.mark.skipif(not emu_bwd.available(), reason="g++ not available")
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_emulated_backward_matches_oracle(case):
+    name, (b, L, H, P, N, G), _, _, _, _, with_D, chunk = case
+    d, dy, dfinal = case_inputs(case)[:3]
+    out = emu_bwd.run(d, dy, dfinal, chunk_size=chunk)
+    assert out["status"] == 0
+    assert out["launches"] == 5
+    if name == "bf16_N256_chunk32":
+        assert out["chunk"] == 32  # 64 would not fit the shared memory of one CTA
+    elif chunk:
+        assert out["chunk"] == chunk
+    ref = oracle_bwd(d, dy, dfinal)
+    compare(out, ref)
+    if d["initial_states"] is None:
+        # the gradient at a zero initial state: the oracle's, with a zero h0 passed
+        d0 = dict(d, initial_states=torch.zeros(b, H, P, N))
+        assert np.allclose(out["dh0"], oracle_bwd(d0, dy, dfinal)["dh0"], rtol=1e-4, atol=1e-5)
+    if not with_D:
+        # dD is the gradient at D = 0: sum over rows and tokens of dy . x
+        want = np.einsum("blhp,blhp->h", dy.double().numpy(), d["x"].double().numpy())
+        assert np.allclose(out["dD"], want, rtol=1e-5, atol=1e-5)
+
+
+def test_reverse_thread_order_gives_the_same_bits():
+    d = inputs(2, 150, 4, 24, 40, 2, "f32", 0.3, seed=11)
+    dy = dy_like(2, 150, 4, 24, torch.float32, 5)
+    dfinal = dfinal_like(2, 4, 24, 40, 5)
+    fwd_order = emu_bwd.run(d, dy, dfinal)
+    rev_order = emu_bwd.run(d, dy, dfinal, reverse=True)
+    for k in KEYS:
+        assert np.array_equal(fwd_order[k], rev_order[k]), k
+
+
+def test_threads_under_thread_sanitizer():
+    d = inputs(1, 40, 2, 8, 16, 1, "f32", 0.3, seed=3)
+    dy = dy_like(1, 40, 2, 8, torch.float32, 3)
+    out = emu_bwd.run(d, dy, dfinal_like(1, 2, 8, 16, 3), chunk_size=16, kind="tsan")
+    assert out["status"] == 0
+    assert "ThreadSanitizer" not in out["stderr"]
+    compare(out, oracle_bwd(d, dy, dfinal_like(1, 2, 8, 16, 3)))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(headdim=257), 2),
+    (dict(dstate=300), 2),
+    (dict(chunk_size=65), 2),
+    (dict(chunk_size=-1), 1),
+    (dict(ngroups=3), 1),
+    (dict(seqlen=0), 1),
+])
+def test_emulated_plan_rejects(kw, status):
+    shp = dict(batch=1, seqlen=8, nheads=2, headdim=4, dstate=4, ngroups=1)
+    shp.update(kw)
+    x = torch.zeros(shp["batch"], max(shp["seqlen"], 1), shp["nheads"], shp["headdim"])
+    d = {"x": x, "dt": torch.zeros(x.shape[:3]), "A": torch.zeros(shp["nheads"]),
+         "B": torch.zeros(x.shape[0], x.shape[1], shp["ngroups"], shp["dstate"]),
+         "C": torch.zeros(x.shape[0], x.shape[1], shp["ngroups"], shp["dstate"]), "D": None}
+    # the driver reads sizes from args.txt: write the requested ones
+    out = _run_with_sizes(d, shp, kw.get("chunk_size", 0))
+    assert out == status
+
+
+def _run_with_sizes(d, shp, chunk):
+    exe = emu_bwd.build("asan")
+    with tempfile.TemporaryDirectory() as tmp:
+        for k in ("x", "dt", "A", "B", "C"):
+            d[k].numpy().tofile(os.path.join(tmp, k + ".bin"))
+        d["x"].numpy().tofile(os.path.join(tmp, "dy.bin"))
+        kv = dict(shp, chunk_size=chunk, dtype=0, has_D=0, has_h0=0, has_seq=0, has_dfinal=0, want_dD=0,
+                  want_dh0=0, reverse=0)
+        with open(os.path.join(tmp, "args.txt"), "w") as f:
+            f.write("".join(f"{k} {v}\n" for k, v in kv.items()))
+        r = subprocess.run([exe, tmp], capture_output=True, text=True, timeout=120,
+                           env=dict(os.environ, ASAN_OPTIONS="detect_leaks=0"))
+        return int(r.stdout.split()[1])
+
+
+def test_packed_with_dfinal_is_unsupported():
+    d = inputs(1, 32, 2, 4, 4, 1, "f32", packed=(4, 12), seed=2)
+    dy = dy_like(1, 32, 2, 4, torch.float32, 2)
+    assert emu_bwd.run(d, dy, dfinal_like(1, 2, 4, 4, 2))["status"] == 2
+
+
+# Planted mistakes in a copy of the kernels: each must make the emulated run
+# fail (sanitizer abort, non-finite output or a parity miss).
+MUTANTS = [
+    # a missing barrier between the Q x Q matrices and their use
+    ("drop_barrier", r"(    red\[tid\] = part;\n  }\n)  __syncthreads\(\);", r"\1"),
+    # the in-chunk sum of dx runs one token past the chunk
+    ("dx_past_chunk", r"for \(int t = s; t < Qc; \+\+t\) acc = fmaf", "for (int t = s; t <= Qc; ++t) acc = fmaf"),
+    # the adjoint carried across chunks skips the chunk decay
+    ("no_decay_backward", r"lam = fmaf\(dec\[c\], lam, u\);", "lam = lam + u;"),
+    # the row term of dcs loses dt
+    ("rowm_no_dt", r"rowm = fmaf\(Em\[t \* sQ \+ s\] \* w\[s\]", "rowm = fmaf(Em[t * sQ + s]"),
+    # the h_in term of dC is taken for every token
+    ("dC_hin_always", r"    if \(seg\[s\] == -1\) \{\n      float hy", "    if (true) {\n      float hy"),
+]
+
+
+@pytest.mark.parametrize("mutant", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_emulator_catches_planted_mistakes(mutant, monkeypatch):
+    name, pat, rep = mutant
+    src = open(emu_bwd.KERNELS).read()
+    bad, n = re.subn(pat, rep, src)
+    assert n == 1, f"mutant {name} did not apply"
+    with tempfile.TemporaryDirectory() as tmp:
+        os.makedirs(os.path.join(tmp, "k"))
+        with open(os.path.join(tmp, "k", "ssd_bwd.cuh"), "w") as f:
+            f.write(bad)
+        monkeypatch.setattr(emu_bwd, "KERNELS", os.path.join(tmp, "k", "ssd_bwd.cuh"))
+        monkeypatch.setattr(emu_bwd, "OUT", os.path.join(tmp, "out"))
+        d = inputs(2, 80, 2, 8, 16, 1, "f32", 0.5, packed=None, seed=9,
+                    lengths=[[20, 1, 30, 29], [40, 40]] if name == "dC_hin_always" else None)
+        dy = dy_like(2, 80, 2, 8, torch.float32, 9)
+        dfinal = None if name == "dC_hin_always" else dfinal_like(2, 2, 8, 16, 9)
+        ref = oracle_bwd(d, dy, dfinal)
+        caught = False
+        for reverse in (False, True):
+            try:
+                out = emu_bwd.run(d, dy, dfinal, chunk_size=16, reverse=reverse)
+                compare(out, ref)
+            except (AssertionError, RuntimeError):
+                caught = True
+        assert caught, f"mutant {name} survived"

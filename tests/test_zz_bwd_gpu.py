@@ -1,0 +1,83 @@
+"""Parity of the CUDA backward (``ssd_bwd``) with the fp64 backward oracle.
+
+The cases of the host emulation (``test_bwd_emu_cpu.py``) run here compiled
+by nvcc on the GPU, plus sizes only a GPU finishes quickly: a mid-size bf16
+problem and a packed one compared in full, and the benchmark's c1 layout
+(b 8, L 2048, H 80, P 64, N 128, bf16) at full size compared on one batch
+row: every gradient of a row except dA and dD depends on that row's inputs
+only, and dA, dD (sums over rows) are compared at the smaller sizes.  The
+file name sorts it after the forward's GPU files."""
+import numpy as np
+import pytest
+import torch
+
+import mamba_ssd_chunked_03_b200 as ssd
+import oracle
+from bwd_cases import CASES, KEYS, case_inputs, compare, dfinal_like, dy_like, inputs, oracle_bwd
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_bwd(d, dy, dfinal, chunk=0):
+    c = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    g = ssd.bwd(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], dy.cuda(), initial_states=c["initial_states"],
+                seq_idx=c.get("seq_idx"), dfinal_states=None if dfinal is None else dfinal.cuda(), chunk_size=chunk,
+                want_dD=True, want_dinitial_states=True)
+    torch.cuda.synchronize()
+    out = {k: (None if v is None else v.cpu().numpy()) for k, v in g.items()}
+    out["dh0"] = out.pop("dinitial_states")
+    return out
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_backward_matches_oracle(case):
+    d, dy, dfinal, chunk = case_inputs(case)
+    out = _gpu_bwd(d, dy, dfinal, chunk)
+    compare(out, oracle_bwd(d, dy, dfinal))
+    if d["initial_states"] is None:
+        b, H, P, N = d["x"].shape[0], d["x"].shape[2], d["x"].shape[3], d["B"].shape[3]
+        ref0 = oracle_bwd(dict(d, initial_states=torch.zeros(b, H, P, N)), dy, dfinal)
+        compare(out, ref0, keys=("dh0",))
+
+
+def test_backward_is_deterministic():
+    d, dy, dfinal, _ = case_inputs(CASES[1])
+    first = _gpu_bwd(d, dy, dfinal)
+    second = _gpu_bwd(d, dy, dfinal)
+    for k in KEYS:
+        assert np.array_equal(first[k], second[k]), k
+
+
+@pytest.mark.parametrize("packed", [False, True], ids=["dense", "packed"])
+def test_backward_mid_size(packed):
+    b, L, H, P, N, G = (2, 1024, 8, 64, 128, 1) if not packed else (2, 1024, 4, 64, 128, 2)
+    d = inputs(b, L, H, P, N, G, "bf16", h0=0.0 if packed else 0.2, packed=(32, 400) if packed else None, seed=77)
+    dy = dy_like(b, L, H, P, torch.bfloat16, 78)
+    dfinal = None if packed else dfinal_like(b, H, P, N, 79)
+    compare(_gpu_bwd(d, dy, dfinal), oracle_bwd(d, dy, dfinal))
+
+
+def test_backward_c1_layout_one_row():
+    b, L, H, P, N, G = 8, 2048, 80, 64, 128, 1
+    d = inputs(b, L, H, P, N, G, "bf16", h0=0.1, seed=1001)
+    dy = dy_like(b, L, H, P, torch.bfloat16, 5)
+    dfinal = dfinal_like(b, H, P, N, 6)
+    out = _gpu_bwd(d, dy, dfinal)
+    row = {k: (v[:1] if isinstance(v, torch.Tensor) and k not in ("A", "D") else v) for k, v in d.items()}
+    ref = oracle_bwd(row, dy[:1], dfinal[:1])
+    got = {k: out[k][:1] for k in ("dx", "ddt", "dB", "dC", "dh0")}
+    compare(got, ref, keys=("dx", "ddt", "dB", "dC", "dh0"))
+
+
+def test_autograd_function_routes_through_the_library():
+    d, dy, dfinal, _ = case_inputs(CASES[1])
+    c = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    leaves = {k: c[k].clone().requires_grad_(True) for k in ("x", "dt", "A", "B", "C", "D", "initial_states")}
+    y, fin = ssd.ssd_chunked(leaves["x"], leaves["dt"], leaves["A"], leaves["B"], leaves["C"], leaves["D"],
+                             chunk_size=64, initial_states=leaves["initial_states"])
+    loss = (y.double() * dy.cuda().double()).sum() + (fin.double() * dfinal.cuda().double()).sum()
+    loss.backward()
+    ref = oracle_bwd(d, dy, dfinal)
+    got = {"dx": leaves["x"].grad, "ddt": leaves["dt"].grad, "dA": leaves["A"].grad, "dB": leaves["B"].grad,
+           "dC": leaves["C"].grad, "dD": leaves["D"].grad, "dh0": leaves["initial_states"].grad}
+    compare({k: v.float().cpu().numpy() for k, v in got.items()}, ref)
