@@ -1,6 +1,8 @@
 /*
  * ssd.h -- C ABI of libssd, the chunked SSD (structured state space duality)
- * forward for NVIDIA B200 (sm_100a).
+ * forward for NVIDIA B200 (sm_100a), with its backward (ssd_bwd), the
+ * recurrent decode step, the state operations of sequence parallelism and
+ * the Mamba-2 block's conv1d + SiLU.
  *
  * What one call computes, per batch row b and head h, with group
  * g = h / (nheads / ngroups) (contiguous heads share B and C):
