@@ -597,11 +597,7 @@ def run_bwd(args, dist, dev, world, rank):
     g = {k: host[k].to(dev) for k in names}
     A, D = host["A"].to(dev), host["D"].to(dev)
     ws = torch.empty(ssd.bwd_workspace_size(g["x"], g["B"]), dtype=torch.uint8, device=dev)
-    pl = {"Q": 64}
-    for q in (64, 32, 16, 8):  # the library's own choice for chunk_size 0
-        if ssd.bwd_workspace_size(g["x"], g["B"], chunk_size=q) == ws.numel():
-            pl["Q"] = q
-            break
+    Q = ssd.bwd_chunk_size(g["x"], g["B"])  # the library's own choice
     K = args.steps
     events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for e0_, e1_ in events:  # torch creates an event on its first record
@@ -657,7 +653,7 @@ def run_bwd(args, dist, dev, world, rank):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev) / E
 
-    f_states, f_chunk = bwd_flops(b, L, H, P, N, pl["Q"])
+    f_states, f_chunk = bwd_flops(b, L, H, P, N, Q)
     achieved = f_chunk / (kernel_ms / 1e3) / 1e12
     tokens = b * L
     line = {
@@ -666,7 +662,7 @@ def run_bwd(args, dist, dev, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": BWD_WORKLOAD,
                    "l2": "no flush: inputs, gradients and the per-chunk states (GBs) exceed the 126 MB L2",
-                   "parallelism": "replicas" if world > 1 else "single GPU", "bwd_chunk": pl["Q"]},
+                   "parallelism": "replicas" if world > 1 else "single GPU", "bwd_chunk": Q},
         "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
                      "frac": achieved / FP32_PEAK_TFLOPS,
                      "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz",

@@ -331,6 +331,11 @@ typedef struct {
  * are read), or 0 if the sizes are invalid or unsupported. */
 SSD_API size_t ssd_bwd_workspace_size(const ssd_bwd_args* args);
 
+/* The chunk length ssd_bwd uses for these arguments (chunk_size, or the
+ * library's choice when it is 0), or 0 if the sizes are invalid or
+ * unsupported.  Reads only the size fields; no device work. */
+SSD_API int64_t ssd_bwd_chunk_size(const ssd_bwd_args* args);
+
 /* Enqueue the backward on `stream`: five kernels, no allocation, no memset.
  * All pointers are device pointers owned by the caller; outputs must not
  * overlap inputs or the workspace.  Returns SSD_OK once enqueued;

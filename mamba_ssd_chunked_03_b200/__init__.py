@@ -21,7 +21,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["fwd", "bwd", "BwdArgs", "ssd_chunked", "step", "StepArgs", "total_decay", "state_fold", "conv1d_silu", "ConvArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
+__all__ = ["fwd", "bwd", "BwdArgs", "bwd_workspace_size", "bwd_chunk_size", "ssd_chunked", "step", "StepArgs", "total_decay", "state_fold", "conv1d_silu", "ConvArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
            "SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED", "SSD_ERR_WORKSPACE", "SSD_ERR_CUDA",
            "SSD_F32", "SSD_BF16", "SSD_FLAG_GENERIC"]
 
@@ -110,6 +110,8 @@ def _load() -> ctypes.CDLL:
     L.ssd_bwd.restype = ctypes.c_int
     L.ssd_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs)]
     L.ssd_bwd_workspace_size.restype = ctypes.c_size_t
+    L.ssd_bwd_chunk_size.argtypes = [ctypes.POINTER(BwdArgs)]
+    L.ssd_bwd_chunk_size.restype = ctypes.c_int64
     L.ssd_conv1d_silu.argtypes = [ctypes.POINTER(ConvArgs), ctypes.c_void_p]
     L.ssd_conv1d_silu.restype = ctypes.c_int
     L.ssd_total_decay.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int64] * 3 + [
@@ -417,6 +419,12 @@ def bwd_workspace_size(x, B, chunk_size: int = 0) -> int:
     return int(lib.ssd_bwd_workspace_size(ctypes.byref(a)))
 
 
+def bwd_chunk_size(x, B, chunk_size: int = 0) -> int:
+    """The chunk length ``ssd_bwd`` uses for these shapes (0: not supported)."""
+    a = make_bwd_args(x, None, None, B, None, chunk_size=chunk_size)
+    return int(lib.ssd_bwd_chunk_size(ctypes.byref(a)))
+
+
 def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
         D: Optional[torch.Tensor], dy: torch.Tensor, initial_states: Optional[torch.Tensor] = None,
         seq_idx: Optional[torch.Tensor] = None, dfinal_states: Optional[torch.Tensor] = None,
@@ -449,8 +457,8 @@ def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     a.dx, a.ddt, a.dA, a.dB, a.dC = (_ptr(g[k]) for k in ("dx", "ddt", "dA", "dB", "dC"))
     a.dD, a.dinitial_states = _ptr(g["dD"]), _ptr(g["dinitial_states"])
     need = int(lib.ssd_bwd_workspace_size(ctypes.byref(a)))
-    if need == 0:
-        raise SSDError(SSD_ERR_UNSUPPORTED)
+    if need == 0:  # sizes the library rejects: let it say why (nothing is enqueued)
+        raise SSDError(lib.ssd_bwd(ctypes.byref(a), _stream(x)))
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()

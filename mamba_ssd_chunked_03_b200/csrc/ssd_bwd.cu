@@ -28,6 +28,11 @@ extern "C" SSD_API size_t ssd_bwd_workspace_size(const ssd_bwd_args* a) {
   return ssd::bwd::plan(a, &pl) == SSD_OK ? pl.total : 0;
 }
 
+extern "C" SSD_API int64_t ssd_bwd_chunk_size(const ssd_bwd_args* a) {
+  ssd::bwd::Plan pl;
+  return ssd::bwd::plan(a, &pl) == SSD_OK ? pl.d.Q : 0;
+}
+
 extern "C" SSD_API ssd_status ssd_bwd(const ssd_bwd_args* a, void* stream) {
   CudaLaunch launch{static_cast<cudaStream_t>(stream)};
   return ssd::bwd::run(a, launch);

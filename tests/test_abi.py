@@ -344,3 +344,13 @@ def test_bwd_workspace_size():
     # dstate 256 does not fit a 64-token chunk: the library halves it
     assert size(dstate=256) == size(dstate=256, chunk_size=32)
     assert size(dstate=256, chunk_size=64) == 0
+
+
+def test_bwd_chunk_size_query():
+    q = lambda **kw: ssd.lib.ssd_bwd_chunk_size(ctypes.byref(_bwd_args(**kw)))
+    assert q() == 64
+    assert q(chunk_size=16) == 16
+    assert q(dstate=256) == 32          # 64 would not fit one CTA's shared memory
+    assert q(dstate=256, headdim=256) == 32
+    assert q(chunk_size=65) == 0 and q(batch=0) == 0
+    assert ssd.lib.ssd_bwd_chunk_size(None) == 0

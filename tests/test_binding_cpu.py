@@ -58,3 +58,17 @@ def test_total_decay_and_fold_reject_cpu_tensors():
         ssd.total_decay(torch.zeros(1, 4, 2), torch.zeros(2))
     with pytest.raises(ValueError):
         ssd.state_fold(torch.zeros(2, 1, 2, 4, 4), torch.zeros(2, 1, 2), None, 1, (1, 2, 4, 4))
+
+
+def test_bwd_rejects_bad_arguments():
+    d = _fwd_args()
+    dy = torch.zeros_like(d["x"])
+    with pytest.raises(ValueError, match="CUDA"):
+        ssd.bwd(**d, dy=dy)  # CPU tensors
+    with pytest.raises(TypeError):
+        ssd.bwd(**_fwd_args(x=torch.zeros(1, 8, 2, 4, dtype=torch.float16)), dy=dy)
+
+
+def test_autograd_wrapper_rejects_cpu_tensors():
+    with pytest.raises(ValueError, match="CUDA"):
+        ssd.ssd_chunked(**_fwd_args())
