@@ -290,10 +290,13 @@ SSD_API ssd_status ssd_conv1d_silu(const ssd_conv_args* args, void* stream);
  * dtype.  Chunking re-associates the same sums, so the result equals the
  * adjoint recurrence up to rounding for every chunk size. */
 typedef struct {
-  /* sizes as in ssd_fwd_args; headdim and dstate at most 256.  chunk_size is
-   * the chunk length of the backward itself, unrelated to the forward's: 0
-   * lets the library choose (64, halved while its shared memory would not
-   * fit), or 1..64 (SSD_ERR_UNSUPPORTED if that does not fit). */
+  /* sizes as in ssd_fwd_args; headdim and dstate at most 256, and one
+   * headdim x dstate state must fit a CTA's shared memory next to an 8-token
+   * chunk (so not both 256).  chunk_size is the chunk length of the backward
+   * itself, unrelated to the forward's: 0 lets the library choose (64,
+   * halved while its shared memory would not fit: 32 for dstate 256 at
+   * headdim 64, 16 for 128 x 256), or 1..64 (SSD_ERR_UNSUPPORTED if that
+   * does not fit). */
   int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk_size;
   ssd_dtype dtype;                /* of x, B, C and dy                                */
   const void* x;                  /* (b,L,H,P) dtype                                  */

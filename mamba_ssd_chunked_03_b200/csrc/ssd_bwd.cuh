@@ -144,6 +144,67 @@ __device__ __forceinline__ void chunk_cumsum(const KArgs& a, const ChunkPos& q, 
   }
 }
 
+// ---- register-tiled products of small matrices in shared memory
+//
+// A thread owns a kT x kT block of an M x Nn product: rows r_i = tr + i TR and
+// columns c_j = tc + j TC (TR = ceil(M / kT), TC = ceil(Nn / kT)).  The
+// threads of a warp take consecutive tc, so they read consecutive columns of
+// one operand and the same few rows of the other (a broadcast); row strides
+// are padded where a column walk would otherwise meet one bank.  Indices past
+// the edge are clamped for loads, and their results are never stored.
+constexpr int kT = 4;
+
+struct Tile {
+  int tc;               // column-block index (the partial-sum slot of a row)
+  int r[kT], c[kT];     // clamped row and column indices
+  bool rv[kT], cv[kT];  // inside the product?
+};
+
+__device__ __forceinline__ int tiles_of(int M, int Nn) { return ((M + kT - 1) / kT) * ((Nn + kT - 1) / kT); }
+
+__device__ __forceinline__ Tile make_tile(int tile, int M, int Nn) {
+  const int TR = (M + kT - 1) / kT, TC = (Nn + kT - 1) / kT;
+  const int tr = tile / TC;
+  Tile t;
+  t.tc = tile % TC;
+#pragma unroll
+  for (int i = 0; i < kT; ++i) {
+    const int r = tr + i * TR;
+    t.rv[i] = r < M;
+    t.r[i] = r < M ? r : M - 1;
+    const int c = t.tc + i * TC;
+    t.cv[i] = c < Nn;
+    t.c[i] = c < Nn ? c : Nn - 1;
+  }
+  return t;
+}
+
+__device__ __forceinline__ void tile_zero(float (&acc)[kT][kT]) {
+#pragma unroll
+  for (int i = 0; i < kT; ++i)
+#pragma unroll
+    for (int j = 0; j < kT; ++j) acc[i][j] = 0.f;
+}
+
+// acc[i][j] += sum_{k0 <= k < k1} A(r_i, k) B(k, c_j), with A(m, k) = a[m am + k ak]
+// (times ks[k] when kScale) and B(k, n) = b[k bk + n bn].
+template <bool kScale>
+__device__ __forceinline__ void tile_mac(float (&acc)[kT][kT], const Tile& t, const float* a, int am, int ak,
+                                         const float* ks, const float* b, int bk, int bn, int k0, int k1) {
+  for (int k = k0; k < k1; ++k) {
+    float av[kT], bv[kT];
+    const float sk = kScale ? ks[k] : 1.f;
+#pragma unroll
+    for (int i = 0; i < kT; ++i) av[i] = kScale ? a[t.r[i] * am + k * ak] * sk : a[t.r[i] * am + k * ak];
+#pragma unroll
+    for (int j = 0; j < kT; ++j) bv[j] = b[k * bk + t.c[j] * bn];
+#pragma unroll
+    for (int i = 0; i < kT; ++i)
+#pragma unroll
+      for (int j = 0; j < kT; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+  }
+}
+
 // Shared-memory floats of k_bwd_chunk_states for chunk length Q.
 inline size_t smem_states_floats(int64_t Q, int64_t P, int64_t N) { return (size_t)(2 * Q * P + 2 * Q * N + 4 * Q); }
 
@@ -188,18 +249,26 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk_states(const KArgs a) {
   }
   if (tid == 0) a.dec[(q.b * d.H + q.h) * d.nc + q.c] = seg[Qc - 1] == -1 ? expf(cs[Qc - 1]) : 0.f;
   __syncthreads();
+  // S (P x N) = sum_t cS_t x_t B_t^T and T = sum_t cT_t dy_t C_t^T, over the chunk's tokens
   const int64_t off = ((q.b * d.H + q.h) * d.nc + q.c) * d.P * d.N;
   float* So = a.S + off;
   float* To = a.T + off;
-  for (int e = tid; e < P * N; e += kThreads) {
-    const int p = e / N, n = e % N;
-    float s = 0.f, u = 0.f;
-    for (int t = 0; t < Qc; ++t) {
-      s = fmaf(cS[t] * xs[t * P + p], Bs[t * N + n], s);
-      u = fmaf(cT[t] * dys[t * P + p], Cs[t * N + n], u);
-    }
-    So[e] = s;
-    To[e] = u;
+  const int nt = tiles_of(P, N);
+  for (int tile = tid; tile < nt; tile += kThreads) {
+    const Tile tl = make_tile(tile, P, N);
+    float s[kT][kT], u[kT][kT];
+    tile_zero(s);
+    tile_zero(u);
+    tile_mac<true>(s, tl, xs, 1, P, cS, Bs, N, 1, 0, Qc);
+    tile_mac<true>(u, tl, dys, 1, P, cT, Cs, N, 1, 0, Qc);
+#pragma unroll
+    for (int i = 0; i < kT; ++i)
+#pragma unroll
+      for (int j = 0; j < kT; ++j)
+        if (tl.rv[i] && tl.cv[j]) {
+          So[tl.r[i] * N + tl.c[j]] = s[i][j];
+          To[tl.r[i] * N + tl.c[j]] = u[i][j];
+        }
   }
 }
 
@@ -231,10 +300,18 @@ __global__ void __launch_bounds__(kThreads) k_bwd_state_passing(const KArgs a) {
   if (a.dh0) a.dh0[i] = lam;
 }
 
+// Columns of k_bwd_chunk's partial-sum array: one per column block of a
+// Q x P or Q x N product, and at least 8 (four row and four column quarters).
+__host__ __device__ inline int64_t part_cols(int64_t P, int64_t N) {
+  const int64_t m = ((P > N ? P : N) + kT - 1) / kT;
+  return m > 8 ? m : 8;
+}
+
 // Shared-memory floats of k_bwd_chunk for chunk length Q (rows padded by one
 // float so that column walks do not collide in a bank).
 inline size_t smem_chunk_floats(int64_t Q, int64_t P, int64_t N) {
-  return (size_t)(4 * Q * (P + 1) + 2 * Q * (N + 1) + 3 * Q * (Q + 1) + 6 * Q + kThreads);
+  return (size_t)(2 * Q * (P + 1) + 2 * Q * (N + 1) + P * (N + 1) + 3 * Q * (Q + 1) + Q * part_cols(P, N) +
+                  10 * Q + kThreads);
 }
 
 template <typename T>
@@ -242,21 +319,25 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
   const Dims& d = a.d;
   const ChunkPos q = chunk_pos(d, blockIdx.x);
   const int P = (int)d.P, N = (int)d.N, Q = (int)d.Q, Qc = q.Qc;
-  const int sP = P + 1, sN = N + 1, sQ = Q + 1;
+  const int sP = P + 1, sN = N + 1, sQ = Q + 1, PC = (int)part_cols(d.P, d.N);
   const int tid = threadIdx.x;
   SSD_DYN_SMEM(sm);
   float* xs = sm;             // Q x sP: x_t
   float* dys = xs + Q * sP;   // Q x sP: dy_t
-  float* LB = dys + Q * sP;   // Q x sP: (Lam B_s)_p
-  float* HC = LB + Q * sP;    // Q x sP: (h_in C_t)_p
-  float* Bs = HC + Q * sP;    // Q x sN
+  float* Bs = dys + Q * sP;   // Q x sN
   float* Cs = Bs + Q * sN;    // Q x sN
-  float* Em = Cs + Q * sN;    // Q x sQ: E(t,s)
-  float* CB = Em + Q * sQ;    // Q x sQ: C_t.B_s (s <= t)
-  float* XY = CB + Q * sQ;    // Q x sQ: dy_t.x_s (s <= t)
-  float* cs = XY + Q * sQ;    // Q
+  float* SB = Cs + Q * sN;    // P x sN: Lam, then h_in
+  float* Km = SB + P * sN;    // Q x sQ: E(t,s) C_t.B_s
+  float* Zm = Km + Q * sQ;    // Q x sQ: E(t,s) dy_t.x_s
+  float* Mm = Zm + Q * sQ;    // Q x sQ: E(t,s) (C_t.B_s)(dy_t.x_s)
+  float* part = Mm + Q * sQ;  // Q x PC: partial sums per row
+  float* cs = part + Q * PC;  // Q
   float* w = cs + Q;          // Q: dt
-  float* dw = w + Q;          // Q
+  float* el = w + Q;          // Q: E(last, s)
+  float* ein = el + Q;        // Q: e_t
+  float* dg = ein + Q;        // Q: dy_t.x_t
+  float* nv = dg + Q;         // Q: x_s^T Lam B_s
+  float* dw = nv + Q;         // Q
   float* dcs = dw + Q;        // Q
   float* nn = dcs + Q;        // Q: N_s
   float* red = nn + Q;        // kThreads
@@ -282,92 +363,158 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
     Bs[t * sN + n] = ld(B, gi);
     Cs[t * sN + n] = ld(C, gi);
   }
+  {
+    float part_lh = 0.f;  // <Lam, h_in>, this thread's share
+    for (int e = tid; e < P * N; e += kThreads) {
+      const float l = Lam[e];
+      SB[(e / N) * sN + e % N] = l;
+      part_lh = fmaf(l, Hin[e], part_lh);
+    }
+    red[tid] = part_lh;
+  }
   for (int t = tid; t < Qc; t += kThreads) w[t] = a.dt[(q.b * d.L + q.t0 + t) * d.H + q.h];
   if (tid == 0) chunk_cumsum(a, q, cs, seg);
   __syncthreads();
 
-  // the chunk's Q x Q matrices, lower triangle
-  for (int i = tid; i < Qc * Qc; i += kThreads) {
-    const int t = i / Qc, s = i % Qc;
-    float e = 0.f, cb = 0.f, xy = 0.f;
-    if (s <= t) {
-      if (seg[s] == seg[t]) e = expf(cs[t] - cs[s]);
-      for (int n = 0; n < N; ++n) cb = fmaf(Cs[t * sN + n], Bs[s * sN + n], cb);
-      for (int p = 0; p < P; ++p) xy = fmaf(dys[t * sP + p], xs[s * sP + p], xy);
-    }
-    Em[t * sQ + s] = e;
-    CB[t * sQ + s] = cb;
-    XY[t * sQ + s] = xy;
+  const int last = Qc - 1;
+  // the chunk's Q x Q matrices: C_t.B_s and dy_t.x_s, masked and decayed
+  for (int tile = tid; tile < tiles_of(Qc, Qc); tile += kThreads) {
+    const Tile tl = make_tile(tile, Qc, Qc);
+    float cb[kT][kT], xy[kT][kT];
+    tile_zero(cb);
+    tile_zero(xy);
+    tile_mac<false>(cb, tl, Cs, sN, 1, nullptr, Bs, 1, sN, 0, N);
+    tile_mac<false>(xy, tl, dys, sP, 1, nullptr, xs, 1, sP, 0, P);
+#pragma unroll
+    for (int i = 0; i < kT; ++i)
+#pragma unroll
+      for (int j = 0; j < kT; ++j) {
+        if (!tl.rv[i] || !tl.cv[j]) continue;
+        const int t = tl.r[i], s = tl.c[j];
+        const float e = (s <= t && seg[s] == seg[t]) ? expf(cs[t] - cs[s]) : 0.f;
+        Km[t * sQ + s] = e * cb[i][j];
+        Zm[t * sQ + s] = e * xy[i][j];
+        Mm[t * sQ + s] = e * cb[i][j] * xy[i][j];
+        if (s == t) dg[t] = xy[i][j];
+      }
   }
-  // Lam B_s and h_in C_t
-  for (int i = tid; i < P * Qc; i += kThreads) {
-    const int p = i / Qc, s = i % Qc;
-    float lb = 0.f, hc = 0.f;
-    for (int n = 0; n < N; ++n) {
-      lb = fmaf(Lam[p * N + n], Bs[s * sN + n], lb);
-      hc = fmaf(Hin[p * N + n], Cs[s * sN + n], hc);
-    }
-    LB[s * sP + p] = lb;
-    HC[s * sP + p] = hc;
-  }
-  // <Lam, h_in>, this thread's share
-  {
-    float part = 0.f;
-    for (int e = tid; e < P * N; e += kThreads) part = fmaf(Lam[e], Hin[e], part);
-    red[tid] = part;
+  for (int t = tid; t < Qc; t += kThreads) {
+    el[t] = seg[t] == seg[last] ? expf(cs[last] - cs[t]) : 0.f;
+    ein[t] = seg[t] == -1 ? expf(cs[t]) : 0.f;
   }
   __syncthreads();
 
-  const int last = Qc - 1;
   const float Dh = a.D ? a.D[q.h] : 0.f;
-  // dx
-  for (int i = tid; i < Qc * P; i += kThreads) {
-    const int s = i / P, p = i % P;
-    float acc = 0.f;
-    for (int t = s; t < Qc; ++t) acc = fmaf(Em[t * sQ + s] * CB[t * sQ + s], dys[t * sP + p], acc);
-    acc = fmaf(Em[last * sQ + s], LB[s * sP + p], acc);
-    a.dx[((q.b * d.L + q.t0 + s) * d.H + q.h) * d.P + p] = fmaf(w[s], acc, Dh * dys[s * sP + p]);
-  }
-  // dB and dC of this head
-  for (int i = tid; i < Qc * N; i += kThreads) {
-    const int s = i / N, n = i % N;
-    float accB = 0.f;
-    for (int t = s; t < Qc; ++t) accB = fmaf(Em[t * sQ + s] * XY[t * sQ + s], Cs[t * sN + n], accB);
-    float lx = 0.f;
-    for (int p = 0; p < P; ++p) lx = fmaf(Lam[p * N + n], xs[s * sP + p], lx);
-    accB = fmaf(Em[last * sQ + s], lx, accB);
-    float accC = 0.f;
-    for (int r = 0; r <= s; ++r) accC = fmaf(Em[s * sQ + r] * w[r] * XY[s * sQ + r], Bs[r * sN + n], accC);
-    if (seg[s] == -1) {
-      float hy = 0.f;
-      for (int p = 0; p < P; ++p) hy = fmaf(Hin[p * N + n], dys[s * sP + p], hy);
-      accC = fmaf(expf(cs[s]), hy, accC);
+  // dx (Q x P): w_s [sum_t K(t,s) dy_t + E(last,s) Lam B_s] + D dy_s; with the
+  // row partials of x_s . (Lam B_s)
+  for (int tile = tid; tile < tiles_of(Qc, P); tile += kThreads) {
+    const Tile tl = make_tile(tile, Qc, P);
+    float acc[kT][kT], lb[kT][kT];
+    tile_zero(acc);
+    tile_zero(lb);
+    tile_mac<false>(acc, tl, Km, 1, sQ, nullptr, dys, sP, 1, tl.r[0], Qc);
+    tile_mac<false>(lb, tl, Bs, sN, 1, nullptr, SB, 1, sN, 0, N);
+#pragma unroll
+    for (int i = 0; i < kT; ++i) {
+      if (!tl.rv[i]) continue;
+      const int s = tl.r[i];
+      float nx = 0.f;
+#pragma unroll
+      for (int j = 0; j < kT; ++j) {
+        if (!tl.cv[j]) continue;
+        const int p = tl.c[j];
+        a.dx[((q.b * d.L + q.t0 + s) * d.H + q.h) * d.P + p] =
+            fmaf(w[s], fmaf(el[s], lb[i][j], acc[i][j]), Dh * dys[s * sP + p]);
+        nx = fmaf(xs[s * sP + p], lb[i][j], nx);
+      }
+      part[s * PC + tl.tc] = nx;
     }
-    const int64_t gi = ((q.b * d.L + q.t0 + s) * d.H + q.h) * d.N + n;
-    a.dBh[gi] = w[s] * accB;
-    a.dCh[gi] = accC;
   }
-  // per token: dw and dcs (before the last token's extra terms)
+  // dB of this head (Q x N): w_s [sum_t Z(t,s) C_t + E(last,s) Lam^T x_s]
+  for (int tile = tid; tile < tiles_of(Qc, N); tile += kThreads) {
+    const Tile tl = make_tile(tile, Qc, N);
+    float bi[kT][kT], bl[kT][kT];
+    tile_zero(bi);
+    tile_zero(bl);
+    tile_mac<false>(bi, tl, Zm, 1, sQ, nullptr, Cs, sN, 1, tl.r[0], Qc);
+    tile_mac<false>(bl, tl, xs, sP, 1, nullptr, SB, sN, 1, 0, P);
+#pragma unroll
+    for (int i = 0; i < kT; ++i)
+#pragma unroll
+      for (int j = 0; j < kT; ++j)
+        if (tl.rv[i] && tl.cv[j]) {
+          const int s = tl.r[i];
+          a.dBh[((q.b * d.L + q.t0 + s) * d.H + q.h) * d.N + tl.c[j]] = w[s] * fmaf(el[s], bl[i][j], bi[i][j]);
+        }
+  }
+  __syncthreads();
+
+  const int tcp = (P + kT - 1) / kT;
+  for (int s = tid; s < Qc; s += kThreads) {
+    float v = 0.f;
+    for (int k = 0; k < tcp; ++k) v += part[s * PC + k];
+    nv[s] = v;
+  }
+  for (int e = tid; e < P * N; e += kThreads) SB[(e / N) * sN + e % N] = Hin[e];
+  __syncthreads();
+
+  // dC of this head (Q x N): sum_s Z(t,s) w_s B_s + e_t h_in^T dy_t; with the
+  // row partials of C_t . (h_in^T dy_t)
+  for (int tile = tid; tile < tiles_of(Qc, N); tile += kThreads) {
+    const Tile tl = make_tile(tile, Qc, N);
+    int kmax = 0;
+#pragma unroll
+    for (int i = 0; i < kT; ++i)
+      if (tl.rv[i]) kmax = tl.r[i] + 1;
+    float ci[kT][kT], ch[kT][kT];
+    tile_zero(ci);
+    tile_zero(ch);
+    tile_mac<true>(ci, tl, Zm, sQ, 1, w, Bs, sN, 1, 0, kmax);
+    tile_mac<false>(ch, tl, dys, sP, 1, nullptr, SB, sN, 1, 0, P);
+#pragma unroll
+    for (int i = 0; i < kT; ++i) {
+      if (!tl.rv[i]) continue;
+      const int t = tl.r[i];
+      float cy = 0.f;
+#pragma unroll
+      for (int j = 0; j < kT; ++j) {
+        if (!tl.cv[j]) continue;
+        const int n = tl.c[j];
+        a.dCh[((q.b * d.L + q.t0 + t) * d.H + q.h) * d.N + n] = fmaf(ein[t], ch[i][j], ci[i][j]);
+        cy = fmaf(Cs[t * sN + n], ch[i][j], cy);
+      }
+      part[t * PC + tl.tc] = cy;
+    }
+  }
+  __syncthreads();
+
+  // per token: the h_in term of dcs (kept in dcs for now), then the row and
+  // column sums of M in quarters, four threads per token
+  const int tcn = (N + kT - 1) / kT;
   for (int t = tid; t < Qc; t += kThreads) {
-    float nx = 0.f;
-    for (int p = 0; p < P; ++p) nx = fmaf(xs[t * sP + p], LB[t * sP + p], nx);
-    float y0 = 0.f;
-    if (seg[t] == -1) {
-      for (int p = 0; p < P; ++p) y0 = fmaf(dys[t * sP + p], HC[t * sP + p], y0);
-      y0 *= expf(cs[t]);
+    float v = 0.f;
+    for (int k = 0; k < tcn; ++k) v += part[t * PC + k];
+    dcs[t] = ein[t] * v;
+  }
+  __syncthreads();
+  for (int i = tid; i < 4 * Qc; i += kThreads) {
+    const int t = i >> 2, qq = i & 3;
+    const int lo = Qc * qq / 4, hi = Qc * (qq + 1) / 4;
+    float col = 0.f, row = 0.f;
+    for (int u = lo; u < hi; ++u) {
+      if (u > t) col += Mm[u * sQ + t];
+      if (u < t) row = fmaf(Mm[t * sQ + u], w[u], row);
     }
-    float dwt = 0.f, colm = 0.f;
-    for (int u = t; u < Qc; ++u) {
-      const float m = Em[u * sQ + t] * CB[u * sQ + t] * XY[u * sQ + t];
-      dwt += m;
-      if (u > t) colm += m;
-    }
-    float rowm = 0.f;
-    for (int s = 0; s < t; ++s) rowm = fmaf(Em[t * sQ + s] * w[s], CB[t * sQ + s] * XY[t * sQ + s], rowm);
-    const float el = Em[last * sQ + t];
-    dw[t] = fmaf(el, nx, dwt);
-    nn[t] = el * w[t] * nx;
-    dcs[t] = rowm - w[t] * colm + y0 - nn[t];
+    part[t * PC + qq] = col;
+    part[t * PC + 4 + qq] = row;
+  }
+  __syncthreads();
+  for (int t = tid; t < Qc; t += kThreads) {
+    const float col = part[t * PC] + part[t * PC + 1] + part[t * PC + 2] + part[t * PC + 3];
+    const float row = part[t * PC + 4] + part[t * PC + 5] + part[t * PC + 6] + part[t * PC + 7];
+    dw[t] = fmaf(el[t], nv[t], col + Mm[t * sQ + t]);
+    nn[t] = el[t] * w[t] * nv[t];
+    dcs[t] = row - w[t] * col + dcs[t] - nn[t];
   }
   __syncthreads();
 
@@ -387,7 +534,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
       const float dl = seg[k] == k ? 0.f : run;  // a segment's first token has no decay
       a.ddt[(q.b * d.L + q.t0 + k) * d.H + q.h] = fmaf(Ah, dl, dw[k]);
       dA += (double)w[k] * (double)dl;
-      dD += (double)XY[k * sQ + k];
+      dD += (double)dg[k];
     }
     const int64_t pi = q.h * (d.b * d.nc) + q.b * d.nc + q.c;
     a.dA_part[pi] = dA;

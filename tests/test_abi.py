@@ -351,6 +351,7 @@ def test_bwd_chunk_size_query():
     assert q() == 64
     assert q(chunk_size=16) == 16
     assert q(dstate=256) == 32          # 64 would not fit one CTA's shared memory
-    assert q(dstate=256, headdim=256) == 32
+    assert q(dstate=256, headdim=128) == 16
+    assert q(dstate=256, headdim=256) == 0  # one 256 x 256 state alone exceeds a CTA's shared memory
     assert q(chunk_size=65) == 0 and q(batch=0) == 0
     assert ssd.lib.ssd_bwd_chunk_size(None) == 0

@@ -113,15 +113,17 @@ def test_packed_with_dfinal_is_unsupported():
 # fail (sanitizer abort, non-finite output or a parity miss).
 MUTANTS = [
     # a missing barrier between the Q x Q matrices and their use
-    ("drop_barrier", r"(    red\[tid\] = part;\n  }\n)  __syncthreads\(\);", r"\1"),
+    ("drop_barrier", r"(    ein\[t\] = seg\[t\] == -1 \? expf\(cs\[t\]\) : 0\.f;\n  }\n)  __syncthreads\(\);", r"\1"),
     # the in-chunk sum of dx runs one token past the chunk
-    ("dx_past_chunk", r"for \(int t = s; t < Qc; \+\+t\) acc = fmaf", "for (int t = s; t <= Qc; ++t) acc = fmaf"),
+    ("dx_past_chunk", r"(tile_mac<false>\(acc, tl, Km, 1, sQ, nullptr, dys, sP, 1, tl\.r\[0\], )Qc\);", r"\1Qc + 1);"),
     # the adjoint carried across chunks skips the chunk decay
     ("no_decay_backward", r"lam = fmaf\(dec\[c\], lam, u\);", "lam = lam + u;"),
     # the row term of dcs loses dt
-    ("rowm_no_dt", r"rowm = fmaf\(Em\[t \* sQ \+ s\] \* w\[s\]", "rowm = fmaf(Em[t * sQ + s]"),
-    # the h_in term of dC is taken for every token
-    ("dC_hin_always", r"    if \(seg\[s\] == -1\) \{\n      float hy", "    if (true) {\n      float hy"),
+    ("rowm_no_dt", r"row = fmaf\(Mm\[t \* sQ \+ u\], w\[u\], row\);", "row += Mm[t * sQ + u];"),
+    # the h_in terms are taken for every token, also after a sequence boundary
+    ("hin_always", r"ein\[t\] = seg\[t\] == -1 \? expf\(cs\[t\]\) : 0\.f;", "ein[t] = expf(cs[t]);"),
+    # tiles numbered with the wrong divisor: parts of a non-square product are never written
+    ("tile_index", r"const int tr = tile / TC;", "const int tr = tile / TR;"),
 ]
 
 
@@ -138,9 +140,9 @@ def test_emulator_catches_planted_mistakes(mutant, monkeypatch):
         monkeypatch.setattr(emu_bwd, "KERNELS", os.path.join(tmp, "k", "ssd_bwd.cuh"))
         monkeypatch.setattr(emu_bwd, "OUT", os.path.join(tmp, "out"))
         d = inputs(2, 80, 2, 8, 16, 1, "f32", 0.5, packed=None, seed=9,
-                    lengths=[[20, 1, 30, 29], [40, 40]] if name == "dC_hin_always" else None)
+                    lengths=[[20, 1, 30, 29], [40, 40]] if name == "hin_always" else None)
         dy = dy_like(2, 80, 2, 8, torch.float32, 9)
-        dfinal = None if name == "dC_hin_always" else dfinal_like(2, 2, 8, 16, 9)
+        dfinal = None if name == "hin_always" else dfinal_like(2, 2, 8, 16, 9)
         ref = oracle_bwd(d, dy, dfinal)
         caught = False
         for reverse in (False, True):
