@@ -146,12 +146,14 @@ __device__ __forceinline__ void chunk_cumsum(const KArgs& a, const ChunkPos& q, 
 
 // ---- register-tiled products of small matrices in shared memory
 //
-// A thread owns a kT x kT block of an M x Nn product: rows r_i = tr + i TR and
-// columns c_j = tc + j TC (TR = ceil(M / kT), TC = ceil(Nn / kT)).  The
+// A thread owns a kT x kT block of an M x Nn product: rows r_i = kT tr + i and
+// columns c_j = tc + j TC (TC = ceil(Nn / kT)), with tile = tr TC + tc.  The
 // threads of a warp take consecutive tc, so they read consecutive columns of
 // one operand and the same few rows of the other (a broadcast); row strides
-// are padded where a column walk would otherwise meet one bank.  Indices past
-// the edge are clamped for loads, and their results are never stored.
+// are padded where a column walk would otherwise meet one bank.  Contiguous
+// rows let a triangular product stop at the thread's own first or last row.
+// Indices past the edge are clamped for loads, and their results are never
+// stored.
 constexpr int kT = 4;
 
 struct Tile {
@@ -163,13 +165,13 @@ struct Tile {
 __device__ __forceinline__ int tiles_of(int M, int Nn) { return ((M + kT - 1) / kT) * ((Nn + kT - 1) / kT); }
 
 __device__ __forceinline__ Tile make_tile(int tile, int M, int Nn) {
-  const int TR = (M + kT - 1) / kT, TC = (Nn + kT - 1) / kT;
+  const int TC = (Nn + kT - 1) / kT;
   const int tr = tile / TC;
   Tile t;
   t.tc = tile % TC;
 #pragma unroll
   for (int i = 0; i < kT; ++i) {
-    const int r = tr + i * TR;
+    const int r = tr * kT + i;
     t.rv[i] = r < M;
     t.r[i] = r < M ? r : M - 1;
     const int c = t.tc + i * TC;

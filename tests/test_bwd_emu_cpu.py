@@ -123,7 +123,7 @@ MUTANTS = [
     # the h_in terms are taken for every token, also after a sequence boundary
     ("hin_always", r"ein\[t\] = seg\[t\] == -1 \? expf\(cs\[t\]\) : 0\.f;", "ein[t] = expf(cs[t]);"),
     # tiles numbered with the wrong divisor: parts of a non-square product are never written
-    ("tile_index", r"const int tr = tile / TC;", "const int tr = tile / TR;"),
+    ("tile_index", r"const int tr = tile / TC;", "const int tr = tile / (TC + 1);"),
 ]
 
 
