@@ -16,6 +16,20 @@ That is the state passing of "SSM 家族全景图（下）：Mamba-2 与 Jamba" 
 kernels; this module only calls them and moves the states between ranks.
 Packed sequences (seq_idx) are not split this way.
 
+The backward (``bwd_seqpar``) is the same exchange run the other way.  The
+gradient with respect to the state entering rank k's range is
+D_k Lam_k + T_k, where Lam_k is the gradient with respect to the state
+leaving it and T_k comes from the range's own outputs alone (the backward's
+dinitial_states when no state gradient comes in).  So:
+
+1. every rank recovers h_in as in the forward, and runs its backward without
+   an incoming state gradient: T_k;
+2. the ranks all-gather (T_k, D_k);
+3. rank r folds Lam_r from the sequence's dfinal through ranks R-1..r+1
+   (``ssd_state_fold`` over the reversed lists) and runs its backward again
+   with h_in and Lam_r, which gives its tokens' gradients;
+4. dA and dD, which sum over all tokens, are all-reduced.
+
 The three per-rank operations are taken from ``ops`` (default: the library),
 so the exchange logic can be exercised on CPU ranks with another
 implementation of them.
@@ -26,7 +40,7 @@ from typing import Optional
 
 import torch
 
-from . import fwd, state_fold, total_decay
+from . import bwd, fwd, state_fold, total_decay
 
 
 class LibraryOps:
@@ -44,6 +58,11 @@ class LibraryOps:
     def state_fold(states, decays, initial_states, rank, shape):
         return state_fold(states, decays, initial_states, rank, shape)
 
+    @staticmethod
+    def local_backward(x, dt, A, B, C, D, dy, initial_states, dfinal_states):
+        return bwd(x, dt, A, B, C, D, dy, initial_states=initial_states, dfinal_states=dfinal_states,
+                   want_dD=D is not None, want_dinitial_states=True)
+
 
 def local_summary(x, dt, A, B, C, D, chunk_size: int = 64, ops=LibraryOps):
     """(S, D_total) of this rank's range: its end state from a zero state and
@@ -58,13 +77,8 @@ def carry_in(states, decays, initial_states, rank: int, shape, ops=LibraryOps):
     return ops.state_fold(states, decays, initial_states, rank, shape)
 
 
-def fwd_seqpar(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
-               D: Optional[torch.Tensor], chunk_size: int = 64, initial_states: Optional[torch.Tensor] = None,
-               group=None, ops=LibraryOps):
-    """The forward of this rank's token range of a sequence split over the
-    ranks of ``group``, in rank order.  ``initial_states`` (the state before
-    the sequence's first token, or None) must be the same on every rank.
-    Returns (y of this rank's tokens, the state at the end of its range)."""
+def _state_in(x, dt, A, B, C, D, chunk_size, initial_states, group, ops):
+    """(h_in of this rank, the gathered total decays (R,b,H), the state shape)."""
     import torch.distributed as dist
     R = dist.get_world_size(group)
     r = dist.get_rank(group)
@@ -73,5 +87,45 @@ def fwd_seqpar(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tens
     all_d = [torch.empty_like(dec) for _ in range(R)]
     dist.all_gather(all_S, S.contiguous(), group=group)
     dist.all_gather(all_d, dec.contiguous(), group=group)
-    h_in = carry_in(torch.stack(all_S), torch.stack(all_d), initial_states, r, tuple(S.shape), ops)
+    decays = torch.stack(all_d)
+    return carry_in(torch.stack(all_S), decays, initial_states, r, tuple(S.shape), ops), decays, tuple(S.shape)
+
+
+def fwd_seqpar(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+               D: Optional[torch.Tensor], chunk_size: int = 64, initial_states: Optional[torch.Tensor] = None,
+               group=None, ops=LibraryOps):
+    """The forward of this rank's token range of a sequence split over the
+    ranks of ``group``, in rank order.  ``initial_states`` (the state before
+    the sequence's first token, or None) must be the same on every rank.
+    Returns (y of this rank's tokens, the state at the end of its range)."""
+    h_in, _, _ = _state_in(x, dt, A, B, C, D, chunk_size, initial_states, group, ops)
     return ops.local_forward(x, dt, A, B, C, D, chunk_size, h_in)
+
+
+def bwd_seqpar(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+               D: Optional[torch.Tensor], dy: torch.Tensor, chunk_size: int = 64,
+               initial_states: Optional[torch.Tensor] = None, dfinal_states: Optional[torch.Tensor] = None,
+               group=None, ops=LibraryOps) -> dict:
+    """The backward of ``fwd_seqpar`` for this rank's token range.  ``dy`` is
+    dLoss/dy of this rank's tokens; ``initial_states`` and ``dfinal_states``
+    (dLoss/d(the sequence's final state)), each None or the same on every
+    rank.  Returns a dict: dx, ddt, dB, dC of this rank's tokens; dA and dD
+    summed over all ranks; dinitial_states on rank 0 (None elsewhere)."""
+    import torch.distributed as dist
+    R = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    h_in, decays, shape = _state_in(x, dt, A, B, C, D, chunk_size, initial_states, group, ops)
+    T = ops.local_backward(x, dt, A, B, C, D, dy, h_in, None)["dinitial_states"]
+    all_T = [torch.empty_like(T) for _ in range(R)]
+    dist.all_gather(all_T, T.contiguous(), group=group)
+    after = list(range(R - 1, r, -1))  # the ranks after this one, last first
+    lam = ops.state_fold(torch.stack([all_T[k] for k in after]) if after else None,
+                         torch.stack([decays[k] for k in after]) if after else None,
+                         dfinal_states, len(after), shape)
+    g = ops.local_backward(x, dt, A, B, C, D, dy, h_in, lam)
+    dist.all_reduce(g["dA"], group=group)
+    if g.get("dD") is not None:
+        dist.all_reduce(g["dD"], group=group)
+    if r != 0:
+        g["dinitial_states"] = None
+    return g

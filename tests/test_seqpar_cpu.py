@@ -1,7 +1,7 @@
 """Sequence parallelism on the CPU: the composition rule the split relies on,
-pinned on the oracle, and the exchange logic of ``seqpar.fwd_seqpar`` on two
-gloo ranks (with the per-rank operations done by the oracle, since these
-ranks have no GPU).
+pinned on the oracle, and the exchange logic of ``seqpar.fwd_seqpar`` and
+``seqpar.bwd_seqpar`` on two and three gloo ranks (with the per-rank
+operations done by the oracle, since these ranks have no GPU).
 
 The rule: over a contiguous token range the recurrence is affine in the
 state, h_out = D h_in + S, with S the range's end state from a zero state and
@@ -50,6 +50,15 @@ class OracleOps:
         for k in range(rank):
             h = decays[k].double()[:, :, None, None] * h + states[k].double()
         return h.float()
+
+    @staticmethod
+    def local_backward(x, dt, A, B, C, D, dy, initial_states, dfinal_states):
+        b, _, H, P = x.shape
+        h0 = initial_states if initial_states is not None else torch.zeros(b, H, P, B.shape[3])
+        g = oracle.ssd_bwd(x, dt, A, B, C, D, h0, dy, dfinal_states, None)
+        out = {k: (None if v is None else torch.from_numpy(v).float()) for k, v in g.items() if k != "dh0"}
+        out["dinitial_states"] = torch.from_numpy(g["dh0"]).float()
+        return out
 
 
 @pytest.mark.parametrize("cuts", [[0, 90, 91, 200], [0, 64, 128, 200], [0, 200]])
@@ -116,3 +125,55 @@ def test_fwd_seqpar_gloo_ranks(cuts):
         y = np.concatenate([out[r][0] for r in range(world)], axis=1)
         assert np.abs(y - yw).max() <= 1e-5 * max(1.0, np.abs(yw).max())
         assert np.abs(out[world - 1][1] - fw).max() <= 1e-5 * max(1.0, np.abs(fw).max())
+
+
+def _bwd_data():
+    shape = si.SSDShape("sp", 2, 200, 3, 8, 8, 1, 64, "f32", h0_std=0.5, seed=5)
+    d = si.make_inputs(shape)
+    g = torch.Generator().manual_seed(21)
+    dy = torch.randn(2, 200, 3, 8, generator=g)
+    dfinal = torch.randn(2, 3, 8, 8, generator=g)
+    return d, dy, dfinal
+
+
+def _bwd_rank_main(rank, world, port, cuts, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from mamba_ssd_chunked_03_b200 import seqpar
+        d, dy, dfinal = _bwd_data()
+        lo, hi = cuts[rank], cuts[rank + 1]
+        p = _split(d, lo, hi)
+        g = seqpar.bwd_seqpar(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], dy[:, lo:hi].contiguous(), 64,
+                              d["initial_states"], dfinal, ops=OracleOps)
+        out[rank] = {k: (None if v is None else v.numpy()) for k, v in g.items()}
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("cuts", [[0, 117, 200], [0, 64, 65, 200]], ids=["2_ranks", "3_ranks"])
+def test_bwd_seqpar_gloo_ranks(cuts):
+    world = len(cuts) - 1
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_bwd_rank_main, args=(r, world, port, cuts, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(180)
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        d, dy, dfinal = _bwd_data()
+        ref = oracle.ssd_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["initial_states"], dy, dfinal, None)
+        tol = lambda w: 1e-5 * max(1.0, np.abs(w).max())
+        for k in ("dx", "ddt", "dB", "dC"):
+            got = np.concatenate([out[r][k] for r in range(world)], axis=1)
+            assert np.abs(got - ref[k]).max() <= tol(ref[k]), k
+        for r in range(world):  # the shared parameters: every rank holds the sum
+            assert np.abs(out[r]["dA"] - ref["dA"]).max() <= tol(ref["dA"])
+            assert np.abs(out[r]["dD"] - ref["dD"]).max() <= tol(ref["dD"])
+        assert np.abs(out[0]["dinitial_states"] - ref["dh0"]).max() <= tol(ref["dh0"])
+        assert all(out[r]["dinitial_states"] is None for r in range(1, world))

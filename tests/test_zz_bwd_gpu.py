@@ -81,3 +81,44 @@ def test_autograd_function_routes_through_the_library():
     got = {"dx": leaves["x"].grad, "ddt": leaves["dt"].grad, "dA": leaves["A"].grad, "dB": leaves["B"].grad,
            "dC": leaves["C"].grad, "dD": leaves["D"].grad, "dh0": leaves["initial_states"].grad}
     compare({k: v.float().cpu().numpy() for k, v in got.items()}, ref)
+
+
+@pytest.mark.parametrize("cuts", [[0, 333, 700], [0, 64, 65, 700]], ids=["2_ranks", "3_ranks"])
+def test_simulated_seqpar_backward_matches_the_whole_sequence(cuts):
+    """The exchange of ``seqpar.bwd_seqpar`` with the library's kernels, ranks
+    simulated in one process (gathers done by stacking).  The states crossing
+    ranks come from the fp32 forward, so the bound is ten times the
+    single-call one."""
+    from mamba_ssd_chunked_03_b200 import seqpar
+    import ssd_inputs as si
+    b, L, H, P, N = 2, 700, 4, 64, 128
+    d = si.make_inputs(si.SSDShape("split_bwd", b, L, H, P, N, 2, 64, "f32", h0_std=0.3, seed=23))
+    dy = dy_like(b, L, H, P, torch.float32, 31)
+    dfinal = dfinal_like(b, H, P, N, 31)
+    ref = oracle_bwd(d, dy, dfinal)
+    g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    ops = seqpar.LibraryOps
+    spans = list(zip(cuts[:-1], cuts[1:]))
+    parts = [{k: (g[k][:, lo:hi].contiguous() if k in ("x", "dt", "B", "C") else g[k]) for k in g} for lo, hi in spans]
+    dys = [dy[:, lo:hi].contiguous().cuda() for lo, hi in spans]
+    summ = [seqpar.local_summary(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], 64) for p in parts]
+    S, Dk = torch.stack([s for s, _ in summ]), torch.stack([k for _, k in summ])
+    shape = (b, H, P, N)
+    h_in = [seqpar.carry_in(S, Dk, g["initial_states"], r, shape) for r in range(len(parts))]
+    T = [ops.local_backward(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], dys[r], h_in[r], None)["dinitial_states"]
+         for r, p in enumerate(parts)]
+    R = len(parts)
+    out = []
+    for r, p in enumerate(parts):
+        after = list(range(R - 1, r, -1))
+        lam = ops.state_fold(torch.stack([T[k] for k in after]) if after else None,
+                             torch.stack([Dk[k] for k in after]) if after else None, dfinal.cuda(), len(after), shape)
+        out.append(ops.local_backward(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], dys[r], h_in[r], lam))
+    torch.cuda.synchronize()
+    got = {k: torch.cat([o[k] for o in out], dim=1).cpu().numpy() for k in ("dx", "ddt", "dB", "dC")}
+    got["dA"] = sum(o["dA"] for o in out).cpu().numpy()
+    got["dD"] = sum(o["dD"] for o in out).cpu().numpy()
+    got["dh0"] = out[0]["dinitial_states"].cpu().numpy()
+    for k, v in got.items():
+        rel = np.linalg.norm(v - ref[k]) / np.linalg.norm(ref[k])
+        assert rel <= 1e-4, (k, rel)
