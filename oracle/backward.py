@@ -26,6 +26,12 @@ Backward, with G_t = dLoss/dh_t (P x N) swept from the last token:
 where <., .> sums over all entries.  A reset token (a_t = 0) passes no
 gradient to h_{t-1}, dt_t's decay term or A.  Plain fp64 numpy, token by token
 (the states are recomputed first, as the pages describe), for small inputs.
+
+With the Mamba-2 block's gate ("SSM 家族全景图（下）：Mamba-2 与 Jamba",
+section 5) the output is out = y * SiLU(z), SiLU(v) = v / (1 + e^-v).  Given
+dout, the gate's own gradient is dz = dout * y * SiLU'(z), with
+SiLU'(v) = s (1 + v (1 - s)) and s = 1 / (1 + e^-v), and the SSD receives
+dy = dout * SiLU(z) (``ssd_bwd_gated``).
 """
 from __future__ import annotations
 
@@ -34,6 +40,15 @@ from typing import Optional
 import numpy as np
 
 from . import as_f64, as_i32
+
+
+def _upstream(a):
+    """An upstream gradient at the precision given: fp64 arrays as they are
+    (a gradient formed in fp64, such as the gate's dout * SiLU(z)), anything
+    else widened through fp32 like the inputs."""
+    if isinstance(a, np.ndarray) and a.dtype == np.float64:
+        return np.ascontiguousarray(a)
+    return as_f64(a)
 
 
 def ssd_bwd(x, dt, A, B, C, D, initial_states, dy, dfinal=None, seq_idx=None) -> dict:
@@ -46,8 +61,8 @@ def ssd_bwd(x, dt, A, B, C, D, initial_states, dy, dfinal=None, seq_idx=None) ->
     x, dt, A, B, C = as_f64(x), as_f64(dt), as_f64(A), as_f64(B), as_f64(C)
     Dv = None if D is None else as_f64(D)
     h0 = None if initial_states is None else as_f64(initial_states)
-    dy = as_f64(dy)
-    dfin = None if dfinal is None else as_f64(dfinal)
+    dy = _upstream(dy)
+    dfin = None if dfinal is None else _upstream(dfinal)
     seq = None if seq_idx is None else as_i32(seq_idx)
     if seq is not None and dfin is not None:
         raise ValueError("dfinal with packed sequences is not supported here")
@@ -100,3 +115,31 @@ def ssd_bwd(x, dt, A, B, C, D, initial_states, dy, dfinal=None, seq_idx=None) ->
         dB[:, :, grp[h_]] += dBh[:, :, h_]
         dC[:, :, grp[h_]] += dCh[:, :, h_]
     return {"dx": dx, "ddt": ddt, "dA": dA, "dB": dB, "dC": dC, "dD": dD, "dh0": dh0}
+
+
+def silu(v):
+    """SiLU(v) = v / (1 + e^-v), elementwise, fp64."""
+    v = np.asarray(v, dtype=np.float64)
+    return v / (1.0 + np.exp(-v))
+
+
+def silu_grad(v):
+    """dSiLU/dv = s (1 + v (1 - s)) with s = 1 / (1 + e^-v), elementwise, fp64."""
+    v = np.asarray(v, dtype=np.float64)
+    s = 1.0 / (1.0 + np.exp(-v))
+    return s * (1.0 + v * (1.0 - s))
+
+
+def ssd_bwd_gated(x, dt, A, B, C, D, initial_states, z, dout, dfinal=None, seq_idx=None, backward_fn=None) -> dict:
+    """Gradients of sum(dout * y * SiLU(z)) + sum(dfinal * final): the ungated
+    output y comes from the forward oracle (fp64), the SSD's gradients from
+    ``backward_fn`` (default ``ssd_bwd``) on dy = dout * SiLU(z).  Returns the
+    same dict plus dz."""
+    from . import ssd_fwd
+    seq = None if seq_idx is None else as_i32(seq_idx)
+    num_seqs = None if seq is None else int(seq.max()) + 1
+    y, _ = ssd_fwd(x, dt, A, B, C, D, initial_states, seq_idx=seq, num_seqs=num_seqs)
+    zz, do = as_f64(z), as_f64(dout)
+    g = (backward_fn or ssd_bwd)(x, dt, A, B, C, D, initial_states, do * silu(zz), dfinal, seq)
+    g["dz"] = do * y * silu_grad(zz)
+    return g

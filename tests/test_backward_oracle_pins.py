@@ -14,10 +14,12 @@ from oracle import backward
 import ssd_inputs as si
 
 
-def _autograd(d, dy, dfinal):
-    """fp64 recurrence in PyTorch; returns the gradient of sum(dy*y) + sum(dfinal*final)."""
+def _autograd(d, dy, dfinal, z=None):
+    """fp64 recurrence in PyTorch; returns the gradient of sum(dy*y) + sum(dfinal*final),
+    or, with a gate z, of sum(dy * y * z * sigmoid(z)) + sum(dfinal*final) (plus dz)."""
     t64 = {k: (v.double().clone().requires_grad_(True) if isinstance(v, torch.Tensor) and k != "seq_idx" else v)
            for k, v in d.items()}
+    zt = None if z is None else torch.from_numpy(np.asarray(z, dtype=np.float64)).requires_grad_(True)
     x, dt, A, B, C, D, h0 = (t64[k] for k in ("x", "dt", "A", "B", "C", "D", "initial_states"))
     b, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
@@ -35,13 +37,19 @@ def _autograd(d, dy, dfinal):
         if D is not None:
             y = y + D[None, :, None] * x[:, t]
         ys.append(y)
-    loss = (torch.stack(ys, 1) * torch.from_numpy(dy)).sum()
+    yy = torch.stack(ys, 1)
+    if zt is not None:
+        yy = yy * zt * torch.sigmoid(zt)
+    loss = (yy * torch.from_numpy(dy)).sum()
     if dfinal is not None:
         loss = loss + (h * torch.from_numpy(dfinal)).sum()
     loss.backward()
     g = lambda k: None if t64[k] is None else t64[k].grad.numpy()
-    return {"dx": g("x"), "ddt": g("dt"), "dA": g("A"), "dB": g("B"), "dC": g("C"), "dD": g("D"),
-            "dh0": g("initial_states")}
+    out = {"dx": g("x"), "ddt": g("dt"), "dA": g("A"), "dB": g("B"), "dC": g("C"), "dD": g("D"),
+           "dh0": g("initial_states")}
+    if zt is not None:
+        out["dz"] = zt.grad.numpy()
+    return out
 
 
 CASES = [
@@ -126,3 +134,37 @@ def test_c_backward_matches_the_numpy_backward(case):
             assert got[k] is None, k
             continue
         assert np.allclose(got[k], w, rtol=1e-11, atol=1e-11 * max(1.0, np.abs(w).max())), k
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"b{c[0]}L{c[1]}H{c[2]}G{c[5]}{'_packed' if c[9] else ''}")
+def test_gated_backward_matches_autograd(case):
+    """The gate out = y * SiLU(z): dz and the SSD's gradients through it,
+    against autograd of y * z * sigmoid(z) written out here."""
+    b, L, H, P, N, G, h0s, withD, withF, packed = case
+    d = si.make_inputs(si.SSDShape("bwd_gate", b, L, H, P, N, G, 64, "f32", h0_std=h0s, seed=L * 5 + H))
+    if not withD:
+        d["D"] = None
+    if packed is not None:
+        d["seq_idx"], d["num_seqs"] = si.seq_idx_from_lengths(packed)
+        withF = False
+    rng = np.random.default_rng(L + 7)
+    f32 = lambda a: a.astype(np.float32).astype(np.float64)
+    dout = f32(rng.standard_normal((b, L, H, P)))
+    z = f32(2.0 * rng.standard_normal((b, L, H, P)))  # both signs, well into the curved part of SiLU
+    dfinal = f32(rng.standard_normal((b, H, P, N))) if withF else None
+    got = backward.ssd_bwd_gated(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["initial_states"], z, dout,
+                                 dfinal, d.get("seq_idx"))
+    want = _autograd(d, dout, dfinal, z=z)
+    for k, w in want.items():
+        if w is None:
+            assert got[k] is None, k
+            continue
+        assert np.allclose(got[k], w, rtol=1e-9, atol=1e-9 * max(1.0, np.abs(w).max())), k
+
+
+def test_silu_grad_is_the_derivative():
+    v = np.linspace(-8.0, 8.0, 161)
+    h = 1e-6
+    fd = (backward.silu(v + h) - backward.silu(v - h)) / (2 * h)
+    assert np.allclose(backward.silu_grad(v), fd, rtol=1e-7, atol=1e-9)
+    assert backward.silu_grad(0.0) == 0.5  # s(0) = 1/2, and the v (1 - s) term vanishes

@@ -122,6 +122,8 @@ BACKWARD_MUTANTS = {
     "dB_not_summed_over_group": ("dB[:, :, grp[h_]] += dBh[:, :, h_]", "dB[:, :, grp[h_]] = dBh[:, :, h_]"),
     "reset_ignored": ("a = np.where(reset[:, :, None], 0.0, a)", "a = a"),
     "skip_term_dropped_from_dx": ("dx += Dv[None, None, :, None] * dy", "dx += 0.0 * dy"),
+    "gate_grad_is_the_logistic_slope": ("return s * (1.0 + v * (1.0 - s))", "return s * (1.0 - s)"),
+    "gate_not_applied_to_dy": ("do * silu(zz), dfinal, seq)", "do, dfinal, seq)"),
 }
 
 
@@ -151,4 +153,9 @@ def test_backward_mutant_fails_a_pin(name, monkeypatch, tmp_path):
         bw.test_backward_matches_finite_differences_of_the_forward_oracle()
     except AssertionError:
         failed += 1
+    for case in bw.CASES:
+        try:
+            bw.test_gated_backward_matches_autograd(case)
+        except AssertionError:
+            failed += 1
     assert failed > 0, f"no pin caught {name}"
