@@ -328,6 +328,12 @@ typedef struct {
                                      recorded on `stream` right before and right after
                                      k_bwd_chunk, the kernel that dominates the call.
                                      Both or neither.                                */
+  const void* z;                  /* (b,L,H,P) dtype gate, or NULL.  With z the forward
+                                     returned out = y * SiLU(z) (ssd_fwd_args.z) and dy
+                                     is dLoss/dout: the kernels recompute y, write
+                                     dz = dy * y * SiLU'(z) and take dy * SiLU(z) as
+                                     the gradient of y.                              */
+  float* dz;                      /* (b,L,H,P) fp32 output dLoss/dz; required iff z  */
 } ssd_bwd_args;
 
 /* Bytes of device workspace ssd_bwd needs (only sizes, chunk_size and dtype
@@ -343,8 +349,8 @@ SSD_API int64_t ssd_bwd_chunk_size(const ssd_bwd_args* args);
  * All pointers are device pointers owned by the caller; outputs must not
  * overlap inputs or the workspace.  Returns SSD_OK once enqueued;
  * SSD_ERR_INVALID_ARG for a null required pointer, a bad size or enum, or a
- * misaligned workspace or a single timing event; SSD_ERR_UNSUPPORTED as
- * described above;
+ * misaligned workspace, a single timing event, or z without dz (or dz
+ * without z); SSD_ERR_UNSUPPORTED as described above;
  * SSD_ERR_WORKSPACE when the workspace is missing or too small; SSD_ERR_CUDA
  * when a launch fails (outputs then undefined). */
 SSD_API ssd_status ssd_bwd(const ssd_bwd_args* args, void* stream);

@@ -83,6 +83,7 @@ class BwdArgs(ctypes.Structure):
         ("dinitial_states", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("timing_events", ctypes.c_void_p * 2),
+        ("z", ctypes.c_void_p), ("dz", ctypes.c_void_p),
     ]
 
 
@@ -429,7 +430,8 @@ def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
         D: Optional[torch.Tensor], dy: torch.Tensor, initial_states: Optional[torch.Tensor] = None,
         seq_idx: Optional[torch.Tensor] = None, dfinal_states: Optional[torch.Tensor] = None,
         chunk_size: int = 0, want_dD: bool = True, want_dinitial_states: Optional[bool] = None,
-        workspace: Optional[torch.Tensor] = None, timing_events: Optional[tuple] = None) -> dict:
+        workspace: Optional[torch.Tensor] = None, timing_events: Optional[tuple] = None,
+        z: Optional[torch.Tensor] = None) -> dict:
     """The SSD backward via ``ssd_bwd``: gradients of a loss given
     dy = dLoss/dy (like x) and dfinal_states = dLoss/dfinal_states
     ((b,H,P,N) fp32 or None; not with seq_idx).  Inputs as for ``fwd``.
@@ -437,10 +439,15 @@ def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     ``want_dD``) and dinitial_states (by default only when initial_states
     is given).  ``chunk_size`` is the backward's own chunk length (0: the
     library chooses).  ``timing_events``: optional (start, end)
-    torch.cuda.Event pair recorded around the dominant kernel."""
+    torch.cuda.Event pair recorded around the dominant kernel.  ``z``: the
+    forward's gate (like x); dy is then the gradient of y * SiLU(z), and the
+    dict also holds dz (fp32)."""
     _check(x, dt, A, B, C, D, initial_states, seq_idx)
     if dy.dtype != x.dtype or tuple(dy.shape) != tuple(x.shape) or dy.device != x.device or not dy.is_contiguous():
         raise ValueError("dy must be a contiguous tensor like x")
+    if z is not None and (z.dtype != x.dtype or tuple(z.shape) != tuple(x.shape) or z.device != x.device
+                          or not z.is_contiguous()):
+        raise ValueError("z must be a contiguous tensor like x")
     b, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
     if dfinal_states is not None and (dfinal_states.dtype != torch.float32 or tuple(dfinal_states.shape) != (b, H, P, N)
@@ -452,10 +459,12 @@ def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     g = {"dx": torch.empty(b, L, H, P, **f32), "ddt": torch.empty(b, L, H, **f32), "dA": torch.empty(H, **f32),
          "dB": torch.empty(b, L, G, N, **f32), "dC": torch.empty(b, L, G, N, **f32),
          "dD": torch.empty(H, **f32) if want_dD else None,
-         "dinitial_states": torch.empty(b, H, P, N, **f32) if want_dinitial_states else None}
+         "dinitial_states": torch.empty(b, H, P, N, **f32) if want_dinitial_states else None,
+         "dz": torch.empty(b, L, H, P, **f32) if z is not None else None}
     a = make_bwd_args(x, dt, A, B, C, D, dy, initial_states, seq_idx, dfinal_states, chunk_size)
     a.dx, a.ddt, a.dA, a.dB, a.dC = (_ptr(g[k]) for k in ("dx", "ddt", "dA", "dB", "dC"))
     a.dD, a.dinitial_states = _ptr(g["dD"]), _ptr(g["dinitial_states"])
+    a.z, a.dz = _ptr(z), _ptr(g["dz"])
     need = int(lib.ssd_bwd_workspace_size(ctypes.byref(a)))
     if need == 0:  # sizes the library rejects: let it say why (nothing is enqueued)
         raise SSDError(lib.ssd_bwd(ctypes.byref(a), _stream(x)))
@@ -477,34 +486,35 @@ class _SSDChunked(torch.autograd.Function):
     """``fwd`` forward, ``bwd`` backward; gradients returned in each input's dtype."""
 
     @staticmethod
-    def forward(ctx, x, dt, A, B, C, D, initial_states, seq_idx, num_seqs, chunk_size):
+    def forward(ctx, x, dt, A, B, C, D, initial_states, seq_idx, num_seqs, chunk_size, z):
         ctx.set_materialize_grads(False)
         y, fin = fwd(x, dt, A, B, C, D, chunk_size=chunk_size, initial_states=initial_states, seq_idx=seq_idx,
-                     num_seqs=num_seqs)
-        ctx.save_for_backward(x, dt, A, B, C, D, initial_states, seq_idx)
+                     num_seqs=num_seqs, z=z)
+        ctx.save_for_backward(x, dt, A, B, C, D, initial_states, seq_idx, z)
         return y, fin
 
     @staticmethod
     def backward(ctx, dy, dfin):
-        x, dt, A, B, C, D, h0, seq = ctx.saved_tensors
+        x, dt, A, B, C, D, h0, seq, z = ctx.saved_tensors
         if seq is not None and dfin is not None:
             raise NotImplementedError("the gradient through per-sequence final states is not supported")
         dy = torch.zeros_like(x) if dy is None else dy.to(x.dtype).contiguous()
         dfin = None if dfin is None else dfin.to(torch.float32).contiguous()
         need = ctx.needs_input_grad
         g = bwd(x, dt, A, B, C, D, dy, initial_states=h0, seq_idx=seq, dfinal_states=dfin,
-                want_dD=D is not None and need[5], want_dinitial_states=h0 is not None and need[6])
+                want_dD=D is not None and need[5], want_dinitial_states=h0 is not None and need[6], z=z)
         return (g["dx"].to(x.dtype), g["ddt"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype), g["dD"],
-                g["dinitial_states"], None, None, None)
+                g["dinitial_states"], None, None, None, None if z is None else g["dz"].to(z.dtype))
 
 
 def ssd_chunked(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
                 D: Optional[torch.Tensor] = None, chunk_size: int = 64,
                 initial_states: Optional[torch.Tensor] = None, seq_idx: Optional[torch.Tensor] = None,
-                num_seqs: Optional[int] = None):
-    """Differentiable SSD forward: returns (y, final_states) like ``fwd``, and
-    its backward runs ``ssd_bwd`` (the states are recomputed, nothing but the
-    inputs is kept).  With seq_idx the final states carry no gradient."""
+                num_seqs: Optional[int] = None, z: Optional[torch.Tensor] = None):
+    """Differentiable SSD forward: returns (y, final_states) like ``fwd``
+    (y * SiLU(z) with a gate z), and its backward runs ``ssd_bwd`` (the
+    states and y are recomputed, nothing but the inputs is kept).  With
+    seq_idx the final states carry no gradient."""
     if seq_idx is not None and num_seqs is None:
         num_seqs = int(seq_idx.max().item()) + 1
-    return _SSDChunked.apply(x, dt, A, B, C, D, initial_states, seq_idx, num_seqs, chunk_size)
+    return _SSDChunked.apply(x, dt, A, B, C, D, initial_states, seq_idx, num_seqs, chunk_size, z)

@@ -30,6 +30,9 @@
 // M(t,s) = E(t,s) w_s (C_t.B_s)(dy_t.x_s) and N_s = E(last,s) w_s x_s^T Lam B_s;
 // dl_k = sum of dcs_t over t >= k in k's segment, ddt_k = dw_k + A dl_k and
 // dA = sum_k dt_k dl_k.  A token that starts a segment has no decay term.
+// With the block's gate (out = y SiLU(z)), k_bwd_chunk first recomputes the
+// chunk's y from the same K and h_in, writes dz = dout y SiLU'(z), and all of
+// the above then runs on dy = dout SiLU(z).
 //
 // Five kernels, in stream order:
 //   k_bwd_chunk_states   per (b, c, h): the chunk's end state from a zero
@@ -90,6 +93,8 @@ struct KArgs {
   float* dC;
   float* dD;
   float* dh0;
+  const void* z;    // (b,L,H,P) gate or null
+  float* dz;        // (b,L,H,P) with z
   // workspace
   float* S;         // (b,H,nc,P,N): chunk end states from zero, then each chunk's h_in
   float* T;         // (b,H,nc,P,N): each chunk's sum_t e_t dy_t C_t^T, then its Lam
@@ -102,6 +107,13 @@ struct KArgs {
 
 __device__ __forceinline__ float ld(const float* p, int64_t i) { return p[i]; }
 __device__ __forceinline__ float ld(const __nv_bfloat16* p, int64_t i) { return __bfloat162float(p[i]); }
+
+// The gate: SiLU(v) = v / (1 + e^-v) and its slope s (1 + v (1 - s)), s = 1 / (1 + e^-v).
+__device__ __forceinline__ float gate_silu(float v) { return v / (1.f + expf(-v)); }
+__device__ __forceinline__ float gate_slope(float v) {
+  const float s = 1.f / (1.f + expf(-v));
+  return s * fmaf(v, 1.f - s, 1.f);
+}
 
 // Chunk c's coordinates from a CTA index ordered (b, c, h), h fastest.
 struct ChunkPos {
@@ -228,13 +240,14 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk_states(const KArgs a) {
 
   const T* x = static_cast<const T*>(a.x);
   const T* dy = static_cast<const T*>(a.dy);
+  const T* z = static_cast<const T*>(a.z);
   const T* B = static_cast<const T*>(a.B);
   const T* C = static_cast<const T*>(a.C);
   for (int i = tid; i < Qc * P; i += kThreads) {
     const int t = i / P, p = i % P;
     const int64_t gi = ((q.b * d.L + q.t0 + t) * d.H + q.h) * d.P + p;
     xs[i] = ld(x, gi);
-    dys[i] = ld(dy, gi);
+    dys[i] = z ? ld(dy, gi) * gate_silu(ld(z, gi)) : ld(dy, gi);  // the gradient reaching y
   }
   for (int i = tid; i < Qc * N; i += kThreads) {
     const int t = i / N, n = i % N;
@@ -325,10 +338,10 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
   const int tid = threadIdx.x;
   SSD_DYN_SMEM(sm);
   float* xs = sm;             // Q x sP: x_t
-  float* dys = xs + Q * sP;   // Q x sP: dy_t
+  float* dys = xs + Q * sP;   // Q x sP: dy_t (with a gate: first dout_t, then dout_t SiLU(z_t))
   float* Bs = dys + Q * sP;   // Q x sN
   float* Cs = Bs + Q * sN;    // Q x sN
-  float* SB = Cs + Q * sN;    // P x sN: Lam, then h_in
+  float* SB = Cs + Q * sN;    // P x sN: h_in, then Lam
   float* Km = SB + P * sN;    // Q x sQ: E(t,s) C_t.B_s
   float* Zm = Km + Q * sQ;    // Q x sQ: E(t,s) dy_t.x_s
   float* Mm = Zm + Q * sQ;    // Q x sQ: E(t,s) (C_t.B_s)(dy_t.x_s)
@@ -347,11 +360,13 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
 
   const T* x = static_cast<const T*>(a.x);
   const T* dy = static_cast<const T*>(a.dy);
+  const T* z = static_cast<const T*>(a.z);
   const T* B = static_cast<const T*>(a.B);
   const T* C = static_cast<const T*>(a.C);
   const int64_t soff = ((q.b * d.H + q.h) * d.nc + q.c) * d.P * d.N;
   const float* Hin = a.S + soff;  // P x N
   const float* Lam = a.T + soff;  // P x N
+  const float Dh = a.D ? a.D[q.h] : 0.f;
 
   for (int i = tid; i < Qc * P; i += kThreads) {
     const int t = i / P, p = i % P;
@@ -368,9 +383,9 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
   {
     float part_lh = 0.f;  // <Lam, h_in>, this thread's share
     for (int e = tid; e < P * N; e += kThreads) {
-      const float l = Lam[e];
-      SB[(e / N) * sN + e % N] = l;
-      part_lh = fmaf(l, Hin[e], part_lh);
+      const float h = Hin[e];
+      SB[(e / N) * sN + e % N] = h;
+      part_lh = fmaf(Lam[e], h, part_lh);
     }
     red[tid] = part_lh;
   }
@@ -379,14 +394,12 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
   __syncthreads();
 
   const int last = Qc - 1;
-  // the chunk's Q x Q matrices: C_t.B_s and dy_t.x_s, masked and decayed
+  // K = E o (C B^T) on the chunk's Q x Q triangle, and the decays to the chunk's ends
   for (int tile = tid; tile < tiles_of(Qc, Qc); tile += kThreads) {
     const Tile tl = make_tile(tile, Qc, Qc);
-    float cb[kT][kT], xy[kT][kT];
+    float cb[kT][kT];
     tile_zero(cb);
-    tile_zero(xy);
     tile_mac<false>(cb, tl, Cs, sN, 1, nullptr, Bs, 1, sN, 0, N);
-    tile_mac<false>(xy, tl, dys, sP, 1, nullptr, xs, 1, sP, 0, P);
 #pragma unroll
     for (int i = 0; i < kT; ++i)
 #pragma unroll
@@ -395,9 +408,6 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
         const int t = tl.r[i], s = tl.c[j];
         const float e = (s <= t && seg[s] == seg[t]) ? expf(cs[t] - cs[s]) : 0.f;
         Km[t * sQ + s] = e * cb[i][j];
-        Zm[t * sQ + s] = e * xy[i][j];
-        Mm[t * sQ + s] = e * cb[i][j] * xy[i][j];
-        if (s == t) dg[t] = xy[i][j];
       }
   }
   for (int t = tid; t < Qc; t += kThreads) {
@@ -406,7 +416,96 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
   }
   __syncthreads();
 
-  const float Dh = a.D ? a.D[q.h] : 0.f;
+  if (z) {
+    // the gate: recompute y_t = sum_s K(t,s) dt_s x_s + e_t h_in C_t + D x_t, write
+    // dz = dout y SiLU'(z), and carry on with dy = dout SiLU(z)
+    for (int tile = tid; tile < tiles_of(Qc, P); tile += kThreads) {
+      const Tile tl = make_tile(tile, Qc, P);
+      int kmax = 0;
+#pragma unroll
+      for (int i = 0; i < kT; ++i)
+        if (tl.rv[i]) kmax = tl.r[i] + 1;
+      float yi[kT][kT], yh[kT][kT];
+      tile_zero(yi);
+      tile_zero(yh);
+      tile_mac<true>(yi, tl, Km, sQ, 1, w, xs, sP, 1, 0, kmax);
+      tile_mac<false>(yh, tl, Cs, sN, 1, nullptr, SB, 1, sN, 0, N);
+#pragma unroll
+      for (int i = 0; i < kT; ++i)
+#pragma unroll
+        for (int j = 0; j < kT; ++j) {
+          if (!tl.rv[i] || !tl.cv[j]) continue;
+          const int t = tl.r[i], p = tl.c[j];
+          const int64_t gi = ((q.b * d.L + q.t0 + t) * d.H + q.h) * d.P + p;
+          const float y = fmaf(ein[t], yh[i][j], fmaf(Dh, xs[t * sP + p], yi[i][j]));
+          const float zz = ld(z, gi), dout = dys[t * sP + p];
+          a.dz[gi] = dout * y * gate_slope(zz);
+          dys[t * sP + p] = dout * gate_silu(zz);
+        }
+    }
+    __syncthreads();
+  }
+
+  // Z = E o (dy x^T) and M = K o (dy x^T); the diagonal dy_t.x_t
+  for (int tile = tid; tile < tiles_of(Qc, Qc); tile += kThreads) {
+    const Tile tl = make_tile(tile, Qc, Qc);
+    float xy[kT][kT];
+    tile_zero(xy);
+    tile_mac<false>(xy, tl, dys, sP, 1, nullptr, xs, 1, sP, 0, P);
+#pragma unroll
+    for (int i = 0; i < kT; ++i)
+#pragma unroll
+      for (int j = 0; j < kT; ++j) {
+        if (!tl.rv[i] || !tl.cv[j]) continue;
+        const int t = tl.r[i], s = tl.c[j];
+        const float e = (s <= t && seg[s] == seg[t]) ? expf(cs[t] - cs[s]) : 0.f;
+        Zm[t * sQ + s] = e * xy[i][j];
+        Mm[t * sQ + s] = Km[t * sQ + s] * xy[i][j];
+        if (s == t) dg[t] = xy[i][j];
+      }
+  }
+  __syncthreads();
+
+  // dC of this head (Q x N): sum_s Z(t,s) w_s B_s + e_t h_in^T dy_t; with the
+  // row partials of C_t . (h_in^T dy_t)
+  for (int tile = tid; tile < tiles_of(Qc, N); tile += kThreads) {
+    const Tile tl = make_tile(tile, Qc, N);
+    int kmax = 0;
+#pragma unroll
+    for (int i = 0; i < kT; ++i)
+      if (tl.rv[i]) kmax = tl.r[i] + 1;
+    float ci[kT][kT], ch[kT][kT];
+    tile_zero(ci);
+    tile_zero(ch);
+    tile_mac<true>(ci, tl, Zm, sQ, 1, w, Bs, sN, 1, 0, kmax);
+    tile_mac<false>(ch, tl, dys, sP, 1, nullptr, SB, sN, 1, 0, P);
+#pragma unroll
+    for (int i = 0; i < kT; ++i) {
+      if (!tl.rv[i]) continue;
+      const int t = tl.r[i];
+      float cy = 0.f;
+#pragma unroll
+      for (int j = 0; j < kT; ++j) {
+        if (!tl.cv[j]) continue;
+        const int n = tl.c[j];
+        a.dCh[((q.b * d.L + q.t0 + t) * d.H + q.h) * d.N + n] = fmaf(ein[t], ch[i][j], ci[i][j]);
+        cy = fmaf(Cs[t * sN + n], ch[i][j], cy);
+      }
+      part[t * PC + tl.tc] = cy;
+    }
+  }
+  __syncthreads();
+
+  // the h_in term of dcs (kept in dcs for now); Lam replaces h_in
+  const int tcn = (N + kT - 1) / kT;
+  for (int t = tid; t < Qc; t += kThreads) {
+    float v = 0.f;
+    for (int k = 0; k < tcn; ++k) v += part[t * PC + k];
+    dcs[t] = ein[t] * v;
+  }
+  for (int e = tid; e < P * N; e += kThreads) SB[(e / N) * sN + e % N] = Lam[e];
+  __syncthreads();
+
   // dx (Q x P): w_s [sum_t K(t,s) dy_t + E(last,s) Lam B_s] + D dy_s; with the
   // row partials of x_s . (Lam B_s)
   for (int tile = tid; tile < tiles_of(Qc, P); tile += kThreads) {
@@ -457,48 +556,9 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
     for (int k = 0; k < tcp; ++k) v += part[s * PC + k];
     nv[s] = v;
   }
-  for (int e = tid; e < P * N; e += kThreads) SB[(e / N) * sN + e % N] = Hin[e];
   __syncthreads();
 
-  // dC of this head (Q x N): sum_s Z(t,s) w_s B_s + e_t h_in^T dy_t; with the
-  // row partials of C_t . (h_in^T dy_t)
-  for (int tile = tid; tile < tiles_of(Qc, N); tile += kThreads) {
-    const Tile tl = make_tile(tile, Qc, N);
-    int kmax = 0;
-#pragma unroll
-    for (int i = 0; i < kT; ++i)
-      if (tl.rv[i]) kmax = tl.r[i] + 1;
-    float ci[kT][kT], ch[kT][kT];
-    tile_zero(ci);
-    tile_zero(ch);
-    tile_mac<true>(ci, tl, Zm, sQ, 1, w, Bs, sN, 1, 0, kmax);
-    tile_mac<false>(ch, tl, dys, sP, 1, nullptr, SB, sN, 1, 0, P);
-#pragma unroll
-    for (int i = 0; i < kT; ++i) {
-      if (!tl.rv[i]) continue;
-      const int t = tl.r[i];
-      float cy = 0.f;
-#pragma unroll
-      for (int j = 0; j < kT; ++j) {
-        if (!tl.cv[j]) continue;
-        const int n = tl.c[j];
-        a.dCh[((q.b * d.L + q.t0 + t) * d.H + q.h) * d.N + n] = fmaf(ein[t], ch[i][j], ci[i][j]);
-        cy = fmaf(Cs[t * sN + n], ch[i][j], cy);
-      }
-      part[t * PC + tl.tc] = cy;
-    }
-  }
-  __syncthreads();
-
-  // per token: the h_in term of dcs (kept in dcs for now), then the row and
-  // column sums of M in quarters, four threads per token
-  const int tcn = (N + kT - 1) / kT;
-  for (int t = tid; t < Qc; t += kThreads) {
-    float v = 0.f;
-    for (int k = 0; k < tcn; ++k) v += part[t * PC + k];
-    dcs[t] = ein[t] * v;
-  }
-  __syncthreads();
+  // per token: the row and column sums of M in quarters, four threads per token
   for (int i = tid; i < 4 * Qc; i += kThreads) {
     const int t = i >> 2, qq = i & 3;
     const int lo = Qc * qq / 4, hi = Qc * (qq + 1) / 4;
@@ -649,6 +709,7 @@ inline ssd_status check_call(const ssd_bwd_args* a, const Plan& pl) {
   if (!a->workspace || a->workspace_bytes < pl.total) return SSD_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(a->workspace) % 256 != 0) return SSD_ERR_INVALID_ARG;
   if ((a->timing_events[0] == nullptr) != (a->timing_events[1] == nullptr)) return SSD_ERR_INVALID_ARG;
+  if ((a->z == nullptr) != (a->dz == nullptr)) return SSD_ERR_INVALID_ARG;
   return SSD_OK;
 }
 
@@ -672,6 +733,8 @@ inline KArgs make_kargs(const ssd_bwd_args* a, const Plan& pl) {
   k.dC = a->dC;
   k.dD = a->dD;
   k.dh0 = a->dinitial_states;
+  k.z = a->z;
+  k.dz = a->dz;
   char* ws = static_cast<char*>(a->workspace);
   k.S = reinterpret_cast<float*>(ws + pl.off_S);
   k.T = reinterpret_cast<float*>(ws + pl.off_T);

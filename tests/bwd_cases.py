@@ -5,6 +5,7 @@ import numpy as np
 import torch
 
 import oracle
+from oracle import backward
 import ssd_inputs as si
 
 # The kernels compute in fp32 and the oracle in fp64 on the same (fp32- or
@@ -13,7 +14,7 @@ import ssd_inputs as si
 # relative at these sizes); both bounds leave a wide margin over that.
 REL_L2 = 1e-5
 MAX_ABS = 1e-4
-KEYS = ("dx", "ddt", "dA", "dB", "dC", "dD", "dh0")
+KEYS = ("dx", "ddt", "dA", "dB", "dC", "dD", "dh0", "dz")
 
 CASES = [
     # id, (b, L, H, P, N, G), dtype, h0 std, dfinal, packed (lo, hi) or per-row lengths, D, chunk
@@ -28,6 +29,9 @@ CASES = [
     ("bf16_N256_chunk32", (1, 70, 2, 64, 256, 1), "bf16", 0.2, True, None, True, 0),
     ("f32_hpg4", (1, 40, 8, 8, 16, 2), "f32", 0.0, True, None, True, 8),
 ]
+# the same with the block's gate (out = y SiLU(z)): dy is then the gradient of the gated output
+GATED = {"f32_ragged_Q16", "bf16_packed", "f32_packed_edges", "bf16_N256_chunk32"}
+CASES += [("gated_" + c[0],) + c[1:] for c in CASES if c[0] in GATED]
 
 
 def dy_like(b, L, H, P, dtype, seed):
@@ -48,19 +52,29 @@ def inputs(b, L, H, P, N, G, dtype="f32", h0=0.0, packed=None, seed=1, has_D=Tru
     return d
 
 
+def gate_like(b, L, H, P, dtype, seed):
+    """z ~ N(0, 2^2): both signs, well into the curved part of SiLU."""
+    g = torch.Generator().manual_seed(seed + 2)
+    return (2.0 * torch.randn(b, L, H, P, generator=g)).to(dtype)
+
+
 def case_inputs(case):
-    """(inputs, dy, dfinal, chunk) of one CASES entry."""
+    """(inputs, dy, dfinal, chunk) of one CASES entry; a gated case carries
+    its gate in inputs["z"]."""
     name, (b, L, H, P, N, G), dtype, h0, with_df, packed, with_D, chunk = case
     d = inputs(b, L, H, P, N, G, dtype, h0, packed if isinstance(packed, tuple) else None, seed=L * 3 + H,
                has_D=with_D, lengths=packed if isinstance(packed, list) else None)
+    d["z"] = gate_like(b, L, H, P, d["x"].dtype, L + N) if name.startswith("gated_") else None
     dy = dy_like(b, L, H, P, d["x"].dtype, L + P)
     dfinal = dfinal_like(b, H, P, N, L) if with_df else None
     return d, dy, dfinal, chunk
 
 
 def oracle_bwd(d, dy, dfinal):
-    return oracle.ssd_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["initial_states"], dy, dfinal,
-                          d["seq_idx"])
+    args = (d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["initial_states"])
+    if d.get("z") is not None:
+        return backward.ssd_bwd_gated(*args, d["z"], dy, dfinal, d["seq_idx"], backward_fn=oracle.ssd_bwd)
+    return oracle.ssd_bwd(*args, dy, dfinal, d["seq_idx"])
 
 
 def compare(out, ref, keys=KEYS):

@@ -6,8 +6,8 @@
 //
 // reads DIR/args.txt ("key value" lines: the size fields of ssd_bwd_args,
 // dtype 0|1 and has_* / want_* flags) and the input arrays DIR/<name>.bin
-// (raw, row-major: x dt A B C D h0 seq dy dfinal), writes the gradients as
-// raw fp32 to DIR/<name>.bin (dx ddt dA dB dC dD dh0) and prints the status.
+// (raw, row-major: x dt A B C D h0 seq dy dfinal z), writes the gradients as
+// raw fp32 to DIR/<name>.bin (dx ddt dA dB dC dD dh0 dz) and prints the status.
 // "reverse 1" runs each block's fibers in reverse thread order.
 // Every buffer is allocated to its exact size, so AddressSanitizer sees any
 // access past it; outputs, workspace and shared memory start as NaN bytes,
@@ -207,6 +207,7 @@ int main(int argc, char** argv) {
   a.seq_idx = static_cast<const int32_t*>(in("seq", kv["has_seq"] != 0));
   a.dy = in("dy", true);
   a.dfinal_states = static_cast<const float*>(in("dfinal", kv["has_dfinal"] != 0));
+  a.z = in("z", kv["has_z"] != 0);
 
   const size_t b = a.batch, L = a.seqlen, H = a.nheads, P = a.headdim, N = a.dstate, G = a.ngroups;
   const size_t nx = b * L * H * P, ndt = b * L * H, nB = b * L * G * N, nh = b * H * P * N;
@@ -217,6 +218,7 @@ int main(int argc, char** argv) {
   a.dC = nan_floats(nB);
   a.dD = kv["want_dD"] ? nan_floats(H) : nullptr;
   a.dinitial_states = kv["want_dh0"] ? nan_floats(nh) : nullptr;
+  a.dz = a.z ? nan_floats(nx) : nullptr;
 
   ssd::bwd::Plan pl;
   ssd_status st = ssd::bwd::plan(&a, &pl);
@@ -239,6 +241,7 @@ int main(int argc, char** argv) {
   write_file(dir + "/dC.bin", a.dC, nB * 4);
   if (a.dD) write_file(dir + "/dD.bin", a.dD, H * 4);
   if (a.dinitial_states) write_file(dir + "/dh0.bin", a.dinitial_states, nh * 4);
+  if (a.dz) write_file(dir + "/dz.bin", a.dz, nx * 4);
   std::free(ws);
   return 0;
 }

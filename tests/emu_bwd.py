@@ -56,10 +56,12 @@ def _raw(t) -> bytes:
 
 
 def run(inp: dict, dy, dfinal=None, chunk_size: int = 0, want_dD: bool = True, want_dh0: bool = True,
-        kind: str = "asan", reverse: bool = False, timeout: int = 600) -> dict:
+        kind: str = "asan", reverse: bool = False, timeout: int = 600, z=None) -> dict:
     """Run the emulated backward on ``inp`` (``ssd_inputs.make_inputs`` form)
     with upstream gradient ``dy`` (x's dtype) and ``dfinal`` (fp32 or None).
     ``reverse`` runs each block's threads in reverse order (fiber builds).
+    ``z``: the forward's gate (x's dtype), dy then being the gradient of the
+    gated output.
     Returns {"status", "chunk", and the fp32 gradients as numpy arrays}."""
     exe = build(kind)
     x = inp["x"]
@@ -67,7 +69,8 @@ def run(inp: dict, dy, dfinal=None, chunk_size: int = 0, want_dD: bool = True, w
     G, N = inp["B"].shape[2], inp["B"].shape[3]
     with tempfile.TemporaryDirectory() as d:
         arrays = {"x": x, "dt": inp["dt"], "A": inp["A"], "B": inp["B"], "C": inp["C"], "D": inp.get("D"),
-                  "h0": inp.get("initial_states"), "seq": inp.get("seq_idx"), "dy": dy, "dfinal": dfinal}
+                  "h0": inp.get("initial_states"), "seq": inp.get("seq_idx"), "dy": dy, "dfinal": dfinal,
+                  "z": z}
         for k, v in arrays.items():
             if v is not None:
                 with open(os.path.join(d, k + ".bin"), "wb") as f:
@@ -76,7 +79,7 @@ def run(inp: dict, dy, dfinal=None, chunk_size: int = 0, want_dD: bool = True, w
                   dtype=1 if x.dtype == torch.bfloat16 else 0, has_D=int(arrays["D"] is not None),
                   has_h0=int(arrays["h0"] is not None), has_seq=int(arrays["seq"] is not None),
                   has_dfinal=int(dfinal is not None), want_dD=int(want_dD), want_dh0=int(want_dh0),
-                  reverse=int(reverse))
+                  reverse=int(reverse), has_z=int(z is not None))
         with open(os.path.join(d, "args.txt"), "w") as f:
             f.write("".join(f"{k} {v}\n" for k, v in kv.items()))
         env = dict(os.environ)
@@ -90,7 +93,7 @@ def run(inp: dict, dy, dfinal=None, chunk_size: int = 0, want_dD: bool = True, w
         if out["status"] != 0:
             return out
         shapes = {"dx": (b, L, H, P), "ddt": (b, L, H), "dA": (H,), "dB": (b, L, G, N), "dC": (b, L, G, N),
-                  "dD": (H,), "dh0": (b, H, P, N)}
+                  "dD": (H,), "dh0": (b, H, P, N), "dz": (b, L, H, P)}
         for k, shp in shapes.items():
             path = os.path.join(d, k + ".bin")
             out[k] = np.fromfile(path, dtype=np.float32).reshape(shp) if os.path.exists(path) else None

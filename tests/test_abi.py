@@ -322,6 +322,8 @@ def _bwd_args(**kw):
     ({"headdim": 257}, ssd.SSD_ERR_UNSUPPORTED),
     ({"chunk_size": 65}, ssd.SSD_ERR_UNSUPPORTED),
     ({"timing_events": (ctypes.c_void_p * 2)(1 << 12, None)}, ssd.SSD_ERR_INVALID_ARG),  # one event only
+    ({"z": 1 << 26}, ssd.SSD_ERR_INVALID_ARG),                                           # a gate without dz
+    ({"dz": 1 << 26}, ssd.SSD_ERR_INVALID_ARG),                                          # dz without a gate
 ])
 def test_bwd_rejects_bad_arguments(kw, status):
     assert ssd.lib.ssd_bwd(ctypes.byref(_bwd_args(**kw)), None) == status

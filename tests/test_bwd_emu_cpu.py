@@ -21,7 +21,7 @@ import pytest
 import torch
 
 import emu_bwd
-from bwd_cases import CASES, KEYS, case_inputs, compare, dfinal_like, dy_like, inputs, oracle_bwd
+from bwd_cases import CASES, KEYS, case_inputs, compare, dfinal_like, dy_like, gate_like, inputs, oracle_bwd
 
 pytestmark = pytest.mark.skipif(not emu_bwd.available(), reason="g++ not available")
 
@@ -30,7 +30,7 @@ pytestmark = pytest.mark.skipif(not emu_bwd.available(), reason="g++ not availab
 def test_emulated_backward_matches_oracle(case):
     name, (b, L, H, P, N, G), _, _, _, _, with_D, chunk = case
     d, dy, dfinal = case_inputs(case)[:3]
-    out = emu_bwd.run(d, dy, dfinal, chunk_size=chunk)
+    out = emu_bwd.run(d, dy, dfinal, chunk_size=chunk, z=d["z"])
     assert out["status"] == 0
     assert out["launches"] == 5
     if name == "bf16_N256_chunk32":
@@ -44,8 +44,12 @@ def test_emulated_backward_matches_oracle(case):
         d0 = dict(d, initial_states=torch.zeros(b, H, P, N))
         assert np.allclose(out["dh0"], oracle_bwd(d0, dy, dfinal)["dh0"], rtol=1e-4, atol=1e-5)
     if not with_D:
-        # dD is the gradient at D = 0: sum over rows and tokens of dy . x
-        want = np.einsum("blhp,blhp->h", dy.double().numpy(), d["x"].double().numpy())
+        # dD is the gradient at D = 0: sum over rows and tokens of dy . x (dy reaching y, after the gate)
+        dyy = dy.double().numpy()
+        if d["z"] is not None:
+            zz = d["z"].double().numpy()
+            dyy = dyy * zz / (1.0 + np.exp(-zz))
+        want = np.einsum("blhp,blhp->h", dyy, d["x"].double().numpy())
         assert np.allclose(out["dD"], want, rtol=1e-5, atol=1e-5)
 
 
@@ -112,8 +116,8 @@ def test_packed_with_dfinal_is_unsupported():
 # Planted mistakes in a copy of the kernels: each must make the emulated run
 # fail (sanitizer abort, non-finite output or a parity miss).
 MUTANTS = [
-    # a missing barrier between the Q x Q matrices and their use
-    ("drop_barrier", r"(    ein\[t\] = seg\[t\] == -1 \? expf\(cs\[t\]\) : 0\.f;\n  }\n)  __syncthreads\(\);", r"\1"),
+    # a missing barrier between the Q x Q matrices and their use by other threads
+    ("drop_barrier", r"(        if \(s == t\) dg\[t\] = xy\[i\]\[j\];\n      }\n  }\n)  __syncthreads\(\);", r"\1"),
     # the in-chunk sum of dx runs one token past the chunk
     ("dx_past_chunk", r"(tile_mac<false>\(acc, tl, Km, 1, sQ, nullptr, dys, sP, 1, tl\.r\[0\], )Qc\);", r"\1Qc + 1);"),
     # the adjoint carried across chunks skips the chunk decay
@@ -124,6 +128,11 @@ MUTANTS = [
     ("hin_always", r"ein\[t\] = seg\[t\] == -1 \? expf\(cs\[t\]\) : 0\.f;", "ein[t] = expf(cs[t]);"),
     # tiles numbered with the wrong divisor: parts of a non-square product are never written
     ("tile_index", r"const int tr = tile / TC;", "const int tr = tile / (TC + 1);"),
+    # the gate's slope taken as the logistic's (run with a gate)
+    ("gate_slope", r"return s \* fmaf\(v, 1\.f - s, 1\.f\);", "return s * (1.f - s);"),
+    # no barrier between rewriting dy through the gate and reading it (run with a gate)
+    ("gate_barrier", r"(          dys\[t \* sP \+ p\] = dout \* gate_silu\(zz\);\n        }\n    }\n)    __syncthreads\(\);",
+     r"\1"),
 ]
 
 
@@ -141,13 +150,14 @@ def test_emulator_catches_planted_mistakes(mutant, monkeypatch):
         monkeypatch.setattr(emu_bwd, "OUT", os.path.join(tmp, "out"))
         d = inputs(2, 80, 2, 8, 16, 1, "f32", 0.5, packed=None, seed=9,
                     lengths=[[20, 1, 30, 29], [40, 40]] if name == "hin_always" else None)
+        d["z"] = gate_like(2, 80, 2, 8, torch.float32, 9) if name.startswith("gate") else None
         dy = dy_like(2, 80, 2, 8, torch.float32, 9)
         dfinal = None if name == "hin_always" else dfinal_like(2, 2, 8, 16, 9)
         ref = oracle_bwd(d, dy, dfinal)
         caught = False
         for reverse in (False, True):
             try:
-                out = emu_bwd.run(d, dy, dfinal, chunk_size=16, reverse=reverse)
+                out = emu_bwd.run(d, dy, dfinal, chunk_size=16, reverse=reverse, z=d["z"])
                 compare(out, ref)
             except (AssertionError, RuntimeError):
                 caught = True

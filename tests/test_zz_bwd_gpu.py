@@ -22,7 +22,7 @@ def _gpu_bwd(d, dy, dfinal, chunk=0):
     c = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     g = ssd.bwd(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], dy.cuda(), initial_states=c["initial_states"],
                 seq_idx=c.get("seq_idx"), dfinal_states=None if dfinal is None else dfinal.cuda(), chunk_size=chunk,
-                want_dD=True, want_dinitial_states=True)
+                want_dD=True, want_dinitial_states=True, z=c.get("z"))
     torch.cuda.synchronize()
     out = {k: (None if v is None else v.cpu().numpy()) for k, v in g.items()}
     out["dh0"] = out.pop("dinitial_states")
@@ -122,3 +122,17 @@ def test_simulated_seqpar_backward_matches_the_whole_sequence(cuts):
     for k, v in got.items():
         rel = np.linalg.norm(v - ref[k]) / np.linalg.norm(ref[k])
         assert rel <= 1e-4, (k, rel)
+
+
+def test_autograd_function_through_the_gate():
+    """ssd_chunked with a gate z: y * SiLU(z) forward, dz and the SSD's
+    gradients backward."""
+    d, dy, _, _ = case_inputs(next(c for c in CASES if c[0] == "gated_f32_ragged_Q16"))
+    c = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    leaves = {k: c[k].clone().requires_grad_(True) for k in ("x", "dt", "A", "B", "C", "D", "initial_states", "z")}
+    y, _ = ssd.ssd_chunked(leaves["x"], leaves["dt"], leaves["A"], leaves["B"], leaves["C"], leaves["D"],
+                           chunk_size=64, initial_states=leaves["initial_states"], z=leaves["z"])
+    (y.double() * dy.cuda().double()).sum().backward()
+    ref = oracle_bwd(d, dy, None)
+    names = {"dx": "x", "ddt": "dt", "dA": "A", "dB": "B", "dC": "C", "dD": "D", "dh0": "initial_states", "dz": "z"}
+    compare({k: leaves[v].grad.float().cpu().numpy() for k, v in names.items()}, ref)
