@@ -72,11 +72,17 @@ def test_mutant_is_caught(name):
 # Planted mistakes in a copy of oracle/block.py (conv1d + SiLU, gate): each must
 # fail some pin of tests/test_block_oracle_pins.py.
 BLOCK_MUTANTS = {
-    "tap_direction_reversed": ("pre += w[None, None, :, k] * src", "pre += w[None, None, :, K - 1 - k] * src"),
+    "tap_direction_reversed": ("pre += w[None, None, :, k] * src",
+                               "pre += w[None, None, :, w.shape[1] - 1 - k] * src"),
     "taps_shifted_by_one": ("shift = K - 1 - k", "shift = K - k"),
     "bias_dropped": ("pre = np.zeros((b, L, C)) if bias is None", "pre = np.zeros((b, L, C)) if True"),
     "packing_cut_ignored": ("            src *= same[:, :, None]\n", ""),
     "silu_sign_flipped": ("return v / (1.0 + np.exp(-v))", "return v / (1.0 + np.exp(v))"),
+    "conv_grad_lands_on_the_output_token": ("du[:, : L - shift] += (w[None, None, :, k] * g * valid)[:, shift:]",
+                                            "du += w[None, None, :, k] * g * valid"),
+    "conv_grad_without_the_silu_slope": ("g = as_f64(dout) * silu_grad(_pre(u, w, bias, seq_idx))",
+                                         "g = as_f64(dout) + 0.0 * _pre(u, w, bias, seq_idx)"),
+    "conv_grad_ignores_the_packing_cut": ("            valid[:, shift:, 0] = seq[:, shift:] == seq[:, : L - shift]\n", ""),
 }
 
 
@@ -100,7 +106,9 @@ def test_block_mutant_fails_a_pin(name, monkeypatch, tmp_path):
     pins_run = [lambda: bpins.test_silu_is_x_times_the_logistic(),
                 *[functools.partial(bpins.test_each_channel_is_a_numpy_convolution, K) for K in (1, 2, 4)],
                 bpins.test_an_impulse_gives_back_the_filter, bpins.test_the_first_token_sees_only_itself,
-                bpins.test_packed_sequences_equal_their_parts_run_alone, bpins.test_gate]
+                bpins.test_packed_sequences_equal_their_parts_run_alone, bpins.test_gate,
+                *[functools.partial(bpins.test_conv_backward_matches_autograd, *c) for c in
+                  [(4, True, None), (4, True, [[7, 1, 22], [30]])]]]
     failed = 0
     for pin in pins_run:
         try:
