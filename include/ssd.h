@@ -264,6 +264,43 @@ typedef struct {
 
 SSD_API ssd_status ssd_conv1d_silu(const ssd_conv_args* args, void* stream);
 
+/* The backward of ssd_conv1d_silu: given dout = dLoss/dout, with the
+ * pre-activation a (bias + the taps) recomputed and g = dout * SiLU'(a)
+ * (SiLU'(v) = s (1 + v (1 - s)), s = 1 / (1 + e^-v)):
+ *
+ *   du[b,s,c]   = sum over the taps k that reach s from t = s + (K-1) - k
+ *                 (same sequence, t < L) of weight[c,k] g[b,t,c]
+ *   dweight[c,k] = sum_{b,t} g[b,t,c] u[b, t-(K-1)+k, c]   (taps the forward takes)
+ *   dbias[c]     = sum_{b,t} g[b,t,c]
+ *
+ * Sizes, u, weight, bias and seq_idx as in ssd_conv_args, width 1..4 (else
+ * SSD_ERR_UNSUPPORTED).  Gradients are fp32.  dweight and dbias are summed in
+ * a fixed order (fp64 over per-strip partials), so results are deterministic.
+ * Device pointers owned by the caller; outputs must not overlap the inputs
+ * or the workspace.  Asynchronous on `stream`; nothing is enqueued when the
+ * arguments are rejected (SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED,
+ * SSD_ERR_WORKSPACE as for ssd_bwd). */
+typedef struct {
+  int64_t batch, seqlen, channels, width;
+  ssd_dtype dtype;         /* of u and dout                                  */
+  const void* u;           /* (b,L,channels) dtype                           */
+  const float* weight;     /* (channels,width) fp32                          */
+  const float* bias;       /* (channels) fp32, or NULL for 0                 */
+  const int32_t* seq_idx;  /* (b,L) int32 packed-sequence ids, or NULL       */
+  const void* dout;        /* (b,L,channels) dtype, dLoss/dout               */
+  float* du;               /* (b,L,channels) fp32, output                    */
+  float* dweight;          /* (channels,width) fp32, output                  */
+  float* dbias;            /* (channels) fp32 output, or NULL to skip        */
+  void* workspace;         /* ssd_conv1d_silu_bwd_workspace_size bytes,
+                              256-byte aligned; contents on entry do not matter */
+  size_t workspace_bytes;
+} ssd_conv_bwd_args;
+
+/* Workspace bytes ssd_conv1d_silu_bwd needs (sizes only), or 0 if invalid. */
+SSD_API size_t ssd_conv1d_silu_bwd_workspace_size(const ssd_conv_bwd_args* args);
+
+SSD_API ssd_status ssd_conv1d_silu_bwd(const ssd_conv_bwd_args* args, void* stream);
+
 /* The backward pass of ssd_fwd: the gradients of a loss with respect to every
  * input, given dy = dLoss/dy and optionally dfinal = dLoss/dfinal_states.
  * The pages give the forward recurrence (sources above) and say that the

@@ -21,7 +21,8 @@ from typing import Optional
 
 import torch
 
-__all__ = ["fwd", "bwd", "BwdArgs", "bwd_workspace_size", "bwd_chunk_size", "ssd_chunked", "step", "StepArgs", "total_decay", "state_fold", "conv1d_silu", "ConvArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
+__all__ = ["fwd", "bwd", "BwdArgs", "bwd_workspace_size", "bwd_chunk_size", "ssd_chunked",
+           "conv1d_silu_bwd", "ConvBwdArgs", "causal_conv1d_silu", "step", "StepArgs", "total_decay", "state_fold", "conv1d_silu", "ConvArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
            "SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED", "SSD_ERR_WORKSPACE", "SSD_ERR_CUDA",
            "SSD_F32", "SSD_BF16", "SSD_FLAG_GENERIC"]
 
@@ -87,6 +88,17 @@ class BwdArgs(ctypes.Structure):
     ]
 
 
+class ConvBwdArgs(ctypes.Structure):
+    """Mirror of ``ssd_conv_bwd_args``."""
+    _fields_ = [(n, ctypes.c_int64) for n in ("batch", "seqlen", "channels", "width")] + [
+        ("dtype", ctypes.c_int),
+        ("u", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+        ("seq_idx", ctypes.c_void_p), ("dout", ctypes.c_void_p),
+        ("du", ctypes.c_void_p), ("dweight", ctypes.c_void_p), ("dbias", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -113,6 +125,10 @@ def _load() -> ctypes.CDLL:
     L.ssd_bwd_workspace_size.restype = ctypes.c_size_t
     L.ssd_bwd_chunk_size.argtypes = [ctypes.POINTER(BwdArgs)]
     L.ssd_bwd_chunk_size.restype = ctypes.c_int64
+    L.ssd_conv1d_silu_bwd.argtypes = [ctypes.POINTER(ConvBwdArgs), ctypes.c_void_p]
+    L.ssd_conv1d_silu_bwd.restype = ctypes.c_int
+    L.ssd_conv1d_silu_bwd_workspace_size.argtypes = [ctypes.POINTER(ConvBwdArgs)]
+    L.ssd_conv1d_silu_bwd_workspace_size.restype = ctypes.c_size_t
     L.ssd_conv1d_silu.argtypes = [ctypes.POINTER(ConvArgs), ctypes.c_void_p]
     L.ssd_conv1d_silu.restype = ctypes.c_int
     L.ssd_total_decay.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int64] * 3 + [
@@ -518,3 +534,62 @@ def ssd_chunked(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Ten
     if seq_idx is not None and num_seqs is None:
         num_seqs = int(seq_idx.max().item()) + 1
     return _SSDChunked.apply(x, dt, A, B, C, D, initial_states, seq_idx, num_seqs, chunk_size, z)
+
+
+def conv1d_silu_bwd(u: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor], dout: torch.Tensor,
+                    seq_idx: Optional[torch.Tensor] = None, want_dbias: bool = True) -> tuple:
+    """``ssd_conv1d_silu_bwd``: (du (b,L,C), dweight (C,K), dbias (C) or None),
+    all fp32, for dout = dLoss/d(conv1d_silu(u, weight, bias, seq_idx))."""
+    if u.dim() != 3 or weight.dim() != 2 or weight.shape[0] != u.shape[2]:
+        raise ValueError("expected u (b,L,C) and weight (C,K)")
+    if dout.dtype != u.dtype or tuple(dout.shape) != tuple(u.shape):
+        raise ValueError("dout must be like u")
+    if u.dtype not in (torch.float32, torch.bfloat16) or weight.dtype != torch.float32 \
+            or (bias is not None and (bias.dtype != torch.float32 or tuple(bias.shape) != (u.shape[2],))):
+        raise TypeError("u float32 or bfloat16; weight and bias float32 (bias of shape (C,))")
+    if seq_idx is not None and (seq_idx.dtype != torch.int32 or tuple(seq_idx.shape) != tuple(u.shape[:2])):
+        raise ValueError("seq_idx must be int32 (b,L)")
+    for name, t in (("u", u), ("weight", weight), ("bias", bias), ("seq_idx", seq_idx), ("dout", dout)):
+        if t is not None and (t.device != u.device or u.device.type != "cuda" or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor on {u.device}")
+    b, L, C = u.shape
+    f32 = dict(device=u.device, dtype=torch.float32)
+    du, dw = torch.empty(b, L, C, **f32), torch.empty(weight.shape, **f32)
+    db = torch.empty(C, **f32) if want_dbias else None
+    a = ConvBwdArgs()
+    a.batch, a.seqlen, a.channels, a.width = b, L, C, weight.shape[1]
+    a.dtype = SSD_BF16 if u.dtype == torch.bfloat16 else SSD_F32
+    a.u, a.weight, a.bias, a.seq_idx, a.dout = _ptr(u), _ptr(weight), _ptr(bias), _ptr(seq_idx), _ptr(dout)
+    a.du, a.dweight, a.dbias = _ptr(du), _ptr(dw), _ptr(db)
+    need = int(lib.ssd_conv1d_silu_bwd_workspace_size(ctypes.byref(a)))
+    if need == 0:
+        raise SSDError(lib.ssd_conv1d_silu_bwd(ctypes.byref(a), _stream(u)))
+    ws = torch.empty(need, dtype=torch.uint8, device=u.device)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), need
+    st = lib.ssd_conv1d_silu_bwd(ctypes.byref(a), _stream(u))
+    if st != SSD_OK:
+        raise SSDError(st)
+    return du, dw, db
+
+
+class _CausalConv1dSilu(torch.autograd.Function):
+    """``conv1d_silu`` forward, ``conv1d_silu_bwd`` backward."""
+
+    @staticmethod
+    def forward(ctx, u, weight, bias, seq_idx):
+        ctx.save_for_backward(u, weight, bias, seq_idx)
+        return conv1d_silu(u, weight, bias, seq_idx)
+
+    @staticmethod
+    def backward(ctx, dout):
+        u, weight, bias, seq_idx = ctx.saved_tensors
+        du, dw, db = conv1d_silu_bwd(u, weight, bias, dout.to(u.dtype).contiguous(), seq_idx,
+                                     want_dbias=bias is not None and ctx.needs_input_grad[2])
+        return du.to(u.dtype), dw, db, None
+
+
+def causal_conv1d_silu(u: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                       seq_idx: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Differentiable ``conv1d_silu``: the backward runs ``ssd_conv1d_silu_bwd``
+    (the pre-activation is recomputed, nothing but the inputs is kept)."""
+    return _CausalConv1dSilu.apply(u, weight, bias, seq_idx)

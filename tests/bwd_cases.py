@@ -91,3 +91,42 @@ def compare(out, ref, keys=KEYS):
         mad = np.abs(got - want).max()
         assert rel <= REL_L2, f"{k}: rel L2 {rel:.3g}"
         assert mad <= MAX_ABS * max(1.0, np.abs(want).max()), f"{k}: max abs {mad:.3g}"
+
+
+# conv1d + SiLU backward: id, (b, L, C, K), dtype, per-row packed lengths or None, bias
+CONV_CASES = [
+    ("f32_K4_strips", (2, 70, 300, 4), "f32", None, True),
+    ("bf16_K3_packed", (2, 64, 260, 3), "bf16", [[7, 1, 40, 16], [1, 63]], False),
+    ("f32_K1", (1, 33, 5, 1), "f32", None, True),
+    ("f32_one_token", (1, 1, 8, 4), "f32", None, True),
+    ("f32_K2_packed_on_a_strip_edge", (1, 64, 8, 2), "f32", [[32, 32]], True),
+    ("bf16_K4_c1_channels", (1, 100, 5376, 4), "bf16", None, True),
+]
+
+
+def conv_case_inputs(case):
+    """(u, weight, bias, dout, seq_idx) of one CONV_CASES entry."""
+    name, (b, L, C, K), dtype, packed, with_bias = case
+    g = torch.Generator().manual_seed(L * 7 + C + K)
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    u = torch.randn(b, L, C, generator=g).to(dt)
+    w = torch.randn(C, K, generator=g) * 0.5
+    bias = torch.randn(C, generator=g) * 0.1 if with_bias else None
+    dout = torch.randn(b, L, C, generator=g).to(dt)
+    seq = si.seq_idx_from_lengths(packed)[0] if packed else None
+    return u, w, bias, dout, seq
+
+
+def conv_compare(du, dw, db, ref):
+    """du, dw, dbias against the fp64 oracle's (du, dw, dbias): the same bounds
+    as the SSD backward (fp32 sums of at most K terms per du, b L terms per
+    dw and dbias, the latter in fp64 over per-strip partials)."""
+    for name, got, want in (("du", du, ref[0]), ("dw", dw, ref[1]), ("dbias", db, ref[2])):
+        if got is None:
+            continue
+        got = np.asarray(got, dtype=np.float64)
+        assert got.shape == want.shape, name
+        assert np.isfinite(got).all(), name
+        rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+        assert rel <= REL_L2, f"{name}: rel L2 {rel:.3g}"
+        assert np.abs(got - want).max() <= MAX_ABS * max(1.0, np.abs(want).max()), name

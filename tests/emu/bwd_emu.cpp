@@ -20,6 +20,7 @@
 #include <vector>
 
 #include "cuda_emu.h"
+#include "emu_launch.h"
 #include "ssd.h"
 #include "ssd_bwd.cuh"
 
@@ -55,111 +56,8 @@ float* nan_floats(size_t n) {
   return p;
 }
 
-#ifdef SSD_EMU_THREADS
-// Each block: kThreads host threads meeting at a std::barrier.
-struct EmuLaunch {
-  int launches = 0;
-  bool reverse = false;  // (thread order only matters for fibers)
-  bool operator()(void (*kern)(ssd::bwd::KArgs), unsigned grid, size_t smem, const ssd::bwd::KArgs& k) {
-    using ssd::bwd::kThreads;
-    if (smem > ssd::bwd::kSmemLimit) return false;
-    ++launches;
-    gridDim = dim3{grid, 1, 1};
-    blockDim = dim3{(unsigned)kThreads, 1, 1};
-    for (unsigned bi = 0; bi < grid; ++bi) {
-      void* sm = smem ? std::malloc(smem) : nullptr;
-      if (sm) std::memset(sm, 0xff, smem);
-      std::barrier<> bar(kThreads);
-      emu::g_barrier = &bar;
-      emu::g_smem = static_cast<float*>(sm);
-      std::vector<std::thread> th;
-      th.reserve(kThreads);
-      for (int t = 0; t < kThreads; ++t) {
-        th.emplace_back([&bar, kern, &k, bi, t] {
-          threadIdx = dim3{(unsigned)t, 1, 1};
-          blockIdx = dim3{bi, 1, 1};
-          kern(k);
-          bar.arrive_and_drop();  // an exited thread no longer holds back __syncthreads
-        });
-      }
-      for (auto& x : th) x.join();
-      std::free(sm);
-    }
-    return true;
-  }
-  bool record(void*) { return true; }  // no events on the host
-};
-#else
-// Each block: kThreads fibers on this host thread.  A round resumes every
-// live fiber once, in thread order (or reversed), and each runs up to its
-// next __syncthreads or its end; so no fiber starts phase k+1 before all
-// have finished phase k, as a CTA barrier guarantees, and a value read
-// across threads without a barrier between is seen unwritten (NaN) in one
-// of the two orders.
-constexpr size_t kFiberStack = 256 * 1024;
-void (*g_kern)(ssd::bwd::KArgs) = nullptr;
-const ssd::bwd::KArgs* g_args = nullptr;
-std::vector<char> g_done;
-int g_cur = 0;
-
-void fiber_entry() {
-  g_kern(*g_args);
-  g_done[g_cur] = 1;  // returning resumes the scheduler (uc_link)
-}
-
-struct EmuLaunch {
-  int launches = 0;
-  bool reverse = false;
-  std::vector<ucontext_t> ctx;
-  std::vector<char*> stacks;
-  ~EmuLaunch() {
-    for (char* p : stacks) std::free(p);
-  }
-  bool operator()(void (*kern)(ssd::bwd::KArgs), unsigned grid, size_t smem, const ssd::bwd::KArgs& k) {
-    using ssd::bwd::kThreads;
-    if (smem > ssd::bwd::kSmemLimit) return false;
-    ++launches;
-    if (stacks.empty()) {
-      ctx.resize(kThreads);
-      for (int t = 0; t < kThreads; ++t) stacks.push_back(static_cast<char*>(std::malloc(kFiberStack)));
-    }
-    gridDim = dim3{grid, 1, 1};
-    blockDim = dim3{(unsigned)kThreads, 1, 1};
-    g_kern = kern;
-    g_args = &k;
-    g_done.assign(kThreads, 0);
-    for (unsigned bi = 0; bi < grid; ++bi) {
-      void* sm = smem ? std::malloc(smem) : nullptr;
-      if (sm) std::memset(sm, 0xff, smem);
-      emu::g_smem = static_cast<float*>(sm);
-      blockIdx = dim3{bi, 1, 1};
-      for (int t = 0; t < kThreads; ++t) {
-        getcontext(&ctx[t]);
-        ctx[t].uc_stack.ss_sp = stacks[t];
-        ctx[t].uc_stack.ss_size = kFiberStack;
-        ctx[t].uc_link = &emu::g_sched;
-        makecontext(&ctx[t], fiber_entry, 0);
-        g_done[t] = 0;
-      }
-      int live = kThreads;
-      while (live > 0) {
-        for (int j = 0; j < kThreads; ++j) {
-          const int t = reverse ? kThreads - 1 - j : j;
-          if (g_done[t]) continue;
-          threadIdx = dim3{(unsigned)t, 1, 1};
-          g_cur = t;
-          emu::g_self = &ctx[t];
-          swapcontext(&emu::g_sched, &ctx[t]);
-          if (g_done[t]) --live;
-        }
-      }
-      std::free(sm);
-    }
-    return true;
-  }
-  bool record(void*) { return true; }  // no events on the host
-};
-#endif
+static_assert(emu::kThreads == ssd::bwd::kThreads, "the emulator launches the kernels' block size");
+using EmuLaunch = emu::Launch<ssd::bwd::KArgs>;
 
 }  // namespace
 

@@ -1,7 +1,7 @@
 """Build and run the test-only host emulation of the backward kernels
-(``tests/emu/bwd_emu.cpp``): the kernels of ``csrc/ssd_bwd.cuh`` and the
-host plan that launches them, compiled by g++ with a sanitizer and run on
-small inputs on the CPU.  Used by the CPU tests only, to check indexing,
+(``tests/emu/bwd_emu.cpp`` for ``csrc/ssd_bwd.cuh``, ``tests/emu/conv_bwd_emu.cpp``
+for ``csrc/ssd_conv_bwd.cuh``): the kernels and the host plan that launches
+them, compiled by g++ with a sanitizer and run on small inputs on the CPU.  Used by the CPU tests only, to check indexing,
 barriers and arithmetic before the code runs on a GPU; the GPU tests are the
 parity claim."""
 from __future__ import annotations
@@ -18,6 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "emu", "bwd_emu.cpp")
 SHIM = os.path.join(HERE, "emu", "cuda_emu.h")
+LAUNCH = os.path.join(HERE, "emu", "emu_launch.h")
 KERNELS = os.path.join(ROOT, "mamba_ssd_chunked_03_b200", "csrc", "ssd_bwd.cuh")
 HEADER = os.path.join(ROOT, "include", "ssd.h")
 OUT = os.path.join(HERE, "emu", "_build")
@@ -31,16 +32,21 @@ def available() -> bool:
     return shutil.which("g++") is not None
 
 
-def build(kind: str = "asan") -> str:
+CONV_SRC = os.path.join(HERE, "emu", "conv_bwd_emu.cpp")
+CONV_KERNELS = os.path.join(ROOT, "mamba_ssd_chunked_03_b200", "csrc", "ssd_conv_bwd.cuh")
+
+
+def build(kind: str = "asan", which: str = "ssd") -> str:
     os.makedirs(OUT, exist_ok=True)
-    exe = os.path.join(OUT, f"bwd_emu_{kind}")
-    deps = [SRC, SHIM, KERNELS, HEADER, os.path.abspath(__file__)]
+    src, kernels = (SRC, KERNELS) if which == "ssd" else (CONV_SRC, CONV_KERNELS)
+    exe = os.path.join(OUT, f"{'bwd' if which == 'ssd' else 'conv_bwd'}_emu_{kind}")
+    deps = [src, SHIM, LAUNCH, kernels, HEADER, os.path.abspath(__file__)]
     if os.path.exists(exe) and os.path.getmtime(exe) >= max(os.path.getmtime(d) for d in deps):
         return exe
     tmp = exe + f".tmp{os.getpid()}"
     cmd = ["g++", "-std=c++20", "-O1", "-g", "-fno-omit-frame-pointer", *SANITIZERS[kind], "-pthread",
-           "-I", os.path.join(ROOT, "include"), "-I", os.path.dirname(KERNELS), "-I", os.path.dirname(SHIM),
-           SRC, "-o", tmp]
+           "-I", os.path.join(ROOT, "include"), "-I", os.path.dirname(kernels), "-I", os.path.dirname(SHIM),
+           src, "-o", tmp]
     subprocess.run(cmd, check=True)
     os.replace(tmp, exe)
     return exe
@@ -97,4 +103,37 @@ def run(inp: dict, dy, dfinal=None, chunk_size: int = 0, want_dD: bool = True, w
         for k, shp in shapes.items():
             path = os.path.join(d, k + ".bin")
             out[k] = np.fromfile(path, dtype=np.float32).reshape(shp) if os.path.exists(path) else None
+        return out
+
+
+def run_conv(u, weight, bias, dout, seq_idx=None, want_dbias: bool = True, kind: str = "asan",
+             reverse: bool = False, timeout: int = 600) -> dict:
+    """Run the emulated conv1d + SiLU backward.  Returns {"status",
+    "launches", and du (b,L,C), dw (C,K), dbias (C) as fp32 numpy arrays}."""
+    exe = build(kind, which="conv")
+    b, L, C = u.shape
+    K = weight.shape[1]
+    with tempfile.TemporaryDirectory() as d:
+        for name, v in (("u", u), ("w", weight), ("bias", bias), ("seq", seq_idx), ("dout", dout)):
+            if v is not None:
+                with open(os.path.join(d, name + ".bin"), "wb") as f:
+                    f.write(_raw(v))
+        kv = dict(batch=b, seqlen=L, channels=C, width=K, dtype=1 if u.dtype == torch.bfloat16 else 0,
+                  has_bias=int(bias is not None), has_seq=int(seq_idx is not None), want_dbias=int(want_dbias),
+                  reverse=int(reverse))
+        with open(os.path.join(d, "args.txt"), "w") as f:
+            f.write("".join(f"{k} {v}\n" for k, v in kv.items()))
+        env = dict(os.environ)
+        env.setdefault("ASAN_OPTIONS", "detect_leaks=0")
+        r = subprocess.run([exe, d], capture_output=True, text=True, timeout=timeout, env=env)
+        words = r.stdout.split()
+        if r.returncode not in (0, 1) or len(words) < 4 or words[0] != "status":
+            raise RuntimeError(f"emulator failed (rc {r.returncode}):\n{r.stdout}\n{r.stderr[-4000:]}")
+        out = {"status": int(words[1]), "launches": int(words[3])}
+        if out["status"] != 0:
+            return out
+        out["du"] = np.fromfile(os.path.join(d, "du.bin"), dtype=np.float32).reshape(b, L, C)
+        out["dw"] = np.fromfile(os.path.join(d, "dw.bin"), dtype=np.float32).reshape(C, K)
+        p = os.path.join(d, "dbias.bin")
+        out["dbias"] = np.fromfile(p, dtype=np.float32) if os.path.exists(p) else None
         return out

@@ -357,3 +357,47 @@ def test_bwd_chunk_size_query():
     assert q(dstate=256, headdim=256) == 0  # one 256 x 256 state alone exceeds a CTA's shared memory
     assert q(chunk_size=65) == 0 and q(batch=0) == 0
     assert ssd.lib.ssd_bwd_chunk_size(None) == 0
+
+
+def test_conv_bwd_struct_layout_matches_the_compiled_header():
+    names = [f[0] for f in ssd.ConvBwdArgs._fields_]
+    got = _c_layout(names, "ssd_conv_bwd_args")
+    assert got[:-1] == [getattr(ssd.ConvBwdArgs, n).offset for n in names]
+    assert got[-1] == ctypes.sizeof(ssd.ConvBwdArgs)
+
+
+def _conv_bwd_args(**kw):
+    a = ssd.ConvBwdArgs()
+    a.batch, a.seqlen, a.channels, a.width = 2, 64, 64, 4
+    a.dtype = ssd.SSD_BF16
+    for i, n in enumerate(("u", "weight", "dout", "du", "dweight")):
+        setattr(a, n, 4096 * (i + 1))  # never dereferenced: every case below is rejected on the host
+    a.workspace = 1 << 30
+    a.workspace_bytes = ssd.lib.ssd_conv1d_silu_bwd_workspace_size(ctypes.byref(a))
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({"batch": 0}, ssd.SSD_ERR_INVALID_ARG),
+    ({"dtype": 5}, ssd.SSD_ERR_INVALID_ARG),
+    ({"u": None}, ssd.SSD_ERR_INVALID_ARG),
+    ({"dout": None}, ssd.SSD_ERR_INVALID_ARG),
+    ({"dweight": None}, ssd.SSD_ERR_INVALID_ARG),
+    ({"workspace": None}, ssd.SSD_ERR_WORKSPACE),
+    ({"workspace_bytes": 16}, ssd.SSD_ERR_WORKSPACE),
+    ({"workspace": (1 << 30) + 32}, ssd.SSD_ERR_INVALID_ARG),
+    ({"width": 5}, ssd.SSD_ERR_UNSUPPORTED),
+])
+def test_conv_bwd_rejects_bad_arguments(kw, status):
+    assert ssd.lib.ssd_conv1d_silu_bwd(ctypes.byref(_conv_bwd_args(**kw)), None) == status
+
+
+def test_conv_bwd_workspace_size():
+    size = lambda **kw: ssd.lib.ssd_conv1d_silu_bwd_workspace_size(ctypes.byref(_conv_bwd_args(**kw)))
+    # per (row, strip of 32 tokens) and channel: K dweight partials and one dbias partial, fp32
+    assert size() == 2 * 2 * 64 * 5 * 4
+    assert size(seqlen=65) == 2 * 3 * 64 * 5 * 4
+    assert size(batch=0) == 0 and size(width=5) == 0
+    assert ssd.lib.ssd_conv1d_silu_bwd(None, None) == ssd.SSD_ERR_INVALID_ARG

@@ -13,7 +13,9 @@ import torch
 
 import mamba_ssd_chunked_03_b200 as ssd
 import oracle
-from bwd_cases import CASES, KEYS, case_inputs, compare, dfinal_like, dy_like, inputs, oracle_bwd
+from bwd_cases import (CASES, CONV_CASES, KEYS, case_inputs, compare, conv_case_inputs, conv_compare, dfinal_like,
+                       dy_like, inputs, oracle_bwd)
+from oracle import block
 
 pytestmark = pytest.mark.gpu
 
@@ -136,3 +138,24 @@ def test_autograd_function_through_the_gate():
     ref = oracle_bwd(d, dy, None)
     names = {"dx": "x", "ddt": "dt", "dA": "A", "dB": "B", "dC": "C", "dD": "D", "dh0": "initial_states", "dz": "z"}
     compare({k: leaves[v].grad.float().cpu().numpy() for k, v in names.items()}, ref)
+
+
+@pytest.mark.parametrize("case", CONV_CASES, ids=lambda c: c[0])
+def test_conv_backward_matches_oracle(case):
+    u, w, bias, dout, seq = conv_case_inputs(case)
+    cu = lambda t: None if t is None else t.cuda()
+    du, dw, db = ssd.conv1d_silu_bwd(cu(u), cu(w), cu(bias), cu(dout), cu(seq))
+    torch.cuda.synchronize()
+    conv_compare(du.cpu().numpy(), dw.cpu().numpy(), None if db is None else db.cpu().numpy(),
+                 block.conv1d_silu_bwd(u, w, bias, dout, seq))
+
+
+def test_conv_autograd_function_routes_through_the_library():
+    u, w, bias, dout, seq = conv_case_inputs(CONV_CASES[1])
+    bias = torch.randn(w.shape[0]) * 0.1
+    leaves = [t.cuda().requires_grad_(True) for t in (u.float(), w, bias)]
+    out = ssd.causal_conv1d_silu(leaves[0].to(u.dtype), leaves[1], leaves[2], seq.cuda())
+    (out.double() * dout.cuda().double()).sum().backward()
+    du, dw, db = block.conv1d_silu_bwd(u, w, bias, dout, seq)
+    conv_compare(leaves[0].grad.cpu().numpy(), leaves[1].grad.cpu().numpy(), leaves[2].grad.cpu().numpy(),
+                 (du, dw, db))
