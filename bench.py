@@ -220,6 +220,8 @@ def run_reference_op(args):
     import oracle
     if args.op == "bwd":
         return run_reference_bwd(args)
+    if args.op == "conv_bwd":
+        return run_reference_conv_bwd(args)
     if args.op == "step":
         b, H, P, N, G = args.step_batch, 80, 64, 128, 1
         shape = si.SSDShape("decode", b, 1, H, P, N, G, 64, "bf16", h0_std=0.5, seed=11)
@@ -253,6 +255,35 @@ def run_reference_op(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload, "sample": sample},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference_conv_bwd(args):
+    """``--impl reference --op conv_bwd``: the conv backward oracle, one batch
+    row of c1's xBC tensor per step, on the host."""
+    from oracle import block
+    b, L, C, K = 8, 2048, 80 * 64 + 2 * 1 * 128, 4
+    gen = torch.Generator().manual_seed(13)
+    u = torch.randn(1, L, C, generator=gen).to(torch.bfloat16)
+    w, bias = torch.randn(C, K, generator=gen) * 0.5, torch.randn(C, generator=gen) * 0.1
+    dout = torch.randn(1, L, C, generator=gen).to(torch.bfloat16)
+    for _ in range(args.warmup):
+        block.conv1d_silu_bwd(u, w, bias, dout)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        block.conv1d_silu_bwd(u, w, bias, dout)
+    el = time.perf_counter() - t
+    value = L * args.steps / el
+    sample = f"{args.steps} batch rows of b{b} L{L} channels {C} width {K} (numpy, one process)"
+    line = {
+        "impl": "reference", "metric": "Mamba-2 block causal conv1d + SiLU backward tokens/s", "value": value,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "config": {"workload": "conv1d+SiLU backward, c1 xBC", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -504,6 +535,104 @@ def run_conv(args, dist, dev, world, rank):
     return 0
 
 
+def run_conv_bwd(args, dist, dev, world, rank):
+    """``--op conv_bwd``: the conv1d + SiLU backward on c1's xBC tensor (b 8,
+    L 2048, 5376 channels, width 4, bf16 in, fp32 gradients).  Bound by HBM:
+    u and dout read once, du written once (fp32), plus the per-strip weight
+    partials."""
+    import mamba_ssd_chunked_03_b200 as ssd
+    b, L, C, K = 8, 2048, 80 * 64 + 2 * 1 * 128, 4
+    gen = torch.Generator().manual_seed(13 + rank)
+    u_h = torch.randn(b, L, C, generator=gen).to(torch.bfloat16)
+    w_h = torch.randn(C, K, generator=gen) * 0.5
+    bias_h = torch.randn(C, generator=gen) * 0.1
+    dout_h = torch.randn(b, L, C, generator=gen).to(torch.bfloat16)
+    u, w, bias, dout = u_h.to(dev), w_h.to(dev), bias_h.to(dev), dout_h.to(dev)
+
+    def step():
+        return ssd.conv1d_silu_bwd(u, w, bias, dout)
+
+    K_ = args.steps
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_uuid(dev))
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K_):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clock_stats = clocks.stop()
+    ms_step = max_over_ranks(e0.elapsed_time(e1), dist, dev) / K_
+
+    pinned_u, pinned_d = u_h.pin_memory(), dout_h.pin_memory()
+    du_host = torch.empty(b, L, C, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        u.copy_(pinned_u, non_blocking=True)
+        dout.copy_(pinned_d, non_blocking=True)
+        du_, _, _ = step()
+        du_host.copy_(du_, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    E = max(3, min(K_, 20))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(E):
+        e2e_step()
+    a1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev) / E
+
+    strips = -(-L // 32)
+    nbytes = 2 * b * L * C * 2 + b * L * C * 4 + 2 * b * strips * C * (K + 1) * 4 + C * (K + 1) * 4
+    peaks = load_peaks()
+    achieved = nbytes / (ms_step / 1e3) / 1e9
+    tokens = b * L
+    line = {
+        "metric": "Mamba-2 block causal conv1d + SiLU backward tokens/s", "value": tokens * world / (ms_step / 1e3),
+        "unit": "tokens/s", "n_gpus": world, "steps": K_, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"conv1d+SiLU backward: b{b} L{L} channels {C} (c1 xBC) width {K}, bf16 in, "
+                               f"fp32 gradients",
+                   "l2": f"no flush: u + dout + du {nbytes / 1e6:.0f} MB > 126 MB L2",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                     "frac_datasheet": achieved / DATASHEET_HBM_GBS, "kernel": "k_conv_bwd (with its reduce)",
+                     "kernel_ms": ms_step, "traffic": None, "algorithmic_bytes": nbytes},
+        "e2e": {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 2 * b * L * C * 2, "d2h_bytes_per_step": b * L * C * 4, "steps": E},
+        "gpu_launches": 2 * K_,
+        "clocks": clock_stats,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import block  # test infrastructure: only this CPU-baseline leg uses it here
+        reps, t = 0, time.perf_counter()
+        while True:
+            block.conv1d_silu_bwd(u_h[:1], w_h, bias_h, dout_h[:1])  # one batch row per repetition
+            reps += 1
+            el = time.perf_counter() - t
+            if el >= min(args.cpu_seconds, 10.0):
+                break
+        line["cpu_baseline"] = {"value": reps * L / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{reps} batch rows of {L} tokens (numpy, one process), {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
 # ----------------------------------------------------------------------------- backward
 
 BWD_SHAPE = si.SSDShape("c1_bwd", 8, 2048, 80, 64, 128, 1, 64, "bf16", seed=1001)
@@ -698,9 +827,10 @@ def main():
     ap.add_argument("--generic", action="store_true", help="force the generic CUDA-core kernels")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--op", default="fwd", choices=["fwd", "step", "conv", "bwd"],
+    ap.add_argument("--op", default="fwd", choices=["fwd", "step", "conv", "bwd", "conv_bwd"],
                     help="fwd: the chunked forward (default); step: the recurrent decode step; "
-                         "conv: the block's causal conv1d + SiLU; bwd: the backward on c1's layout")
+                         "conv: the block's causal conv1d + SiLU; bwd: the backward on c1's layout; "
+                         "conv_bwd: the conv1d + SiLU backward")
     ap.add_argument("--step-batch", type=int, default=256, help="rows of the decode step (--op step)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -730,6 +860,8 @@ def main():
         return run_conv(args, dist, dev, world, rank)
     if args.op == "bwd":
         return run_bwd(args, dist, dev, world, rank)
+    if args.op == "conv_bwd":
+        return run_conv_bwd(args, dist, dev, world, rank)
 
     host = si.make_inputs(shape, seed=shape.seed + rank)
     num_seqs = host.get("num_seqs")

@@ -73,7 +73,7 @@ def test_reference_arm_under_torchrun_prints_once():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
 
 
-@pytest.mark.parametrize("op", ["step", "conv", "bwd"])
+@pytest.mark.parametrize("op", ["step", "conv", "bwd", "conv_bwd"])
 def test_reference_arm_of_the_other_ops(op):
     cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--op", op, "--steps", "1",
            "--warmup", "3", "--step-batch", "8"]
