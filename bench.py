@@ -719,7 +719,7 @@ def run_bwd(args, dist, dev, world, rank):
     Its kernels run on the CUDA cores, so the roofline is fp32 FMA throughput
     (bound "alu") on k_bwd_chunk, the dominant kernel."""
     import mamba_ssd_chunked_03_b200 as ssd
-    shape = BWD_SHAPE
+    shape = BWD_SHAPE.with_(batch=args.bwd_rows, nheads=args.bwd_heads)
     b, L, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
     host = bwd_inputs(shape, rank)
     names = ("x", "dt", "B", "C", "dy")
@@ -789,8 +789,10 @@ def run_bwd(args, dist, dev, world, rank):
         "metric": "SSD bwd tokens/s", "value": tokens * world / (ms_step / 1e3), "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": BWD_WORKLOAD,
-                   "l2": "no flush: inputs, gradients and the per-chunk states (GBs) exceed the 126 MB L2",
+        "config": {"workload": BWD_WORKLOAD if (b, H) == (8, 80) else
+                   BWD_WORKLOAD.replace("b8 ", f"b{b} ").replace("H80 ", f"H{H} "),
+                   "l2": "no flush: inputs, gradients and the per-chunk states exceed the 126 MB L2"
+                         if (b, H) == (8, 80) else "small case for profiling",
                    "parallelism": "replicas" if world > 1 else "single GPU", "bwd_chunk": Q},
         "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
                      "frac": achieved / FP32_PEAK_TFLOPS,
@@ -832,6 +834,8 @@ def main():
                          "conv: the block's causal conv1d + SiLU; bwd: the backward on c1's layout; "
                          "conv_bwd: the conv1d + SiLU backward")
     ap.add_argument("--step-batch", type=int, default=256, help="rows of the decode step (--op step)")
+    ap.add_argument("--bwd-rows", type=int, default=8, help="batch rows of --op bwd (8: c1)")
+    ap.add_argument("--bwd-heads", type=int, default=80, help="heads of --op bwd (80: c1)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
