@@ -59,7 +59,7 @@ def load_library(path: str) -> ctypes.CDLL:
     f.argtypes = [i64] * 6 + [vp] * 8 + [i64, vp, vp, vp, i64, ctypes.c_int]
     f.restype = ctypes.c_int
     g = lib.oracle_ssd_bwd
-    g.argtypes = [i64] * 6 + [vp] * 17 + [ctypes.c_int]
+    g.argtypes = [i64] * 6 + [vp] * 17 + [ctypes.c_int, vp, vp]
     g.restype = ctypes.c_int
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
@@ -151,7 +151,9 @@ def ssd_fwd(x, dt, A, B, C, D=None, initial_states=None, seq_idx=None, num_seqs=
 def ssd_bwd(x, dt, A, B, C, D=None, initial_states=None, dy=None, dfinal=None, seq_idx=None,
             nthreads: int = 0) -> dict:
     """The backward pass in C (fp64, OpenMP over (b, h)): gradients of
-    sum(dy * y) + sum(dfinal * final) as a dict like ``backward.ssd_bwd``."""
+    sum(dy * y) + sum(dfinal * final) as a dict like ``backward.ssd_bwd``,
+    plus dA_abs and dD_abs (H): the sums of the magnitudes of the terms
+    that dA and dD add up."""
     x32, dt32, A32, B32, C32 = (as_f32(v) for v in (x, dt, A, B, C))
     D32, h032, si = as_f32(D), as_f32(initial_states), as_i32(seq_idx)
     dy32, df32 = as_f32(dy), as_f32(dfinal)
@@ -164,6 +166,8 @@ def ssd_bwd(x, dt, A, B, C, D=None, initial_states=None, dy=None, dfinal=None, s
     dCh = np.zeros((b, L, H, N))
     dA_u = np.zeros(b * H)
     dD_u = np.zeros(b * H)
+    dA_abs = np.zeros(b * H)
+    dD_abs = np.zeros(b * H)
     dh0 = np.zeros((b, H, P, N)) if h032 is not None else None
 
     def ptr(a):
@@ -171,7 +175,8 @@ def ssd_bwd(x, dt, A, B, C, D=None, initial_states=None, dy=None, dfinal=None, s
 
     rc = _get_lib().oracle_ssd_bwd(b, L, H, P, N, G, ptr(x32), ptr(dt32), ptr(A32), ptr(B32), ptr(C32),
                                    ptr(D32), ptr(h032), ptr(si), ptr(dy32), ptr(df32), ptr(dx), ptr(ddt),
-                                   ptr(dBh), ptr(dCh), ptr(dA_u), ptr(dD_u), ptr(dh0), int(nthreads))
+                                   ptr(dBh), ptr(dCh), ptr(dA_u), ptr(dD_u), ptr(dh0), int(nthreads), ptr(dA_abs),
+                                   ptr(dD_abs))
     if rc != 0:
         raise RuntimeError(f"oracle_ssd_bwd failed with code {rc}")
     grp = np.arange(H) // (H // G)
@@ -181,4 +186,5 @@ def ssd_bwd(x, dt, A, B, C, D=None, initial_states=None, dy=None, dfinal=None, s
         dB[:, :, grp[h]] += dBh[:, :, h]
         dC[:, :, grp[h]] += dCh[:, :, h]
     return {"dx": dx, "ddt": ddt, "dA": dA_u.reshape(b, H).sum(axis=0), "dB": dB, "dC": dC,
-            "dD": None if D32 is None else dD_u.reshape(b, H).sum(axis=0), "dh0": dh0}
+            "dD": None if D32 is None else dD_u.reshape(b, H).sum(axis=0), "dh0": dh0,
+            "dA_abs": dA_abs.reshape(b, H).sum(axis=0), "dD_abs": dD_abs.reshape(b, H).sum(axis=0)}

@@ -109,7 +109,8 @@ static void oracle_bwd_unit(int64_t b, int64_t h, int64_t L, int64_t H, int64_t 
                             const float* x, const float* dt, const float* A, const float* Bm, const float* Cm,
                             const float* D, const float* h0, const int32_t* seq_idx, const float* dy,
                             const float* dfinal, double* dx, double* ddt, double* dA_unit, double* dBh,
-                            double* dCh, double* dD_unit, double* dh0, double* ckpt, double* blk, double* Gs) {
+                            double* dCh, double* dD_unit, double* dh0, double* ckpt, double* blk, double* Gs,
+                            double* dA_abs_unit, double* dD_abs_unit) {
   const int64_t g = h / (H / G), PN = P * N, nb = (L + 63) / 64;
   const double rate = (double)A[h];
   const double skip = D ? (double)D[h] : 0.0;
@@ -137,7 +138,7 @@ static void oracle_bwd_unit(int64_t b, int64_t h, int64_t L, int64_t H, int64_t 
   } else {
     memset(Gs, 0, sizeof(double) * (size_t)PN);
   }
-  double dA_acc = 0.0, dD_acc = 0.0;
+  double dA_acc = 0.0, dD_acc = 0.0, dA_abs = 0.0, dD_abs = 0.0;
   for (int64_t k = nb - 1; k >= 0; --k) {
     const int64_t t0 = 64 * k, t1 = (t0 + 64 < L) ? t0 + 64 : L;
     /* rebuild the block's states: blk[j] = h_{t0 + j}; the state before t0 is ckpt[k] */
@@ -178,6 +179,7 @@ static void oracle_bwd_unit(int64_t b, int64_t h, int64_t L, int64_t H, int64_t 
         dx[(tok * H + h) * P + p] = step * gb + skip * (double)dyt[p];
         g_in += gb * (double)xt[p];
         dD_acc += (double)dyt[p] * (double)xt[p];
+        dD_abs += fabs((double)dyt[p] * (double)xt[p]);
       }
       for (int64_t n = 0; n < N; ++n) {
         double gx = 0.0, hy = 0.0;
@@ -190,6 +192,7 @@ static void oracle_bwd_unit(int64_t b, int64_t h, int64_t L, int64_t H, int64_t 
       }
       ddt[tok * H + h] = g_in + rate * decay * g_dec;
       dA_acc += step * decay * g_dec;
+      dA_abs += fabs(step * decay * g_dec);
     }
   }
   if (dh0) {
@@ -198,6 +201,8 @@ static void oracle_bwd_unit(int64_t b, int64_t h, int64_t L, int64_t H, int64_t 
   }
   *dA_unit = dA_acc;
   *dD_unit = dD_acc;
+  if (dA_abs_unit) *dA_abs_unit = dA_abs;
+  if (dD_abs_unit) *dD_abs_unit = dD_abs;
 }
 
 /*
@@ -205,13 +210,17 @@ static void oracle_bwd_unit(int64_t b, int64_t h, int64_t L, int64_t H, int64_t 
  * NULL (not with seq_idx); outputs dx (b,L,H,P), ddt (b,L,H), dBh, dCh
  * (b,L,H,N) per head (the caller sums each group's heads), dA_units and
  * dD_units (b*H) per unit (the caller sums over the batch), dh0 (b,H,P,N) or
- * NULL.  Returns 0, -1 on a bad argument, -2 if memory runs out.
+ * NULL; dA_abs_units and dD_abs_units (b*H) or NULL: per unit, the sums of
+ * the magnitudes of the terms that dA and dD add up (the scale a rounding
+ * error in those sums is measured against).  Returns 0, -1 on a bad
+ * argument, -2 if memory runs out.
  */
 int oracle_ssd_bwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim, int64_t dstate,
                    int64_t ngroups, const float* x, const float* dt, const float* A, const float* B,
                    const float* C, const float* D, const float* initial_states, const int32_t* seq_idx,
                    const float* dy, const float* dfinal, double* dx, double* ddt, double* dBh, double* dCh,
-                   double* dA_units, double* dD_units, double* dh0, int nthreads) {
+                   double* dA_units, double* dD_units, double* dh0, int nthreads, double* dA_abs_units,
+                   double* dD_abs_units) {
   if (batch <= 0 || seqlen <= 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0) return -1;
   if (nheads % ngroups != 0 || (seq_idx && dfinal)) return -1;
   if (!x || !dt || !A || !B || !C || !dy || !dx || !ddt || !dBh || !dCh || !dA_units || !dD_units) return -1;
@@ -236,7 +245,8 @@ int oracle_ssd_bwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdi
       if (!ckpt || !blk || !Gs) continue;
       oracle_bwd_unit(u / nheads, u % nheads, seqlen, nheads, headdim, dstate, ngroups, x, dt, A, B, C, D,
                       initial_states, seq_idx, dy, dfinal, dx, ddt, dA_units + u, dBh, dCh, dD_units + u,
-                      initial_states ? dh0 : NULL, ckpt, blk, Gs);
+                      initial_states ? dh0 : NULL, ckpt, blk, Gs, dA_abs_units ? dA_abs_units + u : NULL,
+                      dD_abs_units ? dD_abs_units + u : NULL);
     }
     free(ckpt);
     free(blk);

@@ -21,7 +21,8 @@ import pytest
 import torch
 
 import emu_bwd
-from bwd_cases import CASES, KEYS, case_inputs, compare, dfinal_like, dy_like, gate_like, inputs, oracle_bwd
+from bwd_cases import (CASES, KEYS, RANDOM_SEEDS, case_inputs, compare, dfinal_like, dy_like, gate_like, inputs,
+                       oracle_bwd, random_case)
 
 pytestmark = pytest.mark.skipif(not emu_bwd.available(), reason="g++ not available")
 
@@ -162,3 +163,11 @@ def test_emulator_catches_planted_mistakes(mutant, monkeypatch):
             except (AssertionError, RuntimeError):
                 caught = True
         assert caught, f"mutant {name} survived"
+
+
+@pytest.mark.parametrize("seed", RANDOM_SEEDS)
+def test_emulated_backward_on_random_shapes(seed):
+    d, dy, dfinal, chunk, _ = random_case(seed)
+    out = emu_bwd.run(d, dy, dfinal, chunk_size=chunk, z=d["z"], reverse=seed % 2 == 1)
+    assert out["status"] == 0
+    compare(out, oracle_bwd(d, dy, dfinal))

@@ -13,8 +13,8 @@ import torch
 
 import mamba_ssd_chunked_03_b200 as ssd
 import oracle
-from bwd_cases import (CASES, CONV_CASES, KEYS, case_inputs, compare, conv_case_inputs, conv_compare, dfinal_like,
-                       dy_like, inputs, oracle_bwd)
+from bwd_cases import (CASES, CONV_CASES, KEYS, RANDOM_SEEDS, case_inputs, compare, conv_case_inputs, conv_compare,
+                       dfinal_like, dy_like, inputs, oracle_bwd, random_case)
 from oracle import block
 
 pytestmark = pytest.mark.gpu
@@ -121,9 +121,7 @@ def test_simulated_seqpar_backward_matches_the_whole_sequence(cuts):
     got["dA"] = sum(o["dA"] for o in out).cpu().numpy()
     got["dD"] = sum(o["dD"] for o in out).cpu().numpy()
     got["dh0"] = out[0]["dinitial_states"].cpu().numpy()
-    for k, v in got.items():
-        rel = np.linalg.norm(v - ref[k]) / np.linalg.norm(ref[k])
-        assert rel <= 1e-4, (k, rel)
+    compare(got, ref, keys=("dx", "ddt", "dA", "dB", "dC", "dD", "dh0"), rel_l2=1e-4)
 
 
 def test_autograd_function_through_the_gate():
@@ -159,3 +157,10 @@ def test_conv_autograd_function_routes_through_the_library():
     du, dw, db = block.conv1d_silu_bwd(u, w, bias, dout, seq)
     conv_compare(leaves[0].grad.cpu().numpy(), leaves[1].grad.cpu().numpy(), leaves[2].grad.cpu().numpy(),
                  (du, dw, db))
+
+
+@pytest.mark.parametrize("seed", RANDOM_SEEDS)
+def test_backward_on_random_shapes(seed):
+    """The seeded random problems of the host emulation's sweep, on the GPU."""
+    d, dy, dfinal, chunk, _ = random_case(seed)
+    compare(_gpu_bwd(d, dy, dfinal, chunk), oracle_bwd(d, dy, dfinal))
