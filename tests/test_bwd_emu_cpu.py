@@ -171,3 +171,14 @@ def test_emulated_backward_on_random_shapes(seed):
     out = emu_bwd.run(d, dy, dfinal, chunk_size=chunk, z=d["z"], reverse=seed % 2 == 1)
     assert out["status"] == 0
     compare(out, oracle_bwd(d, dy, dfinal))
+
+
+@pytest.mark.parametrize("packed", [False, True], ids=["dense", "packed"])
+def test_emulated_backward_on_the_gpu_tests_mid_sizes(packed):
+    """The mid-size problems of the GPU tests, under the sanitizers too."""
+    b, L, H, P, N, G = (2, 1024, 8, 64, 128, 1) if not packed else (2, 1024, 4, 64, 128, 2)
+    d = inputs(b, L, H, P, N, G, "bf16", h0=0.0 if packed else 0.2, packed=(32, 400) if packed else None, seed=77)
+    d["z"] = None
+    dy = dy_like(b, L, H, P, torch.bfloat16, 78)
+    dfinal = None if packed else dfinal_like(b, H, P, N, 79)
+    compare(emu_bwd.run(d, dy, dfinal, timeout=1200), oracle_bwd(d, dy, dfinal))
