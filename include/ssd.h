@@ -370,8 +370,16 @@ typedef struct {
                                      is dLoss/dout: the kernels recompute y, write
                                      dz = dy * y * SiLU'(z) and take dy * SiLU(z) as
                                      the gradient of y.                              */
-  float* dz;                      /* (b,L,H,P) fp32 output dLoss/dz; required iff z  */
+  float* dz;                      /* (b,L,H,P) fp32 output dLoss/dz; required iff z
+                                     (unless SSD_BWD_DINITIAL_ONLY)                  */
+  uint32_t flags;                 /* SSD_BWD_* or 0                                  */
 } ssd_bwd_args;
+
+/* ssd_bwd flags */
+#define SSD_BWD_DINITIAL_ONLY 1u /* compute dinitial_states alone (required then; dx, ddt,
+                                    dA, dB, dC, dD, dz may be NULL and are not written):
+                                    two of the five kernels.  Sequence parallelism needs
+                                    only this from its first backward pass.          */
 
 /* Bytes of device workspace ssd_bwd needs (only sizes, chunk_size and dtype
  * are read), or 0 if the sizes are invalid or unsupported. */
@@ -386,8 +394,8 @@ SSD_API int64_t ssd_bwd_chunk_size(const ssd_bwd_args* args);
  * All pointers are device pointers owned by the caller; outputs must not
  * overlap inputs or the workspace.  Returns SSD_OK once enqueued;
  * SSD_ERR_INVALID_ARG for a null required pointer, a bad size or enum, or a
- * misaligned workspace, a single timing event, or z without dz (or dz
- * without z); SSD_ERR_UNSUPPORTED as described above;
+ * misaligned workspace, a single timing event, z without dz (or dz
+ * without z), or an unknown flag; SSD_ERR_UNSUPPORTED as described above;
  * SSD_ERR_WORKSPACE when the workspace is missing or too small; SSD_ERR_CUDA
  * when a launch fails (outputs then undefined). */
 SSD_API ssd_status ssd_bwd(const ssd_bwd_args* args, void* stream);

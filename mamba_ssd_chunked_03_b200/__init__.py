@@ -32,6 +32,7 @@ SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_WORKSPACE, SSD_ERR_CUD
 SSD_F32, SSD_BF16 = 0, 1
 SSD_FLAG_GENERIC = 1
 SSD_FLAG_CHECK_SEQ = 2
+SSD_BWD_DINITIAL_ONLY = 1
 
 
 class Args(ctypes.Structure):
@@ -85,6 +86,7 @@ class BwdArgs(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("timing_events", ctypes.c_void_p * 2),
         ("z", ctypes.c_void_p), ("dz", ctypes.c_void_p),
+        ("flags", ctypes.c_uint32),
     ]
 
 
@@ -447,7 +449,7 @@ def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
         seq_idx: Optional[torch.Tensor] = None, dfinal_states: Optional[torch.Tensor] = None,
         chunk_size: int = 0, want_dD: bool = True, want_dinitial_states: Optional[bool] = None,
         workspace: Optional[torch.Tensor] = None, timing_events: Optional[tuple] = None,
-        z: Optional[torch.Tensor] = None) -> dict:
+        z: Optional[torch.Tensor] = None, dinitial_only: bool = False) -> dict:
     """The SSD backward via ``ssd_bwd``: gradients of a loss given
     dy = dLoss/dy (like x) and dfinal_states = dLoss/dfinal_states
     ((b,H,P,N) fp32 or None; not with seq_idx).  Inputs as for ``fwd``.
@@ -457,7 +459,8 @@ def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     library chooses).  ``timing_events``: optional (start, end)
     torch.cuda.Event pair recorded around the dominant kernel.  ``z``: the
     forward's gate (like x); dy is then the gradient of y * SiLU(z), and the
-    dict also holds dz (fp32)."""
+    dict also holds dz (fp32).  ``dinitial_only``: compute dinitial_states
+    alone (two of the five kernels); the other entries are None."""
     _check(x, dt, A, B, C, D, initial_states, seq_idx)
     if dy.dtype != x.dtype or tuple(dy.shape) != tuple(x.shape) or dy.device != x.device or not dy.is_contiguous():
         raise ValueError("dy must be a contiguous tensor like x")
@@ -472,15 +475,20 @@ def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     if want_dinitial_states is None:
         want_dinitial_states = initial_states is not None
     f32 = dict(device=x.device, dtype=torch.float32)
-    g = {"dx": torch.empty(b, L, H, P, **f32), "ddt": torch.empty(b, L, H, **f32), "dA": torch.empty(H, **f32),
-         "dB": torch.empty(b, L, G, N, **f32), "dC": torch.empty(b, L, G, N, **f32),
-         "dD": torch.empty(H, **f32) if want_dD else None,
-         "dinitial_states": torch.empty(b, H, P, N, **f32) if want_dinitial_states else None,
-         "dz": torch.empty(b, L, H, P, **f32) if z is not None else None}
+    if dinitial_only:
+        g = {k: None for k in ("dx", "ddt", "dA", "dB", "dC", "dD", "dz")}
+        g["dinitial_states"] = torch.empty(b, H, P, N, **f32)
+    else:
+        g = {"dx": torch.empty(b, L, H, P, **f32), "ddt": torch.empty(b, L, H, **f32),
+             "dA": torch.empty(H, **f32), "dB": torch.empty(b, L, G, N, **f32), "dC": torch.empty(b, L, G, N, **f32),
+             "dD": torch.empty(H, **f32) if want_dD else None,
+             "dinitial_states": torch.empty(b, H, P, N, **f32) if want_dinitial_states else None,
+             "dz": torch.empty(b, L, H, P, **f32) if z is not None else None}
     a = make_bwd_args(x, dt, A, B, C, D, dy, initial_states, seq_idx, dfinal_states, chunk_size)
     a.dx, a.ddt, a.dA, a.dB, a.dC = (_ptr(g[k]) for k in ("dx", "ddt", "dA", "dB", "dC"))
     a.dD, a.dinitial_states = _ptr(g["dD"]), _ptr(g["dinitial_states"])
     a.z, a.dz = _ptr(z), _ptr(g["dz"])
+    a.flags = SSD_BWD_DINITIAL_ONLY if dinitial_only else 0
     need = int(lib.ssd_bwd_workspace_size(ctypes.byref(a)))
     if need == 0:  # sizes the library rejects: let it say why (nothing is enqueued)
         raise SSDError(lib.ssd_bwd(ctypes.byref(a), _stream(x)))

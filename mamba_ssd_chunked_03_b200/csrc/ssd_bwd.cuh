@@ -703,13 +703,16 @@ inline ssd_status plan(const ssd_bwd_args* a, Plan* pl) {
 
 // Arguments and workspace for one call; the workspace is required.
 inline ssd_status check_call(const ssd_bwd_args* a, const Plan& pl) {
-  if (!a->x || !a->dt || !a->A || !a->B || !a->C || !a->dy || !a->dx || !a->ddt || !a->dA || !a->dB || !a->dC)
-    return SSD_ERR_INVALID_ARG;
+  if (a->flags & ~SSD_BWD_DINITIAL_ONLY) return SSD_ERR_INVALID_ARG;
+  const bool only_dh0 = (a->flags & SSD_BWD_DINITIAL_ONLY) != 0;
+  if (!a->x || !a->dt || !a->A || !a->B || !a->C || !a->dy) return SSD_ERR_INVALID_ARG;
+  if (only_dh0 ? !a->dinitial_states : (!a->dx || !a->ddt || !a->dA || !a->dB || !a->dC)) return SSD_ERR_INVALID_ARG;
   if (a->seq_idx && a->dfinal_states) return SSD_ERR_UNSUPPORTED;
   if (!a->workspace || a->workspace_bytes < pl.total) return SSD_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(a->workspace) % 256 != 0) return SSD_ERR_INVALID_ARG;
   if ((a->timing_events[0] == nullptr) != (a->timing_events[1] == nullptr)) return SSD_ERR_INVALID_ARG;
-  if ((a->z == nullptr) != (a->dz == nullptr)) return SSD_ERR_INVALID_ARG;
+  if (!only_dh0 && (a->z == nullptr) != (a->dz == nullptr)) return SSD_ERR_INVALID_ARG;
+  if (a->dz && !a->z) return SSD_ERR_INVALID_ARG;
   return SSD_OK;
 }
 
@@ -752,11 +755,15 @@ inline unsigned blocks_for(int64_t n) { return (unsigned)((n + kThreads - 1) / k
 // shared bytes, args)`, which returns false when a launch fails;
 // `launch.record(event)` records a caller's timing event (false on failure).
 template <typename T, class Launch>
-ssd_status enqueue_typed(const KArgs& k, const Plan& pl, void* const events[2], Launch& launch) {
+ssd_status enqueue_typed(const KArgs& k, const Plan& pl, void* const events[2], bool only_dh0, Launch& launch) {
   const Dims& d = pl.d;
   const unsigned chunk_ctas = (unsigned)(d.b * d.nc * d.H);
   if (!launch(&k_bwd_chunk_states<T>, chunk_ctas, pl.smem_states, k)) return SSD_ERR_CUDA;
   if (!launch(&k_bwd_state_passing, blocks_for(d.b * d.H * d.P * d.N), (size_t)0, k)) return SSD_ERR_CUDA;
+  if (only_dh0) {  // k_bwd_chunk is not run: its timing events mark the same point
+    if (events[0] && !(launch.record(events[0]) && launch.record(events[1]))) return SSD_ERR_CUDA;
+    return SSD_OK;
+  }
   if (events[0] && !launch.record(events[0])) return SSD_ERR_CUDA;
   if (!launch(&k_bwd_chunk<T>, chunk_ctas, pl.smem_chunk, k)) return SSD_ERR_CUDA;
   if (events[1] && !launch.record(events[1])) return SSD_ERR_CUDA;
@@ -773,8 +780,9 @@ ssd_status run(const ssd_bwd_args* a, Launch& launch) {
   st = check_call(a, pl);
   if (st != SSD_OK) return st;
   const KArgs k = make_kargs(a, pl);
-  return a->dtype == SSD_BF16 ? enqueue_typed<__nv_bfloat16>(k, pl, a->timing_events, launch)
-                               : enqueue_typed<float>(k, pl, a->timing_events, launch);
+  const bool only_dh0 = (a->flags & SSD_BWD_DINITIAL_ONLY) != 0;
+  return a->dtype == SSD_BF16 ? enqueue_typed<__nv_bfloat16>(k, pl, a->timing_events, only_dh0, launch)
+                               : enqueue_typed<float>(k, pl, a->timing_events, only_dh0, launch);
 }
 
 }  // namespace bwd

@@ -22,8 +22,10 @@ D_k Lam_k + T_k, where Lam_k is the gradient with respect to the state
 leaving it and T_k comes from the range's own outputs alone (the backward's
 dinitial_states when no state gradient comes in).  So:
 
-1. every rank recovers h_in as in the forward, and runs its backward without
-   an incoming state gradient: T_k;
+1. every rank recovers h_in as in the forward, and computes T_k: the
+   backward's dinitial_states with no incoming state gradient (which does not
+   depend on h_in; ``ssd_bwd`` with ``SSD_BWD_DINITIAL_ONLY`` runs two of its
+   five kernels for it);
 2. the ranks all-gather (T_k, D_k);
 3. rank r folds Lam_r from the sequence's dfinal through ranks R-1..r+1
    (``ssd_state_fold`` over the reversed lists) and runs its backward again
@@ -62,6 +64,12 @@ class LibraryOps:
     def local_backward(x, dt, A, B, C, D, dy, initial_states, dfinal_states):
         return bwd(x, dt, A, B, C, D, dy, initial_states=initial_states, dfinal_states=dfinal_states,
                    want_dD=D is not None, want_dinitial_states=True)
+
+    @staticmethod
+    def adjoint_summary(x, dt, A, B, C, D, dy):
+        """T: dLoss/d(the state entering the range) from the range's own
+        outputs (no state gradient coming in), without the other gradients."""
+        return bwd(x, dt, A, B, C, D, dy, dinitial_only=True)["dinitial_states"]
 
 
 def local_summary(x, dt, A, B, C, D, chunk_size: int = 64, ops=LibraryOps):
@@ -115,7 +123,10 @@ def bwd_seqpar(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tens
     R = dist.get_world_size(group)
     r = dist.get_rank(group)
     h_in, decays, shape = _state_in(x, dt, A, B, C, D, chunk_size, initial_states, group, ops)
-    T = ops.local_backward(x, dt, A, B, C, D, dy, h_in, None)["dinitial_states"]
+    if hasattr(ops, "adjoint_summary"):
+        T = ops.adjoint_summary(x, dt, A, B, C, D, dy)
+    else:
+        T = ops.local_backward(x, dt, A, B, C, D, dy, h_in, None)["dinitial_states"]
     all_T = [torch.empty_like(T) for _ in range(R)]
     dist.all_gather(all_T, T.contiguous(), group=group)
     after = list(range(R - 1, r, -1))  # the ranks after this one, last first

@@ -8,7 +8,8 @@
 // dtype 0|1 and has_* / want_* flags) and the input arrays DIR/<name>.bin
 // (raw, row-major: x dt A B C D h0 seq dy dfinal z), writes the gradients as
 // raw fp32 to DIR/<name>.bin (dx ddt dA dB dC dD dh0 dz) and prints the status.
-// "reverse 1" runs each block's fibers in reverse thread order.
+// "reverse 1" runs each block's fibers in reverse thread order; "flags" are
+// ssd_bwd_args.flags (with SSD_BWD_DINITIAL_ONLY only dh0 is allocated).
 // Every buffer is allocated to its exact size, so AddressSanitizer sees any
 // access past it; outputs, workspace and shared memory start as NaN bytes,
 // so a value read before it was written shows up in the result.
@@ -86,6 +87,8 @@ int main(int argc, char** argv) {
   a.ngroups = kv["ngroups"];
   a.chunk_size = kv["chunk_size"];
   a.dtype = (ssd_dtype)kv["dtype"];
+  a.flags = (uint32_t)kv["flags"];
+  const bool only_dh0 = (a.flags & SSD_BWD_DINITIAL_ONLY) != 0;
   auto in = [&](const char* name, bool present) -> const void* {
     if (!present) return nullptr;
     Buf b = read_file(dir + "/" + name + ".bin");
@@ -109,14 +112,16 @@ int main(int argc, char** argv) {
 
   const size_t b = a.batch, L = a.seqlen, H = a.nheads, P = a.headdim, N = a.dstate, G = a.ngroups;
   const size_t nx = b * L * H * P, ndt = b * L * H, nB = b * L * G * N, nh = b * H * P * N;
-  a.dx = nan_floats(nx);
-  a.ddt = nan_floats(ndt);
-  a.dA = nan_floats(H);
-  a.dB = nan_floats(nB);
-  a.dC = nan_floats(nB);
-  a.dD = kv["want_dD"] ? nan_floats(H) : nullptr;
+  if (!only_dh0) {
+    a.dx = nan_floats(nx);
+    a.ddt = nan_floats(ndt);
+    a.dA = nan_floats(H);
+    a.dB = nan_floats(nB);
+    a.dC = nan_floats(nB);
+    a.dD = kv["want_dD"] ? nan_floats(H) : nullptr;
+    a.dz = a.z ? nan_floats(nx) : nullptr;
+  }
   a.dinitial_states = kv["want_dh0"] ? nan_floats(nh) : nullptr;
-  a.dz = a.z ? nan_floats(nx) : nullptr;
 
   ssd::bwd::Plan pl;
   ssd_status st = ssd::bwd::plan(&a, &pl);
@@ -132,11 +137,11 @@ int main(int argc, char** argv) {
   st = ssd::bwd::run(&a, launch);
   std::printf("status %d launches %d chunk %lld\n", (int)st, launch.launches, (long long)pl.d.Q);
   if (st != SSD_OK) return 1;
-  write_file(dir + "/dx.bin", a.dx, nx * 4);
-  write_file(dir + "/ddt.bin", a.ddt, ndt * 4);
-  write_file(dir + "/dA.bin", a.dA, H * 4);
-  write_file(dir + "/dB.bin", a.dB, nB * 4);
-  write_file(dir + "/dC.bin", a.dC, nB * 4);
+  if (a.dx) write_file(dir + "/dx.bin", a.dx, nx * 4);
+  if (a.ddt) write_file(dir + "/ddt.bin", a.ddt, ndt * 4);
+  if (a.dA) write_file(dir + "/dA.bin", a.dA, H * 4);
+  if (a.dB) write_file(dir + "/dB.bin", a.dB, nB * 4);
+  if (a.dC) write_file(dir + "/dC.bin", a.dC, nB * 4);
   if (a.dD) write_file(dir + "/dD.bin", a.dD, H * 4);
   if (a.dinitial_states) write_file(dir + "/dh0.bin", a.dinitial_states, nh * 4);
   if (a.dz) write_file(dir + "/dz.bin", a.dz, nx * 4);

@@ -62,7 +62,7 @@ def _raw(t) -> bytes:
 
 
 def run(inp: dict, dy, dfinal=None, chunk_size: int = 0, want_dD: bool = True, want_dh0: bool = True,
-        kind: str = "asan", reverse: bool = False, timeout: int = 600, z=None) -> dict:
+        kind: str = "asan", reverse: bool = False, timeout: int = 600, z=None, flags: int = 0) -> dict:
     """Run the emulated backward on ``inp`` (``ssd_inputs.make_inputs`` form)
     with upstream gradient ``dy`` (x's dtype) and ``dfinal`` (fp32 or None).
     ``reverse`` runs each block's threads in reverse order (fiber builds).
@@ -85,7 +85,7 @@ def run(inp: dict, dy, dfinal=None, chunk_size: int = 0, want_dD: bool = True, w
                   dtype=1 if x.dtype == torch.bfloat16 else 0, has_D=int(arrays["D"] is not None),
                   has_h0=int(arrays["h0"] is not None), has_seq=int(arrays["seq"] is not None),
                   has_dfinal=int(dfinal is not None), want_dD=int(want_dD), want_dh0=int(want_dh0),
-                  reverse=int(reverse), has_z=int(z is not None))
+                  reverse=int(reverse), has_z=int(z is not None), flags=int(flags))
         with open(os.path.join(d, "args.txt"), "w") as f:
             f.write("".join(f"{k} {v}\n" for k, v in kv.items()))
         env = dict(os.environ)

@@ -401,3 +401,12 @@ def test_conv_bwd_workspace_size():
     assert size(seqlen=65) == 2 * 3 * 64 * 5 * 4
     assert size(batch=0) == 0 and size(width=5) == 0
     assert ssd.lib.ssd_conv1d_silu_bwd(None, None) == ssd.SSD_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({"flags": 2}, ssd.SSD_ERR_INVALID_ARG),                               # unknown flag
+    ({"flags": 1}, ssd.SSD_ERR_INVALID_ARG),                               # dinitial_states missing
+    ({"flags": 1, "dinitial_states": 1 << 27, "dz": 1 << 26}, ssd.SSD_ERR_INVALID_ARG),  # dz without a gate
+])
+def test_bwd_dinitial_only_rejections(kw, status):
+    assert ssd.lib.ssd_bwd(ctypes.byref(_bwd_args(**kw)), None) == status

@@ -182,3 +182,12 @@ def test_emulated_backward_on_the_gpu_tests_mid_sizes(packed):
     dy = dy_like(b, L, H, P, torch.bfloat16, 78)
     dfinal = None if packed else dfinal_like(b, H, P, N, 79)
     compare(emu_bwd.run(d, dy, dfinal, timeout=1200), oracle_bwd(d, dy, dfinal))
+
+
+def test_dinitial_only_gives_the_same_bits_and_writes_nothing_else():
+    d, dy, dfinal, chunk = case_inputs(CASES[1])
+    full = emu_bwd.run(d, dy, None, chunk_size=chunk, z=d["z"])
+    only = emu_bwd.run(d, dy, None, chunk_size=chunk, z=d["z"], flags=1)
+    assert only["status"] == 0 and only["launches"] == 2
+    assert np.array_equal(only["dh0"], full["dh0"])
+    assert all(only[k] is None for k in ("dx", "ddt", "dA", "dB", "dC", "dD", "dz"))
