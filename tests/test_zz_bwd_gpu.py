@@ -148,10 +148,13 @@ def test_conv_backward_matches_oracle(case):
 
 
 def test_conv_autograd_function_routes_through_the_library():
-    u, w, bias, dout, seq = conv_case_inputs(CONV_CASES[1])
-    bias = torch.randn(w.shape[0]) * 0.1
-    leaves = [t.cuda().requires_grad_(True) for t in (u.float(), w, bias)]
-    out = ssd.causal_conv1d_silu(leaves[0].to(u.dtype), leaves[1], leaves[2], seq.cuda())
+    """fp32 u, so that the gradient handed back in u's dtype is the library's
+    fp32 du unrounded (packed rows, as the forward kernel takes channels % 4)."""
+    u, w, bias, dout, _ = conv_case_inputs(CONV_CASES[0])
+    import ssd_inputs as si
+    seq = si.seq_idx_from_lengths([[20, 1, 49], [35, 35]])[0]
+    leaves = [t.cuda().requires_grad_(True) for t in (u, w, bias)]
+    out = ssd.causal_conv1d_silu(leaves[0], leaves[1], leaves[2], seq.cuda())
     (out.double() * dout.cuda().double()).sum().backward()
     du, dw, db = block.conv1d_silu_bwd(u, w, bias, dout, seq)
     conv_compare(leaves[0].grad.cpu().numpy(), leaves[1].grad.cpu().numpy(), leaves[2].grad.cpu().numpy(),
