@@ -168,3 +168,21 @@ def test_silu_grad_is_the_derivative():
     fd = (backward.silu(v + h) - backward.silu(v - h)) / (2 * h)
     assert np.allclose(backward.silu_grad(v), fd, rtol=1e-7, atol=1e-9)
     assert backward.silu_grad(0.0) == 0.5  # s(0) = 1/2, and the v (1 - s) term vanishes
+
+
+def test_one_token_closed_form():
+    """L = 1, P = N = 1: y = (a h0 + dt x B) C + D x with a = exp(dt A), so by
+    hand dx = (dt B C + D) dy, dB = dt x C dy, dC = h dy, dD = x dy,
+    ddt = (x B + A a h0) C dy, dA = dt a h0 C dy, dh0 = a C dy (a final-state
+    gradient adds dfinal times the same derivatives of h)."""
+    x, dt, A, B, C, D, h0, dy, df = 0.75, 0.125, -2.0, -1.5, 0.5, 0.25, 0.625, 1.25, -0.375
+    t = lambda v, shape: torch.full(shape, v, dtype=torch.float32)
+    got = backward.ssd_bwd(t(x, (1, 1, 1, 1)), t(dt, (1, 1, 1)), t(A, (1,)), t(B, (1, 1, 1, 1)), t(C, (1, 1, 1, 1)),
+                           t(D, (1,)), t(h0, (1, 1, 1, 1)), np.full((1, 1, 1, 1), dy), np.full((1, 1, 1, 1), df))
+    a = np.exp(dt * A)
+    h = a * h0 + dt * x * B
+    g = C * dy + df  # dLoss/dh
+    want = {"dx": dt * B * g + D * dy, "dB": dt * x * g, "dC": h * dy, "dD": x * dy,
+            "ddt": x * B * g + A * a * h0 * g, "dA": dt * a * h0 * g, "dh0": a * g}
+    for k, w in want.items():
+        assert np.allclose(np.asarray(got[k]).ravel()[0], w, rtol=1e-14, atol=0), (k, got[k], w)

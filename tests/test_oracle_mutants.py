@@ -166,4 +166,8 @@ def test_backward_mutant_fails_a_pin(name, monkeypatch, tmp_path):
             bw.test_gated_backward_matches_autograd(case)
         except AssertionError:
             failed += 1
+    try:
+        bw.test_one_token_closed_form()
+    except AssertionError:
+        failed += 1
     assert failed > 0, f"no pin caught {name}"
