@@ -168,62 +168,74 @@ __device__ __forceinline__ void chunk_cumsum(const KArgs& a, const ChunkPos& q, 
 // stored.
 constexpr int kT = 4;
 
-struct Tile {
+template <int TM, int TN>
+struct TileT {
   int tc;               // column-block index (the partial-sum slot of a row)
-  int r[kT], c[kT];     // clamped row and column indices
-  bool rv[kT], cv[kT];  // inside the product?
+  int r[TM], c[TN];     // clamped row and column indices
+  bool rv[TM], cv[TN];  // inside the product?
 };
+using Tile = TileT<kT, kT>;
 
-__device__ __forceinline__ int tiles_of(int M, int Nn) { return ((M + kT - 1) / kT) * ((Nn + kT - 1) / kT); }
+template <int TM = kT, int TN = kT>
+__device__ __forceinline__ int tiles_of(int M, int Nn) {
+  return ((M + TM - 1) / TM) * ((Nn + TN - 1) / TN);
+}
 
-__device__ __forceinline__ Tile make_tile(int tile, int M, int Nn) {
-  const int TC = (Nn + kT - 1) / kT;
+template <int TM = kT, int TN = kT>
+__device__ __forceinline__ TileT<TM, TN> make_tile(int tile, int M, int Nn) {
+  const int TC = (Nn + TN - 1) / TN;
   const int tr = tile / TC;
-  Tile t;
+  TileT<TM, TN> t;
   t.tc = tile % TC;
 #pragma unroll
-  for (int i = 0; i < kT; ++i) {
-    const int r = tr * kT + i;
+  for (int i = 0; i < TM; ++i) {
+    const int r = tr * TM + i;
     t.rv[i] = r < M;
     t.r[i] = r < M ? r : M - 1;
-    const int c = t.tc + i * TC;
-    t.cv[i] = c < Nn;
-    t.c[i] = c < Nn ? c : Nn - 1;
+  }
+#pragma unroll
+  for (int j = 0; j < TN; ++j) {
+    const int c = t.tc + j * TC;
+    t.cv[j] = c < Nn;
+    t.c[j] = c < Nn ? c : Nn - 1;
   }
   return t;
 }
 
-__device__ __forceinline__ void tile_zero(float (&acc)[kT][kT]) {
+template <int TM, int TN>
+__device__ __forceinline__ void tile_zero(float (&acc)[TM][TN]) {
 #pragma unroll
-  for (int i = 0; i < kT; ++i)
+  for (int i = 0; i < TM; ++i)
 #pragma unroll
-    for (int j = 0; j < kT; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
 }
 
 // acc[i][j] += sum_{k0 <= k < k1} A(r_i, k) B(k, c_j), with A(m, k) = a[m am + k ak]
 // (times ks[k] when kScale) and B(k, n) = b[k bk + n bn].
-template <bool kScale>
-__device__ __forceinline__ void tile_mac(float (&acc)[kT][kT], const Tile& t, const float* a, int am, int ak,
-                                         const float* ks, const float* b, int bk, int bn, int k0, int k1) {
+template <bool kScale, int TM, int TN>
+__device__ __forceinline__ void tile_mac(float (&acc)[TM][TN], const TileT<TM, TN>& t, const float* a, int am,
+                                         int ak, const float* ks, const float* b, int bk, int bn, int k0, int k1) {
   for (int k = k0; k < k1; ++k) {
-    float av[kT], bv[kT];
+    float av[TM], bv[TN];
     const float sk = kScale ? ks[k] : 1.f;
 #pragma unroll
-    for (int i = 0; i < kT; ++i) av[i] = kScale ? a[t.r[i] * am + k * ak] * sk : a[t.r[i] * am + k * ak];
+    for (int i = 0; i < TM; ++i) av[i] = kScale ? a[t.r[i] * am + k * ak] * sk : a[t.r[i] * am + k * ak];
 #pragma unroll
-    for (int j = 0; j < kT; ++j) bv[j] = b[k * bk + t.c[j] * bn];
+    for (int j = 0; j < TN; ++j) bv[j] = b[k * bk + t.c[j] * bn];
 #pragma unroll
-    for (int i = 0; i < kT; ++i)
+    for (int i = 0; i < TM; ++i)
 #pragma unroll
-      for (int j = 0; j < kT; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
   }
 }
 
 // Shared-memory floats of k_bwd_chunk_states for chunk length Q.
 inline size_t smem_states_floats(int64_t Q, int64_t P, int64_t N) { return (size_t)(2 * Q * P + 2 * Q * N + 4 * Q); }
 
+// Two CTAs per SM (2 x 99 KB of shared memory at headdim 64, dstate 128): at
+// most 128 registers a thread.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) k_bwd_chunk_states(const KArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) k_bwd_chunk_states(const KArgs a) {
   const Dims& d = a.d;
   const ChunkPos q = chunk_pos(d, blockIdx.x);
   const int P = (int)d.P, N = (int)d.N, Q = (int)d.Q, Qc = q.Qc;
@@ -268,18 +280,20 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk_states(const KArgs a) {
   const int64_t off = ((q.b * d.H + q.h) * d.nc + q.c) * d.P * d.N;
   float* So = a.S + off;
   float* To = a.T + off;
-  const int nt = tiles_of(P, N);
+  // 8 x 4 blocks: P x N = 8192 outputs at headdim 64, dstate 128 is one block per thread
+  constexpr int TM = 8, TN = 4;
+  const int nt = tiles_of<TM, TN>(P, N);
   for (int tile = tid; tile < nt; tile += kThreads) {
-    const Tile tl = make_tile(tile, P, N);
-    float s[kT][kT], u[kT][kT];
+    const TileT<TM, TN> tl = make_tile<TM, TN>(tile, P, N);
+    float s[TM][TN], u[TM][TN];
     tile_zero(s);
     tile_zero(u);
     tile_mac<true>(s, tl, xs, 1, P, cS, Bs, N, 1, 0, Qc);
     tile_mac<true>(u, tl, dys, 1, P, cT, Cs, N, 1, 0, Qc);
 #pragma unroll
-    for (int i = 0; i < kT; ++i)
+    for (int i = 0; i < TM; ++i)
 #pragma unroll
-      for (int j = 0; j < kT; ++j)
+      for (int j = 0; j < TN; ++j)
         if (tl.rv[i] && tl.cv[j]) {
           So[tl.r[i] * N + tl.c[j]] = s[i][j];
           To[tl.r[i] * N + tl.c[j]] = u[i][j];
