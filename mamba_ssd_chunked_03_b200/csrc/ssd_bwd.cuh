@@ -167,6 +167,7 @@ __device__ __forceinline__ void chunk_cumsum(const KArgs& a, const ChunkPos& q, 
 // Indices past the edge are clamped for loads, and their results are never
 // stored.
 constexpr int kT = 4;
+constexpr int kTN = 8;  // rows of the blocks of the Q x dstate products
 
 template <int TM, int TN>
 struct TileT {
@@ -480,21 +481,21 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
   }
   __syncthreads();
 
-  // dC of this head (Q x N): sum_s Z(t,s) w_s B_s + e_t h_in^T dy_t; with the
-  // row partials of C_t . (h_in^T dy_t)
-  for (int tile = tid; tile < tiles_of(Qc, N); tile += kThreads) {
-    const Tile tl = make_tile(tile, Qc, N);
+  // dC of this head (Q x N, 8 x 4 blocks: one per thread at Q 64, dstate 128):
+  // sum_s Z(t,s) w_s B_s + e_t h_in^T dy_t; with the row partials of C_t . (h_in^T dy_t)
+  for (int tile = tid; tile < tiles_of<kTN, kT>(Qc, N); tile += kThreads) {
+    const TileT<kTN, kT> tl = make_tile<kTN, kT>(tile, Qc, N);
     int kmax = 0;
 #pragma unroll
-    for (int i = 0; i < kT; ++i)
+    for (int i = 0; i < kTN; ++i)
       if (tl.rv[i]) kmax = tl.r[i] + 1;
-    float ci[kT][kT], ch[kT][kT];
+    float ci[kTN][kT], ch[kTN][kT];
     tile_zero(ci);
     tile_zero(ch);
     tile_mac<true>(ci, tl, Zm, sQ, 1, w, Bs, sN, 1, 0, kmax);
     tile_mac<false>(ch, tl, dys, sP, 1, nullptr, SB, sN, 1, 0, P);
 #pragma unroll
-    for (int i = 0; i < kT; ++i) {
+    for (int i = 0; i < kTN; ++i) {
       if (!tl.rv[i]) continue;
       const int t = tl.r[i];
       float cy = 0.f;
@@ -545,16 +546,16 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
       part[s * PC + tl.tc] = nx;
     }
   }
-  // dB of this head (Q x N): w_s [sum_t Z(t,s) C_t + E(last,s) Lam^T x_s]
-  for (int tile = tid; tile < tiles_of(Qc, N); tile += kThreads) {
-    const Tile tl = make_tile(tile, Qc, N);
-    float bi[kT][kT], bl[kT][kT];
+  // dB of this head (Q x N, 8 x 4 blocks): w_s [sum_t Z(t,s) C_t + E(last,s) Lam^T x_s]
+  for (int tile = tid; tile < tiles_of<kTN, kT>(Qc, N); tile += kThreads) {
+    const TileT<kTN, kT> tl = make_tile<kTN, kT>(tile, Qc, N);
+    float bi[kTN][kT], bl[kTN][kT];
     tile_zero(bi);
     tile_zero(bl);
     tile_mac<false>(bi, tl, Zm, 1, sQ, nullptr, Cs, sN, 1, tl.r[0], Qc);
     tile_mac<false>(bl, tl, xs, sP, 1, nullptr, SB, sN, 1, 0, P);
 #pragma unroll
-    for (int i = 0; i < kT; ++i)
+    for (int i = 0; i < kTN; ++i)
 #pragma unroll
       for (int j = 0; j < kT; ++j)
         if (tl.rv[i] && tl.cv[j]) {
