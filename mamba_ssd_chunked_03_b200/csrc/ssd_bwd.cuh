@@ -158,16 +158,16 @@ __device__ __forceinline__ void chunk_cumsum(const KArgs& a, const ChunkPos& q, 
 
 // ---- register-tiled products of small matrices in shared memory
 //
-// A thread owns a kT x kT block of an M x Nn product: rows r_i = kT tr + i and
-// columns c_j = tc + j TC (TC = ceil(Nn / kT)), with tile = tr TC + tc.  The
+// A thread owns a TM x TN block of an M x Nn product: rows r_i = TM tr + i and
+// columns c_j = tc + j TC (TC = ceil(Nn / TN)), with tile = tr TC + tc.  The
 // threads of a warp take consecutive tc, so they read consecutive columns of
 // one operand and the same few rows of the other (a broadcast); row strides
 // are padded where a column walk would otherwise meet one bank.  Contiguous
 // rows let a triangular product stop at the thread's own first or last row.
 // Indices past the edge are clamped for loads, and their results are never
-// stored.
-constexpr int kT = 4;
-constexpr int kTN = 8;  // rows of the blocks of the Q x dstate products
+// stored.  Each block costs TM + TN shared loads per TM TN multiply-adds.
+constexpr int kT = 4;   // 4 x 4 blocks by default
+constexpr int kTN = 8;  // rows of the 8 x 4 blocks of the Q x dstate and headdim x dstate products
 
 template <int TM, int TN>
 struct TileT {
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_bwd_chunk_states(const KArgs a)
   float* So = a.S + off;
   float* To = a.T + off;
   // 8 x 4 blocks: P x N = 8192 outputs at headdim 64, dstate 128 is one block per thread
-  constexpr int TM = 8, TN = 4;
+  constexpr int TM = kTN, TN = kT;
   const int nt = tiles_of<TM, TN>(P, N);
   for (int tile = tid; tile < nt; tile += kThreads) {
     const TileT<TM, TN> tl = make_tile<TM, TN>(tile, P, N);
