@@ -324,7 +324,9 @@ SSD_API ssd_status ssd_conv1d_silu_bwd(const ssd_conv_bwd_args* args, void* stre
  * adjoint state is carried backwards across chunks, and every chunk then
  * forms its gradients from its own tokens and those two states.  All
  * arithmetic is fp32; every gradient is written as fp32, whatever the input
- * dtype.  Chunking re-associates the same sums, so the result equals the
+ * dtype.  A_h <= 0 is assumed, as for ssd_fwd: the in-chunk decays
+ * exp(cs_t - cs_s) and exp(cs_t) are then at most 1 (with A_h > 0 they can
+ * overflow fp32).  Chunking re-associates the same sums, so the result equals the
  * adjoint recurrence up to rounding for every chunk size. */
 typedef struct {
   /* sizes as in ssd_fwd_args; headdim and dstate at most 256, and one

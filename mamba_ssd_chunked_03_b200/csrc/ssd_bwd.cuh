@@ -315,17 +315,42 @@ __global__ void __launch_bounds__(kThreads) k_bwd_state_passing(const KArgs a) {
   float* S = a.S + bh * d.nc * PN + e;
   float* T = a.T + bh * d.nc * PN + e;
   const float* dec = a.dec + bh * d.nc;
+  // Four chunks' values are loaded before any of them is overwritten, so that
+  // four loads are in flight at a time (the addresses differ, which the
+  // compiler cannot see).
   float run = a.h0 ? a.h0[i] : 0.f;
-  for (int64_t c = 0; c < d.nc; ++c) {
-    const float s = S[c * PN];
+  int64_t c = 0;
+  for (; c + 4 <= d.nc; c += 4) {
+    float v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = S[(c + j) * PN];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      S[(c + j) * PN] = run;
+      run = fmaf(dec[c + j], run, v[j]);
+    }
+  }
+  for (; c < d.nc; ++c) {
+    const float v = S[c * PN];
     S[c * PN] = run;
-    run = fmaf(dec[c], run, s);
+    run = fmaf(dec[c], run, v);
   }
   float lam = a.dfinal ? a.dfinal[i] : 0.f;
-  for (int64_t c = d.nc - 1; c >= 0; --c) {
-    const float u = T[c * PN];
+  c = d.nc - 1;
+  for (; c - 3 >= 0; c -= 4) {
+    float v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = T[(c - j) * PN];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      T[(c - j) * PN] = lam;
+      lam = fmaf(dec[c - j], lam, v[j]);
+    }
+  }
+  for (; c >= 0; --c) {
+    const float v = T[c * PN];
     T[c * PN] = lam;
-    lam = fmaf(dec[c], lam, u);
+    lam = fmaf(dec[c], lam, v);
   }
   if (a.dh0) a.dh0[i] = lam;
 }

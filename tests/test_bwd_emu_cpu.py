@@ -122,7 +122,7 @@ MUTANTS = [
     # the in-chunk sum of dx runs one token past the chunk
     ("dx_past_chunk", r"(tile_mac<false>\(acc, tl, Km, 1, sQ, nullptr, dys, sP, 1, tl\.r\[0\], )Qc\);", r"\1Qc + 1);"),
     # the adjoint carried across chunks skips the chunk decay
-    ("no_decay_backward", r"lam = fmaf\(dec\[c\], lam, u\);", "lam = lam + u;"),
+    ("no_decay_backward", r"lam = fmaf\(dec\[c - j\], lam, v\[j\]\);", "lam = lam + v[j];"),
     # the row term of dcs loses dt
     ("rowm_no_dt", r"row = fmaf\(Mm\[t \* sQ \+ u\], w\[u\], row\);", "row += Mm[t * sQ + u];"),
     # the h_in terms are taken for every token, also after a sequence boundary
