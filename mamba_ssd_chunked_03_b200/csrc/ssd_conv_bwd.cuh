@@ -95,14 +95,24 @@ __global__ void __launch_bounds__(kThreads) k_conv_bwd(const KArgs a) {
 #pragma unroll
   for (int k = 0; k < K; ++k) dw[k] = 0.f;
 
+  // the next token's inputs are loaded before this token's du store, which the
+  // compiler cannot tell apart from them: two tokens' loads in flight
+  float nu = t0 < te ? cv_ld(u, t0 * a.C) : 0.f;
+  float nd = t0 < te ? cv_ld(dout, t0 * a.C) : 0.f;
+  int ns = (t0 < te && seq) ? seq[t0] : 0;
   for (int64_t t = t0; t < te; ++t) {
-    const float cur = cv_ld(u, t * a.C);
-    const int st = seq ? seq[t] : 0;
+    const float cur = nu, dcur = nd;
+    const int st = ns;
+    if (t + 1 < te) {
+      nu = cv_ld(u, (t + 1) * a.C);
+      nd = cv_ld(dout, (t + 1) * a.C);
+      ns = seq ? seq[t + 1] : 0;
+    }
     float pre = fmaf(w[K - 1], cur, bias);
 #pragma unroll
     for (int j = 0; j < K - 1; ++j)
       if (wseq[j] == st) pre = fmaf(w[j], win[j], pre);
-    const float g = cv_ld(dout, t * a.C) * silu_slope(pre);
+    const float g = dcur * silu_slope(pre);
     if (t < t1) {
       db += g;
       dw[K - 1] = fmaf(g, cur, dw[K - 1]);
