@@ -32,9 +32,13 @@ dinitial_states when no state gradient comes in).  So:
    with h_in and Lam_r, which gives its tokens' gradients;
 4. dA and dD, which sum over all tokens, are all-reduced.
 
-The three per-rank operations are taken from ``ops`` (default: the library),
-so the exchange logic can be exercised on CPU ranks with another
-implementation of them.
+With the block's gate z (out = y * SiLU(z)) only the outputs change: the
+exchanged states do not depend on z, so the forward passes z to its final
+local pass, and the backward to its adjoint summary and final pass.
+
+The per-rank operations are taken from ``ops`` (default: the library), so the
+exchange logic can be exercised on CPU ranks with another implementation of
+them.
 """
 from __future__ import annotations
 
@@ -49,8 +53,8 @@ class LibraryOps:
     """The per-rank operations, on the library's kernels."""
 
     @staticmethod
-    def local_forward(x, dt, A, B, C, D, chunk_size, initial_states):
-        return fwd(x, dt, A, B, C, D, chunk_size=chunk_size, initial_states=initial_states)
+    def local_forward(x, dt, A, B, C, D, chunk_size, initial_states, z=None):
+        return fwd(x, dt, A, B, C, D, chunk_size=chunk_size, initial_states=initial_states, z=z)
 
     @staticmethod
     def total_decay(dt, A):
@@ -61,15 +65,15 @@ class LibraryOps:
         return state_fold(states, decays, initial_states, rank, shape)
 
     @staticmethod
-    def local_backward(x, dt, A, B, C, D, dy, initial_states, dfinal_states):
+    def local_backward(x, dt, A, B, C, D, dy, initial_states, dfinal_states, z=None):
         return bwd(x, dt, A, B, C, D, dy, initial_states=initial_states, dfinal_states=dfinal_states,
-                   want_dD=D is not None, want_dinitial_states=True)
+                   want_dD=D is not None, want_dinitial_states=True, z=z)
 
     @staticmethod
-    def adjoint_summary(x, dt, A, B, C, D, dy):
+    def adjoint_summary(x, dt, A, B, C, D, dy, z=None):
         """T: dLoss/d(the state entering the range) from the range's own
         outputs (no state gradient coming in), without the other gradients."""
-        return bwd(x, dt, A, B, C, D, dy, dinitial_only=True)["dinitial_states"]
+        return bwd(x, dt, A, B, C, D, dy, dinitial_only=True, z=z)["dinitial_states"]
 
 
 def local_summary(x, dt, A, B, C, D, chunk_size: int = 64, ops=LibraryOps):
@@ -101,39 +105,44 @@ def _state_in(x, dt, A, B, C, D, chunk_size, initial_states, group, ops):
 
 def fwd_seqpar(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
                D: Optional[torch.Tensor], chunk_size: int = 64, initial_states: Optional[torch.Tensor] = None,
-               group=None, ops=LibraryOps):
+               group=None, ops=LibraryOps, z: Optional[torch.Tensor] = None):
     """The forward of this rank's token range of a sequence split over the
     ranks of ``group``, in rank order.  ``initial_states`` (the state before
-    the sequence's first token, or None) must be the same on every rank.
-    Returns (y of this rank's tokens, the state at the end of its range)."""
+    the sequence's first token, or None) must be the same on every rank;
+    ``z``, this rank's gate (like x), or None.  Returns (y of this rank's
+    tokens, y * SiLU(z) with a gate, and the state at the end of its range)."""
     h_in, _, _ = _state_in(x, dt, A, B, C, D, chunk_size, initial_states, group, ops)
-    return ops.local_forward(x, dt, A, B, C, D, chunk_size, h_in)
+    if z is None:
+        return ops.local_forward(x, dt, A, B, C, D, chunk_size, h_in)
+    return ops.local_forward(x, dt, A, B, C, D, chunk_size, h_in, z=z)
 
 
 def bwd_seqpar(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
                D: Optional[torch.Tensor], dy: torch.Tensor, chunk_size: int = 64,
                initial_states: Optional[torch.Tensor] = None, dfinal_states: Optional[torch.Tensor] = None,
-               group=None, ops=LibraryOps) -> dict:
+               group=None, ops=LibraryOps, z: Optional[torch.Tensor] = None) -> dict:
     """The backward of ``fwd_seqpar`` for this rank's token range.  ``dy`` is
-    dLoss/dy of this rank's tokens; ``initial_states`` and ``dfinal_states``
-    (dLoss/d(the sequence's final state)), each None or the same on every
-    rank.  Returns a dict: dx, ddt, dB, dC of this rank's tokens; dA and dD
-    summed over all ranks; dinitial_states on rank 0 (None elsewhere)."""
+    dLoss/dy of this rank's tokens (of y * SiLU(z) with this rank's gate z);
+    ``initial_states`` and ``dfinal_states`` (dLoss/d(the sequence's final
+    state)), each None or the same on every rank.  Returns a dict: dx, ddt,
+    dB, dC (and dz) of this rank's tokens; dA and dD summed over all ranks;
+    dinitial_states on rank 0 (None elsewhere)."""
     import torch.distributed as dist
     R = dist.get_world_size(group)
     r = dist.get_rank(group)
     h_in, decays, shape = _state_in(x, dt, A, B, C, D, chunk_size, initial_states, group, ops)
+    gate = {} if z is None else {"z": z}
     if hasattr(ops, "adjoint_summary"):
-        T = ops.adjoint_summary(x, dt, A, B, C, D, dy)
+        T = ops.adjoint_summary(x, dt, A, B, C, D, dy, **gate)
     else:
-        T = ops.local_backward(x, dt, A, B, C, D, dy, h_in, None)["dinitial_states"]
+        T = ops.local_backward(x, dt, A, B, C, D, dy, h_in, None, **gate)["dinitial_states"]
     all_T = [torch.empty_like(T) for _ in range(R)]
     dist.all_gather(all_T, T.contiguous(), group=group)
     after = list(range(R - 1, r, -1))  # the ranks after this one, last first
     lam = ops.state_fold(torch.stack([all_T[k] for k in after]) if after else None,
                          torch.stack([decays[k] for k in after]) if after else None,
                          dfinal_states, len(after), shape)
-    g = ops.local_backward(x, dt, A, B, C, D, dy, h_in, lam)
+    g = ops.local_backward(x, dt, A, B, C, D, dy, h_in, lam, **gate)
     dist.all_reduce(g["dA"], group=group)
     if g.get("dD") is not None:
         dist.all_reduce(g["dD"], group=group)

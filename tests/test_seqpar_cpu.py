@@ -18,6 +18,7 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import oracle
+from oracle import backward, block
 import ssd_inputs as si
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -35,8 +36,10 @@ class OracleOps:
     """The per-rank operations of seqpar, on the oracle (fp64)."""
 
     @staticmethod
-    def local_forward(x, dt, A, B, C, D, chunk_size, initial_states):
+    def local_forward(x, dt, A, B, C, D, chunk_size, initial_states, z=None):
         y, f = oracle.ssd_fwd(x, dt, A, B, C, D, initial_states)
+        if z is not None:
+            y = block.gate(y, z)
         return torch.from_numpy(y), torch.from_numpy(f).float()
 
     @staticmethod
@@ -52,11 +55,16 @@ class OracleOps:
         return h.float()
 
     @staticmethod
-    def local_backward(x, dt, A, B, C, D, dy, initial_states, dfinal_states):
+    def local_backward(x, dt, A, B, C, D, dy, initial_states, dfinal_states, z=None):
         b, _, H, P = x.shape
         h0 = initial_states if initial_states is not None else torch.zeros(b, H, P, B.shape[3])
-        g = oracle.ssd_bwd(x, dt, A, B, C, D, h0, dy, dfinal_states, None)
-        out = {k: (None if v is None else torch.from_numpy(v).float()) for k, v in g.items() if k != "dh0"}
+        if z is None:
+            g = oracle.ssd_bwd(x, dt, A, B, C, D, h0, dy, dfinal_states, None)
+        else:
+            g = backward.ssd_bwd_gated(x, dt, A, B, C, D, h0, z, dy, dfinal_states, None,
+                                       backward_fn=oracle.ssd_bwd)
+        out = {k: (None if v is None else torch.from_numpy(np.asarray(v)).float()) for k, v in g.items()
+               if k != "dh0"}
         out["dinitial_states"] = torch.from_numpy(g["dh0"]).float()
         return out
 
@@ -127,49 +135,54 @@ def test_fwd_seqpar_gloo_ranks(cuts):
         assert np.abs(out[world - 1][1] - fw).max() <= 1e-5 * max(1.0, np.abs(fw).max())
 
 
-def _bwd_data():
+def _bwd_data(gated=False):
     shape = si.SSDShape("sp", 2, 200, 3, 8, 8, 1, 64, "f32", h0_std=0.5, seed=5)
     d = si.make_inputs(shape)
     g = torch.Generator().manual_seed(21)
     dy = torch.randn(2, 200, 3, 8, generator=g)
     dfinal = torch.randn(2, 3, 8, 8, generator=g)
+    d["z"] = 2.0 * torch.randn(2, 200, 3, 8, generator=g) if gated else None
     return d, dy, dfinal
 
 
-def _bwd_rank_main(rank, world, port, cuts, out):
+def _bwd_rank_main(rank, world, port, cuts, out, gated=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         from mamba_ssd_chunked_03_b200 import seqpar
-        d, dy, dfinal = _bwd_data()
+        d, dy, dfinal = _bwd_data(gated)
         lo, hi = cuts[rank], cuts[rank + 1]
         p = _split(d, lo, hi)
+        z = None if d["z"] is None else d["z"][:, lo:hi].contiguous()
         g = seqpar.bwd_seqpar(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], dy[:, lo:hi].contiguous(), 64,
-                              d["initial_states"], dfinal, ops=OracleOps)
+                              d["initial_states"], dfinal, ops=OracleOps, z=z)
         out[rank] = {k: (None if v is None else v.numpy()) for k, v in g.items()}
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("cuts", [[0, 117, 200], [0, 64, 65, 200]], ids=["2_ranks", "3_ranks"])
-def test_bwd_seqpar_gloo_ranks(cuts):
+@pytest.mark.parametrize("cuts,gated", [([0, 117, 200], False), ([0, 64, 65, 200], False), ([0, 90, 200], True)],
+                         ids=["2_ranks", "3_ranks", "2_ranks_gated"])
+def test_bwd_seqpar_gloo_ranks(cuts, gated):
     world = len(cuts) - 1
     ctx = mp.get_context("spawn")
     with ctx.Manager() as m:
         out = m.dict()
         port = _free_port()
-        procs = [ctx.Process(target=_bwd_rank_main, args=(r, world, port, cuts, out)) for r in range(world)]
+        procs = [ctx.Process(target=_bwd_rank_main, args=(r, world, port, cuts, out, gated)) for r in range(world)]
         for p in procs:
             p.start()
         for p in procs:
             p.join(180)
         assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
-        d, dy, dfinal = _bwd_data()
-        ref = oracle.ssd_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["initial_states"], dy, dfinal, None)
+        d, dy, dfinal = _bwd_data(gated)
+        args = (d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["initial_states"])
+        ref = (oracle.ssd_bwd(*args, dy, dfinal, None) if not gated else
+               backward.ssd_bwd_gated(*args, d["z"], dy, dfinal, None, backward_fn=oracle.ssd_bwd))
         tol = lambda w: 1e-5 * max(1.0, np.abs(w).max())
-        for k in ("dx", "ddt", "dB", "dC"):
+        for k in ("dx", "ddt", "dB", "dC") + (("dz",) if gated else ()):
             got = np.concatenate([out[r][k] for r in range(world)], axis=1)
             assert np.abs(got - ref[k]).max() <= tol(ref[k]), k
         for r in range(world):  # the shared parameters: every rank holds the sum
