@@ -6,7 +6,7 @@ problem and a packed one compared in full, and the benchmark's c1 layout
 (b 8, L 2048, H 80, P 64, N 128, bf16) at full size compared on one batch
 row: every gradient of a row except dA and dD depends on that row's inputs
 only, and dA, dD (sums over rows) are compared at the smaller sizes.  The
-file name sorts it after the forward's GPU files."""
+file name sorts it after every other GPU file."""
 import numpy as np
 import pytest
 import torch
