@@ -98,7 +98,11 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, cuts, out):
+def _gate(seed=22):
+    return 2.0 * torch.randn(2, 200, 3, 8, generator=torch.Generator().manual_seed(seed))
+
+
+def _rank_main(rank, world, port, cuts, out, gated=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -107,22 +111,24 @@ def _rank_main(rank, world, port, cuts, out):
         shape = si.SSDShape("sp", 2, 200, 3, 8, 8, 1, 64, "f32", h0_std=0.5, seed=5)
         d = si.make_inputs(shape)
         p = _split(d, cuts[rank], cuts[rank + 1])
+        z = _gate()[:, cuts[rank]:cuts[rank + 1]].contiguous() if gated else None
         y, f = seqpar.fwd_seqpar(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], 64, d["initial_states"],
-                                 ops=OracleOps)
+                                 ops=OracleOps, z=z)
         out[rank] = (np.asarray(y), np.asarray(f))
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("cuts", [[0, 117, 200], [0, 64, 65, 200]], ids=["2_ranks", "3_ranks"])
-def test_fwd_seqpar_gloo_ranks(cuts):
+@pytest.mark.parametrize("cuts,gated", [([0, 117, 200], False), ([0, 64, 65, 200], False), ([0, 90, 200], True)],
+                         ids=["2_ranks", "3_ranks", "2_ranks_gated"])
+def test_fwd_seqpar_gloo_ranks(cuts, gated):
     world = len(cuts) - 1
     ctx = mp.get_context("spawn")
     with ctx.Manager() as m:
         out = m.dict()
         port = _free_port()
-        procs = [ctx.Process(target=_rank_main, args=(r, world, port, cuts, out)) for r in range(world)]
+        procs = [ctx.Process(target=_rank_main, args=(r, world, port, cuts, out, gated)) for r in range(world)]
         for p in procs:
             p.start()
         for p in procs:
@@ -130,6 +136,8 @@ def test_fwd_seqpar_gloo_ranks(cuts):
         assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
         shape = si.SSDShape("sp", 2, 200, 3, 8, 8, 1, 64, "f32", h0_std=0.5, seed=5)
         yw, fw = _whole(si.make_inputs(shape))
+        if gated:
+            yw = block.gate(yw, _gate())
         y = np.concatenate([out[r][0] for r in range(world)], axis=1)
         assert np.abs(y - yw).max() <= 1e-5 * max(1.0, np.abs(yw).max())
         assert np.abs(out[world - 1][1] - fw).max() <= 1e-5 * max(1.0, np.abs(fw).max())
