@@ -1,7 +1,7 @@
-"""CPU oracle for the SSD forward -- TEST INFRASTRUCTURE ONLY.
+"""CPU oracle for the SSD forward and backward -- TEST INFRASTRUCTURE ONLY.
 
-Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may import this package.  The product path (the CUDA library and
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline and
+reference legs of ``bench.py`` may import this package.  The product path (the CUDA library and
 its Python binding) never imports, links or calls it, and this package never
 imports the product path.  The only module both sides use is ``ssd_inputs``,
 which draws random tensors and holds none of the method's arithmetic.
@@ -13,11 +13,14 @@ Contents:
                               written out (tiny inputs; a pin for the oracle).
   * ``block.conv1d_silu``, ``block.gate`` -- the Mamba-2 block pieces around the SSD
                               (causal depthwise conv1d + SiLU; the SiLU gate).
+  * ``block.conv1d_silu_bwd`` -- their backward (du, dweight, dbias).
   * ``backward.ssd_bwd``     -- the backward pass: the adjoint of the recurrence
                               (derived; the pages give no formulas), fp64 numpy.
+  * ``backward.ssd_bwd_gated`` -- the backward through the gate y * SiLU(z).
   * ``ssd_bwd``              -- the same adjoint in C + OpenMP (``ssd_oracle.c``),
                               states recomputed from 64-token checkpoints, for
-                              larger inputs.
+                              larger inputs; also the magnitude sums of the terms
+                              of dA and dD (the scale of their rounding).
   * ``chunked.ssd_chunked``  -- the four chunked steps written out literally in
                               fp64 numpy (a pin for the decomposition the CUDA
                               kernels use).
