@@ -380,7 +380,7 @@ typedef struct {
 /* ssd_bwd flags */
 #define SSD_BWD_DINITIAL_ONLY 1u /* compute dinitial_states alone (required then; dx, ddt,
                                     dA, dB, dC, dD, dz may be NULL and are not written):
-                                    two of the five kernels.  Sequence parallelism needs
+                                    two of the six kernels.  Sequence parallelism needs
                                     only this from its first backward pass.          */
 
 /* Bytes of device workspace ssd_bwd needs (only sizes, chunk_size and dtype
@@ -392,7 +392,7 @@ SSD_API size_t ssd_bwd_workspace_size(const ssd_bwd_args* args);
  * unsupported.  Reads only the size fields; no device work. */
 SSD_API int64_t ssd_bwd_chunk_size(const ssd_bwd_args* args);
 
-/* Enqueue the backward on `stream`: five kernels, no allocation, no memset.
+/* Enqueue the backward on `stream`: six kernels, no allocation, no memset.
  * All pointers are device pointers owned by the caller; outputs must not
  * overlap inputs or the workspace.  Returns SSD_OK once enqueued;
  * SSD_ERR_INVALID_ARG for a null required pointer, a bad size or enum, or a

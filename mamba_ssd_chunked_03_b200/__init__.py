@@ -460,7 +460,7 @@ def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     torch.cuda.Event pair recorded around the dominant kernel.  ``z``: the
     forward's gate (like x); dy is then the gradient of y * SiLU(z), and the
     dict also holds dz (fp32).  ``dinitial_only``: compute dinitial_states
-    alone (two of the five kernels); the other entries are None."""
+    alone (two of the six kernels); the other entries are None."""
     _check(x, dt, A, B, C, D, initial_states, seq_idx)
     if dy.dtype != x.dtype or tuple(dy.shape) != tuple(x.shape) or dy.device != x.device or not dy.is_contiguous():
         raise ValueError("dy must be a contiguous tensor like x")

@@ -34,12 +34,14 @@
 // chunk's y from the same K and h_in, writes dz = dout y SiLU'(z), and all of
 // the above then runs on dy = dout SiLU(z).
 //
-// Five kernels, in stream order:
+// Six kernels, in stream order:
 //   k_bwd_chunk_states   per (b, c, h): the chunk's end state from a zero
 //                        state, its adjoint input sum_t e_t dy_t C_t^T, and
 //                        its decay e_last
 //   k_bwd_state_passing  per state entry: h_in of every chunk (forward) and
 //                        Lam of every chunk (backward), dinitial_states
+//   k_bwd_chunk_cb       per (b, c, g): C_t.B_s of the chunk, which the
+//                        group's heads share
 //   k_bwd_chunk          per (b, c, h): the formulas above from the chunk's
 //                        tokens, h_in and Lam; dB and dC per head
 //   k_bwd_group_sum      dB, dC summed over each group's heads
@@ -99,6 +101,7 @@ struct KArgs {
   float* S;         // (b,H,nc,P,N): chunk end states from zero, then each chunk's h_in
   float* T;         // (b,H,nc,P,N): each chunk's sum_t e_t dy_t C_t^T, then its Lam
   float* dec;       // (b,H,nc): e_last of each chunk
+  float* CB;        // (b,nc,G,Q,Q): C_t.B_s of each chunk, shared by the group's heads
   float* dBh;       // (b,L,H,N): dB per head
   float* dCh;       // (b,L,H,N): dC per head
   double* dA_part;  // (H, b*nc)
@@ -227,6 +230,46 @@ __device__ __forceinline__ void tile_mac(float (&acc)[TM][TN], const TileT<TM, T
     for (int i = 0; i < TM; ++i)
 #pragma unroll
       for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+  }
+}
+
+// Shared-memory floats of k_bwd_chunk_cb for chunk length Q.
+inline size_t smem_cb_floats(int64_t Q, int64_t N) { return (size_t)(2 * Q * (N + 1)); }
+
+// C_t.B_s (Q x Q, over dstate) of every chunk and group: the heads of a group
+// share it.  One CTA per (b, c, g), g fastest.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_bwd_chunk_cb(const KArgs a) {
+  const Dims& d = a.d;
+  const int64_t bid = blockIdx.x;
+  const int64_t g = bid % d.G, c = (bid / d.G) % d.nc, b = bid / (d.G * d.nc);
+  const int64_t t0 = c * d.Q;
+  const int Qc = (int)(d.L - t0 < d.Q ? d.L - t0 : d.Q);
+  const int N = (int)d.N, Q = (int)d.Q, sN = N + 1;
+  const int tid = threadIdx.x;
+  SSD_DYN_SMEM(sm);
+  float* Bs = sm;            // Q x sN
+  float* Cs = Bs + Q * sN;   // Q x sN
+  const T* B = static_cast<const T*>(a.B);
+  const T* C = static_cast<const T*>(a.C);
+  for (int i = tid; i < Qc * N; i += kThreads) {
+    const int t = i / N, n = i % N;
+    const int64_t gi = ((b * d.L + t0 + t) * d.G + g) * d.N + n;
+    Bs[t * sN + n] = ld(B, gi);
+    Cs[t * sN + n] = ld(C, gi);
+  }
+  __syncthreads();
+  float* out = a.CB + ((b * d.nc + c) * d.G + g) * d.Q * d.Q;
+  for (int tile = tid; tile < tiles_of(Qc, Qc); tile += kThreads) {
+    const Tile tl = make_tile(tile, Qc, Qc);
+    float cb[kT][kT];
+    tile_zero(cb);
+    tile_mac<false>(cb, tl, Cs, sN, 1, nullptr, Bs, 1, sN, 0, N);
+#pragma unroll
+    for (int i = 0; i < kT; ++i)
+#pragma unroll
+      for (int j = 0; j < kT; ++j)
+        if (tl.rv[i] && tl.cv[j]) out[tl.r[i] * Q + tl.c[j]] = cb[i][j];
   }
 }
 
@@ -434,21 +477,15 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
   __syncthreads();
 
   const int last = Qc - 1;
-  // K = E o (C B^T) on the chunk's Q x Q triangle, and the decays to the chunk's ends
-  for (int tile = tid; tile < tiles_of(Qc, Qc); tile += kThreads) {
-    const Tile tl = make_tile(tile, Qc, Qc);
-    float cb[kT][kT];
-    tile_zero(cb);
-    tile_mac<false>(cb, tl, Cs, sN, 1, nullptr, Bs, 1, sN, 0, N);
-#pragma unroll
-    for (int i = 0; i < kT; ++i)
-#pragma unroll
-      for (int j = 0; j < kT; ++j) {
-        if (!tl.rv[i] || !tl.cv[j]) continue;
-        const int t = tl.r[i], s = tl.c[j];
-        const float e = (s <= t && seg[s] == seg[t]) ? expf(cs[t] - cs[s]) : 0.f;
-        Km[t * sQ + s] = e * cb[i][j];
-      }
+  // K = E o (C B^T) on the chunk's Q x Q triangle (C B^T from k_bwd_chunk_cb, once
+  // per group), and the decays to the chunk's ends
+  {
+    const float* cb = a.CB + ((q.b * d.nc + q.c) * d.G + q.g) * d.Q * d.Q;
+    for (int i = tid; i < Qc * Qc; i += kThreads) {
+      const int t = i / Qc, s = i % Qc;
+      const float e = (s <= t && seg[s] == seg[t]) ? expf(cs[t] - cs[s]) : 0.f;
+      Km[t * sQ + s] = s <= t ? e * cb[t * Q + s] : 0.f;
+    }
   }
   for (int t = tid; t < Qc; t += kThreads) {
     el[t] = seg[t] == seg[last] ? expf(cs[last] - cs[t]) : 0.f;
@@ -681,7 +718,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd_param_sum(const KArgs a) {
 struct Plan {
   Dims d;
   size_t smem_states, smem_chunk;  // bytes
-  size_t off_S, off_T, off_dec, off_dBh, off_dCh, off_dA, off_dD, total;
+  size_t smem_cb;                  // bytes
+  size_t off_S, off_T, off_dec, off_CB, off_dBh, off_dCh, off_dA, off_dD, total;
 };
 
 inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -718,6 +756,7 @@ inline ssd_status plan(const ssd_bwd_args* a, Plan* pl) {
   if (chunk_ctas >= 2147483647.0 || state_ctas >= 2147483647.0 || group_ctas >= 2147483647.0)
     return SSD_ERR_UNSUPPORTED;
   pl->smem_states = smem_states_floats(Q, d.P, d.N) * 4;
+  pl->smem_cb = smem_cb_floats(Q, d.N) * 4;
   pl->smem_chunk = smem_chunk_floats(Q, d.P, d.N) * 4;
   const size_t states = (size_t)(d.b * d.H * d.nc) * (size_t)(d.P * d.N) * 4;
   const size_t per_head = (size_t)(d.b * d.L * d.H) * (size_t)d.N * 4;
@@ -729,6 +768,8 @@ inline ssd_status plan(const ssd_bwd_args* a, Plan* pl) {
   o = align256(o + states);
   pl->off_dec = o;
   o = align256(o + (size_t)(d.b * d.H * d.nc) * 4);
+  pl->off_CB = o;
+  o = align256(o + (size_t)(d.b * d.nc * d.G) * (size_t)(d.Q * d.Q) * 4);
   pl->off_dBh = o;
   o = align256(o + per_head);
   pl->off_dCh = o;
@@ -782,6 +823,7 @@ inline KArgs make_kargs(const ssd_bwd_args* a, const Plan& pl) {
   k.S = reinterpret_cast<float*>(ws + pl.off_S);
   k.T = reinterpret_cast<float*>(ws + pl.off_T);
   k.dec = reinterpret_cast<float*>(ws + pl.off_dec);
+  k.CB = reinterpret_cast<float*>(ws + pl.off_CB);
   k.dBh = reinterpret_cast<float*>(ws + pl.off_dBh);
   k.dCh = reinterpret_cast<float*>(ws + pl.off_dCh);
   k.dA_part = reinterpret_cast<double*>(ws + pl.off_dA);
@@ -791,7 +833,7 @@ inline KArgs make_kargs(const ssd_bwd_args* a, const Plan& pl) {
 
 inline unsigned blocks_for(int64_t n) { return (unsigned)((n + kThreads - 1) / kThreads); }
 
-// Validate, then enqueue the five kernels through `launch(kernel, grid,
+// Validate, then enqueue the six kernels through `launch(kernel, grid,
 // shared bytes, args)`, which returns false when a launch fails;
 // `launch.record(event)` records a caller's timing event (false on failure).
 template <typename T, class Launch>
@@ -804,6 +846,7 @@ ssd_status enqueue_typed(const KArgs& k, const Plan& pl, void* const events[2], 
     if (events[0] && !(launch.record(events[0]) && launch.record(events[1]))) return SSD_ERR_CUDA;
     return SSD_OK;
   }
+  if (!launch(&k_bwd_chunk_cb<T>, (unsigned)(d.b * d.nc * d.G), pl.smem_cb, k)) return SSD_ERR_CUDA;
   if (events[0] && !launch.record(events[0])) return SSD_ERR_CUDA;
   if (!launch(&k_bwd_chunk<T>, chunk_ctas, pl.smem_chunk, k)) return SSD_ERR_CUDA;
   if (events[1] && !launch.record(events[1])) return SSD_ERR_CUDA;

@@ -25,7 +25,7 @@ dinitial_states when no state gradient comes in).  So:
 1. every rank recovers h_in as in the forward, and computes T_k: the
    backward's dinitial_states with no incoming state gradient (which does not
    depend on h_in; ``ssd_bwd`` with ``SSD_BWD_DINITIAL_ONLY`` runs two of its
-   five kernels for it);
+   six kernels for it);
 2. the ranks all-gather (T_k, D_k);
 3. rank r folds Lam_r from the sequence's dfinal through ranks R-1..r+1
    (``ssd_state_fold`` over the reversed lists) and runs its backward again
