@@ -639,22 +639,23 @@ BWD_SHAPE = si.SSDShape("c1_bwd", 8, 2048, 80, 64, 128, 1, 64, "bf16", seed=1001
 BWD_WORKLOAD = "SSD bwd on the c1 layout: b8 L2048 H80 P64 N128 G1 bf16, from dy, fp32 gradients"
 
 
-def bwd_flops(b, L, H, P, N, Q):
-    """Algorithmic FLOPs (2 per multiply-add) of the backward's two per-chunk
-    kernels, (k_bwd_chunk_states, k_bwd_chunk), for chunk length Q.  Per chunk
-    of Qc tokens, with T2 = Qc (Qc + 1) / 2 lower-triangle pairs:
-    k_bwd_chunk_states forms two P x N sums of Qc outer products (2 Qc P N);
-    k_bwd_chunk forms C B^T and dy x^T on the triangle (T2 (N + P)), Lam B^T
-    and h_in C^T (2 Qc P N), the triangle products for dx, dB, dC
-    (T2 (P + 2 N)), the state terms of dB and dC (2 Qc P N) and <Lam, h_in>
-    (P N)."""
-    states = chunk = 0
+def bwd_flops(b, L, H, P, N, Q, G=1):
+    """Algorithmic FLOPs (2 per multiply-add) of the backward's per-chunk
+    kernels, (k_bwd_chunk_states, k_bwd_chunk_cb, k_bwd_chunk), for chunk
+    length Q.  Per chunk of Qc tokens, with T2 = Qc (Qc + 1) / 2
+    lower-triangle pairs: k_bwd_chunk_states forms two P x N sums of Qc outer
+    products (2 Qc P N per head); k_bwd_chunk_cb forms C B^T on the triangle
+    (T2 N per group); k_bwd_chunk forms dy x^T on the triangle (T2 P), Lam B^T
+    (Qc P N), the triangle products for dx, dB, dC (T2 (P + 2 N)), the state
+    terms of dB and dC (2 Qc P N) and <Lam, h_in> (P N) per head."""
+    states = cb = chunk = 0
     for c in range(-(-L // Q)):
         qc = min(Q, L - c * Q)
         t2 = qc * (qc + 1) // 2
         states += 2 * qc * P * N
-        chunk += t2 * (3 * N + 2 * P) + 4 * qc * P * N + P * N
-    return 2 * b * H * states, 2 * b * H * chunk
+        cb += t2 * N
+        chunk += t2 * (2 * N + 2 * P) + 3 * qc * P * N + P * N
+    return 2 * b * H * states, 2 * b * G * cb, 2 * b * H * chunk
 
 
 def bwd_inputs(shape, rank=0):
@@ -782,7 +783,7 @@ def run_bwd(args, dist, dev, world, rank):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev) / E
 
-    f_states, f_chunk = bwd_flops(b, L, H, P, N, Q)
+    f_states, f_cb, f_chunk = bwd_flops(b, L, H, P, N, Q, shape.ngroups)
     achieved = f_chunk / (kernel_ms / 1e3) / 1e12
     tokens = b * L
     line = {
@@ -800,7 +801,8 @@ def run_bwd(args, dist, dev, world, rank):
                      "kernel": "k_bwd_chunk", "kernel_ms": kernel_ms,
                      "kernel_ms_p10_p50_p90": [per[int(0.1 * (K - 1))], per[int(0.5 * (K - 1))],
                                                per[int(0.9 * (K - 1))]],
-                     "traffic": None, "algorithmic_flops": f_chunk, "states_kernel_flops": f_states},
+                     "traffic": None, "algorithmic_flops": f_chunk, "states_kernel_flops": f_states,
+                     "cb_kernel_flops": f_cb},
         "e2e": {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": E},
         "gpu_launches": 6 * K,
