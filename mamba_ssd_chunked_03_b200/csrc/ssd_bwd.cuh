@@ -47,6 +47,8 @@
 //   k_bwd_group_sum      dB, dC summed over each group's heads
 //   k_bwd_param_sum      dA, dD summed over rows and chunks (fp64)
 //
+// With SSD_BWD_DINITIAL_ONLY only the first two run.
+//
 // All fp32 on the CUDA cores; every loop is bounded by the chunk's own token
 // count, and nothing waits on another CTA.  The kernels use only standard
 // CUDA built-ins so that the same source also runs, for tests only, under a
