@@ -175,3 +175,16 @@ def random_case(seed: int):
 
 
 RANDOM_SEEDS = list(range(1000, 1012))
+
+
+def out_of_order_case():
+    """A packed batch whose ids do not increase along the tokens (a change of
+    id starts a sequence, whatever its value), with a gate: (inputs, dy,
+    dfinal, chunk)."""
+    b, L, H, P, N, G = 2, 90, 4, 16, 24, 2
+    d = inputs(b, L, H, P, N, G, "f32", 0.3, None, seed=5)
+    seq = torch.tensor([[7] * 20 + [3] * 1 + [5] * 40 + [0] * 29,
+                        [2] * 45 + [9] * 45], dtype=torch.int32)
+    d["seq_idx"], d["num_seqs"] = seq, 10
+    d["z"] = gate_like(b, L, H, P, torch.float32, 5)
+    return d, dy_like(b, L, H, P, torch.float32, 5), None, 16

@@ -191,3 +191,10 @@ def test_dinitial_only_gives_the_same_bits_and_writes_nothing_else():
     assert only["status"] == 0 and only["launches"] == 2
     assert np.array_equal(only["dh0"], full["dh0"])
     assert all(only[k] is None for k in ("dx", "ddt", "dA", "dB", "dC", "dD", "dz"))
+
+
+def test_emulated_backward_with_ids_out_of_order():
+    from bwd_cases import out_of_order_case
+    d, dy, dfinal, chunk = out_of_order_case()
+    out = emu_bwd.run(d, dy, dfinal, chunk_size=chunk, z=d["z"])
+    compare(out, oracle_bwd(d, dy, dfinal))

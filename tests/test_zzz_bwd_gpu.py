@@ -166,3 +166,9 @@ def test_backward_on_random_shapes(seed):
     """The seeded random problems of the host emulation's sweep, on the GPU."""
     d, dy, dfinal, chunk, _ = random_case(seed)
     compare(_gpu_bwd(d, dy, dfinal, chunk), oracle_bwd(d, dy, dfinal))
+
+
+def test_backward_with_ids_out_of_order():
+    from bwd_cases import out_of_order_case
+    d, dy, dfinal, chunk = out_of_order_case()
+    compare(_gpu_bwd(d, dy, dfinal, chunk), oracle_bwd(d, dy, dfinal))
