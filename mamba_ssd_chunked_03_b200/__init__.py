@@ -1,11 +1,12 @@
-"""Chunked SSD (Mamba-2 structured state space duality) forward on B200.
+"""Chunked SSD (Mamba-2 structured state space duality) forward and backward on B200.
 
 Thin Python binding over the C ABI in ``include/ssd.h`` (``libssd.so``, built
 in-tree by ``mamba_ssd_chunked_03_b200/build.py``).  This module only marshals
 arguments: it checks tensor placement, dtypes and shapes, allocates outputs
-and the workspace with PyTorch on the current stream, and calls ``ssd_fwd``.
-Every step of the forward runs in the library's CUDA kernels; there is no
-Python or CPU fallback, and importing fails loudly if the library is missing.
+and the workspace with PyTorch on the current stream, and calls the library
+(``ssd_fwd``, ``ssd_bwd``, ``ssd_step``, ``ssd_conv1d_silu`` and the rest).
+Every step runs in the library's CUDA kernels; there is no Python or CPU
+fallback, and importing fails loudly if the library is missing.
 
     y, final_states = fwd(x, dt, A, B, C, D, chunk_size=64,
                           initial_states=None, seq_idx=None, num_seqs=None)
@@ -21,7 +22,8 @@ from typing import Optional
 
 import torch
 
-__all__ = ["fwd", "bwd", "BwdArgs", "bwd_workspace_size", "bwd_chunk_size", "ssd_chunked",
+__all__ = ["fwd", "bwd", "BwdArgs", "bwd_workspace_size", "bwd_chunk_size", "ssd_chunked", "make_args",
+           "make_bwd_args", "main_kernel", "device_status",
            "conv1d_silu_bwd", "ConvBwdArgs", "causal_conv1d_silu", "step", "StepArgs", "total_decay", "state_fold", "conv1d_silu", "ConvArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
            "SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED", "SSD_ERR_WORKSPACE", "SSD_ERR_CUDA",
            "SSD_F32", "SSD_BF16", "SSD_FLAG_GENERIC"]
