@@ -25,11 +25,16 @@
 //   dLam' = e_last Lam + sum_t e_t dy_t C_t^T     (= dLoss/dh_in)
 //
 // and, for the log-decays l_k = dt_k A (cs_t = sum of l_k over the segment
-// up to t), dcs_t = sum_{s<t} M(t,s) - sum_{u>t} M(u,t) + e_t dy_t.(h_in C_t)
-// - N_t (+ e_last <Lam,h_in> + sum_s N_s at the last token), with
-// M(t,s) = E(t,s) w_s (C_t.B_s)(dy_t.x_s) and N_s = E(last,s) w_s x_s^T Lam B_s;
-// dl_k = sum of dcs_t over t >= k in k's segment, ddt_k = dw_k + A dl_k and
+// up to t), with M(t,s) = E(t,s) w_s (C_t.B_s)(dy_t.x_s) and
+// N_s = E(last,s) w_s x_s^T Lam B_s:
+//
+//   dl_k = sum_{s < k <= t} M(t,s) + sum_{t >= k} e_t dy_t.(h_in C_t)
+//          + sum_{s < k} N_s + e_last <Lam, h_in>
+//
+// (every term whose decay spans token k), ddt_k = dw_k + A dl_k and
 // dA = sum_k dt_k dl_k.  A token that starts a segment has no decay term.
+// The pair sum is formed directly over the block s < k <= t; written as row
+// sums minus column sums, the pairs after k would cancel only to rounding.
 // With the block's gate (out = y SiLU(z)), k_bwd_chunk first recomputes the
 // chunk's y from the same K and h_in, writes dz = dout y SiLU'(z), and all of
 // the above then runs on dy = dout SiLU(z).
@@ -637,42 +642,49 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
   }
   __syncthreads();
 
-  // per token: the row and column sums of M in quarters, four threads per token
+  // per token k, four threads each: a quarter of the column sum of M below the
+  // diagonal (for dw) and of the block sum S_k = sum_{u >= k, s < k} M(u,s) w_s,
+  // the pairs whose decay spans k
   for (int i = tid; i < 4 * Qc; i += kThreads) {
-    const int t = i >> 2, qq = i & 3;
-    const int lo = Qc * qq / 4, hi = Qc * (qq + 1) / 4;
-    float col = 0.f, row = 0.f;
+    const int k = i >> 2, qq = i & 3;
+    const int lo = k + (Qc - k) * qq / 4, hi = k + (Qc - k) * (qq + 1) / 4;
+    float col = 0.f, blk = 0.f;
     for (int u = lo; u < hi; ++u) {
-      if (u > t) col += Mm[u * sQ + t];
-      if (u < t) row = fmaf(Mm[t * sQ + u], w[u], row);
+      if (u > k) col += Mm[u * sQ + k];
+      for (int s2 = 0; s2 < k; ++s2) blk = fmaf(Mm[u * sQ + s2], w[s2], blk);
     }
-    part[t * PC + qq] = col;
-    part[t * PC + 4 + qq] = row;
+    part[k * PC + qq] = col;
+    part[k * PC + 4 + qq] = blk;
   }
   __syncthreads();
   for (int t = tid; t < Qc; t += kThreads) {
     const float col = part[t * PC] + part[t * PC + 1] + part[t * PC + 2] + part[t * PC + 3];
-    const float row = part[t * PC + 4] + part[t * PC + 5] + part[t * PC + 6] + part[t * PC + 7];
+    const float blk = part[t * PC + 4] + part[t * PC + 5] + part[t * PC + 6] + part[t * PC + 7];
     dw[t] = fmaf(el[t], nv[t], col + Mm[t * sQ + t]);
     nn[t] = el[t] * w[t] * nv[t];
-    dcs[t] = row - w[t] * col + dcs[t] - nn[t];
+    part[t * PC] = blk;  // S_t
   }
   __syncthreads();
 
   if (tid == 0) {
+    // dl_k = S_k + sum_{t >= k} (h_in term)_t + sum_{s < k} N_s + e_last <Lam, h_in>;
+    // the h_in terms live in the first sequence only and N in the last, so
+    // none of the sums crosses a boundary that matters
     float lh = 0.f;
     for (int i = 0; i < kThreads; ++i) lh += red[i];
-    float sn = 0.f;
-    for (int t = 0; t < Qc; ++t) sn += nn[t];
     const float e_last = seg[last] == -1 ? expf(cs[last]) : 0.f;
-    dcs[last] += sn + e_last * lh;
+    float before = 0.f;  // sum_{s < k} N_s, kept in nn as an exclusive prefix
+    for (int k = 0; k <= last; ++k) {
+      const float v = nn[k];
+      nn[k] = before;
+      before += v;
+    }
     const float Ah = a.A[q.h];
     double dA = 0.0, dD = 0.0;
-    float run = 0.f;
+    float after = 0.f;  // sum_{t >= k} of the h_in term (kept in dcs)
     for (int k = last; k >= 0; --k) {
-      if (k == last || seg[k] != seg[k + 1]) run = 0.f;
-      run += dcs[k];
-      const float dl = seg[k] == k ? 0.f : run;  // a segment's first token has no decay
+      after += dcs[k];
+      const float dl = seg[k] == k ? 0.f : part[k * PC] + after + nn[k] + e_last * lh;  // none at a sequence start
       a.ddt[(q.b * d.L + q.t0 + k) * d.H + q.h] = fmaf(Ah, dl, dw[k]);
       dA += (double)w[k] * (double)dl;
       dD += (double)dg[k];

@@ -123,8 +123,8 @@ MUTANTS = [
     ("dx_past_chunk", r"(tile_mac<false>\(acc, tl, Km, 1, sQ, nullptr, dys, sP, 1, tl\.r\[0\], )Qc\);", r"\1Qc + 1);"),
     # the adjoint carried across chunks skips the chunk decay
     ("no_decay_backward", r"lam = fmaf\(dec\[c - j\], lam, v\[j\]\);", "lam = lam + v[j];"),
-    # the row term of dcs loses dt
-    ("rowm_no_dt", r"row = fmaf\(Mm\[t \* sQ \+ u\], w\[u\], row\);", "row += Mm[t * sQ + u];"),
+    # the pair sum of dl loses dt
+    ("pairs_no_dt", r"blk = fmaf\(Mm\[u \* sQ \+ s2\], w\[s2\], blk\);", "blk += Mm[u * sQ + s2];"),
     # the h_in terms are taken for every token, also after a sequence boundary
     ("hin_always", r"ein\[t\] = seg\[t\] == -1 \? expf\(cs\[t\]\) : 0\.f;", "ein[t] = expf(cs[t]);"),
     # tiles numbered with the wrong divisor: parts of a non-square product are never written
