@@ -65,17 +65,20 @@ def silu_grad(v: np.ndarray) -> np.ndarray:
     return s * (1.0 + v * (1.0 - s))
 
 
-def conv1d_silu_bwd(u, weight, bias, dout, seq_idx=None) -> tuple:
+def conv1d_silu_bwd(u, weight, bias, dout, seq_idx=None, with_scale: bool = False) -> tuple:
     """Gradients of sum(dout * conv1d_silu(u, weight, bias, seq_idx)):
     (du (b, L, C), dweight (C, K), dbias (C)), fp64.  With g = dout * SiLU'(pre),
     each tap k that the forward takes (reading token t - shift for output t)
     sends w[c, k] g[t] back to du[t - shift] and adds g[t] u[t - shift] to
-    dweight[c, k]; dbias = sum over rows and tokens of g."""
+    dweight[c, k]; dbias = sum over rows and tokens of g.  With ``with_scale``
+    two more arrays follow: the sums of the magnitudes of the terms of dweight
+    and of dbias (the scale a rounding error in those sums is measured against)."""
     u, w = as_f64(u), as_f64(weight)
     b, L, C = u.shape
     g = as_f64(dout) * silu_grad(_pre(u, w, bias, seq_idx))
     du = np.zeros((b, L, C))
     dw = np.zeros(w.shape)
+    dw_abs = np.zeros(w.shape)
     for k, shift, src in _taps(u, w.shape[1], seq_idx):
         valid = np.zeros((b, L, 1))  # the tap reads a real input (not the zero before a row or sequence)
         valid[:, shift:] = 1.0
@@ -84,6 +87,9 @@ def conv1d_silu_bwd(u, weight, bias, dout, seq_idx=None) -> tuple:
             valid[:, shift:, 0] = seq[:, shift:] == seq[:, : L - shift]
         du[:, : L - shift] += (w[None, None, :, k] * g * valid)[:, shift:]
         dw[:, k] = np.einsum("blc,blc->c", g, src)
+        dw_abs[:, k] = np.einsum("blc,blc->c", np.abs(g), np.abs(src))
+    if with_scale:
+        return du, dw, g.sum(axis=(0, 1)), dw_abs, np.abs(g).sum(axis=(0, 1))
     return du, dw, g.sum(axis=(0, 1))
 
 

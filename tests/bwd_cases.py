@@ -125,15 +125,22 @@ def conv_case_inputs(case):
 
 
 def conv_compare(du, dw, db, ref):
-    """du, dw, dbias against the fp64 oracle's (du, dw, dbias): the same bounds
-    as the SSD backward (fp32 sums of at most K terms per du, b L terms per
-    dw and dbias, the latter in fp64 over per-strip partials)."""
+    """du, dw, dbias against the fp64 oracle's (du, dw, dbias[, dw_abs,
+    dbias_abs]): du by the SSD backward's bounds (fp32 sums of at most K
+    terms); dw and dbias, signed sums over every token, element by element
+    within REL_L2 times the sums of their terms' magnitudes when the oracle
+    gives them (``with_scale``), else by the same relative bounds."""
+    scales = {"dw": ref[3], "dbias": ref[4]} if len(ref) > 3 else {}
     for name, got, want in (("du", du, ref[0]), ("dw", dw, ref[1]), ("dbias", db, ref[2])):
         if got is None:
             continue
         got = np.asarray(got, dtype=np.float64)
         assert got.shape == want.shape, name
         assert np.isfinite(got).all(), name
+        if name in scales:
+            err = np.abs(got - want)
+            assert (err <= REL_L2 * scales[name] + 1e-30).all(), f"{name}: {err.max():.3g}"
+            continue
         rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
         assert rel <= REL_L2, f"{name}: rel L2 {rel:.3g}"
         assert np.abs(got - want).max() <= MAX_ABS * max(1.0, np.abs(want).max()), name

@@ -18,7 +18,7 @@ def test_emulated_conv_backward_matches_oracle(case, reverse):
     u, w, bias, dout, seq = conv_case_inputs(case)
     out = emu_bwd.run_conv(u, w, bias, dout, seq, reverse=reverse)
     assert out["status"] == 0 and out["launches"] == 2
-    conv_compare(out["du"], out["dw"], out["dbias"], block.conv1d_silu_bwd(u, w, bias, dout, seq))
+    conv_compare(out["du"], out["dw"], out["dbias"], block.conv1d_silu_bwd(u, w, bias, dout, seq, with_scale=True))
 
 
 def test_emulated_conv_backward_without_dbias():

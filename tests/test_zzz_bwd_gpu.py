@@ -144,7 +144,7 @@ def test_conv_backward_matches_oracle(case):
     du, dw, db = ssd.conv1d_silu_bwd(cu(u), cu(w), cu(bias), cu(dout), cu(seq))
     torch.cuda.synchronize()
     conv_compare(du.cpu().numpy(), dw.cpu().numpy(), None if db is None else db.cpu().numpy(),
-                 block.conv1d_silu_bwd(u, w, bias, dout, seq))
+                 block.conv1d_silu_bwd(u, w, bias, dout, seq, with_scale=True))
 
 
 def test_conv_autograd_function_routes_through_the_library():
@@ -156,9 +156,8 @@ def test_conv_autograd_function_routes_through_the_library():
     leaves = [t.cuda().requires_grad_(True) for t in (u, w, bias)]
     out = ssd.causal_conv1d_silu(leaves[0], leaves[1], leaves[2], seq.cuda())
     (out.double() * dout.cuda().double()).sum().backward()
-    du, dw, db = block.conv1d_silu_bwd(u, w, bias, dout, seq)
     conv_compare(leaves[0].grad.cpu().numpy(), leaves[1].grad.cpu().numpy(), leaves[2].grad.cpu().numpy(),
-                 (du, dw, db))
+                 block.conv1d_silu_bwd(u, w, bias, dout, seq, with_scale=True))
 
 
 @pytest.mark.parametrize("seed", RANDOM_SEEDS)
