@@ -74,6 +74,12 @@ typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
 #define SSD_FLAG_CHECK_SEQ 2u /* check the seq_idx precondition first: ssd_fwd copies
                                  seq_idx to the host (waiting for `stream`) and
                                  returns ssd_check_seq_idx's verdict if it fails */
+#define SSD_FLAG_TEST_STALL 4u /* for tests of the failure path only: the two-head
+                                  kernel's state hand-over between CTAs waits on a
+                                  flag that nothing sets, so that bounded wait runs
+                                  out (after 1 s) and ssd_fwd_device_status reports
+                                  SSD_ERR_TIMEOUT; y is then incomplete.  Shapes
+                                  without a hand-over are not affected. */
 
 typedef struct {
   /* sizes: b = batch, L = seqlen, H = nheads, P = headdim, N = dstate,

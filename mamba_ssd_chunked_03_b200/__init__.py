@@ -34,6 +34,7 @@ SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_WORKSPACE, SSD_ERR_CUD
 SSD_F32, SSD_BF16 = 0, 1
 SSD_FLAG_GENERIC = 1
 SSD_FLAG_CHECK_SEQ = 2
+SSD_FLAG_TEST_STALL = 4  # failure-path tests only: the two-head kernel's hand-over wait runs out
 SSD_BWD_DINITIAL_ONLY = 1
 
 
@@ -263,7 +264,8 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
         num_seqs: Optional[int] = None, return_final_states: bool = True,
         y: Optional[torch.Tensor] = None, final_states: Optional[torch.Tensor] = None,
         workspace: Optional[torch.Tensor] = None, generic: bool = False,
-        timing_events: Optional[tuple] = None, z: Optional[torch.Tensor] = None, check_seq: bool = False):
+        timing_events: Optional[tuple] = None, z: Optional[torch.Tensor] = None, check_seq: bool = False,
+        check_status: bool = False, flags: int = 0):
     """SSD forward.  Returns (y, final_states or None).
 
     x (b,L,H,P) fp32|bf16, dt (b,L,H) fp32, A (H) fp32, B/C (b,L,G,N) x.dtype,
@@ -277,6 +279,11 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     y * SiLU(z).
     ``check_seq``: check the seq_idx precondition on a host copy first
     (synchronous; raises SSDError on a violation).
+    ``check_status``: wait for the call and raise SSDError(SSD_ERR_TIMEOUT)
+    if a bounded device-side wait gave up (y is then incomplete); without it
+    the call is asynchronous and such a failure is seen only through
+    ``device_status``.
+    ``flags``: further SSD_FLAG_* bits passed through to ssd_fwd.
     """
     _check(x, dt, A, B, C, D, initial_states, seq_idx)
     if z is not None and (z.dtype != x.dtype or tuple(z.shape) != tuple(x.shape) or z.device != x.device
@@ -297,6 +304,7 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
                   generic=generic, z=z)
     if check_seq:
         a.flags |= SSD_FLAG_CHECK_SEQ
+    a.flags |= int(flags)
     need = int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
     if need > 0:
         if workspace is None or workspace.numel() * workspace.element_size() < need:
@@ -311,6 +319,10 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
     st = lib.ssd_fwd(ctypes.byref(a), ctypes.c_void_p(stream))
     if st != SSD_OK:
         raise SSDError(st)
+    if check_status:
+        st = int(lib.ssd_fwd_device_status(ctypes.byref(a), ctypes.c_void_p(stream)))
+        if st != SSD_OK:
+            raise SSDError(st)
     return y, final_states
 
 

@@ -22,7 +22,7 @@ ssd_status check_sizes(const ssd_fwd_args* a) {
   if (a->nheads % a->ngroups != 0) return SSD_ERR_INVALID_ARG;
   if (!is_pow2(a->chunk_size) || a->chunk_size < 16 || a->chunk_size > 256) return SSD_ERR_INVALID_ARG;
   if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
-  if (a->flags & ~(SSD_FLAG_GENERIC | SSD_FLAG_CHECK_SEQ)) return SSD_ERR_INVALID_ARG;
+  if (a->flags & ~(SSD_FLAG_GENERIC | SSD_FLAG_CHECK_SEQ | SSD_FLAG_TEST_STALL)) return SSD_ERR_INVALID_ARG;
   if (a->seq_idx && a->num_seqs <= 0) return SSD_ERR_INVALID_ARG;
   if (a->seq_idx && a->num_seqs > (int64_t)1 << 31) return SSD_ERR_INVALID_ARG;
   // implemented shape set
@@ -64,6 +64,7 @@ Problem resolve(const ssd_fwd_args* a) {
   p.num_seqs = a->seq_idx ? a->num_seqs : 0;
   p.y = a->y;
   p.final_states = a->final_states;
+  p.stall = (a->flags & SSD_FLAG_TEST_STALL) != 0;
   return p;
 }
 

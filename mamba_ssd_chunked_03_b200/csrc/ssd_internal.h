@@ -25,6 +25,7 @@ struct Problem {
   void* y;
   float* final_states;
   const void* z;  // gate: y * SiLU(z), or null
+  bool stall;     // SSD_FLAG_TEST_STALL: the two-head kernel's hand-over waits never succeed
 };
 
 constexpr size_t kWsAlign = 256;

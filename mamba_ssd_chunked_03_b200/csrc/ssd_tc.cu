@@ -694,7 +694,7 @@ TcWorkspace tc_carve(const Problem& p, void* ws, size_t* total) {
   w.err = reinterpret_cast<int*>(base);
   w.failed_count = reinterpret_cast<int*>(base + sizeof(int));
   w.flags = pair ? reinterpret_cast<int*>(base + 2 * sizeof(int)) : nullptr;
-  const size_t nflags = (size_t)kPairFlagsPerCta * kPairGridMax;
+  const size_t nflags = (size_t)kPairFlagsPerCta * kPairGridMax + 1;  // + the never-set flag
   w.pair_bad = pair ? reinterpret_cast<int*>(base + (2 + nflags) * sizeof(int)) : nullptr;
   size_t zero_ints = 2 + (pair ? nflags + (size_t)(p.b * p.H / 2) : 0);
   w.unit_bad = p.seq ? reinterpret_cast<int*>(base + zero_ints * sizeof(int)) : nullptr;

@@ -70,12 +70,15 @@ struct FastArgs {
   RunList runs;
   int* unit_bad;
   const __nv_bfloat16* z;  // gate (b, L, H, 64): y * SiLU(z), or null
+  int stall;               // two-head kernel: hand-overs wait on the never-set flag (failure-path tests)
 };
 
 // persistent grid of the two-head kernel, at most; per-CTA hand-over size
 constexpr int kPairGridMax = 256;
 constexpr int kPairHandoffFloats = 2 * 128 * 64;
-constexpr int kPairFlagsPerCta = 8;  // one per state warp
+constexpr int kPairFlagsPerCta = 16;  // one per state warp
+// the flag after the last CTA's: cleared every call and never set (SSD_FLAG_TEST_STALL)
+constexpr int kPairNeverFlag = kPairGridMax * kPairFlagsPerCta;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -829,6 +829,7 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
   fa.z = static_cast<const __nv_bfloat16*>(p.z);
   fa.runs = w.runs;
   fa.unit_bad = w.unit_bad;
+  fa.stall = p.stall ? 1 : 0;
   // (a gated call takes the single-head kernel, whose epilogue applies the gate)
   if (!varlen && !p.z && NS == 128 && tc_pair_supported(p)) {
     CUtensorMap ty, tdt;

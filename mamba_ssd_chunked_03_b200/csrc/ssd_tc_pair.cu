@@ -2,42 +2,49 @@
 // factorised-decay formulation): one CTA owns two heads (h, h+1) of the same
 // batch row and B/C group and walks their chunks together.  The heads share
 // the C, B and W' = masked C B^T tiles, and every MMA covers both heads at
-// once with N = 128:
+// once with M = 128 rows (p of head h, then p of head h+1):
 //
-//   Yd   = W' [X'_h | X'_h+1]                     (M = 64 tokens,  K = 64 tokens)
-//   S'^T = B^T [X'_h | X'_h+1]                    (M = 128 states, K = 64 tokens)
-//   Yd  += C [H_h | H_h+1]^T                      (M = 64 tokens,  K = N)
-//   y_t  = u_t Yd_t + D x_t,   H <- 2^cs_e (H + S')
+//   Yd^T  = X'^T W'^T                 (N = 64 tokens t,  K = 64 tokens s)
+//   S     = X'^T B                    (N = 128 states,   K = 64 tokens s)
+//   Yd^T += H C^T                     (N = 64 tokens t,  K = N states)
+//   y_t   = u_t Yd_t + D x_t,   H <- 2^cs_e (H + S)
 //
 // per head, with cs_t the in-chunk cumulative sum of dt A (log2 units),
 // u_t = 2^cs_t, v_s = 2^-cs_s dt_s and X' = diag(v) x: u_t v_s = exp of the
 // decay from s to t times dt_s.  The factors are taken about the chunk's
 // first token (ssd_tc_fast.cu takes them about its middle), so the state
-// enters the C H^T product as it is, with no per-chunk rescaling; a chunk
+// enters the H C^T product as it is, with no per-chunk rescaling; a chunk
 // whose total decay exceeds 2^kRangeLog2 sends the pair to the exact kernel.
-// The chunked steps are those
-// of "SSM 家族全景图（下）：Mamba-2 与 Jamba" section 三.4; the D feed-through
-// is from "从Transformer的二次复杂度困境到Mamba的线性突围" (continuous SSM).
+// The chunked steps are those of "SSM 家族全景图（下）：Mamba-2 与 Jamba"
+// section 三.4; the D feed-through is from "从Transformer的二次复杂度困境到Mamba
+// 的线性突围" (continuous SSM).
 //
-// The D x_t feed-through is taken from the scaled tile: D x_t = (D / v_t) X'_t,
-// so the epilogue needs no second read of x.  It writes y over X' in the
-// same shared-memory slot (each thread overwrites exactly what it read) and
-// a bulk tensor store per head moves the tile out.
+// Both A operands live in tensor memory: X'^T (scaled from the x tile through
+// 8 x 8 transposing loads) and the bf16 copy of the state.  Shared memory
+// carries only the TMA tiles (x, W', B, C, dt), the MMAs' B operands and the
+// y tile, which the epilogue writes over x in the same slot before a bulk
+// tensor store per head moves it out.  The chunk-to-chunk chain is short: S
+// of chunk g lands, the state warps load it, fold it into the fp32 state and
+// store the next bf16 state; only then do they scale the x tile of chunk
+// g + 2, off that chain, and the next chunk's S and W' products do not wait
+// for the state.
 //
-// Warp roles (512 threads), each a loop over the chunks that only waits on
+// Warp roles (896 threads), each a loop over the chunks that only waits on
 // the barriers it needs:
-//   warp 0      TMA loads (one thread): x 3 chunks ahead (L2 prefetch 6 ahead),
-//               W', B, C 2 ahead
+//   warp 0      TMA loads (one thread): W', B, C 2 chunks ahead
 //   warp 1      MMA issue (descriptors formed by the warp, one elected lane issues)
-//   warp 2      dt scan of both heads: u, v, D / v and the chunk scalars; it
-//               also loads dt by TMA into an 8-deep ring of its own
-//   warp 3      y stores (one thread); frees an x slot once its tile is read out
-//   warps 4-7   the epilogue of both heads
-//   warps 8-11, 12-15   one head each: state update (fp32 state in registers),
-//               publishing the bf16 e^m H tile, and scaling the head's next
-//               x tile into X' in place
-// x tiles sit in a 4-deep ring; W'+B, C, the e^m H tiles, Yd and S are
-// double-buffered.  Every wait is bounded; a CTA that times out records the
+//   warp 2      dt scan of both heads: u, v and the chunk scalars; it also
+//               loads dt by TMA into an 8-deep ring of its own
+//   warp 3      y stores and x loads (one thread): an x slot of the 8-slot
+//               ring is refilled 8 chunks ahead once its y tile is read out
+//   warps 4-11  the epilogue: warp 4 + 4 half + q owns TMEM rows 32q.. (head
+//               q/2, p = 32 (q&1) + lane) and tokens [32 half, 32 half + 32)
+//   warps 12-27 the state: warp 12 + 4 nq + q owns TMEM rows 32q.. and states
+//               n in [32 nq, 32 nq + 32): fp32 state in registers, its bf16
+//               copy in TMEM, and tokens [16 nq, 16 nq + 16) of the x scaling
+//               into X'^T two chunks ahead
+// TMEM (512 columns): Yd^T x2 (64 columns each), S x1 (128), the bf16 state x2
+// (64), X'^T x4 (32).  Every wait is bounded; a CTA that times out records the
 // error, drains its copies, stores and MMAs, frees its TMEM and exits.
 //
 // The grid is persistent: with G CTAs, CTA i owns the contiguous range
@@ -65,22 +72,21 @@ using namespace tc;
 
 struct PairCfg {
   static constexpr int NS = 128, NB = 2;
-  static constexpr int kThreads = 512;
+  static constexpr int kThreads = 896;
   static constexpr uint32_t kTile = 8192;
-  static constexpr int kXSlots = 4;
-  static constexpr uint32_t oX = 0;                        // [4 slots][2 heads] x -> X' -> y, in place
-  static constexpr uint32_t oW = oX + 2 * kXSlots * kTile; // [2] W' tiles
-  static constexpr uint32_t oB = oW + 2 * kTile;           // [2] B, 2 n-blocks each
-  static constexpr uint32_t oC = oB + 2 * NB * kTile;      // [2] C, 2 n-blocks each
-  static constexpr uint32_t oH = oC + 2 * NB * kTile;      // [2 bufs][2 heads] e^m H, 16 KB each
-  static constexpr uint32_t kHTile = NB * kTile;
-  static constexpr uint32_t oDt = oH + 4 * kHTile;          // [8] dt boxes: 64 tokens x 4 heads fp32
+  static constexpr int kXSlots = 8;  // x ring (power of two)
+  static constexpr uint32_t oX = 0;                         // [8 slots][2 heads] x -> y, in place
+  static constexpr uint32_t oW = oX + 2 * kXSlots * kTile;  // [2] W' tiles
+  static constexpr uint32_t oB = oW + 2 * kTile;            // [2] B, 2 n-blocks each
+  static constexpr uint32_t oC = oB + 2 * NB * kTile;       // [2] C, 2 n-blocks each
+  static constexpr uint32_t oDt = oC + 2 * NB * kTile;      // [8] dt boxes: 64 tokens x 4 heads fp32
   static constexpr uint32_t kDtBox = 64 * 16;
   static constexpr uint32_t oEnd = oDt + 8 * kDtBox;
   static constexpr uint32_t kSmemBytes = oEnd + 1024;
-  // TMEM: Yd[2] at 0 / 128 (M = 64 layout, head j in columns 64j..64j+63),
-  //       S[2]  at 256 / 384 (M = 128 layout, head j in columns 64j..)
-  static constexpr uint32_t tYd0 = 0, tS0 = 256, kTmemCols = 512;
+  // TMEM (M = 128 layout, row = lane = 64 j + p for head h0 + j):
+  //   Yd^T[2] fp32, 64 columns (t) each;  S fp32, 128 columns (n);
+  //   H[2] bf16, 64 columns (two n per column);  X'^T[4] bf16, 32 columns (two s per column)
+  static constexpr uint32_t tYd0 = 0, tS = 128, tH0 = 256, tX0 = 384, kTmemCols = 512;
 };
 
 constexpr int kPairMaxSeg = 32;  // segments (pairs touched) per CTA, at most
@@ -88,16 +94,17 @@ constexpr int kPairMaxSeg = 32;  // segments (pairs touched) per CTA, at most
 // Ring barriers are indexed like the buffers they guard, so no barrier can
 // complete a second phase before every waiter has seen the first.
 struct __align__(16) PairSmem {
-  uint64_t full_x[4], x_empty[4];        // x ring: TMA landed / y tile read out by the store
+  uint64_t full_x[8], x_empty[8];        // x ring: TMA landed / scaled (state-only pass)
   uint64_t full_dt[8];                   // dt ring (the scan warp's own)
   uint64_t full_wb[2], full_c[2];        // W' + B, C of a chunk landed
   uint64_t scan_full[4], scan_empty[4];  // scan results of a chunk ready / consumed
-  uint64_t xp_ready[4];                  // X' of a chunk scaled
+  uint64_t xp_ready[4];                  // X'^T of a chunk in TMEM
   uint64_t s_full[2];                    // S of a chunk in TMEM (its W' and B reads are done)
-  uint64_t mma_done[2];                  // every MMA of a chunk done: Yd final, C and e^m H free
-  uint64_t h_ready[2];                   // e^m H of a chunk published
-  uint64_t acc_free[2];                  // Yd (epilogue) and S (state) TMEM buffers read out
-  uint64_t y_staged[4];                  // y of a chunk written over its x slot
+  uint64_t s_free[2];                    // S of a chunk read out by the state warps
+  uint64_t mma_done[2];                  // every MMA of a chunk done: Yd final, C free
+  uint64_t h_ready[2];                   // bf16 state for a chunk written to TMEM
+  uint64_t acc_free[2];                  // Yd of a chunk read out by the epilogue
+  uint64_t y_staged[8];                  // y of a chunk written over its x slot
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -109,13 +116,12 @@ struct __align__(16) PairSmem {
   int seg_i0[kPairMaxSeg];  // split mode: the first CTA whose range holds the segment's pair start
   alignas(16) float u[4][2][64];  // written as float4
   alignas(16) float v[4][2][64];
-  alignas(16) float g[4][2][64];  // D / v_t: D x_t = g_t X'_t
-  float sc[4][2][4];  // [0]: d = 2^cs_e, the chunk's total decay
+  float sc[4][2][4];  // [0]: d = 2^cs_e, the chunk's total decay; [1]: D of the head
 };
 
-static_assert(offsetof(PairSmem, u) % 16 == 0 && offsetof(PairSmem, v) % 16 == 0 &&
-                  offsetof(PairSmem, g) % 16 == 0,
+static_assert(offsetof(PairSmem, u) % 16 == 0 && offsetof(PairSmem, v) % 16 == 0,
               "scan results are stored as float4");
+static_assert(PairCfg::kSmemBytes + sizeof(PairSmem) <= 227 * 1024, "shared memory per CTA");
 
 // Position of one of a CTA's step streams (each role walks its steps in
 // order): segment k, chunk c.  next() moves to the following step.
@@ -139,7 +145,7 @@ struct PairCursor {
 // W', C, y) and leaves the end state in handoff and the segment's total decay
 // per head in seg_decay.
 template <bool kStateOnly>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(896, 1)
     k_ssd_fwd_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_dt,
@@ -156,23 +162,28 @@ __global__ void __launch_bounds__(512, 1)
   const int nc = (int)a.nc;
 
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       mbar_init(&s.full_x[i], 1);
-      mbar_init(&s.x_empty[i], 1);
+      // the state-only pass stores no y: the x scalers (state warps) free the slot
+      mbar_init(&s.x_empty[i], 512);
+      mbar_init(&s.y_staged[i], 256);
+      mbar_init(&s.full_dt[i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&s.scan_full[i], 32);
-      mbar_init(&s.scan_empty[i], kStateOnly ? 256 : 384);  // epilogue warps and state warps
-      mbar_init(&s.xp_ready[i], 256);  // both heads' state warps
-      mbar_init(&s.y_staged[i], 128);
+      // the state warps, and in the fused pass the epilogue warps
+      mbar_init(&s.scan_empty[i], kStateOnly ? 512 : 256 + 512);
+      mbar_init(&s.xp_ready[i], 512);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.full_wb[i], 1);
       mbar_init(&s.full_c[i], 1);
       mbar_init(&s.s_full[i], 1);
+      mbar_init(&s.s_free[i], 512);
       mbar_init(&s.mma_done[i], 1);
-      mbar_init(&s.h_ready[i], 256);
-      mbar_init(&s.acc_free[i], kStateOnly ? 256 : 384);  // epilogue (Yd) and state (S) readers
+      mbar_init(&s.h_ready[i], 512);
+      mbar_init(&s.acc_free[i], 256);
     }
-    for (int i = 0; i < 8; ++i) mbar_init(&s.full_dt[i], 1);
     mbar_init(&s.drain, 1);
     s.abort_flag = *reinterpret_cast<volatile int*>(a.err) != 0;
     s.never = 0;
@@ -246,25 +257,14 @@ __global__ void __launch_bounds__(512, 1)
   const int total = s.total;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA loads
+    // ------------------------------------------------------------ TMA loads: W', B, C
     if (lane == 0) {
-      int last_x = -1, last_wb = -1, last_c = -1;
+      int last_wb = -1, last_c = -1;
       // (the argument is this CTA's step number; each stream has a cursor on
       // its pair and chunk, advanced as the stream issues its steps in order)
-      PairCursor ux, uwb, uc, upf;
-      ux.start(s);
+      PairCursor uwb, uc;
       uwb.start(s);
       uc.start(s);
-      upf.start(s);
-      for (int k = 0; k < 3; ++k) upf.next(s);
-      auto issue_x = [&](int gg) {
-        const int sl = gg & 3, bb = s.seg_b[ux.k], hh = s.seg_h0[ux.k];
-        mbar_arrive_expect_tx(&s.full_x[sl], 2 * K::kTile);
-        for (int j = 0; j < 2; ++j)
-          tma_load_3d(sm + K::oX + (sl * 2 + j) * K::kTile, &tm_x, &s.full_x[sl], (hh + j) * 64, ux.c * 64, bb);
-        ux.next(s);
-        last_x = gg;
-      };
       auto issue_wb = [&](int gg) {
         const int i = gg & 1, bb = s.seg_b[uwb.k], grp = s.seg_grp[uwb.k];
         mbar_arrive_expect_tx(&s.full_wb[i], (kStateOnly ? K::NB : 1 + K::NB) * K::kTile);
@@ -285,18 +285,7 @@ __global__ void __launch_bounds__(512, 1)
         uc.next(s);
         last_c = gg;
       };
-      // x comes from HBM and takes several chunk periods to arrive; L2
-      // prefetches run 6 chunks ahead of use, the loads into the ring 3
-      auto prefetch_x = [&](int) {
-        const int bb = s.seg_b[upf.k], hh = s.seg_h0[upf.k];
-        for (int j = 0; j < 2; ++j) tma_prefetch_l2_3d(&tm_x, (hh + j) * 64, upf.c * 64, bb);
-        upf.next(s);
-      };
       if (!*abort_flag) {
-        #pragma unroll 1
-        for (int c = 3; c < 6 && c < total; ++c) prefetch_x(c);
-        #pragma unroll 1
-        for (int c = 0; c < 3 && c < total; ++c) issue_x(c);  // slot 3 starts free
         if (!kStateOnly) griddep_wait();  // W' comes from the C B^T kernel launched before this one
         #pragma unroll 1
         for (int c = 0; c < 2 && c < total; ++c) {
@@ -307,27 +296,15 @@ __global__ void __launch_bounds__(512, 1)
       bool ok = !*abort_flag;
       // each tile is refilled for a later chunk as soon as its last reader is done
       #pragma unroll 1
-      for (int c = 0; c < total && ok; ++c) {
-        if (c + 2 < total) {
-          ok = mbar_wait(&s.s_full[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
-          if (ok) issue_wb(c + 2);
-          if (!kStateOnly) {
-            ok = ok && mbar_wait(&s.mma_done[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
-            if (ok) issue_c(c + 2);
-          }
-        }
-        // x of step c + 3 goes where step c - 1 was, once its y tile has been stored
-        if (ok && c + 3 < total) {
-          ok = c < 1 || mbar_wait(&s.x_empty[(c - 1) & 3], ((c - 1) >> 2) & 1, abort_flag, kWaitLimitNs);
-          if (ok) issue_x(c + 3);
-          if (ok && c + 6 < total) prefetch_x(c + 6);
+      for (int c = 0; c + 2 < total && ok; ++c) {
+        ok = mbar_wait(&s.s_full[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
+        if (ok) issue_wb(c + 2);
+        if (!kStateOnly) {
+          ok = ok && mbar_wait(&s.mma_done[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
+          if (ok) issue_c(c + 2);
         }
       }
       if (*abort_flag) {  // let this CTA's own copies land before its smem is released
-        // (within one ring-depth window every slot holds a single chunk)
-        #pragma unroll 1
-        for (int c = last_x - 3 < 0 ? 0 : last_x - 3; c <= last_x; ++c)
-          mbar_wait(&s.full_x[c & 3], (c >> 2) & 1, never, kWaitLimitNs);
         #pragma unroll 1
         for (int c = last_wb - 1 < 0 ? 0 : last_wb - 1; c <= last_wb; ++c)
           mbar_wait(&s.full_wb[c & 1], (c >> 1) & 1, never, kWaitLimitNs);
@@ -341,49 +318,51 @@ __global__ void __launch_bounds__(512, 1)
     // The whole warp walks the loop and forms the descriptors (warp-uniform
     // values); one elected lane issues the MMAs and commits.
     const uint32_t aW = smem_u32(sm + K::oW), aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB);
-    const uint32_t aX = smem_u32(sm + K::oX), aH = smem_u32(sm + K::oH);
-    constexpr uint32_t id_y = idesc_bf16(64, 128, 0, 1);    // A K-major, B MN-major (2 heads)
-    constexpr uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // both MN-major
+    constexpr uint32_t id_y = idesc_bf16(128, 64, 0, 0);   // A in TMEM, B K-major
+    constexpr uint32_t id_s = idesc_bf16(128, 128, 0, 1);  // A in TMEM, B MN-major
     #pragma unroll 1
     for (int c = 0; c < total; ++c) {
-      const int i = c & 1;
+      const int i = c & 1, xb = c & 3;
       const uint32_t ph = (c >> 1) & 1;
       bool ok = mbar_wait_warp(&s.full_wb[i], ph, abort_flag, kWaitLimitNs);
-      ok = ok && mbar_wait_warp(&s.xp_ready[c & 3], (c >> 2) & 1, abort_flag, kWaitLimitNs);
-      if (c >= 2) ok = ok && mbar_wait_warp(&s.acc_free[i], ((c - 2) >> 1) & 1, abort_flag, kWaitLimitNs);
+      ok = ok && mbar_wait_warp(&s.xp_ready[xb], (c >> 2) & 1, abort_flag, kWaitLimitNs);
+      if (!kStateOnly && c >= 2) ok = ok && mbar_wait_warp(&s.acc_free[i], ((c - 2) >> 1) & 1, abort_flag, kWaitLimitNs);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t yd = tmem + K::tYd0 + 128 * i;
-      const uint32_t st = tmem + K::tS0 + 128 * i;
-      // X' of both heads, this chunk; a K step of 16 tokens is 16 rows (2048 B)
-      const uint64_t dxp = sw128_desc(aX + (c & 3) * 2 * K::kTile, K::kTile, 1024);
-      const uint64_t dw = sw128_desc(aW + i * K::kTile, 16, 1024);  // a K step is 32 B along the row
+      const uint32_t yd = tmem + K::tYd0 + 64 * i;
+      const uint32_t ax = tmem + K::tX0 + 32 * xb;  // X'^T of both heads, this chunk
+      const uint64_t dw = sw128_desc(aW + i * K::kTile, 16, 1024);
       const uint64_t db = sw128_desc(aB + i * K::NB * K::kTile, K::kTile, 1024);
-      if (elect_one()) {
-        // Yd = W' [X'_0 | X'_1]   (K = 64 tokens)
-        if (!kStateOnly) {
+      if (!kStateOnly) {
+        // Yd^T = X'^T W'^T   (K = 64 tokens s; a K step is 32 bytes along the row)
+        if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(yd, dw + 2 * kk, dxp + 128 * kk, id_y, kk > 0);
+          for (int kk = 0; kk < 4; ++kk) mma_bf16_ts(yd, ax + 8 * kk, dw + 2 * kk, id_y, kk > 0);
         }
-        // S'^T = B^T [X'_0 | X'_1]   (M = 128 states, K = 64 tokens)
+        __syncwarp();
+      }
+      // S = X'^T B   (N = 128 states, K = 64 tokens s; a K step is 16 rows), once
+      // the state warps have read out the previous chunk's S
+      if (c >= 1 && !mbar_wait_warp(&s.s_free[(c - 1) & 1], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(st, db + 128 * kk, dxp + 128 * kk, id_s, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ts(tmem + K::tS, ax + 8 * kk, db + 128 * kk, id_s, kk > 0);
         mma_commit(&s.s_full[i]);
-        if (kStateOnly) mma_commit(&s.x_empty[c & 3]);  // X' read: the slot may be refilled
       }
       __syncwarp();
       if (kStateOnly) continue;
-      // Yd += C [e^m H_0 | e^m H_1]^T   (K = N)
+      // Yd^T += H C^T   (K = N states)
       ok = mbar_wait_warp(&s.h_ready[i], ph, abort_flag, kWaitLimitNs);
       ok = ok && mbar_wait_warp(&s.full_c[i], ph, abort_flag, kWaitLimitNs);
       if (!ok) break;
       tc_fence_after();
       const uint64_t dc = sw128_desc(aC + i * K::NB * K::kTile, 16, 1024);
-      const uint64_t dh = sw128_desc(aH + i * 2 * K::kHTile, K::kHTile, 1024);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < NS / 16; ++kk)
-          mma_bf16_ss(yd, dc + ((kk >> 2) * K::kTile + (kk & 3) * 32) / 16, dh + 128 * kk, id_y, 1);
+          mma_bf16_ts(yd, tmem + K::tH0 + 64 * i + 8 * kk, dc + ((kk >> 2) * K::kTile + (kk & 3) * 32) / 16, id_y,
+                      1);
         mma_commit(&s.mma_done[i]);
       }
       __syncwarp();
@@ -454,17 +433,13 @@ __global__ void __launch_bounds__(512, 1)
       const int e = nvalid - 1;
       const float mine = (e & 3) == 0 ? cs[0] : (e & 3) == 1 ? cs[1] : (e & 3) == 2 ? cs[2] : cs[3];
       const float cse = __shfl_sync(0xffffffffu, mine, e >> 2, 16);
-      float u4[4], v4[4], g4[4];
+      float u4[4], v4[4];
       bool bad = false;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         u4[k] = exp2f(cs[k]);
         v4[k] = exp2f(-cs[k]) * d[k];
-        // D x_t is recovered from X'_t = v_t x_t, so a valid token needs v_t well
-        // inside the normal range (the fast division is exact to 2 ulp there)
-        g4[k] = dsk != 0.f ? __fdividef(dsk, v4[k]) : 0.f;
-        bad |= !(fabsf(cs[k]) <= kRangeLog2) ||
-               (dsk != 0.f && 4 * l16 + k < nvalid && !(fabsf(v4[k]) >= 1e-30f && fabsf(v4[k]) <= 1e30f));
+        bad |= !(fabsf(cs[k]) <= kRangeLog2);
       }
       // a chunk the factorised form cannot take: the exact kernel redoes the
       // pair (once, however many chunks or CTAs find it)
@@ -476,9 +451,9 @@ __global__ void __launch_bounds__(512, 1)
       }
       *reinterpret_cast<float4*>(&s.u[slot][j][4 * l16]) = make_float4(u4[0], u4[1], u4[2], u4[3]);
       *reinterpret_cast<float4*>(&s.v[slot][j][4 * l16]) = make_float4(v4[0], v4[1], v4[2], v4[3]);
-      *reinterpret_cast<float4*>(&s.g[slot][j][4 * l16]) = make_float4(g4[0], g4[1], g4[2], g4[3]);
       if (l16 == 0) {
         s.sc[slot][j][0] = exp2f(cse);
+        s.sc[slot][j][1] = dsk;
       }
       mbar_arrive(&s.scan_full[slot]);
     }
@@ -487,110 +462,198 @@ __global__ void __launch_bounds__(512, 1)
       for (int c = last_dt - 7 < 0 ? 0 : last_dt - 7; c <= last_dt; ++c)
         mbar_wait(&s.full_dt[c & 7], (c >> 3) & 1, never, kWaitLimitNs);
   } else if (warp == 3) {
-    // ------------------------------------------------------------ y stores
-    // (the state-only pass stores no y: its MMAs free the x slots)
-    if (!kStateOnly && lane == 0) {
-      PairCursor uy;
+    // ---------------------------------------------- y stores and x loads
+    // An x slot is refilled (8 steps ahead) as soon as the y tile written
+    // over it has been read out by its store; in the state-only pass, which
+    // stores no y, as soon as the state warps have scaled it.  x comes from
+    // HBM: L2 prefetches run 3 steps ahead of the loads.
+    if (lane == 0) {
+      int last_x = -1;
+      PairCursor ux, uy, upf;
+      ux.start(s);
       uy.start(s);
-      #pragma unroll 1
-      for (int c = 0; c < total; ++c, uy.next(s)) {
-        const int sl = c & 3;
-        if (!mbar_wait(&s.y_staged[sl], (c >> 2) & 1, abort_flag, kWaitLimitNs)) break;
+      upf.start(s);
+      for (int k = 0; k < K::kXSlots + 3; ++k) upf.next(s);
+      auto issue_x = [&](int gg) {
+        const int sl = gg & (K::kXSlots - 1), bb = s.seg_b[ux.k], hh = s.seg_h0[ux.k];
+        mbar_arrive_expect_tx(&s.full_x[sl], 2 * K::kTile);
         for (int j = 0; j < 2; ++j)
-          tma_store_3d(&tm_y, sm + K::oX + (sl * 2 + j) * K::kTile, (s.seg_h0[uy.k] + j) * 64, uy.c * 64,
-                       s.seg_b[uy.k]);
-        bulk_commit_group();
-        bulk_wait_read<0>();  // the tiles have been read out: the slot may be refilled
-        mbar_arrive(&s.x_empty[sl]);
+          tma_load_3d(sm + K::oX + (sl * 2 + j) * K::kTile, &tm_x, &s.full_x[sl], (hh + j) * 64, ux.c * 64, bb);
+        ux.next(s);
+        last_x = gg;
+      };
+      auto prefetch_x = [&]() {
+        const int bb = s.seg_b[upf.k], hh = s.seg_h0[upf.k];
+        for (int j = 0; j < 2; ++j) tma_prefetch_l2_3d(&tm_x, (hh + j) * 64, upf.c * 64, bb);
+        upf.next(s);
+      };
+      if (!*abort_flag) {
+        #pragma unroll 1
+        for (int c = K::kXSlots; c < K::kXSlots + 3 && c < total; ++c) prefetch_x();
+        #pragma unroll 1
+        for (int c = 0; c < K::kXSlots && c < total; ++c) issue_x(c);  // the ring starts free
       }
+      #pragma unroll 1
+      for (int c = 0; c < total && !*abort_flag; ++c) {
+        const int sl = c & (K::kXSlots - 1);
+        if (!kStateOnly) {
+          if (!mbar_wait(&s.y_staged[sl], (c >> 3) & 1, abort_flag, kWaitLimitNs)) break;
+          for (int j = 0; j < 2; ++j)
+            tma_store_3d(&tm_y, sm + K::oX + (sl * 2 + j) * K::kTile, (s.seg_h0[uy.k] + j) * 64, uy.c * 64,
+                         s.seg_b[uy.k]);
+          bulk_commit_group();
+          bulk_wait_read<0>();  // the tiles have been read out: the slot may be refilled
+          uy.next(s);
+        } else if (!mbar_wait(&s.x_empty[sl], (c >> 3) & 1, abort_flag, kWaitLimitNs)) {
+          break;
+        }
+        if (c + K::kXSlots < total) {
+          issue_x(c + K::kXSlots);
+          if (c + K::kXSlots + 3 < total) prefetch_x();
+        }
+      }
+      if (*abort_flag)  // let this CTA's own x copies land before its smem is released
+        #pragma unroll 1
+        for (int c = last_x - (K::kXSlots - 1) < 0 ? 0 : last_x - (K::kXSlots - 1); c <= last_x; ++c)
+          mbar_wait(&s.full_x[c & (K::kXSlots - 1)], (c >> 3) & 1, never, kWaitLimitNs);
       bulk_wait<0>();  // stores complete before the CTA's shared memory is released
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------ epilogue warps (both heads)
+    // Warp 4 + 4 half + q reads Yd^T rows 32q.. (head q/2, p = 32 (q&1) + ..)
+    // at tokens [32 half, 32 half + 32) with the 16x256b shape, which gives
+    // each thread (p, t..t+1) pairs: 8 x 8 blocks in the layout of an 8 x 8
+    // transpose.  Per block, x is loaded as (t, p..p+1) and transposed to
+    // (p, t..t+1), y = u_t Yd + D x is formed in fp32, and the bf16 result is
+    // transposed back and stored where x was read.
     if constexpr (!kStateOnly) {
-      const int q = warp & 3;              // TMEM lane quadrant
+      const int q = warp & 3;
+      const int j = q >> 1;                   // head h0 + j
+      const int ch = 32 * ((warp - 4) >> 2);  // first token of this warp's half
       const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
-      const int te = 16 * q + (lane & 15);   // epilogue row (token) of this thread
-      const int half = lane >> 4;            // epilogue columns p in [32 half, 32 half + 32)
       #pragma unroll 1
-      for (int c = 1; c <= total; ++c) {
-        // ---- epilogue for step c-1, both heads: y = u_t Yd + (D / v_t) X'_t, written over X'
-        if (c >= 1) {
-          const int ip = (c - 1) & 1, slp = (c - 1) & 3;
-          if (!mbar_wait_warp(&s.mma_done[ip], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) break;
-          tc_fence_after();
-          #pragma unroll 1
-          for (int j = 0; j < 2; ++j) {
-            uint32_t r[32];
-            SSD_TMEM_LD_16x32bx2_X32_HALF32(tq + K::tYd0 + 128 * ip + 64 * j, r);
-            SSD_TMEM_WAIT_LD_32(r);
-            const float ut = s.u[slp][j][te], gt = s.g[slp][j][te];
-            unsigned char* row = sm + K::oX + (slp * 2 + j) * K::kTile + te * 128;
-  #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              // 16-byte column 4 half + k of row te, at its swizzled position
-              uint4* px = reinterpret_cast<uint4*>(row + (((4 * half + k) ^ (te & 7)) << 4));
-              const uint4 xv = *px;
-              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-              uint32_t o[4];
-  #pragma unroll
-              for (int k2 = 0; k2 < 4; ++k2) {
-                float x0, x1;
-                unpack_bf16x2(xw[k2], x0, x1);
-                const int jj = 8 * k + 2 * k2;
-                o[k2] = pack_bf16x2(fmaf(ut, __uint_as_float(r[jj]), gt * x0),
-                                    fmaf(ut, __uint_as_float(r[jj + 1]), gt * x1));
-              }
-              *px = make_uint4(o[0], o[1], o[2], o[3]);
-            }
+      for (int c = 0; c < total; ++c) {
+        const int ip = c & 1, sl = c & (K::kXSlots - 1), sc4 = c & 3;
+        if (!mbar_wait_warp(&s.mma_done[ip], (c >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+        tc_fence_after();
+        const float dj = s.sc[sc4][j][1];
+        // Both 16-lane Yd loads and the x loads are issued before any y store.
+        // x block group G = 2 lh + e (rows p = 32 (q&1) + 16 lh + 8 e + ..) is
+        // read with one transposing 4-matrix load, matrix jj holding tokens
+        // ch + 8 jj + ..: register jj then pairs with the Yd registers
+        // 16 lh + 4 jj + 2 e (+1).  y goes back the same way.
+        const uint32_t xt_a = smem_u32(sm + K::oX + (sl * 2 + j) * K::kTile);
+        uint32_t r[32];
+        uint32_t* r_hi = r + 16;
+        SSD_TMEM_LD_16x256b_X4(tq + K::tYd0 + 64 * ip + ch, r);
+        SSD_TMEM_LD_16x256b_X4(tq + (16u << 16) + K::tYd0 + 64 * ip + ch, r_hi);
+        const uint32_t trow = ch + 8 * (lane >> 3) + (lane & 7);  // the row this thread addresses
+        uint32_t xv[4][4];
+#pragma unroll
+        for (int G = 0; G < 4; ++G)
+          ldmatrix_x4_trans(xt_a + sw128(trow * 128 + (32 * (q & 1) + 8 * G) * 2), xv[G]);
+        SSD_TMEM_WAIT_LD_32(r);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float2 u2 = *reinterpret_cast<const float2*>(&s.u[sc4][j][ch + 8 * jj + 2 * (lane & 3)]);
+#pragma unroll
+          for (int G = 0; G < 4; ++G) {
+            float x0, x1;
+            unpack_bf16x2(xv[G][jj], x0, x1);
+            const uint32_t* rr = r + 16 * (G >> 1) + 4 * jj + 2 * (G & 1);  // (p, t), (p, t+1)
+            xv[G][jj] = pack_bf16x2(fmaf(u2.x, __uint_as_float(rr[0]), dj * x0),
+                                    fmaf(u2.y, __uint_as_float(rr[1]), dj * x1));
           }
-          tc_fence_before();
-          mbar_arrive(&s.acc_free[ip]);  // this thread's reads of Yd of chunk c-1 are done
-          fence_proxy_async_smem();
-          mbar_arrive(&s.y_staged[slp]);
-          mbar_arrive(&s.scan_empty[slp]);
         }
+#pragma unroll
+        for (int G = 0; G < 4; ++G)
+          stmatrix_x4_trans(xt_a + sw128(trow * 128 + (32 * (q & 1) + 8 * G) * 2), xv[G]);
+        tc_fence_before();
+        mbar_arrive(&s.acc_free[ip]);  // this thread's reads of Yd of step c are done
+        fence_proxy_async_smem();
+        mbar_arrive(&s.y_staged[sl]);
+        mbar_arrive(&s.scan_empty[sc4]);
       }
     }
   } else {
-    // ------------------------------------------------ per-head state warps
-    const int j = (warp - 8) >> 2;       // head h0 + j of the current pair
-    const int q = warp & 3;              // TMEM lane quadrant
+    // ------------------------------------------------ state warps
+    // The warp holds rows 32q.. (head q/2) and states n in [32 nq, 32 nq + 32)
+    // of S and H in the layout of the 16x256b TMEM shape: H[16 m2 + 4 jj + 2 hi + e]
+    // is row p = 32 (q&1) + 16 m2 + 8 hi + lane/4, state n = 32 nq + 8 jj +
+    // 2 (lane%4) + e.  Each thread then owns (n, n+1) pairs, so a warp's global
+    // accesses of a state touch 8 rows x 32 contiguous bytes per instruction.
+    const int q = warp & 3;
+    const int j = q >> 1;                // head h0 + j
+    const int nq = (warp - 12) >> 2;
+    const int uw = warp - 12;            // this warp's part of a state hand-over
     const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
-    const int n = 32 * q + lane;         // state row
-    const int uw = warp - 8;             // this warp's part of a state hand-over
-    const int ut = tid - 256 - 128 * j;  // 0..127 within this head's group
-    const int srow = ut >> 1, shalf = ut & 1;
-    // X' = diag(v) x for step cc of this head: each thread scales half a
-    // 128-byte row in place, at the swizzled positions of its 16-byte columns
-    // (the caller has seen scan_full and full_x of step cc; it fences and
-    // arrives on xp_ready)
-    auto scale_tile = [&](int cc) {
-      const int sl = cc & 3;
-      const __nv_bfloat162 w2 = __float2bfloat162_rn(s.v[sl][j][srow]);
-      unsigned char* row = sm + K::oX + (sl * 2 + j) * K::kTile + srow * 128;
+    float H[32];
+    float dprod = 1.f;  // state-only pass: the segment's total decay so far
+    // row p and state n of the pair (H[hk], H[hk + 1]) for m = 2 m2 + hi
+    auto st_row = [&](int m) { return 32 * (q & 1) + 16 * (m >> 1) + 8 * (m & 1) + (lane >> 2); };
+    auto st_col = [&](int jj) { return 32 * nq + 8 * jj + 2 * (lane & 3); };
+    auto st_idx = [&](int m, int jj) { return 16 * (m >> 1) + 4 * jj + 2 * (m & 1); };
+    // the bf16 copy of H for step gg (the state before it) into its TMEM buffer
+    // (column c holds states 2c, 2c+1); the MMAs that read that buffer two
+    // steps earlier are done (every MMA before the last S this warp has seen is)
+    auto publish = [&](int gg) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint4* px = reinterpret_cast<uint4*>(row + (((4 * shalf + k) ^ (srow & 7)) << 4));
-        uint4 vv = *px;
-        __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&vv);
+      for (int m2 = 0; m2 < 2; ++m2) {
+        uint32_t r[8];
 #pragma unroll
-        for (int q2 = 0; q2 < 4; ++q2) e2[q2] = __hmul2(e2[q2], w2);
-        *px = vv;
+        for (int jj = 0; jj < 4; ++jj) {
+          r[2 * jj] = pack_bf16x2(H[16 * m2 + 4 * jj], H[16 * m2 + 4 * jj + 1]);
+          r[2 * jj + 1] = pack_bf16x2(H[16 * m2 + 4 * jj + 2], H[16 * m2 + 4 * jj + 3]);
+        }
+        SSD_TMEM_ST_16x128b_X4(tq + ((uint32_t)(16 * m2) << 16) + K::tH0 + 64 * (gg & 1) + 16 * nq, r);
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&s.h_ready[gg & 1]);
     };
-    auto scale_chunk = [&](int cc) -> bool {
-      const int sl = cc & 3;
-      if (!mbar_wait_warp(&s.scan_full[sl], (cc >> 2) & 1, abort_flag, kWaitLimitNs) ||
-          !mbar_wait_warp(&s.full_x[sl], (cc >> 2) & 1, abort_flag, kWaitLimitNs))
+    // X'^T of step cc, rows 32q.. (p = 32 (q&1) + ..) and tokens
+    // [16 nq, 16 nq + 16), into TMEM in 8 x 8 blocks.  Per half mh (rows
+    // 16 mh.. of the warp's 32) one transposing 4-matrix load reads matrix
+    // k = 2 e + jj: x at tokens 16 nq + 8 jj + .. and p = 32 (q&1) + 16 mh +
+    // 8 e + ..; register k then holds (p, s..s+1), which is scaled by v_s,
+    // v_s+1 and stored with the 16x128b shape (two tokens per column, repeat
+    // jj, lanes + 8 e).  The X'^T buffer of step cc was last read by the MMAs
+    // of step cc - 4, which are done once S of step cc - 2 is.
+    auto scale = [&](int cc) -> bool {
+      const int sl = cc & (K::kXSlots - 1), xb = cc & 3;
+      if (!mbar_wait_warp(&s.scan_full[cc & 3], (cc >> 2) & 1, abort_flag, kWaitLimitNs) ||
+          !mbar_wait_warp(&s.full_x[sl], (cc >> 3) & 1, abort_flag, kWaitLimitNs))
         return false;
-      scale_tile(cc);
-      fence_proxy_async_smem();
-      mbar_arrive(&s.xp_ready[sl]);
+      tc_fence_after();
+      const uint32_t xt_a = smem_u32(sm + K::oX + (sl * 2 + j) * K::kTile);
+      const int k = lane >> 3;  // the matrix this thread addresses a row of
+      const uint32_t srow = 16 * nq + 8 * (k & 1) + (lane & 7);
+      __nv_bfloat162 w2[2];
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const float2 v2 = *reinterpret_cast<const float2*>(&s.v[cc & 3][j][16 * nq + 8 * jj + 2 * (lane & 3)]);
+        w2[jj] = __floats2bfloat162_rn(v2.x, v2.y);
+      }
+#pragma unroll
+      for (int mh = 0; mh < 2; ++mh) {
+        uint32_t xv[4];
+        ldmatrix_x4_trans(xt_a + sw128(srow * 128 + (32 * (q & 1) + 16 * mh + 8 * (k >> 1)) * 2), xv);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const __nv_bfloat162 x2 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&xv[m]), w2[m & 1]);
+          xv[m] = *reinterpret_cast<const uint32_t*>(&x2);
+        }
+        const uint32_t taddr = tq + ((uint32_t)(16 * mh) << 16) + K::tX0 + 32 * xb + 8 * nq;
+        asm volatile("tcgen05.st.sync.aligned.16x128b.x2.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(xv[0]),
+                     "r"(xv[2]), "r"(xv[1]), "r"(xv[3])
+                     : "memory");
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&s.xp_ready[xb]);
+      if (kStateOnly) mbar_arrive(&s.x_empty[sl]);  // no epilogue reads this x tile
       return true;
     };
-    float H[64];
-    float dprod = 1.f;  // state-only pass: the segment's total decay so far
     // state at the start of segment k: h0 (or zero) at a pair's first chunk,
     // otherwise this warp's part of the hand-over the previous CTA wrote, or
     // in split mode h0 carried through the state-only pass's local states of
@@ -600,85 +663,100 @@ __global__ void __launch_bounds__(512, 1)
       const int64_t h = s.seg_h0[k] + j, bb = s.seg_b[k];
       if (kStateOnly) {
 #pragma unroll
-        for (int p = 0; p < 64; ++p) H[p] = 0.f;
+        for (int kk = 0; kk < 32; ++kk) H[kk] = 0.f;
         dprod = 1.f;
         return true;
       }
       if (s.seg_c0[k] == 0 || a.split) {
-        if (a.h0 && n < a.Nr) {
-          const float* src = a.h0 + ((bb * a.H + h) * 64) * a.Nr + n;
+        if (a.h0 && 32 * nq < a.Nr) {  // (16-byte aligned: the library checks it)
+          const float* src = a.h0 + (bb * a.H + h) * 64 * a.Nr;
 #pragma unroll
-          for (int p = 0; p < 64; ++p) H[p] = src[p * a.Nr];
+          for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const float2 v = *reinterpret_cast<const float2*>(src + (int64_t)st_row(m) * a.Nr + st_col(jj));
+              H[st_idx(m, jj)] = v.x;
+              H[st_idx(m, jj) + 1] = v.y;
+            }
         } else {
 #pragma unroll
-          for (int p = 0; p < 64; ++p) H[p] = 0.f;
+          for (int kk = 0; kk < 32; ++kk) H[kk] = 0.f;
         }
         if (s.seg_c0[k] == 0) return true;
         griddep_wait();  // the state-only pass launched before this kernel
         #pragma unroll 1
         for (int ip = s.seg_i0[k]; ip < (int)blockIdx.x; ++ip) {
           const float dd = __ldcg(a.seg_decay + 2 * ip + j);
-          const float4* src =
-              reinterpret_cast<const float4*>(a.handoff + (size_t)ip * kPairHandoffFloats + ((size_t)j * 128 + n) * 64);
+          const float* src = a.handoff + (size_t)ip * kPairHandoffFloats + (size_t)j * 64 * 128;
 #pragma unroll
-          for (int p = 0; p < 16; ++p) {
-            const float4 v = __ldcg(src + p);
-            H[4 * p] = fmaf(dd, H[4 * p], v.x);
-            H[4 * p + 1] = fmaf(dd, H[4 * p + 1], v.y);
-            H[4 * p + 2] = fmaf(dd, H[4 * p + 2], v.z);
-            H[4 * p + 3] = fmaf(dd, H[4 * p + 3], v.w);
-          }
+          for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const float2 v = __ldcg(reinterpret_cast<const float2*>(src + st_row(m) * 128 + st_col(jj)));
+              H[st_idx(m, jj)] = fmaf(dd, H[st_idx(m, jj)], v.x);
+              H[st_idx(m, jj) + 1] = fmaf(dd, H[st_idx(m, jj) + 1], v.y);
+            }
         }
         return true;
       }
       const int slot = (int)blockIdx.x - 1;
       bool ok = true;
-      if (lane == 0) ok = wait_flag_acquire(a.flags + slot * kPairFlagsPerCta + uw, abort_flag, kWaitLimitNs);
+      const int* flag = a.flags + (a.stall ? kPairNeverFlag : slot * kPairFlagsPerCta + uw);
+      if (lane == 0) ok = wait_flag_acquire(flag, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) return false;
-      const float4* src =
-          reinterpret_cast<const float4*>(a.handoff + (size_t)slot * kPairHandoffFloats + ((size_t)j * 128 + n) * 64);
+      const float* src = a.handoff + (size_t)slot * kPairHandoffFloats + (size_t)j * 64 * 128;
 #pragma unroll
-      for (int p = 0; p < 16; ++p) {
-        const float4 v = __ldcg(src + p);
-        H[4 * p] = v.x;
-        H[4 * p + 1] = v.y;
-        H[4 * p + 2] = v.z;
-        H[4 * p + 3] = v.w;
-      }
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(src + st_row(m) * 128 + st_col(jj)));
+          H[st_idx(m, jj)] = v.x;
+          H[st_idx(m, jj) + 1] = v.y;
+        }
       return true;
     };
     // state at the end of segment k: the pair's final state, or the hand-over
     // to the next CTA (data, then this warp's release flag)
     auto seg_end = [&](int k) {
       const int64_t h = s.seg_h0[k] + j, bb = s.seg_b[k];
-      if (kStateOnly) {  // the local end state and the total decay, for the CTAs after this one
-        float4* dst = reinterpret_cast<float4*>(a.handoff + (size_t)blockIdx.x * kPairHandoffFloats +
-                                                ((size_t)j * 128 + n) * 64);
+      float* hand = a.handoff + (size_t)blockIdx.x * kPairHandoffFloats + (size_t)j * 64 * 128;
+      auto put_handoff = [&]() {
 #pragma unroll
-        for (int p = 0; p < 16; ++p) __stcg(dst + p, make_float4(H[4 * p], H[4 * p + 1], H[4 * p + 2], H[4 * p + 3]));
-        if (n == 0) __stcg(a.seg_decay + 2 * blockIdx.x + j, dprod);
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+            __stcg(reinterpret_cast<float2*>(hand + st_row(m) * 128 + st_col(jj)),
+                   make_float2(H[st_idx(m, jj)], H[st_idx(m, jj) + 1]));
+      };
+      if (kStateOnly) {  // the local end state and the total decay, for the CTAs after this one
+        put_handoff();
+        if (lane == 0 && nq == 0 && (q & 1) == 0) __stcg(a.seg_decay + 2 * blockIdx.x + j, dprod);
         return;
       }
       if (s.seg_c0[k] + s.seg_len[k] == nc) {
-        if (a.final_states && n < a.Nr) {
-          float* dst = a.final_states + ((bb * a.H + h) * 64) * a.Nr + n;
+        if (a.final_states && 32 * nq < a.Nr) {  // (16-byte aligned: the library checks it)
+          float* dst = a.final_states + (bb * a.H + h) * 64 * a.Nr;
 #pragma unroll
-          for (int p = 0; p < 64; ++p) dst[(int64_t)p * a.Nr] = H[p];
+          for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+              *reinterpret_cast<float2*>(dst + (int64_t)st_row(m) * a.Nr + st_col(jj)) =
+                  make_float2(H[st_idx(m, jj)], H[st_idx(m, jj) + 1]);
         }
         return;
       }
       if (a.split) return;  // the CTAs after this one start from the state-only pass
-      float4* dst = reinterpret_cast<float4*>(a.handoff + (size_t)blockIdx.x * kPairHandoffFloats +
-                                              ((size_t)j * 128 + n) * 64);
-#pragma unroll
-      for (int p = 0; p < 16; ++p) __stcg(dst + p, make_float4(H[4 * p], H[4 * p + 1], H[4 * p + 2], H[4 * p + 3]));
+      put_handoff();
       __threadfence();
       __syncwarp();
       if (lane == 0) store_flag_release(a.flags + (int)blockIdx.x * kPairFlagsPerCta + uw, 1);
     };
-    // Steps in order: publish e^m H for step g (the state before g), scale the
-    // x tile of step g+1, then fold step g's chunk state into H.
-    bool failed = total > 0 && !scale_chunk(0);
+    // Per step g: wait for S of g, fold it into H (H <- d (H + S)), publish
+    // the bf16 H for step g + 1 unless the segment ends there, then scale the
+    // x tile of step g + 2.
+    bool failed = false;
+    #pragma unroll 1
+    for (int c = 0; c < 2 && c < total && !failed; ++c) failed = !scale(c);
     const int nseg = s.nseg;
     #pragma unroll 1
     for (int k = 0; k < nseg && !failed; ++k) {
@@ -686,83 +764,47 @@ __global__ void __launch_bounds__(512, 1)
         failed = true;
         break;
       }
-      const int g_end = s.seg_g0[k] + s.seg_len[k];
+      const int g0 = s.seg_g0[k], g_end = g0 + s.seg_len[k];
+      if (!kStateOnly) publish(g0);
       #pragma unroll 1
-      for (int g = s.seg_g0[k]; g < g_end; ++g) {
-        const int i = g & 1, n1 = g + 1, s1 = n1 & 3;
-        const bool more = n1 < total;
-        // the barriers this step's publish and the next tile's scaling need,
-        // probed together (their latencies overlap), then waited for if not yet
-        const bool d_ok = kStateOnly || g < 2 || mbar_probe(&s.mma_done[i], ((g - 2) >> 1) & 1);
-        const bool v_ok = !more || mbar_probe(&s.scan_full[s1], (n1 >> 2) & 1);
-        const bool x_ok = !more || mbar_probe(&s.full_x[s1], (n1 >> 2) & 1);
-        if constexpr (!kStateOnly) {
-          if (!__all_sync(0xffffffffu, d_ok) &&
-              !mbar_wait_warp(&s.mma_done[i], ((g - 2) >> 1) & 1, abort_flag, kWaitLimitNs)) {
-            failed = true;
-            break;
-          }
-          {
-            unsigned char* base = sm + K::oH + (i * 2 + j) * K::kHTile + (uint32_t)n * 128;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              uint4 vv;
-              vv.x = pack_bf16x2(H[8 * kk + 0], H[8 * kk + 1]);
-              vv.y = pack_bf16x2(H[8 * kk + 2], H[8 * kk + 3]);
-              vv.z = pack_bf16x2(H[8 * kk + 4], H[8 * kk + 5]);
-              vv.w = pack_bf16x2(H[8 * kk + 6], H[8 * kk + 7]);
-              *reinterpret_cast<uint4*>(base + ((kk ^ (n & 7)) << 4)) = vv;
-            }
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(&s.h_ready[i]);
-        }
-        if (more) {
-          if ((!__all_sync(0xffffffffu, v_ok) &&
-               !mbar_wait_warp(&s.scan_full[s1], (n1 >> 2) & 1, abort_flag, kWaitLimitNs)) ||
-              (!__all_sync(0xffffffffu, x_ok) &&
-               !mbar_wait_warp(&s.full_x[s1], (n1 >> 2) & 1, abort_flag, kWaitLimitNs))) {
-            failed = true;
-            break;
-          }
-          scale_tile(n1);
-          fence_proxy_async_smem();
-          mbar_arrive(&s.xp_ready[s1]);
-        }
-        // ---- state update with step g's chunk state
+      for (int g = g0; g < g_end; ++g) {
+        const int i = g & 1;
         if (!mbar_wait_warp(&s.s_full[i], (g >> 1) & 1, abort_flag, kWaitLimitNs)) {
           failed = true;
           break;
         }
         tc_fence_after();
         {
-          // H <- d (H + S'), two lanes of fp32 per instruction
+          uint32_t r[32];
+          uint32_t* r_hi = r + 16;
+          SSD_TMEM_LD_16x256b_X4(tq + K::tS + 32 * nq, r);
+          SSD_TMEM_LD_16x256b_X4(tq + (16u << 16) + K::tS + 32 * nq, r_hi);
+          SSD_TMEM_WAIT_LD_32(r);
+          tc_fence_before();
+          mbar_arrive(&s.s_free[i]);  // this thread's reads of S of step g are done
+          // H <- d (H + S), two lanes of fp32 per instruction
           const float dd = s.sc[g & 3][j][0];
           const float2 d2 = make_float2(dd, dd);
           if (kStateOnly) dprod *= dd;
 #pragma unroll
-          for (int hlf = 0; hlf < 2; ++hlf) {
-            uint32_t r[32];
-            SSD_TMEM_LD_32x32b_X32(tq + K::tS0 + 128 * i + 64 * j + 32 * hlf, r);
-            SSD_TMEM_WAIT_LD_32(r);
-#pragma unroll
-            for (int kk = 0; kk < 32; kk += 2) {
-              const float2 h2 = __fadd2_rn(make_float2(H[32 * hlf + kk], H[32 * hlf + kk + 1]),
-                                           make_float2(__uint_as_float(r[kk]), __uint_as_float(r[kk + 1])));
-              const float2 o2 = __fmul2_rn(d2, h2);
-              H[32 * hlf + kk] = o2.x;
-              H[32 * hlf + kk + 1] = o2.y;
-            }
+          for (int kk = 0; kk < 32; kk += 2) {
+            const float2 h2 = __fadd2_rn(make_float2(H[kk], H[kk + 1]),
+                                         make_float2(__uint_as_float(r[kk]), __uint_as_float(r[kk + 1])));
+            const float2 o2 = __fmul2_rn(d2, h2);
+            H[kk] = o2.x;
+            H[kk + 1] = o2.y;
           }
         }
-        tc_fence_before();
-        mbar_arrive(&s.acc_free[i]);        // this thread's reads of S of step g are done
-        mbar_arrive(&s.scan_empty[g & 3]);  // and of that step's scalars
+        mbar_arrive(&s.scan_empty[g & 3]);  // this step's scalars are read
+        if (!kStateOnly && g + 1 < g_end) publish(g + 1);
+        if (g + 2 < total && !scale(g + 2)) {
+          failed = true;
+          break;
+        }
       }
       if (!failed) seg_end(k);
     }
   }
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -59,7 +59,7 @@ def call(a):
     ("chunk_size", 8, ssd.SSD_ERR_INVALID_ARG),    # below 16
     ("chunk_size", 512, ssd.SSD_ERR_INVALID_ARG),  # above 256
     ("dtype", 7, ssd.SSD_ERR_INVALID_ARG),
-    ("flags", 4, ssd.SSD_ERR_INVALID_ARG),
+    ("flags", 8, ssd.SSD_ERR_INVALID_ARG),
     ("headdim", 12, ssd.SSD_ERR_UNSUPPORTED),
     ("dstate", 512, ssd.SSD_ERR_UNSUPPORTED),
     ("x", None, ssd.SSD_ERR_INVALID_ARG),
@@ -282,7 +282,9 @@ def test_check_flag_is_accepted_and_unknown_flags_rejected():
     a = base_args()
     a.flags = ssd.SSD_FLAG_CHECK_SEQ
     assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"tcgen05"
-    a.flags = 4
+    a.flags = ssd.SSD_FLAG_TEST_STALL
+    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"tcgen05"
+    a.flags = 8
     assert call(a) == ssd.SSD_ERR_INVALID_ARG
 
 

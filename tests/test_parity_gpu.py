@@ -3,11 +3,10 @@ inputs.  Tolerances (stated by the task's target and written here): relative
 L2 over y <= 1e-5 on the fp32 path and <= 1e-2 on the bf16-input /
 fp32-accumulate path; final states max|diff| <= tol * max(1, max|ref|).
 
-Small cases are compared element by element over the whole output; they span
-several chunks, ragged tails, groups, packed boundaries inside chunks and on
-chunk edges.  Full-size workloads are compared on sampled (batch, head)
-units, which the oracle computes one by one, in the launch configuration the
-benchmark times.
+Every case is compared element by element over the whole output.  The small
+cases span several chunks, ragged tails, groups, packed boundaries inside
+chunks and on chunk edges; the full-size workloads run in the launch
+configuration the benchmark times, with the oracle on every unit.
 """
 import numpy as np
 import pytest
@@ -309,36 +308,27 @@ def test_rejected_call_raises_and_leaves_outputs():
     assert bool((y == 7.0).all())
 
 
-# ---- full-size workloads, sampled units --------------------------------------
-
-def _sample_units(b, H, k, seed):
-    rng = np.random.default_rng(seed)
-    units = set([0, b * H - 1])
-    while len(units) < k:
-        units.add(int(rng.integers(0, b * H)))
-    return sorted(units)
-
+# ---- full-size workloads, every unit -----------------------------------------
 
 FULL = ["c1", "c3", "c4"] + [f"c2_N{n}_Q{q}" for n in (64, 128, 256) for q in (64, 128, 256)]
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_sampled(name):
+def test_full_size(name):
+    """The whole y and every final state of each benchmark workload, in the
+    launch configuration the benchmark times, against the oracle run on every
+    (batch, head) unit.  Besides the stated bound over the whole tensor, each
+    unit's own slice of y is held to it, so that one wrong hand-over or split
+    point between CTAs cannot hide in the average."""
     s = si.CONFIGS[name]
     d = si.make_inputs(s)
     y, f = run_gpu(d, s.chunk_size)
     assert np.isfinite(y).all() and np.isfinite(f).all()
-    H = s.nheads
-    k = 4 if s.seqlen * s.dstate > 2048 * 128 else 6
-    units = _sample_units(s.batch, H, k, seed=len(name))
-    yr, fr = run_oracle(d, units=units)
-    ys = np.stack([y[u // H, :, u % H] for u in units])
-    yrs = np.stack([yr[u // H, :, u % H] for u in units])
-    assert rel_l2(ys, yrs) <= 1e-2, rel_l2(ys, yrs)
-    if d["seq_idx"] is None:
-        fs = np.stack([f[u // H, u % H] for u in units])
-        frs = np.stack([fr[u // H, u % H] for u in units])
-    else:
-        heads = sorted({u % H for u in units})
-        fs, frs = f[:, heads], fr[:, heads]
-    assert state_err(fs, frs) <= 1e-2, state_err(fs, frs)
+    yr, fr = run_oracle(d)
+    assert rel_l2(y, yr) <= 1e-2, rel_l2(y, yr)
+    assert state_err(f, fr) <= 1e-2, state_err(f, fr)
+    err = y - yr
+    num = np.sqrt((err * err).sum(axis=(1, 3)))    # (b, H): per unit
+    den = np.sqrt((yr * yr).sum(axis=(1, 3)))
+    worst = float((num / np.maximum(den, 1e-300)).max())
+    assert worst <= 1e-2, worst
