@@ -316,18 +316,28 @@ __global__ void __launch_bounds__(896, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     // The whole warp walks the loop and forms the descriptors (warp-uniform
-    // values); one elected lane issues the MMAs and commits.
+    // values); one elected lane issues the MMAs and commits.  A step's
+    // barriers are probed together with non-blocking tests, whose latencies
+    // overlap, and only one not yet complete is then waited for.
+    auto need = [&](bool done, uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, done) || mbar_wait_warp(bar, parity, abort_flag, kWaitLimitNs);
+    };
     const uint32_t aW = smem_u32(sm + K::oW), aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB);
     constexpr uint32_t id_y = idesc_bf16(128, 64, 0, 0);   // A in TMEM, B K-major
     constexpr uint32_t id_s = idesc_bf16(128, 128, 0, 1);  // A in TMEM, B MN-major
     #pragma unroll 1
     for (int c = 0; c < total; ++c) {
       const int i = c & 1, xb = c & 3;
-      const uint32_t ph = (c >> 1) & 1;
-      bool ok = mbar_wait_warp(&s.full_wb[i], ph, abort_flag, kWaitLimitNs);
-      ok = ok && mbar_wait_warp(&s.xp_ready[xb], (c >> 2) & 1, abort_flag, kWaitLimitNs);
-      if (!kStateOnly && c >= 2) ok = ok && mbar_wait_warp(&s.acc_free[i], ((c - 2) >> 1) & 1, abort_flag, kWaitLimitNs);
-      if (!ok) break;
+      const uint32_t ph = (c >> 1) & 1, pxp = (c >> 2) & 1, pacc = ((c - 2) >> 1) & 1, psf = ((c - 1) >> 1) & 1;
+      const bool acc = !kStateOnly && c >= 2, sfree = c >= 1;
+      const bool p_wb = mbar_probe(&s.full_wb[i], ph);
+      const bool p_xp = mbar_probe(&s.xp_ready[xb], pxp);
+      const bool p_acc = !acc || mbar_probe(&s.acc_free[i], pacc);
+      const bool p_sf = !sfree || mbar_probe(&s.s_free[(c - 1) & 1], psf);
+      const bool p_c = kStateOnly || mbar_probe(&s.full_c[i], ph);
+      if (!need(p_wb, &s.full_wb[i], ph) || !need(p_xp, &s.xp_ready[xb], pxp) ||
+          (acc && !need(p_acc, &s.acc_free[i], pacc)))
+        break;
       tc_fence_after();
       const uint32_t yd = tmem + K::tYd0 + 64 * i;
       const uint32_t ax = tmem + K::tX0 + 32 * xb;  // X'^T of both heads, this chunk
@@ -343,7 +353,7 @@ __global__ void __launch_bounds__(896, 1)
       }
       // S = X'^T B   (N = 128 states, K = 64 tokens s; a K step is 16 rows), once
       // the state warps have read out the previous chunk's S
-      if (c >= 1 && !mbar_wait_warp(&s.s_free[(c - 1) & 1], ((c - 1) >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+      if (sfree && !need(p_sf, &s.s_free[(c - 1) & 1], psf)) break;
       tc_fence_after();
       if (elect_one()) {
 #pragma unroll
@@ -353,9 +363,8 @@ __global__ void __launch_bounds__(896, 1)
       __syncwarp();
       if (kStateOnly) continue;
       // Yd^T += H C^T   (K = N states)
-      ok = mbar_wait_warp(&s.h_ready[i], ph, abort_flag, kWaitLimitNs);
-      ok = ok && mbar_wait_warp(&s.full_c[i], ph, abort_flag, kWaitLimitNs);
-      if (!ok) break;
+      const bool p_h = mbar_probe(&s.h_ready[i], ph);
+      if (!need(p_h, &s.h_ready[i], ph) || !need(p_c, &s.full_c[i], ph)) break;
       tc_fence_after();
       const uint64_t dc = sw128_desc(aC + i * K::NB * K::kTile, 16, 1024);
       if (elect_one()) {
@@ -621,8 +630,11 @@ __global__ void __launch_bounds__(896, 1)
     // of step cc - 4, which are done once S of step cc - 2 is.
     auto scale = [&](int cc) -> bool {
       const int sl = cc & (K::kXSlots - 1), xb = cc & 3;
-      if (!mbar_wait_warp(&s.scan_full[cc & 3], (cc >> 2) & 1, abort_flag, kWaitLimitNs) ||
-          !mbar_wait_warp(&s.full_x[sl], (cc >> 3) & 1, abort_flag, kWaitLimitNs))
+      const bool p_v = mbar_probe(&s.scan_full[cc & 3], (cc >> 2) & 1);
+      const bool p_x = mbar_probe(&s.full_x[sl], (cc >> 3) & 1);
+      if ((!__all_sync(0xffffffffu, p_v) &&
+           !mbar_wait_warp(&s.scan_full[cc & 3], (cc >> 2) & 1, abort_flag, kWaitLimitNs)) ||
+          (!__all_sync(0xffffffffu, p_x) && !mbar_wait_warp(&s.full_x[sl], (cc >> 3) & 1, abort_flag, kWaitLimitNs)))
         return false;
       tc_fence_after();
       const uint32_t xt_a = smem_u32(sm + K::oX + (sl * 2 + j) * K::kTile);
@@ -716,7 +728,17 @@ __global__ void __launch_bounds__(896, 1)
       return true;
     };
     // state at the end of segment k: the pair's final state, or the hand-over
-    // to the next CTA (data, then this warp's release flag)
+    // to the next CTA: the data now, this warp's release flag (after a fence)
+    // a few steps later, when the stores have long reached L2 and the fence
+    // no longer waits for them.  The next CTA reads the hand-over only at the
+    // end of its own range.
+    int release_at = -1;  // step after which the pending hand-over flag is released
+    auto release = [&]() {
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) store_flag_release(a.flags + (int)blockIdx.x * kPairFlagsPerCta + uw, 1);
+      release_at = -1;
+    };
     auto seg_end = [&](int k) {
       const int64_t h = s.seg_h0[k] + j, bb = s.seg_b[k];
       float* hand = a.handoff + (size_t)blockIdx.x * kPairHandoffFloats + (size_t)j * 64 * 128;
@@ -747,9 +769,7 @@ __global__ void __launch_bounds__(896, 1)
       }
       if (a.split) return;  // the CTAs after this one start from the state-only pass
       put_handoff();
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) store_flag_release(a.flags + (int)blockIdx.x * kPairFlagsPerCta + uw, 1);
+      release_at = s.seg_g0[k] + s.seg_len[k] + 2;
     };
     // Per step g: wait for S of g, fold it into H (H <- d (H + S)), publish
     // the bf16 H for step g + 1 unless the segment ends there, then scale the
@@ -801,9 +821,11 @@ __global__ void __launch_bounds__(896, 1)
           failed = true;
           break;
         }
+        if (g == release_at) release();
       }
       if (!failed) seg_end(k);
     }
+    if (release_at >= 0 && !failed) release();
   }
   tc_fence_before();
   __syncthreads();
