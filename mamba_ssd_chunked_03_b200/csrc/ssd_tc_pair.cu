@@ -92,7 +92,10 @@ struct PairCfg {
 constexpr int kPairMaxSeg = 32;  // segments (pairs touched) per CTA, at most
 
 // Ring barriers are indexed like the buffers they guard, so no barrier can
-// complete a second phase before every waiter has seen the first.
+// complete a second phase before every waiter has seen the first.  A warp
+// arrives once (lane 0, after each lane's own wait or fence and a __syncwarp,
+// which orders the warp's accesses before that release), so the counts below
+// are in warps: 32 times fewer shared-memory atomics than per-thread arrivals.
 struct __align__(16) PairSmem {
   uint64_t full_x[8], x_empty[8];        // x ring: TMA landed / scaled (state-only pass)
   uint64_t full_dt[8];                   // dt ring (the scan warp's own)
@@ -165,24 +168,24 @@ __global__ void __launch_bounds__(896, 1)
     for (int i = 0; i < 8; ++i) {
       mbar_init(&s.full_x[i], 1);
       // the state-only pass stores no y: the x scalers (state warps) free the slot
-      mbar_init(&s.x_empty[i], 512);
-      mbar_init(&s.y_staged[i], 256);
+      mbar_init(&s.x_empty[i], 16);
+      mbar_init(&s.y_staged[i], 8);
       mbar_init(&s.full_dt[i], 1);
     }
     for (int i = 0; i < 4; ++i) {
-      mbar_init(&s.scan_full[i], 32);
+      mbar_init(&s.scan_full[i], 1);
       // the state warps, and in the fused pass the epilogue warps
-      mbar_init(&s.scan_empty[i], kStateOnly ? 512 : 256 + 512);
-      mbar_init(&s.xp_ready[i], 512);
+      mbar_init(&s.scan_empty[i], kStateOnly ? 16 : 8 + 16);
+      mbar_init(&s.xp_ready[i], 16);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.full_wb[i], 1);
       mbar_init(&s.full_c[i], 1);
       mbar_init(&s.s_full[i], 1);
-      mbar_init(&s.s_free[i], 512);
+      mbar_init(&s.s_free[i], 16);
       mbar_init(&s.mma_done[i], 1);
-      mbar_init(&s.h_ready[i], 512);
-      mbar_init(&s.acc_free[i], 256);
+      mbar_init(&s.h_ready[i], 16);
+      mbar_init(&s.acc_free[i], 8);
     }
     mbar_init(&s.drain, 1);
     s.abort_flag = *reinterpret_cast<volatile int*>(a.err) != 0;
@@ -322,7 +325,11 @@ __global__ void __launch_bounds__(896, 1)
     auto need = [&](bool done, uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, done) || mbar_wait_warp(bar, parity, abort_flag, kWaitLimitNs);
     };
-    const uint32_t aW = smem_u32(sm + K::oW), aC = smem_u32(sm + K::oC), aB = smem_u32(sm + K::oB);
+    // descriptors of buffer 0; buffer 1 lies a whole number of 8 KB tiles further
+    const uint64_t dw0 = sw128_desc(smem_u32(sm + K::oW), 16, 1024);
+    const uint64_t db0 = sw128_desc(smem_u32(sm + K::oB), K::kTile, 1024);
+    const uint64_t dc0 = sw128_desc(smem_u32(sm + K::oC), 16, 1024);
+    constexpr uint32_t kTileDesc = K::kTile >> 4;  // an 8 KB tile in descriptor address units
     constexpr uint32_t id_y = idesc_bf16(128, 64, 0, 0);   // A in TMEM, B K-major
     constexpr uint32_t id_s = idesc_bf16(128, 128, 0, 1);  // A in TMEM, B MN-major
     #pragma unroll 1
@@ -341,8 +348,8 @@ __global__ void __launch_bounds__(896, 1)
       tc_fence_after();
       const uint32_t yd = tmem + K::tYd0 + 64 * i;
       const uint32_t ax = tmem + K::tX0 + 32 * xb;  // X'^T of both heads, this chunk
-      const uint64_t dw = sw128_desc(aW + i * K::kTile, 16, 1024);
-      const uint64_t db = sw128_desc(aB + i * K::NB * K::kTile, K::kTile, 1024);
+      const uint64_t dw = dw0 + i * kTileDesc;
+      const uint64_t db = db0 + i * K::NB * kTileDesc;
       if (!kStateOnly) {
         // Yd^T = X'^T W'^T   (K = 64 tokens s; a K step is 32 bytes along the row)
         if (elect_one()) {
@@ -366,7 +373,7 @@ __global__ void __launch_bounds__(896, 1)
       const bool p_h = mbar_probe(&s.h_ready[i], ph);
       if (!need(p_h, &s.h_ready[i], ph) || !need(p_c, &s.full_c[i], ph)) break;
       tc_fence_after();
-      const uint64_t dc = sw128_desc(aC + i * K::NB * K::kTile, 16, 1024);
+      const uint64_t dc = dc0 + i * K::NB * kTileDesc;
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < NS / 16; ++kk)
@@ -464,7 +471,8 @@ __global__ void __launch_bounds__(896, 1)
         s.sc[slot][j][0] = exp2f(cse);
         s.sc[slot][j][1] = dsk;
       }
-      mbar_arrive(&s.scan_full[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.scan_full[slot]);
     }
     if (lane == 0 && *abort_flag)  // let the dt copies in flight land
       #pragma unroll 1
@@ -562,26 +570,31 @@ __global__ void __launch_bounds__(896, 1)
         for (int G = 0; G < 4; ++G)
           ldmatrix_x4_trans(xt_a + sw128(trow * 128 + (32 * (q & 1) + 8 * G) * 2), xv[G]);
         SSD_TMEM_WAIT_LD_32(r);
+        const float2 dj2 = make_float2(dj, dj);
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           const float2 u2 = *reinterpret_cast<const float2*>(&s.u[sc4][j][ch + 8 * jj + 2 * (lane & 3)]);
 #pragma unroll
           for (int G = 0; G < 4; ++G) {
-            float x0, x1;
-            unpack_bf16x2(xv[G][jj], x0, x1);
-            const uint32_t* rr = r + 16 * (G >> 1) + 4 * jj + 2 * (G & 1);  // (p, t), (p, t+1)
-            xv[G][jj] = pack_bf16x2(fmaf(u2.x, __uint_as_float(rr[0]), dj * x0),
-                                    fmaf(u2.y, __uint_as_float(rr[1]), dj * x1));
+            // y = u_t Yd + D x_t for the pair (p, t), (p, t+1), two lanes of fp32 per instruction
+            const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xv[G][jj]));
+            const uint32_t* rr = r + 16 * (G >> 1) + 4 * jj + 2 * (G & 1);
+            const float2 o2 =
+                __ffma2_rn(u2, make_float2(__uint_as_float(rr[0]), __uint_as_float(rr[1])), __fmul2_rn(dj2, x2));
+            xv[G][jj] = pack_bf16x2(o2.x, o2.y);
           }
         }
 #pragma unroll
         for (int G = 0; G < 4; ++G)
           stmatrix_x4_trans(xt_a + sw128(trow * 128 + (32 * (q & 1) + 8 * G) * 2), xv[G]);
-        tc_fence_before();
-        mbar_arrive(&s.acc_free[ip]);  // this thread's reads of Yd of step c are done
-        fence_proxy_async_smem();
-        mbar_arrive(&s.y_staged[sl]);
-        mbar_arrive(&s.scan_empty[sc4]);
+        tc_fence_before();         // this thread's reads of Yd of step c are done
+        fence_proxy_async_smem();  // its y stores are visible to the bulk store
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&s.acc_free[ip]);
+          mbar_arrive(&s.y_staged[sl]);
+          mbar_arrive(&s.scan_empty[sc4]);
+        }
       }
     }
   } else {
@@ -618,7 +631,8 @@ __global__ void __launch_bounds__(896, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&s.h_ready[gg & 1]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.h_ready[gg & 1]);
     };
     // X'^T of step cc, rows 32q.. (p = 32 (q&1) + ..) and tokens
     // [16 nq, 16 nq + 16), into TMEM in 8 x 8 blocks.  Per half mh (rows
@@ -662,8 +676,11 @@ __global__ void __launch_bounds__(896, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&s.xp_ready[xb]);
-      if (kStateOnly) mbar_arrive(&s.x_empty[sl]);  // no epilogue reads this x tile
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s.xp_ready[xb]);
+        if (kStateOnly) mbar_arrive(&s.x_empty[sl]);  // no epilogue reads this x tile
+      }
       return true;
     };
     // state at the start of segment k: h0 (or zero) at a pair's first chunk,
@@ -800,8 +817,9 @@ __global__ void __launch_bounds__(896, 1)
           SSD_TMEM_LD_16x256b_X4(tq + K::tS + 32 * nq, r);
           SSD_TMEM_LD_16x256b_X4(tq + (16u << 16) + K::tS + 32 * nq, r_hi);
           SSD_TMEM_WAIT_LD_32(r);
-          tc_fence_before();
-          mbar_arrive(&s.s_free[i]);  // this thread's reads of S of step g are done
+          tc_fence_before();  // this thread's reads of S of step g are done
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.s_free[i]);
           // H <- d (H + S), two lanes of fp32 per instruction
           const float dd = s.sc[g & 3][j][0];
           const float2 d2 = make_float2(dd, dd);
@@ -815,7 +833,8 @@ __global__ void __launch_bounds__(896, 1)
             H[kk + 1] = o2.y;
           }
         }
-        mbar_arrive(&s.scan_empty[g & 3]);  // this step's scalars are read
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.scan_empty[g & 3]);  // this step's scalars are read
         if (!kStateOnly && g + 1 < g_end) publish(g + 1);
         if (g + 2 < total && !scale(g + 2)) {
           failed = true;
