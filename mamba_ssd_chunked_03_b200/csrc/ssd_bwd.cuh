@@ -147,23 +147,33 @@ __device__ __forceinline__ ChunkPos chunk_pos(const Dims& d, int64_t bid) {
 // first token of t's packed sequence, or -1 while that sequence began before
 // the chunk (those tokens see h_in).  A token whose id differs from the
 // previous token's starts a sequence: its own decay is not applied (a_t = 0),
-// so the sum restarts at 0 there.  One thread runs this.
-__device__ __forceinline__ void chunk_cumsum(const KArgs& a, const ChunkPos& q, float* cs, int* seg) {
+// so the sum restarts at 0 there.  Every thread of the block calls it: the
+// log-decays and the sequence starts are loaded in parallel into cs and seg,
+// then one thread runs the scan over shared memory.  It ends with a barrier.
+__device__ __forceinline__ void chunk_cumsum(const KArgs& a, const ChunkPos& q, float* cs, int* seg, int tid) {
   const float Ah = a.A[q.h];
   const int32_t* sq = a.seq ? a.seq + q.b * a.d.L : nullptr;
-  float acc = 0.f;
-  int s0 = -1;
-  for (int t = 0; t < q.Qc; ++t) {
+  for (int t = tid; t < q.Qc; t += kThreads) {
     const int64_t l = q.t0 + t;
-    if (sq && l > 0 && sq[l] != sq[l - 1]) {
-      s0 = t;
-      acc = 0.f;
-    } else {
-      acc += a.dt[(q.b * a.d.L + l) * a.d.H + q.h] * Ah;
-    }
-    cs[t] = acc;
-    seg[t] = s0;
+    cs[t] = a.dt[(q.b * a.d.L + l) * a.d.H + q.h] * Ah;
+    seg[t] = sq && l > 0 && sq[l] != sq[l - 1];  // a sequence starts at t
   }
+  __syncthreads();
+  if (tid == 0) {
+    float acc = 0.f;
+    int s0 = -1;
+    for (int t = 0; t < q.Qc; ++t) {
+      if (seg[t]) {
+        s0 = t;
+        acc = 0.f;
+      } else {
+        acc += cs[t];
+      }
+      cs[t] = acc;
+      seg[t] = s0;
+    }
+  }
+  __syncthreads();
 }
 
 // ---- register-tiled products of small matrices in shared memory
@@ -318,8 +328,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_bwd_chunk_states(const KArgs a)
     Bs[i] = ld(B, gi);
     Cs[i] = ld(C, gi);
   }
-  if (tid == 0) chunk_cumsum(a, q, cs, seg);
-  __syncthreads();
+  chunk_cumsum(a, q, cs, seg, tid);
   for (int t = tid; t < Qc; t += kThreads) {
     const float w = a.dt[(q.b * d.L + q.t0 + t) * d.H + q.h];
     cS[t] = seg[t] == seg[Qc - 1] ? w * expf(cs[Qc - 1] - cs[t]) : 0.f;
@@ -365,42 +374,33 @@ __global__ void __launch_bounds__(kThreads) k_bwd_state_passing(const KArgs a) {
   float* S = a.S + bh * d.nc * PN + e;
   float* T = a.T + bh * d.nc * PN + e;
   const float* dec = a.dec + bh * d.nc;
-  // Four chunks' values are loaded before any of them is overwritten, so that
-  // four loads are in flight at a time (the addresses differ, which the
-  // compiler cannot see).
+  // The two scans run side by side, kBatch chunks at a time: a batch of S
+  // (walking forward) and one of T (walking back) are loaded before either is
+  // overwritten, so that 2 kBatch loads are in flight per thread (the
+  // addresses differ, which the compiler cannot see).  The scans are each
+  // thread's own, so a batch is a plain reordering of the loads.
+  constexpr int kBatch = 16;
   float run = a.h0 ? a.h0[i] : 0.f;
-  int64_t c = 0;
-  for (; c + 4 <= d.nc; c += 4) {
-    float v[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = S[(c + j) * PN];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      S[(c + j) * PN] = run;
-      run = fmaf(dec[c + j], run, v[j]);
-    }
-  }
-  for (; c < d.nc; ++c) {
-    const float v = S[c * PN];
-    S[c * PN] = run;
-    run = fmaf(dec[c], run, v);
-  }
   float lam = a.dfinal ? a.dfinal[i] : 0.f;
-  c = d.nc - 1;
-  for (; c - 3 >= 0; c -= 4) {
-    float v[4];
+  const int64_t nc = d.nc;
+  for (int64_t c = 0; c < nc; c += kBatch) {
+    const int n = (int)(nc - c < kBatch ? nc - c : kBatch);
+    const int64_t cb = nc - 1 - c;  // the backward scan's chunk for j = 0
+    float vs[kBatch], vt[kBatch];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = T[(c - j) * PN];
+    for (int j = 0; j < kBatch; ++j)
+      if (j < n) {
+        vs[j] = S[(c + j) * PN];
+        vt[j] = T[(cb - j) * PN];
+      }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      T[(c - j) * PN] = lam;
-      lam = fmaf(dec[c - j], lam, v[j]);
-    }
-  }
-  for (; c >= 0; --c) {
-    const float v = T[c * PN];
-    T[c * PN] = lam;
-    lam = fmaf(dec[c], lam, v);
+    for (int j = 0; j < kBatch; ++j)
+      if (j < n) {
+        S[(c + j) * PN] = run;
+        run = fmaf(dec[c + j], run, vs[j]);
+        T[(cb - j) * PN] = lam;
+        lam = fmaf(dec[cb - j], lam, vt[j]);
+      }
   }
   if (a.dh0) a.dh0[i] = lam;
 }
@@ -480,8 +480,12 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
     red[tid] = part_lh;
   }
   for (int t = tid; t < Qc; t += kThreads) w[t] = a.dt[(q.b * d.L + q.t0 + t) * d.H + q.h];
-  if (tid == 0) chunk_cumsum(a, q, cs, seg);
-  __syncthreads();
+  chunk_cumsum(a, q, cs, seg, tid);
+  // <Lam, h_in>: the threads' shares summed pairwise (red[0] holds it)
+  for (int off = kThreads / 2; off > 0; off >>= 1) {
+    if (tid < off) red[tid] += red[tid + off];
+    __syncthreads();
+  }
 
   const int last = Qc - 1;
   // K = E o (C B^T) on the chunk's Q x Q triangle (C B^T from k_bwd_chunk_cb, once
@@ -670,8 +674,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
     // dl_k = S_k + sum_{t >= k} (h_in term)_t + sum_{s < k} N_s + e_last <Lam, h_in>;
     // the h_in terms live in the first sequence only and N in the last, so
     // none of the sums crosses a boundary that matters
-    float lh = 0.f;
-    for (int i = 0; i < kThreads; ++i) lh += red[i];
+    const float lh = red[0];
     const float e_last = seg[last] == -1 ? expf(cs[last]) : 0.f;
     float before = 0.f;  // sum_{s < k} N_s, kept in nn as an exclusive prefix
     for (int k = 0; k <= last; ++k) {
