@@ -386,6 +386,17 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
         "=r"(r[15])                                                                                         \
       : "r"(taddr))
 
+// 16 lanes x 32 bit, twice, 16 columns per half: threads 0-15 write lanes
+// base..base+15 at columns [c, c+16), threads 16-31 the same lanes at
+// columns [c+32, c+48) (the store form of SSD_TMEM_LD_16x32bx2_X16_HALF32).
+#define SSD_TMEM_ST_16x32bx2_X16_HALF32(taddr, r)                                                          \
+  asm volatile(                                                                                              \
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 32, {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+      "%15,%16};" ::"r"(taddr),                                                                              \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),       \
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])                      \
+      : "memory")
+
 // 32 lanes x 32 bit, 32 consecutive columns: thread i writes lane base + i.
 #define SSD_TMEM_ST_32x32b_X32(taddr, r)                                                                     \
   asm volatile(                                                                                              \

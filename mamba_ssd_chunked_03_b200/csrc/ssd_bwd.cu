@@ -1,10 +1,11 @@
-// ssd_bwd and ssd_bwd_workspace_size: the backward kernels of ssd_bwd.cuh,
-// launched on the caller's stream.
+// ssd_bwd and ssd_bwd_workspace_size: the backward kernels of ssd_bwd.cuh and
+// ssd_bwd_tc.cuh, launched on the caller's stream.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "ssd.h"
 #include "ssd_bwd.cuh"
+#include "ssd_bwd_tc.cuh"
 
 namespace {
 
@@ -19,6 +20,8 @@ struct CudaLaunch {
     return cudaGetLastError() == cudaSuccess;
   }
   bool record(void* event) const { return cudaEventRecord(static_cast<cudaEvent_t>(event), stream) == cudaSuccess; }
+  bool chunk_tc_ok(const ssd::bwd::KArgs& k) const { return ssd::bwd::chunk_tc_supported(k); }
+  bool chunk_tc(const ssd::bwd::KArgs& k) const { return ssd::bwd::chunk_tc_launch(k, stream) == cudaSuccess; }
 };
 
 }  // namespace

@@ -51,6 +51,9 @@
 //                        tokens, h_in and Lam; dB and dC per head
 //   k_bwd_group_sum      dB, dC summed over each group's heads
 //   k_bwd_param_sum      dA, dD summed over rows and chunks (fp64)
+//   (k_bwd_chunk_cb and k_bwd_chunk give way to k_bwd_chunk_tc of
+//   ssd_bwd_tc.cuh, the same formulas on the tensor cores, where that kernel
+//   takes the call)
 //
 // With SSD_BWD_DINITIAL_ONLY only the first two run.
 //
@@ -64,6 +67,9 @@
 
 #include <stddef.h>
 #include <stdint.h>
+
+#include <type_traits>
+#include <utility>
 
 #include "ssd.h"
 
@@ -850,6 +856,15 @@ inline KArgs make_kargs(const ssd_bwd_args* a, const Plan& pl) {
 
 inline unsigned blocks_for(int64_t n) { return (unsigned)((n + kThreads - 1) / kThreads); }
 
+// A launcher may offer the tensor-core chunk kernel (ssd_bwd_tc.cuh, GPU
+// builds): chunk_tc_ok(k) says whether it takes the call, chunk_tc(k) runs it.
+// The host emulation of the kernels offers none and runs the CUDA-core ones.
+template <class L, class = void>
+struct has_chunk_tc : std::false_type {};
+template <class L>
+struct has_chunk_tc<L, std::void_t<decltype(std::declval<L&>().chunk_tc(std::declval<const KArgs&>()))>>
+    : std::true_type {};
+
 // Validate, then enqueue the six kernels through `launch(kernel, grid,
 // shared bytes, args)`, which returns false when a launch fails;
 // `launch.record(event)` records a caller's timing event (false on failure).
@@ -863,10 +878,19 @@ ssd_status enqueue_typed(const KArgs& k, const Plan& pl, void* const events[2], 
     if (events[0] && !(launch.record(events[0]) && launch.record(events[1]))) return SSD_ERR_CUDA;
     return SSD_OK;
   }
-  if (!launch(&k_bwd_chunk_cb<T>, (unsigned)(d.b * d.nc * d.G), pl.smem_cb, k)) return SSD_ERR_CUDA;
-  if (events[0] && !launch.record(events[0])) return SSD_ERR_CUDA;
-  if (!launch(&k_bwd_chunk<T>, chunk_ctas, pl.smem_chunk, k)) return SSD_ERR_CUDA;
-  if (events[1] && !launch.record(events[1])) return SSD_ERR_CUDA;
+  bool tensor_cores = false;
+  if constexpr (has_chunk_tc<Launch>::value && std::is_same<T, __nv_bfloat16>::value) tensor_cores = launch.chunk_tc_ok(k);
+  if (tensor_cores) {  // C B^T is formed inside the kernel
+    if (events[0] && !launch.record(events[0])) return SSD_ERR_CUDA;
+    if constexpr (has_chunk_tc<Launch>::value)
+      if (!launch.chunk_tc(k)) return SSD_ERR_CUDA;
+    if (events[1] && !launch.record(events[1])) return SSD_ERR_CUDA;
+  } else {
+    if (!launch(&k_bwd_chunk_cb<T>, (unsigned)(d.b * d.nc * d.G), pl.smem_cb, k)) return SSD_ERR_CUDA;
+    if (events[0] && !launch.record(events[0])) return SSD_ERR_CUDA;
+    if (!launch(&k_bwd_chunk<T>, chunk_ctas, pl.smem_chunk, k)) return SSD_ERR_CUDA;
+    if (events[1] && !launch.record(events[1])) return SSD_ERR_CUDA;
+  }
   if (!launch(&k_bwd_group_sum, blocks_for(d.b * d.L * d.G * d.N), (size_t)0, k)) return SSD_ERR_CUDA;
   if (!launch(&k_bwd_param_sum, blocks_for(d.H), (size_t)0, k)) return SSD_ERR_CUDA;
   return SSD_OK;

@@ -1,0 +1,562 @@
+// The backward's per-chunk gradients on the tensor cores (tcgen05 MMAs with
+// fp32 accumulators in tensor memory): the formulas of k_bwd_chunk in
+// ssd_bwd.cuh, with every contraction an MMA.  One CTA per (batch row, chunk,
+// head), for headdim 64, dstate 128, 64-token chunks, bf16 inputs and no gate;
+// other calls take the CUDA-core kernels.
+//
+// Per chunk (E(t,s) = exp(cs_t - cs_s) inside one packed sequence, w = dt,
+// e_t, el_s = E(last, s), h_in the state entering the chunk, Lam the
+// gradient with respect to the state leaving it):
+//
+//   CB = C B^T,  G = dy x^T                              (bf16 operands as loaded)
+//   K = E o CB,  Z = E o G,  Zw = Z diag(w),  M = K o G   (CUDA cores)
+//   dx = diag(w) [K^T dy + diag(el) B Lam^T] + D dy
+//   dB = diag(w) [Z^T C + diag(el) x Lam]
+//   dC = Zw B + diag(e) dy h_in
+//
+// and the decay gradients from row sums of M and of the products, as in
+// ssd_bwd.cuh.  The fp32 operands (K, Z, Zw, Lam, h_in) enter the MMAs as
+// three bf16 terms, v = hi + mid + lo with hi = bf16(v), mid = bf16(v - hi),
+// lo = bf16(v - hi - mid): the terms miss v by at most 2^-24 |v|, and each
+// product of a term with a bf16 input is exact in fp32, so the contractions
+// keep fp32 accuracy.
+//
+// A row-scaled term shares its accumulator with the unscaled one: the product
+// with Lam is formed first, read out, scaled by el_s and written back, and
+// the other product accumulates on top of it.  Tensor memory (the M = 64
+// layout: row m at lane 32 (m / 16) + m % 16), 448 of 512 columns:
+//   [0, 64)    dx        [64, 192)  dB
+//   [192, 256) CB, then with [256, 320) (G) the product dy h_in
+//   [320, 448) Zw B
+// Shared memory holds x, dy, B and C as the TMA loads them (bf16, 128-byte
+// rows, 128-byte swizzle), the three-term split tiles written by the threads
+// in the same layout, and M in fp32 for the decay sums.  Every wait is
+// bounded (1 s); a CTA whose wait gives up lets its copies and MMAs finish,
+// frees its tensor memory and exits without writing gradients.
+//
+// Included by ssd_bwd.cu only (after ssd_bwd.cuh): the host emulation of the
+// CUDA-core kernels includes ssd_bwd.cuh alone.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "sm100.cuh"
+#include "ssd_bwd.cuh"
+#include "ssd_internal.h"
+#include "ssd_tc_common.cuh"
+
+namespace ssd {
+namespace bwd {
+namespace {
+
+using namespace sm100;
+
+struct TcCfg {
+  static constexpr int Q = 64;
+  static constexpr uint32_t kTile = 8192;          // 64 rows x 128 bytes
+  static constexpr uint32_t oX = 0;                 // x  [s][p]
+  static constexpr uint32_t oDY = oX + kTile;       // dy [t][p]
+  static constexpr uint32_t oB = oDY + kTile;       // B  [s][n], n-blocks 0-63, 64-127
+  static constexpr uint32_t oC = oB + 2 * kTile;    // C  [t][n]
+  static constexpr uint32_t oK = oC + 2 * kTile;    // K  terms [3][t][s]
+  static constexpr uint32_t oZ = oK + 3 * kTile;    // Z  terms [3][t][s]
+  static constexpr uint32_t oZw = oZ + 3 * kTile;   // Zw terms [3][t][s]
+  static constexpr uint32_t oS = oZw + 3 * kTile;   // Lam, then h_in: terms [3][n-block][p][n]
+  static constexpr uint32_t oM = oS + 6 * kTile;    // M fp32 [t][s], rows of kMs
+  static constexpr int kMs = Q + 1;
+  static constexpr uint32_t oEnd = oM + Q * kMs * 4;
+  static constexpr uint32_t kSmemBytes = oEnd + 1024;
+  // tensor memory columns
+  static constexpr uint32_t tDx = 0, tDB = 64, tCB = 192, tG = 256, tDC2 = 192, tDC1 = 320, kTmemCols = 512;
+};
+
+struct __align__(16) TcSmem {
+  uint64_t bar_in, bar_p1, bar_p2, bar_drain;
+  uint32_t tmem_base;
+  int abort_flag, never;
+  float cs[64], w[64], el[64], ein[64], dg[64], nv[64], dw[64], dcs[64], nn[64];
+  float nxp[64][4], cyp[64][4];  // row sums, four shares a row
+  float pair[64][8];             // the decay pair sums, in quarters
+  float red[kThreads];
+  int seg[64];
+};
+
+// v = hi + mid + lo, each rounded to bf16 (see the file comment)
+__device__ __forceinline__ void split3(float v, __nv_bfloat16& hi, __nv_bfloat16& mid, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(hi);
+  mid = __float2bfloat16_rn(r1);
+  lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+}
+
+// 8 bf16 values as one 16-byte chunk of a 128-byte row
+__device__ __forceinline__ uint4 pack8(const __nv_bfloat16 (&v)[8]) {
+  uint4 u;
+  u.x = (uint32_t)__bfloat16_as_ushort(v[0]) | ((uint32_t)__bfloat16_as_ushort(v[1]) << 16);
+  u.y = (uint32_t)__bfloat16_as_ushort(v[2]) | ((uint32_t)__bfloat16_as_ushort(v[3]) << 16);
+  u.z = (uint32_t)__bfloat16_as_ushort(v[4]) | ((uint32_t)__bfloat16_as_ushort(v[5]) << 16);
+  u.w = (uint32_t)__bfloat16_as_ushort(v[6]) | ((uint32_t)__bfloat16_as_ushort(v[7]) << 16);
+  return u;
+}
+
+// Byte offset of 16-byte chunk k16 of row r in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw_chunk(int r, int k16) {
+  return (uint32_t)r * 128 + ((uint32_t)(k16 ^ (r & 7)) << 4);
+}
+
+// 8 bf16 of row r, chunk k16 of a swizzled tile, as floats
+__device__ __forceinline__ void load8(const unsigned char* tile, int r, int k16, float* f) {
+  const uint4 u = *reinterpret_cast<const uint4*>(tile + sw_chunk(r, k16));
+  const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w4[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
+  }
+}
+
+// Three-term split of 8 consecutive values of row r (chunk k16) into three
+// tiles `stride` bytes apart.
+__device__ __forceinline__ void store_terms8(unsigned char* tile, uint32_t stride, int r, int k16, const float* v) {
+  __nv_bfloat16 h[8], m[8], l[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) split3(v[i], h[i], m[i], l[i]);
+  const uint32_t off = sw_chunk(r, k16);
+  *reinterpret_cast<uint4*>(tile + off) = pack8(h);
+  *reinterpret_cast<uint4*>(tile + stride + off) = pack8(m);
+  *reinterpret_cast<uint4*>(tile + 2 * stride + off) = pack8(l);
+}
+
+// A state (P x N fp32; this thread: row p, states n in [n0, n0 + 32)) as three
+// terms, each two 64-column blocks [p][n] of the split area.
+__device__ __forceinline__ void store_state_terms(unsigned char* area, int p, int n0, const float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int n = n0 + 8 * c;
+    store_terms8(area + (n >> 6) * TcCfg::kTile, 2 * TcCfg::kTile, p, (n & 63) >> 3, v + 8 * c);
+  }
+}
+
+// Descriptor of K step kk of a K-major operand: 16 bf16 (32 bytes) along the
+// row, the next 64-column tile after 4 steps.
+__device__ __forceinline__ uint64_t kmaj(uint64_t d0, int kk) {
+  return d0 + (uint64_t)(((kk >> 2) * TcCfg::kTile + (kk & 3) * 32) >> 4);
+}
+// ... of an MN-major operand: 16 rows (2048 bytes)
+__device__ __forceinline__ uint64_t mnmaj(uint64_t d0, int kk) { return d0 + (uint64_t)((kk * 2048) >> 4); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_bwd_chunk_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dy,
+                   const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
+                   const KArgs a) {
+  using K = TcCfg;
+  constexpr uint64_t kLimit = tc::kWaitLimitNs;
+  const Dims& d = a.d;
+  const ChunkPos q = chunk_pos(d, blockIdx.x);
+  const int Qc = q.Qc, last = Qc - 1;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                       ~uintptr_t(1023));
+  float* Mm = reinterpret_cast<float*>(sm + K::oM);
+  __shared__ TcSmem s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // TMEM reads: warp (qd, hf) reads rows 16 qd + (lane & 15) of its lane
+  // quadrant; 64-column accumulators give it columns c0 + [0, 16), 128-column
+  // ones columns c1 + [0, 32)
+  const int qd = warp & 3, hf = warp >> 2;
+  const int row = 16 * qd + (lane & 15);
+  const int c0 = 16 * hf + 32 * (lane >> 4);
+  const int c1 = 64 * hf + 32 * (lane >> 4);
+  volatile int* abort_flag = &s.abort_flag;
+  volatile int* never = &s.never;
+
+  if (tid == 0) {
+    mbar_init(&s.bar_in, 1);
+    mbar_init(&s.bar_p1, 1);
+    mbar_init(&s.bar_p2, 1);
+    mbar_init(&s.bar_drain, 1);
+    s.abort_flag = 0;
+    s.never = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_dy);
+    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_c);
+  }
+  if (warp == 0) {
+    tmem_alloc(&s.tmem_base, K::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  const uint32_t tq = tmem + ((uint32_t)(32 * qd) << 16);
+  if (tid == 0) {
+    const int col = (int)(q.h * d.P), tok = (int)q.t0, bb = (int)q.b, grp = (int)q.g;
+    mbar_arrive_expect_tx(&s.bar_in, 6 * K::kTile);
+    tma_load_3d(sm + K::oX, &tm_x, &s.bar_in, col, tok, bb);
+    tma_load_3d(sm + K::oDY, &tm_dy, &s.bar_in, col, tok, bb);
+    for (int jb = 0; jb < 2; ++jb) {
+      tma_load_4d(sm + K::oB + jb * K::kTile, &tm_b, &s.bar_in, 64 * jb, grp, tok, bb);
+      tma_load_4d(sm + K::oC + jb * K::kTile, &tm_c, &s.bar_in, 64 * jb, grp, tok, bb);
+    }
+  }
+
+  // the chunk's states: this thread's row p = tid / 4, states n in [32 (tid % 4), +32)
+  const int sp = tid >> 2, sn0 = 32 * (tid & 3);
+  const int64_t soff = ((q.b * d.H + q.h) * d.nc + q.c) * d.P * d.N + (int64_t)sp * d.N + sn0;
+  float hin[32];
+  {
+    float lam[32];
+    const float4* pl = reinterpret_cast<const float4*>(a.T + soff);
+    const float4* ph = reinterpret_cast<const float4*>(a.S + soff);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 v = __ldcg(pl + i), u = __ldcg(ph + i);
+      lam[4 * i] = v.x, lam[4 * i + 1] = v.y, lam[4 * i + 2] = v.z, lam[4 * i + 3] = v.w;
+      hin[4 * i] = u.x, hin[4 * i + 1] = u.y, hin[4 * i + 2] = u.z, hin[4 * i + 3] = u.w;
+    }
+    float lh = 0.f;  // <Lam, h_in>, this thread's share
+#pragma unroll
+    for (int i = 0; i < 32; ++i) lh = fmaf(lam[i], hin[i], lh);
+    s.red[tid] = lh;
+    store_state_terms(sm + K::oS, sp, sn0, lam);
+  }
+  for (int t = tid; t < 64; t += kThreads) {
+    s.w[t] = t < Qc ? a.dt[(q.b * d.L + q.t0 + t) * d.H + q.h] : 0.f;
+    s.cs[t] = 0.f;
+    s.seg[t] = 0;
+    s.el[t] = 0.f;
+    s.ein[t] = 0.f;
+    s.dg[t] = 0.f;
+  }
+  __syncthreads();
+  chunk_cumsum(a, q, s.cs, s.seg, tid);  // ends with a barrier
+  for (int off = kThreads / 2; off > 0; off >>= 1) {
+    if (tid < off) s.red[tid] += s.red[tid + off];
+    __syncthreads();
+  }
+  for (int t = tid; t < Qc; t += kThreads) {
+    s.el[t] = s.seg[t] == s.seg[last] ? expf(s.cs[last] - s.cs[t]) : 0.f;
+    s.ein[t] = s.seg[t] == -1 ? expf(s.cs[t]) : 0.f;
+  }
+  fence_proxy_async_smem();  // the Lam terms are read by the MMAs
+  __syncthreads();
+
+  // descriptors: K-major tiles (rows along K) and MN-major ones (rows along K,
+  // the 64-element blocks of M or N one tile apart)
+  const uint64_t dX = sw128_desc(smem_u32(sm + K::oX), 16, 1024);
+  const uint64_t dDY = sw128_desc(smem_u32(sm + K::oDY), 16, 1024);
+  const uint64_t dB = sw128_desc(smem_u32(sm + K::oB), 16, 1024);
+  const uint64_t dC = sw128_desc(smem_u32(sm + K::oC), 16, 1024);
+  const uint64_t dDYmn = sw128_desc(smem_u32(sm + K::oDY), K::kTile, 1024);
+  const uint64_t dBmn = sw128_desc(smem_u32(sm + K::oB), K::kTile, 1024);
+  const uint64_t dCmn = sw128_desc(smem_u32(sm + K::oC), K::kTile, 1024);
+  constexpr uint32_t id_kk64 = idesc_bf16(64, 64, 0, 0);
+  constexpr uint32_t id_km128 = idesc_bf16(64, 128, 0, 1);
+  constexpr uint32_t id_mm64 = idesc_bf16(64, 64, 1, 1);
+  constexpr uint32_t id_mm128 = idesc_bf16(64, 128, 1, 1);
+  // term t3 of a split: the Q x Q ones one tile apart, the states two
+  auto qq_term = [&](uint32_t base, int t3, bool mn) {
+    return sw128_desc(smem_u32(sm + base + (uint32_t)t3 * K::kTile), mn ? K::kTile : 16, 1024);
+  };
+  auto st_term = [&](int t3, bool mn) {
+    return sw128_desc(smem_u32(sm + K::oS + (uint32_t)t3 * 2 * K::kTile), mn ? K::kTile : 16, 1024);
+  };
+
+  // ---- MMAs, first round: CB, G, B Lam^T, x Lam
+  bool ok = mbar_wait(&s.bar_in, 0, abort_flag, kLimit);  // every thread reads the tiles later
+  if (warp == 0 && __all_sync(0xffffffffu, ok)) {
+    tc_fence_after();
+    if (elect_one()) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)  // CB = C B^T (K = n)
+        mma_bf16_ss(tmem + K::tCB, kmaj(dC, kk), kmaj(dB, kk), id_kk64, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)  // G = dy x^T (K = p)
+        mma_bf16_ss(tmem + K::tG, kmaj(dDY, kk), kmaj(dX, kk), id_kk64, kk > 0);
+#pragma unroll
+      for (int t3 = 0; t3 < 3; ++t3) {
+        const uint64_t lk = st_term(t3, false), lm = st_term(t3, true);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // dx <- B Lam^T (K = n)
+          mma_bf16_ss(tmem + K::tDx, kmaj(dB, kk), kmaj(lk, kk), id_kk64, t3 > 0 || kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dB <- x Lam (K = p)
+          mma_bf16_ss(tmem + K::tDB, kmaj(dX, kk), mnmaj(lm, kk), id_km128, t3 > 0 || kk > 0);
+      }
+      mma_commit(&s.bar_p1);
+    }
+    __syncwarp();
+  }
+  ok = ok && mbar_wait(&s.bar_p1, 0, abort_flag, kLimit);
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    tc_fence_after();
+    // ---- the Q x Q matrices: row t, columns s in [c0, c0 + 16)
+    {
+      uint32_t rcb[16], rg[16];
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tCB + 16 * hf, rcb);
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tG + 16 * hf, rg);
+      SSD_TMEM_WAIT_LD_16(rcb);
+      SSD_TMEM_WAIT_LD_16(rg);
+      const int t = row;
+      const float cst = s.cs[t];
+      const int segt = s.seg[t];
+      float kv[16], zv[16], zwv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int sc = c0 + i;
+        const float g = __uint_as_float(rg[i]);
+        const bool in = t < Qc && sc <= t && s.seg[sc] == segt;
+        const float e = in ? expf(cst - s.cs[sc]) : 0.f;
+        kv[i] = e * __uint_as_float(rcb[i]);
+        zv[i] = e * g;
+        zwv[i] = zv[i] * s.w[sc];
+        Mm[t * K::kMs + sc] = kv[i] * g;
+        if (sc == t && t < Qc) s.dg[t] = g;
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int k16 = (c0 >> 3) + c;
+        store_terms8(sm + K::oK, K::kTile, t, k16, kv + 8 * c);
+        store_terms8(sm + K::oZ, K::kTile, t, k16, zv + 8 * c);
+        store_terms8(sm + K::oZw, K::kTile, t, k16, zwv + 8 * c);
+      }
+    }
+    // ---- B Lam^T: the row sums x_s . (Lam B_s), then scaled by el_s and written back
+    {
+      uint32_t r[16];
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDx + 16 * hf, r);
+      SSD_TMEM_WAIT_LD_16(r);
+      const int sr = row;
+      float xv[16];
+      load8(sm + K::oX, sr, c0 >> 3, xv);
+      load8(sm + K::oX, sr, (c0 >> 3) + 1, xv + 8);
+      float nx = 0.f;
+      const float els = s.el[sr];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float v = __uint_as_float(r[i]);
+        nx = fmaf(xv[i], v, nx);
+        r[i] = __float_as_uint(els * v);
+      }
+      s.nxp[sr][2 * hf + (lane >> 4)] = nx;
+      SSD_TMEM_ST_16x32bx2_X16_HALF32(tq + K::tDx + 16 * hf, r);
+    }
+    // ---- x Lam: scaled by el_s and written back
+    {
+      const float els = s.el[row];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[16];
+        SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDB + 64 * hf + 16 * half, r);
+        SSD_TMEM_WAIT_LD_16(r);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(els * __uint_as_float(r[i]));
+        SSD_TMEM_ST_16x32bx2_X16_HALF32(tq + K::tDB + 64 * hf + 16 * half, r);
+      }
+    }
+    // ---- h_in terms over the Lam terms (the MMAs that read those are done)
+    store_state_terms(sm + K::oS, sp, sn0, hin);
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  fence_proxy_async_smem();  // the split tiles are read by the MMAs
+  ok = __syncthreads_and(ok);
+
+  // ---- MMAs, second round: K^T dy, Z^T C (accumulating), dy h_in, Zw B
+  if (ok && warp == 0) {
+    tc_fence_after();
+    if (elect_one()) {
+#pragma unroll
+      for (int t3 = 0; t3 < 3; ++t3) {
+        const uint64_t k_mn = qq_term(K::oK, t3, true), z_mn = qq_term(K::oZ, t3, true);
+        const uint64_t zw_k = qq_term(K::oZw, t3, false), h_mn = st_term(t3, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // K = t, t, p, s
+          mma_bf16_ss(tmem + K::tDx, mnmaj(k_mn, kk), mnmaj(dDYmn, kk), id_mm64, 1);
+          mma_bf16_ss(tmem + K::tDB, mnmaj(z_mn, kk), mnmaj(dCmn, kk), id_mm128, 1);
+          mma_bf16_ss(tmem + K::tDC2, kmaj(dDY, kk), mnmaj(h_mn, kk), id_km128, t3 > 0 || kk > 0);
+          mma_bf16_ss(tmem + K::tDC1, kmaj(zw_k, kk), mnmaj(dBmn, kk), id_km128, t3 > 0 || kk > 0);
+        }
+      }
+      mma_commit(&s.bar_p2);
+    }
+    __syncwarp();
+  }
+  ok = ok && mbar_wait(&s.bar_p2, 0, abort_flag, kLimit);
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    tc_fence_after();
+    const int64_t tok = q.b * d.L + q.t0 + row;  // this thread's token row
+    const bool valid = row < Qc;
+    // ---- dx = w_s [K^T dy + el_s B Lam^T] + D dy_s (columns p in [c0, c0 + 16))
+    {
+      uint32_t r[16];
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDx + 16 * hf, r);
+      SSD_TMEM_WAIT_LD_16(r);
+      float dyv[16];
+      load8(sm + K::oDY, row, c0 >> 3, dyv);
+      load8(sm + K::oDY, row, (c0 >> 3) + 1, dyv + 8);
+      const float ws = s.w[row], Dh = a.D ? a.D[q.h] : 0.f;
+      if (valid) {
+        float4* dst = reinterpret_cast<float4*>(a.dx + (tok * d.H + q.h) * d.P + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_float4(fmaf(ws, __uint_as_float(r[4 * i]), Dh * dyv[4 * i]),
+                               fmaf(ws, __uint_as_float(r[4 * i + 1]), Dh * dyv[4 * i + 1]),
+                               fmaf(ws, __uint_as_float(r[4 * i + 2]), Dh * dyv[4 * i + 2]),
+                               fmaf(ws, __uint_as_float(r[4 * i + 3]), Dh * dyv[4 * i + 3]));
+      }
+    }
+    // ---- dB of this head = w_s [Z^T C + el_s x Lam] (states n in [c1, c1 + 32))
+    {
+      uint32_t r[32];
+      uint32_t* r_hi = r + 16;
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDB + 64 * hf, r);
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDB + 64 * hf + 16, r_hi);
+      SSD_TMEM_WAIT_LD_32(r);
+      const float ws = s.w[row];
+      if (valid) {
+        float4* dst = reinterpret_cast<float4*>(a.dBh + (tok * d.H + q.h) * d.N + c1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(ws * __uint_as_float(r[4 * i]), ws * __uint_as_float(r[4 * i + 1]),
+                               ws * __uint_as_float(r[4 * i + 2]), ws * __uint_as_float(r[4 * i + 3]));
+      }
+    }
+    // ---- dC of this head = Zw B + e_t dy h_in, and the row sums C_t . (h_in^T dy_t)
+    {
+      uint32_t r2[32], r1[32];
+      uint32_t* r2_hi = r2 + 16;
+      uint32_t* r1_hi = r1 + 16;
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDC2 + 64 * hf, r2);
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDC2 + 64 * hf + 16, r2_hi);
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDC1 + 64 * hf, r1);
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDC1 + 64 * hf + 16, r1_hi);
+      SSD_TMEM_WAIT_LD_32(r2);
+      SSD_TMEM_WAIT_LD_32(r1);
+      float cv[32];
+      const unsigned char* ctile = sm + K::oC + hf * K::kTile;  // states 64 hf ..
+#pragma unroll
+      for (int c = 0; c < 4; ++c) load8(ctile, row, 4 * (lane >> 4) + c, cv + 8 * c);
+      const float et = s.ein[row];
+      float cy = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) cy = fmaf(cv[i], __uint_as_float(r2[i]), cy);
+      s.cyp[row][2 * hf + (lane >> 4)] = cy;
+      if (valid) {
+        float4* dst = reinterpret_cast<float4*>(a.dCh + (tok * d.H + q.h) * d.N + c1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(fmaf(et, __uint_as_float(r2[4 * i]), __uint_as_float(r1[4 * i])),
+                               fmaf(et, __uint_as_float(r2[4 * i + 1]), __uint_as_float(r1[4 * i + 1])),
+                               fmaf(et, __uint_as_float(r2[4 * i + 2]), __uint_as_float(r1[4 * i + 2])),
+                               fmaf(et, __uint_as_float(r2[4 * i + 3]), __uint_as_float(r1[4 * i + 3])));
+      }
+    }
+  }
+  tc_fence_before();
+  ok = __syncthreads_and(ok);
+
+  if (ok) {
+    // ---- the decay gradients (the tail of k_bwd_chunk, on the row sums above)
+    for (int t = tid; t < Qc; t += kThreads) {
+      s.nv[t] = s.nxp[t][0] + s.nxp[t][1] + s.nxp[t][2] + s.nxp[t][3];
+      s.dcs[t] = s.ein[t] * (s.cyp[t][0] + s.cyp[t][1] + s.cyp[t][2] + s.cyp[t][3]);
+    }
+    // per token k, four threads each: a quarter of the column sum of M below
+    // the diagonal (for dw) and of the block sum S_k = sum_{u >= k, s < k}
+    // M(u,s) w_s, the pairs whose decay spans k
+    for (int i = tid; i < 4 * Qc; i += kThreads) {
+      const int k = i >> 2, qq = i & 3;
+      const int lo = k + (Qc - k) * qq / 4, hi = k + (Qc - k) * (qq + 1) / 4;
+      float col = 0.f, blk = 0.f;
+      for (int u = lo; u < hi; ++u) {
+        if (u > k) col += Mm[u * K::kMs + k];
+        for (int s2 = 0; s2 < k; ++s2) blk = fmaf(Mm[u * K::kMs + s2], s.w[s2], blk);
+      }
+      s.pair[k][qq] = col;
+      s.pair[k][4 + qq] = blk;
+    }
+    __syncthreads();
+    for (int t = tid; t < Qc; t += kThreads) {
+      const float col = s.pair[t][0] + s.pair[t][1] + s.pair[t][2] + s.pair[t][3];
+      const float blk = s.pair[t][4] + s.pair[t][5] + s.pair[t][6] + s.pair[t][7];
+      s.dw[t] = fmaf(s.el[t], s.nv[t], col + Mm[t * K::kMs + t]);
+      s.nn[t] = s.el[t] * s.w[t] * s.nv[t];
+      s.pair[t][0] = blk;  // S_t
+    }
+    __syncthreads();
+    if (tid == 0) {
+      // dl_k = S_k + sum_{t >= k} (h_in term)_t + sum_{s < k} N_s + e_last <Lam, h_in>
+      const float lh = s.red[0];
+      const float e_last = s.seg[last] == -1 ? expf(s.cs[last]) : 0.f;
+      float before = 0.f;  // sum_{s < k} N_s, kept in nn as an exclusive prefix
+      for (int k = 0; k <= last; ++k) {
+        const float v = s.nn[k];
+        s.nn[k] = before;
+        before += v;
+      }
+      const float Ah = a.A[q.h];
+      double dA = 0.0, dD = 0.0;
+      float after = 0.f;  // sum_{t >= k} of the h_in term
+      for (int k = last; k >= 0; --k) {
+        after += s.dcs[k];
+        const float dl = s.seg[k] == k ? 0.f : s.pair[k][0] + after + s.nn[k] + e_last * lh;
+        a.ddt[(q.b * d.L + q.t0 + k) * d.H + q.h] = fmaf(Ah, dl, s.dw[k]);
+        dA += (double)s.w[k] * (double)dl;
+        dD += (double)s.dg[k];
+      }
+      const int64_t pi = q.h * (d.b * d.nc) + q.b * d.nc + q.c;
+      a.dA_part[pi] = dA;
+      a.dD_part[pi] = dD;
+    }
+  } else if (warp == 0) {
+    // a wait gave up: let this CTA's copies and MMAs finish before its memory goes
+    mbar_wait(&s.bar_in, 0, never, kLimit);
+    if (elect_one()) {
+      mma_commit(&s.bar_drain);
+      mbar_wait(&s.bar_drain, 0, never, kLimit);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+// The tensor-core chunk kernel takes bf16 calls without a gate at headdim 64,
+// dstate 128 and 64-token chunks (TMA needs 16-byte aligned x, dy, B, C; the
+// gradient stores are 16-byte vectors).
+inline bool chunk_tc_supported(const KArgs& k) {
+  const Dims& d = k.d;
+  return d.P == 64 && d.N == 128 && d.Q == 64 && !k.z && aligned16(k.x) && aligned16(k.dy) && aligned16(k.B) &&
+         aligned16(k.C) && aligned16(k.dx) && d.L < ((int64_t)1 << 31) && d.H * d.P < ((int64_t)1 << 31);
+}
+
+inline cudaError_t chunk_tc_launch(const KArgs& k, cudaStream_t st) {
+  const Dims& d = k.d;
+  CUtensorMap tx, tdy, tb, tc_;
+  if (!tc::make_map_3d(&tx, k.x, d.H * d.P, d.L, d.b) || !tc::make_map_3d(&tdy, k.dy, d.H * d.P, d.L, d.b) ||
+      !tc::make_map_bc(&tb, k.B, d.N, d.G, d.L, d.b) || !tc::make_map_bc(&tc_, k.C, d.N, d.G, d.L, d.b))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)TcCfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  k_bwd_chunk_tc<<<(unsigned)(d.b * d.nc * d.H), kThreads, TcCfg::kSmemBytes, st>>>(tx, tdy, tb, tc_, k);
+  return cudaGetLastError();
+}
+
+}  // namespace bwd
+}  // namespace ssd
