@@ -196,6 +196,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   const uint32_t tq = tmem + ((uint32_t)(32 * qd) << 16);
   if (tid == 0) {
+    // the chunk states of the CTA one wave later, into L2 (a hint: the grid
+    // runs one CTA an SM, so that CTA comes about an SM count later)
+    uint32_t nsm;
+    asm("mov.u32 %0, %%nsmid;" : "=r"(nsm));
+    const int64_t nb = (int64_t)blockIdx.x + nsm;
+    if (nb < (int64_t)gridDim.x) {
+      const ChunkPos qn = chunk_pos(d, nb);
+      const int64_t o = ((qn.b * d.H + qn.h) * d.nc + qn.c) * d.P * d.N;
+      const uint32_t bytes = (uint32_t)(d.P * d.N * 4);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.S + o), "r"(bytes) : "memory");
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.T + o), "r"(bytes) : "memory");
+    }
     const int col = (int)(q.h * d.P), tok = (int)q.t0, bb = (int)q.b, grp = (int)q.g;
     mbar_arrive_expect_tx(&s.bar_in, 6 * K::kTile);
     tma_load_3d(sm + K::oX, &tm_x, &s.bar_in, col, tok, bb);
@@ -470,16 +482,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       s.nv[t] = s.nxp[t][0] + s.nxp[t][1] + s.nxp[t][2] + s.nxp[t][3];
       s.dcs[t] = s.ein[t] * (s.cyp[t][0] + s.cyp[t][1] + s.cyp[t][2] + s.cyp[t][3]);
     }
-    // per token k, four threads each: a quarter of the column sum of M below
-    // the diagonal (for dw) and of the block sum S_k = sum_{u >= k, s < k}
-    // M(u,s) w_s, the pairs whose decay spans k
+    // The pairs whose decay spans token k: S_k = sum_{u >= k} R(u, k) with the
+    // row prefix R(u, k) = sum_{s < k} M(u, s) w_s, and the column sum of M
+    // below the diagonal (for dw).  R goes where the K terms were (the MMAs
+    // that read them are done).  Row u's prefix: four threads, 16 columns each.
+    float* Rm = reinterpret_cast<float*>(sm + K::oK);  // [u][k], rows of kMs
+    {
+      const int u = tid >> 2, sg = tid & 3;
+      float pre[16], run = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int sc = 16 * sg + j;
+        pre[j] = run;
+        run = fmaf(Mm[u * K::kMs + sc], s.w[sc], run);
+      }
+      s.pair[u][sg] = run;  // this segment's total
+      __syncwarp();
+      float off = 0.f;  // the segments before this one (same warp: threads 4u .. 4u + 3)
+      for (int g2 = 0; g2 < sg; ++g2) off += s.pair[u][g2];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) Rm[u * K::kMs + 16 * sg + j] = off + pre[j];
+    }
+    __syncthreads();
     for (int i = tid; i < 4 * Qc; i += kThreads) {
       const int k = i >> 2, qq = i & 3;
       const int lo = k + (Qc - k) * qq / 4, hi = k + (Qc - k) * (qq + 1) / 4;
       float col = 0.f, blk = 0.f;
       for (int u = lo; u < hi; ++u) {
         if (u > k) col += Mm[u * K::kMs + k];
-        for (int s2 = 0; s2 < k; ++s2) blk = fmaf(Mm[u * K::kMs + s2], s.w[s2], blk);
+        blk += Rm[u * K::kMs + k];
       }
       s.pair[k][qq] = col;
       s.pair[k][4 + qq] = blk;
@@ -493,32 +524,222 @@ __global__ void __launch_bounds__(kThreads, 1)
       s.pair[t][0] = blk;  // S_t
     }
     __syncthreads();
-    if (tid == 0) {
-      // dl_k = S_k + sum_{t >= k} (h_in term)_t + sum_{s < k} N_s + e_last <Lam, h_in>
+    if (warp == 0) {
+      // dl_k = S_k + sum_{t >= k} (h_in term)_t + sum_{s < k} N_s + e_last <Lam, h_in>,
+      // tokens k = lane and lane + 32, the sums as warp scans
       const float lh = s.red[0];
       const float e_last = s.seg[last] == -1 ? expf(s.cs[last]) : 0.f;
-      float before = 0.f;  // sum_{s < k} N_s, kept in nn as an exclusive prefix
-      for (int k = 0; k <= last; ++k) {
-        const float v = s.nn[k];
-        s.nn[k] = before;
-        before += v;
+      const int k0 = lane, k1 = lane + 32;
+      const bool v0 = k0 <= last, v1 = k1 <= last;
+      const float n0 = v0 ? s.nn[k0] : 0.f, n1 = v1 ? s.nn[k1] : 0.f;
+      const float h0v = v0 ? s.dcs[k0] : 0.f, h1v = v1 ? s.dcs[k1] : 0.f;
+      float pre0 = n0, pre1 = n1, suf0 = h0v, suf1 = h1v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float a0 = __shfl_up_sync(0xffffffffu, pre0, o), a1 = __shfl_up_sync(0xffffffffu, pre1, o);
+        const float b0 = __shfl_down_sync(0xffffffffu, suf0, o), b1 = __shfl_down_sync(0xffffffffu, suf1, o);
+        if (lane >= o) pre0 += a0, pre1 += a1;
+        if (lane + o < 32) suf0 += b0, suf1 += b1;
       }
+      pre1 += __shfl_sync(0xffffffffu, pre0, 31);  // the first 32 tokens' total
+      suf0 += __shfl_sync(0xffffffffu, suf1, 0);   // the last 32 tokens' total
       const float Ah = a.A[q.h];
       double dA = 0.0, dD = 0.0;
-      float after = 0.f;  // sum_{t >= k} of the h_in term
-      for (int k = last; k >= 0; --k) {
-        after += s.dcs[k];
-        const float dl = s.seg[k] == k ? 0.f : s.pair[k][0] + after + s.nn[k] + e_last * lh;
-        a.ddt[(q.b * d.L + q.t0 + k) * d.H + q.h] = fmaf(Ah, dl, s.dw[k]);
-        dA += (double)s.w[k] * (double)dl;
-        dD += (double)s.dg[k];
+      if (v0) {
+        const float dl = s.seg[k0] == k0 ? 0.f : s.pair[k0][0] + suf0 + (pre0 - n0) + e_last * lh;
+        a.ddt[(q.b * d.L + q.t0 + k0) * d.H + q.h] = fmaf(Ah, dl, s.dw[k0]);
+        dA += (double)s.w[k0] * (double)dl;
+        dD += (double)s.dg[k0];
       }
-      const int64_t pi = q.h * (d.b * d.nc) + q.b * d.nc + q.c;
-      a.dA_part[pi] = dA;
-      a.dD_part[pi] = dD;
+      if (v1) {
+        const float dl = s.seg[k1] == k1 ? 0.f : s.pair[k1][0] + suf1 + (pre1 - n1) + e_last * lh;
+        a.ddt[(q.b * d.L + q.t0 + k1) * d.H + q.h] = fmaf(Ah, dl, s.dw[k1]);
+        dA += (double)s.w[k1] * (double)dl;
+        dD += (double)s.dg[k1];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        dA += __shfl_xor_sync(0xffffffffu, dA, o);
+        dD += __shfl_xor_sync(0xffffffffu, dD, o);
+      }
+      if (lane == 0) {
+        const int64_t pi = q.h * (d.b * d.nc) + q.b * d.nc + q.c;
+        a.dA_part[pi] = dA;
+        a.dD_part[pi] = dD;
+      }
     }
   } else if (warp == 0) {
     // a wait gave up: let this CTA's copies and MMAs finish before its memory goes
+    mbar_wait(&s.bar_in, 0, never, kLimit);
+    if (elect_one()) {
+      mma_commit(&s.bar_drain);
+      mbar_wait(&s.bar_drain, 0, never, kLimit);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
+}
+
+// The chunk states of the backward's recomputation on the tensor cores (the
+// formulas of k_bwd_chunk_states): per (batch row, chunk, head)
+//
+//   S = (diag(cS) x)^T B,   cS_t = dt_t E(last, t)     the chunk's end state from zero
+//   T = (diag(cT) dy)^T C,  cT_t = e_t                  its part of dLoss/dh_in
+//
+// with the scaled x and dy as three bf16 terms (fp32 accuracy, as above) and
+// B, C as loaded; M = 64 (p), N = 128 (n), K = 64 tokens.  256 TMEM columns
+// and 97 KB of shared memory, so two CTAs share an SM.
+struct StCfg {
+  static constexpr uint32_t kTile = 8192;
+  static constexpr uint32_t oX = 0;                  // x  [t][p]
+  static constexpr uint32_t oDY = oX + kTile;        // dy [t][p]
+  static constexpr uint32_t oB = oDY + kTile;        // B  [t][n]
+  static constexpr uint32_t oC = oB + 2 * kTile;     // C  [t][n]
+  static constexpr uint32_t oXs = oC + 2 * kTile;    // cS x terms [3][t][p]
+  static constexpr uint32_t oDs = oXs + 3 * kTile;   // cT dy terms [3][t][p]
+  static constexpr uint32_t oEnd = oDs + 3 * kTile;
+  static constexpr uint32_t kSmemBytes = oEnd + 1024;
+  static constexpr uint32_t tS = 0, tT = 128, kTmemCols = 256;
+};
+
+struct __align__(16) StSmem {
+  uint64_t bar_in, bar_mma, bar_drain;
+  uint32_t tmem_base;
+  int abort_flag, never;
+  float cs[64], cS[64], cT[64];
+  int seg[64];
+};
+
+__global__ void __launch_bounds__(kThreads, 2)
+    k_bwd_chunk_states_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dy,
+                          const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
+                          const KArgs a) {
+  using K = StCfg;
+  constexpr uint64_t kLimit = tc::kWaitLimitNs;
+  const Dims& d = a.d;
+  const ChunkPos q = chunk_pos(d, blockIdx.x);
+  const int Qc = q.Qc, last = Qc - 1;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                       ~uintptr_t(1023));
+  __shared__ StSmem s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, hf = warp >> 2;
+  const int row = 16 * qd + (lane & 15);          // state row p this thread reads from TMEM
+  const int c1 = 64 * hf + 32 * (lane >> 4);      // and its states n in [c1, c1 + 32)
+  volatile int* abort_flag = &s.abort_flag;
+  volatile int* never = &s.never;
+
+  if (tid == 0) {
+    mbar_init(&s.bar_in, 1);
+    mbar_init(&s.bar_mma, 1);
+    mbar_init(&s.bar_drain, 1);
+    s.abort_flag = 0;
+    s.never = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_dy);
+    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_c);
+  }
+  if (warp == 0) {
+    tmem_alloc(&s.tmem_base, K::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  const uint32_t tq = tmem + ((uint32_t)(32 * qd) << 16);
+  if (tid == 0) {
+    const int col = (int)(q.h * d.P), tok = (int)q.t0, bb = (int)q.b, grp = (int)q.g;
+    mbar_arrive_expect_tx(&s.bar_in, 6 * K::kTile);
+    tma_load_3d(sm + K::oX, &tm_x, &s.bar_in, col, tok, bb);
+    tma_load_3d(sm + K::oDY, &tm_dy, &s.bar_in, col, tok, bb);
+    for (int jb = 0; jb < 2; ++jb) {
+      tma_load_4d(sm + K::oB + jb * K::kTile, &tm_b, &s.bar_in, 64 * jb, grp, tok, bb);
+      tma_load_4d(sm + K::oC + jb * K::kTile, &tm_c, &s.bar_in, 64 * jb, grp, tok, bb);
+    }
+  }
+  for (int t = tid; t < 64; t += kThreads) {
+    s.cs[t] = 0.f;
+    s.seg[t] = 0;
+    s.cS[t] = 0.f;
+    s.cT[t] = 0.f;
+  }
+  __syncthreads();
+  chunk_cumsum(a, q, s.cs, s.seg, tid);  // ends with a barrier
+  for (int t = tid; t < Qc; t += kThreads) {
+    const float w = a.dt[(q.b * d.L + q.t0 + t) * d.H + q.h];
+    s.cS[t] = s.seg[t] == s.seg[last] ? w * expf(s.cs[last] - s.cs[t]) : 0.f;
+    s.cT[t] = s.seg[t] == -1 ? expf(s.cs[t]) : 0.f;
+  }
+  if (tid == 0) a.dec[(q.b * d.H + q.h) * d.nc + q.c] = s.seg[last] == -1 ? expf(s.cs[last]) : 0.f;
+  __syncthreads();
+  bool ok = mbar_wait(&s.bar_in, 0, abort_flag, kLimit);
+  if (ok) {
+    // the scaled x and dy as three bf16 terms: row t = tid / 4, columns p in [16 (tid % 4), +16)
+    const int t = tid >> 2, k0 = 2 * (tid & 3);
+    float v[16];
+    load8(sm + K::oX, t, k0, v);
+    load8(sm + K::oX, t, k0 + 1, v + 8);
+    const float fs = s.cS[t], ft = s.cT[t];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] *= fs;
+    store_terms8(sm + K::oXs, K::kTile, t, k0, v);
+    store_terms8(sm + K::oXs, K::kTile, t, k0 + 1, v + 8);
+    load8(sm + K::oDY, t, k0, v);
+    load8(sm + K::oDY, t, k0 + 1, v + 8);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] *= ft;
+    store_terms8(sm + K::oDs, K::kTile, t, k0, v);
+    store_terms8(sm + K::oDs, K::kTile, t, k0 + 1, v + 8);
+  }
+  fence_proxy_async_smem();  // the terms are read by the MMAs
+  ok = __syncthreads_and(ok);
+  if (ok && warp == 0) {
+    tc_fence_after();
+    const uint64_t dBmn = sw128_desc(smem_u32(sm + K::oB), K::kTile, 1024);
+    const uint64_t dCmn = sw128_desc(smem_u32(sm + K::oC), K::kTile, 1024);
+    constexpr uint32_t id = idesc_bf16(64, 128, 1, 1);  // A = terms^T (MN-major), B MN-major
+    if (elect_one()) {
+#pragma unroll
+      for (int t3 = 0; t3 < 3; ++t3) {
+        const uint64_t xs = sw128_desc(smem_u32(sm + K::oXs + t3 * K::kTile), K::kTile, 1024);
+        const uint64_t ds = sw128_desc(smem_u32(sm + K::oDs + t3 * K::kTile), K::kTile, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // K = tokens
+          mma_bf16_ss(tmem + K::tS, mnmaj(xs, kk), mnmaj(dBmn, kk), id, t3 > 0 || kk > 0);
+          mma_bf16_ss(tmem + K::tT, mnmaj(ds, kk), mnmaj(dCmn, kk), id, t3 > 0 || kk > 0);
+        }
+      }
+      mma_commit(&s.bar_mma);
+    }
+    __syncwarp();
+  }
+  ok = ok && mbar_wait(&s.bar_mma, 0, abort_flag, kLimit);
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    tc_fence_after();
+    const int64_t off = ((q.b * d.H + q.h) * d.nc + q.c) * d.P * d.N + (int64_t)row * d.N + c1;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      uint32_t r[32];
+      uint32_t* r_hi = r + 16;
+      const uint32_t col = (which ? K::tT : K::tS) + 64 * hf;
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + col, r);
+      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + col + 16, r_hi);
+      SSD_TMEM_WAIT_LD_32(r);
+      float4* dst = reinterpret_cast<float4*>((which ? a.T : a.S) + off);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
+                             __uint_as_float(r[4 * i + 3]));
+    }
+  } else if (warp == 0) {
     mbar_wait(&s.bar_in, 0, never, kLimit);
     if (elect_one()) {
       mma_commit(&s.bar_drain);
@@ -536,8 +757,8 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 }  // namespace
 
-// The tensor-core chunk kernel takes bf16 calls without a gate at headdim 64,
-// dstate 128 and 64-token chunks (TMA needs 16-byte aligned x, dy, B, C; the
+// The tensor-core kernels take bf16 calls without a gate at headdim 64, dstate
+// 128 and 64-token chunks (TMA needs 16-byte aligned x, dy, B, C; the
 // gradient stores are 16-byte vectors).
 inline bool chunk_tc_supported(const KArgs& k) {
   const Dims& d = k.d;
@@ -545,12 +766,28 @@ inline bool chunk_tc_supported(const KArgs& k) {
          aligned16(k.C) && aligned16(k.dx) && d.L < ((int64_t)1 << 31) && d.H * d.P < ((int64_t)1 << 31);
 }
 
+// the four tensor maps of the tensor-core kernels (x, dy, B, C)
+inline bool chunk_tc_maps(const KArgs& k, CUtensorMap* tx, CUtensorMap* tdy, CUtensorMap* tb, CUtensorMap* tc_) {
+  const Dims& d = k.d;
+  return tc::make_map_3d(tx, k.x, d.H * d.P, d.L, d.b) && tc::make_map_3d(tdy, k.dy, d.H * d.P, d.L, d.b) &&
+         tc::make_map_bc(tb, k.B, d.N, d.G, d.L, d.b) && tc::make_map_bc(tc_, k.C, d.N, d.G, d.L, d.b);
+}
+
+inline cudaError_t chunk_states_tc_launch(const KArgs& k, cudaStream_t st) {
+  const Dims& d = k.d;
+  CUtensorMap tx, tdy, tb, tc_;
+  if (!chunk_tc_maps(k, &tx, &tdy, &tb, &tc_)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)StCfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  k_bwd_chunk_states_tc<<<(unsigned)(d.b * d.nc * d.H), kThreads, StCfg::kSmemBytes, st>>>(tx, tdy, tb, tc_, k);
+  return cudaGetLastError();
+}
+
 inline cudaError_t chunk_tc_launch(const KArgs& k, cudaStream_t st) {
   const Dims& d = k.d;
   CUtensorMap tx, tdy, tb, tc_;
-  if (!tc::make_map_3d(&tx, k.x, d.H * d.P, d.L, d.b) || !tc::make_map_3d(&tdy, k.dy, d.H * d.P, d.L, d.b) ||
-      !tc::make_map_bc(&tb, k.B, d.N, d.G, d.L, d.b) || !tc::make_map_bc(&tc_, k.C, d.N, d.G, d.L, d.b))
-    return cudaErrorInvalidValue;
+  if (!chunk_tc_maps(k, &tx, &tdy, &tb, &tc_)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)TcCfg::kSmemBytes);
   if (e != cudaSuccess) return e;
