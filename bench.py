@@ -658,6 +658,20 @@ def bwd_flops(b, L, H, P, N, Q, G=1):
     return 2 * b * H * states, 2 * b * G * cb, 2 * b * H * chunk
 
 
+def bwd_chunk_bytes(b, L, H, P, N, Q, G=1):
+    """Algorithmic HBM bytes of the backward's per-chunk kernel (k_bwd_chunk_tc,
+    or k_bwd_chunk on the CUDA cores), each tensor touched once: per (row,
+    chunk, head) the entering state h_in and its adjoint Lam read (2 P N fp32),
+    x and dy read (2 Qc P bf16), dt read and ddt written (2 Qc fp32), dx
+    written (Qc P fp32) and the head's dB and dC written (2 Qc N fp32); per
+    (row, chunk, group) B and C read (2 Qc N bf16)."""
+    tot = 0
+    for c in range(-(-L // Q)):
+        qc = min(Q, L - c * Q)
+        tot += H * (2 * P * N * 4 + 2 * qc * P * 2 + 2 * qc * 4 + qc * P * 4 + 2 * qc * N * 4) + G * 2 * qc * N * 2
+    return b * tot
+
+
 def bwd_inputs(shape, rank=0):
     host = si.make_inputs(shape, seed=shape.seed + rank)
     g = torch.Generator().manual_seed(shape.seed + 17 + rank)
@@ -717,8 +731,10 @@ def run_reference_bwd(args):
 def run_bwd(args, dist, dev, world, rank):
     """``--op bwd``: the backward ``ssd_bwd`` on c1's layout (b 8, L 2048,
     H 80, P 64, N 128, G 1, bf16) from a random dy, all gradients in fp32.
-    Its kernels run on the CUDA cores, so the roofline is fp32 FMA throughput
-    (bound "alu") on k_bwd_chunk, the dominant kernel."""
+    Its dominant kernel, k_bwd_chunk_tc, forms every contraction with tcgen05
+    MMAs; at speed of light it is bound by its HBM traffic (the chunk states
+    and adjoints read, the gradients written), so the roofline is that
+    traffic over its time against the measured HBM peak."""
     import mamba_ssd_chunked_03_b200 as ssd
     shape = BWD_SHAPE.with_(batch=args.bwd_rows, nheads=args.bwd_heads)
     b, L, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
@@ -784,7 +800,9 @@ def run_bwd(args, dist, dev, world, rank):
     e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev) / E
 
     f_states, f_cb, f_chunk = bwd_flops(b, L, H, P, N, Q, shape.ngroups)
-    achieved = f_chunk / (kernel_ms / 1e3) / 1e12
+    by_chunk = bwd_chunk_bytes(b, L, H, P, N, Q, shape.ngroups)
+    achieved = by_chunk / (kernel_ms / 1e3) / 1e9
+    peaks = load_peaks()
     tokens = b * L
     line = {
         "metric": "SSD bwd tokens/s", "value": tokens * world / (ms_step / 1e3), "unit": "tokens/s",
@@ -795,17 +813,17 @@ def run_bwd(args, dist, dev, world, rank):
                    "l2": "no flush: inputs, gradients and the per-chunk states exceed the 126 MB L2"
                          if (b, H) == (8, 80) else "small case for profiling",
                    "parallelism": "replicas" if world > 1 else "single GPU", "bwd_chunk": Q},
-        "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
-                     "frac": achieved / FP32_PEAK_TFLOPS,
-                     "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz",
-                     "kernel": "k_bwd_chunk", "kernel_ms": kernel_ms,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                     "kernel": "k_bwd_chunk_tc (tcgen05)", "kernel_ms": kernel_ms,
                      "kernel_ms_p10_p50_p90": [per[int(0.1 * (K - 1))], per[int(0.5 * (K - 1))],
                                                per[int(0.9 * (K - 1))]],
-                     "traffic": None, "algorithmic_flops": f_chunk, "states_kernel_flops": f_states,
-                     "cb_kernel_flops": f_cb},
+                     "traffic": None, "algorithmic_bytes": by_chunk, "algorithmic_flops": f_chunk,
+                     "tflops": f_chunk / (kernel_ms / 1e3) / 1e12, "states_kernel_flops": f_states,
+                     "cb_flops_in_kernel": f_cb},
         "e2e": {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": E},
-        "gpu_launches": 6 * K,
+        "gpu_launches": 5 * K,
         "clocks": clock_stats,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -143,21 +143,28 @@ SSD_API size_t ssd_fwd_workspace_size(const ssd_fwd_args* args);
 SSD_API ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream);
 
 /* ssd_fwd for callers that cannot allocate device memory when they call:
- * identical arguments and results (it always runs the generic CUDA-core
- * kernels), but the workspace fields are ignored and no memory is allocated
- * or freed.  Meant for code where no device allocator is reachable or allowed
- * once work has started, such as a plugin inside a host runtime that owns all
- * device memory, or a latency-critical loop that must not call cudaMalloc.
- * The pages describe no such entry point; it has no counterpart there.
+ * identical arguments and results, but the workspace fields are ignored and
+ * no memory is allocated or freed.  Meant for code where no device allocator
+ * is reachable or allowed once work has started, such as a plugin inside a
+ * host runtime that owns all device memory, or a latency-critical loop that
+ * must not call cudaMalloc.  The pages describe no such entry point; it has
+ * no counterpart there.
  *
  * Scratch comes from one fixed 32 MiB device array inside the library.  Every
  * GPU that loads this part of the library keeps that array until the process
- * exits.  Problems whose generic workspace (ssd_fwd_workspace_size with
- * SSD_FLAG_GENERIC) exceeds 32 MiB are rejected with SSD_ERR_WORKSPACE before
- * anything is enqueued.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.  A failed lookup returns SSD_ERR_CUDA.
+ * exits.  The call takes the kernel path ssd_fwd would take (the tensor-core
+ * kernels where they apply, unless SSD_FLAG_GENERIC is set) when that path's
+ * workspace fits the array, else the generic CUDA-core kernels; problems
+ * whose generic workspace (ssd_fwd_workspace_size with SSD_FLAG_GENERIC) also
+ * exceeds 32 MiB are rejected with SSD_ERR_WORKSPACE before anything is
+ * enqueued.  SSD_FLAG_CHECK_SEQ is honoured; SSD_FLAG_TEST_STALL is not.
+ *  - The array's device address is looked up (cudaGetSymbolAddress) with the
+ *    calling device current: on the first call on each device, and again on
+ *    every call made outside stream capture, so that a device reset (which
+ *    reloads the library's device code) is picked up by the next such call.
+ *    A call made while `stream` is capturing uses the address found before;
+ *    make the first call on a device before any capture.  A failed lookup
+ *    returns SSD_ERR_CUDA.
  *  - All calls on a device share the one array and it keeps the last call's
  *    contents; each call rewrites every part it reads (and clears what must
  *    start at zero), so sequential calls are independent.  Calls that overlap
@@ -398,7 +405,16 @@ SSD_API size_t ssd_bwd_workspace_size(const ssd_bwd_args* args);
  * unsupported.  Reads only the size fields; no device work. */
 SSD_API int64_t ssd_bwd_chunk_size(const ssd_bwd_args* args);
 
-/* Enqueue the backward on `stream`: six kernels, no allocation, no memset.
+/* The kernels ssd_bwd runs for these arguments: "tcgen05" when the chunk
+ * states and the per-chunk gradients are formed on the tensor cores (bf16, no
+ * gate, headdim 64, dstate 128, 64-token chunks, x, dy, B, C and dx 16-byte
+ * aligned), "generic" when the CUDA-core kernels run, "invalid" for sizes
+ * ssd_bwd rejects.  Reads sizes and pointer values only; no device work.
+ * Static string. */
+SSD_API const char* ssd_bwd_path(const ssd_bwd_args* args);
+
+/* Enqueue the backward on `stream`: five kernels on the tensor-core path, six
+ * otherwise (ssd_bwd_path), no allocation, no memset.
  * All pointers are device pointers owned by the caller; outputs must not
  * overlap inputs or the workspace.  Returns SSD_OK once enqueued;
  * SSD_ERR_INVALID_ARG for a null required pointer, a bad size or enum, or a

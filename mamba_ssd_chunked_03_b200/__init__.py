@@ -22,11 +22,11 @@ from typing import Optional
 
 import torch
 
-__all__ = ["fwd", "bwd", "BwdArgs", "bwd_workspace_size", "bwd_chunk_size", "ssd_chunked", "make_args",
+__all__ = ["fwd", "bwd", "BwdArgs", "bwd_workspace_size", "bwd_chunk_size", "bwd_path", "ssd_chunked", "make_args",
            "make_bwd_args", "main_kernel", "device_status",
            "conv1d_silu_bwd", "ConvBwdArgs", "causal_conv1d_silu", "step", "StepArgs", "total_decay", "state_fold", "conv1d_silu", "ConvArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
            "SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED", "SSD_ERR_WORKSPACE", "SSD_ERR_CUDA",
-           "SSD_F32", "SSD_BF16", "SSD_FLAG_GENERIC"]
+           "SSD_ERR_TIMEOUT", "SSD_F32", "SSD_BF16", "SSD_FLAG_GENERIC", "SSD_FLAG_CHECK_SEQ", "SSD_FLAG_TEST_STALL"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
 
@@ -130,6 +130,8 @@ def _load() -> ctypes.CDLL:
     L.ssd_bwd_workspace_size.restype = ctypes.c_size_t
     L.ssd_bwd_chunk_size.argtypes = [ctypes.POINTER(BwdArgs)]
     L.ssd_bwd_chunk_size.restype = ctypes.c_int64
+    L.ssd_bwd_path.argtypes = [ctypes.POINTER(BwdArgs)]
+    L.ssd_bwd_path.restype = ctypes.c_char_p
     L.ssd_conv1d_silu_bwd.argtypes = [ctypes.POINTER(ConvBwdArgs), ctypes.c_void_p]
     L.ssd_conv1d_silu_bwd.restype = ctypes.c_int
     L.ssd_conv1d_silu_bwd_workspace_size.argtypes = [ctypes.POINTER(ConvBwdArgs)]
@@ -456,6 +458,15 @@ def bwd_chunk_size(x, B, chunk_size: int = 0) -> int:
     """The chunk length ``ssd_bwd`` uses for these shapes (0: not supported)."""
     a = make_bwd_args(x, None, None, B, None, chunk_size=chunk_size)
     return int(lib.ssd_bwd_chunk_size(ctypes.byref(a)))
+
+
+def bwd_path(x, dy, B, C, z=None, chunk_size: int = 0, dx: Optional[torch.Tensor] = None) -> str:
+    """Kernels ``bwd`` runs for these tensors: "tcgen05" (the chunk states and
+    per-chunk gradients on the tensor cores) or "generic" (CUDA cores)."""
+    a = make_bwd_args(x, None, None, B, C, dy=dy, chunk_size=chunk_size)
+    a.z = _ptr(z)
+    a.dx = _ptr(dx)
+    return lib.ssd_bwd_path(ctypes.byref(a)).decode()
 
 
 def bwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,

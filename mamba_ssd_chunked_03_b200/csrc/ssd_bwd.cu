@@ -39,6 +39,12 @@ extern "C" SSD_API int64_t ssd_bwd_chunk_size(const ssd_bwd_args* a) {
   return ssd::bwd::plan(a, &pl) == SSD_OK ? pl.d.Q : 0;
 }
 
+extern "C" SSD_API const char* ssd_bwd_path(const ssd_bwd_args* a) {
+  ssd::bwd::Plan pl;
+  if (ssd::bwd::plan(a, &pl) != SSD_OK) return "invalid";
+  return a->dtype == SSD_BF16 && ssd::bwd::chunk_tc_supported(ssd::bwd::make_kargs(a, pl)) ? "tcgen05" : "generic";
+}
+
 extern "C" SSD_API ssd_status ssd_bwd(const ssd_bwd_args* a, void* stream) {
   CudaLaunch launch{static_cast<cudaStream_t>(stream)};
   return ssd::bwd::run(a, launch);

@@ -1,6 +1,6 @@
 """Cases, inputs and the comparison rule shared by the backward tests (the
 host emulation in ``test_bwd_emu_cpu.py`` and the GPU parity tests in
-``test_zzz_bwd_gpu.py``)."""
+``test_bwd_gpu.py``)."""
 import numpy as np
 import torch
 

@@ -9,7 +9,7 @@ threads: a shared-memory race aborts), and fills outputs, workspace and
 shared memory with NaN first, so a value read before it was written shows up.
 Each block's threads also run in reverse order once, which exposes a missing
 barrier in the other direction.  Planted mistakes in a copy of the kernels
-must be caught.  The GPU parity tests (``test_zzz_bwd_gpu.py``) run the same
+must be caught.  The GPU parity tests (``test_bwd_gpu.py``) run the same
 kernels compiled by nvcc."""
 import os
 import re

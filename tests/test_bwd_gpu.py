@@ -5,8 +5,10 @@ by nvcc on the GPU, plus sizes only a GPU finishes quickly: a mid-size bf16
 problem and a packed one compared in full, and the benchmark's c1 layout
 (b 8, L 2048, H 80, P 64, N 128, bf16) at full size compared on one batch
 row: every gradient of a row except dA and dD depends on that row's inputs
-only, and dA, dD (sums over rows) are compared at the smaller sizes.  The
-file name sorts it after every other GPU file."""
+only, and dA, dD (sums over rows) are compared at the smaller sizes.  bf16
+calls at headdim 64, dstate 128 without a gate run the tensor-core kernels
+(k_bwd_chunk_states_tc, k_bwd_chunk_tc); the others the CUDA-core ones, so
+both are held to the same tolerances here."""
 import numpy as np
 import pytest
 import torch
@@ -171,3 +173,36 @@ def test_backward_with_ids_out_of_order():
     from bwd_cases import out_of_order_case
     d, dy, dfinal, chunk = out_of_order_case()
     compare(_gpu_bwd(d, dy, dfinal, chunk), oracle_bwd(d, dy, dfinal))
+
+
+TC_EDGE = [
+    # b, L, H, P, N, G, dtype, h0, dfinal, has_D, per-row lengths (packed) or None
+    (1, 200, 4, 64, 128, 2, "bf16", 0.3, True, False, None),      # ragged last chunk (8 tokens), no D
+    (2, 65, 2, 64, 128, 1, "bf16", 0.0, True, True, None),        # one full chunk and one token
+    (1, 300, 4, 64, 128, 2, "bf16", 0.0, False, True, [[1, 63, 1, 100, 135]]),  # one-token sequences, a
+                                                                   # boundary on a chunk edge
+]
+
+
+@pytest.mark.parametrize("case", TC_EDGE, ids=lambda c: f"L{c[1]}_H{c[2]}_G{c[5]}_{'packed' if c[10] else 'dense'}")
+def test_tensor_core_backward_edge_cases(case):
+    b, L, H, P, N, G, dtype, h0, with_df, has_D, lengths = case
+    d = inputs(b, L, H, P, N, G, dtype, h0, None, seed=L + H, has_D=has_D, lengths=lengths)
+    g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    dy = dy_like(b, L, H, P, torch.bfloat16, L + 1)
+    assert ssd.bwd_path(g["x"], dy.cuda(), g["B"], g["C"]) == "tcgen05"
+    dfinal = dfinal_like(b, H, P, N, L + 2) if with_df else None
+    compare(_gpu_bwd(d, dy, dfinal), oracle_bwd(d, dy, dfinal))
+
+
+def test_tensor_core_dinitial_only_matches_a_full_call():
+    b, L, H, P, N, G = 2, 300, 4, 64, 128, 2
+    d = inputs(b, L, H, P, N, G, "bf16", 0.2, None, seed=91)
+    g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    dy = dy_like(b, L, H, P, torch.bfloat16, 92).cuda()
+    full = ssd.bwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], dy, initial_states=g["initial_states"],
+                   want_dinitial_states=True)
+    only = ssd.bwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], dy, initial_states=g["initial_states"],
+                   want_dinitial_states=True, dinitial_only=True)
+    torch.cuda.synchronize()
+    assert torch.equal(full["dinitial_states"], only["dinitial_states"])

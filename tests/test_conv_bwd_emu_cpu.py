@@ -1,7 +1,7 @@
 """The conv1d + SiLU backward kernels (``csrc/ssd_conv_bwd.cuh``) on the CPU
 through the test-only emulation in ``tests/emu`` (AddressSanitizer + UBSan,
 exact-size buffers, NaN-filled outputs and workspace), against the fp64
-oracle, before any GPU runs them.  ``test_zzz_bwd_gpu.py`` runs the same
+oracle, before any GPU runs them.  ``test_bwd_gpu.py`` runs the same
 cases on the GPU."""
 import pytest
 

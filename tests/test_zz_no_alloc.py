@@ -3,12 +3,14 @@ memory when they call (for instance a plugin inside a host runtime that owns
 all device memory, or a latency-critical loop that must not call cudaMalloc).
 
 It takes the same arguments as ssd_fwd but brings its own scratch: a fixed
-32 MiB device array inside the library.  These tests call it through the C
+32 MiB device array inside the library, and it takes ssd_fwd's kernel path
+when that path's workspace fits the array.  These tests call it through the C
 ABI and compare it with ssd_fwd on several calls in a row (the array keeps
 the previous call's contents, so a stale value would show up in a later
-call), and check that a problem too large for the array is refused without
-touching the outputs.  This file is collected last so that a failure here
-cannot hide other tests in a run that stops at the first failure.
+call), compare a tensor-core call with the oracle, and check that a problem
+too large for the array is refused without touching the outputs.  This file
+is collected last so that a failure here cannot hide other tests in a run
+that stops at the first failure.
 """
 import ctypes
 
@@ -17,7 +19,7 @@ import torch
 
 import mamba_ssd_chunked_03_b200 as ssd
 import ssd_inputs as si
-from gpu_util import TOL, rel_l2, state_err, to_dev
+from gpu_util import TOL, rel_l2, run_oracle, state_err, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -96,3 +98,18 @@ def test_problem_larger_than_the_scratch_is_refused():
     torch.cuda.synchronize()
     assert st == ssd.SSD_ERR_WORKSPACE
     assert bool(torch.isnan(y).all()) and bool(torch.isnan(f).all())
+
+
+def test_tensor_core_path_matches_the_oracle():
+    # two-head tensor-core kernel (N 128, heads per group even), ragged tail, h0
+    s = si.SSDShape("na_tc", 2, 300, 8, 64, 128, 2, 64, "bf16", h0_std=0.2, seed=25)
+    d = si.make_inputs(s)
+    g = to_dev(d)
+    a = ssd.make_args(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], s.chunk_size)
+    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"tcgen05"
+    yr, fr = run_oracle(d)
+    for _ in range(2):  # two calls in a row on the shared array
+        y, f = _noalloc(g, s.chunk_size)
+        y64, f64 = y.double().cpu().numpy(), f.double().cpu().numpy()
+        assert rel_l2(y64, yr) <= TOL["bf16"], rel_l2(y64, yr)
+        assert state_err(f64, fr) <= TOL["bf16"], state_err(f64, fr)
