@@ -358,8 +358,11 @@ typedef struct {
   const void* C;                  /* (b,L,G,N) dtype                                  */
   const float* D;                 /* (H) fp32, or NULL for D = 0                      */
   const float* initial_states;    /* (b,H,P,N) fp32, or NULL = 0                      */
-  const int32_t* seq_idx;         /* (b,L) int32 packed-sequence ids, or NULL; the
-                                     precondition of ssd_fwd_args (not checked)       */
+  const int32_t* seq_idx;         /* (b,L) int32 packed-sequence ids, or NULL.  Any
+                                     change of id between neighbouring tokens starts a
+                                     new sequence (a_t = 0 there); ids need not
+                                     increase or stay in one row, since the backward
+                                     takes no per-sequence final states.              */
   const void* dy;                 /* (b,L,H,P) dtype, dLoss/dy                        */
   const float* dfinal_states;     /* (b,H,P,N) fp32 dLoss/dfinal_states, or NULL = 0.
                                      Not with seq_idx (SSD_ERR_UNSUPPORTED).          */

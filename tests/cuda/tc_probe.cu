@@ -15,9 +15,6 @@
 // modes 0-2 read TMEM with the 16-lane x2 shape, modes 3 and 5 with 32x32b,
 // modes 4 and 6 with 16x256b.
 //
-// tc_probe_mma_rate times 64 back-to-back MMAs (M = 128, K = 16) from one
-// thread: clock cycles to issue them and until all have completed.
-//
 // tc_probe_layout records the lane / column maps of the 16x256b load, the
 // 16x128b store and the 8 x 8 transpose, so the tests can check them exactly.
 #include <cuda_bf16.h>
@@ -270,128 +267,3 @@ extern "C" __attribute__((visibility("default"))) int tc_probe_layout(uint32_t* 
   return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
 
-// variant: 0 A in TMEM, N = 64 (B K-major); 1 A in TMEM, N = 128; 2 A in TMEM,
-// N = 256; 3 A in shared memory (K-major), N = 64; 4 A in TMEM, N = 192
-// (B MN-major over three 64-wide blocks 8 KB apart)
-// load (warps 4-7, 300 bounded iterations each, alongside the MMAs): bit 0
-// TMEM loads (32x32b.x32, columns 320..351), bit 1 shared-memory transposing
-// loads and stores (bytes 32768..49151), bit 2 TMEM stores (columns 320..351),
-// bit 3 fp32 FMA chains (eight independent per thread).
-// variant 5 issues the fused kernel's per-chunk sequence four times: 4 x N = 64
-// into columns 0.., 4 x N = 128 into columns 64.., 8 x N = 64 into columns 0..,
-// with B descriptors stepping through shared memory as there.
-__global__ void __launch_bounds__(256) rate_kernel(int variant, int load, long long* __restrict__ out) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t bar;
-  __shared__ uint32_t tmem_base;
-  __shared__ int abort_flag;
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  for (int i = tid; i < 49152 / 16; i += 256) reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
-  if (tid == 0) {
-    mbar_init(&bar, 1);
-    abort_flag = 0;
-    fence_mbar_init();
-  }
-  fence_proxy_async_smem();
-  __syncthreads();
-  if (warp == 0) {
-    tmem_alloc(&tmem_base, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base;
-  if (warp < 4) {  // A columns 256..263: zeros
-    uint32_t r[32];
-    for (int c = 0; c < 32; ++c) r[c] = 0;
-    SSD_TMEM_ST_32x32b_X32(tmem + ((uint32_t)(32 * warp) << 16) + 256, r);
-  }
-  tmem_wait_st();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (tid == 0) {
-    const uint32_t s0 = smem_u32(smem);
-    const int N = variant == 1 ? 128 : variant == 2 ? 256 : variant == 4 ? 192 : 64;
-    const uint64_t bd = variant == 4 ? sw128_desc(s0 + 16384, 8192, 1024) : sw128_desc(s0 + 16384, 16, 1024);
-    const uint64_t ad = sw128_desc(s0, 16, 1024);
-    const uint32_t id = idesc_bf16(128, N, 0, variant == 4);
-    const long long t0 = clock64();
-    if (variant == 5) {
-      const uint32_t id64 = idesc_bf16(128, 64, 0, 0), id128 = idesc_bf16(128, 128, 0, 1);
-#pragma unroll 1
-      for (int rep = 0; rep < 4; ++rep) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ts(tmem, tmem + 256, sw128_desc(s0 + 16384 + kk * 32, 16, 1024), id64, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ts(tmem + 64, tmem + 256, sw128_desc(s0 + 24576 + kk * 2048, 8192, 1024), id128, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem, tmem + 256, sw128_desc(s0 + 16384 + (kk >> 2) * 4096 + (kk & 3) * 32, 16, 1024), id64, 1);
-      }
-    } else if (variant == 3) {
-#pragma unroll
-      for (int k = 0; k < 64; ++k) mma_bf16_ss(tmem, ad, bd, id, k > 0);
-    } else {
-#pragma unroll
-      for (int k = 0; k < 64; ++k) mma_bf16_ts(tmem, tmem + 256, bd, id, k > 0);
-    }
-    const long long t1 = clock64();
-    mma_commit(&bar);
-    const bool ok = mbar_wait(&bar, 0, &abort_flag, 1000000000ull);
-    const long long t2 = clock64();
-    out[0] = t1 - t0;
-    out[1] = ok ? t2 - t0 : -1;
-  } else if (warp >= 4 && load) {
-    const uint32_t tq = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 320;
-    const uint32_t sbase = smem_u32(smem) + 32768 + (warp - 4) * 4096;
-    uint32_t acc = 0, r[32];
-    for (int c = 0; c < 32; ++c) r[c] = c;
-    for (int it = 0; it < 300; ++it) {
-      if (load & 1) {
-        SSD_TMEM_LD_32x32b_X32(tq, r);
-        SSD_TMEM_WAIT_LD_32(r);
-        acc ^= r[it & 31];
-      }
-      if (load & 4) {
-        SSD_TMEM_ST_32x32b_X32(tq, r);
-        tmem_wait_st();
-      }
-      if (load & 8) {
-        float f[8];
-        for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(r[k]) * 1e-30f;
-#pragma unroll 1
-        for (int k2 = 0; k2 < 16; ++k2)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) f[k] = fmaf(f[k], 0.999f, 1e-7f);
-        for (int k = 0; k < 8; ++k) acc ^= __float_as_uint(f[k]);
-      }
-      if (load & 2) {
-        uint32_t v[4];
-        for (int k = 0; k < 4; ++k) {
-          ldmatrix_x4_trans(sbase + 1024 * k + (lane & 7) * 128 + ((lane >> 3) << 4), v);
-          acc ^= v[0] ^ v[3];
-          stmatrix_x4_trans(sbase + 1024 * k + (lane & 7) * 128 + ((lane >> 3) << 4), v);
-        }
-      }
-    }
-    out[2 + (tid - 128)] = acc;
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 512);
-}
-
-extern "C" __attribute__((visibility("default"))) int tc_probe_mma_rate(int variant, int load, long long* out,
-                                                                        void* stream) {
-  if (variant < 0 || variant > 5 || load < 0 || load > 15) return 1;
-  const size_t smem = 49152 + 1024;
-  if (cudaFuncSetAttribute(rate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return 2;
-  rate_kernel<<<1, 256, smem, static_cast<cudaStream_t>(stream)>>>(variant, load, out);
-  return cudaGetLastError() == cudaSuccess ? 0 : 3;
-}

@@ -97,24 +97,3 @@ def test_fragment_layouts():
                  for ni, n in enumerate(names)}
         raise AssertionError(f"{len(bad)} mismatches: {first}")
 
-
-def test_mma_issue_rate_is_recorded():
-    """Times 64 back-to-back MMAs per shape, alone and beside other warps'
-    TMEM or shared-memory traffic (a measurement, printed; the test only
-    checks that every variant completed)."""
-    lib = ctypes.CDLL(LIB)
-    lib.tc_probe_mma_rate.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
-    names = ["A tmem N64", "A tmem N128", "A tmem N256", "A smem N64", "A tmem N192 (B MN)",
-             "chunk sequence"]
-    loads = {0: "alone", 1: "tmem ld", 2: "smem ldst", 4: "tmem st", 8: "fma", 15: "all"}
-    for v, name in enumerate(names):
-        for ld, lname in loads.items():
-            if ld and v not in (0, 5):
-                continue
-            out = torch.zeros(2 + 128, dtype=torch.int64, device="cuda")
-            for _ in range(3):  # warm the instruction cache
-                assert lib.tc_probe_mma_rate(v, ld, out.data_ptr(), torch.cuda.current_stream().cuda_stream) == 0
-            torch.cuda.synchronize()
-            issue, done = (int(t) for t in out[:2].cpu())
-            assert done > 0, name
-            print(f"mma rate {name} [{lname}]: issue {issue / 64:.1f} cycles/MMA, complete {done / 64:.1f} cycles/MMA")
