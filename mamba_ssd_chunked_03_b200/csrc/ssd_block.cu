@@ -11,7 +11,13 @@
 // 16 of fp32) over a strip of kStrip tokens; its filter taps, bias and the K-1
 // previous inputs (with their sequence ids) stay in registers while it walks
 // the strip.  Consecutive threads take consecutive channel vectors, so every
-// load and store of a warp is contiguous.
+// load and store of a warp is contiguous.  The strip is read kGroup tokens at
+// a time, all of a group's loads issued before its first output is formed, so
+// that each thread keeps several loads in flight; the channel pairs are
+// computed in packed fp32x2 arithmetic, and SiLU takes the hardware exponential
+// and an approximate divide: a relative error of a few millionths, far below
+// the bf16 rounding of the output, for a third of the instructions of the
+// correctly rounded forms (which left the kernel issue-bound).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -22,8 +28,10 @@ namespace ssd {
 namespace {
 
 constexpr int kStrip = 32;        // tokens per thread
+constexpr int kGroup = 4;         // tokens loaded before any of them is used
 constexpr int kConvThreads = 128;
 constexpr int kMaxWidth = 4;
+constexpr int kVec = 4;           // channels per thread
 
 struct ConvArgs {
   int64_t L, C;
@@ -34,110 +42,128 @@ struct ConvArgs {
   void* out;
 };
 
+// A thread's 4 channels as they sit in memory, and as two fp32 pairs.
 template <typename T>
 struct Vec;
 template <>
 struct Vec<__nv_bfloat16> {
-  static constexpr int n = 4;  // 8-byte vectors: half the registers of 16-byte ones, twice the resident warps
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[4]) {
-    const uint2 q = *reinterpret_cast<const uint2*>(p);
-    const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&q.x);
-    const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162*>(&q.y);
-    v[0] = __low2float(h0);
-    v[1] = __high2float(h0);
-    v[2] = __low2float(h1);
-    v[3] = __high2float(h1);
+  using Raw = uint2;  // 8 bytes: half the registers of 8-channel vectors, twice the resident warps
+  static __device__ __forceinline__ float2 pair(uint32_t q) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q));
   }
-  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[4]) {
-    const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
-    const __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
-    *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<const uint32_t*>(&h0),
-                                              *reinterpret_cast<const uint32_t*>(&h1));
+  static __device__ __forceinline__ uint32_t pack(float2 v) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+    return *reinterpret_cast<const uint32_t*>(&h);
   }
+  static __device__ __forceinline__ void unpack(Raw q, float2 (&v)[2]) { v[0] = pair(q.x), v[1] = pair(q.y); }
+  static __device__ __forceinline__ Raw pack(const float2 (&v)[2]) { return make_uint2(pack(v[0]), pack(v[1])); }
 };
 template <>
 struct Vec<float> {
-  static constexpr int n = 4;
-  static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
-    const float4 q = *reinterpret_cast<const float4*>(p);
-    v[0] = q.x, v[1] = q.y, v[2] = q.z, v[3] = q.w;
+  using Raw = float4;
+  static __device__ __forceinline__ void unpack(Raw q, float2 (&v)[2]) {
+    v[0] = make_float2(q.x, q.y), v[1] = make_float2(q.z, q.w);
   }
-  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
-    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-  }
+  static __device__ __forceinline__ Raw pack(const float2 (&v)[2]) { return make_float4(v[0].x, v[0].y, v[1].x, v[1].y); }
 };
 
-__device__ __forceinline__ float silu(float v) { return v / (1.f + expf(-v)); }
+__device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.f + __expf(-v)); }
 
-// grid: (channel vectors / kConvThreads, token strips, batch rows)
-template <typename T, int K>
+// grid: (channel vectors / kConvThreads, token strips, batch rows).  SEQ: the
+// row carries sequence ids (taps into an earlier sequence add nothing).
+template <typename T, int K, bool SEQ>
 __global__ void __launch_bounds__(kConvThreads) k_conv1d_silu(const ConvArgs a) {
-  constexpr int V = Vec<T>::n;
-  const int64_t c0 = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) * V;
+  using Raw = typename Vec<T>::Raw;
+  constexpr int NP = kVec / 2;  // channel pairs per thread
+  const int64_t c0 = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) * kVec;
   if (c0 >= a.C) return;
   const int64_t b = blockIdx.z;
   const int64_t t0 = (int64_t)blockIdx.y * kStrip;
-  const T* u = static_cast<const T*>(a.u) + b * a.L * a.C + c0;
-  T* out = static_cast<T*>(a.out) + b * a.L * a.C + c0;
-  const int32_t* seq = a.seq ? a.seq + b * a.L : nullptr;
-  float w[V][K], bias[V];
+  const int64_t rs = a.C / kVec;  // a token row, in vectors
+  const Raw* __restrict__ u = reinterpret_cast<const Raw*>(static_cast<const T*>(a.u) + b * a.L * a.C + c0);
+  Raw* __restrict__ out = reinterpret_cast<Raw*>(static_cast<T*>(a.out) + b * a.L * a.C + c0);
+  const int32_t* __restrict__ seq = SEQ ? a.seq + b * a.L : nullptr;
+  float2 w[NP][K], bias[NP];
 #pragma unroll
-  for (int v = 0; v < V; ++v) {
-    bias[v] = a.bias ? a.bias[c0 + v] : 0.f;
+  for (int p = 0; p < NP; ++p) {
+    const int64_t c = c0 + 2 * p;
+    bias[p] = a.bias ? make_float2(a.bias[c], a.bias[c + 1]) : make_float2(0.f, 0.f);
 #pragma unroll
-    for (int k = 0; k < K; ++k) w[v][k] = a.w[(c0 + v) * K + k];
+    for (int k = 0; k < K; ++k) w[p][k] = make_float2(a.w[c * K + k], a.w[(c + 1) * K + k]);
   }
   // win[j]: the input at token t-(K-1)+j for j < K-1 (zero before token 0),
   // with its sequence id (-1 there)
-  float win[K > 1 ? K - 1 : 1][V];
+  float2 win[K > 1 ? K - 1 : 1][NP];
   int wseq[K > 1 ? K - 1 : 1];
 #pragma unroll
   for (int j = 0; j < K - 1; ++j) {
     const int64_t s = t0 - (K - 1) + j;
     if (s >= 0) {
-      Vec<T>::load(u + s * a.C, win[j]);
-      wseq[j] = seq ? seq[s] : 0;
+      Vec<T>::unpack(__ldg(u + s * rs), win[j]);
+      wseq[j] = SEQ ? seq[s] : 0;
     } else {
 #pragma unroll
-      for (int v = 0; v < V; ++v) win[j][v] = 0.f;
+      for (int p = 0; p < NP; ++p) win[j][p] = make_float2(0.f, 0.f);
       wseq[j] = -1;
     }
   }
   const int64_t t_end = t0 + kStrip < a.L ? t0 + kStrip : a.L;
-  for (int64_t t = t0; t < t_end; ++t) {
-    float cur[V];
-    Vec<T>::load(u + t * a.C, cur);
-    const int st = seq ? seq[t] : 0;
-    float acc[V];
+  for (int64_t tg = t0; tg < t_end; tg += kGroup) {
+    Raw raw[kGroup];
+    int sq[kGroup];
 #pragma unroll
-    for (int v = 0; v < V; ++v) acc[v] = fmaf(w[v][K - 1], cur[v], bias[v]);
-#pragma unroll
-    for (int j = 0; j < K - 1; ++j) {
-      if (wseq[j] == st) {  // same sequence (ids are >= 0; a tap before token 0 carries -1)
-#pragma unroll
-        for (int v = 0; v < V; ++v) acc[v] = fmaf(w[v][j], win[j][v], acc[v]);
+    for (int g = 0; g < kGroup; ++g) {
+      if (tg + g < t_end) {
+        raw[g] = __ldcs(u + (tg + g) * rs);
+        sq[g] = SEQ ? seq[tg + g] : 0;
       }
     }
 #pragma unroll
-    for (int v = 0; v < V; ++v) acc[v] = silu(acc[v]);
-    Vec<T>::store(out + t * a.C, acc);
+    for (int g = 0; g < kGroup; ++g) {
+      if (tg + g < t_end) {
+        float2 cur[NP], acc[NP];
+        Vec<T>::unpack(raw[g], cur);
 #pragma unroll
-    for (int j = 0; j + 1 < K - 1; ++j) {
+        for (int p = 0; p < NP; ++p) acc[p] = __ffma2_rn(w[p][K - 1], cur[p], bias[p]);
 #pragma unroll
-      for (int v = 0; v < V; ++v) win[j][v] = win[j + 1][v];
-      wseq[j] = wseq[j + 1];
+        for (int j = 0; j < K - 1; ++j) {
+          // same sequence (ids are >= 0; a tap before token 0 carries -1 and a zero input)
+          if (!SEQ || wseq[j] == sq[g]) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) acc[p] = __ffma2_rn(w[p][j], win[j][p], acc[p]);
+          }
+        }
+#pragma unroll
+        for (int p = 0; p < NP; ++p) acc[p] = make_float2(silu(acc[p].x), silu(acc[p].y));
+        __stcs(out + (tg + g) * rs, Vec<T>::pack(acc));
+#pragma unroll
+        for (int j = 0; j + 1 < K - 1; ++j) {
+#pragma unroll
+          for (int p = 0; p < NP; ++p) win[j][p] = win[j + 1][p];
+          wseq[j] = wseq[j + 1];
+        }
+        if (K > 1) {
+#pragma unroll
+          for (int p = 0; p < NP; ++p) win[K > 1 ? K - 2 : 0][p] = cur[p];
+          wseq[K > 1 ? K - 2 : 0] = sq[g];
+        }
+      }
     }
-    if (K > 1) {
-#pragma unroll
-      for (int v = 0; v < V; ++v) win[K > 1 ? K - 2 : 0][v] = cur[v];
-      wseq[K > 1 ? K - 2 : 0] = st;
-    }
+  }
+}
+
+template <typename T, bool SEQ>
+void launch_width(const ConvArgs& a, int width, dim3 grid, cudaStream_t st) {
+  switch (width) {
+    case 1: k_conv1d_silu<T, 1, SEQ><<<grid, kConvThreads, 0, st>>>(a); break;
+    case 2: k_conv1d_silu<T, 2, SEQ><<<grid, kConvThreads, 0, st>>>(a); break;
+    case 3: k_conv1d_silu<T, 3, SEQ><<<grid, kConvThreads, 0, st>>>(a); break;
+    default: k_conv1d_silu<T, 4, SEQ><<<grid, kConvThreads, 0, st>>>(a); break;
   }
 }
 
 template <typename T>
 cudaError_t launch_conv(const ssd_conv_args* p, cudaStream_t st) {
-  constexpr int V = Vec<T>::n;
   ConvArgs a;
   a.L = p->seqlen;
   a.C = p->channels;
@@ -146,14 +172,12 @@ cudaError_t launch_conv(const ssd_conv_args* p, cudaStream_t st) {
   a.bias = p->bias;
   a.seq = p->seq_idx;
   a.out = p->out;
-  const dim3 grid((unsigned)((p->channels / V + kConvThreads - 1) / kConvThreads),
+  const dim3 grid((unsigned)((p->channels / kVec + kConvThreads - 1) / kConvThreads),
                   (unsigned)((p->seqlen + kStrip - 1) / kStrip), (unsigned)p->batch);
-  switch (p->width) {
-    case 1: k_conv1d_silu<T, 1><<<grid, kConvThreads, 0, st>>>(a); break;
-    case 2: k_conv1d_silu<T, 2><<<grid, kConvThreads, 0, st>>>(a); break;
-    case 3: k_conv1d_silu<T, 3><<<grid, kConvThreads, 0, st>>>(a); break;
-    default: k_conv1d_silu<T, 4><<<grid, kConvThreads, 0, st>>>(a); break;
-  }
+  if (a.seq)
+    launch_width<T, true>(a, (int)p->width, grid, st);
+  else
+    launch_width<T, false>(a, (int)p->width, grid, st);
   return cudaGetLastError();
 }
 

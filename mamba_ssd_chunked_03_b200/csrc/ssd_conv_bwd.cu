@@ -1,6 +1,7 @@
 // ssd_conv1d_silu_bwd and its workspace query: the kernels of
 // ssd_conv_bwd.cuh, launched on the caller's stream.
 #include <cuda_bf16.h>
+#include <cuda_pipeline.h>
 #include <cuda_runtime.h>
 
 #include "ssd.h"
@@ -12,6 +13,9 @@ struct CudaLaunch {
   cudaStream_t stream;
   bool operator()(void (*kern)(ssd::convbwd::KArgs), unsigned grid, size_t smem, const ssd::convbwd::KArgs& k) const {
     if (grid == 0) return true;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return false;
     kern<<<grid, ssd::convbwd::kThreads, smem, stream>>>(k);
     return cudaGetLastError() == cudaSuccess;
   }

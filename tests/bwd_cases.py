@@ -108,6 +108,10 @@ CONV_CASES = [
     ("f32_one_token", (1, 1, 8, 4), "f32", None, True),
     ("f32_K2_packed_on_a_strip_edge", (1, 64, 8, 2), "f32", [[32, 32]], True),
     ("bf16_K4_c1_channels", (1, 100, 5376, 4), "bf16", None, True),
+    # 64-token bf16 strips with a ragged last one; a partial second channel block
+    ("bf16_K4_strips", (2, 150, 264, 4), "bf16", None, True),
+    # sequence starts on either side of the 64-token strip edges (rows staged by 16-byte copies)
+    ("bf16_K4_packed_strips", (1, 200, 16, 4), "bf16", [[63, 2, 65, 70]], False),
 ]
 
 

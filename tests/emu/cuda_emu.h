@@ -59,6 +59,16 @@ inline void __syncthreads() { swapcontext(emu::g_self, &emu::g_sched); }
 
 #define SSD_DYN_SMEM(name) float* name = emu::g_smem
 
+// The fast-math intrinsics, at host precision.
+inline float __expf(float v) { return std::exp(v); }
+inline float __fdividef(float a, float b) { return a / b; }
+
+// The cuda_pipeline primitives: an asynchronous copy to shared memory lands
+// at once here; the wait and the CTA barrier after it order it as on a GPU.
+inline void __pipeline_memcpy_async(void* dst, const void* src, size_t n) { std::memcpy(dst, src, n); }
+inline void __pipeline_commit() {}
+inline void __pipeline_wait_prior(size_t) {}
+
 // bf16 is the upper half of an IEEE binary32: widening is a shift.
 struct __nv_bfloat16 {
   uint16_t bits;

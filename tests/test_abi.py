@@ -398,9 +398,12 @@ def test_conv_bwd_rejects_bad_arguments(kw, status):
 
 def test_conv_bwd_workspace_size():
     size = lambda **kw: ssd.lib.ssd_conv1d_silu_bwd_workspace_size(ctypes.byref(_conv_bwd_args(**kw)))
-    # per (row, strip of 32 tokens) and channel: K dweight partials and one dbias partial, fp32
-    assert size() == 2 * 2 * 64 * 5 * 4
-    assert size(seqlen=65) == 2 * 3 * 64 * 5 * 4
+    # per (row, strip) and channel: K dweight partials and one dbias partial, fp32;
+    # a strip is 64 tokens of bf16 inputs and 32 of fp32 ones
+    assert size() == 2 * 1 * 64 * 5 * 4
+    assert size(seqlen=65) == 2 * 2 * 64 * 5 * 4
+    assert size(dtype=ssd.SSD_F32) == 2 * 2 * 64 * 5 * 4
+    assert size(dtype=ssd.SSD_F32, seqlen=65) == 2 * 3 * 64 * 5 * 4
     assert size(batch=0) == 0 and size(width=5) == 0
     assert ssd.lib.ssd_conv1d_silu_bwd(None, None) == ssd.SSD_ERR_INVALID_ARG
 
