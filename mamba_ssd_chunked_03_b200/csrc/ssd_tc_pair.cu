@@ -74,14 +74,16 @@ struct PairCfg {
   static constexpr int NS = 128, NB = 2;
   static constexpr int kThreads = 896;
   static constexpr uint32_t kTile = 8192;
-  static constexpr int kXSlots = 8;  // x ring (power of two)
-  static constexpr uint32_t oX = 0;                         // [8 slots][2 heads] x -> y, in place
-  static constexpr uint32_t oW = oX + 2 * kXSlots * kTile;  // [2] W' tiles
-  static constexpr uint32_t oB = oW + 2 * kTile;            // [2] B, 2 n-blocks each
-  static constexpr uint32_t oC = oB + 2 * NB * kTile;       // [2] C, 2 n-blocks each
-  static constexpr uint32_t oDt = oC + 2 * NB * kTile;      // [8] dt boxes: 64 tokens x 4 heads fp32
+  // ring depths (steps of lead): x tiles (y is staged in place), W' + B, C, dt
+  static constexpr int kXSlots = 8, kWbSlots = 2, kCSlots = 2, kDtSlots = 8;
+  static constexpr int kWbMax = kWbSlots > 4 ? kWbSlots : 4;  // the state-only pass runs B 4 deep
+  static constexpr uint32_t oX = 0;                                // [slots][2 heads] x -> y, in place
+  static constexpr uint32_t oW = oX + 2 * kXSlots * kTile;         // [slots] W' tiles
+  static constexpr uint32_t oB = oW + kWbSlots * kTile;            // [slots] B, 2 n-blocks each
+  static constexpr uint32_t oC = oB + kWbSlots * NB * kTile;       // [slots] C, 2 n-blocks each
+  static constexpr uint32_t oDt = oC + kCSlots * NB * kTile;       // [slots] dt boxes: 64 tokens x 4 heads fp32
   static constexpr uint32_t kDtBox = 64 * 16;
-  static constexpr uint32_t oEnd = oDt + 8 * kDtBox;
+  static constexpr uint32_t oEnd = oDt + kDtSlots * kDtBox;
   static constexpr uint32_t kSmemBytes = oEnd + 1024;
   // TMEM (M = 128 layout, row = lane = 64 j + p for head h0 + j):
   //   Yd^T[2] fp32, 64 columns (t) each;  S fp32, 128 columns (n);
@@ -91,23 +93,35 @@ struct PairCfg {
 
 constexpr int kPairMaxSeg = 32;  // segments (pairs touched) per CTA, at most
 
+// Slot and phase parity of step c in a ring of n buffers.
+template <int n>
+__device__ __forceinline__ int ring_slot(int c) {
+  return c % n;
+}
+template <int n>
+__device__ __forceinline__ uint32_t ring_par(int c) {
+  return (uint32_t)(c / n) & 1u;
+}
+
 // Ring barriers are indexed like the buffers they guard, so no barrier can
 // complete a second phase before every waiter has seen the first.  A warp
 // arrives once (lane 0, after each lane's own wait or fence and a __syncwarp,
 // which orders the warp's accesses before that release), so the counts below
 // are in warps: 32 times fewer shared-memory atomics than per-thread arrivals.
 struct __align__(16) PairSmem {
-  uint64_t full_x[8], x_empty[8];        // x ring: TMA landed / scaled (state-only pass)
-  uint64_t full_dt[8];                   // dt ring (the scan warp's own)
-  uint64_t full_wb[2], full_c[2];        // W' + B, C of a chunk landed
+  uint64_t full_x[PairCfg::kXSlots], x_empty[PairCfg::kXSlots];  // x ring: TMA landed / scaled (state-only pass)
+  uint64_t full_dt[PairCfg::kDtSlots];   // dt ring (the scan warp's own)
+  uint64_t full_wb[PairCfg::kWbMax];     // W' + B of a chunk landed (state-only pass: B)
+  uint64_t wb_free[PairCfg::kWbMax];     // ... and read by its MMAs
+  uint64_t full_c[PairCfg::kCSlots], c_free[PairCfg::kCSlots];  // C of a chunk landed / read
   uint64_t scan_full[4], scan_empty[4];  // scan results of a chunk ready / consumed
   uint64_t xp_ready[4];                  // X'^T of a chunk in TMEM
-  uint64_t s_full[2];                    // S of a chunk in TMEM (its W' and B reads are done)
+  uint64_t s_full[2];                    // S of a chunk in TMEM
   uint64_t s_free[2];                    // S of a chunk read out by the state warps
   uint64_t mma_done[2];                  // every MMA of a chunk done: Yd final, C free
   uint64_t h_ready[2];                   // bf16 state for a chunk written to TMEM
   uint64_t acc_free[2];                  // Yd of a chunk read out by the epilogue
-  uint64_t y_staged[8];                  // y of a chunk written over its x slot
+  uint64_t y_staged[PairCfg::kXSlots];   // y of a chunk written over its x slot
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -127,15 +141,20 @@ static_assert(offsetof(PairSmem, u) % 16 == 0 && offsetof(PairSmem, v) % 16 == 0
 static_assert(PairCfg::kSmemBytes + sizeof(PairSmem) <= 227 * 1024, "shared memory per CTA");
 
 // Position of one of a CTA's step streams (each role walks its steps in
-// order): segment k, chunk c.  next() moves to the following step.
+// order): segment k, chunk c.  next() moves to the following step.  kRev (the
+// state-only pass, which has one segment) walks the segment's chunks from its
+// last to its first.
+template <bool kRev>
 struct PairCursor {
   int k, c;
   __device__ __forceinline__ void start(const PairSmem& s) {
     k = 0;
-    c = s.seg_c0[0];
+    c = kRev ? s.seg_c0[0] + s.seg_len[0] - 1 : s.seg_c0[0];
   }
   __device__ __forceinline__ void next(const PairSmem& s) {
-    if (++c == s.seg_c0[k] + s.seg_len[k] && k + 1 < s.nseg) {
+    if (kRev) {
+      --c;
+    } else if (++c == s.seg_c0[k] + s.seg_len[k] && k + 1 < s.nseg) {
       ++k;
       c = s.seg_c0[k];
     }
@@ -146,7 +165,11 @@ struct PairCursor {
 // segment of its range that ends inside a pair (there is at most one: the
 // head of its last pair), runs it from a zero state with x and B alone (no
 // W', C, y) and leaves the end state in handoff and the segment's total decay
-// per head in seg_decay.
+// per head in seg_decay.  It walks the segment from its last chunk to its
+// first and scales each token's x by its decay to the segment's end (a factor
+// of at most one, known as the walk goes: the chunks after it are done), so
+// the end state is one MMA accumulation, S += X''^T B, that stays in tensor
+// memory until the last chunk; no step waits for the state warps.
 template <bool kStateOnly>
 __global__ void __launch_bounds__(896, 1)
     k_ssd_fwd_pair(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
@@ -154,6 +177,13 @@ __global__ void __launch_bounds__(896, 1)
                    const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_dt,
                    const FastArgs a) {
   using K = PairCfg;
+  using Cursor = PairCursor<kStateOnly>;
+  // B (with W') ring depth.  The state-only pass needs no W' or C: its B ring
+  // takes their space and runs 4 steps ahead, since its steps wait on nothing
+  // else.
+  constexpr int kBR = kStateOnly ? 4 : PairCfg::kWbSlots;
+  static_assert(4 * PairCfg::NB * PairCfg::kTile <= PairCfg::oDt - PairCfg::oW, "state-only B ring");
+  constexpr uint32_t oBr = kStateOnly ? PairCfg::oW : PairCfg::oB;
   constexpr int NS = K::NS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -165,12 +195,16 @@ __global__ void __launch_bounds__(896, 1)
   const int nc = (int)a.nc;
 
   if (tid == 0) {
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < K::kXSlots; ++i) {
       mbar_init(&s.full_x[i], 1);
       // the state-only pass stores no y: the x scalers (state warps) free the slot
       mbar_init(&s.x_empty[i], 16);
       mbar_init(&s.y_staged[i], 8);
-      mbar_init(&s.full_dt[i], 1);
+    }
+    for (int i = 0; i < K::kDtSlots; ++i) mbar_init(&s.full_dt[i], 1);
+    for (int i = 0; i < K::kCSlots; ++i) {
+      mbar_init(&s.full_c[i], 1);
+      mbar_init(&s.c_free[i], 1);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&s.scan_full[i], 1);
@@ -178,9 +212,11 @@ __global__ void __launch_bounds__(896, 1)
       mbar_init(&s.scan_empty[i], kStateOnly ? 16 : 8 + 16);
       mbar_init(&s.xp_ready[i], 16);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < K::kWbMax; ++i) {
       mbar_init(&s.full_wb[i], 1);
-      mbar_init(&s.full_c[i], 1);
+      mbar_init(&s.wb_free[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.s_free[i], 16);
       mbar_init(&s.mma_done[i], 1);
@@ -265,23 +301,22 @@ __global__ void __launch_bounds__(896, 1)
       int last_wb = -1, last_c = -1;
       // (the argument is this CTA's step number; each stream has a cursor on
       // its pair and chunk, advanced as the stream issues its steps in order)
-      PairCursor uwb, uc;
+      Cursor uwb, uc;
       uwb.start(s);
       uc.start(s);
       auto issue_wb = [&](int gg) {
-        const int i = gg & 1, bb = s.seg_b[uwb.k], grp = s.seg_grp[uwb.k];
+        const int i = ring_slot<kBR>(gg), bb = s.seg_b[uwb.k], grp = s.seg_grp[uwb.k];
         mbar_arrive_expect_tx(&s.full_wb[i], (kStateOnly ? K::NB : 1 + K::NB) * K::kTile);
         if (!kStateOnly)
           tma_load_3d(sm + K::oW + i * K::kTile, &tm_w, &s.full_wb[i], 0, ((bb * nc + uwb.c) * (int)a.G + grp) * 64,
                       0);
         for (int jb = 0; jb < K::NB; ++jb)
-          tma_load_4d(sm + K::oB + (i * K::NB + jb) * K::kTile, &tm_b, &s.full_wb[i], 64 * jb, grp, uwb.c * 64,
-                      bb);
+          tma_load_4d(sm + oBr + (i * K::NB + jb) * K::kTile, &tm_b, &s.full_wb[i], 64 * jb, grp, uwb.c * 64, bb);
         uwb.next(s);
         last_wb = gg;
       };
       auto issue_c = [&](int gg) {
-        const int i = gg & 1, bb = s.seg_b[uc.k], grp = s.seg_grp[uc.k];
+        const int i = ring_slot<K::kCSlots>(gg), bb = s.seg_b[uc.k], grp = s.seg_grp[uc.k];
         mbar_arrive_expect_tx(&s.full_c[i], K::NB * K::kTile);
         for (int jb = 0; jb < K::NB; ++jb)
           tma_load_4d(sm + K::oC + (i * K::NB + jb) * K::kTile, &tm_c, &s.full_c[i], 64 * jb, grp, uc.c * 64, bb);
@@ -291,29 +326,31 @@ __global__ void __launch_bounds__(896, 1)
       if (!*abort_flag) {
         if (!kStateOnly) griddep_wait();  // W' comes from the C B^T kernel launched before this one
         #pragma unroll 1
-        for (int c = 0; c < 2 && c < total; ++c) {
-          issue_wb(c);
-          if (!kStateOnly) issue_c(c);
-        }
+        for (int c = 0; c < kBR && c < total; ++c) issue_wb(c);
+        if (!kStateOnly)
+          #pragma unroll 1
+          for (int c = 0; c < K::kCSlots && c < total; ++c) issue_c(c);
       }
       bool ok = !*abort_flag;
-      // each tile is refilled for a later chunk as soon as its last reader is done
+      // each tile is refilled for a later chunk as soon as its MMAs are done
       #pragma unroll 1
-      for (int c = 0; c + 2 < total && ok; ++c) {
-        ok = mbar_wait(&s.s_full[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
-        if (ok) issue_wb(c + 2);
-        if (!kStateOnly) {
-          ok = ok && mbar_wait(&s.mma_done[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
-          if (ok) issue_c(c + 2);
+      for (int c = 0; c < total && ok; ++c) {
+        if (c + kBR < total) {
+          ok = mbar_wait(&s.wb_free[ring_slot<kBR>(c)], ring_par<kBR>(c), abort_flag, kWaitLimitNs);
+          if (ok) issue_wb(c + kBR);
+        }
+        if (!kStateOnly && ok && c + K::kCSlots < total) {
+          ok = mbar_wait(&s.c_free[ring_slot<K::kCSlots>(c)], ring_par<K::kCSlots>(c), abort_flag, kWaitLimitNs);
+          if (ok) issue_c(c + K::kCSlots);
         }
       }
       if (*abort_flag) {  // let this CTA's own copies land before its smem is released
         #pragma unroll 1
-        for (int c = last_wb - 1 < 0 ? 0 : last_wb - 1; c <= last_wb; ++c)
-          mbar_wait(&s.full_wb[c & 1], (c >> 1) & 1, never, kWaitLimitNs);
+        for (int c = last_wb - (kBR - 1) < 0 ? 0 : last_wb - (kBR - 1); c <= last_wb; ++c)
+          mbar_wait(&s.full_wb[ring_slot<kBR>(c)], ring_par<kBR>(c), never, kWaitLimitNs);
         #pragma unroll 1
-        for (int c = last_c - 1 < 0 ? 0 : last_c - 1; c <= last_c; ++c)
-          mbar_wait(&s.full_c[c & 1], (c >> 1) & 1, never, kWaitLimitNs);
+        for (int c = last_c - (K::kCSlots - 1) < 0 ? 0 : last_c - (K::kCSlots - 1); c <= last_c; ++c)
+          mbar_wait(&s.full_c[ring_slot<K::kCSlots>(c)], ring_par<K::kCSlots>(c), never, kWaitLimitNs);
       }
     }
   } else if (warp == 1) {
@@ -327,29 +364,31 @@ __global__ void __launch_bounds__(896, 1)
     };
     // descriptors of buffer 0; buffer 1 lies a whole number of 8 KB tiles further
     const uint64_t dw0 = sw128_desc(smem_u32(sm + K::oW), 16, 1024);
-    const uint64_t db0 = sw128_desc(smem_u32(sm + K::oB), K::kTile, 1024);
+    const uint64_t db0 = sw128_desc(smem_u32(sm + oBr), K::kTile, 1024);
     const uint64_t dc0 = sw128_desc(smem_u32(sm + K::oC), 16, 1024);
     constexpr uint32_t kTileDesc = K::kTile >> 4;  // an 8 KB tile in descriptor address units
     constexpr uint32_t id_y = idesc_bf16(128, 64, 0, 0);   // A in TMEM, B K-major
     constexpr uint32_t id_s = idesc_bf16(128, 128, 0, 1);  // A in TMEM, B MN-major
     #pragma unroll 1
     for (int c = 0; c < total; ++c) {
-      const int i = c & 1, xb = c & 3;
+      const int i = c & 1, xb = c & 3, ib = ring_slot<kBR>(c), ic = ring_slot<K::kCSlots>(c);
       const uint32_t ph = (c >> 1) & 1, pxp = (c >> 2) & 1, pacc = ((c - 2) >> 1) & 1, psf = ((c - 1) >> 1) & 1;
-      const bool acc = !kStateOnly && c >= 2, sfree = c >= 1;
-      const bool p_wb = mbar_probe(&s.full_wb[i], ph);
+      const uint32_t pb = ring_par<kBR>(c), pc = ring_par<K::kCSlots>(c);
+      // (the state-only pass accumulates S over its whole segment: no S is read out between steps)
+      const bool acc = !kStateOnly && c >= 2, sfree = !kStateOnly && c >= 1;
+      const bool p_wb = mbar_probe(&s.full_wb[ib], pb);
       const bool p_xp = mbar_probe(&s.xp_ready[xb], pxp);
       const bool p_acc = !acc || mbar_probe(&s.acc_free[i], pacc);
       const bool p_sf = !sfree || mbar_probe(&s.s_free[(c - 1) & 1], psf);
-      const bool p_c = kStateOnly || mbar_probe(&s.full_c[i], ph);
-      if (!need(p_wb, &s.full_wb[i], ph) || !need(p_xp, &s.xp_ready[xb], pxp) ||
+      const bool p_c = kStateOnly || mbar_probe(&s.full_c[ic], pc);
+      if (!need(p_wb, &s.full_wb[ib], pb) || !need(p_xp, &s.xp_ready[xb], pxp) ||
           (acc && !need(p_acc, &s.acc_free[i], pacc)))
         break;
       tc_fence_after();
       const uint32_t yd = tmem + K::tYd0 + 64 * i;
       const uint32_t ax = tmem + K::tX0 + 32 * xb;  // X'^T of both heads, this chunk
-      const uint64_t dw = dw0 + i * kTileDesc;
-      const uint64_t db = db0 + i * K::NB * kTileDesc;
+      const uint64_t dw = dw0 + ib * kTileDesc;
+      const uint64_t db = db0 + ib * K::NB * kTileDesc;
       if (!kStateOnly) {
         // Yd^T = X'^T W'^T   (K = 64 tokens s; a K step is 32 bytes along the row)
         if (elect_one()) {
@@ -364,22 +403,25 @@ __global__ void __launch_bounds__(896, 1)
       tc_fence_after();
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_bf16_ts(tmem + K::tS, ax + 8 * kk, db + 128 * kk, id_s, kk > 0);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ts(tmem + K::tS, ax + 8 * kk, db + 128 * kk, id_s, kk > 0 || (kStateOnly && c > 0));
         mma_commit(&s.s_full[i]);
+        mma_commit(&s.wb_free[ib]);  // the step's W' and B have been read
       }
       __syncwarp();
       if (kStateOnly) continue;
       // Yd^T += H C^T   (K = N states)
       const bool p_h = mbar_probe(&s.h_ready[i], ph);
-      if (!need(p_h, &s.h_ready[i], ph) || !need(p_c, &s.full_c[i], ph)) break;
+      if (!need(p_h, &s.h_ready[i], ph) || !need(p_c, &s.full_c[ic], pc)) break;
       tc_fence_after();
-      const uint64_t dc = dc0 + i * K::NB * kTileDesc;
+      const uint64_t dc = dc0 + ic * K::NB * kTileDesc;
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < NS / 16; ++kk)
           mma_bf16_ts(yd, tmem + K::tH0 + 64 * i + 8 * kk, dc + ((kk >> 2) * K::kTile + (kk & 3) * 32) / 16, id_y,
                       1);
         mma_commit(&s.mma_done[i]);
+        mma_commit(&s.c_free[ic]);  // the step's C has been read
       }
       __syncwarp();
     }
@@ -396,21 +438,23 @@ __global__ void __launch_bounds__(896, 1)
     // so that no register load is in flight when the results are released.
     const int j = lane >> 4, l16 = lane & 15;
     int last_dt = -1;
-    PairCursor ud, us;
+    Cursor ud, us;
     ud.start(s);
     us.start(s);
     auto issue_dt = [&](int gg) {
-      mbar_arrive_expect_tx(&s.full_dt[gg & 7], K::kDtBox);
-      tma_load_3d(sm + K::oDt + (gg & 7) * K::kDtBox, &tm_dt, &s.full_dt[gg & 7], s.seg_h0[ud.k] & ~3, ud.c * 64,
+      const int sl = ring_slot<K::kDtSlots>(gg);
+      mbar_arrive_expect_tx(&s.full_dt[sl], K::kDtBox);
+      tma_load_3d(sm + K::oDt + sl * K::kDtBox, &tm_dt, &s.full_dt[sl], s.seg_h0[ud.k] & ~3, ud.c * 64,
                   s.seg_b[ud.k]);
       ud.next(s);
       last_dt = gg;
     };
     if (lane == 0 && !*abort_flag)
       #pragma unroll 1
-      for (int c = 0; c < 8 && c < total; ++c) issue_dt(c);
+      for (int c = 0; c < K::kDtSlots && c < total; ++c) issue_dt(c);
     int cur_seg = -1, col = 0;
     float a2 = 0.f, dsk = 0.f;
+    float suf = 0.f;  // state-only pass: log2 decay from the end of this chunk to the segment's end
     #pragma unroll 1
     for (int g = 0; g < total; ++g, us.next(s)) {
       const int slot = g & 3;
@@ -422,17 +466,18 @@ __global__ void __launch_bounds__(896, 1)
         dsk = a.D ? a.D[hh + j] : 0.f;
       }
       if (g >= 4 && !mbar_wait_warp(&s.scan_empty[slot], ((g - 4) >> 2) & 1, abort_flag, kWaitLimitNs)) break;
-      if (!mbar_wait_warp(&s.full_dt[g & 7], (g >> 3) & 1, abort_flag, kWaitLimitNs)) break;
-      const float* dts = reinterpret_cast<const float*>(sm + K::oDt + (g & 7) * K::kDtBox);
+      if (!mbar_wait_warp(&s.full_dt[ring_slot<K::kDtSlots>(g)], ring_par<K::kDtSlots>(g), abort_flag, kWaitLimitNs))
+        break;
+      const float* dts = reinterpret_cast<const float*>(sm + K::oDt + ring_slot<K::kDtSlots>(g) * K::kDtBox);
       const int c = us.c;
       const int nvalid = (int)((int64_t)(c + 1) * 64 <= a.L ? 64 : a.L - (int64_t)c * 64);
       float d[4], cs[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) d[k] = dts[(4 * l16 + k) * 4 + col];
       __syncwarp();
-      if (lane == 0 && g + 8 < total) {  // the slot has been read: refill it 8 steps ahead
+      if (lane == 0 && g + K::kDtSlots < total) {  // the slot has been read: refill it
         fence_proxy_async_smem();
-        issue_dt(g + 8);
+        issue_dt(g + K::kDtSlots);
       }
       cs[0] = d[0] * a2;
 #pragma unroll
@@ -454,9 +499,12 @@ __global__ void __launch_bounds__(896, 1)
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         u4[k] = exp2f(cs[k]);
-        v4[k] = exp2f(-cs[k]) * d[k];
+        // fused pass: v_s = 2^-cs_s dt_s (the chunk's first token as reference);
+        // state-only pass: 2^(suf + cs_e - cs_s) dt_s, the decay to the segment's end
+        v4[k] = kStateOnly ? exp2f(suf + cse - cs[k]) * d[k] : exp2f(-cs[k]) * d[k];
         bad |= !(fabsf(cs[k]) <= kRangeLog2);
       }
+      if (kStateOnly) suf += cse;
       // a chunk the factorised form cannot take: the exact kernel redoes the
       // pair (once, however many chunks or CTAs find it)
       if (__any_sync(0xffffffffu, bad) && lane == 0 && atomicExch(&a.pair_bad[s.seg_pair[us.k]], 1) == 0) {
@@ -476,33 +524,37 @@ __global__ void __launch_bounds__(896, 1)
     }
     if (lane == 0 && *abort_flag)  // let the dt copies in flight land
       #pragma unroll 1
-      for (int c = last_dt - 7 < 0 ? 0 : last_dt - 7; c <= last_dt; ++c)
-        mbar_wait(&s.full_dt[c & 7], (c >> 3) & 1, never, kWaitLimitNs);
+      for (int c = last_dt - (K::kDtSlots - 1) < 0 ? 0 : last_dt - (K::kDtSlots - 1); c <= last_dt; ++c)
+        mbar_wait(&s.full_dt[ring_slot<K::kDtSlots>(c)], ring_par<K::kDtSlots>(c), never, kWaitLimitNs);
   } else if (warp == 3) {
     // ---------------------------------------------- y stores and x loads
     // An x slot is refilled (8 steps ahead) as soon as the y tile written
     // over it has been read out by its store; in the state-only pass, which
     // stores no y, as soon as the state warps have scaled it.  x comes from
-    // HBM: L2 prefetches run 3 steps ahead of the loads.
+    // HBM: L2 prefetches run 6 steps ahead of the loads (the steps 8-10 after
+    // the first x loads are not prefetched).
     if (lane == 0) {
-      int last_x = -1;
-      PairCursor ux, uy, upf;
+      int last_x = -1, pf = K::kXSlots + 3;  // pf: the step upf is at
+      Cursor ux, uy, upf;
       ux.start(s);
       uy.start(s);
       upf.start(s);
-      for (int k = 0; k < K::kXSlots + 3; ++k) upf.next(s);
+      for (int k = 0; k < pf; ++k) upf.next(s);
       auto issue_x = [&](int gg) {
-        const int sl = gg & (K::kXSlots - 1), bb = s.seg_b[ux.k], hh = s.seg_h0[ux.k];
+        const int sl = ring_slot<K::kXSlots>(gg), bb = s.seg_b[ux.k], hh = s.seg_h0[ux.k];
         mbar_arrive_expect_tx(&s.full_x[sl], 2 * K::kTile);
         for (int j = 0; j < 2; ++j)
           tma_load_3d(sm + K::oX + (sl * 2 + j) * K::kTile, &tm_x, &s.full_x[sl], (hh + j) * 64, ux.c * 64, bb);
         ux.next(s);
         last_x = gg;
       };
-      auto prefetch_x = [&]() {
-        const int bb = s.seg_b[upf.k], hh = s.seg_h0[upf.k];
-        for (int j = 0; j < 2; ++j) tma_prefetch_l2_3d(&tm_x, (hh + j) * 64, upf.c * 64, bb);
+      auto prefetch_x = [&]() {  // step pf, if it is one of this CTA's
+        if (pf < total) {
+          const int bb = s.seg_b[upf.k], hh = s.seg_h0[upf.k];
+          for (int j = 0; j < 2; ++j) tma_prefetch_l2_3d(&tm_x, (hh + j) * 64, upf.c * 64, bb);
+        }
         upf.next(s);
+        ++pf;
       };
       if (!*abort_flag) {
         #pragma unroll 1
@@ -512,27 +564,27 @@ __global__ void __launch_bounds__(896, 1)
       }
       #pragma unroll 1
       for (int c = 0; c < total && !*abort_flag; ++c) {
-        const int sl = c & (K::kXSlots - 1);
+        const int sl = ring_slot<K::kXSlots>(c);
         if (!kStateOnly) {
-          if (!mbar_wait(&s.y_staged[sl], (c >> 3) & 1, abort_flag, kWaitLimitNs)) break;
+          if (!mbar_wait(&s.y_staged[sl], ring_par<K::kXSlots>(c), abort_flag, kWaitLimitNs)) break;
           for (int j = 0; j < 2; ++j)
             tma_store_3d(&tm_y, sm + K::oX + (sl * 2 + j) * K::kTile, (s.seg_h0[uy.k] + j) * 64, uy.c * 64,
                          s.seg_b[uy.k]);
           bulk_commit_group();
           bulk_wait_read<0>();  // the tiles have been read out: the slot may be refilled
           uy.next(s);
-        } else if (!mbar_wait(&s.x_empty[sl], (c >> 3) & 1, abort_flag, kWaitLimitNs)) {
+        } else if (!mbar_wait(&s.x_empty[sl], ring_par<K::kXSlots>(c), abort_flag, kWaitLimitNs)) {
           break;
         }
         if (c + K::kXSlots < total) {
           issue_x(c + K::kXSlots);
-          if (c + K::kXSlots + 3 < total) prefetch_x();
+          prefetch_x();
         }
       }
       if (*abort_flag)  // let this CTA's own x copies land before its smem is released
         #pragma unroll 1
         for (int c = last_x - (K::kXSlots - 1) < 0 ? 0 : last_x - (K::kXSlots - 1); c <= last_x; ++c)
-          mbar_wait(&s.full_x[c & (K::kXSlots - 1)], (c >> 3) & 1, never, kWaitLimitNs);
+          mbar_wait(&s.full_x[ring_slot<K::kXSlots>(c)], ring_par<K::kXSlots>(c), never, kWaitLimitNs);
       bulk_wait<0>();  // stores complete before the CTA's shared memory is released
     }
   } else if (warp < 12) {
@@ -550,7 +602,7 @@ __global__ void __launch_bounds__(896, 1)
       const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
       #pragma unroll 1
       for (int c = 0; c < total; ++c) {
-        const int ip = c & 1, sl = c & (K::kXSlots - 1), sc4 = c & 3;
+        const int ip = c & 1, sl = ring_slot<K::kXSlots>(c), sc4 = c & 3;
         if (!mbar_wait_warp(&s.mma_done[ip], (c >> 1) & 1, abort_flag, kWaitLimitNs)) break;
         tc_fence_after();
         const float dj = s.sc[sc4][j][1];
@@ -643,12 +695,13 @@ __global__ void __launch_bounds__(896, 1)
     // jj, lanes + 8 e).  The X'^T buffer of step cc was last read by the MMAs
     // of step cc - 4, which are done once S of step cc - 2 is.
     auto scale = [&](int cc) -> bool {
-      const int sl = cc & (K::kXSlots - 1), xb = cc & 3;
+      const int sl = ring_slot<K::kXSlots>(cc), xb = cc & 3;
       const bool p_v = mbar_probe(&s.scan_full[cc & 3], (cc >> 2) & 1);
-      const bool p_x = mbar_probe(&s.full_x[sl], (cc >> 3) & 1);
+      const bool p_x = mbar_probe(&s.full_x[sl], ring_par<K::kXSlots>(cc));
       if ((!__all_sync(0xffffffffu, p_v) &&
            !mbar_wait_warp(&s.scan_full[cc & 3], (cc >> 2) & 1, abort_flag, kWaitLimitNs)) ||
-          (!__all_sync(0xffffffffu, p_x) && !mbar_wait_warp(&s.full_x[sl], (cc >> 3) & 1, abort_flag, kWaitLimitNs)))
+          (!__all_sync(0xffffffffu, p_x) &&
+           !mbar_wait_warp(&s.full_x[sl], ring_par<K::kXSlots>(cc), abort_flag, kWaitLimitNs)))
         return false;
       tc_fence_after();
       const uint32_t xt_a = smem_u32(sm + K::oX + (sl * 2 + j) * K::kTile);
@@ -811,7 +864,11 @@ __global__ void __launch_bounds__(896, 1)
           break;
         }
         tc_fence_after();
-        {
+        if constexpr (kStateOnly) {
+          // S accumulates in TMEM; the wait above only orders the reuse of
+          // X'^T buffers (scale below)
+          dprod *= s.sc[g & 3][j][0];
+        } else {
           uint32_t r[32];
           uint32_t* r_hi = r + 16;
           SSD_TMEM_LD_16x256b_X4(tq + K::tS + 32 * nq, r);
@@ -823,7 +880,6 @@ __global__ void __launch_bounds__(896, 1)
           // H <- d (H + S), two lanes of fp32 per instruction
           const float dd = s.sc[g & 3][j][0];
           const float2 d2 = make_float2(dd, dd);
-          if (kStateOnly) dprod *= dd;
 #pragma unroll
           for (int kk = 0; kk < 32; kk += 2) {
             const float2 h2 = __fadd2_rn(make_float2(H[kk], H[kk + 1]),
@@ -841,6 +897,16 @@ __global__ void __launch_bounds__(896, 1)
           break;
         }
         if (g == release_at) release();
+      }
+      if (kStateOnly && !failed && g_end > g0) {
+        // the segment's end state: every MMA is done (S of its last step was waited for)
+        uint32_t r[32];
+        uint32_t* r_hi = r + 16;
+        SSD_TMEM_LD_16x256b_X4(tq + K::tS + 32 * nq, r);
+        SSD_TMEM_LD_16x256b_X4(tq + (16u << 16) + K::tS + 32 * nq, r_hi);
+        SSD_TMEM_WAIT_LD_32(r);
+#pragma unroll
+        for (int kk = 0; kk < 32; ++kk) H[kk] = __uint_as_float(r[kk]);
       }
       if (!failed) seg_end(k);
     }
