@@ -367,14 +367,38 @@ __global__ void __launch_bounds__(kThreads, 2) k_bwd_chunk_states(const KArgs a)
   }
 }
 
-// One thread per state entry (b, h, p, n): the forward scan turns S into the
-// state entering each chunk, the backward scan turns T into the gradient with
-// respect to the state leaving each chunk; what the backward scan carries out
-// of chunk 0 is dLoss/dinitial_states.
+// V consecutive state entries (b, h, p, n..n+V-1) per thread: the forward
+// scan turns S into the state entering each chunk, the backward scan turns T
+// into the gradient with respect to the state leaving each chunk; what the
+// backward scan carries out of chunk 0 is dLoss/dinitial_states.  V = 4 when
+// P N is a multiple of 4 (S and T are 256-byte aligned workspace, so each
+// chunk's row is then read and written as 16-byte vectors), else 1; h0,
+// dfinal and dh0 are the caller's and are accessed one float at a time.
+template <int V>
+__device__ __forceinline__ void ld_v(const float* p, float (&o)[V]) {
+  if constexpr (V == 4) {
+    const float4 q = *reinterpret_cast<const float4*>(p);
+    o[0] = q.x, o[1] = q.y, o[2] = q.z, o[3] = q.w;
+  } else {
+#pragma unroll
+    for (int k = 0; k < V; ++k) o[k] = p[k];
+  }
+}
+template <int V>
+__device__ __forceinline__ void st_v(float* p, const float (&o)[V]) {
+  if constexpr (V == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(o[0], o[1], o[2], o[3]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < V; ++k) p[k] = o[k];
+  }
+}
+
+template <int V>
 __global__ void __launch_bounds__(kThreads) k_bwd_state_passing(const KArgs a) {
   const Dims& d = a.d;
   const int64_t PN = d.P * d.N;
-  const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  const int64_t i = ((int64_t)blockIdx.x * kThreads + threadIdx.x) * V;  // the thread's first entry
   if (i >= d.b * d.H * PN) return;
   const int64_t bh = i / PN, e = i % PN;
   float* S = a.S + bh * d.nc * PN + e;
@@ -385,30 +409,40 @@ __global__ void __launch_bounds__(kThreads) k_bwd_state_passing(const KArgs a) {
   // overwritten, so that 2 kBatch loads are in flight per thread (the
   // addresses differ, which the compiler cannot see).  The scans are each
   // thread's own, so a batch is a plain reordering of the loads.
-  constexpr int kBatch = 16;
-  float run = a.h0 ? a.h0[i] : 0.f;
-  float lam = a.dfinal ? a.dfinal[i] : 0.f;
+  constexpr int kBatch = V == 4 ? 8 : 16;
+  float run[V], lam[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    run[k] = a.h0 ? a.h0[i + k] : 0.f;
+    lam[k] = a.dfinal ? a.dfinal[i + k] : 0.f;
+  }
   const int64_t nc = d.nc;
   for (int64_t c = 0; c < nc; c += kBatch) {
     const int n = (int)(nc - c < kBatch ? nc - c : kBatch);
     const int64_t cb = nc - 1 - c;  // the backward scan's chunk for j = 0
-    float vs[kBatch], vt[kBatch];
+    float vs[kBatch][V], vt[kBatch][V];
 #pragma unroll
     for (int j = 0; j < kBatch; ++j)
       if (j < n) {
-        vs[j] = S[(c + j) * PN];
-        vt[j] = T[(cb - j) * PN];
+        ld_v<V>(S + (c + j) * PN, vs[j]);
+        ld_v<V>(T + (cb - j) * PN, vt[j]);
       }
 #pragma unroll
     for (int j = 0; j < kBatch; ++j)
       if (j < n) {
-        S[(c + j) * PN] = run;
-        run = fmaf(dec[c + j], run, vs[j]);
-        T[(cb - j) * PN] = lam;
-        lam = fmaf(dec[cb - j], lam, vt[j]);
+        st_v<V>(S + (c + j) * PN, run);
+        st_v<V>(T + (cb - j) * PN, lam);
+        const float ds = dec[c + j], dl = dec[cb - j];
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+          run[k] = fmaf(ds, run[k], vs[j][k]);
+          lam[k] = fmaf(dl, lam[k], vt[j][k]);
+        }
       }
   }
-  if (a.dh0) a.dh0[i] = lam;
+  if (a.dh0)
+#pragma unroll
+    for (int k = 0; k < V; ++k) a.dh0[i + k] = lam[k];
 }
 
 // Columns of k_bwd_chunk's partial-sum array: one per column block of a
@@ -881,7 +915,10 @@ ssd_status enqueue_typed(const KArgs& k, const Plan& pl, void* const events[2], 
   } else if (!launch(&k_bwd_chunk_states<T>, chunk_ctas, pl.smem_states, k)) {
     return SSD_ERR_CUDA;
   }
-  if (!launch(&k_bwd_state_passing, blocks_for(d.b * d.H * d.P * d.N), (size_t)0, k)) return SSD_ERR_CUDA;
+  const int64_t n_states = d.b * d.H * d.P * d.N;
+  if (!((d.P * d.N) % 4 == 0 ? launch(&k_bwd_state_passing<4>, blocks_for(n_states / 4), (size_t)0, k)
+                              : launch(&k_bwd_state_passing<1>, blocks_for(n_states), (size_t)0, k)))
+    return SSD_ERR_CUDA;
   if (only_dh0) {  // k_bwd_chunk is not run: its timing events mark the same point
     if (events[0] && !(launch.record(events[0]) && launch.record(events[1]))) return SSD_ERR_CUDA;
     return SSD_OK;

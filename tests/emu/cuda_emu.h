@@ -59,6 +59,12 @@ inline void __syncthreads() { swapcontext(emu::g_self, &emu::g_sched); }
 
 #define SSD_DYN_SMEM(name) float* name = emu::g_smem
 
+// The 16-byte vector type of 4 floats.
+struct float4 {
+  float x, y, z, w;
+};
+inline float4 make_float4(float x, float y, float z, float w) { return float4{x, y, z, w}; }
+
 // The fast-math intrinsics, at host precision.
 inline float __expf(float v) { return std::exp(v); }
 inline float __fdividef(float a, float b) { return a / b; }

@@ -122,7 +122,7 @@ MUTANTS = [
     # the in-chunk sum of dx runs one token past the chunk
     ("dx_past_chunk", r"(tile_mac<false>\(acc, tl, Km, 1, sQ, nullptr, dys, sP, 1, tl\.r\[0\], )Qc\);", r"\1Qc + 1);"),
     # the adjoint carried across chunks skips the chunk decay
-    ("no_decay_backward", r"lam = fmaf\(dec\[cb - j\], lam, vt\[j\]\);", "lam = lam + vt[j];"),
+    ("no_decay_backward", r"lam\[k\] = fmaf\(dl, lam\[k\], vt\[j\]\[k\]\);", "lam[k] = lam[k] + vt[j][k];"),
     # the pair sum of dl loses dt
     ("pairs_no_dt", r"blk = fmaf\(Mm\[u \* sQ \+ s2\], w\[s2\], blk\);", "blk += Mm[u * sQ + s2];"),
     # the h_in terms are taken for every token, also after a sequence boundary
