@@ -717,7 +717,8 @@ TcWorkspace tc_carve(const Problem& p, void* ws, size_t* total) {
     w.runs.len = r + 1 + 2 * ns;
     w.runs.id = r + 1 + 3 * ns;
     w.runs.c0 = r + 1 + 4 * ns;
-    off = align_up(off + sizeof(int) * (2 + 5 * ns), kWsAlign);
+    w.runs.order = r + 2 + 5 * ns;
+    off = align_up(off + sizeof(int) * (2 + 6 * ns), kWsAlign);
   }
   w.handoff = pair ? reinterpret_cast<float*>(base + off) : nullptr;
   if (pair) off = align_up(off + sizeof(float) * (size_t)kPairGridMax * kPairHandoffFloats, kWsAlign);

@@ -33,7 +33,11 @@ struct RunList {
   int* len;    // [num_seqs] its tokens
   int* id;     // [num_seqs] its sequence id
   int* c0;     // [num_seqs + 1] its first chunk in the flattened chunk list
+  int* order;  // [num_seqs] the runs longest first (by chunks; ties in run order), which
+               // the single-head kernel takes in that order so that the long runs do not
+               // trail at the end of the grid; run order past kRunSortMax runs
 };
+constexpr int kRunSortMax = 1024;  // runs k_seq_runs ranks (one per thread)
 
 struct CbArgs {
   int64_t L, G, nc;

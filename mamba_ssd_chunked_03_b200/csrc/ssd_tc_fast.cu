@@ -154,8 +154,22 @@ __global__ void __launch_bounds__(1024) k_seq_runs(const SeqRunArgs a) {
       *a.runs.count = 0;
       *a.failed_count = (int)(a.b * a.H);
     }
-  } else if (tid == 0) {
-    *a.runs.count = (int)nr;
+  } else {
+    // the runs longest first: rank = runs with more chunks, or as many and earlier
+    if (nr <= kRunSortMax) {
+      for (int64_t r = tid; r < nr; r += 1024) {
+        const int cr = (a.runs.len[r] + 63) / 64;
+        int rank = 0;
+        for (int64_t q = 0; q < nr; ++q) {
+          const int cq = (a.runs.len[q] + 63) / 64;
+          rank += cq > cr || (cq == cr && q < r);
+        }
+        a.runs.order[rank] = (int)r;
+      }
+    } else {
+      for (int64_t r = tid; r < nr; r += 1024) a.runs.order[r] = (int)r;
+    }
+    if (tid == 0) *a.runs.count = (int)nr;
   }
 }
 
@@ -337,8 +351,9 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
   int64_t b, out_row, cbase;
   int t_base, len;
   if (a.varlen) {
-    const int64_t ru = unit / a.H;
-    if (ru >= *a.runs.count) return;  // past the runs (uniform)
+    const int64_t pos = unit / a.H;
+    if (pos >= *a.runs.count) return;  // past the runs (uniform)
+    const int64_t ru = a.runs.order[pos];  // the longest runs first
     b = a.runs.b[ru];
     t_base = a.runs.t0[ru];
     len = a.runs.len[ru];
