@@ -93,14 +93,15 @@ struct PairCfg {
 
 constexpr int kPairMaxSeg = 32;  // segments (pairs touched) per CTA, at most
 
-// Slot and phase parity of step c in a ring of n buffers.
+// Slot and phase parity of step c (>= 0) in a ring of n buffers (unsigned
+// arithmetic: a mask and a shift when n is a power of two).
 template <int n>
 __device__ __forceinline__ int ring_slot(int c) {
-  return c % n;
+  return (int)((uint32_t)c % (uint32_t)n);
 }
 template <int n>
 __device__ __forceinline__ uint32_t ring_par(int c) {
-  return (uint32_t)(c / n) & 1u;
+  return ((uint32_t)c / (uint32_t)n) & 1u;
 }
 
 // Ring barriers are indexed like the buffers they guard, so no barrier can
@@ -112,8 +113,8 @@ struct __align__(16) PairSmem {
   uint64_t full_x[PairCfg::kXSlots], x_empty[PairCfg::kXSlots];  // x ring: TMA landed / scaled (state-only pass)
   uint64_t full_dt[PairCfg::kDtSlots];   // dt ring (the scan warp's own)
   uint64_t full_wb[PairCfg::kWbMax];     // W' + B of a chunk landed (state-only pass: B)
-  uint64_t wb_free[PairCfg::kWbMax];     // ... and read by its MMAs
-  uint64_t full_c[PairCfg::kCSlots], c_free[PairCfg::kCSlots];  // C of a chunk landed / read
+  uint64_t wb_free[PairCfg::kWbMax];     // ... and read by its MMAs (state-only pass)
+  uint64_t full_c[PairCfg::kCSlots];     // C of a chunk landed
   uint64_t scan_full[4], scan_empty[4];  // scan results of a chunk ready / consumed
   uint64_t xp_ready[4];                  // X'^T of a chunk in TMEM
   uint64_t s_full[2];                    // S of a chunk in TMEM
@@ -182,6 +183,8 @@ __global__ void __launch_bounds__(896, 1)
   // takes their space and runs 4 steps ahead, since its steps wait on nothing
   // else.
   constexpr int kBR = kStateOnly ? 4 : PairCfg::kWbSlots;
+  // (the fused pass refills W', B and C on s_full and mma_done, which are 2 deep)
+  static_assert(PairCfg::kWbSlots == 2 && PairCfg::kCSlots == 2, "fused-pass W'/B and C rings");
   static_assert(4 * PairCfg::NB * PairCfg::kTile <= PairCfg::oDt - PairCfg::oW, "state-only B ring");
   constexpr uint32_t oBr = kStateOnly ? PairCfg::oW : PairCfg::oB;
   constexpr int NS = K::NS;
@@ -202,10 +205,7 @@ __global__ void __launch_bounds__(896, 1)
       mbar_init(&s.y_staged[i], 8);
     }
     for (int i = 0; i < K::kDtSlots; ++i) mbar_init(&s.full_dt[i], 1);
-    for (int i = 0; i < K::kCSlots; ++i) {
-      mbar_init(&s.full_c[i], 1);
-      mbar_init(&s.c_free[i], 1);
-    }
+    for (int i = 0; i < K::kCSlots; ++i) mbar_init(&s.full_c[i], 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&s.scan_full[i], 1);
       // the state warps, and in the fused pass the epilogue warps
@@ -332,15 +332,20 @@ __global__ void __launch_bounds__(896, 1)
           for (int c = 0; c < K::kCSlots && c < total; ++c) issue_c(c);
       }
       bool ok = !*abort_flag;
-      // each tile is refilled for a later chunk as soon as its MMAs are done
+      // each tile is refilled for a later chunk as soon as its MMAs are done:
+      // the fused pass takes the two barriers its MMA warp commits anyway (S
+      // done frees W' and B, every MMA done frees C: one commit more each on
+      // the MMA warp's path measured 3% slower); the state-only pass has
+      // barriers of its own for its deeper B ring
       #pragma unroll 1
       for (int c = 0; c < total && ok; ++c) {
         if (c + kBR < total) {
-          ok = mbar_wait(&s.wb_free[ring_slot<kBR>(c)], ring_par<kBR>(c), abort_flag, kWaitLimitNs);
+          ok = kStateOnly ? mbar_wait(&s.wb_free[ring_slot<kBR>(c)], ring_par<kBR>(c), abort_flag, kWaitLimitNs)
+                          : mbar_wait(&s.s_full[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
           if (ok) issue_wb(c + kBR);
         }
         if (!kStateOnly && ok && c + K::kCSlots < total) {
-          ok = mbar_wait(&s.c_free[ring_slot<K::kCSlots>(c)], ring_par<K::kCSlots>(c), abort_flag, kWaitLimitNs);
+          ok = mbar_wait(&s.mma_done[c & 1], (c >> 1) & 1, abort_flag, kWaitLimitNs);
           if (ok) issue_c(c + K::kCSlots);
         }
       }
@@ -406,7 +411,7 @@ __global__ void __launch_bounds__(896, 1)
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16_ts(tmem + K::tS, ax + 8 * kk, db + 128 * kk, id_s, kk > 0 || (kStateOnly && c > 0));
         mma_commit(&s.s_full[i]);
-        mma_commit(&s.wb_free[ib]);  // the step's W' and B have been read
+        if (kStateOnly) mma_commit(&s.wb_free[ib]);  // the step's B has been read
       }
       __syncwarp();
       if (kStateOnly) continue;
@@ -421,7 +426,6 @@ __global__ void __launch_bounds__(896, 1)
           mma_bf16_ts(yd, tmem + K::tH0 + 64 * i + 8 * kk, dc + ((kk >> 2) * K::kTile + (kk & 3) * 32) / 16, id_y,
                       1);
         mma_commit(&s.mma_done[i]);
-        mma_commit(&s.c_free[ic]);  // the step's C has been read
       }
       __syncwarp();
     }
