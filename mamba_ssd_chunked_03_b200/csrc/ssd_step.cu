@@ -12,7 +12,9 @@
 // 8 b H P N bytes); x, B, C, y are small.  One CTA per (row, head): its 8
 // warps take the state rows p, each lane four consecutive states n (float4
 // loads and stores, coalesced along the row), B and C held in registers, and
-// y_p reduced across the warp.
+// y_p reduced across the warp.  A warp loads the state of kRowsInFlight of its
+// rows before it updates any of them, so that many loads are in flight at
+// once (one row at a time left the step bound by load latency).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -24,6 +26,7 @@ namespace {
 
 constexpr int kStepThreads = 256;
 constexpr int kStepMaxN = 256;  // states per row a lane group covers: 4 per lane, twice
+constexpr int kRowsInFlight = 8;  // rows a warp loads before updating them
 
 struct StepArgs {
   int64_t H, P, N, hpg, G;
@@ -51,7 +54,8 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
   return make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
 }
 
-template <typename T>
+// NK: 128-state halves of a row a lane covers (1 for N <= 128, 2 up to 256)
+template <typename T, int NK>
 __global__ void __launch_bounds__(kStepThreads) k_ssd_step(const StepArgs a) {
   const int64_t bh = blockIdx.x;  // b * H + h
   const int64_t b = bh / a.H, h = bh % a.H, g = h / a.hpg;
@@ -63,36 +67,54 @@ __global__ void __launch_bounds__(kStepThreads) k_ssd_step(const StepArgs a) {
   const T* Cp = static_cast<const T*>(a.C) + (b * a.G + g) * a.N;
   const T* xp = static_cast<const T*>(a.x) + bh * a.P;
   T* yp = static_cast<T*>(a.y) + bh * a.P;
-  float* S = a.state + bh * a.P * a.N;
-  // this lane's states: n = 4 lane + 128 k, k < 2
-  float4 bv[2], cv[2];
+  float* __restrict__ S = a.state + bh * a.P * a.N;
+  // this lane's states: n = 4 lane + 128 k, k < NK
+  float4 bv[NK], cv[NK];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
+  for (int k = 0; k < NK; ++k) {
     const int n = 4 * lane + 128 * k;
     bv[k] = n < a.N ? load4(Bp + n) : make_float4(0.f, 0.f, 0.f, 0.f);
     cv[k] = n < a.N ? load4(Cp + n) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int64_t p = warp; p < a.P; p += kStepThreads / 32) {
-    const float xv = to_f(xp[p]);
-    const float u = dtv * xv;
-    float acc = 0.f;
+  constexpr int kWarps = kStepThreads / 32;
+  for (int64_t p0 = warp; p0 < a.P; p0 += kRowsInFlight * kWarps) {
+    float4 sv[kRowsInFlight][NK];
+    float xv[kRowsInFlight];
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int n = 4 * lane + 128 * k;
-      if (n < a.N) {
-        float4* sp = reinterpret_cast<float4*>(S + p * a.N + n);
-        float4 s = *sp;
-        s.x = fmaf(decay, s.x, u * bv[k].x);
-        s.y = fmaf(decay, s.y, u * bv[k].y);
-        s.z = fmaf(decay, s.z, u * bv[k].z);
-        s.w = fmaf(decay, s.w, u * bv[k].w);
-        *sp = s;
-        acc = fmaf(s.x, cv[k].x, fmaf(s.y, cv[k].y, fmaf(s.z, cv[k].z, fmaf(s.w, cv[k].w, acc))));
+    for (int r = 0; r < kRowsInFlight; ++r) {
+      const int64_t p = p0 + (int64_t)r * kWarps;
+      if (p < a.P) {
+        xv[r] = to_f(xp[p]);
+#pragma unroll
+        for (int k = 0; k < NK; ++k) {
+          const int n = 4 * lane + 128 * k;
+          if (n < a.N) sv[r][k] = *reinterpret_cast<const float4*>(S + p * a.N + n);
+        }
       }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) from_f(yp + p, fmaf(dsk, xv, acc));
+    for (int r = 0; r < kRowsInFlight; ++r) {
+      const int64_t p = p0 + (int64_t)r * kWarps;
+      if (p >= a.P) break;  // (uniform across the warp)
+      const float u = dtv * xv[r];
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < NK; ++k) {
+        const int n = 4 * lane + 128 * k;
+        if (n < a.N) {
+          float4 st = sv[r][k];
+          st.x = fmaf(decay, st.x, u * bv[k].x);
+          st.y = fmaf(decay, st.y, u * bv[k].y);
+          st.z = fmaf(decay, st.z, u * bv[k].z);
+          st.w = fmaf(decay, st.w, u * bv[k].w);
+          *reinterpret_cast<float4*>(S + p * a.N + n) = st;
+          acc = fmaf(st.x, cv[k].x, fmaf(st.y, cv[k].y, fmaf(st.z, cv[k].z, fmaf(st.w, cv[k].w, acc))));
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) from_f(yp + p, fmaf(dsk, xv[r], acc));
+    }
   }
 }
 
@@ -129,9 +151,13 @@ extern "C" SSD_API ssd_status ssd_step(const ssd_step_args* a, void* stream) {
   s.y = a->y;
   const unsigned grid = (unsigned)(a->batch * a->nheads);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (a->dtype == SSD_BF16)
-    k_ssd_step<__nv_bfloat16><<<grid, kStepThreads, 0, st>>>(s);
-  else
-    k_ssd_step<float><<<grid, kStepThreads, 0, st>>>(s);
+  const bool two = a->dstate > 128;
+  if (a->dtype == SSD_BF16) {
+    if (two) k_ssd_step<__nv_bfloat16, 2><<<grid, kStepThreads, 0, st>>>(s);
+    else k_ssd_step<__nv_bfloat16, 1><<<grid, kStepThreads, 0, st>>>(s);
+  } else {
+    if (two) k_ssd_step<float, 2><<<grid, kStepThreads, 0, st>>>(s);
+    else k_ssd_step<float, 1><<<grid, kStepThreads, 0, st>>>(s);
+  }
   return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
