@@ -33,6 +33,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "ssd.h"
 
 #ifndef SSD_DYN_SMEM
@@ -153,7 +155,14 @@ __global__ void __launch_bounds__(kThreads) k_conv_bwd(const KArgs a) {
 #pragma unroll
   for (int k = 0; k < K; ++k) dw[k] = 0.f;
 
-  for (int64_t t = t0; t < te; ++t) {
+  // One token of the walk.  IN: the token is the strip's own (dw and dbias
+  // take its terms); ST: 0 no du store (the first K-1 tokens), 1 store (token
+  // t-(K-1) is in the strip), 2 store if it is.  The walk runs in these three
+  // phases so that the checks leave its main loop, which is unrolled: the
+  // window and pending-sum shifts then become register renames.
+  auto token = [&](int64_t t, auto in_strip, auto store_mode) {
+    constexpr bool IN = decltype(in_strip)::value;
+    constexpr int ST = decltype(store_mode)::value;
     const float cur = cv_ld(tu, (t - t0 + (K - 1)) * kThreads);
     const float dcur = cv_ld(td, (t - t0) * kThreads);
     const int st = SEQ ? seq[t] : 0;
@@ -166,7 +175,7 @@ __global__ void __launch_bounds__(kThreads) k_conv_bwd(const KArgs a) {
     for (int j = 0; j < K - 1; ++j)
       if (take[j]) pre = fmaf(w[j], win[j], pre);
     const float g = dcur * silu_slope(pre);
-    if (t < t1) {
+    if constexpr (IN) {
       db += g;
       dw[K - 1] = fmaf(g, cur, dw[K - 1]);
 #pragma unroll
@@ -179,7 +188,11 @@ __global__ void __launch_bounds__(kThreads) k_conv_bwd(const KArgs a) {
       if (take[j]) pend[j] = fmaf(w[j], g, pend[j]);
     // token t-(K-1) has all its contributions now
     const int64_t done = t - (K - 1);
-    if (done >= t0 && done < t1) du[done * a.C] = pend[0];
+    if constexpr (ST == 1) {
+      du[done * a.C] = pend[0];
+    } else if constexpr (ST == 2) {
+      if (done >= t0 && done < t1) du[done * a.C] = pend[0];
+    }
 #pragma unroll
     for (int j = 0; j + 1 < K; ++j) pend[j] = pend[j + 1];
     pend[K - 1] = 0.f;
@@ -192,7 +205,14 @@ __global__ void __launch_bounds__(kThreads) k_conv_bwd(const KArgs a) {
       win[K > 1 ? K - 2 : 0] = cur;
       wseq[K > 1 ? K - 2 : 0] = st;
     }
-  }
+  };
+  using yes = std::true_type;
+  using no = std::false_type;
+  const int64_t tw = t0 + (K - 1) < t1 ? t0 + (K - 1) : t1;  // the first token whose t-(K-1) is in the strip
+  for (int64_t t = t0; t < tw; ++t) token(t, yes{}, std::integral_constant<int, 0>{});
+#pragma unroll 4
+  for (int64_t t = tw; t < t1; ++t) token(t, yes{}, std::integral_constant<int, 1>{});
+  for (int64_t t = t1; t < te; ++t) token(t, no{}, std::integral_constant<int, 2>{});
   // at the end of the row the last tokens of the strip are complete too
 #pragma unroll
   for (int j = 0; j < K - 1; ++j) {
