@@ -106,26 +106,69 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t v, int64_t* tota
 __global__ void __launch_bounds__(1024) k_seq_runs(const SeqRunArgs a) {
   __shared__ int64_t warp_sums[32];
   __shared__ int bad;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   if (tid == 0) bad = 0;
   const int64_t total = a.b * a.L;
-  const int64_t per = (total + 1023) / 1024;
-  const int64_t lo = tid * per < total ? tid * per : total;
-  const int64_t hi = lo + per < total ? lo + per : total;
-  auto is_start = [&](int64_t i) { return i % a.L == 0 || a.seq[i] != a.seq[i - 1]; };
-  int64_t cnt = 0;
-  for (int64_t i = lo; i < hi; ++i) cnt += is_start(i);
-  int64_t nr = 0;
-  int64_t k = block_exclusive_scan(cnt, &nr, warp_sums);
-  const bool fits = nr <= a.num_seqs;
-  if (fits)
-    for (int64_t i = lo; i < hi; ++i)
-      if (is_start(i)) {
-        a.runs.b[k] = (int)(i / a.L);
-        a.runs.t0[k] = (int)(i % a.L);
-        a.runs.id[k] = a.seq[i];
-        ++k;
+  // Each warp takes a contiguous range of tokens (a multiple of 32) and reads
+  // it 32 consecutive tokens at a time, 16 iterations of loads in flight: a
+  // token opens a run at its row's start or where its id differs from the
+  // token before (the lane below, or the previous iteration's last lane).
+  // Each lane keeps its token's position in the row as a counter.
+  const int64_t per_w = ((total + 31) / 32 + 31) / 32 * 32;
+  const int64_t wlo = (int64_t)wid * per_w < total ? (int64_t)wid * per_w : total;
+  const int64_t whi = wlo + per_w < total ? wlo + per_w : total;
+  const int64_t i0 = wlo + lane;
+  const int64_t row0 = i0 / a.L, pos0 = i0 - row0 * a.L;
+  const int before = wlo > 0 && wlo < total ? a.seq[wlo - 1] : 0;
+  constexpr int kBatch = 16;
+  // walk the range; visit(base, ballot of starts, is_start, id, row, pos) per 32 tokens
+  auto walk = [&](auto&& visit) {
+    int64_t pos = pos0, row = row0;
+    int carry = before;
+    for (int64_t b0 = wlo; b0 < whi; b0 += 32 * kBatch) {
+      int cur[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int64_t i = b0 + 32 * u + lane;
+        cur[u] = i < whi ? a.seq[i] : 0;
       }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int64_t base = b0 + 32 * u;
+        if (base >= whi) break;  // (uniform across the warp)
+        int prev = __shfl_up_sync(0xffffffffu, cur[u], 1);
+        if (lane == 0) prev = carry;
+        const bool st = base + lane < whi && (pos == 0 || cur[u] != prev);
+        const uint32_t bal = __ballot_sync(0xffffffffu, st);
+        visit(bal, st, cur[u], row, pos);
+        carry = __shfl_sync(0xffffffffu, cur[u], 31);
+        pos += 32;
+        while (pos >= a.L) {
+          pos -= a.L;
+          ++row;
+        }
+      }
+    }
+  };
+  int64_t cnt = 0;
+  walk([&](uint32_t bal, bool, int, int64_t, int64_t) { cnt += __popc(bal); });
+  // warp counts -> each warp's first run index (lane 0 contributes the warp's count)
+  int64_t nr = 0;
+  const int64_t k0 = block_exclusive_scan(lane == 0 ? cnt : 0, &nr, warp_sums);
+  const int64_t kw = __shfl_sync(0xffffffffu, k0, 0);
+  const bool fits = nr <= a.num_seqs;
+  if (fits) {
+    int64_t k = kw;
+    walk([&](uint32_t bal, bool st, int id, int64_t row, int64_t pos) {
+      if (st) {
+        const int64_t at = k + __popc(bal & ((1u << lane) - 1u));
+        a.runs.b[at] = (int)row;
+        a.runs.t0[at] = (int)pos;
+        a.runs.id[at] = id;
+      }
+      k += __popc(bal);
+    });
+  }
   __syncthreads();
   // lengths, the id checks and the chunk counts, per block of runs
   const int64_t rper = (nr + 1023) / 1024;
