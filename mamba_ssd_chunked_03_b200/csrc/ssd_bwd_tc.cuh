@@ -66,6 +66,11 @@ struct TcCfg {
   static constexpr uint32_t oZw = oZ + 3 * kTile;   // Zw terms [3][t][s]
   static constexpr uint32_t oS = oZw + 3 * kTile;   // Lam, then h_in: terms [3][n-block][p][n]
   static constexpr uint32_t oM = oS + 6 * kTile;    // M fp32 [t][s], rows of kMs
+  // the gradients staged for their bulk stores, over the Z, Zw and state terms
+  // (dead once the second round of MMAs is done; the tail's R is in K's place):
+  // 32-column fp32 boxes, 64 rows of 128 bytes, 128-byte swizzle
+  static constexpr uint32_t oStage = oZ, oStDx = 0, oStDB = 2 * kTile, oStDC = 6 * kTile;
+  static_assert(oStDC + 4 * kTile <= oM - oZ, "gradient staging");
   static constexpr int kMs = Q + 1;
   static constexpr uint32_t oEnd = oM + Q * kMs * 4;
   static constexpr uint32_t kSmemBytes = oEnd + 1024;
@@ -151,7 +156,8 @@ __device__ __forceinline__ uint64_t mnmaj(uint64_t d0, int kk) { return d0 + (ui
 __global__ void __launch_bounds__(kThreads, 1)
     k_bwd_chunk_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dy,
                    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
-                   const KArgs a) {
+                   const __grid_constant__ CUtensorMap tm_dx, const __grid_constant__ CUtensorMap tm_dbh,
+                   const __grid_constant__ CUtensorMap tm_dch, const KArgs a) {
   using K = TcCfg;
   constexpr uint64_t kLimit = tc::kWaitLimitNs;
   const Dims& d = a.d;
@@ -161,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                        ~uintptr_t(1023));
   float* Mm = reinterpret_cast<float*>(sm + K::oM);
+  unsigned char* stage = sm + K::oStage;
   __shared__ TcSmem s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // TMEM reads: warp (qd, hf) reads rows 16 qd + (lane & 15) of its lane
@@ -405,8 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   ok = __syncthreads_and(ok);
   if (ok) {
     tc_fence_after();
-    const int64_t tok = q.b * d.L + q.t0 + row;  // this thread's token row
-    const bool valid = row < Qc;
+    // this thread's token row is staged whole (rows past the chunk's last token are
+    // beyond L and the bulk stores clip them)
     // ---- dx = w_s [K^T dy + el_s B Lam^T] + D dy_s (columns p in [c0, c0 + 16))
     {
       uint32_t r[16];
@@ -416,15 +423,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       load8(sm + K::oDY, row, c0 >> 3, dyv);
       load8(sm + K::oDY, row, (c0 >> 3) + 1, dyv + 8);
       const float ws = s.w[row], Dh = a.D ? a.D[q.h] : 0.f;
-      if (valid) {
-        float4* dst = reinterpret_cast<float4*>(a.dx + (tok * d.H + q.h) * d.P + c0);
+      // columns c0 .. c0 + 15: box c0 / 32, 16-byte chunks 4 hf .. 4 hf + 3 of its row
+      unsigned char* box = stage + K::oStDx + (uint32_t)(c0 >> 5) * K::kTile;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_float4(fmaf(ws, __uint_as_float(r[4 * i]), Dh * dyv[4 * i]),
-                               fmaf(ws, __uint_as_float(r[4 * i + 1]), Dh * dyv[4 * i + 1]),
-                               fmaf(ws, __uint_as_float(r[4 * i + 2]), Dh * dyv[4 * i + 2]),
-                               fmaf(ws, __uint_as_float(r[4 * i + 3]), Dh * dyv[4 * i + 3]));
-      }
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4*>(box + sw_chunk(row, 4 * hf + i)) =
+            make_float4(fmaf(ws, __uint_as_float(r[4 * i]), Dh * dyv[4 * i]),
+                        fmaf(ws, __uint_as_float(r[4 * i + 1]), Dh * dyv[4 * i + 1]),
+                        fmaf(ws, __uint_as_float(r[4 * i + 2]), Dh * dyv[4 * i + 2]),
+                        fmaf(ws, __uint_as_float(r[4 * i + 3]), Dh * dyv[4 * i + 3]));
     }
     // ---- dB of this head = w_s [Z^T C + el_s x Lam] (states n in [c1, c1 + 32))
     {
@@ -434,13 +441,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDB + 64 * hf + 16, r_hi);
       SSD_TMEM_WAIT_LD_32(r);
       const float ws = s.w[row];
-      if (valid) {
-        float4* dst = reinterpret_cast<float4*>(a.dBh + (tok * d.H + q.h) * d.N + c1);
+      unsigned char* box = stage + K::oStDB + (uint32_t)(c1 >> 5) * K::kTile;  // a whole 32-column row
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(ws * __uint_as_float(r[4 * i]), ws * __uint_as_float(r[4 * i + 1]),
-                               ws * __uint_as_float(r[4 * i + 2]), ws * __uint_as_float(r[4 * i + 3]));
-      }
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<float4*>(box + sw_chunk(row, i)) =
+            make_float4(ws * __uint_as_float(r[4 * i]), ws * __uint_as_float(r[4 * i + 1]),
+                        ws * __uint_as_float(r[4 * i + 2]), ws * __uint_as_float(r[4 * i + 3]));
     }
     // ---- dC of this head = Zw B + e_t dy h_in, and the row sums C_t . (h_in^T dy_t)
     {
@@ -462,21 +468,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 32; ++i) cy = fmaf(cv[i], __uint_as_float(r2[i]), cy);
       s.cyp[row][2 * hf + (lane >> 4)] = cy;
-      if (valid) {
-        float4* dst = reinterpret_cast<float4*>(a.dCh + (tok * d.H + q.h) * d.N + c1);
+      unsigned char* box = stage + K::oStDC + (uint32_t)(c1 >> 5) * K::kTile;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(fmaf(et, __uint_as_float(r2[4 * i]), __uint_as_float(r1[4 * i])),
-                               fmaf(et, __uint_as_float(r2[4 * i + 1]), __uint_as_float(r1[4 * i + 1])),
-                               fmaf(et, __uint_as_float(r2[4 * i + 2]), __uint_as_float(r1[4 * i + 2])),
-                               fmaf(et, __uint_as_float(r2[4 * i + 3]), __uint_as_float(r1[4 * i + 3])));
-      }
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<float4*>(box + sw_chunk(row, i)) =
+            make_float4(fmaf(et, __uint_as_float(r2[4 * i]), __uint_as_float(r1[4 * i])),
+                        fmaf(et, __uint_as_float(r2[4 * i + 1]), __uint_as_float(r1[4 * i + 1])),
+                        fmaf(et, __uint_as_float(r2[4 * i + 2]), __uint_as_float(r1[4 * i + 2])),
+                        fmaf(et, __uint_as_float(r2[4 * i + 3]), __uint_as_float(r1[4 * i + 3])));
     }
+    fence_proxy_async_smem();  // the staged gradients are read by the bulk stores
   }
   tc_fence_before();
   ok = __syncthreads_and(ok);
 
   if (ok) {
+    if (tid == 0) {
+      // dx, dB and dC of this head and chunk: 32-column boxes, rows past L clipped
+      const int h = (int)q.h, tk = (int)q.t0, bb = (int)q.b;
+      for (int k = 0; k < 2; ++k) tma_store_4d(&tm_dx, stage + K::oStDx + k * K::kTile, 32 * k, h, tk, bb);
+      for (int k = 0; k < 4; ++k) {
+        tma_store_4d(&tm_dbh, stage + K::oStDB + k * K::kTile, 32 * k, h, tk, bb);
+        tma_store_4d(&tm_dch, stage + K::oStDC + k * K::kTile, 32 * k, h, tk, bb);
+      }
+      bulk_commit_group();
+    }
     // ---- the decay gradients (the tail of k_bwd_chunk, on the row sums above)
     for (int t = tid; t < Qc; t += kThreads) {
       s.nv[t] = s.nxp[t][0] + s.nxp[t][1] + s.nxp[t][2] + s.nxp[t][3];
@@ -577,6 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
+  if (tid == 0) bulk_wait<0>();  // the gradient stores have read their staging before the CTA's memory goes
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -786,12 +803,17 @@ inline cudaError_t chunk_states_tc_launch(const KArgs& k, cudaStream_t st) {
 
 inline cudaError_t chunk_tc_launch(const KArgs& k, cudaStream_t st) {
   const Dims& d = k.d;
-  CUtensorMap tx, tdy, tb, tc_;
+  CUtensorMap tx, tdy, tb, tc_, tdx, tdb, tdc;
   if (!chunk_tc_maps(k, &tx, &tdy, &tb, &tc_)) return cudaErrorInvalidValue;
+  // the gradient tiles' bulk stores: dx (b, L, H, P) and the per-head dB, dC (b, L, H, N), fp32
+  if (!tc::make_map_f32_tiles(&tdx, k.dx, d.P, d.H, d.L, d.b) || !tc::make_map_f32_tiles(&tdb, k.dBh, d.N, d.H, d.L, d.b) ||
+      !tc::make_map_f32_tiles(&tdc, k.dCh, d.N, d.H, d.L, d.b))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)TcCfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  k_bwd_chunk_tc<<<(unsigned)(d.b * d.nc * d.H), kThreads, TcCfg::kSmemBytes, st>>>(tx, tdy, tb, tc_, k);
+  k_bwd_chunk_tc<<<(unsigned)(d.b * d.nc * d.H), kThreads, TcCfg::kSmemBytes, st>>>(tx, tdy, tb, tc_, tdx, tdb, tdc,
+                                                                                       k);
   return cudaGetLastError();
 }
 

@@ -114,6 +114,18 @@ bool make_map_dt(CUtensorMap* m, const float* dt, int64_t H, int64_t L, int64_t 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_map_f32_tiles(CUtensorMap* m, float* base, int64_t inner, int64_t H, int64_t L, int64_t b) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || (inner * 4) % 16 != 0) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)b};
+  const cuuint64_t strides[3] = {(cuuint64_t)(inner * 4), (cuuint64_t)(H * inner * 4), (cuuint64_t)(L * H * inner * 4)};
+  const cuuint32_t box[4] = {32, 1, 64, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tc
 
 namespace {

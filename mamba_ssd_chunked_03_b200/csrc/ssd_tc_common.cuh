@@ -109,6 +109,10 @@ bool make_map_bc(CUtensorMap* m, const void* base, int64_t N, int64_t G, int64_t
 // fp32 tensor map over dt (b, L, H) with a 4-head x 64-token box, no swizzle;
 // needs H * 4 bytes to be a multiple of 16.  Tokens past L read as zeros.
 bool make_map_dt(CUtensorMap* m, const float* dt, int64_t H, int64_t L, int64_t b);
+// fp32 tensor map over (b, L, H, inner) as 4-D (element, head, token, row) with
+// a 32 x 1 x 64 x 1 box (128-byte rows) and 128-byte swizzle, for bulk stores
+// of per-chunk gradient tiles; tokens past L are clipped.
+bool make_map_f32_tiles(CUtensorMap* m, float* base, int64_t inner, int64_t H, int64_t L, int64_t b);
 
 }  // namespace tc
 
