@@ -620,6 +620,10 @@ struct StCfg {
   static constexpr uint32_t oEnd = oDs + 3 * kTile;
   static constexpr uint32_t kSmemBytes = oEnd + 1024;
   static constexpr uint32_t tS = 0, tT = 128, kTmemCols = 256;
+  // S and T staged for their bulk stores over B, C and the terms (dead once the
+  // MMAs are done): 32-column fp32 boxes of 64 rows, 128-byte swizzle
+  static constexpr uint32_t oStS = oB, oStT = oB + 4 * kTile;
+  static_assert(oStT + 4 * kTile <= oEnd, "state staging");
 };
 
 struct __align__(16) StSmem {
@@ -633,6 +637,7 @@ struct __align__(16) StSmem {
 __global__ void __launch_bounds__(kThreads, 2)
     k_bwd_chunk_states_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dy,
                           const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
+                          const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_t,
                           const KArgs a) {
   using K = StCfg;
   constexpr uint64_t kLimit = tc::kWaitLimitNs;
@@ -741,7 +746,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   ok = __syncthreads_and(ok);
   if (ok) {
     tc_fence_after();
-    const int64_t off = ((q.b * d.H + q.h) * d.nc + q.c) * d.P * d.N + (int64_t)row * d.N + c1;
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
       uint32_t r[32];
@@ -750,13 +754,27 @@ __global__ void __launch_bounds__(kThreads, 2)
       SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + col, r);
       SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + col + 16, r_hi);
       SSD_TMEM_WAIT_LD_32(r);
-      float4* dst = reinterpret_cast<float4*>((which ? a.T : a.S) + off);
+      // this thread's row, states [c1, c1 + 32): a whole row of box c1 / 32
+      unsigned char* box = sm + (which ? K::oStT : K::oStS) + (uint32_t)(c1 >> 5) * K::kTile;
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
-                             __uint_as_float(r[4 * i + 3]));
+        *reinterpret_cast<float4*>(box + sw_chunk(row, i)) =
+            make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
+                        __uint_as_float(r[4 * i + 3]));
     }
-  } else if (warp == 0) {
+    fence_proxy_async_smem();  // the staged states are read by the bulk stores
+  }
+  ok = __syncthreads_and(ok);
+  if (ok && tid == 0) {
+    const int unit = (int)((q.b * d.H + q.h) * d.nc + q.c);
+    for (int k = 0; k < 4; ++k) {
+      tma_store_3d(&tm_s, sm + K::oStS + k * K::kTile, 32 * k, 0, unit);
+      tma_store_3d(&tm_t, sm + K::oStT + k * K::kTile, 32 * k, 0, unit);
+    }
+    bulk_commit_group();
+    bulk_wait<0>();  // the stores have read their staging before the CTA's memory goes
+  }
+  if (!ok && warp == 0) {
     mbar_wait(&s.bar_in, 0, never, kLimit);
     if (elect_one()) {
       mma_commit(&s.bar_drain);
@@ -792,12 +810,17 @@ inline bool chunk_tc_maps(const KArgs& k, CUtensorMap* tx, CUtensorMap* tdy, CUt
 
 inline cudaError_t chunk_states_tc_launch(const KArgs& k, cudaStream_t st) {
   const Dims& d = k.d;
-  CUtensorMap tx, tdy, tb, tc_;
+  CUtensorMap tx, tdy, tb, tc_, ts, tt;
   if (!chunk_tc_maps(k, &tx, &tdy, &tb, &tc_)) return cudaErrorInvalidValue;
+  // the states' bulk stores: S and T are (b, H, nc, P, N) fp32, one P x N block per chunk and head
+  if (!tc::make_map_f32_blocks(&ts, k.S, d.N, d.P, d.b * d.H * d.nc) ||
+      !tc::make_map_f32_blocks(&tt, k.T, d.N, d.P, d.b * d.H * d.nc))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)StCfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  k_bwd_chunk_states_tc<<<(unsigned)(d.b * d.nc * d.H), kThreads, StCfg::kSmemBytes, st>>>(tx, tdy, tb, tc_, k);
+  k_bwd_chunk_states_tc<<<(unsigned)(d.b * d.nc * d.H), kThreads, StCfg::kSmemBytes, st>>>(tx, tdy, tb, tc_, ts, tt,
+                                                                                               k);
   return cudaGetLastError();
 }
 

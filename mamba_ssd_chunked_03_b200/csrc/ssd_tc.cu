@@ -126,6 +126,18 @@ bool make_map_f32_tiles(CUtensorMap* m, float* base, int64_t inner, int64_t H, i
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_map_f32_blocks(CUtensorMap* m, float* base, int64_t inner, int64_t rows, int64_t units) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || (inner * 4) % 16 != 0 || rows > 256 || units >= ((int64_t)1 << 31)) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)units};
+  const cuuint64_t strides[2] = {(cuuint64_t)(inner * 4), (cuuint64_t)(rows * inner * 4)};
+  const cuuint32_t box[3] = {32, (cuuint32_t)rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tc
 
 namespace {

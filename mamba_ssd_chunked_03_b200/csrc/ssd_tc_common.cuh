@@ -113,6 +113,10 @@ bool make_map_dt(CUtensorMap* m, const float* dt, int64_t H, int64_t L, int64_t 
 // a 32 x 1 x 64 x 1 box (128-byte rows) and 128-byte swizzle, for bulk stores
 // of per-chunk gradient tiles; tokens past L are clipped.
 bool make_map_f32_tiles(CUtensorMap* m, float* base, int64_t inner, int64_t H, int64_t L, int64_t b);
+// fp32 tensor map over units of a rows x inner block each (units, rows, inner
+// contiguous) with a 32 x rows x 1 box and 128-byte swizzle: one unit's
+// 32-column slice per bulk store.
+bool make_map_f32_blocks(CUtensorMap* m, float* base, int64_t inner, int64_t rows, int64_t units);
 
 }  // namespace tc
 
