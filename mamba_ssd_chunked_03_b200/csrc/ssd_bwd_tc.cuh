@@ -72,20 +72,28 @@ struct TcCfg {
   static constexpr uint32_t oStage = oZ, oStDx = 0, oStDB = 2 * kTile, oStDC = 6 * kTile;
   static_assert(oStDC + 4 * kTile <= oM - oZ, "gradient staging");
   static constexpr int kMs = Q + 1;
-  static constexpr uint32_t oEnd = oM + Q * kMs * 4;
+  // the chunk's states as their bulk loads leave them, fp32 [p][n]: h_in in a
+  // region of its own (read again for its terms after the first MMAs), Lam over
+  // the K and Z terms (split into its terms before those are written)
+  static constexpr uint32_t kStateBytes = 64 * 128 * 4;
+  static constexpr uint32_t oHin = (oM + Q * kMs * 4 + 127) & ~127u;
+  static constexpr uint32_t oLam = oK;
+  static_assert(oLam + kStateBytes <= oZw, "Lam staging");
+  static constexpr uint32_t oEnd = oHin + kStateBytes;
   static constexpr uint32_t kSmemBytes = oEnd + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   // tensor memory columns
   static constexpr uint32_t tDx = 0, tDB = 64, tCB = 192, tG = 256, tDC2 = 192, tDC1 = 320, kTmemCols = 512;
 };
 
 struct __align__(16) TcSmem {
-  uint64_t bar_in, bar_p1, bar_p2, bar_drain;
+  uint64_t bar_in, bar_st, bar_p1, bar_p2, bar_drain;
   uint32_t tmem_base;
   int abort_flag, never;
   float cs[64], w[64], el[64], ein[64], dg[64], nv[64], dw[64], dcs[64], nn[64];
   float nxp[64][4], cyp[64][4];  // row sums, four shares a row
   float pair[64][8];             // the decay pair sums, in quarters
-  float red[kThreads];
+  float red[kThreads / 32];  // <Lam, h_in>, a share per warp
   int seg[64];
 };
 
@@ -135,14 +143,89 @@ __device__ __forceinline__ void store_terms8(unsigned char* tile, uint32_t strid
   *reinterpret_cast<uint4*>(tile + 2 * stride + off) = pack8(l);
 }
 
-// A state (P x N fp32; this thread: row p, states n in [n0, n0 + 32)) as three
-// terms, each two 64-column blocks [p][n] of the split area.
-__device__ __forceinline__ void store_state_terms(unsigned char* area, int p, int n0, const float (&v)[32]) {
+// The chunk's per-token scalars for tokens 2 lane and 2 lane + 1, by one warp:
+// w = dt, the in-chunk cumulative log-decay cs and the in-chunk index seg of
+// the token's sequence start (-1: it began before the chunk), as chunk_cumsum
+// defines them, then el = E(last, t) and ein = e_t.  cs is a segmented scan
+// (a start contributes 0 and restarts the sum) and seg a max scan of the
+// starts, both over the warp's shuffles.  Tokens past the chunk's end get 0
+// everywhere.
+struct DtScan {
+  float w[2], cs[2], el[2], ein[2];
+  int seg[2];
+};
+__device__ __forceinline__ DtScan dt_scan_warp(const KArgs& a, const ChunkPos& q, int lane) {
+  const Dims& d = a.d;
+  const float Ah = a.A[q.h];
+  const float* dtp = a.dt + (q.b * d.L + q.t0) * d.H + q.h;
+  const int32_t* sq = a.seq ? a.seq + q.b * d.L + q.t0 : nullptr;
+  DtScan r;
+  bool v[2], f[2];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const int n = n0 + 8 * c;
-    store_terms8(area + (n >> 6) * TcCfg::kTile, 2 * TcCfg::kTile, p, (n & 63) >> 3, v + 8 * c);
+  for (int e = 0; e < 2; ++e) {
+    const int t = 2 * lane + e;
+    v[e] = t < q.Qc;
+    r.w[e] = v[e] ? dtp[(int64_t)t * d.H] : 0.f;
+    f[e] = v[e] && sq && q.t0 + t > 0 && sq[t] != sq[t - 1];  // a sequence starts at t
   }
+  const float a0 = f[0] ? 0.f : r.w[0] * Ah;
+  const float a1 = f[1] ? 0.f : a0 + r.w[1] * Ah;
+  float sum = a1;                                         // the lane's sum since its last start
+  int rs = f[0] || f[1];                                  // ... and whether it has one
+  int st = f[1] ? 2 * lane + 1 : f[0] ? 2 * lane : -1;  // its last start
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float ps = __shfl_up_sync(0xffffffffu, sum, o);
+    const int pr = __shfl_up_sync(0xffffffffu, rs, o);
+    const int pst = __shfl_up_sync(0xffffffffu, st, o);
+    if (lane >= o) {
+      if (!rs) sum += ps;
+      rs |= pr;
+      st = max(st, pst);
+    }
+  }
+  float pre = __shfl_up_sync(0xffffffffu, sum, 1);
+  int pst = __shfl_up_sync(0xffffffffu, st, 1);
+  if (lane == 0) pre = 0.f, pst = -1;
+  r.cs[0] = f[0] ? 0.f : a0 + pre;
+  r.cs[1] = f[1] ? 0.f : f[0] ? a1 : a1 + pre;
+  r.seg[0] = f[0] ? 2 * lane : pst;
+  r.seg[1] = f[1] ? 2 * lane + 1 : r.seg[0];
+  const int last = q.Qc - 1;
+  const float csl = __shfl_sync(0xffffffffu, (last & 1) ? r.cs[1] : r.cs[0], last >> 1);
+  const int segl = __shfl_sync(0xffffffffu, (last & 1) ? r.seg[1] : r.seg[0], last >> 1);
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    if (!v[e]) r.cs[e] = 0.f, r.seg[e] = 0;
+    r.el[e] = v[e] && r.seg[e] == segl ? expf(csl - r.cs[e]) : 0.f;
+    r.ein[e] = v[e] && r.seg[e] == -1 ? expf(r.cs[e]) : 0.f;
+  }
+  return r;
+}
+
+// The three-term split of a fp32 state [p][n] as its bulk load leaves it in
+// shared memory: this thread's 16-byte chunk k16 = tid % 16 of rows
+// p = tid / 16 + 16 j, into the MN-major term tiles at `area` (two 64-column
+// blocks a term); returns the thread's share of <v, w> when `w` is given.
+__device__ __forceinline__ float split_state(unsigned char* area, const float* v, const float* w, int tid) {
+  const int k16 = tid & 15;
+  float dot = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int p = (tid >> 4) + 16 * j;
+    const float4* vr = reinterpret_cast<const float4*>(v + p * 128 + 8 * k16);
+    const float4 x0 = vr[0], x1 = vr[1];
+    const float e[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    if (w) {
+      const float4* wr = reinterpret_cast<const float4*>(w + p * 128 + 8 * k16);
+      const float4 y0 = wr[0], y1 = wr[1];
+      const float f[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dot = fmaf(e[i], f[i], dot);
+    }
+    store_terms8(area + (k16 >> 3) * TcCfg::kTile, 2 * TcCfg::kTile, p, k16 & 7, e);
+  }
+  return dot;
 }
 
 // Descriptor of K step kk of a K-major operand: 16 bf16 (32 bytes) along the
@@ -182,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&s.bar_in, 1);
+    mbar_init(&s.bar_st, 1);
     mbar_init(&s.bar_p1, 1);
     mbar_init(&s.bar_p2, 1);
     mbar_init(&s.bar_drain, 1);
@@ -203,6 +287,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   const uint32_t tq = tmem + ((uint32_t)(32 * qd) << 16);
   if (tid == 0) {
+    // this chunk's states first (the threads wait on them first): Lam and h_in,
+    // one contiguous P x N block each
+    const int64_t so = ((q.b * d.H + q.h) * d.nc + q.c) * d.P * d.N;
+    mbar_arrive_expect_tx(&s.bar_st, 2 * K::kStateBytes);
+    bulk_load(sm + K::oLam, a.T + so, K::kStateBytes, &s.bar_st);
+    bulk_load(sm + K::oHin, a.S + so, K::kStateBytes, &s.bar_st);
     // the chunk states of the CTA one wave later, into L2 (a hint: the grid
     // runs one CTA an SM, so that CTA comes about an SM count later)
     uint32_t nsm;
@@ -224,47 +314,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_4d(sm + K::oC + jb * K::kTile, &tm_c, &s.bar_in, 64 * jb, grp, tok, bb);
     }
   }
-
-  // the chunk's states: this thread's row p = tid / 4, states n in [32 (tid % 4), +32)
-  const int sp = tid >> 2, sn0 = 32 * (tid & 3);
-  const int64_t soff = ((q.b * d.H + q.h) * d.nc + q.c) * d.P * d.N + (int64_t)sp * d.N + sn0;
-  float hin[32];
-  {
-    float lam[32];
-    const float4* pl = reinterpret_cast<const float4*>(a.T + soff);
-    const float4* ph = reinterpret_cast<const float4*>(a.S + soff);
+  if (warp == 0) {  // the per-token scalars, while the loads are in flight
+    const DtScan r = dt_scan_warp(a, q, lane);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 v = __ldcg(pl + i), u = __ldcg(ph + i);
-      lam[4 * i] = v.x, lam[4 * i + 1] = v.y, lam[4 * i + 2] = v.z, lam[4 * i + 3] = v.w;
-      hin[4 * i] = u.x, hin[4 * i + 1] = u.y, hin[4 * i + 2] = u.z, hin[4 * i + 3] = u.w;
+    for (int e = 0; e < 2; ++e) {
+      const int t = 2 * lane + e;
+      s.w[t] = r.w[e];
+      s.cs[t] = r.cs[e];
+      s.seg[t] = r.seg[e];
+      s.el[t] = r.el[e];
+      s.ein[t] = r.ein[e];
+      s.dg[t] = 0.f;
     }
-    float lh = 0.f;  // <Lam, h_in>, this thread's share
+  }
+  // the Lam terms (the h_in ones come after the first MMAs) and <Lam, h_in>
+  bool ok = mbar_wait(&s.bar_st, 0, abort_flag, kLimit);
+  if (ok) {
+    float lh = split_state(sm + K::oS, reinterpret_cast<const float*>(sm + K::oLam),
+                           reinterpret_cast<const float*>(sm + K::oHin), tid);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) lh = fmaf(lam[i], hin[i], lh);
-    s.red[tid] = lh;
-    store_state_terms(sm + K::oS, sp, sn0, lam);
-  }
-  for (int t = tid; t < 64; t += kThreads) {
-    s.w[t] = t < Qc ? a.dt[(q.b * d.L + q.t0 + t) * d.H + q.h] : 0.f;
-    s.cs[t] = 0.f;
-    s.seg[t] = 0;
-    s.el[t] = 0.f;
-    s.ein[t] = 0.f;
-    s.dg[t] = 0.f;
-  }
-  __syncthreads();
-  chunk_cumsum(a, q, s.cs, s.seg, tid);  // ends with a barrier
-  for (int off = kThreads / 2; off > 0; off >>= 1) {
-    if (tid < off) s.red[tid] += s.red[tid + off];
-    __syncthreads();
-  }
-  for (int t = tid; t < Qc; t += kThreads) {
-    s.el[t] = s.seg[t] == s.seg[last] ? expf(s.cs[last] - s.cs[t]) : 0.f;
-    s.ein[t] = s.seg[t] == -1 ? expf(s.cs[t]) : 0.f;
+    for (int o = 16; o > 0; o >>= 1) lh += __shfl_xor_sync(0xffffffffu, lh, o);
+    if (lane == 0) s.red[warp] = lh;
   }
   fence_proxy_async_smem();  // the Lam terms are read by the MMAs
-  __syncthreads();
+  ok = __syncthreads_and(ok);
 
   // descriptors: K-major tiles (rows along K) and MN-major ones (rows along K,
   // the 64-element blocks of M or N one tile apart)
@@ -288,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   // ---- MMAs, first round: CB, G, B Lam^T, x Lam
-  bool ok = mbar_wait(&s.bar_in, 0, abort_flag, kLimit);  // every thread reads the tiles later
+  ok = ok && mbar_wait(&s.bar_in, 0, abort_flag, kLimit);  // every thread reads the tiles later
   if (warp == 0 && __all_sync(0xffffffffu, ok)) {
     tc_fence_after();
     if (elect_one()) {
@@ -381,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // ---- h_in terms over the Lam terms (the MMAs that read those are done)
-    store_state_terms(sm + K::oS, sp, sn0, hin);
+    split_state(sm + K::oS, reinterpret_cast<const float*>(sm + K::oHin), nullptr, tid);
     tmem_wait_st();
   }
   tc_fence_before();
@@ -543,7 +616,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
       // dl_k = S_k + sum_{t >= k} (h_in term)_t + sum_{s < k} N_s + e_last <Lam, h_in>,
       // tokens k = lane and lane + 32, the sums as warp scans
-      const float lh = s.red[0];
+      float lh = 0.f;
+#pragma unroll
+      for (int i = 0; i < kThreads / 32; ++i) lh += s.red[i];
       const float e_last = s.seg[last] == -1 ? expf(s.cs[last]) : 0.f;
       const int k0 = lane, k1 = lane + 32;
       const bool v0 = k0 <= last, v1 = k1 <= last;
@@ -586,6 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 0) {
     // a wait gave up: let this CTA's copies and MMAs finish before its memory goes
+    mbar_wait(&s.bar_st, 0, never, kLimit);
     mbar_wait(&s.bar_in, 0, never, kLimit);
     if (elect_one()) {
       mma_commit(&s.bar_drain);
@@ -630,8 +706,7 @@ struct __align__(16) StSmem {
   uint64_t bar_in, bar_mma, bar_drain;
   uint32_t tmem_base;
   int abort_flag, never;
-  float cs[64], cS[64], cT[64];
-  int seg[64];
+  float cS[64], cT[64];
 };
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -686,20 +761,16 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_load_4d(sm + K::oC + jb * K::kTile, &tm_c, &s.bar_in, 64 * jb, grp, tok, bb);
     }
   }
-  for (int t = tid; t < 64; t += kThreads) {
-    s.cs[t] = 0.f;
-    s.seg[t] = 0;
-    s.cS[t] = 0.f;
-    s.cT[t] = 0.f;
+  if (warp == 0) {  // the per-token scale factors, while the loads are in flight
+    const DtScan r = dt_scan_warp(a, q, lane);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      s.cS[2 * lane + e] = r.w[e] * r.el[e];
+      s.cT[2 * lane + e] = r.ein[e];
+    }
+    // the chunk's decay, e of its last token (0 when a sequence starts inside it)
+    if (lane == (last >> 1)) a.dec[(q.b * d.H + q.h) * d.nc + q.c] = (last & 1) ? r.ein[1] : r.ein[0];
   }
-  __syncthreads();
-  chunk_cumsum(a, q, s.cs, s.seg, tid);  // ends with a barrier
-  for (int t = tid; t < Qc; t += kThreads) {
-    const float w = a.dt[(q.b * d.L + q.t0 + t) * d.H + q.h];
-    s.cS[t] = s.seg[t] == s.seg[last] ? w * expf(s.cs[last] - s.cs[t]) : 0.f;
-    s.cT[t] = s.seg[t] == -1 ? expf(s.cs[t]) : 0.f;
-  }
-  if (tid == 0) a.dec[(q.b * d.H + q.h) * d.nc + q.c] = s.seg[last] == -1 ? expf(s.cs[last]) : 0.f;
   __syncthreads();
   bool ok = mbar_wait(&s.bar_in, 0, abort_flag, kLimit);
   if (ok) {
