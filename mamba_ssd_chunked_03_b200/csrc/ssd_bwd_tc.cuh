@@ -29,10 +29,13 @@
 //   [192, 256) CB, then with [256, 320) (G) the product dy h_in
 //   [320, 448) Zw B
 // Shared memory holds x, dy, B and C as the TMA loads them (bf16, 128-byte
-// rows, 128-byte swizzle), the three-term split tiles written by the threads
-// in the same layout, and M in fp32 for the decay sums.  Every wait is
-// bounded (1 s); a CTA whose wait gives up lets its copies and MMAs finish,
-// frees its tensor memory and exits without writing gradients.
+// rows, 128-byte swizzle), the chunk's Lam and h_in as two bulk copies leave
+// them (fp32), the three-term split tiles written by the threads in the
+// tiles' layout, and M in fp32 for the decay sums.  The MMAs run in five
+// groups with a completion barrier each (C B^T and G; the Lam products; dx;
+// dB; dC), so the threads start on each result while the next is formed.
+// Every wait is bounded (1 s); a CTA whose wait gives up lets its copies and
+// MMAs finish, frees its tensor memory and exits without writing gradients.
 //
 // Included by ssd_bwd.cu only (after ssd_bwd.cuh): the host emulation of the
 // CUDA-core kernels includes ssd_bwd.cuh alone.
@@ -66,20 +69,23 @@ struct TcCfg {
   static constexpr uint32_t oZw = oZ + 3 * kTile;   // Zw terms [3][t][s]
   static constexpr uint32_t oS = oZw + 3 * kTile;   // Lam, then h_in: terms [3][n-block][p][n]
   static constexpr uint32_t oM = oS + 6 * kTile;    // M fp32 [t][s], rows of kMs
-  // the gradients staged for their bulk stores, over the Z, Zw and state terms
-  // (dead once the second round of MMAs is done; the tail's R is in K's place):
-  // 32-column fp32 boxes, 64 rows of 128 bytes, 128-byte swizzle
-  static constexpr uint32_t oStage = oZ, oStDx = 0, oStDB = 2 * kTile, oStDC = 6 * kTile;
-  static_assert(oStDC + 4 * kTile <= oM - oZ, "gradient staging");
   static constexpr int kMs = Q + 1;
   // the chunk's states as their bulk loads leave them, fp32 [p][n]: h_in in a
   // region of its own (read again for its terms after the first MMAs), Lam over
   // the K and Z terms (split into its terms before those are written)
   static constexpr uint32_t kStateBytes = 64 * 128 * 4;
-  static constexpr uint32_t oHin = (oM + Q * kMs * 4 + 127) & ~127u;
+  static constexpr uint32_t oHin = (oM + Q * kMs * 4 + 1023) & ~1023u;
   static constexpr uint32_t oLam = oK;
   static_assert(oLam + kStateBytes <= oZw, "Lam staging");
   static constexpr uint32_t oEnd = oHin + kStateBytes;
+  // The gradients staged for their bulk stores (32-column fp32 boxes, 64 rows
+  // of 128 bytes, 128-byte swizzle), each where nothing still running reads:
+  // dx over the K terms (read only by the dx MMAs), dB over the h_in copy
+  // (dead once its terms are written), dC over the Z and Zw terms (all MMAs
+  // done); the tail's R over the state terms.
+  static constexpr uint32_t oStDx = oK, oStDB = oHin, oStDC = oZ, oR = oS;
+  static_assert(oStDx + 2 * kTile <= oZ && oStDB + 4 * kTile <= oEnd && oStDC + 4 * kTile <= oS, "staging");
+  static_assert(oR + Q * kMs * 4 <= oM, "R");
   static constexpr uint32_t kSmemBytes = oEnd + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   // tensor memory columns
@@ -87,7 +93,8 @@ struct TcCfg {
 };
 
 struct __align__(16) TcSmem {
-  uint64_t bar_in, bar_st, bar_p1, bar_p2, bar_drain;
+  // MMA completions: p1a C B^T and G, p1 the Lam products; p2a dx, p2b dB, p2 dC
+  uint64_t bar_in, bar_st, bar_p1a, bar_p1, bar_p2a, bar_p2b, bar_p2, bar_drain;
   uint32_t tmem_base;
   int abort_flag, never;
   float cs[64], w[64], el[64], ein[64], dg[64], nv[64], dw[64], dcs[64], nn[64];
@@ -141,6 +148,22 @@ __device__ __forceinline__ void store_terms8(unsigned char* tile, uint32_t strid
   *reinterpret_cast<uint4*>(tile + off) = pack8(h);
   *reinterpret_cast<uint4*>(tile + stride + off) = pack8(m);
   *reinterpret_cast<uint4*>(tile + 2 * stride + off) = pack8(l);
+}
+
+// chunk_pos in 32-bit arithmetic: the tensor-core kernels' grids (one CTA per
+// row, chunk and head) stay below 2^31 CTAs.
+__device__ __forceinline__ ChunkPos chunk_pos_u32(const Dims& d, uint32_t bid) {
+  const uint32_t H = (uint32_t)d.H, nc = (uint32_t)d.nc;
+  const uint32_t bc = bid / H, bb = bc / nc;
+  ChunkPos q;
+  q.h = bid - bc * H;
+  q.c = bc - bb * nc;
+  q.b = bb;
+  q.g = (uint32_t)q.h / (uint32_t)d.hpg;
+  q.t0 = q.c * d.Q;
+  const int64_t left = d.L - q.t0;
+  q.Qc = (int)(left < d.Q ? left : d.Q);
+  return q;
 }
 
 // The chunk's per-token scalars for tokens 2 lane and 2 lane + 1, by one warp:
@@ -244,13 +267,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   using K = TcCfg;
   constexpr uint64_t kLimit = tc::kWaitLimitNs;
   const Dims& d = a.d;
-  const ChunkPos q = chunk_pos(d, blockIdx.x);
+  const ChunkPos q = chunk_pos_u32(d, blockIdx.x);
   const int Qc = q.Qc, last = Qc - 1;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                        ~uintptr_t(1023));
   float* Mm = reinterpret_cast<float*>(sm + K::oM);
-  unsigned char* stage = sm + K::oStage;
   __shared__ TcSmem s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // TMEM reads: warp (qd, hf) reads rows 16 qd + (lane & 15) of its lane
@@ -266,7 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(&s.bar_in, 1);
     mbar_init(&s.bar_st, 1);
+    mbar_init(&s.bar_p1a, 1);
     mbar_init(&s.bar_p1, 1);
+    mbar_init(&s.bar_p2a, 1);
+    mbar_init(&s.bar_p2b, 1);
     mbar_init(&s.bar_p2, 1);
     mbar_init(&s.bar_drain, 1);
     s.abort_flag = 0;
@@ -299,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm("mov.u32 %0, %%nsmid;" : "=r"(nsm));
     const int64_t nb = (int64_t)blockIdx.x + nsm;
     if (nb < (int64_t)gridDim.x) {
-      const ChunkPos qn = chunk_pos(d, nb);
+      const ChunkPos qn = chunk_pos_u32(d, (uint32_t)nb);
       const int64_t o = ((qn.b * d.H + qn.h) * d.nc + qn.c) * d.P * d.N;
       const uint32_t bytes = (uint32_t)(d.P * d.N * 4);
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.S + o), "r"(bytes) : "memory");
@@ -314,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_4d(sm + K::oC + jb * K::kTile, &tm_c, &s.bar_in, 64 * jb, grp, tok, bb);
     }
   }
-  if (warp == 0) {  // the per-token scalars, while the loads are in flight
+  if (warp == 1) {  // the per-token scalars, while the loads are in flight
     const DtScan r = dt_scan_warp(a, q, lane);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -371,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)  // G = dy x^T (K = p)
         mma_bf16_ss(tmem + K::tG, kmaj(dDY, kk), kmaj(dX, kk), id_kk64, kk > 0);
+      mma_commit(&s.bar_p1a);  // the Q x Q phase starts on these while the rest run
 #pragma unroll
       for (int t3 = 0; t3 < 3; ++t3) {
         const uint64_t lk = st_term(t3, false), lm = st_term(t3, true);
@@ -385,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
-  ok = ok && mbar_wait(&s.bar_p1, 0, abort_flag, kLimit);
+  ok = ok && mbar_wait(&s.bar_p1a, 0, abort_flag, kLimit);
   ok = __syncthreads_and(ok);
   if (ok) {
     tc_fence_after();
@@ -420,6 +446,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         store_terms8(sm + K::oZw, K::kTile, t, k16, zwv + 8 * c);
       }
     }
+  }
+  ok = ok && mbar_wait(&s.bar_p1, 0, abort_flag, kLimit);  // the Lam products
+  if (ok) {
+    tc_fence_after();
     // ---- B Lam^T: the row sums x_s . (Lam B_s), then scaled by el_s and written back
     {
       uint32_t r[16];
@@ -453,36 +483,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         SSD_TMEM_ST_16x32bx2_X16_HALF32(tq + K::tDB + 64 * hf + 16 * half, r);
       }
     }
-    // ---- h_in terms over the Lam terms (the MMAs that read those are done)
-    split_state(sm + K::oS, reinterpret_cast<const float*>(sm + K::oHin), nullptr, tid);
     tmem_wait_st();
   }
   tc_fence_before();
   fence_proxy_async_smem();  // the split tiles are read by the MMAs
   ok = __syncthreads_and(ok);
 
-  // ---- MMAs, second round: K^T dy, Z^T C (accumulating), dy h_in, Zw B
+  // ---- MMAs, second round: K^T dy, Z^T C (accumulating on the scaled Lam
+  // products), Zw B; then, once its terms are written, dy h_in.  dx, dB and dC
+  // complete on barriers of their own, so the read-out of one overlaps the next.
   if (ok && warp == 0) {
     tc_fence_after();
     if (elect_one()) {
 #pragma unroll
       for (int t3 = 0; t3 < 3; ++t3) {
-        const uint64_t k_mn = qq_term(K::oK, t3, true), z_mn = qq_term(K::oZ, t3, true);
-        const uint64_t zw_k = qq_term(K::oZw, t3, false), h_mn = st_term(t3, true);
+        const uint64_t k_mn = qq_term(K::oK, t3, true);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // K = t, t, p, s
+        for (int kk = 0; kk < 4; ++kk)  // K = t
           mma_bf16_ss(tmem + K::tDx, mnmaj(k_mn, kk), mnmaj(dDYmn, kk), id_mm64, 1);
+      }
+      mma_commit(&s.bar_p2a);
+#pragma unroll
+      for (int t3 = 0; t3 < 3; ++t3) {
+        const uint64_t z_mn = qq_term(K::oZ, t3, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // K = t
           mma_bf16_ss(tmem + K::tDB, mnmaj(z_mn, kk), mnmaj(dCmn, kk), id_mm128, 1);
-          mma_bf16_ss(tmem + K::tDC2, kmaj(dDY, kk), mnmaj(h_mn, kk), id_km128, t3 > 0 || kk > 0);
+      }
+      mma_commit(&s.bar_p2b);
+#pragma unroll
+      for (int t3 = 0; t3 < 3; ++t3) {
+        const uint64_t zw_k = qq_term(K::oZw, t3, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // K = s
           mma_bf16_ss(tmem + K::tDC1, kmaj(zw_k, kk), mnmaj(dBmn, kk), id_km128, t3 > 0 || kk > 0);
-        }
+      }
+    }
+    __syncwarp();
+  }
+  // ---- h_in terms over the Lam terms (the MMAs that read those are done)
+  if (ok) split_state(sm + K::oS, reinterpret_cast<const float*>(sm + K::oHin), nullptr, tid);
+  fence_proxy_async_smem();  // the h_in terms are read by the MMAs
+  ok = __syncthreads_and(ok);
+  if (ok && warp == 0) {
+    tc_fence_after();
+    if (elect_one()) {
+#pragma unroll
+      for (int t3 = 0; t3 < 3; ++t3) {
+        const uint64_t h_mn = st_term(t3, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // K = p
+          mma_bf16_ss(tmem + K::tDC2, kmaj(dDY, kk), mnmaj(h_mn, kk), id_km128, t3 > 0 || kk > 0);
       }
       mma_commit(&s.bar_p2);
     }
     __syncwarp();
   }
-  ok = ok && mbar_wait(&s.bar_p2, 0, abort_flag, kLimit);
-  ok = __syncthreads_and(ok);
+  ok = ok && mbar_wait(&s.bar_p2a, 0, abort_flag, kLimit);
   if (ok) {
     tc_fence_after();
     // this thread's token row is staged whole (rows past the chunk's last token are
@@ -497,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       load8(sm + K::oDY, row, (c0 >> 3) + 1, dyv + 8);
       const float ws = s.w[row], Dh = a.D ? a.D[q.h] : 0.f;
       // columns c0 .. c0 + 15: box c0 / 32, 16-byte chunks 4 hf .. 4 hf + 3 of its row
-      unsigned char* box = stage + K::oStDx + (uint32_t)(c0 >> 5) * K::kTile;
+      unsigned char* box = sm + K::oStDx + (uint32_t)(c0 >> 5) * K::kTile;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         *reinterpret_cast<float4*>(box + sw_chunk(row, 4 * hf + i)) =
@@ -506,6 +563,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         fmaf(ws, __uint_as_float(r[4 * i + 2]), Dh * dyv[4 * i + 2]),
                         fmaf(ws, __uint_as_float(r[4 * i + 3]), Dh * dyv[4 * i + 3]));
     }
+  }
+  ok = ok && mbar_wait(&s.bar_p2b, 0, abort_flag, kLimit);
+  if (ok) {
+    tc_fence_after();
     // ---- dB of this head = w_s [Z^T C + el_s x Lam] (states n in [c1, c1 + 32))
     {
       uint32_t r[32];
@@ -514,13 +575,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDB + 64 * hf + 16, r_hi);
       SSD_TMEM_WAIT_LD_32(r);
       const float ws = s.w[row];
-      unsigned char* box = stage + K::oStDB + (uint32_t)(c1 >> 5) * K::kTile;  // a whole 32-column row
+      unsigned char* box = sm + K::oStDB + (uint32_t)(c1 >> 5) * K::kTile;  // a whole 32-column row
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         *reinterpret_cast<float4*>(box + sw_chunk(row, i)) =
             make_float4(ws * __uint_as_float(r[4 * i]), ws * __uint_as_float(r[4 * i + 1]),
                         ws * __uint_as_float(r[4 * i + 2]), ws * __uint_as_float(r[4 * i + 3]));
     }
+  }
+  ok = ok && mbar_wait(&s.bar_p2, 0, abort_flag, kLimit);
+  if (ok) {
+    tc_fence_after();
     // ---- dC of this head = Zw B + e_t dy h_in, and the row sums C_t . (h_in^T dy_t)
     {
       uint32_t r2[32], r1[32];
@@ -541,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 32; ++i) cy = fmaf(cv[i], __uint_as_float(r2[i]), cy);
       s.cyp[row][2 * hf + (lane >> 4)] = cy;
-      unsigned char* box = stage + K::oStDC + (uint32_t)(c1 >> 5) * K::kTile;
+      unsigned char* box = sm + K::oStDC + (uint32_t)(c1 >> 5) * K::kTile;
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         *reinterpret_cast<float4*>(box + sw_chunk(row, i)) =
@@ -559,10 +624,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
       // dx, dB and dC of this head and chunk: 32-column boxes, rows past L clipped
       const int h = (int)q.h, tk = (int)q.t0, bb = (int)q.b;
-      for (int k = 0; k < 2; ++k) tma_store_4d(&tm_dx, stage + K::oStDx + k * K::kTile, 32 * k, h, tk, bb);
+      for (int k = 0; k < 2; ++k) tma_store_4d(&tm_dx, sm + K::oStDx + k * K::kTile, 32 * k, h, tk, bb);
       for (int k = 0; k < 4; ++k) {
-        tma_store_4d(&tm_dbh, stage + K::oStDB + k * K::kTile, 32 * k, h, tk, bb);
-        tma_store_4d(&tm_dch, stage + K::oStDC + k * K::kTile, 32 * k, h, tk, bb);
+        tma_store_4d(&tm_dbh, sm + K::oStDB + k * K::kTile, 32 * k, h, tk, bb);
+        tma_store_4d(&tm_dch, sm + K::oStDC + k * K::kTile, 32 * k, h, tk, bb);
       }
       bulk_commit_group();
     }
@@ -573,9 +638,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // The pairs whose decay spans token k: S_k = sum_{u >= k} R(u, k) with the
     // row prefix R(u, k) = sum_{s < k} M(u, s) w_s, and the column sum of M
-    // below the diagonal (for dw).  R goes where the K terms were (the MMAs
+    // below the diagonal (for dw).  R goes over the state terms (the MMAs
     // that read them are done).  Row u's prefix: four threads, 16 columns each.
-    float* Rm = reinterpret_cast<float*>(sm + K::oK);  // [u][k], rows of kMs
+    float* Rm = reinterpret_cast<float*>(sm + K::oR);  // [u][k], rows of kMs
     {
       const int u = tid >> 2, sg = tid & 3;
       float pre[16], run = 0.f;
@@ -717,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   using K = StCfg;
   constexpr uint64_t kLimit = tc::kWaitLimitNs;
   const Dims& d = a.d;
-  const ChunkPos q = chunk_pos(d, blockIdx.x);
+  const ChunkPos q = chunk_pos_u32(d, blockIdx.x);
   const int Qc = q.Qc, last = Qc - 1;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
