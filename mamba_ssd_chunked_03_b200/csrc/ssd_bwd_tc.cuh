@@ -227,15 +227,16 @@ __device__ __forceinline__ DtScan dt_scan_warp(const KArgs& a, const ChunkPos& q
 }
 
 // The three-term split of a fp32 state [p][n] as its bulk load leaves it in
-// shared memory: this thread's 16-byte chunk k16 = tid % 16 of rows
-// p = tid / 16 + 16 j, into the MN-major term tiles at `area` (two 64-column
-// blocks a term); returns the thread's share of <v, w> when `w` is given.
-__device__ __forceinline__ float split_state(unsigned char* area, const float* v, const float* w, int tid) {
-  const int k16 = tid & 15;
+// shared memory, into the MN-major term tiles at `area` (two 64-column blocks
+// a term): items i = first, first + stride, .. < 1024, item i being the
+// 16-byte chunk k16 = i % 16 of row p = i / 16.  Returns the thread's share of
+// <v, w> when `w` is given.
+__device__ __forceinline__ float split_state(unsigned char* area, const float* v, const float* w, int first,
+                                             int stride) {
   float dot = 0.f;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int p = (tid >> 4) + 16 * j;
+#pragma unroll 2
+  for (int it = first; it < 64 * 16; it += stride) {
+    const int p = it >> 4, k16 = it & 15;
     const float4* vr = reinterpret_cast<const float4*>(v + p * 128 + 8 * k16);
     const float4 x0 = vr[0], x1 = vr[1];
     const float e[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
@@ -301,6 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_dy);
     tma_prefetch_desc(&tm_b);
     tma_prefetch_desc(&tm_c);
+    tma_prefetch_desc(&tm_dx);
+    tma_prefetch_desc(&tm_dbh);
+    tma_prefetch_desc(&tm_dch);
   }
   if (warp == 0) {
     tmem_alloc(&s.tmem_base, K::kTmemCols);
@@ -339,31 +343,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_4d(sm + K::oC + jb * K::kTile, &tm_c, &s.bar_in, 64 * jb, grp, tok, bb);
     }
   }
-  if (warp == 1) {  // the per-token scalars, while the loads are in flight
-    const DtScan r = dt_scan_warp(a, q, lane);
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int t = 2 * lane + e;
-      s.w[t] = r.w[e];
-      s.cs[t] = r.cs[e];
-      s.seg[t] = r.seg[e];
-      s.el[t] = r.el[e];
-      s.ein[t] = r.ein[e];
-      s.dg[t] = 0.f;
-    }
-  }
-  // the Lam terms (the h_in ones come after the first MMAs) and <Lam, h_in>
-  bool ok = mbar_wait(&s.bar_st, 0, abort_flag, kLimit);
-  if (ok) {
-    float lh = split_state(sm + K::oS, reinterpret_cast<const float*>(sm + K::oLam),
-                           reinterpret_cast<const float*>(sm + K::oHin), tid);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) lh += __shfl_xor_sync(0xffffffffu, lh, o);
-    if (lane == 0) s.red[warp] = lh;
-  }
-  fence_proxy_async_smem();  // the Lam terms are read by the MMAs
-  ok = __syncthreads_and(ok);
-
   // descriptors: K-major tiles (rows along K) and MN-major ones (rows along K,
   // the 64-element blocks of M or N one tile apart)
   const uint64_t dX = sw128_desc(smem_u32(sm + K::oX), 16, 1024);
@@ -385,18 +364,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     return sw128_desc(smem_u32(sm + K::oS + (uint32_t)t3 * 2 * K::kTile), mn ? K::kTile : 16, 1024);
   };
 
-  // ---- MMAs, first round: CB, G, B Lam^T, x Lam
+  // Warp 0 forms C B^T and G as soon as their tiles land, warp 1 the per-token
+  // scalars, warps 2-7 the Lam terms (the h_in ones come after the first MMAs)
+  // and <Lam, h_in>.
+  bool ok = true;
+  float lh = 0.f;
+  if (warp == 0) {
+    ok = mbar_wait(&s.bar_in, 0, abort_flag, kLimit);
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // CB = C B^T (K = n)
+          mma_bf16_ss(tmem + K::tCB, kmaj(dC, kk), kmaj(dB, kk), id_kk64, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // G = dy x^T (K = p)
+          mma_bf16_ss(tmem + K::tG, kmaj(dDY, kk), kmaj(dX, kk), id_kk64, kk > 0);
+        mma_commit(&s.bar_p1a);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    const DtScan r = dt_scan_warp(a, q, lane);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int t = 2 * lane + e;
+      s.w[t] = r.w[e];
+      s.cs[t] = r.cs[e];
+      s.seg[t] = r.seg[e];
+      s.el[t] = r.el[e];
+      s.ein[t] = r.ein[e];
+      s.dg[t] = 0.f;
+    }
+  } else {
+    ok = mbar_wait(&s.bar_st, 0, abort_flag, kLimit);
+    if (ok)
+      lh = split_state(sm + K::oS, reinterpret_cast<const float*>(sm + K::oLam),
+                       reinterpret_cast<const float*>(sm + K::oHin), tid - 64, kThreads - 64);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lh += __shfl_xor_sync(0xffffffffu, lh, o);
+  if (lane == 0) s.red[warp] = lh;
+  fence_proxy_async_smem();  // the Lam terms are read by the MMAs
+  ok = __syncthreads_and(ok);
+
+  // ---- MMAs, first round, continued: B Lam^T, x Lam
   ok = ok && mbar_wait(&s.bar_in, 0, abort_flag, kLimit);  // every thread reads the tiles later
   if (warp == 0 && __all_sync(0xffffffffu, ok)) {
     tc_fence_after();
     if (elect_one()) {
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)  // CB = C B^T (K = n)
-        mma_bf16_ss(tmem + K::tCB, kmaj(dC, kk), kmaj(dB, kk), id_kk64, kk > 0);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)  // G = dy x^T (K = p)
-        mma_bf16_ss(tmem + K::tG, kmaj(dDY, kk), kmaj(dX, kk), id_kk64, kk > 0);
-      mma_commit(&s.bar_p1a);  // the Q x Q phase starts on these while the rest run
 #pragma unroll
       for (int t3 = 0; t3 < 3; ++t3) {
         const uint64_t lk = st_term(t3, false), lm = st_term(t3, true);
@@ -412,7 +428,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
   ok = ok && mbar_wait(&s.bar_p1a, 0, abort_flag, kLimit);
-  ok = __syncthreads_and(ok);
   if (ok) {
     tc_fence_after();
     // ---- the Q x Q matrices: row t, columns s in [c0, c0 + 16)
@@ -521,8 +536,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
-  // ---- h_in terms over the Lam terms (the MMAs that read those are done)
-  if (ok) split_state(sm + K::oS, reinterpret_cast<const float*>(sm + K::oHin), nullptr, tid);
+  // ---- h_in terms over the Lam terms (the MMAs that read those are done), by
+  // warps 1-7 while warp 0 issues
+  if (ok && warp > 0) split_state(sm + K::oS, reinterpret_cast<const float*>(sm + K::oHin), nullptr, tid - 32, kThreads - 32);
   fence_proxy_async_smem();  // the h_in terms are read by the MMAs
   ok = __syncthreads_and(ok);
   if (ok && warp == 0) {
