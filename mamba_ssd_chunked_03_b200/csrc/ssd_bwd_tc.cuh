@@ -97,30 +97,14 @@ struct __align__(16) TcSmem {
   uint64_t bar_in, bar_st, bar_p1a, bar_p1, bar_p2a, bar_p2b, bar_p2, bar_drain;
   uint32_t tmem_base;
   int abort_flag, never;
-  float cs[64], w[64], el[64], ein[64], dg[64], nv[64], dw[64], dcs[64], nn[64];
+  __align__(16) float cs[64];  // cs, w and seg are read as 16-byte vectors
+  __align__(16) float w[64];
+  __align__(16) int seg[64];
+  float el[64], ein[64], dg[64], nv[64], dw[64], dcs[64], nn[64];
   float nxp[64][4], cyp[64][4];  // row sums, four shares a row
   float pair[64][8];             // the decay pair sums, in quarters
   float red[kThreads / 32];  // <Lam, h_in>, a share per warp
-  int seg[64];
 };
-
-// v = hi + mid + lo, each rounded to bf16 (see the file comment)
-__device__ __forceinline__ void split3(float v, __nv_bfloat16& hi, __nv_bfloat16& mid, __nv_bfloat16& lo) {
-  hi = __float2bfloat16_rn(v);
-  const float r1 = v - __bfloat162float(hi);
-  mid = __float2bfloat16_rn(r1);
-  lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-}
-
-// 8 bf16 values as one 16-byte chunk of a 128-byte row
-__device__ __forceinline__ uint4 pack8(const __nv_bfloat16 (&v)[8]) {
-  uint4 u;
-  u.x = (uint32_t)__bfloat16_as_ushort(v[0]) | ((uint32_t)__bfloat16_as_ushort(v[1]) << 16);
-  u.y = (uint32_t)__bfloat16_as_ushort(v[2]) | ((uint32_t)__bfloat16_as_ushort(v[3]) << 16);
-  u.z = (uint32_t)__bfloat16_as_ushort(v[4]) | ((uint32_t)__bfloat16_as_ushort(v[5]) << 16);
-  u.w = (uint32_t)__bfloat16_as_ushort(v[6]) | ((uint32_t)__bfloat16_as_ushort(v[7]) << 16);
-  return u;
-}
 
 // Byte offset of 16-byte chunk k16 of row r in a 128-byte-swizzled tile.
 __device__ __forceinline__ uint32_t sw_chunk(int r, int k16) {
@@ -138,16 +122,33 @@ __device__ __forceinline__ void load8(const unsigned char* tile, int r, int k16,
   }
 }
 
+// split3 of two values at once, as packed bf16 pairs (the first value in the
+// low half): bf16x2 roundings and fp32x2 differences, each difference exact
+// as in split3, so the terms are split3's.
+__device__ __forceinline__ void split3x2(float a, float b, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
+  const float2 v = make_float2(a, b), neg = make_float2(-1.f, -1.f);
+  const __nv_bfloat162 h = __float22bfloat162_rn(v);
+  const float2 r1 = __ffma2_rn(__bfloat1622float2(h), neg, v);
+  const __nv_bfloat162 m = __float22bfloat162_rn(r1);
+  const float2 r2 = __ffma2_rn(__bfloat1622float2(m), neg, r1);
+  const __nv_bfloat162 l = __float22bfloat162_rn(r2);
+  hi = reinterpret_cast<const uint32_t&>(h);
+  mid = reinterpret_cast<const uint32_t&>(m);
+  lo = reinterpret_cast<const uint32_t&>(l);
+}
+
 // Three-term split of 8 consecutive values of row r (chunk k16) into three
 // tiles `stride` bytes apart.
 __device__ __forceinline__ void store_terms8(unsigned char* tile, uint32_t stride, int r, int k16, const float* v) {
-  __nv_bfloat16 h[8], m[8], l[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) split3(v[i], h[i], m[i], l[i]);
+  uint4 h, m, l;
+  split3x2(v[0], v[1], h.x, m.x, l.x);
+  split3x2(v[2], v[3], h.y, m.y, l.y);
+  split3x2(v[4], v[5], h.z, m.z, l.z);
+  split3x2(v[6], v[7], h.w, m.w, l.w);
   const uint32_t off = sw_chunk(r, k16);
-  *reinterpret_cast<uint4*>(tile + off) = pack8(h);
-  *reinterpret_cast<uint4*>(tile + stride + off) = pack8(m);
-  *reinterpret_cast<uint4*>(tile + 2 * stride + off) = pack8(l);
+  *reinterpret_cast<uint4*>(tile + off) = h;
+  *reinterpret_cast<uint4*>(tile + stride + off) = m;
+  *reinterpret_cast<uint4*>(tile + 2 * stride + off) = l;
 }
 
 // chunk_pos in 32-bit arithmetic: the tensor-core kernels' grids (one CTA per
@@ -440,16 +441,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = row;
       const float cst = s.cs[t];
       const int segt = s.seg[t];
+      float csv[16], wv[16];
+      int sgv[16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 c4 = reinterpret_cast<const float4*>(s.cs + c0)[j];
+        const float4 w4 = reinterpret_cast<const float4*>(s.w + c0)[j];
+        const int4 g4 = reinterpret_cast<const int4*>(s.seg + c0)[j];
+        csv[4 * j] = c4.x, csv[4 * j + 1] = c4.y, csv[4 * j + 2] = c4.z, csv[4 * j + 3] = c4.w;
+        wv[4 * j] = w4.x, wv[4 * j + 1] = w4.y, wv[4 * j + 2] = w4.z, wv[4 * j + 3] = w4.w;
+        sgv[4 * j] = g4.x, sgv[4 * j + 1] = g4.y, sgv[4 * j + 2] = g4.z, sgv[4 * j + 3] = g4.w;
+      }
       float kv[16], zv[16], zwv[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int sc = c0 + i;
         const float g = __uint_as_float(rg[i]);
-        const bool in = t < Qc && sc <= t && s.seg[sc] == segt;
-        const float e = in ? expf(cst - s.cs[sc]) : 0.f;
+        const bool in = t < Qc && sc <= t && sgv[i] == segt;
+        const float e = in ? expf(cst - csv[i]) : 0.f;
         kv[i] = e * __uint_as_float(rcb[i]);
         zv[i] = e * g;
-        zwv[i] = zv[i] * s.w[sc];
+        zwv[i] = zv[i] * wv[i];
         Mm[t * K::kMs + sc] = kv[i] * g;
         if (sc == t && t < Qc) s.dg[t] = g;
       }
