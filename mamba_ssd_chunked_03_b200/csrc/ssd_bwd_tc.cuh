@@ -762,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
-  if (tid == 0) bulk_wait<0>();  // the gradient stores have read their staging before the CTA's memory goes
+  if (tid == 0) bulk_wait_read<0>();  // the gradient stores have read their staging before the CTA's memory goes
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -854,7 +854,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_load_4d(sm + K::oC + jb * K::kTile, &tm_c, &s.bar_in, 64 * jb, grp, tok, bb);
     }
   }
-  if (warp == 0) {  // the per-token scale factors, while the loads are in flight
+  if (warp == 1) {  // the per-token scale factors, while the loads are in flight
     const DtScan r = dt_scan_warp(a, q, lane);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -936,7 +936,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_store_3d(&tm_t, sm + K::oStT + k * K::kTile, 32 * k, 0, unit);
     }
     bulk_commit_group();
-    bulk_wait<0>();  // the stores have read their staging before the CTA's memory goes
+    bulk_wait_read<0>();  // the stores have read their staging before the CTA's memory goes
   }
   if (!ok && warp == 0) {
     mbar_wait(&s.bar_in, 0, never, kLimit);
