@@ -22,8 +22,8 @@ struct CudaLaunch {
   bool record(void* event) const { return cudaEventRecord(static_cast<cudaEvent_t>(event), stream) == cudaSuccess; }
   bool chunk_tc_ok(const ssd::bwd::KArgs& k) const { return ssd::bwd::chunk_tc_supported(k); }
   bool chunk_tc(const ssd::bwd::KArgs& k) const { return ssd::bwd::chunk_tc_launch(k, stream) == cudaSuccess; }
-  bool chunk_states_tc(const ssd::bwd::KArgs& k) const {
-    return ssd::bwd::chunk_states_tc_launch(k, stream) == cudaSuccess;
+  bool state_walk_tc(const ssd::bwd::KArgs& k, bool only_dh0) const {
+    return ssd::bwd::state_walk_tc_launch(k, only_dh0, stream) == cudaSuccess;
   }
 };
 

@@ -51,9 +51,10 @@
 //                        tokens, h_in and Lam; dB and dC per head
 //   k_bwd_group_sum      dB, dC summed over each group's heads
 //   k_bwd_param_sum      dA, dD summed over rows and chunks (fp64)
-//   (k_bwd_chunk_states, k_bwd_chunk_cb and k_bwd_chunk give way to
-//   k_bwd_chunk_states_tc and k_bwd_chunk_tc of ssd_bwd_tc.cuh, the same
-//   formulas on the tensor cores, where those take the call)
+//   (k_bwd_chunk_states and k_bwd_state_passing give way to
+//   k_bwd_state_walk_tc, k_bwd_chunk_cb and k_bwd_chunk to k_bwd_chunk_tc, of
+//   ssd_bwd_tc.cuh: the same formulas on the tensor cores, where those take
+//   the call)
 //
 // With SSD_BWD_DINITIAL_ONLY only the first two run.
 //
@@ -891,8 +892,9 @@ inline KArgs make_kargs(const ssd_bwd_args* a, const Plan& pl) {
 inline unsigned blocks_for(int64_t n) { return (unsigned)((n + kThreads - 1) / kThreads); }
 
 // A launcher may offer the tensor-core kernels (ssd_bwd_tc.cuh, GPU builds):
-// chunk_tc_ok(k) says whether they take the call, chunk_states_tc(k) and
-// chunk_tc(k) run them in place of k_bwd_chunk_states and k_bwd_chunk.
+// chunk_tc_ok(k) says whether they take the call, state_walk_tc(k, only_dh0)
+// runs the chunk states and their scans in place of k_bwd_chunk_states and
+// k_bwd_state_passing, and chunk_tc(k) runs in place of k_bwd_chunk.
 // The host emulation of the kernels offers none and runs the CUDA-core ones.
 template <class L, class = void>
 struct has_chunk_tc : std::false_type {};
@@ -909,16 +911,16 @@ ssd_status enqueue_typed(const KArgs& k, const Plan& pl, void* const events[2], 
   const unsigned chunk_ctas = (unsigned)(d.b * d.nc * d.H);
   bool tensor_cores = false;
   if constexpr (has_chunk_tc<Launch>::value && std::is_same<T, __nv_bfloat16>::value) tensor_cores = launch.chunk_tc_ok(k);
-  if (tensor_cores) {
+  if (tensor_cores) {  // the chunk states and their scans in one pass
     if constexpr (has_chunk_tc<Launch>::value)
-      if (!launch.chunk_states_tc(k)) return SSD_ERR_CUDA;
-  } else if (!launch(&k_bwd_chunk_states<T>, chunk_ctas, pl.smem_states, k)) {
-    return SSD_ERR_CUDA;
+      if (!launch.state_walk_tc(k, only_dh0)) return SSD_ERR_CUDA;
+  } else {
+    if (!launch(&k_bwd_chunk_states<T>, chunk_ctas, pl.smem_states, k)) return SSD_ERR_CUDA;
+    const int64_t n_states = d.b * d.H * d.P * d.N;
+    if (!((d.P * d.N) % 4 == 0 ? launch(&k_bwd_state_passing<4>, blocks_for(n_states / 4), (size_t)0, k)
+                                : launch(&k_bwd_state_passing<1>, blocks_for(n_states), (size_t)0, k)))
+      return SSD_ERR_CUDA;
   }
-  const int64_t n_states = d.b * d.H * d.P * d.N;
-  if (!((d.P * d.N) % 4 == 0 ? launch(&k_bwd_state_passing<4>, blocks_for(n_states / 4), (size_t)0, k)
-                              : launch(&k_bwd_state_passing<1>, blocks_for(n_states), (size_t)0, k)))
-    return SSD_ERR_CUDA;
   if (only_dh0) {  // k_bwd_chunk is not run: its timing events mark the same point
     if (events[0] && !(launch.record(events[0]) && launch.record(events[1]))) return SSD_ERR_CUDA;
     return SSD_OK;

@@ -769,71 +769,111 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
 }
 
-// The chunk states of the backward's recomputation on the tensor cores (the
-// formulas of k_bwd_chunk_states): per (batch row, chunk, head)
+// The chunk states and their scan in one pass: one CTA walks the chunks of
+// one (batch row, head), forward or backward,
 //
-//   S = (diag(cS) x)^T B,   cS_t = dt_t E(last, t)     the chunk's end state from zero
-//   T = (diag(cT) dy)^T C,  cT_t = e_t                  its part of dLoss/dh_in
+//   forward:  h_in(0) = h0,        h_in(c+1) = dec_c h_in(c) + S_c
+//   backward: Lam(nc-1) = dfinal,  Lam(c-1)   = dec_c Lam(c) + T_c,   dh0 = Lam(-1)
 //
-// with the scaled x and dy as three bf16 terms (fp32 accuracy, as above) and
-// B, C as loaded; M = 64 (p), N = 128 (n), K = 64 tokens.  256 TMEM columns
-// and 97 KB of shared memory, so two CTAs share an SM.
-struct StCfg {
+// with the chunk's products (the formulas of k_bwd_chunk_states)
+//
+//   S_c = (diag(cS) x_c)^T B_c,   cS_t = dt_t E(last, t)
+//   T_c = (diag(cT) dy_c)^T C_c,  cT_t = e_t
+//
+// formed by tcgen05 MMAs (M = 64 rows p, N = 128 states, K = 64 tokens) with
+// the scaled x or dy as three bf16 terms, and the scans of k_bwd_state_passing;
+// h_in goes to S and Lam to T, and the per-chunk products never reach memory.
+// Roles
+// (384 threads):
+//   warp 0      TMA loads (one thread): x or dy, and B or C, 3 chunks ahead
+//   warp 1      MMAs (one elected lane) into two 128-column accumulators
+//   warp 2      per-chunk scalars (dt_scan_warp): the token scales and dec_c
+//   warps 3-7   the scaled tile's three-term split, two chunks' terms in flight
+//   warps 8-11  the state: warp 8 + q owns rows 16 q .. 16 q + 15 (TMEM lane
+//               quadrant q) and all 128 states, in fp32 registers; each chunk's
+//               entering state is staged (128-byte swizzled 32-column boxes)
+//               and sent by bulk tensor stores, two stagings in flight
+// Every wait is bounded; a CTA that gives up drains its copies, MMAs and
+// stores, frees its tensor memory and exits.
+struct WalkCfg {
+  static constexpr int kThreads = 384;
+  static constexpr int kRing = 3;  // input slots
+  static constexpr int kScan = 4;  // per-chunk scalar slots
+  static constexpr int kSplitWarp0 = 3, kSplitWarps = 5, kStateWarp0 = 8, kStateWarps = 4;
   static constexpr uint32_t kTile = 8192;
-  static constexpr uint32_t oX = 0;                  // x  [t][p]
-  static constexpr uint32_t oDY = oX + kTile;        // dy [t][p]
-  static constexpr uint32_t oB = oDY + kTile;        // B  [t][n]
-  static constexpr uint32_t oC = oB + 2 * kTile;     // C  [t][n]
-  static constexpr uint32_t oXs = oC + 2 * kTile;    // cS x terms [3][t][p]
-  static constexpr uint32_t oDs = oXs + 3 * kTile;   // cT dy terms [3][t][p]
-  static constexpr uint32_t oEnd = oDs + 3 * kTile;
+  static constexpr uint32_t kInSlot = 3 * kTile;  // x or dy [t][p], then B or C [t][n] (two n-blocks)
+  static constexpr uint32_t oIn = 0;
+  static constexpr uint32_t kTermSlot = 3 * kTile;  // the three terms [t][p]
+  static constexpr uint32_t oTerms = oIn + kRing * kInSlot;
+  static constexpr uint32_t kStageSlot = 4 * kTile;  // a state: four 32-column fp32 boxes
+  static constexpr uint32_t oStage = oTerms + 2 * kTermSlot;
+  static constexpr uint32_t oEnd = oStage + 2 * kStageSlot;
   static constexpr uint32_t kSmemBytes = oEnd + 1024;
-  static constexpr uint32_t tS = 0, tT = 128, kTmemCols = 256;
-  // S and T staged for their bulk stores over B, C and the terms (dead once the
-  // MMAs are done): 32-column fp32 boxes of 64 rows, 128-byte swizzle
-  static constexpr uint32_t oStS = oB, oStT = oB + 4 * kTile;
-  static_assert(oStT + 4 * kTile <= oEnd, "state staging");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static constexpr uint32_t kTmemCols = 256;
 };
 
-struct __align__(16) StSmem {
-  uint64_t bar_in, bar_mma, bar_drain;
+struct __align__(16) WalkSmem {
+  uint64_t full_in[WalkCfg::kRing], in_free[WalkCfg::kRing];
+  uint64_t scan_full[WalkCfg::kScan], scan_empty[WalkCfg::kScan];
+  uint64_t terms_full[2], terms_free[2];
+  uint64_t mma_done[2], acc_free[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort_flag, never;
-  float cS[64], cT[64];
+  float f[WalkCfg::kScan][64];  // token scales: dt_t E(last, t) forward, e_t backward
+  float dec[WalkCfg::kScan];    // the chunk's decay
 };
 
-__global__ void __launch_bounds__(kThreads, 2)
-    k_bwd_chunk_states_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dy,
-                          const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
-                          const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_t,
-                          const KArgs a) {
-  using K = StCfg;
+// Grid: both directions of every (row, head) (blockIdx.x = 2 unit + dir), or
+// only the backward ones (blockIdx.x = unit) when `both` is 0.
+__global__ void __launch_bounds__(WalkCfg::kThreads, 1)
+    k_bwd_state_walk_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dy,
+                        const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
+                        const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_t,
+                        const KArgs a, int both) {
+  using K = WalkCfg;
   constexpr uint64_t kLimit = tc::kWaitLimitNs;
   const Dims& d = a.d;
-  const ChunkPos q = chunk_pos_u32(d, blockIdx.x);
-  const int Qc = q.Qc, last = Qc - 1;
+  const uint32_t unit = both ? blockIdx.x >> 1 : blockIdx.x;  // b H + h
+  const int dir = both ? (int)(blockIdx.x & 1) : 1;           // 0 forward (h_in), 1 backward (Lam)
+  const uint32_t H = (uint32_t)d.H;
+  const int64_t bb = unit / H, hh = unit - (uint32_t)bb * H, gg = (uint32_t)hh / (uint32_t)d.hpg;
+  const int nc = (int)d.nc;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                        ~uintptr_t(1023));
-  __shared__ StSmem s;
+  __shared__ WalkSmem s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, hf = warp >> 2;
-  const int row = 16 * qd + (lane & 15);          // state row p this thread reads from TMEM
-  const int c1 = 64 * hf + 32 * (lane >> 4);      // and its states n in [c1, c1 + 32)
   volatile int* abort_flag = &s.abort_flag;
   volatile int* never = &s.never;
+  const CUtensorMap* mX = dir ? &tm_dy : &tm_x;
+  const CUtensorMap* mY = dir ? &tm_c : &tm_b;
+  const CUtensorMap* mO = dir ? &tm_t : &tm_s;
+  auto chunk_of = [&](int k) { return dir ? nc - 1 - k : k; };
 
   if (tid == 0) {
-    mbar_init(&s.bar_in, 1);
-    mbar_init(&s.bar_mma, 1);
-    mbar_init(&s.bar_drain, 1);
+    for (int i = 0; i < K::kRing; ++i) {
+      mbar_init(&s.full_in[i], 1);
+      mbar_init(&s.in_free[i], K::kSplitWarps + 1);  // the split warps (x or dy) and the MMAs' commit (B or C)
+    }
+    for (int i = 0; i < K::kScan; ++i) {
+      mbar_init(&s.scan_full[i], 1);
+      mbar_init(&s.scan_empty[i], K::kSplitWarps + K::kStateWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.terms_full[i], K::kSplitWarps);
+      mbar_init(&s.terms_free[i], 1);
+      mbar_init(&s.mma_done[i], 1);
+      mbar_init(&s.acc_free[i], K::kStateWarps);
+    }
+    mbar_init(&s.drain, 1);
     s.abort_flag = 0;
     s.never = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_dy);
-    tma_prefetch_desc(&tm_b);
-    tma_prefetch_desc(&tm_c);
+    tma_prefetch_desc(mX);
+    tma_prefetch_desc(mY);
+    tma_prefetch_desc(mO);
   }
   if (warp == 0) {
     tmem_alloc(&s.tmem_base, K::kTmemCols);
@@ -843,108 +883,172 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  const uint32_t tq = tmem + ((uint32_t)(32 * qd) << 16);
-  if (tid == 0) {
-    const int col = (int)(q.h * d.P), tok = (int)q.t0, bb = (int)q.b, grp = (int)q.g;
-    mbar_arrive_expect_tx(&s.bar_in, 6 * K::kTile);
-    tma_load_3d(sm + K::oX, &tm_x, &s.bar_in, col, tok, bb);
-    tma_load_3d(sm + K::oDY, &tm_dy, &s.bar_in, col, tok, bb);
-    for (int jb = 0; jb < 2; ++jb) {
-      tma_load_4d(sm + K::oB + jb * K::kTile, &tm_b, &s.bar_in, 64 * jb, grp, tok, bb);
-      tma_load_4d(sm + K::oC + jb * K::kTile, &tm_c, &s.bar_in, 64 * jb, grp, tok, bb);
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA loads
+    if (lane == 0) {
+      int last = -1;
+      for (int k = 0; k < nc; ++k) {
+        const int sl = k % K::kRing;
+        if (k >= K::kRing && !mbar_wait(&s.in_free[sl], ((k / K::kRing) - 1) & 1, abort_flag, kLimit)) break;
+        const int tok = chunk_of(k) * 64;
+        unsigned char* base = sm + K::oIn + sl * K::kInSlot;
+        mbar_arrive_expect_tx(&s.full_in[sl], K::kInSlot);
+        tma_load_3d(base, mX, &s.full_in[sl], (int)(hh * d.P), tok, (int)bb);
+        for (int jb = 0; jb < 2; ++jb)
+          tma_load_4d(base + (1 + jb) * K::kTile, mY, &s.full_in[sl], 64 * jb, (int)gg, tok, (int)bb);
+        last = k;
+      }
+      if (*abort_flag)  // let the copies in flight land before the CTA's memory goes
+        for (int k = last - (K::kRing - 1) < 0 ? 0 : last - (K::kRing - 1); k <= last; ++k)
+          mbar_wait(&s.full_in[k % K::kRing], (k / K::kRing) & 1, never, kLimit);
     }
-  }
-  if (warp == 1) {  // the per-token scale factors, while the loads are in flight
-    const DtScan r = dt_scan_warp(a, q, lane);
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      s.cS[2 * lane + e] = r.w[e] * r.el[e];
-      s.cT[2 * lane + e] = r.ein[e];
-    }
-    // the chunk's decay, e of its last token (0 when a sequence starts inside it)
-    if (lane == (last >> 1)) a.dec[(q.b * d.H + q.h) * d.nc + q.c] = (last & 1) ? r.ein[1] : r.ein[0];
-  }
-  __syncthreads();
-  bool ok = mbar_wait(&s.bar_in, 0, abort_flag, kLimit);
-  if (ok) {
-    // the scaled x and dy as three bf16 terms: row t = tid / 4, columns p in [16 (tid % 4), +16)
-    const int t = tid >> 2, k0 = 2 * (tid & 3);
-    float v[16];
-    load8(sm + K::oX, t, k0, v);
-    load8(sm + K::oX, t, k0 + 1, v + 8);
-    const float fs = s.cS[t], ft = s.cT[t];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] *= fs;
-    store_terms8(sm + K::oXs, K::kTile, t, k0, v);
-    store_terms8(sm + K::oXs, K::kTile, t, k0 + 1, v + 8);
-    load8(sm + K::oDY, t, k0, v);
-    load8(sm + K::oDY, t, k0 + 1, v + 8);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] *= ft;
-    store_terms8(sm + K::oDs, K::kTile, t, k0, v);
-    store_terms8(sm + K::oDs, K::kTile, t, k0 + 1, v + 8);
-  }
-  fence_proxy_async_smem();  // the terms are read by the MMAs
-  ok = __syncthreads_and(ok);
-  if (ok && warp == 0) {
-    tc_fence_after();
-    const uint64_t dBmn = sw128_desc(smem_u32(sm + K::oB), K::kTile, 1024);
-    const uint64_t dCmn = sw128_desc(smem_u32(sm + K::oC), K::kTile, 1024);
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMAs: S or T of chunk k = terms^T (B or C)
     constexpr uint32_t id = idesc_bf16(64, 128, 1, 1);  // A = terms^T (MN-major), B MN-major
-    if (elect_one()) {
+    for (int k = 0; k < nc; ++k) {
+      const int sl = k % K::kRing, ts = k & 1;
+      bool ok = mbar_wait_warp(&s.full_in[sl], (k / K::kRing) & 1, abort_flag, kLimit);
+      ok = ok && mbar_wait_warp(&s.terms_full[ts], (k >> 1) & 1, abort_flag, kLimit);
+      if (ok && k >= 2) ok = mbar_wait_warp(&s.acc_free[ts], ((k >> 1) - 1) & 1, abort_flag, kLimit);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t dY = sw128_desc(smem_u32(sm + K::oIn + sl * K::kInSlot + K::kTile), K::kTile, 1024);
 #pragma unroll
-      for (int t3 = 0; t3 < 3; ++t3) {
-        const uint64_t xs = sw128_desc(smem_u32(sm + K::oXs + t3 * K::kTile), K::kTile, 1024);
-        const uint64_t ds = sw128_desc(smem_u32(sm + K::oDs + t3 * K::kTile), K::kTile, 1024);
+        for (int t3 = 0; t3 < 3; ++t3) {
+          const uint64_t xs = sw128_desc(smem_u32(sm + K::oTerms + ts * K::kTermSlot + t3 * K::kTile), K::kTile, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // K = tokens
-          mma_bf16_ss(tmem + K::tS, mnmaj(xs, kk), mnmaj(dBmn, kk), id, t3 > 0 || kk > 0);
-          mma_bf16_ss(tmem + K::tT, mnmaj(ds, kk), mnmaj(dCmn, kk), id, t3 > 0 || kk > 0);
+          for (int kk = 0; kk < 4; ++kk)  // K = tokens
+            mma_bf16_ss(tmem + 128 * ts, mnmaj(xs, kk), mnmaj(dY, kk), id, t3 > 0 || kk > 0);
+        }
+        mma_commit(&s.mma_done[ts]);
+        mma_commit(&s.in_free[sl]);
+        mma_commit(&s.terms_free[ts]);
+      }
+      __syncwarp();
+    }
+    if (elect_one()) {  // every MMA (and its commits) done before the CTA's memory goes
+      mma_commit(&s.drain);
+      mbar_wait(&s.drain, 0, never, kLimit);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------ per-chunk scalars
+    for (int k = 0; k < nc; ++k) {
+      const int ss = k % K::kScan;
+      if (k >= K::kScan && !mbar_wait_warp(&s.scan_empty[ss], ((k / K::kScan) - 1) & 1, abort_flag, kLimit)) break;
+      ChunkPos q;
+      q.b = bb, q.h = hh, q.g = gg, q.c = chunk_of(k), q.t0 = q.c * d.Q;
+      const int64_t left = d.L - q.t0;
+      q.Qc = (int)(left < d.Q ? left : d.Q);
+      const int last = q.Qc - 1;
+      const DtScan r = dt_scan_warp(a, q, lane);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) s.f[ss][2 * lane + e] = dir ? r.ein[e] : r.w[e] * r.el[e];
+      if (lane == (last >> 1)) s.dec[ss] = (last & 1) ? r.ein[1] : r.ein[0];  // 0 when a sequence starts inside
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.scan_full[ss]);
+    }
+  } else if (warp < K::kStateWarp0) {
+    // ------------------------------------------------ the scaled tile's terms
+    const int st = tid - 32 * K::kSplitWarp0;
+    for (int k = 0; k < nc; ++k) {
+      const int sl = k % K::kRing, ss = k % K::kScan, ts = k & 1;
+      bool ok = mbar_wait_warp(&s.full_in[sl], (k / K::kRing) & 1, abort_flag, kLimit);
+      ok = ok && mbar_wait_warp(&s.scan_full[ss], (k / K::kScan) & 1, abort_flag, kLimit);
+      if (ok && k >= 2) ok = mbar_wait_warp(&s.terms_free[ts], ((k >> 1) - 1) & 1, abort_flag, kLimit);
+      if (!ok) break;
+      const unsigned char* X = sm + K::oIn + sl * K::kInSlot;
+      unsigned char* terms = sm + K::oTerms + ts * K::kTermSlot;
+      for (int it = st; it < 64 * 8; it += 32 * K::kSplitWarps) {  // row t, 16-byte chunk k16 of p
+        const int t = it >> 3, k16 = it & 7;
+        float v[8];
+        load8(X, t, k16, v);
+        const float ft = s.f[ss][t];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] *= ft;
+        store_terms8(terms, K::kTile, t, k16, v);
+      }
+      fence_proxy_async_smem();  // the terms are read by the MMAs
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s.terms_full[ts]);
+        mbar_arrive(&s.in_free[sl]);
+        mbar_arrive(&s.scan_empty[ss]);
+      }
+    }
+  } else {
+    // ------------------------------------------------ the state
+    const int qd = warp & 3;
+    const int row = 16 * qd + (lane & 15);  // state row p
+    const int cb = 32 * (lane >> 4);        // states n = 64 h2 + cb + [0, 32), h2 = 0, 1
+    const uint32_t tq = tmem + ((uint32_t)(32 * qd) << 16);
+    const bool issuer = warp == K::kStateWarp0 && lane == 0;
+    const int64_t e0 = ((int64_t)unit * d.P + row) * d.N + cb;
+    const float* init = dir ? a.dfinal : a.h0;
+    float hv[64];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) hv[32 * h2 + i] = init ? init[e0 + 64 * h2 + i] : 0.f;
+    bool done = true;
+    for (int k = 0; k < nc; ++k) {
+      const int ab = k & 1, ss = k % K::kScan;
+      unsigned char* stage = sm + K::oStage + ab * K::kStageSlot;
+      if (issuer && k >= 2) bulk_wait_read<1>();  // the stores of chunk k - 2 have read this staging
+      named_barrier_sync(1, 32 * K::kStateWarps);
+      // the state entering (forward) or leaving (backward) chunk k: row `row`, a
+      // whole 32-column row of boxes 2 h2 + cb / 32
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        unsigned char* box = stage + (uint32_t)(2 * h2 + (cb >> 5)) * K::kTile;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<float4*>(box + sw_chunk(row, i)) =
+              make_float4(hv[32 * h2 + 4 * i], hv[32 * h2 + 4 * i + 1], hv[32 * h2 + 4 * i + 2], hv[32 * h2 + 4 * i + 3]);
+      }
+      bool ok = mbar_wait_warp(&s.mma_done[ab], (k >> 1) & 1, abort_flag, kLimit);
+      ok = ok && mbar_wait_warp(&s.scan_full[ss], (k / K::kScan) & 1, abort_flag, kLimit);
+      if (ok) {
+        tc_fence_after();
+        const float dc = s.dec[ss];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t r[32];
+          uint32_t* r_hi = r + 16;
+          // warp-uniform address: lanes 16-31 read 32 columns further (cb)
+          SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + 128 * ab + 64 * h2, r);
+          SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + 128 * ab + 64 * h2 + 16, r_hi);
+          SSD_TMEM_WAIT_LD_32(r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) hv[32 * h2 + i] = fmaf(dc, hv[32 * h2 + i], __uint_as_float(r[i]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&s.acc_free[ab]);
+          mbar_arrive(&s.scan_empty[ss]);
         }
       }
-      mma_commit(&s.bar_mma);
+      fence_proxy_async_smem();  // the staged state is read by the bulk stores
+      if (named_barrier_any(2, 32 * K::kStateWarps, !ok)) {
+        done = false;
+        break;
+      }
+      if (issuer) {
+        const int u = (int)((int64_t)unit * nc + chunk_of(k));
+        for (int j = 0; j < 4; ++j) tma_store_3d(mO, stage + j * K::kTile, 32 * j, 0, u);
+        bulk_commit_group();
+      }
     }
-    __syncwarp();
-  }
-  ok = ok && mbar_wait(&s.bar_mma, 0, abort_flag, kLimit);
-  ok = __syncthreads_and(ok);
-  if (ok) {
-    tc_fence_after();
+    if (done && dir == 1 && a.dh0)
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      uint32_t r[32];
-      uint32_t* r_hi = r + 16;
-      const uint32_t col = (which ? K::tT : K::tS) + 64 * hf;
-      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + col, r);
-      SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + col + 16, r_hi);
-      SSD_TMEM_WAIT_LD_32(r);
-      // this thread's row, states [c1, c1 + 32): a whole row of box c1 / 32
-      unsigned char* box = sm + (which ? K::oStT : K::oStS) + (uint32_t)(c1 >> 5) * K::kTile;
+      for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        *reinterpret_cast<float4*>(box + sw_chunk(row, i)) =
-            make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
-                        __uint_as_float(r[4 * i + 3]));
-    }
-    fence_proxy_async_smem();  // the staged states are read by the bulk stores
-  }
-  ok = __syncthreads_and(ok);
-  if (ok && tid == 0) {
-    const int unit = (int)((q.b * d.H + q.h) * d.nc + q.c);
-    for (int k = 0; k < 4; ++k) {
-      tma_store_3d(&tm_s, sm + K::oStS + k * K::kTile, 32 * k, 0, unit);
-      tma_store_3d(&tm_t, sm + K::oStT + k * K::kTile, 32 * k, 0, unit);
-    }
-    bulk_commit_group();
-    bulk_wait_read<0>();  // the stores have read their staging before the CTA's memory goes
-  }
-  if (!ok && warp == 0) {
-    mbar_wait(&s.bar_in, 0, never, kLimit);
-    if (elect_one()) {
-      mma_commit(&s.bar_drain);
-      mbar_wait(&s.bar_drain, 0, never, kLimit);
-    }
-    __syncwarp();
+        for (int i = 0; i < 32; ++i) a.dh0[e0 + 64 * h2 + i] = hv[32 * h2 + i];
+    if (issuer) bulk_wait_read<0>();  // the stores have read their staging before the CTA's memory goes
   }
   tc_fence_before();
   __syncthreads();
@@ -972,19 +1076,21 @@ inline bool chunk_tc_maps(const KArgs& k, CUtensorMap* tx, CUtensorMap* tdy, CUt
          tc::make_map_bc(tb, k.B, d.N, d.G, d.L, d.b) && tc::make_map_bc(tc_, k.C, d.N, d.G, d.L, d.b);
 }
 
-inline cudaError_t chunk_states_tc_launch(const KArgs& k, cudaStream_t st) {
+// The forward and backward state walks (only the backward one when just
+// dLoss/dh0 is wanted): one CTA per (row, head) and direction.
+inline cudaError_t state_walk_tc_launch(const KArgs& k, bool only_dh0, cudaStream_t st) {
   const Dims& d = k.d;
   CUtensorMap tx, tdy, tb, tc_, ts, tt;
   if (!chunk_tc_maps(k, &tx, &tdy, &tb, &tc_)) return cudaErrorInvalidValue;
-  // the states' bulk stores: S and T are (b, H, nc, P, N) fp32, one P x N block per chunk and head
   if (!tc::make_map_f32_blocks(&ts, k.S, d.N, d.P, d.b * d.H * d.nc) ||
       !tc::make_map_f32_blocks(&tt, k.T, d.N, d.P, d.b * d.H * d.nc))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)StCfg::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_state_walk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)WalkCfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  k_bwd_chunk_states_tc<<<(unsigned)(d.b * d.nc * d.H), kThreads, StCfg::kSmemBytes, st>>>(tx, tdy, tb, tc_, ts, tt,
-                                                                                               k);
+  const unsigned grid = (unsigned)(d.b * d.H * (only_dh0 ? 1 : 2));
+  k_bwd_state_walk_tc<<<grid, WalkCfg::kThreads, WalkCfg::kSmemBytes, st>>>(tx, tdy, tb, tc_, ts, tt, k,
+                                                                            only_dh0 ? 0 : 1);
   return cudaGetLastError();
 }
 
