@@ -823,7 +823,7 @@ def run_bwd(args, dist, dev, world, rank):
                      "cb_flops_in_kernel": f_cb},
         "e2e": {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": E},
-        "gpu_launches": 5 * K,
+        "gpu_launches": (4 if ssd.bwd_path(g["x"], g["dy"], g["B"], g["C"]) == "tcgen05" else 6) * K,
         "clocks": clock_stats,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -7,7 +7,7 @@ problem and a packed one compared in full, and the benchmark's c1 layout
 row: every gradient of a row except dA and dD depends on that row's inputs
 only, and dA, dD (sums over rows) are compared at the smaller sizes.  bf16
 calls at headdim 64, dstate 128 without a gate run the tensor-core kernels
-(k_bwd_chunk_states_tc, k_bwd_chunk_tc); the others the CUDA-core ones, so
+(k_bwd_state_walk_tc, k_bwd_chunk_tc); the others the CUDA-core ones, so
 both are held to the same tolerances here."""
 import numpy as np
 import pytest
