@@ -269,8 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using K = TcCfg;
   constexpr uint64_t kLimit = tc::kWaitLimitNs;
   const Dims& d = a.d;
-  const ChunkPos q = chunk_pos_u32(d, blockIdx.x);
-  const int Qc = q.Qc, last = Qc - 1;
+  const uint32_t n_units = (uint32_t)(d.b * d.nc * d.H);
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                        ~uintptr_t(1023));
@@ -316,26 +315,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   const uint32_t tq = tmem + ((uint32_t)(32 * qd) << 16);
-  if (tid == 0) {
-    // this chunk's states first (the threads wait on them first): Lam and h_in,
-    // one contiguous P x N block each
-    const int64_t so = ((q.b * d.H + q.h) * d.nc + q.c) * d.P * d.N;
-    mbar_arrive_expect_tx(&s.bar_st, 2 * K::kStateBytes);
-    bulk_load(sm + K::oLam, a.T + so, K::kStateBytes, &s.bar_st);
-    bulk_load(sm + K::oHin, a.S + so, K::kStateBytes, &s.bar_st);
-    // the chunk states of the CTA one wave later, into L2 (a hint: the grid
-    // runs one CTA an SM, so that CTA comes about an SM count later)
-    uint32_t nsm;
-    asm("mov.u32 %0, %%nsmid;" : "=r"(nsm));
-    const int64_t nb = (int64_t)blockIdx.x + nsm;
-    if (nb < (int64_t)gridDim.x) {
-      const ChunkPos qn = chunk_pos_u32(d, (uint32_t)nb);
-      const int64_t o = ((qn.b * d.H + qn.h) * d.nc + qn.c) * d.P * d.N;
-      const uint32_t bytes = (uint32_t)(d.P * d.N * 4);
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.S + o), "r"(bytes) : "memory");
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.T + o), "r"(bytes) : "memory");
-    }
-    const int col = (int)(q.h * d.P), tok = (int)q.t0, bb = (int)q.b, grp = (int)q.g;
+  // A unit's loads: its tiles (x, dy, B, C) on bar_in, its states (Lam and
+  // h_in, one contiguous P x N block each) on bar_st.
+  auto issue_tiles = [&](const ChunkPos& u) {
+    const int col = (int)(u.h * d.P), tok = (int)u.t0, bb = (int)u.b, grp = (int)u.g;
     mbar_arrive_expect_tx(&s.bar_in, 6 * K::kTile);
     tma_load_3d(sm + K::oX, &tm_x, &s.bar_in, col, tok, bb);
     tma_load_3d(sm + K::oDY, &tm_dy, &s.bar_in, col, tok, bb);
@@ -343,6 +326,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_4d(sm + K::oB + jb * K::kTile, &tm_b, &s.bar_in, 64 * jb, grp, tok, bb);
       tma_load_4d(sm + K::oC + jb * K::kTile, &tm_c, &s.bar_in, 64 * jb, grp, tok, bb);
     }
+  };
+  auto state_offset = [&](const ChunkPos& u) { return ((u.b * d.H + u.h) * d.nc + u.c) * d.P * d.N; };
+  auto issue_states = [&](const ChunkPos& u) {
+    const int64_t so = state_offset(u);
+    mbar_arrive_expect_tx(&s.bar_st, 2 * K::kStateBytes);
+    bulk_load(sm + K::oLam, a.T + so, K::kStateBytes, &s.bar_st);
+    bulk_load(sm + K::oHin, a.S + so, K::kStateBytes, &s.bar_st);
+  };
+  if (tid == 0) {  // the first unit (the grid has at most one CTA per unit)
+    const ChunkPos u0 = chunk_pos_u32(d, blockIdx.x);
+    issue_states(u0);
+    issue_tiles(u0);
   }
   // descriptors: K-major tiles (rows along K) and MN-major ones (rows along K,
   // the 64-element blocks of M or N one tile apart)
@@ -365,13 +360,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     return sw128_desc(smem_u32(sm + K::oS + (uint32_t)t3 * 2 * K::kTile), mn ? K::kTile : 16, 1024);
   };
 
+  // The CTA's units, one after the other: each unit's loads are issued during
+  // the previous unit's tail, so its start finds them landed.
+  bool ok = true;
+  int it = 0;
+  for (uint32_t unit = blockIdx.x; unit < n_units; unit += gridDim.x, ++it) {
+  const uint32_t par = (uint32_t)it & 1u;  // every barrier completes one phase a unit
+  const ChunkPos q = chunk_pos_u32(d, unit);
+  const int Qc = q.Qc, last = Qc - 1;
+  const uint32_t next = unit + gridDim.x;
+  if (tid == 0 && next < n_units) {  // the next unit's states into L2 (its bulk loads come in the tail)
+    const int64_t o = state_offset(chunk_pos_u32(d, next));
+    const uint32_t bytes = (uint32_t)(d.P * d.N * 4);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.S + o), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.T + o), "r"(bytes) : "memory");
+  }
   // Warp 0 forms C B^T and G as soon as their tiles land, warp 1 the per-token
   // scalars, warps 2-7 the Lam terms (the h_in ones come after the first MMAs)
   // and <Lam, h_in>.
-  bool ok = true;
   float lh = 0.f;
   if (warp == 0) {
-    ok = mbar_wait(&s.bar_in, 0, abort_flag, kLimit);
+    ok = mbar_wait(&s.bar_in, par, abort_flag, kLimit);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       if (elect_one()) {
@@ -398,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       s.dg[t] = 0.f;
     }
   } else {
-    ok = mbar_wait(&s.bar_st, 0, abort_flag, kLimit);
+    ok = mbar_wait(&s.bar_st, par, abort_flag, kLimit);
     if (ok)
       lh = split_state(sm + K::oS, reinterpret_cast<const float*>(sm + K::oLam),
                        reinterpret_cast<const float*>(sm + K::oHin), tid - 64, kThreads - 64);
@@ -410,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   ok = __syncthreads_and(ok);
 
   // ---- MMAs, first round, continued: B Lam^T, x Lam
-  ok = ok && mbar_wait(&s.bar_in, 0, abort_flag, kLimit);  // every thread reads the tiles later
+  ok = ok && mbar_wait(&s.bar_in, par, abort_flag, kLimit);  // every thread reads the tiles later
   if (warp == 0 && __all_sync(0xffffffffu, ok)) {
     tc_fence_after();
     if (elect_one()) {
@@ -428,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
-  ok = ok && mbar_wait(&s.bar_p1a, 0, abort_flag, kLimit);
+  ok = ok && mbar_wait(&s.bar_p1a, par, abort_flag, kLimit);
   if (ok) {
     tc_fence_after();
     // ---- the Q x Q matrices: row t, columns s in [c0, c0 + 16)
@@ -474,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-  ok = ok && mbar_wait(&s.bar_p1, 0, abort_flag, kLimit);  // the Lam products
+  ok = ok && mbar_wait(&s.bar_p1, par, abort_flag, kLimit);  // the Lam products
   if (ok) {
     tc_fence_after();
     // ---- B Lam^T: the row sums x_s . (Lam B_s), then scaled by el_s and written back
@@ -567,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
-  ok = ok && mbar_wait(&s.bar_p2a, 0, abort_flag, kLimit);
+  ok = ok && mbar_wait(&s.bar_p2a, par, abort_flag, kLimit);
   if (ok) {
     tc_fence_after();
     // this thread's token row is staged whole (rows past the chunk's last token are
@@ -592,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         fmaf(ws, __uint_as_float(r[4 * i + 3]), Dh * dyv[4 * i + 3]));
     }
   }
-  ok = ok && mbar_wait(&s.bar_p2b, 0, abort_flag, kLimit);
+  ok = ok && mbar_wait(&s.bar_p2b, par, abort_flag, kLimit);
   if (ok) {
     tc_fence_after();
     // ---- dB of this head = w_s [Z^T C + el_s x Lam] (states n in [c1, c1 + 32))
@@ -611,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ws * __uint_as_float(r[4 * i + 2]), ws * __uint_as_float(r[4 * i + 3]));
     }
   }
-  ok = ok && mbar_wait(&s.bar_p2, 0, abort_flag, kLimit);
+  ok = ok && mbar_wait(&s.bar_p2, par, abort_flag, kLimit);
   if (ok) {
     tc_fence_after();
     // ---- dC of this head = Zw B + e_t dy h_in, and the row sums C_t . (h_in^T dy_t)
@@ -658,6 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_store_4d(&tm_dch, sm + K::oStDC + k * K::kTile, 32 * k, h, tk, bb);
       }
       bulk_commit_group();
+      if (next < n_units) issue_tiles(chunk_pos_u32(d, next));  // the tiles are read no more
     }
     // ---- the decay gradients (the tail of k_bwd_chunk, on the row sums above)
     for (int t = tid; t < Qc; t += kThreads) {
@@ -752,10 +762,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         a.dD_part[pi] = dD;
       }
     }
-  } else if (warp == 0) {
-    // a wait gave up: let this CTA's copies and MMAs finish before its memory goes
-    mbar_wait(&s.bar_st, 0, never, kLimit);
-    mbar_wait(&s.bar_in, 0, never, kLimit);
+  }
+  // the next unit's states go over this unit's staging once the stores have read it
+  if (ok && tid == 0 && next < n_units) {
+    bulk_wait_read<0>();
+    issue_states(chunk_pos_u32(d, next));
+  }
+  tc_fence_before();
+  ok = __syncthreads_and(ok);
+  tc_fence_after();
+  if (!ok) break;
+  }
+  if (!ok && warp == 0) {
+    // a wait gave up: let this CTA's copies (the current unit's: the next
+    // unit's are issued only after a unit went through) and MMAs finish
+    // before its memory goes
+    mbar_wait(&s.bar_st, (uint32_t)it & 1u, never, kLimit);
+    mbar_wait(&s.bar_in, (uint32_t)it & 1u, never, kLimit);
     if (elect_one()) {
       mma_commit(&s.bar_drain);
       mbar_wait(&s.bar_drain, 0, never, kLimit);
@@ -1105,8 +1128,12 @@ inline cudaError_t chunk_tc_launch(const KArgs& k, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)TcCfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  k_bwd_chunk_tc<<<(unsigned)(d.b * d.nc * d.H), kThreads, TcCfg::kSmemBytes, st>>>(tx, tdy, tb, tc_, tdx, tdb, tdc,
-                                                                                       k);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  const int64_t units = d.b * d.nc * d.H;  // a persistent grid, one CTA an SM, walking the units
+  const unsigned grid = (unsigned)(units < sms ? units : sms);
+  k_bwd_chunk_tc<<<grid, kThreads, TcCfg::kSmemBytes, st>>>(tx, tdy, tb, tc_, tdx, tdb, tdc, k);
   return cudaGetLastError();
 }
 
