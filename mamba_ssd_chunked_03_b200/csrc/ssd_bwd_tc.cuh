@@ -695,6 +695,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < 16; ++j) Rm[u * K::kMs + 16 * sg + j] = off + pre[j];
     }
+    // the next unit's states go over this unit's staging once the stores have
+    // read it, early enough to land during the rest of this tail
+    if (tid == 0 && next < n_units) {
+      bulk_wait_read<0>();
+      issue_states(chunk_pos_u32(d, next));
+    }
     __syncthreads();
     for (int i = tid; i < 4 * Qc; i += kThreads) {
       const int k = i >> 2, qq = i & 3;
@@ -762,11 +768,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         a.dD_part[pi] = dD;
       }
     }
-  }
-  // the next unit's states go over this unit's staging once the stores have read it
-  if (ok && tid == 0 && next < n_units) {
-    bulk_wait_read<0>();
-    issue_states(chunk_pos_u32(d, next));
   }
   tc_fence_before();
   ok = __syncthreads_and(ok);
