@@ -178,20 +178,31 @@ struct DtScan {
   float w[2], cs[2], el[2], ein[2];
   int seg[2];
 };
-__device__ __forceinline__ DtScan dt_scan_warp(const KArgs& a, const ChunkPos& q, int lane) {
+// The loads behind a DtScan: dt of the two tokens and whether a sequence
+// starts at each, so that a loop can issue them a few chunks ahead.
+struct DtRaw {
+  float w[2];
+  bool v[2], f[2];
+};
+__device__ __forceinline__ DtRaw dt_load(const KArgs& a, const ChunkPos& q, int lane) {
   const Dims& d = a.d;
-  const float Ah = a.A[q.h];
   const float* dtp = a.dt + (q.b * d.L + q.t0) * d.H + q.h;
   const int32_t* sq = a.seq ? a.seq + q.b * d.L + q.t0 : nullptr;
-  DtScan r;
-  bool v[2], f[2];
+  DtRaw r;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int t = 2 * lane + e;
-    v[e] = t < q.Qc;
-    r.w[e] = v[e] ? dtp[(int64_t)t * d.H] : 0.f;
-    f[e] = v[e] && sq && q.t0 + t > 0 && sq[t] != sq[t - 1];  // a sequence starts at t
+    r.v[e] = t < q.Qc;
+    r.w[e] = r.v[e] ? dtp[(int64_t)t * d.H] : 0.f;
+    r.f[e] = r.v[e] && sq && q.t0 + t > 0 && sq[t] != sq[t - 1];  // a sequence starts at t
   }
+  return r;
+}
+__device__ __forceinline__ DtScan dt_scan_from(const DtRaw& raw, const ChunkPos& q, float Ah, int lane) {
+  DtScan r;
+  const bool* v = raw.v;
+  const bool* f = raw.f;
+  r.w[0] = raw.w[0], r.w[1] = raw.w[1];
   const float a0 = f[0] ? 0.f : r.w[0] * Ah;
   const float a1 = f[1] ? 0.f : a0 + r.w[1] * Ah;
   float sum = a1;                                         // the lane's sum since its last start
@@ -225,6 +236,9 @@ __device__ __forceinline__ DtScan dt_scan_warp(const KArgs& a, const ChunkPos& q
     r.ein[e] = v[e] && r.seg[e] == -1 ? expf(r.cs[e]) : 0.f;
   }
   return r;
+}
+__device__ __forceinline__ DtScan dt_scan_warp(const KArgs& a, const ChunkPos& q, int lane) {
+  return dt_scan_from(dt_load(a, q, lane), q, a.A[q.h], lane);
 }
 
 // The three-term split of a fp32 state [p][n] as its bulk load leaves it in
@@ -960,15 +974,28 @@ __global__ void __launch_bounds__(WalkCfg::kThreads, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------ per-chunk scalars
-    for (int k = 0; k < nc; ++k) {
-      const int ss = k % K::kScan;
-      if (k >= K::kScan && !mbar_wait_warp(&s.scan_empty[ss], ((k / K::kScan) - 1) & 1, abort_flag, kLimit)) break;
+    // (the loads of chunk k + 2 are issued before chunk k is scanned)
+    auto pos = [&](int k) {
       ChunkPos q;
       q.b = bb, q.h = hh, q.g = gg, q.c = chunk_of(k), q.t0 = q.c * d.Q;
       const int64_t left = d.L - q.t0;
       q.Qc = (int)(left < d.Q ? left : d.Q);
+      return q;
+    };
+    const float Ah = a.A[hh];
+    DtRaw r0{}, r1{};
+    if (nc > 0) r0 = dt_load(a, pos(0), lane);
+    if (nc > 1) r1 = dt_load(a, pos(1), lane);
+    for (int k = 0; k < nc; ++k) {
+      const int ss = k % K::kScan;
+      DtRaw r2{};
+      if (k + 2 < nc) r2 = dt_load(a, pos(k + 2), lane);
+      if (k >= K::kScan && !mbar_wait_warp(&s.scan_empty[ss], ((k / K::kScan) - 1) & 1, abort_flag, kLimit)) break;
+      const ChunkPos q = pos(k);
       const int last = q.Qc - 1;
-      const DtScan r = dt_scan_warp(a, q, lane);
+      const DtScan r = dt_scan_from(r0, q, Ah, lane);
+      r0 = r1;
+      r1 = r2;
 #pragma unroll
       for (int e = 0; e < 2; ++e) s.f[ss][2 * lane + e] = dir ? r.ein[e] : r.w[e] * r.el[e];
       if (lane == (last >> 1)) s.dec[ss] = (last & 1) ? r.ein[1] : r.ein[0];  // 0 when a sequence starts inside
