@@ -825,8 +825,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // (384 threads):
 //   warp 0      TMA loads (one thread): x or dy, and B or C, 3 chunks ahead
 //   warp 1      MMAs (one elected lane) into two 128-column accumulators
-//   warp 2      per-chunk scalars (dt_scan_warp): the token scales and dec_c
-//   warps 3-7   the scaled tile's three-term split, two chunks' terms in flight
+//   warps 2, 7  per-chunk scalars (dt_scan_from), alternate chunks each, their
+//               loads issued two of their chunks ahead: the token scales, dec_c
+//   warps 3-6   the scaled tile's three-term split, two chunks' terms in flight
 //   warps 8-11  the state: warp 8 + q owns rows 16 q .. 16 q + 15 (TMEM lane
 //               quadrant q) and all 128 states, in fp32 registers; each chunk's
 //               entering state is staged (128-byte swizzled 32-column boxes)
@@ -837,7 +838,9 @@ struct WalkCfg {
   static constexpr int kThreads = 384;
   static constexpr int kRing = 3;  // input slots
   static constexpr int kScan = 4;  // per-chunk scalar slots
-  static constexpr int kSplitWarp0 = 3, kSplitWarps = 5, kStateWarp0 = 8, kStateWarps = 4;
+  // warps: 0 TMA, 1 MMA, 2 and 7 the scalars (alternate chunks), 3-6 the split, 8-11 the state
+  static constexpr int kScanWarpA = 2, kScanWarpB = 7;
+  static constexpr int kSplitWarp0 = 3, kSplitWarps = 4, kStateWarp0 = 8, kStateWarps = 4;
   static constexpr uint32_t kTile = 8192;
   static constexpr uint32_t kInSlot = 3 * kTile;  // x or dy [t][p], then B or C [t][n] (two n-blocks)
   static constexpr uint32_t oIn = 0;
@@ -972,9 +975,11 @@ __global__ void __launch_bounds__(WalkCfg::kThreads, 1)
       mbar_wait(&s.drain, 0, never, kLimit);
     }
     __syncwarp();
-  } else if (warp == 2) {
+  } else if (warp == K::kScanWarpA || warp == K::kScanWarpB) {
     // ------------------------------------------------ per-chunk scalars
-    // (the loads of chunk k + 2 are issued before chunk k is scanned)
+    // (this warp's chunks k0, k0 + 2, ..; the loads of chunk k + 4 are issued
+    // before chunk k is scanned)
+    const int k0 = warp == K::kScanWarpA ? 0 : 1;
     auto pos = [&](int k) {
       ChunkPos q;
       q.b = bb, q.h = hh, q.g = gg, q.c = chunk_of(k), q.t0 = q.c * d.Q;
@@ -984,12 +989,12 @@ __global__ void __launch_bounds__(WalkCfg::kThreads, 1)
     };
     const float Ah = a.A[hh];
     DtRaw r0{}, r1{};
-    if (nc > 0) r0 = dt_load(a, pos(0), lane);
-    if (nc > 1) r1 = dt_load(a, pos(1), lane);
-    for (int k = 0; k < nc; ++k) {
+    if (k0 < nc) r0 = dt_load(a, pos(k0), lane);
+    if (k0 + 2 < nc) r1 = dt_load(a, pos(k0 + 2), lane);
+    for (int k = k0; k < nc; k += 2) {
       const int ss = k % K::kScan;
       DtRaw r2{};
-      if (k + 2 < nc) r2 = dt_load(a, pos(k + 2), lane);
+      if (k + 4 < nc) r2 = dt_load(a, pos(k + 4), lane);
       if (k >= K::kScan && !mbar_wait_warp(&s.scan_empty[ss], ((k / K::kScan) - 1) & 1, abort_flag, kLimit)) break;
       const ChunkPos q = pos(k);
       const int last = q.Qc - 1;
@@ -1013,7 +1018,10 @@ __global__ void __launch_bounds__(WalkCfg::kThreads, 1)
       if (!ok) break;
       const unsigned char* X = sm + K::oIn + sl * K::kInSlot;
       unsigned char* terms = sm + K::oTerms + ts * K::kTermSlot;
-      for (int it = st; it < 64 * 8; it += 32 * K::kSplitWarps) {  // row t, 16-byte chunk k16 of p
+      static_assert(64 * 8 == 4 * 32 * K::kSplitWarps, "four items a thread");
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {  // row t, 16-byte chunk k16 of p
+        const int it = st + 32 * K::kSplitWarps * j;
         const int t = it >> 3, k16 = it & 7;
         float v[8];
         load8(X, t, k16, v);
