@@ -97,13 +97,16 @@ struct __align__(16) TcSmem {
   uint64_t bar_in, bar_st, bar_p1a, bar_p1, bar_p2a, bar_p2b, bar_p2, bar_drain;
   uint32_t tmem_base;
   int abort_flag, never;
-  __align__(16) float cs[64];  // cs, w and seg are read as 16-byte vectors
-  __align__(16) float w[64];
-  __align__(16) int seg[64];
-  float el[64], ein[64], dg[64], nv[64], dw[64], dcs[64], nn[64];
+  // per-token arrays, one buffer per unit parity (warp 0 reads a unit's while the
+  // other warps write the next one's); cs, w and seg are read as 16-byte vectors
+  __align__(16) float cs[2][64];
+  __align__(16) float w[2][64];
+  __align__(16) int seg[2][64];
+  float el[2][64], ein[2][64], dg[2][64];
+  float nv[64], dw[64], dcs[64], nn[64];
   float nxp[64][4], cyp[64][4];  // row sums, four shares a row
   float pair[64][8];             // the decay pair sums, in quarters
-  float red[kThreads / 32];  // <Lam, h_in>, a share per warp
+  float red[2][kThreads / 32];  // <Lam, h_in>, a share per warp
 };
 
 // Byte offset of 16-byte chunk k16 of row r in a 128-byte-swizzled tile.
@@ -380,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int it = 0;
   for (uint32_t unit = blockIdx.x; unit < n_units; unit += gridDim.x, ++it) {
   const uint32_t par = (uint32_t)it & 1u;  // every barrier completes one phase a unit
+  const int pb = (int)par;                 // the per-token arrays alternate between units
   const ChunkPos q = chunk_pos_u32(d, unit);
   const int Qc = q.Qc, last = Qc - 1;
   const uint32_t next = unit + gridDim.x;
@@ -413,12 +417,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int t = 2 * lane + e;
-      s.w[t] = r.w[e];
-      s.cs[t] = r.cs[e];
-      s.seg[t] = r.seg[e];
-      s.el[t] = r.el[e];
-      s.ein[t] = r.ein[e];
-      s.dg[t] = 0.f;
+      s.w[pb][t] = r.w[e];
+      s.cs[pb][t] = r.cs[e];
+      s.seg[pb][t] = r.seg[e];
+      s.el[pb][t] = r.el[e];
+      s.ein[pb][t] = r.ein[e];
+      s.dg[pb][t] = 0.f;
     }
   } else {
     ok = mbar_wait(&s.bar_st, par, abort_flag, kLimit);
@@ -428,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lh += __shfl_xor_sync(0xffffffffu, lh, o);
-  if (lane == 0) s.red[warp] = lh;
+  if (lane == 0) s.red[pb][warp] = lh;
   fence_proxy_async_smem();  // the Lam terms are read by the MMAs
   ok = __syncthreads_and(ok);
 
@@ -462,15 +466,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       SSD_TMEM_WAIT_LD_16(rcb);
       SSD_TMEM_WAIT_LD_16(rg);
       const int t = row;
-      const float cst = s.cs[t];
-      const int segt = s.seg[t];
+      const float cst = s.cs[pb][t];
+      const int segt = s.seg[pb][t];
       float csv[16], wv[16];
       int sgv[16];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float4 c4 = reinterpret_cast<const float4*>(s.cs + c0)[j];
-        const float4 w4 = reinterpret_cast<const float4*>(s.w + c0)[j];
-        const int4 g4 = reinterpret_cast<const int4*>(s.seg + c0)[j];
+        const float4 c4 = reinterpret_cast<const float4*>(s.cs[pb] + c0)[j];
+        const float4 w4 = reinterpret_cast<const float4*>(s.w[pb] + c0)[j];
+        const int4 g4 = reinterpret_cast<const int4*>(s.seg[pb] + c0)[j];
         csv[4 * j] = c4.x, csv[4 * j + 1] = c4.y, csv[4 * j + 2] = c4.z, csv[4 * j + 3] = c4.w;
         wv[4 * j] = w4.x, wv[4 * j + 1] = w4.y, wv[4 * j + 2] = w4.z, wv[4 * j + 3] = w4.w;
         sgv[4 * j] = g4.x, sgv[4 * j + 1] = g4.y, sgv[4 * j + 2] = g4.z, sgv[4 * j + 3] = g4.w;
@@ -486,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         zv[i] = e * g;
         zwv[i] = zv[i] * wv[i];
         Mm[t * K::kMs + sc] = kv[i] * g;
-        if (sc == t && t < Qc) s.dg[t] = g;
+        if (sc == t && t < Qc) s.dg[pb][t] = g;
       }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -510,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       load8(sm + K::oX, sr, c0 >> 3, xv);
       load8(sm + K::oX, sr, (c0 >> 3) + 1, xv + 8);
       float nx = 0.f;
-      const float els = s.el[sr];
+      const float els = s.el[pb][sr];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float v = __uint_as_float(r[i]);
@@ -522,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---- x Lam: scaled by el_s and written back
     {
-      const float els = s.el[row];
+      const float els = s.el[pb][row];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t r[16];
@@ -603,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float dyv[16];
       load8(sm + K::oDY, row, c0 >> 3, dyv);
       load8(sm + K::oDY, row, (c0 >> 3) + 1, dyv + 8);
-      const float ws = s.w[row], Dh = a.D ? a.D[q.h] : 0.f;
+      const float ws = s.w[pb][row], Dh = a.D ? a.D[q.h] : 0.f;
       // columns c0 .. c0 + 15: box c0 / 32, 16-byte chunks 4 hf .. 4 hf + 3 of its row
       unsigned char* box = sm + K::oStDx + (uint32_t)(c0 >> 5) * K::kTile;
 #pragma unroll
@@ -625,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDB + 64 * hf, r);
       SSD_TMEM_LD_16x32bx2_X16_HALF32(tq + K::tDB + 64 * hf + 16, r_hi);
       SSD_TMEM_WAIT_LD_32(r);
-      const float ws = s.w[row];
+      const float ws = s.w[pb][row];
       unsigned char* box = sm + K::oStDB + (uint32_t)(c1 >> 5) * K::kTile;  // a whole 32-column row
 #pragma unroll
       for (int i = 0; i < 8; ++i)
@@ -652,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const unsigned char* ctile = sm + K::oC + hf * K::kTile;  // states 64 hf ..
 #pragma unroll
       for (int c = 0; c < 4; ++c) load8(ctile, row, 4 * (lane >> 4) + c, cv + 8 * c);
-      const float et = s.ein[row];
+      const float et = s.ein[pb][row];
       float cy = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) cy = fmaf(cv[i], __uint_as_float(r2[i]), cy);
@@ -686,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- the decay gradients (the tail of k_bwd_chunk, on the row sums above)
     for (int t = tid; t < Qc; t += kThreads) {
       s.nv[t] = s.nxp[t][0] + s.nxp[t][1] + s.nxp[t][2] + s.nxp[t][3];
-      s.dcs[t] = s.ein[t] * (s.cyp[t][0] + s.cyp[t][1] + s.cyp[t][2] + s.cyp[t][3]);
+      s.dcs[t] = s.ein[pb][t] * (s.cyp[t][0] + s.cyp[t][1] + s.cyp[t][2] + s.cyp[t][3]);
     }
     // The pairs whose decay spans token k: S_k = sum_{u >= k} R(u, k) with the
     // row prefix R(u, k) = sum_{s < k} M(u, s) w_s, and the column sum of M
@@ -700,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < 16; ++j) {
         const int sc = 16 * sg + j;
         pre[j] = run;
-        run = fmaf(Mm[u * K::kMs + sc], s.w[sc], run);
+        run = fmaf(Mm[u * K::kMs + sc], s.w[pb][sc], run);
       }
       s.pair[u][sg] = run;  // this segment's total
       __syncwarp();
@@ -731,18 +735,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = tid; t < Qc; t += kThreads) {
       const float col = s.pair[t][0] + s.pair[t][1] + s.pair[t][2] + s.pair[t][3];
       const float blk = s.pair[t][4] + s.pair[t][5] + s.pair[t][6] + s.pair[t][7];
-      s.dw[t] = fmaf(s.el[t], s.nv[t], col + Mm[t * K::kMs + t]);
-      s.nn[t] = s.el[t] * s.w[t] * s.nv[t];
+      s.dw[t] = fmaf(s.el[pb][t], s.nv[t], col + Mm[t * K::kMs + t]);
+      s.nn[t] = s.el[pb][t] * s.w[pb][t] * s.nv[t];
       s.pair[t][0] = blk;  // S_t
     }
-    __syncthreads();
+  }
+  tc_fence_before();
+  ok = __syncthreads_and(ok);
+  tc_fence_after();
+  if (!ok) break;
+  // The per-token tail on warp 0 while warps 1-7 begin the next unit (its
+  // per-token arrays are the other buffer).
     if (warp == 0) {
       // dl_k = S_k + sum_{t >= k} (h_in term)_t + sum_{s < k} N_s + e_last <Lam, h_in>,
       // tokens k = lane and lane + 32, the sums as warp scans
       float lh = 0.f;
 #pragma unroll
-      for (int i = 0; i < kThreads / 32; ++i) lh += s.red[i];
-      const float e_last = s.seg[last] == -1 ? expf(s.cs[last]) : 0.f;
+      for (int i = 0; i < kThreads / 32; ++i) lh += s.red[pb][i];
+      const float e_last = s.seg[pb][last] == -1 ? expf(s.cs[pb][last]) : 0.f;
       const int k0 = lane, k1 = lane + 32;
       const bool v0 = k0 <= last, v1 = k1 <= last;
       const float n0 = v0 ? s.nn[k0] : 0.f, n1 = v1 ? s.nn[k1] : 0.f;
@@ -760,16 +770,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float Ah = a.A[q.h];
       double dA = 0.0, dD = 0.0;
       if (v0) {
-        const float dl = s.seg[k0] == k0 ? 0.f : s.pair[k0][0] + suf0 + (pre0 - n0) + e_last * lh;
+        const float dl = s.seg[pb][k0] == k0 ? 0.f : s.pair[k0][0] + suf0 + (pre0 - n0) + e_last * lh;
         a.ddt[(q.b * d.L + q.t0 + k0) * d.H + q.h] = fmaf(Ah, dl, s.dw[k0]);
-        dA += (double)s.w[k0] * (double)dl;
-        dD += (double)s.dg[k0];
+        dA += (double)s.w[pb][k0] * (double)dl;
+        dD += (double)s.dg[pb][k0];
       }
       if (v1) {
-        const float dl = s.seg[k1] == k1 ? 0.f : s.pair[k1][0] + suf1 + (pre1 - n1) + e_last * lh;
+        const float dl = s.seg[pb][k1] == k1 ? 0.f : s.pair[k1][0] + suf1 + (pre1 - n1) + e_last * lh;
         a.ddt[(q.b * d.L + q.t0 + k1) * d.H + q.h] = fmaf(Ah, dl, s.dw[k1]);
-        dA += (double)s.w[k1] * (double)dl;
-        dD += (double)s.dg[k1];
+        dA += (double)s.w[pb][k1] * (double)dl;
+        dD += (double)s.dg[pb][k1];
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
@@ -782,11 +792,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         a.dD_part[pi] = dD;
       }
     }
-  }
-  tc_fence_before();
-  ok = __syncthreads_and(ok);
-  tc_fence_after();
-  if (!ok) break;
   }
   if (!ok && warp == 0) {
     // a wait gave up: let this CTA's copies (the current unit's: the next
