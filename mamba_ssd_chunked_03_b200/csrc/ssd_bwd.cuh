@@ -50,7 +50,8 @@
 //   k_bwd_chunk          per (b, c, h): the formulas above from the chunk's
 //                        tokens, h_in and Lam; dB and dC per head
 //   k_bwd_group_sum      dB, dC summed over each group's heads
-//   k_bwd_param_sum      dA, dD summed over rows and chunks (fp64)
+//   k_bwd_param_sum      dA, dD summed over rows and chunks (fp64, one CTA
+//                        a head, a fixed-order tree)
 //   (k_bwd_chunk_states and k_bwd_state_passing give way to
 //   k_bwd_state_walk_tc, k_bwd_chunk_cb and k_bwd_chunk to k_bwd_chunk_tc, of
 //   ssd_bwd_tc.cuh: the same formulas on the tensor cores, where those take
@@ -757,18 +758,36 @@ __global__ void __launch_bounds__(kThreads) k_bwd_group_sum(const KArgs a) {
 }
 
 // dA, dD (H): the per-chunk partial sums added in fp64, in a fixed order.
+// One CTA per head: each thread sums a fixed stride of the head's per-chunk
+// partials in fp64, then a tree over the threads in a fixed order (2 kThreads
+// doubles of dynamic shared memory), so the result does not vary run to run.
 __global__ void __launch_bounds__(kThreads) k_bwd_param_sum(const KArgs a) {
   const Dims& d = a.d;
-  const int64_t h = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (h >= d.H) return;
+  const int64_t h = blockIdx.x;
+  const int tid = threadIdx.x;
+  SSD_DYN_SMEM(sm);
+  double* ra = reinterpret_cast<double*>(sm);
+  double* rd = ra + kThreads;
   const int64_t n = d.b * d.nc;
   double sa = 0.0, sd = 0.0;
-  for (int64_t i = 0; i < n; ++i) {
+  for (int64_t i = tid; i < n; i += kThreads) {
     sa += a.dA_part[h * n + i];
     sd += a.dD_part[h * n + i];
   }
-  a.dA[h] = (float)sa;
-  if (a.dD) a.dD[h] = (float)sd;
+  ra[tid] = sa;
+  rd[tid] = sd;
+  __syncthreads();
+  for (int off = kThreads / 2; off > 0; off >>= 1) {
+    if (tid < off) {
+      ra[tid] += ra[tid + off];
+      rd[tid] += rd[tid + off];
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    a.dA[h] = (float)ra[0];
+    if (a.dD) a.dD[h] = (float)rd[0];
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -937,7 +956,7 @@ ssd_status enqueue_typed(const KArgs& k, const Plan& pl, void* const events[2], 
     if (events[1] && !launch.record(events[1])) return SSD_ERR_CUDA;
   }
   if (!launch(&k_bwd_group_sum, blocks_for(d.b * d.L * d.G * d.N), (size_t)0, k)) return SSD_ERR_CUDA;
-  if (!launch(&k_bwd_param_sum, blocks_for(d.H), (size_t)0, k)) return SSD_ERR_CUDA;
+  if (!launch(&k_bwd_param_sum, (unsigned)d.H, (size_t)(2 * kThreads * sizeof(double)), k)) return SSD_ERR_CUDA;
   return SSD_OK;
 }
 
