@@ -741,20 +741,31 @@ __global__ void __launch_bounds__(kThreads) k_bwd_chunk(const KArgs a) {
 }
 
 // dB, dC (b,L,G,N): the per-head gradients summed over each group's heads.
+// V consecutive states n..n+V-1 per thread: 16-byte loads and stores when
+// V = 4 (N a multiple of 4, dB and dC 16-byte aligned; dBh, dCh are 256-byte
+// aligned workspace), the heads of the group added in order.
+template <int V>
 __global__ void __launch_bounds__(kThreads) k_bwd_group_sum(const KArgs a) {
   const Dims& d = a.d;
-  const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  const int64_t i = ((int64_t)blockIdx.x * kThreads + threadIdx.x) * V;  // the thread's first output
   if (i >= d.b * d.L * d.G * d.N) return;
   const int64_t n = i % d.N, r = i / d.N;
   const int64_t g = r % d.G, bl = r / d.G;
-  float sb = 0.f, sc = 0.f;
+  const float* pb = a.dBh + (bl * d.H + g * d.hpg) * d.N + n;
+  const float* pc = a.dCh + (bl * d.H + g * d.hpg) * d.N + n;
+  float sb[V], sc[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) sb[k] = sc[k] = 0.f;
+#pragma unroll 4
   for (int64_t j = 0; j < d.hpg; ++j) {
-    const int64_t gi = (bl * d.H + g * d.hpg + j) * d.N + n;
-    sb += a.dBh[gi];
-    sc += a.dCh[gi];
+    float vb[V], vc[V];
+    ld_v<V>(pb + j * d.N, vb);
+    ld_v<V>(pc + j * d.N, vc);
+#pragma unroll
+    for (int k = 0; k < V; ++k) sb[k] += vb[k], sc[k] += vc[k];
   }
-  a.dB[i] = sb;
-  a.dC[i] = sc;
+  st_v<V>(a.dB + i, sb);
+  st_v<V>(a.dC + i, sc);
 }
 
 // dA, dD (H): the per-chunk partial sums added in fp64, in a fixed order.
@@ -955,7 +966,13 @@ ssd_status enqueue_typed(const KArgs& k, const Plan& pl, void* const events[2], 
     if (!launch(&k_bwd_chunk<T>, chunk_ctas, pl.smem_chunk, k)) return SSD_ERR_CUDA;
     if (events[1] && !launch.record(events[1])) return SSD_ERR_CUDA;
   }
-  if (!launch(&k_bwd_group_sum, blocks_for(d.b * d.L * d.G * d.N), (size_t)0, k)) return SSD_ERR_CUDA;
+  // 16-byte vectors when N allows them and the caller's dB, dC are 16-byte aligned
+  const int64_t n_bc = d.b * d.L * d.G * d.N;
+  const bool vec = d.N % 4 == 0 && (reinterpret_cast<uintptr_t>(k.dB) & 15) == 0 &&
+                   (reinterpret_cast<uintptr_t>(k.dC) & 15) == 0;
+  if (!(vec ? launch(&k_bwd_group_sum<4>, blocks_for(n_bc / 4), (size_t)0, k)
+            : launch(&k_bwd_group_sum<1>, blocks_for(n_bc), (size_t)0, k)))
+    return SSD_ERR_CUDA;
   if (!launch(&k_bwd_param_sum, (unsigned)d.H, (size_t)(2 * kThreads * sizeof(double)), k)) return SSD_ERR_CUDA;
   return SSD_OK;
 }
