@@ -287,6 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint64_t kLimit = tc::kWaitLimitNs;
   const Dims& d = a.d;
   const uint32_t n_units = (uint32_t)(d.b * d.nc * d.H);
+  constexpr int kStoreThread = kThreads - 1, kTileThread = kThreads - 33;  // lanes 31 of warps 7 and 6
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                        ~uintptr_t(1023));
@@ -676,7 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   ok = __syncthreads_and(ok);
 
   if (ok) {
-    if (tid == 0) {
+    // The bulk operations of the tail, each on the last lane of a warp with
+    // little of the tail's work (the column sums of its tokens are the shortest)
+    if (tid == kStoreThread) {
       // dx, dB and dC of this head and chunk: 32-column boxes, rows past L clipped
       const int h = (int)q.h, tk = (int)q.t0, bb = (int)q.b;
       for (int k = 0; k < 2; ++k) tma_store_4d(&tm_dx, sm + K::oStDx + k * K::kTile, 32 * k, h, tk, bb);
@@ -685,8 +688,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_store_4d(&tm_dch, sm + K::oStDC + k * K::kTile, 32 * k, h, tk, bb);
       }
       bulk_commit_group();
-      if (next < n_units) issue_tiles(chunk_pos_u32(d, next));  // the tiles are read no more
     }
+    if (tid == kTileThread && next < n_units) issue_tiles(chunk_pos_u32(d, next));  // the tiles are read no more
     // ---- the decay gradients (the tail of k_bwd_chunk, on the row sums above)
     for (int t = tid; t < Qc; t += kThreads) {
       s.nv[t] = s.nxp[t][0] + s.nxp[t][1] + s.nxp[t][2] + s.nxp[t][3];
@@ -715,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // the next unit's states go over this unit's staging once the stores have
     // read it, early enough to land during the rest of this tail
-    if (tid == 0 && next < n_units) {
+    if (tid == kStoreThread && next < n_units) {
       bulk_wait_read<0>();
       issue_states(chunk_pos_u32(d, next));
     }
@@ -805,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
-  if (tid == 0) bulk_wait_read<0>();  // the gradient stores have read their staging before the CTA's memory goes
+  if (tid == kStoreThread) bulk_wait_read<0>();  // the gradient stores have read their staging before the CTA's memory goes
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
