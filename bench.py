@@ -947,20 +947,26 @@ def main():
         return kernel_each[min(KE - 1, int(q * KE))]
     ms = max_over_ranks(ms, dist, dev)
 
-    # end to end through the public API: pinned host inputs -> device -> fwd -> host
+    # end to end through the public API from host memory: ssd_fwd_host takes the
+    # pinned host inputs, copies them in by row pieces on two streams, runs the
+    # forward on each piece and copies y and the final states back, one piece's
+    # copies in overlapping the previous piece's compute and copies out
     names = [k for k in ("x", "dt", "A", "B", "C", "D", "initial_states", "seq_idx") if host.get(k) is not None]
     pinned = {k: host[k].pin_memory() for k in names}
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     f_host = torch.empty(final.shape, dtype=final.dtype).pin_memory()
     h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in names)
     d2h = y_host.numel() * y_host.element_size() + f_host.numel() * f_host.element_size()
+    gen_flag = ssd.SSD_FLAG_GENERIC if args.generic else 0
+    hws = torch.empty(max(1, ssd.fwd_host_workspace_size(
+        host["x"], host["B"], shape.chunk_size, 0, host.get("seq_idx"), num_seqs, True, host.get("D") is not None,
+        False, host.get("initial_states") is not None, gen_flag)), dtype=torch.uint8, device=dev)
+    stream2 = torch.cuda.Stream(dev)
 
     def e2e_step():
-        for k in names:
-            g[k].copy_(pinned[k], non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
-        f_host.copy_(final, non_blocking=True)
+        ssd.fwd_host(pinned["x"], pinned["dt"], pinned["A"], pinned["B"], pinned["C"], pinned.get("D"),
+                     shape.chunk_size, pinned.get("initial_states"), pinned.get("seq_idx"), num_seqs,
+                     y=y_host, final_states=f_host, workspace=hws, device=dev, stream2=stream2, flags=gen_flag)
 
     for _ in range(3):
         e2e_step()

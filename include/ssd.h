@@ -172,6 +172,42 @@ SSD_API ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream);
  *    serialise them. */
 SSD_API ssd_status ssd_fwd_noalloc(const ssd_fwd_args* args, void* stream);
 
+/* ssd_fwd from and to HOST memory, with the copies overlapped: for callers
+ * whose inputs live on the host and who want the outputs back there.  The
+ * pointer fields of `args` (x, dt, A, B, C, D, z, initial_states, seq_idx, y,
+ * final_states) are host addresses, which should be pinned (page-locked,
+ * e.g. cudaHostAlloc) for the copies to run asynchronously and overlap; its
+ * workspace and timing_events fields are ignored.  The pages describe no such
+ * entry point; it has no counterpart there.
+ *
+ * The batch is taken in pieces of `rows_per_piece` rows (0: the library
+ * chooses, about a quarter of the batch), alternately on `stream` and
+ * `stream2`, each with its own set of device buffers.  For one piece the call
+ * enqueues the copies of its rows' inputs in (one cudaMemcpyAsync per
+ * tensor), ssd_fwd on them, and the copies of its y and final states out; so
+ * a piece's copies in run while the previous piece computes and copies out
+ * (on PCIe the two directions run at the same time).  With seq_idx the batch
+ * is one piece: final_states is then indexed by sequence id, and a call on
+ * part of the rows would clear the ids it does not see.  `stream2` may be
+ * NULL: everything then runs on `stream`, in order.
+ *
+ * `device_workspace` (256-byte aligned, at least ssd_fwd_host_workspace_size
+ * bytes, contents on entry irrelevant) holds the two buffer sets.  The call
+ * returns once everything is enqueued; `stream2` first waits for the work
+ * enqueued on `stream` before the call, and `stream` waits for `stream2`'s
+ * part at the end, so the whole call is ordered on `stream` like a single
+ * operation: the host outputs are complete once `stream` reaches that point
+ * (e.g. after cudaStreamSynchronize(stream)).  SSD_FLAG_CHECK_SEQ checks the
+ * host seq_idx directly, before anything is enqueued.  SSD_ERR_INVALID_ARG
+ * for sizes ssd_fwd rejects or a missing pointer, SSD_ERR_WORKSPACE if the
+ * workspace is missing or too small (nothing enqueued); otherwise ssd_fwd's
+ * verdict on the first piece, in which case the first piece's copies in may
+ * have been enqueued, or SSD_ERR_CUDA if a copy, an event or a launch failed.
+ * Outputs are undefined after any error. */
+SSD_API size_t ssd_fwd_host_workspace_size(const ssd_fwd_args* args, int64_t rows_per_piece);
+SSD_API ssd_status ssd_fwd_host(const ssd_fwd_args* args, int64_t rows_per_piece, void* device_workspace,
+                                size_t device_workspace_bytes, void* stream, void* stream2);
+
 /* Number of kernels ssd_fwd enqueues for these arguments (memsets excluded),
  * or 0 if the sizes are invalid. */
 SSD_API int ssd_fwd_launch_count(const ssd_fwd_args* args);

@@ -22,7 +22,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["fwd", "bwd", "BwdArgs", "bwd_workspace_size", "bwd_chunk_size", "bwd_path", "ssd_chunked", "make_args",
+__all__ = ["fwd", "fwd_host", "bwd", "BwdArgs", "bwd_workspace_size", "bwd_chunk_size", "bwd_path", "ssd_chunked", "make_args",
            "make_bwd_args", "main_kernel", "device_status",
            "conv1d_silu_bwd", "ConvBwdArgs", "causal_conv1d_silu", "step", "StepArgs", "total_decay", "state_fold", "conv1d_silu", "ConvArgs", "workspace_size", "launch_count", "kernel_path", "SSDError", "lib", "LIB_PATH", "Args",
            "SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED", "SSD_ERR_WORKSPACE", "SSD_ERR_CUDA",
@@ -114,6 +114,11 @@ def _load() -> ctypes.CDLL:
     L.ssd_fwd.restype = ctypes.c_int
     L.ssd_fwd_workspace_size.argtypes = [ctypes.POINTER(Args)]
     L.ssd_fwd_workspace_size.restype = ctypes.c_size_t
+    L.ssd_fwd_host_workspace_size.argtypes = [ctypes.POINTER(Args), ctypes.c_int64]
+    L.ssd_fwd_host_workspace_size.restype = ctypes.c_size_t
+    L.ssd_fwd_host.argtypes = [ctypes.POINTER(Args), ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t,
+                               ctypes.c_void_p, ctypes.c_void_p]
+    L.ssd_fwd_host.restype = ctypes.c_int
     L.ssd_fwd_launch_count.argtypes = [ctypes.POINTER(Args)]
     L.ssd_fwd_launch_count.restype = ctypes.c_int
     L.ssd_fwd_device_status.argtypes = [ctypes.POINTER(Args), ctypes.c_void_p]
@@ -326,6 +331,97 @@ def fwd(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: 
         if st != SSD_OK:
             raise SSDError(st)
     return y, final_states
+
+
+_second_streams = {}
+
+
+def fwd_host(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+             D: Optional[torch.Tensor] = None, chunk_size: int = 64,
+             initial_states: Optional[torch.Tensor] = None, seq_idx: Optional[torch.Tensor] = None,
+             num_seqs: Optional[int] = None, return_final_states: bool = True,
+             y: Optional[torch.Tensor] = None, final_states: Optional[torch.Tensor] = None,
+             z: Optional[torch.Tensor] = None, rows_per_piece: int = 0, workspace: Optional[torch.Tensor] = None,
+             device=None, stream2=None, check_seq: bool = False, flags: int = 0):
+    """SSD forward from and to HOST tensors via ``ssd_fwd_host``.  Inputs as
+    for ``fwd`` but CPU tensors (pinned, for the copies to overlap); y and
+    final_states come back as CPU tensors (pinned when allocated here).  The
+    batch runs in pieces of ``rows_per_piece`` rows (0: the library chooses)
+    alternating between the current stream of ``device`` and ``stream2`` (a
+    torch.cuda.Stream; one per device is kept here if None), so that a
+    piece's copies in overlap the previous piece's compute and copies out.
+    ``workspace``: a uint8 CUDA tensor of at least the size the library asks
+    for, or None.  ``flags``: further SSD_FLAG_* bits (SSD_FLAG_GENERIC).
+    Asynchronous on the current stream like ``fwd``: synchronize it before
+    reading y."""
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    if x.dim() != 4 or B.dim() != 4 or C.dim() != 4 or dt.dim() != 3 or A.dim() != 1:
+        raise ValueError("expected x (b,L,H,P), dt (b,L,H), A (H), B and C (b,L,G,N)")
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    for name, t in (("x", x), ("dt", dt), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+                    ("initial_states", initial_states), ("seq_idx", seq_idx)):
+        if t is not None and (t.device.type != "cpu" or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CPU tensor")
+    if tuple(B.shape) != (b, L, G, N) or tuple(C.shape) != (b, L, G, N) or B.dtype != x.dtype or C.dtype != x.dtype:
+        raise ValueError("B and C must be (b, L, G, N) in x's dtype")
+    if tuple(dt.shape) != (b, L, H) or tuple(A.shape) != (H,) or dt.dtype != torch.float32 or A.dtype != torch.float32:
+        raise ValueError("dt must be float32 (b, L, H) and A float32 (H,)")
+    if D is not None and (D.dtype != torch.float32 or tuple(D.shape) != (H,)):
+        raise ValueError("D must be float32 (H,)")
+    if z is not None and (z.dtype != x.dtype or tuple(z.shape) != tuple(x.shape)):
+        raise ValueError("z must be like x")
+    if initial_states is not None and (initial_states.dtype != torch.float32
+                                       or tuple(initial_states.shape) != (b, H, P, N)):
+        raise ValueError("initial_states must be float32 (b, H, P, N)")
+    if seq_idx is not None and (seq_idx.dtype != torch.int32 or tuple(seq_idx.shape) != (b, L)):
+        raise ValueError("seq_idx must be int32 (b, L)")
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if seq_idx is not None and num_seqs is None:
+        num_seqs = int(seq_idx.max().item()) + 1
+    if y is None:
+        y = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    if return_final_states and final_states is None:
+        rows = num_seqs if seq_idx is not None else b
+        final_states = torch.empty(rows, H, P, N, dtype=torch.float32, pin_memory=True)
+    if not return_final_states:
+        final_states = None
+    a = make_args(x, dt, A, B, C, D, chunk_size, initial_states, seq_idx, num_seqs, y, final_states, z=z)
+    if check_seq:
+        a.flags |= SSD_FLAG_CHECK_SEQ
+    a.flags |= int(flags)
+    need = int(lib.ssd_fwd_host_workspace_size(ctypes.byref(a), int(rows_per_piece)))
+    if need == 0:
+        raise SSDError(SSD_ERR_INVALID_ARG)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if stream2 is None:
+        stream2 = _second_streams.get(dev.index)
+        if stream2 is None:
+            stream2 = _second_streams[dev.index] = torch.cuda.Stream(dev)
+    st = lib.ssd_fwd_host(ctypes.byref(a), int(rows_per_piece), ctypes.c_void_p(workspace.data_ptr()),
+                          workspace.numel() * workspace.element_size(),
+                          ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream),
+                          ctypes.c_void_p(stream2.cuda_stream))
+    if st != SSD_OK:
+        raise SSDError(st)
+    return y, final_states
+
+
+def fwd_host_workspace_size(x, B, chunk_size: int = 64, rows_per_piece: int = 0, seq_idx=None, num_seqs=None,
+                            final_states: bool = True, has_D: bool = True, z: bool = False,
+                            initial_states: bool = False, flags: int = 0) -> int:
+    """Device workspace bytes ``fwd_host`` needs for these shapes (tensors
+    only supply shapes and dtype)."""
+    a = make_args(x, None, None, B, None, chunk_size=chunk_size, seq_idx=seq_idx, num_seqs=num_seqs)
+    a.flags |= int(flags)
+    flag_ptr = 1 << 8  # presence only; the size query does not dereference
+    a.final_states = flag_ptr if final_states else None
+    a.D = flag_ptr if has_D else None
+    a.z = flag_ptr if z else None
+    a.initial_states = flag_ptr if initial_states else None
+    return int(lib.ssd_fwd_host_workspace_size(ctypes.byref(a), int(rows_per_piece)))
 
 
 def step(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,

@@ -415,3 +415,35 @@ def test_conv_bwd_workspace_size():
 ])
 def test_bwd_dinitial_only_rejections(kw, status):
     assert ssd.lib.ssd_bwd(ctypes.byref(_bwd_args(**kw)), None) == status
+
+
+def _host_call(a, rows=0, ws=None, nbytes=0):
+    return ssd.lib.ssd_fwd_host(ctypes.byref(a), rows, ws, nbytes, None, None)
+
+
+def test_host_workspace_size_by_pieces():
+    """ssd_fwd_host's device workspace for one-row and whole-batch pieces, the
+    library's default piece size, and 0 for invalid sizes."""
+    a = base_args(batch=8)
+    one = ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 8)
+    per_row = ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 1)
+    assert one > 0 and per_row > 0
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 0) == per_row  # b >= 8: b / 8 rows a piece
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 99) == one      # capped at the batch
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), -1) == 0
+    a.seq_idx, a.num_seqs = 1 << 20, 5
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 1) > one  # one piece with sequence ids
+    a.chunk_size = 48
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 1) == 0
+    assert ssd.lib.ssd_fwd_host_workspace_size(None, 1) == 0
+
+
+def test_host_call_checked_before_anything_is_enqueued():
+    a = base_args(batch=4)
+    need = ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 1)
+    assert _host_call(a, 1) == ssd.SSD_ERR_WORKSPACE                     # none given
+    assert _host_call(a, 1, 1 << 24, need - 1) == ssd.SSD_ERR_WORKSPACE  # one byte short
+    assert _host_call(a, 1, (1 << 24) + 16, need) == ssd.SSD_ERR_INVALID_ARG  # not 256-byte aligned
+    assert _host_call(base_args(batch=4, x=None), 1, 1 << 24, need) == ssd.SSD_ERR_INVALID_ARG
+    assert _host_call(base_args(batch=4, chunk_size=48), 1, 1 << 24, need) == ssd.SSD_ERR_INVALID_ARG
+    assert ssd.lib.ssd_fwd_host(None, 1, None, 0, None, None) == ssd.SSD_ERR_INVALID_ARG
