@@ -818,7 +818,9 @@ def run_bwd(args, dist, dev, world, rank):
                      "kernel": "k_bwd_chunk_tc (tcgen05)", "kernel_ms": kernel_ms,
                      "kernel_ms_p10_p50_p90": [per[int(0.1 * (K - 1))], per[int(0.5 * (K - 1))],
                                                per[int(0.9 * (K - 1))]],
-                     "traffic": None, "algorithmic_bytes": by_chunk, "algorithmic_flops": f_chunk,
+                     "traffic": traffic_from_profiles("ssd_bwd_tc.cuh", "k_bwd_chunk_tc", "c1_bwd")
+                     if (b, H) == (8, 80) else None,
+                     "algorithmic_bytes": by_chunk, "algorithmic_flops": f_chunk,
                      "tflops": f_chunk / (kernel_ms / 1e3) / 1e12, "states_kernel_flops": f_states,
                      "cb_flops_in_kernel": f_cb},
         "e2e": {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
