@@ -849,6 +849,7 @@ def main():
     ap.add_argument("--config", default="c1", choices=sorted(si.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--generic", action="store_true", help="force the generic CUDA-core kernels")
+    ap.add_argument("--gated", action="store_true", help="the forward with the gate z (y * SiLU(z)), z ~ N(0,1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--op", default="fwd", choices=["fwd", "step", "conv", "bwd", "conv_bwd"],
@@ -890,6 +891,9 @@ def main():
         return run_conv_bwd(args, dist, dev, world, rank)
 
     host = si.make_inputs(shape, seed=shape.seed + rank)
+    if args.gated:  # the gate, like x
+        zg = torch.Generator().manual_seed(shape.seed + 7919 + rank)
+        host["z"] = torch.randn(host["x"].shape, generator=zg).to(host["x"].dtype)
     num_seqs = host.get("num_seqs")
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
     b, L, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
@@ -900,11 +904,11 @@ def main():
                                   generic=args.generic)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     launches_per_call = ssd.launch_count(g["x"], g["B"], shape.chunk_size, g.get("seq_idx"), num_seqs, True,
-                                         generic=args.generic)
+                                         generic=args.generic, z=g.get("z"))
     path = ssd.kernel_path(g["x"], g["B"], shape.chunk_size, generic=args.generic, seq_idx=g.get("seq_idx"),
                            num_seqs=num_seqs)
     main_kernel = ssd.main_kernel(g["x"], g["dt"], g["B"], shape.chunk_size, generic=args.generic,
-                                  seq_idx=g.get("seq_idx"), num_seqs=num_seqs)
+                                  seq_idx=g.get("seq_idx"), num_seqs=num_seqs, z=g.get("z"))
 
     K = args.steps
     # the fused kernel's own duration is timed in a separate loop: events
@@ -915,7 +919,7 @@ def main():
     def step(events=None):
         ssd.fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk_size=shape.chunk_size,
                 initial_states=g["initial_states"], seq_idx=g.get("seq_idx"), num_seqs=num_seqs,
-                y=y, final_states=final, workspace=ws, generic=args.generic, timing_events=events)
+                y=y, final_states=final, workspace=ws, generic=args.generic, timing_events=events, z=g.get("z"))
 
     for _ in range(args.warmup):
         step()
@@ -953,7 +957,7 @@ def main():
     # pinned host inputs, copies them in by row pieces on two streams, runs the
     # forward on each piece and copies y and the final states back, one piece's
     # copies in overlapping the previous piece's compute and copies out
-    names = [k for k in ("x", "dt", "A", "B", "C", "D", "initial_states", "seq_idx") if host.get(k) is not None]
+    names = [k for k in ("x", "dt", "A", "B", "C", "D", "initial_states", "seq_idx", "z") if host.get(k) is not None]
     pinned = {k: host[k].pin_memory() for k in names}
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     f_host = torch.empty(final.shape, dtype=final.dtype).pin_memory()
@@ -962,13 +966,14 @@ def main():
     gen_flag = ssd.SSD_FLAG_GENERIC if args.generic else 0
     hws = torch.empty(max(1, ssd.fwd_host_workspace_size(
         host["x"], host["B"], shape.chunk_size, 0, host.get("seq_idx"), num_seqs, True, host.get("D") is not None,
-        False, host.get("initial_states") is not None, gen_flag)), dtype=torch.uint8, device=dev)
+        host.get("z") is not None, host.get("initial_states") is not None, gen_flag)), dtype=torch.uint8, device=dev)
     stream2 = torch.cuda.Stream(dev)
 
     def e2e_step():
         ssd.fwd_host(pinned["x"], pinned["dt"], pinned["A"], pinned["B"], pinned["C"], pinned.get("D"),
                      shape.chunk_size, pinned.get("initial_states"), pinned.get("seq_idx"), num_seqs,
-                     y=y_host, final_states=f_host, workspace=hws, device=dev, stream2=stream2, flags=gen_flag)
+                     y=y_host, final_states=f_host, workspace=hws, device=dev, stream2=stream2, flags=gen_flag,
+                     z=pinned.get("z"))
 
     for _ in range(3):
         e2e_step()
@@ -988,6 +993,8 @@ def main():
         dist.barrier()
 
     w = work(shape, num_seqs)
+    if args.gated and main_kernel != "k_ssd_fwd_pair":  # the single-head kernel reads z in its epilogue
+        w["bytes"] += host["z"].numel() * host["z"].element_size()
     peaks = load_peaks()
     ms_step = ms / K
     tokens_job = shape.tokens * world
@@ -1017,7 +1024,11 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if shape.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": describe(shape), "batch": b, "seqlen": L, "nheads": H, "headdim": P,
+        "config": {"workload": describe(shape) + ((", gated: y * SiLU(z), z ~ N(0,1)" + (
+                       "; the gate in k_gate_silu after the two-head kernel (the roofline is the two-head"
+                       " kernel's)" if main_kernel == "k_ssd_fwd_pair" else "; the gate in the fused epilogue"))
+                   if args.gated else ""),
+                   "batch": b, "seqlen": L, "nheads": H, "headdim": P,
                    "dstate": N, "ngroups": shape.ngroups, "chunk_size": shape.chunk_size,
                    "l2": f"no flush: inputs+outputs {w['bytes'] / 1e6:.0f} MB per step > 126 MB L2",
                    "parallelism": "replicas" if world > 1 else "single GPU"},

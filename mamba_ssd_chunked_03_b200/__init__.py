@@ -242,10 +242,10 @@ def device_status(x, B, chunk_size: int, workspace: torch.Tensor, generic: bool 
 
 
 def launch_count(x, B, chunk_size: int, seq_idx=None, num_seqs=None, final_states: bool = True,
-                 generic: bool = False) -> int:
-    """Kernels one ``fwd`` call enqueues for these shapes."""
+                 generic: bool = False, z=None) -> int:
+    """Kernels one ``fwd`` call enqueues for these shapes (``z``: the gate, if any)."""
     a = make_args(x, None, None, B, None, chunk_size=chunk_size, seq_idx=seq_idx, num_seqs=num_seqs,
-                  generic=generic)
+                  generic=generic, z=z)
     if final_states:
         a.final_states = 1 << 8  # presence only; the query does not dereference
     return int(lib.ssd_fwd_launch_count(ctypes.byref(a)))
@@ -257,11 +257,11 @@ def kernel_path(x, B, chunk_size: int, generic: bool = False, seq_idx=None, num_
     return lib.ssd_fwd_path(ctypes.byref(a)).decode()
 
 
-def main_kernel(x, dt, B, chunk_size: int, generic: bool = False, seq_idx=None, num_seqs=None) -> str:
+def main_kernel(x, dt, B, chunk_size: int, generic: bool = False, seq_idx=None, num_seqs=None, z=None) -> str:
     """Name of the fused kernel a call with these tensors is dominated by
-    (the one ``timing_events`` bracket)."""
+    (the one ``timing_events`` bracket; ``z``: the gate, if any)."""
     a = make_args(x, dt, None, B, None, chunk_size=chunk_size, seq_idx=seq_idx, num_seqs=num_seqs,
-                  generic=generic)
+                  generic=generic, z=z)
     return lib.ssd_fwd_main_kernel(ctypes.byref(a)).decode()
 
 

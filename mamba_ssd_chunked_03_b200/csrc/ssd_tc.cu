@@ -780,7 +780,10 @@ size_t tc_workspace_bytes(const Problem& p) { return tc_workspace_need(tc_tiles(
 int tc_launch_count(const Problem& p) {
   if (p.seq) return 4;  // run list, C B^T per run chunk, fused per (run, head), exact
   const Problem t = tc_tiles(p);
-  return tc_kernel_n(t) == 128 && !t.z && tc_pair_supported(t) && tc_pair_split(t) ? 4 : 3;
+  // C B^T, the fused kernel, the exact kernel; the two-head kernel's
+  // state-only pass when it splits, and its gate pass for a gated call
+  if (tc_kernel_n(t) == 128 && tc_pair_supported(t)) return 3 + (tc_pair_split(t) ? 1 : 0) + (t.z ? 1 : 0);
+  return 3;
 }
 
 cudaError_t tc_forward(const Problem& pq, void* ws, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {

@@ -824,9 +824,33 @@ __global__ void __launch_bounds__(320, FastCfg<NS>::kMinBlocks)
   if (warp == 0) tmem_dealloc(tmem, K::kTmemCols);
 }
 
+// The gate for the two-head kernel, whose epilogue leaves it out: y <- y *
+// SiLU(z) in place, 8 bf16 a thread per 16-byte vector (n8 vectors), SiLU as
+// the single-head epilogue forms it.  y is rounded to bf16 before the gate
+// here, once more after it.
+__global__ void __launch_bounds__(256) k_gate_silu(__nv_bfloat16* y, const __nv_bfloat16* z, int64_t n8) {
+  uint4* yv = reinterpret_cast<uint4*>(y);
+  const uint4* zv = reinterpret_cast<const uint4*>(z);
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n8; i += (int64_t)gridDim.x * 256) {
+    const uint4 a = yv[i], g = __ldcs(zv + i);
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float y0, y1, z0, z1;
+      unpack_bf16x2(aw[j], y0, y1);
+      unpack_bf16x2(gw[j], z0, z1);
+      o[j] = pack_bf16x2(y0 * silu(z0), y1 * silu(z1));
+    }
+    __stcs(yv + i, make_uint4(o[0], o[1], o[2], o[3]));
+  }
+}
+
 // ev0 / ev1 (optional) are recorded right before and after the fused kernel.
 // Packed sequences (seq_idx): the run list first, then W' per run chunk and
-// the single-head kernel per (run, head).
+// the single-head kernel per (run, head).  A gated call on the two-head
+// kernel adds k_gate_silu after it (the exact kernel, which may follow,
+// applies the gate itself to the units it redoes).
 template <int NS>
 cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1) {
   const bool varlen = p.seq != nullptr;
@@ -888,14 +912,21 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
   fa.runs = w.runs;
   fa.unit_bad = w.unit_bad;
   fa.stall = p.stall ? 1 : 0;
-  // (a gated call takes the single-head kernel, whose epilogue applies the gate)
-  if (!varlen && !p.z && NS == 128 && tc_pair_supported(p)) {
+  if (!varlen && NS == 128 && tc_pair_supported(p)) {
     CUtensorMap ty, tdt;
     if (!make_map_3d(&ty, p.y, p.H * p.P, p.L, p.b) || !make_map_dt(&tdt, p.dt, p.H, p.L, p.b))
       return cudaErrorInvalidValue;
     if (ev0 && (e = cudaEventRecord(ev0, st)) != cudaSuccess) return e;
     if ((e = tc_pair_launch(p, w, tx, tb, tc_, tw, ty, tdt, fa, st)) != cudaSuccess) return e;
-    return ev1 ? cudaEventRecord(ev1, st) : cudaSuccess;
+    if (ev1 && (e = cudaEventRecord(ev1, st)) != cudaSuccess) return e;
+    if (p.z) {
+      const int64_t n8 = p.b * p.L * p.H * p.P / 8;  // P = 64
+      const int64_t blocks = (n8 + 255) / 256;
+      k_gate_silu<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, st>>>(
+          static_cast<__nv_bfloat16*>(p.y), static_cast<const __nv_bfloat16*>(p.z), n8);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
   }
   e = cudaFuncSetAttribute(k_ssd_fwd_fast<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)FastCfg<NS>::kSmemBytes);
@@ -912,7 +943,7 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
 
 const char* tc_main_kernel(const Problem& p) {
   if (p.seq) return "k_ssd_fwd_fast";  // per (run, head)
-  return tc_kernel_n(p) == 128 && !p.z && tc_pair_supported(tc_tiles(p)) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
+  return tc_kernel_n(p) == 128 && tc_pair_supported(tc_tiles(p)) ? "k_ssd_fwd_pair" : "k_ssd_fwd_fast";
 }
 
 cudaError_t tc_fast_forward(const Problem& p, const TcWorkspace& w, cudaStream_t st, cudaEvent_t ev0,

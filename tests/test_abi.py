@@ -235,16 +235,21 @@ def test_packed_dispatch_queries():
 
 
 def test_gated_dispatch_queries():
-    """A gated call leaves the two-head kernel; an unaligned gate leaves the
-    tensor-core path (its epilogues read z in 16-byte vectors)."""
-    a = base_args(nheads=8, ngroups=1)
-    two_head = ssd.lib.ssd_fwd_main_kernel(ctypes.byref(a))
-    a.z = 1 << 22
-    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"tcgen05"
-    assert ssd.lib.ssd_fwd_main_kernel(ctypes.byref(a)) == b"k_ssd_fwd_fast"
-    assert two_head in (b"k_ssd_fwd_pair", b"k_ssd_fwd_fast")  # the pair kernel also needs dt 16-byte aligned
-    a.z = (1 << 22) + 8
-    assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"generic"
+    """A gated call keeps the ungated call's fused kernel: the two-head kernel
+    takes the gate in a pass of its own (one more launch), the single-head
+    kernel in its epilogue.  An unaligned gate leaves the tensor-core path
+    (z is read in 16-byte vectors)."""
+    for dt in (1 << 20, (1 << 20) + 4):  # the pair kernel also needs dt 16-byte aligned
+        a = base_args(nheads=8, ngroups=1, dt=dt)
+        fused = ssd.lib.ssd_fwd_main_kernel(ctypes.byref(a))
+        n0 = ssd.lib.ssd_fwd_launch_count(ctypes.byref(a))
+        a.z = 1 << 22
+        assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"tcgen05"
+        assert ssd.lib.ssd_fwd_main_kernel(ctypes.byref(a)) == fused
+        assert ssd.lib.ssd_fwd_launch_count(ctypes.byref(a)) == n0 + (1 if fused == b"k_ssd_fwd_pair" else 0)
+        a.z = (1 << 22) + 8
+        assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"generic"
+    assert fused == b"k_ssd_fwd_fast"  # dt not 16-byte aligned
 
 
 def test_workspace_grows_with_packed_sequences():

@@ -51,7 +51,7 @@ def test_conv1d_silu_strip_edges():
 
 GATE_CASES = [
     # name, b, L, H, N, G, dtype, generic, packed, steep
-    ("two_head_shape_takes_single_head", 2, 300, 8, 128, 1, "bf16", False, None, False),
+    ("two_head_shape_gate_pass", 2, 300, 8, 128, 1, "bf16", False, None, False),
     ("single_head_N256", 1, 200, 4, 256, 2, "bf16", False, None, False),
     ("packed_per_sequence", 1, 260, 4, 128, 2, "bf16", False, [[100, 60, 100]], False),
     ("exact_kernel", 2, 300, 4, 128, 2, "bf16", False, None, True),
@@ -74,8 +74,10 @@ def test_gate_is_applied_where_y_is_formed(case):
     gen = torch.Generator().manual_seed(77)
     z = torch.randn(b, L, H, 64, generator=gen).to(d["x"].dtype)
     g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
-    if name == "two_head_shape_takes_single_head":
-        assert ssd.main_kernel(g["x"], g["dt"], g["B"], 64) == "k_ssd_fwd_pair"  # without the gate
+    if name == "two_head_shape_gate_pass":  # the two-head kernel, then the gate pass over y
+        assert ssd.main_kernel(g["x"], g["dt"], g["B"], 64) == "k_ssd_fwd_pair"
+        assert ssd.main_kernel(g["x"], g["dt"], g["B"], 64, z=g["x"]) == "k_ssd_fwd_pair"
+        assert ssd.launch_count(g["x"], g["B"], 64, z=g["x"]) == ssd.launch_count(g["x"], g["B"], 64) + 1
     y, f = ssd.fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk_size=64,
                    initial_states=g["initial_states"], seq_idx=g.get("seq_idx"), num_seqs=d.get("num_seqs"),
                    generic=generic, z=z.cuda())

@@ -6,9 +6,10 @@ piece's compute and copies out) against ``ssd_fwd`` on device buffers, which
 A piece is a forward over fewer rows, which can change how the tensor-core
 path splits the state passing among CTAs.  There the chunk states are formed
 from bf16 operands, so a different split rounds the states, and through them
-y, differently.  The comparison is therefore not bitwise: 1e-5 (relative L2)
-on the fp32 path, 1e-3 on the bf16 one, both well inside the oracle
-tolerances (1e-5 and 1e-2).  Only the
+y, differently; a gated y on the two-head kernel is rounded to bf16 twice
+(before and after the gate pass).  The comparison is therefore not bitwise:
+1e-5 (relative L2) on the fp32 path, 2e-3 on the bf16 one, both well inside
+the oracle tolerances (1e-5 and 1e-2).  Only the
 current stream is synchronised before the host outputs are read: the call
 must order its second stream's part before it."""
 import pytest
@@ -50,7 +51,7 @@ def test_host_entry_matches_the_device_call(name, shape, rows_list, gated):
     y_ref, f_ref = y_ref.cpu(), f_ref.cpu()
     host = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     zh = None if z is None else z.pin_memory()
-    tol = 1e-3 if shape.dtype == "bf16" else 1e-5
+    tol = 2e-3 if shape.dtype == "bf16" else 1e-5
     for rows in rows_list:
         y, f = ssd.fwd_host(host["x"], host["dt"], host["A"], host["B"], host["C"], host["D"], shape.chunk_size,
                             host["initial_states"], host.get("seq_idx"), ns, z=zh, rows_per_piece=rows)
