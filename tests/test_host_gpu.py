@@ -80,3 +80,21 @@ def test_host_entry_reuses_caller_buffers_and_workspace():
         outs.append((y.clone(), f.clone()))
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[1][0], outs[2][0])
     assert torch.equal(outs[0][1], outs[2][1])
+
+
+def test_host_entry_with_pageable_memory():
+    """Host tensors that are not page-locked: the copies are then staged by the
+    driver and do not overlap, but the results are those of pinned buffers."""
+    shape = si.SSDShape("host_pageable", 3, 200, 8, 64, 128, 1, 64, "bf16", h0_std=0.1, seed=11)
+    d = si.make_inputs(shape)
+    pinned = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    y_p, f_p = ssd.fwd_host(pinned["x"], pinned["dt"], pinned["A"], pinned["B"], pinned["C"], pinned["D"], 64,
+                            pinned["initial_states"], rows_per_piece=1)
+    torch.cuda.current_stream().synchronize()
+    y_out = torch.empty(d["x"].shape, dtype=d["x"].dtype)  # pageable outputs too
+    f_out = torch.empty(3, 8, 64, 128, dtype=torch.float32)
+    y, f = ssd.fwd_host(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], 64, d["initial_states"],
+                        y=y_out, final_states=f_out, rows_per_piece=1)
+    torch.cuda.current_stream().synchronize()
+    assert not y.is_pinned()
+    assert torch.equal(y, y_p) and torch.equal(f, f_p)
