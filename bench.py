@@ -740,9 +740,14 @@ def run_bwd(args, dist, dev, world, rank):
     b, L, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
     host = bwd_inputs(shape, rank)
     names = ("x", "dt", "B", "C", "dy")
+    if args.gated:  # the gate, like x: dy is then the gradient of y * SiLU(z)
+        zg = torch.Generator().manual_seed(7919 + rank)
+        host["z"] = torch.randn(host["x"].shape, generator=zg).to(host["x"].dtype)
+        names = names + ("z",)
     g = {k: host[k].to(dev) for k in names}
     A, D = host["A"].to(dev), host["D"].to(dev)
-    ws = torch.empty(ssd.bwd_workspace_size(g["x"], g["B"]), dtype=torch.uint8, device=dev)
+    ws = torch.empty(ssd.bwd_workspace_size(g["x"], g["B"], z=g.get("z")), dtype=torch.uint8, device=dev)
+    bpath = ssd.bwd_path(g["x"], g["dy"], g["B"], g["C"], z=g.get("z"))
     Q = ssd.bwd_chunk_size(g["x"], g["B"])  # the library's own choice
     K = args.steps
     events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -752,7 +757,8 @@ def run_bwd(args, dist, dev, world, rank):
     out = {}
 
     def step(ev=None):
-        out.update(ssd.bwd(g["x"], g["dt"], A, g["B"], g["C"], D, g["dy"], workspace=ws, timing_events=ev))
+        out.update(ssd.bwd(g["x"], g["dt"], A, g["B"], g["C"], D, g["dy"], workspace=ws, timing_events=ev,
+                           z=g.get("z")))
 
     for _ in range(args.warmup):
         step()
@@ -808,24 +814,27 @@ def run_bwd(args, dist, dev, world, rank):
         "metric": "SSD bwd tokens/s", "value": tokens * world / (ms_step / 1e3), "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": BWD_WORKLOAD if (b, H) == (8, 80) else
-                   BWD_WORKLOAD.replace("b8 ", f"b{b} ").replace("H80 ", f"H{H} "),
+        "config": {"workload": (BWD_WORKLOAD if (b, H) == (8, 80) else
+                                BWD_WORKLOAD.replace("b8 ", f"b{b} ").replace("H80 ", f"H{H} "))
+                   + (", gated: dy is the gradient of y * SiLU(z), z ~ N(0,1); dz too" if args.gated else ""),
+                   "path": bpath,
                    "l2": "no flush: inputs, gradients and the per-chunk states exceed the 126 MB L2"
                          if (b, H) == (8, 80) else "small case for profiling",
                    "parallelism": "replicas" if world > 1 else "single GPU", "bwd_chunk": Q},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
-                     "kernel": "k_bwd_chunk_tc (tcgen05)", "kernel_ms": kernel_ms,
+                     "kernel": "k_bwd_chunk_tc (tcgen05)" if bpath == "tcgen05" else "k_bwd_chunk (CUDA cores)",
+                     "kernel_ms": kernel_ms,
                      "kernel_ms_p10_p50_p90": [per[int(0.1 * (K - 1))], per[int(0.5 * (K - 1))],
                                                per[int(0.9 * (K - 1))]],
                      "traffic": traffic_from_profiles("ssd_bwd_tc.cuh", "k_bwd_chunk_tc", "c1_bwd")
-                     if (b, H) == (8, 80) else None,
+                     if (b, H) == (8, 80) and bpath == "tcgen05" else None,
                      "algorithmic_bytes": by_chunk, "algorithmic_flops": f_chunk,
                      "tflops": f_chunk / (kernel_ms / 1e3) / 1e12, "states_kernel_flops": f_states,
                      "cb_flops_in_kernel": f_cb},
         "e2e": {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": E},
-        "gpu_launches": (4 if ssd.bwd_path(g["x"], g["dy"], g["B"], g["C"]) == "tcgen05" else 6) * K,
+        "gpu_launches": (4 if bpath == "tcgen05" else 6) * K,
         "clocks": clock_stats,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

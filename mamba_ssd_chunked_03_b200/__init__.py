@@ -544,9 +544,11 @@ def make_bwd_args(x, dt, A, B, C, D=None, dy=None, initial_states=None, seq_idx=
     return a
 
 
-def bwd_workspace_size(x, B, chunk_size: int = 0) -> int:
-    """Workspace bytes ``ssd_bwd`` needs for these shapes (0: not supported)."""
+def bwd_workspace_size(x, B, chunk_size: int = 0, z=None) -> int:
+    """Workspace bytes ``ssd_bwd`` needs for these shapes (0: not supported);
+    ``z``: the gate, if the call has one."""
     a = make_bwd_args(x, None, None, B, None, chunk_size=chunk_size)
+    a.z = _ptr(z)
     return int(lib.ssd_bwd_workspace_size(ctypes.byref(a)))
 
 
