@@ -218,9 +218,10 @@ SSD_API const char* ssd_fwd_path(const ssd_fwd_args* args);
 
 /* Name of the fused kernel that dominates the call on the tensor-core path
  * ("k_ssd_fwd_pair": two heads per CTA, N = 128, an even number of heads per
- * group, H a multiple of 4 and dt 16-byte aligned; "k_ssd_fwd_fast": one head
- * per CTA otherwise), "generic" on the generic path, or "invalid".  It is the
- * kernel that timing_events bracket.  Static string; no device work. */
+ * group, H a multiple of 4 and dt 16-byte aligned, with a gate z applied to y
+ * by a pass of its own after it; "k_ssd_fwd_fast": one head per CTA otherwise,
+ * the gate in its epilogue), "generic" on the generic path, or "invalid".  It
+ * is the kernel that timing_events bracket.  Static string; no device work. */
 SSD_API const char* ssd_fwd_main_kernel(const ssd_fwd_args* args);
 
 /* After an ssd_fwd call with these arguments: waits for `stream`, then reads
