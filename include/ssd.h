@@ -127,9 +127,11 @@ typedef struct {
                                      the caller; both or neither.                    */
   const void* z;                  /* (b,L,H,P) dtype gate, or NULL: y is returned as
                                      y * SiLU(z) (SiLU(v) = v / (1 + e^-v)), the
-                                     Mamba-2 block's gate path multiplied in where y
-                                     is formed ("SSM 家族全景图（下）：Mamba-2 与
-                                     Jamba", section 5).                             */
+                                     Mamba-2 block's gate path ("SSM 家族全景图（下）：
+                                     Mamba-2 与 Jamba", section 5), multiplied in
+                                     where y is formed; on the two-head kernel by a
+                                     pass over y right after it (y then rounded to
+                                     the output type twice).                        */
 } ssd_fwd_args;
 
 /* Bytes of device workspace ssd_fwd needs for these sizes and options (only
