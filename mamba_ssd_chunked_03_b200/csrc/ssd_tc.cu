@@ -778,7 +778,8 @@ bool tc_supported(const Problem& p, uint32_t flags) {
 size_t tc_workspace_bytes(const Problem& p) { return tc_workspace_need(tc_tiles(p)); }
 
 int tc_launch_count(const Problem& p) {
-  if (p.seq) return 4;  // run list, C B^T per run chunk, fused per (run, head), exact
+  // run list, (final states of absent ids,) C B^T per run chunk, fused per (run, head), exact
+  if (p.seq) return p.final_states ? 5 : 4;
   const Problem t = tc_tiles(p);
   // C B^T, the fused kernel, the exact kernel; the two-head kernel's
   // state-only pass when it splits, and its gate pass for a gated call
@@ -791,11 +792,8 @@ cudaError_t tc_forward(const Problem& pq, void* ws, cudaStream_t st, cudaEvent_t
   const TcWorkspace w = tc_carve(p, ws);
   cudaError_t e = cudaMemsetAsync(w.err, 0, w.zero_bytes, st);
   if (e != cudaSuccess) return e;
-  // packed sequences: ids that never occur keep zero final states
-  if (p.seq && p.final_states &&
-      (e = cudaMemsetAsync(p.final_states, 0, sizeof(float) * (size_t)(p.num_seqs * p.H * p.P * p.N), st)) !=
-          cudaSuccess)
-    return e;
+  // (packed sequences: the final states of ids that never occur are zeroed
+  // after the run list, by k_zero_absent)
   if ((e = tc_fast_forward(p, w, st, ev0, ev1)) != cudaSuccess) return e;
   return tc_kernel_n(p) == 128 ? launch<128>(p, w, st) : launch<256>(p, w, st);
 }

@@ -6,6 +6,7 @@
 // k_seq_runs (packed sequences only): lists each sequence as a run (row,
 //   first token, length, id), so that every sequence is chunked from its own
 //   first token and the two kernels below take it as an independent problem.
+//   k_zero_absent then zeroes the final states of ids that no run carries.
 //
 // k_chunk_cb (one CTA per chunk -- of a batch row, or of a run -- and B/C group): the head-independent
 //   part of the intra-chunk "attention",
@@ -213,6 +214,32 @@ __global__ void __launch_bounds__(1024) k_seq_runs(const SeqRunArgs a) {
       for (int64_t r = tid; r < nr; r += 1024) a.runs.order[r] = (int)r;
     }
     if (tid == 0) *a.runs.count = (int)nr;
+  }
+}
+
+// ============================================================== k_zero_absent
+// The final state of an id that no run carries (an id in [0, num_seqs) that
+// never occurs in seq_idx) is zero; the fused kernel writes every run's.  A
+// usable list with num_seqs runs carries every id, and the kernel exits after
+// one load.  With an unusable list (count 0) every id is zeroed here, and the
+// exact kernel, later on the same stream, writes the ids that occur.
+constexpr int kZeroSlices = 16;  // blocks' shares of one id's H x P x N floats
+
+__global__ void __launch_bounds__(256) k_zero_absent(const RunList runs, float* final_states, int64_t num_seqs,
+                                                     int64_t per_id) {
+  const int nr = *runs.count;
+  if (nr == num_seqs) return;  // (uniform) every id has its run
+  for (int64_t item = blockIdx.x; item < num_seqs * kZeroSlices; item += gridDim.x) {
+    const int64_t id = item / kZeroSlices, sl = item % kZeroSlices;
+    int lo = 0, hi = nr;  // the runs' ids are strictly increasing: the first >= id
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (runs.id[mid] < id) lo = mid + 1; else hi = mid;
+    }
+    if (lo < nr && runs.id[lo] == id) continue;  // (uniform) written by the fused kernel
+    float* dst = final_states + id * per_id;
+    const int64_t a0 = per_id * sl / kZeroSlices, a1 = per_id * (sl + 1) / kZeroSlices;
+    for (int64_t i = a0 + threadIdx.x; i < a1; i += blockDim.x) dst[i] = 0.f;
   }
 }
 
@@ -872,6 +899,12 @@ cudaError_t launch_fast(const Problem& p, const TcWorkspace& w, cudaStream_t st,
     sa.failed_list = w.failed_list;
     k_seq_runs<<<1, 1024, 0, st>>>(sa);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (p.final_states) {
+      const int64_t items = p.num_seqs * kZeroSlices;
+      k_zero_absent<<<(unsigned)(items < 148 * 8 ? items : 148 * 8), 256, 0, st>>>(
+          w.runs, p.final_states, p.num_seqs, p.H * p.P * p.N);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
   }
   CbArgs ca{};
   ca.L = p.L;

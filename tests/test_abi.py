@@ -227,11 +227,14 @@ def test_conv_struct_layout_matches_the_compiled_header():
 
 def test_packed_dispatch_queries():
     """Packed sequences take the per-sequence fast path: run list, C B^T per
-    run chunk, the single-head kernel per (run, head), the exact kernel."""
+    run chunk, the single-head kernel per (run, head), the exact kernel; with
+    final states, the zeroing of ids that never occur after the run list."""
     a = base_args(seq_idx=1 << 21, num_seqs=8)
     assert ssd.lib.ssd_fwd_path(ctypes.byref(a)) == b"tcgen05"
     assert ssd.lib.ssd_fwd_main_kernel(ctypes.byref(a)) == b"k_ssd_fwd_fast"
     assert ssd.lib.ssd_fwd_launch_count(ctypes.byref(a)) == 4
+    a.final_states = 1 << 22
+    assert ssd.lib.ssd_fwd_launch_count(ctypes.byref(a)) == 5
 
 
 def test_gated_dispatch_queries():

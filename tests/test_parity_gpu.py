@@ -139,6 +139,29 @@ def test_packed_absent_ids_get_zero_states():
     assert state_err(f, fr) <= 1e-2
 
 
+@pytest.mark.parametrize("order", ["increasing", "out_of_order"])
+def test_packed_absent_ids_are_zeroed_in_a_dirty_buffer(order):
+    """Ids that never occur get zero final states written, whatever the caller's
+    buffer held (here NaN).  Increasing ids take the per-run kernels; ids out of
+    order leave the run list unusable and every unit to the exact kernel."""
+    shape = si.SSDShape("packed_dirty", 1, 200, 4, 64, 128, 1, 64, "bf16", h0_std=0.2, seed=41)
+    d = si.make_inputs(shape)
+    ids = [0] * 80 + [3] * 120 if order == "increasing" else [3] * 80 + [0] * 120
+    d["seq_idx"], d["num_seqs"] = torch.tensor([ids], dtype=torch.int32), 5
+    g = to_dev(d)
+    final = torch.full((5, 4, 64, 128), float("nan"), device="cuda")
+    y, f = ssd.fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk_size=64,
+                   initial_states=g["initial_states"], seq_idx=g["seq_idx"], num_seqs=5, final_states=final)
+    torch.cuda.synchronize()
+    assert f.data_ptr() == final.data_ptr()
+    yr, fr = run_oracle(d)
+    f = f.cpu().numpy().astype(np.float64)
+    assert rel_l2(y.float().cpu().numpy().astype(np.float64), yr) <= 1e-2
+    assert not np.isnan(f).any()
+    assert not f[[1, 2, 4]].any()
+    assert state_err(f, fr) <= 1e-2, state_err(f, fr)
+
+
 def test_determinism():
     s = si.SSDShape("det", 2, 700, 8, 64, 128, 2, 64, "bf16", h0_std=0.1, seed=77)
     d = si.make_inputs(s)
