@@ -438,12 +438,33 @@ def test_host_workspace_size_by_pieces():
     assert one > 0 and per_row > 0
     assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 0) == per_row  # b >= 8: b / 8 rows a piece
     assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 99) == one      # capped at the batch
-    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), -1) == 0
+    # token pieces (rows_per_piece < 0: that many tokens of every row)
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), -64) > 0
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), -100) == one  # one piece: the whole call
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), -1000) == one
     a.seq_idx, a.num_seqs = 1 << 20, 5
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), -64) == 0  # would split sequences
     assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 1) > one  # one piece with sequence ids
     a.chunk_size = 48
     assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 1) == 0
     assert ssd.lib.ssd_fwd_host_workspace_size(None, 1) == 0
+
+
+def test_host_default_pieces_for_a_small_batch():
+    """Under eight rows and without sequence ids the library cuts every row
+    into eight token pieces of whole 64-token chunks; rows too short for two
+    chunks stay one piece, and so does a call with sequence ids."""
+    a = base_args(batch=1, seqlen=2000)  # ceil(2000 / 8) = 250 -> 256 tokens a piece
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 0) == \
+        ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), -256)
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 0) != \
+        ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 1)  # two buffer sets, not one
+    short = base_args(batch=1, seqlen=100)
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(short), 0) == \
+        ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(short), 1)
+    a.seq_idx, a.num_seqs = 1 << 20, 3
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 0) == \
+        ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 1)
 
 
 def test_host_call_checked_before_anything_is_enqueued():
