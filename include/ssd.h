@@ -182,16 +182,24 @@ SSD_API ssd_status ssd_fwd_noalloc(const ssd_fwd_args* args, void* stream);
  * workspace and timing_events fields are ignored.  The pages describe no such
  * entry point; it has no counterpart there.
  *
- * The batch is taken in pieces of `rows_per_piece` rows (0: the library
- * chooses, about a quarter of the batch), alternately on `stream` and
- * `stream2`, each with its own set of device buffers.  For one piece the call
- * enqueues the copies of its rows' inputs in (one cudaMemcpyAsync per
- * tensor), ssd_fwd on them, and the copies of its y and final states out; so
- * a piece's copies in run while the previous piece computes and copies out
- * (on PCIe the two directions run at the same time).  With seq_idx the batch
- * is one piece: final_states is then indexed by sequence id, and a call on
- * part of the rows would clear the ids it does not see.  `stream2` may be
- * NULL: everything then runs on `stream`, in order.
+ * The work is taken in pieces, alternately on `stream` and `stream2`, each
+ * with its own set of device buffers.  rows_per_piece > 0: pieces of that
+ * many batch rows.  rows_per_piece < 0: pieces of -rows_per_piece tokens of
+ * every row, piece j starting from the state in which piece j - 1 ends (so
+ * y and the final states are those of one call), not with seq_idx.
+ * rows_per_piece = 0: the library chooses eight pieces: batch / 8 rows each
+ * for a batch of 8 or more, else (no seq_idx, rows of 128 tokens or more)
+ * whole 64-token chunks of every row, else one piece.  For one piece the call
+ * enqueues the copies of its inputs in (one cudaMemcpyAsync per tensor, or
+ * one cudaMemcpy2DAsync, a row each, for token pieces), ssd_fwd on them, and
+ * the copies of its y and final states out; so a piece's copies in run while
+ * the previous piece computes and copies out (on PCIe the two directions run
+ * at the same time).  Token pieces hand their state on through two fp32
+ * buffers in the workspace, so a piece's ssd_fwd also waits for the previous
+ * piece's.  With seq_idx the batch is one piece: final_states is then indexed
+ * by sequence id, and a call on part of the rows would clear the ids it does
+ * not see.  `stream2` may be NULL: everything then runs on `stream`, in
+ * order.
  *
  * `device_workspace` (256-byte aligned, at least ssd_fwd_host_workspace_size
  * bytes, contents on entry irrelevant) holds the two buffer sets.  The call
@@ -205,6 +213,9 @@ SSD_API ssd_status ssd_fwd_noalloc(const ssd_fwd_args* args, void* stream);
  * workspace is missing or too small (nothing enqueued); otherwise ssd_fwd's
  * verdict on the first piece, in which case the first piece's copies in may
  * have been enqueued, or SSD_ERR_CUDA if a copy, an event or a launch failed.
+ * SSD_ERR_INVALID_ARG too for token pieces with seq_idx, or whose row (seqlen
+ * x nheads x headdim elements of x) reaches 2^31 bytes, the largest pitch of
+ * a strided copy.
  * Outputs are undefined after any error. */
 SSD_API size_t ssd_fwd_host_workspace_size(const ssd_fwd_args* args, int64_t rows_per_piece);
 SSD_API ssd_status ssd_fwd_host(const ssd_fwd_args* args, int64_t rows_per_piece, void* device_workspace,

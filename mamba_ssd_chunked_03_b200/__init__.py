@@ -346,8 +346,11 @@ def fwd_host(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor
     """SSD forward from and to HOST tensors via ``ssd_fwd_host``.  Inputs as
     for ``fwd`` but CPU tensors (pinned, for the copies to overlap); y and
     final_states come back as CPU tensors (pinned when allocated here).  The
-    batch runs in pieces of ``rows_per_piece`` rows (0: the library chooses)
-    alternating between the current stream of ``device`` and ``stream2`` (a
+    work runs in pieces of ``rows_per_piece`` rows, or (negative) of
+    ``-rows_per_piece`` tokens of every row, each piece starting from the
+    state the previous one ends in (0: the library chooses eight pieces, of
+    rows for a batch of 8 or more, else of 64-token chunks), alternating
+    between the current stream of ``device`` and ``stream2`` (a
     torch.cuda.Stream; one per device is kept here if None), so that a
     piece's copies in overlap the previous piece's compute and copies out.
     ``workspace``: a uint8 CUDA tensor of at least the size the library asks
