@@ -18,6 +18,14 @@
 // the result is that of one call) and the chain alternates between two fp32
 // state buffers.  Piece j's ssd_fwd therefore waits for piece j - 1's; its
 // copies in do not.
+//
+// A single row of packed sequences is cut at sequence starts instead
+// (sequence pieces), found on the host ids near each eighth of the row: every
+// piece is then an independent packed problem with nothing to hand on.  Its
+// final states are computed under the global ids, and piece j copies back
+// the ids after piece j - 1's last up to its own last (through num_seqs - 1
+// for the last piece), so that every id, occurring or not, comes back from
+// exactly one piece.
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -32,6 +40,8 @@ inline size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 // One buffer set (one piece) and where each tensor sits in it.
 struct HostPlan {
   bool tok;        // pieces of `tokens` tokens of every row (else of `rows` rows)
+  bool seqp;       // one row of packed sequences, cut at sequence starts at call time
+                   // (buffer sets sized for the whole row)
   int64_t rows;    // rows per piece (all of them for token pieces)
   int64_t tokens;  // tokens per piece (the whole row for row pieces)
   int64_t pieces;
@@ -74,6 +84,7 @@ bool plan(const ssd_fwd_args* a, int64_t rows_per_piece, HostPlan* p) {
   const bool tok_ok = (size_t)L * (size_t)(H * P) * es0 < ((size_t)1 << 31);
   if (rows_per_piece < 0 && !tok_ok) return false;
   p->tok = false;
+  p->seqp = false;
   p->rows = b;
   p->tokens = L;
   if (rows_per_piece < 0) {
@@ -86,9 +97,11 @@ bool plan(const ssd_fwd_args* a, int64_t rows_per_piece, HostPlan* p) {
   } else if (!a->seq_idx && L >= 2 * 64 && tok_ok) {
     p->tok = true;
     p->tokens = ((L + kAutoPieces - 1) / kAutoPieces + 63) / 64 * 64;
+  } else if (a->seq_idx && b == 1 && L >= 2 * 64) {
+    p->seqp = true;
   }
-  if (a->seq_idx) p->rows = b;  // one piece with sequence ids: final states by id
-  p->pieces = p->tok ? (L + p->tokens - 1) / p->tokens : (b + p->rows - 1) / p->rows;
+  if (a->seq_idx) p->rows = b;  // rows of packed sequences: one piece, final states by id
+  p->pieces = p->seqp ? kAutoPieces : p->tok ? (L + p->tokens - 1) / p->tokens : (b + p->rows - 1) / p->rows;
   if (p->pieces == 1) p->tok = false;
   const int64_t rows = p->rows, T = p->tokens;
   const size_t es = a->dtype == SSD_BF16 ? 2 : 4;
@@ -105,7 +118,7 @@ bool plan(const ssd_fwd_args* a, int64_t rows_per_piece, HostPlan* p) {
   // the last piece may be shorter or have fewer rows: its workspace too
   ssd_fwd_args pl = pa;
   if (p->tok) pl.seqlen = L - (p->pieces - 1) * T;
-  else pl.batch = b - (p->pieces - 1) * rows;
+  else if (!p->seqp) pl.batch = b - (p->pieces - 1) * rows;
   if (ssd_fwd_launch_count(&pl) == 0) return false;
   const size_t wl = ssd_fwd_workspace_size(&pl);
   if (wl > p->ws_bytes) p->ws_bytes = wl;
@@ -166,6 +179,22 @@ cudaError_t d2h_tok(void* dst, const void* src, size_t w, int64_t L, int64_t t0,
                            cudaMemcpyDeviceToHost, s);
 }
 
+// Sequence pieces: the first sequence start at or after each eighth of the
+// row, as cut[0] = 0 < cut[1] < .. < cut[n] = L; n, or 0 when the ids are
+// not strictly increasing runs in [0, num_seqs) (the call then runs whole).
+int64_t seq_cuts(const int32_t* seq, int64_t L, int64_t num_seqs, int64_t cut[kAutoPieces + 1]) {
+  int64_t n = 0;
+  cut[0] = 0;
+  if (seq[0] < 0 || seq[0] >= num_seqs) return 0;
+  for (int64_t t = 1; t < L; ++t) {
+    if (seq[t] == seq[t - 1]) continue;
+    if (seq[t] < seq[t - 1] || seq[t] >= num_seqs) return 0;
+    if (n + 1 < kAutoPieces && t >= (n + 1) * L / kAutoPieces) cut[++n] = t;
+  }
+  cut[++n] = L;
+  return n;
+}
+
 }  // namespace
 
 extern "C" {
@@ -190,7 +219,11 @@ SSD_API ssd_status ssd_fwd_host(const ssd_fwd_args* args, int64_t rows_per_piece
   unsigned char* ws = static_cast<unsigned char*>(device_workspace);
   cudaStream_t s0 = static_cast<cudaStream_t>(stream);
   cudaStream_t s1 = stream2 ? static_cast<cudaStream_t>(stream2) : s0;
-  const bool two = s1 != s0 && p.pieces > 1;
+  int64_t cut[kAutoPieces + 1];
+  const int64_t ncut = p.seqp ? seq_cuts(a->seq_idx, a->seqlen, a->num_seqs, cut) : 0;
+  const bool seqp = ncut > 1;
+  const int64_t pieces = p.seqp ? (seqp ? ncut : 1) : p.pieces;
+  const bool two = s1 != s0 && pieces > 1;
 
   cudaEvent_t fork = nullptr, join = nullptr, done[2] = {nullptr, nullptr};
   auto destroy = [&]() {
@@ -235,10 +268,19 @@ SSD_API ssd_status ssd_fwd_host(const ssd_fwd_args* args, int64_t rows_per_piece
   const unsigned char* hseq = reinterpret_cast<const unsigned char*>(a->seq_idx);
   unsigned char* hy = static_cast<unsigned char*>(a->y);
   unsigned char* hfin = reinterpret_cast<unsigned char*>(a->final_states);
-  for (int64_t j = 0; j < p.pieces && st == SSD_OK; ++j) {
-    // row pieces: rows [r0, r0 + nr), every token; token pieces: every row, tokens [t0, t0 + nt)
-    const int64_t r0 = p.tok ? 0 : j * p.rows, nr = p.tok ? b : (b - r0 < p.rows ? b - r0 : p.rows);
-    const int64_t t0 = p.tok ? j * p.tokens : 0, nt = p.tok ? (L - t0 < p.tokens ? L - t0 : p.tokens) : L;
+  const bool by_tok = p.tok || seqp;  // pieces of tokens of every row
+  for (int64_t j = 0; j < pieces && st == SSD_OK; ++j) {
+    // row pieces: rows [r0, r0 + nr), every token; token and sequence pieces:
+    // every row, tokens [t0, t0 + nt)
+    const int64_t r0 = by_tok ? 0 : j * p.rows, nr = by_tok ? b : (b - r0 < p.rows ? b - r0 : p.rows);
+    int64_t t0 = 0, nt = L;
+    if (p.tok) {
+      t0 = j * p.tokens;
+      nt = L - t0 < p.tokens ? L - t0 : p.tokens;
+    } else if (seqp) {
+      t0 = cut[j];
+      nt = cut[j + 1] - cut[j];
+    }
     cudaStream_t s = (two && (j & 1)) ? s1 : s0;
     unsigned char* set = ws + (two ? (size_t)(j & 1) * p.set_bytes : 0);
     ssd_fwd_args pa = piece_args(a, nr, nt);
@@ -254,21 +296,24 @@ SSD_API ssd_status ssd_fwd_host(const ssd_fwd_args* args, int64_t rows_per_piece
     if (p.tok) {  // from the state the previous piece left, to the other buffer
       pa.initial_states = (j > 0 || a->initial_states) ? state[(j + 1) & 1] : nullptr;
       pa.final_states = state[j & 1];
-    } else {
-      pa.initial_states = a->initial_states ? reinterpret_cast<const float*>(set + p.off_init) : nullptr;
+    } else {  // (sequence pieces: h0 is the state before the row's first token only)
+      pa.initial_states =
+          a->initial_states && (!seqp || j == 0) ? reinterpret_cast<const float*>(set + p.off_init) : nullptr;
       pa.final_states = a->final_states ? reinterpret_cast<float*>(set + p.off_final) : nullptr;
     }
     pa.workspace = p.ws_bytes ? set + p.off_ws : nullptr;
     pa.workspace_bytes = p.ws_bytes;
     bool ok;
-    if (p.tok) {
+    if (by_tok) {
       ok = h2d_tok(set + p.off_x, hx, p.tok_x, L, t0, nt, b, s) == cudaSuccess &&
            h2d_tok(set + p.off_dt, hdt, p.tok_dt, L, t0, nt, b, s) == cudaSuccess &&
            h2d_tok(set + p.off_B, hB, p.tok_bc, L, t0, nt, b, s) == cudaSuccess &&
            h2d_tok(set + p.off_C, hC, p.tok_bc, L, t0, nt, b, s) == cudaSuccess &&
-           (!hz || h2d_tok(set + p.off_z, hz, p.tok_x, L, t0, nt, b, s) == cudaSuccess);
+           (!hz || h2d_tok(set + p.off_z, hz, p.tok_x, L, t0, nt, b, s) == cudaSuccess) &&
+           (!seqp || h2d_tok(set + p.off_seq, hseq, p.tok_seq, L, t0, nt, b, s) == cudaSuccess) &&
+           (!seqp || j > 0 || !hinit || h2d(set + p.off_init, hinit, p.row_init, s) == cudaSuccess);
       // piece j's state comes from piece j - 1 (on the other stream)
-      if (ok && two && j > 0) ok = cudaStreamWaitEvent(s, done[(j - 1) & 1], 0) == cudaSuccess;
+      if (ok && p.tok && two && j > 0) ok = cudaStreamWaitEvent(s, done[(j - 1) & 1], 0) == cudaSuccess;
     } else {
       const size_t row_x = (size_t)L * p.tok_x, row_dt = (size_t)L * p.tok_dt, row_bc = (size_t)L * p.tok_bc,
                    row_seq = (size_t)L * p.tok_seq;
@@ -293,13 +338,21 @@ SSD_API ssd_status ssd_fwd_host(const ssd_fwd_args* args, int64_t rows_per_piece
       fail(SSD_ERR_CUDA);
       break;
     }
-    const cudaError_t ey = p.tok ? d2h_tok(hy, set + p.off_y, p.tok_x, L, t0, nt, b, s)
-                                 : d2h(hy + r0 * L * p.tok_x, set + p.off_y, nr * L * p.tok_x, s);
+    const cudaError_t ey = by_tok ? d2h_tok(hy, set + p.off_y, p.tok_x, L, t0, nt, b, s)
+                                  : d2h(hy + r0 * L * p.tok_x, set + p.off_y, nr * L * p.tok_x, s);
     if (ey != cudaSuccess) {
       fail(SSD_ERR_CUDA);
       break;
     }
-    if (hfin && (!p.tok || j == p.pieces - 1)) {  // token pieces: the last piece's end state
+    if (hfin && seqp) {  // the ids after the previous piece's last, through this piece's last
+      const int64_t lo = j == 0 ? 0 : (int64_t)a->seq_idx[cut[j] - 1] + 1;
+      const int64_t hi = j == pieces - 1 ? a->num_seqs - 1 : (int64_t)a->seq_idx[cut[j + 1] - 1];
+      if (d2h(hfin + lo * p.row_final, set + p.off_final + lo * p.row_final, (size_t)(hi - lo + 1) * p.row_final,
+              s) != cudaSuccess) {
+        fail(SSD_ERR_CUDA);
+        break;
+      }
+    } else if (hfin && (!p.tok || j == p.pieces - 1)) {  // token pieces: the last piece's end state
       const size_t fb = a->seq_idx ? (size_t)a->num_seqs * p.row_final : nr * p.row_final;
       const void* src = p.tok ? static_cast<const void*>(state[j & 1]) : set + p.off_final;
       if (d2h(hfin + (a->seq_idx ? 0 : r0 * p.row_final), src, fb, s) != cudaSuccess) {

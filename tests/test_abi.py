@@ -453,7 +453,9 @@ def test_host_workspace_size_by_pieces():
 def test_host_default_pieces_for_a_small_batch():
     """Under eight rows and without sequence ids the library cuts every row
     into eight token pieces of whole 64-token chunks; rows too short for two
-    chunks stay one piece, and so does a call with sequence ids."""
+    chunks stay one piece.  With sequence ids a single row is cut at sequence
+    starts found at call time, so its two buffer sets are sized for the whole
+    row; more rows with sequence ids stay one piece."""
     a = base_args(batch=1, seqlen=2000)  # ceil(2000 / 8) = 250 -> 256 tokens a piece
     assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 0) == \
         ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), -256)
@@ -463,8 +465,11 @@ def test_host_default_pieces_for_a_small_batch():
     assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(short), 0) == \
         ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(short), 1)
     a.seq_idx, a.num_seqs = 1 << 20, 3
-    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 0) == \
-        ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 1)
+    one = ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 1)
+    assert 2 * one - 4096 < ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(a), 0) < 2 * one
+    two_rows = base_args(batch=2, seqlen=2000, seq_idx=1 << 20, num_seqs=3)
+    assert ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(two_rows), 0) == \
+        ssd.lib.ssd_fwd_host_workspace_size(ctypes.byref(two_rows), 1)
 
 
 def test_host_call_checked_before_anything_is_enqueued():

@@ -107,3 +107,50 @@ def test_host_entry_with_pageable_memory():
     torch.cuda.current_stream().synchronize()
     assert not y.is_pinned()
     assert torch.equal(y, y_p) and torch.equal(f, f_p)
+
+
+def _packed_row_case(lens, ids, num_seqs, seed):
+    L = sum(lens)
+    shape = si.SSDShape("host_seqp", 1, L, 8, 64, 128, 1, 64, "bf16", h0_std=0.2, seed=seed)
+    d = si.make_inputs(shape)
+    d["seq_idx"] = torch.cat([torch.full((n,), i, dtype=torch.int32) for n, i in zip(lens, ids)]).view(1, L)
+    d["num_seqs"] = num_seqs
+    return shape, d
+
+
+def _host_vs_device(d, num_seqs, z):
+    dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    y_ref, f_ref = ssd.fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], 64, dev["initial_states"],
+                           dev["seq_idx"], num_seqs, z=None if z is None else z.cuda())
+    torch.cuda.synchronize()
+    host = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    final = torch.full((num_seqs, 8, 64, 128), float("nan")).pin_memory()
+    y, f = ssd.fwd_host(host["x"], host["dt"], host["A"], host["B"], host["C"], host["D"], 64,
+                        host["initial_states"], host["seq_idx"], num_seqs, final_states=final,
+                        z=None if z is None else z.pin_memory())
+    torch.cuda.current_stream().synchronize()
+    return y, f, y_ref.cpu(), f_ref.cpu()
+
+
+@pytest.mark.parametrize("gated", [False, True], ids=["plain", "gated"])
+def test_host_packed_row_in_sequence_pieces(gated):
+    """One row of packed sequences is cut at sequence starts (here into 7
+    pieces): every id comes back from exactly one piece, ids that never occur
+    (0, 3, 7 and 11, at the ends and between pieces) as zeros over a host
+    buffer that starts as NaN, and h0 enters the row's first sequence only."""
+    lens = [300, 410, 90, 700, 260, 500, 333, 407]
+    shape, d = _packed_row_case(lens, [1, 2, 4, 5, 6, 8, 9, 10], 12, seed=21)
+    z = torch.randn(d["x"].shape, generator=torch.Generator().manual_seed(22)).to(d["x"].dtype) if gated else None
+    y, f, y_ref, f_ref = _host_vs_device(d, 12, z)
+    assert not torch.isnan(f).any()
+    assert not f[[0, 3, 7, 11]].any()
+    assert _rel(y, y_ref) <= 2e-3, _rel(y, y_ref)
+    assert _rel(f, f_ref) <= 2e-3, _rel(f, f_ref)
+
+
+def test_host_packed_row_out_of_order_runs_whole():
+    """Ids that do not increase along the row cannot be cut into independent
+    pieces; the call then runs as one piece, on the exact kernel."""
+    shape, d = _packed_row_case([100, 150, 130], [2, 0, 1], 3, seed=23)
+    y, f, y_ref, f_ref = _host_vs_device(d, 3, None)
+    assert torch.equal(y, y_ref) and torch.equal(f, f_ref)
