@@ -196,10 +196,17 @@ SSD_API ssd_status ssd_fwd_noalloc(const ssd_fwd_args* args, void* stream);
  * the previous piece computes and copies out (on PCIe the two directions run
  * at the same time).  Token pieces hand their state on through two fp32
  * buffers in the workspace, so a piece's ssd_fwd also waits for the previous
- * piece's.  With seq_idx the batch is one piece: final_states is then indexed
- * by sequence id, and a call on part of the rows would clear the ids it does
- * not see.  `stream2` may be NULL: everything then runs on `stream`, in
- * order.
+ * piece's.  With seq_idx and rows_per_piece = 0, a single row of 128 tokens
+ * or more is cut at sequence starts (the first after each eighth of the row,
+ * read from the host seq_idx at call time): each piece is then an independent
+ * packed problem, and piece j returns the final states of the ids after
+ * piece j - 1's last id through its own last id (the last piece through
+ * num_seqs - 1), so that ids that never occur still come back as zeros; the
+ * two buffer sets are then sized for the whole row.  Ids that are not
+ * strictly increasing runs in [0, num_seqs) keep the call in one piece.  Any
+ * other call with seq_idx is one piece: final_states is indexed by sequence
+ * id, and a call on part of the rows would clear the ids it does not see.
+ * `stream2` may be NULL: everything then runs on `stream`, in order.
  *
  * `device_workspace` (256-byte aligned, at least ssd_fwd_host_workspace_size
  * bytes, contents on entry irrelevant) holds the two buffer sets.  The call
