@@ -70,7 +70,9 @@ ssd_fwd_args piece_args(const ssd_fwd_args* a, int64_t rows, int64_t tokens) {
 // Pieces the library picks: eight, so that the first piece's copies in and
 // the last one's copies out, which nothing overlaps, are an eighth of the call
 // each.  Rows when the batch has eight or more, else tokens (in whole 64-token
-// chunks) when the rows are long enough and carry no sequence ids.
+// chunks) when the rows are long enough and carry no sequence ids, else, for
+// a single row with sequence ids, sequence pieces.  (Token and sequence
+// pieces are copied with the row as pitch, which must stay below 2^31 bytes.)
 constexpr int64_t kAutoPieces = 8;
 
 bool plan(const ssd_fwd_args* a, int64_t rows_per_piece, HostPlan* p) {
@@ -79,7 +81,6 @@ bool plan(const ssd_fwd_args* a, int64_t rows_per_piece, HostPlan* p) {
     return false;
   const int64_t b = a->batch, L = a->seqlen, H = a->nheads, P = a->headdim, N = a->dstate, G = a->ngroups;
   if (rows_per_piece < 0 && a->seq_idx) return false;  // token pieces would split sequences
-  // a token piece is copied with the row length as pitch, which must stay below 2^31 bytes
   const size_t es0 = a->dtype == SSD_BF16 ? 2 : 4;
   const bool tok_ok = (size_t)L * (size_t)(H * P) * es0 < ((size_t)1 << 31);
   if (rows_per_piece < 0 && !tok_ok) return false;
@@ -97,7 +98,7 @@ bool plan(const ssd_fwd_args* a, int64_t rows_per_piece, HostPlan* p) {
   } else if (!a->seq_idx && L >= 2 * 64 && tok_ok) {
     p->tok = true;
     p->tokens = ((L + kAutoPieces - 1) / kAutoPieces + 63) / 64 * 64;
-  } else if (a->seq_idx && b == 1 && L >= 2 * 64) {
+  } else if (a->seq_idx && b == 1 && L >= 2 * 64 && tok_ok) {
     p->seqp = true;
   }
   if (a->seq_idx) p->rows = b;  // rows of packed sequences: one piece, final states by id
